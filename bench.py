@@ -1,0 +1,379 @@
+"""Benchmark of the affine-quantised MoE FFN layer on B200.
+
+One JSON line on rank 0.  A step is one forward of the whole layer (router
+qmv, routing, gate/up + SwiGLU, down, combine) for the workload's batch of
+tokens.  Default workload: single-token decode of the 4096-hidden,
+512-expert, top-4, 4-bit layer with a 4-bit shared expert and 8-bit router
+and sigmoid gate.  Inputs are seeded synthetic weights and activations.
+
+L2: the timed steps cycle through `--copies` independent copies of the
+layer (router, shared expert and expert bank each) with a fresh token per
+step, so the bytes touched between two uses of any weight exceed the 126 MB
+L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own replica on its own tokens (the
+decode path does not shard); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (config, tokens per step)
+    "decode_397b_m1": ("decode_397b", 1),
+    "decode_397b_m8": ("decode_397b", 8),
+    "decode_30b_m1": ("decode_30b", 1),
+    "decode_mixed_2bit_m1": ("mixed_2bit", 1),
+}
+METRIC = "qMoE layer tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_397b_m1", choices=sorted(WORKLOADS))
+    ap.add_argument("--copies", type=int, default=8)
+    ap.add_argument("--cpu-sample", type=int, default=16,
+                    help="tokens of the bounded oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.p = None
+        self.path = os.path.join("/tmp", f"moeq_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def cpu_oracle_sample(cfg, n_tokens, seed=0):
+    """The oracle as it stands on a bounded sample: n_tokens single-token
+    forwards of the workload's layer (router, routing, K experts, shared
+    expert), all host cores.  Returns (tokens/s, cores, seconds)."""
+    import numpy as np
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from helpers import oracle_layer, host_router
+    from quantized_mixture_experts_affine_b200 import synth
+    xb = synth.normal_bf16_host(seed, synth.tag(synth.X, 9999), n_tokens * cfg.H).reshape(
+        n_tokens, cfg.H)
+    R = host_router(cfg, seed, 0)
+    logits = oracle.qmv(R, xb)
+    idx, w, _ = oracle.route(logits, cfg.K, cfg.renorm, cfg.router_scale)
+    experts = np.unique(idx)
+    L = oracle_layer(cfg, seed, 0, experts)           # host weights: not timed
+    remap = {int(e): i for i, e in enumerate(experts)}
+    idx_c = np.vectorize(lambda e: remap[int(e)])(idx).astype(np.int32)
+    cores = oracle.get_threads()
+    t0 = time.perf_counter()
+    logits = oracle.qmv(R, xb)
+    oracle.route(logits, cfg.K, cfg.renorm, cfg.router_scale)
+    oracle.expert_ffn(L, xb, idx_c, w)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, cores, dt
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from quantized_mixture_experts_affine_b200.layer import CONFIGS
+    cfg_name, M = WORKLOADS[args.workload]
+    cfg = CONFIGS[cfg_name]
+    # each step: one bounded sample of M tokens of the workload
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        cpu_oracle_sample(cfg, M)
+    times = []
+    cores = 0
+    for s in range(args.steps):
+        v, cores, dt = cpu_oracle_sample(cfg, M, seed=0)
+        times.append(dt)
+    total = sum(times)
+    value = M * args.steps / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "tokens_per_step": M},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} steps x {M} token(s) of {args.workload}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    from quantized_mixture_experts_affine_b200 import moeq, synth
+    from quantized_mixture_experts_affine_b200.layer import CONFIGS, Workspace, synthetic_layer
+
+    rank, world, local = dist_setup(args.gpus)
+    cfg_name, M = WORKLOADS[args.workload]
+    cfg = CONFIGS[cfg_name]
+    K, W = args.steps, args.warmup
+    assert W >= 3, "at least 3 warm-up steps"
+    copies = max(1, args.copies)
+    seed = 1000 * rank
+    layers = [synthetic_layer(cfg, seed, c) for c in range(copies)]
+    total_steps = W + K
+    # a fresh token batch per step
+    xs = synth.normal_bf16_dev(seed, synth.tag(synth.X, 777), total_steps * M * cfg.H).view(
+        total_steps, M, cfg.H)
+    ys = torch.empty((copies, M, cfg.H), dtype=torch.float32, device="cuda")
+    idx = torch.empty((copies, M, cfg.K), dtype=torch.int32, device="cuda")
+    wts = torch.empty((copies, M, cfg.K), dtype=torch.float32, device="cuda")
+    ws = Workspace(layers[0], M, moeq.MODE_DECODE)
+    st = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def step(i, stream):
+        c = i % copies
+        moeq.moeq_layer_forward(layers[c].desc, xs[i], M, ys[c], None, idx[c], wts[c], ws.buf,
+                                ws.bytes, moeq.MODE_DECODE, stream)
+
+    # warm-up (also first-call set-up of the library) outside any capture
+    with torch.cuda.stream(st):
+        for i in range(W):
+            step(i, st)
+    st.synchronize()
+
+    # capture the K timed steps as CUDA graphs of `copies` steps each
+    graphs = []
+    n0 = moeq.moeq_launch_count()
+    with torch.cuda.stream(st):
+        for g0 in range(W, total_steps, copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                for i in range(g0, min(g0 + copies, total_steps)):
+                    step(i, st)
+            graphs.append(g)
+    launches_per_timed_region = moeq.moeq_launch_count() - n0
+    # one untimed replay of the first graph (graph upload)
+    with torch.cuda.stream(st):
+        graphs[0].replay()
+    st.synchronize()
+
+    peak_hbm, peak_bf16, peak_kind = measured_peaks()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(st):
+            ev0.record(st)
+            for g in graphs:
+                g.replay()
+            ev1.record(st)
+        st.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    ms_step = ms_total / K
+    value = M * K * world / (ms_total / 1e3)
+
+    # routing actually taken in the last steps -> distinct expert bytes per step
+    exp_bytes = cfg.expert_bytes()
+    gu_bytes_expert = 2 * synth.packed_bytes(cfg.I, cfg.H, cfg.expert_bits, cfg.G)
+    sh_gu = 2 * synth.packed_bytes(cfg.shared_I, cfg.H, cfg.shared_bits, cfg.G) if cfg.shared else 0
+    idx_np = idx.cpu().numpy()
+    distinct = [len(set(idx_np[c].ravel().tolist())) for c in range(copies)]
+    mean_distinct = sum(distinct) / len(distinct)
+    layer_bytes = cfg.router_bytes() + mean_distinct * exp_bytes + cfg.shared_bytes()
+    gu_bytes = mean_distinct * gu_bytes_expert + sh_gu
+
+    # dominant kernel (gate/up GEMV): per-launch durations over the same steps,
+    # events recorded around it inside captured graphs
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    kgraphs = []
+    with torch.cuda.stream(st):
+        for g0 in range(W, total_steps, copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                for i in range(g0, min(g0 + copies, total_steps)):
+                    moeq.moeq_set_profile_events(starts[i - W], stops[i - W])
+                    step(i, st)
+            moeq.moeq_set_profile_events(None, None)
+            kgraphs.append(g)
+        for g in kgraphs:
+            g.replay()
+    st.synchronize()
+    k_ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops)) / K
+    k_ms = max_over_ranks(k_ms, world)
+    achieved = gu_bytes / (k_ms / 1e3) / 1e9
+
+    # end to end through the public API: pinned host x -> device, forward,
+    # y -> pinned host, every step
+    x_host = xs[:K].cpu().pin_memory()
+    y_host = torch.empty((K, M, cfg.H), dtype=torch.float32).pin_memory()
+    xdev = torch.empty((M, cfg.H), dtype=torch.bfloat16, device="cuda")
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(st):
+        e0.record(st)
+        for i in range(K):
+            c = i % copies
+            xdev.copy_(x_host[i], non_blocking=True)
+            moeq.moeq_layer_forward(layers[c].desc, xdev, M, ys[c], None, idx[c], wts[c], ws.buf,
+                                    ws.bytes, moeq.MODE_DECODE, st)
+            y_host[i].copy_(ys[c], non_blocking=True)
+        e1.record(st)
+    st.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = M * K * world / (e2e_ms / 1e3)
+    status = moeq.moeq_device_status(st)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens_per_step": M, "hidden": cfg.H,
+                   "experts": cfg.E, "top_k": cfg.K, "intermediate": cfg.I,
+                   "expert_bits": cfg.expert_bits, "router_bits": cfg.router_bits,
+                   "shared_expert": cfg.shared, "parallelism": f"replicas{world}",
+                   "l2": f"{copies} layer copies cycled, fresh tokens per step "
+                         f"({copies * layer_bytes / 1e6:.0f} MB touched per cycle > 126 MB L2)",
+                   "cuda_graph": True},
+        "layer_hbm": {"bytes_per_step": layer_bytes, "achieved_gbs": layer_bytes / (ms_step / 1e3) / 1e9,
+                      "peak_gbs": peak_hbm, "frac": layer_bytes / (ms_step / 1e3) / 1e9 / peak_hbm,
+                      "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "k_gemv gate/up+SwiGLU", "achieved": achieved,
+                     "peak": peak_hbm, "unit": "GB/s", "frac": achieved / peak_hbm,
+                     "traffic": None, "bytes_per_launch": gu_bytes, "ms_per_launch": k_ms,
+                     "peak_kind": peak_kind},
+        "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": M * cfg.H * 2,
+                "d2h_bytes_per_step": M * cfg.H * 4},
+        "gpu_launches": int(launches_per_timed_region),
+        "clocks": clk.summary(),
+        "device_status": status,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        v, cores, dt = cpu_oracle_sample(cfg, args.cpu_sample)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{args.cpu_sample} tokens of {args.workload} "
+                                          f"({dt:.1f} s)"}
+    for g in graphs + kgraphs:
+        g.reset()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+/*
+ * moeq.h -- C ABI of libmoeq.so: the forward pass of one affine-quantised
+ * mixture-of-experts FFN layer on an NVIDIA B200 (sm_100a).
+ *
+ * Weight format (sources: "danveloper/flash-moe" issue thread, the
+ * mixed-precision comment; "flash-moe-inference", the matvec_4bit_fma
+ * listing; "markbaseengine/MOE_FIX_SUCCESS_EXPERT_WORKS.md", "Why This
+ * Worked"):
+ *   - a matrix of out_dim rows by in_dim inputs holds unsigned b-bit codes
+ *     q, b in {2, 4, 8}, packed 32/b per uint32 word, row-major
+ *     ([out_dim][in_dim*b/32] words); value j of a word sits in bits
+ *     [j*b, (j+1)*b) (low bits first);
+ *   - each row is cut into groups of group_size consecutive inputs
+ *     (64 on the pages; 32 and 128 are also accepted) and each group has
+ *     one bf16 scale and one bf16 bias, [out_dim][in_dim/group_size] each;
+ *   - the weight is w = q * scale + bias (affine mode);
+ *   - bit widths are per tensor, so an 8-bit router sits beside 4-bit
+ *     experts.
+ * A bank of E experts stores matrix e at w + e*expert_stride_w (words)
+ * and scales/biases + e*expert_stride_sb (entries); strides of 0 mean a
+ * single matrix.
+ *
+ * Conventions for every entry point:
+ *   - all tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates or frees them; descriptor structs may live
+ *     in host memory and are read during the call only;
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream); every call is asynchronous on it and does no host
+ *     synchronisation and no device allocation;
+ *   - arguments are checked on the host before anything is launched; a
+ *     failed check returns an error code and launches nothing;
+ *   - problems only the device can see (a bounded wait that ran out, an
+ *     operand outside the fp16 range of the prefill tiles) set a device
+ *     status word, read and cleared by moeq_device_status;
+ *   - bf16 values travel as their 16-bit patterns (uint16_t);
+ *   - row offsets are 64-bit; no index arithmetic is narrowed to 16 bits.
+ */
+#ifndef MOEQ_H
+#define MOEQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOEQ_OK = 0,
+  MOEQ_ERR_INVALID_ARG = 1,  /* null pointer, size <= 0, K > E, index out of range ... */
+  MOEQ_ERR_UNSUPPORTED = 2,  /* bits not in {2,4,8}, group size not in {32,64,128}, sizes beyond limits */
+  MOEQ_ERR_ALIGNMENT = 3,    /* pointer not 16-byte aligned, in_dim not a multiple of group_size */
+  MOEQ_ERR_WORKSPACE = 4,    /* workspace missing or smaller than moeq_workspace_bytes */
+  MOEQ_ERR_CUDA = 5,         /* a CUDA runtime call failed */
+  MOEQ_ERR_TIMEOUT = 6,      /* device status: a bounded device-side wait ran out */
+  MOEQ_ERR_RANGE = 7         /* device status: a prefill operand exceeded the fp16 range */
+} moeq_status;
+
+typedef enum {
+  MOEQ_MODE_AUTO = 0,    /* decode for M <= 64, prefill otherwise */
+  MOEQ_MODE_DECODE = 1,  /* HBM-bound split-K quantised matvec path */
+  MOEQ_MODE_PREFILL = 2  /* sort-by-expert gather-QMM on tcgen05 tensor cores */
+} moeq_mode;
+
+/* One packed tensor or bank of tensors (device memory). */
+typedef struct {
+  const uint32_t* w;        /* codes, [E][out_dim][in_dim*bits/32] */
+  const uint16_t* scales;   /* bf16 bits, [E][out_dim][in_dim/group_size] */
+  const uint16_t* biases;   /* bf16 bits, same shape as scales */
+  int32_t out_dim;
+  int32_t in_dim;
+  int32_t bits;             /* 2, 4 or 8 */
+  int32_t group_size;       /* values per group along in_dim: 64 (or 32, 128) */
+  int64_t expert_stride_w;  /* words from one expert's matrix to the next (0: single matrix) */
+  int64_t expert_stride_sb; /* scale/bias entries from one expert to the next */
+} moeq_qtensor;
+
+/*
+ * One layer ("markbaseengine/MOE_ROUTER_WORKS_BREAKTHROUGH.md", "Forward
+ * Pass Sequence"; "flash-moe-inference", per-layer pipeline):
+ *   router [E][H]; gate, up [E][I][H]; down [E][H][I];
+ *   optional shared expert: sh_gate, sh_up [I_sh][H], sh_down [H][I_sh],
+ *   and its sigmoid gate sh_expert_gate [1][H] ("danveloper/flash-moe"
+ *   thread: mlp.shared_expert_gate, 8-bit).
+ */
+typedef struct {
+  moeq_qtensor router;
+  moeq_qtensor gate;
+  moeq_qtensor up;
+  moeq_qtensor down;
+  int32_t has_shared;       /* 0 or 1 */
+  moeq_qtensor sh_gate;
+  moeq_qtensor sh_up;
+  moeq_qtensor sh_down;
+  moeq_qtensor sh_expert_gate;
+  int32_t hidden;           /* H */
+  int32_t inter;            /* I */
+  int32_t n_experts;        /* E */
+  int32_t top_k;            /* K, 1 <= K <= min(E, 32) */
+  int32_t renorm;           /* 1: routed weights renormalised to sum 1 over the K chosen */
+  float router_scale;       /* logits are multiplied by this before the softmax (default 1) */
+} moeq_layer;
+
+/*
+ * Unpack and dequantise matrix `expert` of `t` (source: "flash-moe-inference",
+ * dequantised value nibble*scale + bias).
+ *   q_out: nullable, uint8 [out_dim][in_dim], the codes;
+ *   w_out: nullable, fp32 [out_dim][in_dim], fmaf(q, scale, bias) -- one
+ *          correctly rounded fp32 operation, so the result is exact to the bit.
+ * Errors: INVALID_ARG (t NULL, both outputs NULL, expert < 0), UNSUPPORTED,
+ * ALIGNMENT, CUDA.
+ */
+moeq_status moeq_dequant(const moeq_qtensor* t, int32_t expert, uint8_t* q_out, float* w_out,
+                         void* stream);
+
+/*
+ * y[m][r] = sum_g ( s[r,g] * sum_{c in g} q[r,c] x[m][c]  +  b[r,g] * sum_{c in g} x[m][c] )
+ * for m < M tokens: the group form of the fma(q, scale*x, bias*x) factoring
+ * ("flash-moe-inference", matvec_4bit_fma listing), accumulated in fp32.
+ *   x: bf16 [M][in_dim], 16-byte aligned rows; y: fp32 [M][out_dim].
+ * 1 <= M <= 64.  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+moeq_status moeq_qmv(const moeq_qtensor* t, int32_t expert, const uint16_t* x, int32_t M, float* y,
+                     void* stream);
+
+/*
+ * Routing ("markbaseengine/MOE_ROUTER_WORKS_BREAKTHROUGH.md", Forward Pass
+ * Sequence steps 3-4; "flash-moe-inference", softmax + topK):
+ *   p = softmax(router_scale * logits[m]); the K largest p (ties to the
+ *   lower expert index) in order of p descending; w = p_k / sum of the K
+ *   chosen p when renorm, else p_k.
+ *   logits: fp32 [M][E]; idx: int32 [M][K]; w: fp32 [M][K].
+ * 1 <= K <= min(E, 32); E <= 4096; M >= 0 (M = 0 launches nothing).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+moeq_status moeq_route_topk(const float* logits, int32_t M, int32_t E, int32_t K, int32_t renorm,
+                            float router_scale, int32_t* idx, float* w, void* stream);
+
+/*
+ * Experts and combine with the routing given ("flash-moe-inference",
+ * swiglu and moe_combine_residual listings; "markbaseengine/MOE_FIX_SUCCESS_
+ * EXPERT_WORKS.md", fused gate/up):
+ *   y[m] = sum_k w[m][k] * Wd_e (silu(Wg_e x_m) * (Wu_e x_m)),  e = idx[m][k]
+ *          + sigmoid(Wsg x_m) * SharedExpert(x_m)        (if has_shared)
+ *          + residual[m]                                  (if residual != NULL)
+ * summed over k in order 0..K-1.
+ *   x: bf16 [M][H]; idx int32 [M][K] (each in [0,E)); w fp32 [M][K];
+ *   residual: nullable fp32 [M][H]; y: fp32 [M][H].
+ *   ws: device workspace of at least moeq_workspace_bytes(L, M, mode) bytes,
+ *   256-byte aligned, owned by the caller, contents ignored on entry.
+ * mode: DECODE requires M <= 64; PREFILL requires the prefill constraints
+ * (8-bit or 4-bit experts, H and I multiples of 64). The prefill path
+ * computes every output row independently of M, so splitting the tokens
+ * into chunks gives bit-identical results.
+ * idx is not read on the host; an index outside [0,E) found on the device
+ * sets MOEQ_ERR_INVALID_ARG in the device status word and expert 0 is used
+ * in its place.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA.
+ */
+moeq_status moeq_expert_ffn(const moeq_layer* L, const uint16_t* x, int32_t M, const int32_t* idx,
+                            const float* w, const float* residual, float* y, void* ws,
+                            size_t ws_bytes, int32_t mode, void* stream);
+
+/*
+ * The whole layer: router qmv -> route_topk -> expert_ffn, on the device,
+ * with no host round trip.  idx_out/w_out: nullable, receive the routing.
+ * Same buffers, workspace and errors as moeq_expert_ffn.
+ */
+moeq_status moeq_layer_forward(const moeq_layer* L, const uint16_t* x, int32_t M, float* y,
+                               const float* residual, int32_t* idx_out, float* w_out, void* ws,
+                               size_t ws_bytes, int32_t mode, void* stream);
+
+/* Workspace bytes moeq_expert_ffn / moeq_layer_forward need for M tokens
+ * in `mode` (0 if the arguments are invalid). */
+size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mode);
+
+/* Reads and clears the device status word of the current device (synchronises
+ * `stream`).  *status_out receives MOEQ_OK or the first device error seen. */
+moeq_status moeq_device_status(void* stream, int32_t* status_out);
+
+/*
+ * Diagnostics for benchmarks.
+ *
+ * moeq_set_profile_events: when `start` and `stop` are cudaEvent_t handles
+ * (passed as void*), every later moeq_layer_forward / moeq_expert_ffn call
+ * made from the same host thread records `start` on its stream right before
+ * its main weight-streaming kernel (decode: the gate/up GEMV; prefill: the
+ * gate/up gather-QMM) and `stop` right after it, so cudaEventElapsedTime
+ * gives that kernel's duration.  Recording also works while the stream is
+ * being captured into a CUDA graph.  NULL, NULL turns it off.  The caller
+ * owns the events.  Returns INVALID_ARG if exactly one of them is NULL.
+ *
+ * moeq_launch_count: number of kernels this library has launched (or added
+ * to a graph being captured) from any thread since it was loaded.
+ */
+moeq_status moeq_set_profile_events(void* start, void* stop);
+uint64_t moeq_launch_count(void);
+
+/* Text of a status code (static storage). */
+const char* moeq_status_str(int32_t status);
+
+/* Library version string (static storage). */
+const char* moeq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEQ_H */

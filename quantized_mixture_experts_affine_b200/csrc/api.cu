@@ -1,0 +1,490 @@
+// C ABI of libmoeq.so (include/moeq.h): argument checks, workspace layout
+// and the launch sequences of the decode and prefill paths.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moeq.h"
+#include "prefill.h"
+
+#define MOEQ_API extern "C" __attribute__((visibility("default")))
+
+using namespace moeq;
+
+// ------------------------------------------------------------------ device status word
+__device__ int g_moeq_status;
+
+static int* status_ptr() {
+  static std::mutex mu;
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moeq_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = (int*)p;
+  }
+  return ptrs[dev];
+}
+
+// ------------------------------------------------------------------ diagnostics
+static std::atomic<uint64_t> g_launches{0};
+static thread_local cudaEvent_t t_prof_start = nullptr, t_prof_stop = nullptr;
+
+namespace moeq {
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+cudaError_t profile_mark(bool start, cudaStream_t st) {
+  cudaEvent_t e = start ? t_prof_start : t_prof_stop;
+  return e ? cudaEventRecord(e, st) : cudaSuccess;
+}
+}  // namespace moeq
+
+// ------------------------------------------------------------------ checks
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Shape/format checks of one tensor.  n_mats: experts addressable (>= 1).
+static moeq_status check_tensor(const moeq_qtensor* t, int64_t n_mats) {
+  if (!t || !t->w || !t->scales || !t->biases) return MOEQ_ERR_INVALID_ARG;
+  if (t->out_dim <= 0 || t->in_dim <= 0 || n_mats <= 0) return MOEQ_ERR_INVALID_ARG;
+  if (t->bits != 2 && t->bits != 4 && t->bits != 8) return MOEQ_ERR_UNSUPPORTED;
+  if (t->group_size != 32 && t->group_size != 64 && t->group_size != 128)
+    return MOEQ_ERR_UNSUPPORTED;
+  const int vpc = 128 / t->bits;  // codes per 16-byte chunk
+  if (t->in_dim % t->group_size || t->in_dim % vpc) return MOEQ_ERR_ALIGNMENT;
+  if (!aligned(t->w, 16) || !aligned(t->scales, 2) || !aligned(t->biases, 2))
+    return MOEQ_ERR_ALIGNMENT;
+  const int64_t words = (int64_t)t->out_dim * t->in_dim * t->bits / 32;
+  const int64_t groups = (int64_t)t->out_dim * (t->in_dim / t->group_size);
+  if (n_mats > 1) {
+    if (t->expert_stride_w < words || t->expert_stride_sb < groups) return MOEQ_ERR_INVALID_ARG;
+    if ((t->expert_stride_w * 4) % 16) return MOEQ_ERR_ALIGNMENT;
+  }
+  return MOEQ_OK;
+}
+
+// Decode GEMV limit: a row is cut into at most 8 slices of 512 bytes.
+static int slices_of(const moeq_qtensor& t) {
+  const int cpr = t.in_dim / (128 / t.bits);
+  return (cpr + 31) / 32;
+}
+
+static moeq_status check_layer(const moeq_layer* L) {
+  if (!L) return MOEQ_ERR_INVALID_ARG;
+  const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
+  if (H <= 0 || I <= 0 || E <= 0 || K <= 0) return MOEQ_ERR_INVALID_ARG;
+  if (K > E) return MOEQ_ERR_INVALID_ARG;
+  if (K > kMaxK || E > kMaxE) return MOEQ_ERR_UNSUPPORTED;
+  moeq_status s;
+  if ((s = check_tensor(&L->router, 1)) != MOEQ_OK) return s;
+  if ((s = check_tensor(&L->gate, E)) != MOEQ_OK) return s;
+  if ((s = check_tensor(&L->up, E)) != MOEQ_OK) return s;
+  if ((s = check_tensor(&L->down, E)) != MOEQ_OK) return s;
+  if (L->router.out_dim != E || L->router.in_dim != H) return MOEQ_ERR_INVALID_ARG;
+  if (L->gate.out_dim != I || L->gate.in_dim != H) return MOEQ_ERR_INVALID_ARG;
+  if (L->up.out_dim != I || L->up.in_dim != H) return MOEQ_ERR_INVALID_ARG;
+  if (L->down.out_dim != H || L->down.in_dim != I) return MOEQ_ERR_INVALID_ARG;
+  if (L->gate.bits != L->up.bits || L->gate.group_size != L->up.group_size)
+    return MOEQ_ERR_UNSUPPORTED;
+  if (L->has_shared != 0 && L->has_shared != 1) return MOEQ_ERR_INVALID_ARG;
+  if (L->has_shared) {
+    if ((s = check_tensor(&L->sh_gate, 1)) != MOEQ_OK) return s;
+    if ((s = check_tensor(&L->sh_up, 1)) != MOEQ_OK) return s;
+    if ((s = check_tensor(&L->sh_down, 1)) != MOEQ_OK) return s;
+    if ((s = check_tensor(&L->sh_expert_gate, 1)) != MOEQ_OK) return s;
+    const int Is = L->sh_gate.out_dim;
+    if (L->sh_gate.in_dim != H || L->sh_up.in_dim != H || L->sh_up.out_dim != Is)
+      return MOEQ_ERR_INVALID_ARG;
+    if (L->sh_down.out_dim != H || L->sh_down.in_dim != Is) return MOEQ_ERR_INVALID_ARG;
+    if (L->sh_expert_gate.out_dim != 1 || L->sh_expert_gate.in_dim != H)
+      return MOEQ_ERR_INVALID_ARG;
+    if (L->sh_gate.bits != L->sh_up.bits || L->sh_gate.group_size != L->sh_up.group_size)
+      return MOEQ_ERR_UNSUPPORTED;
+  }
+  return MOEQ_OK;
+}
+
+static moeq_status check_decode_shapes(const moeq_layer* L) {
+  const moeq_qtensor* ts[8] = {&L->router, &L->gate, &L->down, &L->sh_gate, &L->sh_down,
+                               &L->sh_expert_gate, nullptr, nullptr};
+  const int n = L->has_shared ? 6 : 3;
+  for (int i = 0; i < n; ++i)
+    if (slices_of(*ts[i]) > 8) return MOEQ_ERR_UNSUPPORTED;
+  return MOEQ_OK;
+}
+
+// ------------------------------------------------------------------ workspace layout
+namespace {
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~(size_t)255;
+    return o;
+  }
+};
+
+struct DecodeWs {
+  size_t logits, sg_logit, sigma, idx, w, h, d, segs_gu, segs_dn, counts, vecs_gu, vecs_dn, total;
+};
+
+DecodeWs decode_ws(const moeq_layer* L, int M) {
+  const int E = L->n_experts, K = L->top_k, H = L->hidden, I = L->inter;
+  const int Is = L->has_shared ? L->sh_gate.out_dim : 0;
+  const size_t n = (size_t)M * K;
+  Carve c;
+  DecodeWs w;
+  w.logits = c.take((size_t)M * E * 4);
+  w.sg_logit = c.take((size_t)M * 4);
+  w.sigma = c.take((size_t)M * 4);
+  w.idx = c.take(n * 4);
+  w.w = c.take(n * 4);
+  w.h = c.take((n * I + (size_t)M * Is) * 4);
+  w.d = c.take((n + (size_t)M) * H * 4);
+  w.segs_gu = c.take((n + 1) * sizeof(Seg));
+  w.segs_dn = c.take((n + 1) * sizeof(Seg));
+  w.counts = c.take(8 * 4);
+  w.vecs_gu = c.take(n * sizeof(VecRef));
+  w.vecs_dn = c.take(n * sizeof(VecRef));
+  w.total = c.off;
+  return w;
+}
+}  // namespace
+
+static int resolve_mode(int mode, int M) {
+  if (mode == MOEQ_MODE_AUTO) return M <= kMaxDecodeM ? MOEQ_MODE_DECODE : MOEQ_MODE_PREFILL;
+  return mode;
+}
+
+// ------------------------------------------------------------------ GEMV helpers
+static constexpr int kR = 8;  // rows per warp-task on the decode path
+
+static int units_for(int out_dim, int slices) {
+  const GemvShape sh = gemv_shape(slices, kR);
+  const int rows = sh.R * sh.rbs;
+  return (out_dim + rows - 1) / rows;
+}
+
+static int grid_cap() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    sms = n;
+  }
+  return sms * 2;
+}
+
+// x [M][in] (bf16) times one matrix -> y with row stride `ystride`.
+static Seg plain_seg(const moeq_qtensor& t, int expert, const void* src, int64_t src_stride,
+                     float* dst, int64_t dst_stride, int n_vec, int unit_begin) {
+  Seg s;
+  memset(&s, 0, sizeof(s));
+  const uint32_t* w = t.w + (int64_t)expert * t.expert_stride_w;
+  const uint16_t* sc = t.scales + (int64_t)expert * t.expert_stride_sb;
+  const uint16_t* bi = t.biases + (int64_t)expert * t.expert_stride_sb;
+  s.w[0] = s.w[1] = w;
+  s.s[0] = s.s[1] = sc;
+  s.b[0] = s.b[1] = bi;
+  s.out_dim = t.out_dim;
+  s.in_dim = t.in_dim;
+  s.G = t.group_size;
+  s.n_vec = n_vec;
+  s.unit_begin = unit_begin;
+  s.vec_mode = 0;
+  s.src_base = src;
+  s.src_stride = src_stride;
+  s.dst_base = dst;
+  s.dst_stride = dst_stride;
+  s.vecs = nullptr;
+  return s;
+}
+
+static cudaError_t run_plain(const Seg* segs, int n, int bits, int nl, int slices,
+                             cudaStream_t st) {
+  GemvArgs a;
+  memset(&a, 0, sizeof(a));
+  int units = 0;
+  for (int i = 0; i < n; ++i) {
+    a.segs[i] = segs[i];
+    a.segs[i].unit_begin = units;
+    units += units_for(segs[i].out_dim, slices);
+  }
+  a.n_segs = n;
+  a.total_units = units;
+  a.slices = slices;
+  a.status = status_ptr();
+  const int grid = units < grid_cap() ? units : grid_cap();
+  return launch_gemv(bits, nl, 1, kR, SRC_BF16, a, grid, st);
+}
+
+static cudaError_t run_dyn(const Seg* segs, const int32_t* count, int bits, int nl, int nmat,
+                           int src, int slices, int max_units, cudaStream_t st) {
+  GemvArgs a;
+  memset(&a, 0, sizeof(a));
+  a.dyn_segs = segs;
+  a.dyn_count = count;
+  a.slices = slices;
+  a.status = status_ptr();
+  const int grid = max_units < grid_cap() ? max_units : grid_cap();
+  return launch_gemv(bits, nl, nmat, kR, src, a, grid, st);
+}
+
+#define CK(x)                                     \
+  do {                                            \
+    if ((x) != cudaSuccess) return MOEQ_ERR_CUDA; \
+  } while (0)
+// one kernel launch through the library
+#define LAUNCH(x)          \
+  do {                     \
+    CK(x);                 \
+    count_launches(1);     \
+  } while (0)
+
+// ------------------------------------------------------------------ decode path
+static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
+                                  const int32_t* idx_in, const float* w_in, const float* residual,
+                                  float* y, int32_t* idx_out, float* w_out, void* ws,
+                                  cudaStream_t st) {
+  const int E = L->n_experts, K = L->top_k, H = L->hidden, I = L->inter;
+  const int n = M * K;
+  const DecodeWs lay = decode_ws(L, M);
+  char* base = (char*)ws;
+  float* logits = (float*)(base + lay.logits);
+  float* sg_logit = (float*)(base + lay.sg_logit);
+  float* sigma = (float*)(base + lay.sigma);
+  int32_t* idx = idx_out ? idx_out : (int32_t*)(base + lay.idx);
+  float* wts = w_out ? w_out : (float*)(base + lay.w);
+  float* h = (float*)(base + lay.h);
+  float* d = (float*)(base + lay.d);
+  Seg* segs_gu = (Seg*)(base + lay.segs_gu);
+  Seg* segs_dn = (Seg*)(base + lay.segs_dn);
+  int32_t* counts = (int32_t*)(base + lay.counts);
+  VecRef* vecs_gu = (VecRef*)(base + lay.vecs_gu);
+  VecRef* vecs_dn = (VecRef*)(base + lay.vecs_dn);
+
+  // 1. router logits and the shared-expert gate logit (one launch when the
+  //    two 8-bit tensors agree in format)
+  const moeq_qtensor& R = L->router;
+  const moeq_qtensor& SG = L->sh_expert_gate;
+  const int sr = slices_of(R);
+  const bool sg_with_router = L->has_shared && SG.bits == R.bits && slices_of(SG) == sr;
+  if (!idx_in) {
+    Seg segs[2];
+    int ns = 0;
+    segs[ns++] = plain_seg(R, 0, x, H, logits, E, M, 0);
+    if (sg_with_router) segs[ns++] = plain_seg(SG, 0, x, H, sg_logit, 1, M, 0);
+    LAUNCH(run_plain(segs, ns, R.bits, 3, sr, st));
+  }
+  if (L->has_shared && (idx_in || !sg_with_router)) {
+    Seg s = plain_seg(SG, 0, x, H, sg_logit, 1, M, 0);
+    LAUNCH(run_plain(&s, 1, SG.bits, 3, slices_of(SG), st));
+  }
+
+  // 2. routing + grouped plan
+  DecodePlanArgs p;
+  memset(&p, 0, sizeof(p));
+  p.logits = idx_in ? nullptr : logits;
+  p.sg_logit = L->has_shared ? sg_logit : nullptr;
+  p.idx_in = idx_in;
+  p.w_in = w_in;
+  p.M = M;
+  p.E = E;
+  p.K = K;
+  p.renorm = L->renorm;
+  p.router_scale = L->router_scale;
+  p.idx_out = idx;
+  p.w_out = wts;
+  p.x = x;
+  p.H = H;
+  p.I = I;
+  p.has_shared = L->has_shared;
+  p.gate = L->gate;
+  p.up = L->up;
+  p.down = L->down;
+  if (L->has_shared) {
+    p.sh_gate = L->sh_gate;
+    p.sh_up = L->sh_up;
+    p.sh_down = L->sh_down;
+  }
+  p.h = h;
+  p.d = d;
+  p.sigma = sigma;
+  p.segs_gu = segs_gu;
+  p.count_gu = counts;
+  p.segs_dn = segs_dn;
+  p.count_dn = counts + 4;
+  p.vecs_gu = vecs_gu;
+  p.vecs_dn = vecs_dn;
+  const int s_gu = slices_of(L->gate), s_dn = slices_of(L->down);
+  p.units_per_seg_gu = units_for(I, s_gu);
+  p.units_per_seg_dn = units_for(H, s_dn);
+  int s_gu_sh = 0, s_dn_sh = 0;
+  if (L->has_shared) {
+    s_gu_sh = slices_of(L->sh_gate);
+    s_dn_sh = slices_of(L->sh_down);
+    p.units_per_seg_gu_sh = units_for(L->sh_gate.out_dim, s_gu_sh);
+    p.units_per_seg_dn_sh = units_for(H, s_dn_sh);
+    p.shared_same_gu = (L->sh_gate.bits == L->gate.bits && s_gu_sh == s_gu);
+    p.shared_same_dn = (L->sh_down.bits == L->down.bits && s_dn_sh == s_dn);
+  }
+  p.status = status_ptr();
+  LAUNCH(launch_decode_plan(p, st));
+
+  // 3. gate/up + SwiGLU, then 4. down, for the routed experts (+ shared)
+  const int max_entries = n < E ? n : E;
+  const int max_gu = max_entries * p.units_per_seg_gu + (p.shared_same_gu ? p.units_per_seg_gu_sh : 0);
+  const int max_dn = max_entries * p.units_per_seg_dn + (p.shared_same_dn ? p.units_per_seg_dn_sh : 0);
+  CK(profile_mark(true, st));
+  LAUNCH(run_dyn(segs_gu, counts, L->gate.bits, 2, 2, SRC_BF16, s_gu, max_gu, st));
+  CK(profile_mark(false, st));
+  if (L->has_shared && !p.shared_same_gu)
+    LAUNCH(run_dyn(segs_gu + n, counts + 2, L->sh_gate.bits, 2, 2, SRC_BF16, s_gu_sh,
+                   p.units_per_seg_gu_sh, st));
+  LAUNCH(run_dyn(segs_dn, counts + 4, L->down.bits, 2, 1, SRC_F32, s_dn, max_dn, st));
+  if (L->has_shared && !p.shared_same_dn)
+    LAUNCH(run_dyn(segs_dn + n, counts + 6, L->sh_down.bits, 2, 1, SRC_F32, s_dn_sh,
+                   p.units_per_seg_dn_sh, st));
+
+  // 5. weighted combine in k order (+ shared, + residual)
+  LAUNCH(launch_combine(d, wts, sigma, L->has_shared, residual, y, M, K, H, st));
+  return MOEQ_OK;
+}
+
+// ------------------------------------------------------------------ entry points
+MOEQ_API const char* moeq_version(void) { return "moeq 0.1 (sm_100a)"; }
+
+MOEQ_API const char* moeq_status_str(int32_t s) {
+  switch (s) {
+    case MOEQ_OK: return "ok";
+    case MOEQ_ERR_INVALID_ARG: return "invalid argument";
+    case MOEQ_ERR_UNSUPPORTED: return "unsupported format or size";
+    case MOEQ_ERR_ALIGNMENT: return "misaligned pointer or dimension";
+    case MOEQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOEQ_ERR_CUDA: return "CUDA runtime error";
+    case MOEQ_ERR_TIMEOUT: return "device wait timed out";
+    case MOEQ_ERR_RANGE: return "operand outside the fp16 range of the prefill tiles";
+    default: return "unknown status";
+  }
+}
+
+MOEQ_API moeq_status moeq_dequant(const moeq_qtensor* t, int32_t expert, uint8_t* q_out,
+                                  float* w_out, void* stream) {
+  if (!t || (!q_out && !w_out) || expert < 0) return MOEQ_ERR_INVALID_ARG;
+  moeq_status s = check_tensor(t, expert + 1);
+  if (s != MOEQ_OK) return s;
+  if (expert > 0 && (t->expert_stride_w <= 0 || t->expert_stride_sb <= 0))
+    return MOEQ_ERR_INVALID_ARG;
+  LAUNCH(launch_dequant(*t, expert, q_out, w_out, (cudaStream_t)stream));
+  return MOEQ_OK;
+}
+
+MOEQ_API moeq_status moeq_qmv(const moeq_qtensor* t, int32_t expert, const uint16_t* x, int32_t M,
+                              float* y, void* stream) {
+  if (!t || !x || !y || expert < 0 || M <= 0) return MOEQ_ERR_INVALID_ARG;
+  if (M > kMaxDecodeM) return MOEQ_ERR_UNSUPPORTED;
+  moeq_status s = check_tensor(t, expert + 1);
+  if (s != MOEQ_OK) return s;
+  if (expert > 0 && (t->expert_stride_w <= 0 || t->expert_stride_sb <= 0))
+    return MOEQ_ERR_INVALID_ARG;
+  if (slices_of(*t) > 8) return MOEQ_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || ((int64_t)t->in_dim * 2) % 16 || !aligned(y, 4)) return MOEQ_ERR_ALIGNMENT;
+  Seg seg = plain_seg(*t, expert, x, t->in_dim, y, t->out_dim, M, 0);
+  LAUNCH(run_plain(&seg, 1, t->bits, 3, slices_of(*t), (cudaStream_t)stream));
+  return MOEQ_OK;
+}
+
+MOEQ_API moeq_status moeq_route_topk(const float* logits, int32_t M, int32_t E, int32_t K,
+                                     int32_t renorm, float router_scale, int32_t* idx, float* w,
+                                     void* stream) {
+  if (M < 0 || E <= 0 || K <= 0 || K > E) return MOEQ_ERR_INVALID_ARG;
+  if (K > kMaxK || E > kMaxE) return MOEQ_ERR_UNSUPPORTED;
+  if (M == 0) return MOEQ_OK;
+  if (!logits || !idx || !w) return MOEQ_ERR_INVALID_ARG;
+  LAUNCH(launch_route_topk(logits, M, E, K, renorm, router_scale, idx, w, (cudaStream_t)stream));
+  return MOEQ_OK;
+}
+
+MOEQ_API size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mode) {
+  if (check_layer(L) != MOEQ_OK || M <= 0) return 0;
+  mode = resolve_mode(mode, M);
+  if (mode == MOEQ_MODE_DECODE) {
+    if (M > kMaxDecodeM) return 0;
+    return decode_ws(L, M).total;
+  }
+  if (mode == MOEQ_MODE_PREFILL) return prefill_workspace_bytes(L, M);
+  return 0;
+}
+
+static moeq_status forward_common(const moeq_layer* L, const uint16_t* x, int32_t M,
+                                  const int32_t* idx_in, const float* w_in, const float* residual,
+                                  float* y, int32_t* idx_out, float* w_out, void* ws,
+                                  size_t ws_bytes, int32_t mode, void* stream) {
+  moeq_status s = check_layer(L);
+  if (s != MOEQ_OK) return s;
+  if (M < 0 || !x || !y) return MOEQ_ERR_INVALID_ARG;
+  if (M == 0) return MOEQ_OK;
+  if (mode < MOEQ_MODE_AUTO || mode > MOEQ_MODE_PREFILL) return MOEQ_ERR_INVALID_ARG;
+  mode = resolve_mode(mode, M);
+  if (!aligned(x, 16) || (L->hidden * 2) % 16 || !aligned(y, 16) || L->hidden % 4)
+    return MOEQ_ERR_ALIGNMENT;
+  if (residual && !aligned(residual, 16)) return MOEQ_ERR_ALIGNMENT;
+  const size_t need = moeq_workspace_bytes(L, M, mode);
+  if (need == 0) return MOEQ_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < need) return MOEQ_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return MOEQ_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (mode == MOEQ_MODE_DECODE) {
+    if (M > kMaxDecodeM) return MOEQ_ERR_UNSUPPORTED;
+    if ((s = check_decode_shapes(L)) != MOEQ_OK) return s;
+    return decode_forward(L, x, M, idx_in, w_in, residual, y, idx_out, w_out, ws, st);
+  }
+  return prefill_forward(L, x, M, idx_in, w_in, residual, y, idx_out, w_out, ws, ws_bytes,
+                         status_ptr(), st);
+}
+
+MOEQ_API moeq_status moeq_expert_ffn(const moeq_layer* L, const uint16_t* x, int32_t M,
+                                     const int32_t* idx, const float* w, const float* residual,
+                                     float* y, void* ws, size_t ws_bytes, int32_t mode,
+                                     void* stream) {
+  if (M > 0 && (!idx || !w)) return MOEQ_ERR_INVALID_ARG;
+  return forward_common(L, x, M, idx, w, residual, y, nullptr, nullptr, ws, ws_bytes, mode,
+                        stream);
+}
+
+MOEQ_API moeq_status moeq_layer_forward(const moeq_layer* L, const uint16_t* x, int32_t M,
+                                        float* y, const float* residual, int32_t* idx_out,
+                                        float* w_out, void* ws, size_t ws_bytes, int32_t mode,
+                                        void* stream) {
+  return forward_common(L, x, M, nullptr, nullptr, residual, y, idx_out, w_out, ws, ws_bytes,
+                        mode, stream);
+}
+
+MOEQ_API moeq_status moeq_set_profile_events(void* start, void* stop) {
+  if ((start == nullptr) != (stop == nullptr)) return MOEQ_ERR_INVALID_ARG;
+  t_prof_start = (cudaEvent_t)start;
+  t_prof_stop = (cudaEvent_t)stop;
+  return MOEQ_OK;
+}
+
+MOEQ_API uint64_t moeq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+MOEQ_API moeq_status moeq_device_status(void* stream, int32_t* status_out) {
+  if (!status_out) return MOEQ_ERR_INVALID_ARG;
+  int* p = status_ptr();
+  if (!p) return MOEQ_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  int v = 0;
+  CK(cudaMemcpyAsync(&v, p, sizeof(int), cudaMemcpyDeviceToHost, st));
+  CK(cudaMemsetAsync(p, 0, sizeof(int), st));
+  CK(cudaStreamSynchronize(st));
+  *status_out = v;
+  return MOEQ_OK;
+}

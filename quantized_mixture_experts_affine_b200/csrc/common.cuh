@@ -1,0 +1,104 @@
+// Device helpers shared by the layer kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moeq.h"
+
+namespace moeq {
+
+// ------------------------------------------------------------------ limits
+constexpr int kMaxDecodeM = 64;      // tokens per decode call
+constexpr int kMaxK = 32;            // top-K
+constexpr int kMaxE = 4096;          // experts
+constexpr int kXBlock = 32;          // values per fixed-point block of an input vector
+constexpr int kWaitSpins = 1 << 22;  // bounded device-side waits
+
+// ------------------------------------------------------------------ status word
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// ------------------------------------------------------------------ conversions
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+  return __uint_as_float(((uint32_t)h) << 16);
+}
+
+// ------------------------------------------------------------------ loads
+// Streaming 16-byte load of packed weights: read once, do not keep in L1.
+__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t ldg_u16(const uint16_t* p) { return __ldg(p); }
+
+// ------------------------------------------------------------------ integer dot products
+// d = c + sum_i a.byte[i] * b.byte[i]; a unsigned codes, b signed or unsigned limb.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// ------------------------------------------------------------------ warp reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Sum within aligned segments of `width` lanes (power of two <= 32).
+__device__ __forceinline__ float segment_sum(float v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ------------------------------------------------------------------ code registers
+// A 16-byte chunk of a packed row holds VPC = 128/BITS codes in 4 words.
+// It is split into NC = VPC/4 "code registers", each holding 4 codes in its
+// 4 bytes, ready for dp4a:
+//   BITS 8: reg k      = word k                      (values 4k .. 4k+3)
+//   BITS 4: reg 2k     = word k & 0x0F0F0F0F         (values 8k + 0,2,4,6)
+//           reg 2k+1   = (word k >> 4) & 0x0F0F0F0F  (values 8k + 1,3,5,7)
+//   BITS 2: reg 4k+i   = (word k >> 2i) & 0x03030303 (values 16k + i + 0,4,8,12)
+// value_of(BITS, reg, byte) gives the position of a code within the chunk.
+template <int BITS>
+struct Chunk {
+  static constexpr int VPC = 128 / BITS;  // values per chunk
+  static constexpr int NC = VPC / 4;      // code registers per chunk
+  static constexpr int NBLK = VPC >= kXBlock ? VPC / kXBlock : 1;  // x blocks touched
+  __host__ __device__ static constexpr int value_of(int reg, int byte) {
+    return BITS == 8 ? reg * 4 + byte
+         : BITS == 4 ? (reg >> 1) * 8 + (reg & 1) + 2 * byte
+                     : (reg >> 2) * 16 + (reg & 3) + 4 * byte;
+  }
+  __device__ __forceinline__ static void split(const uint4& w, uint32_t (&c)[NC]) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (BITS == 8) {
+        c[k] = ws[k];
+      } else if (BITS == 4) {
+        c[2 * k] = ws[k] & 0x0F0F0F0Fu;
+        c[2 * k + 1] = (ws[k] >> 4) & 0x0F0F0F0Fu;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[4 * k + i] = (ws[k] >> (2 * i)) & 0x03030303u;
+      }
+    }
+  }
+};
+
+}  // namespace moeq

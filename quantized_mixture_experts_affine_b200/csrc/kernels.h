@@ -1,0 +1,115 @@
+// Host-side launchers shared between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moeq.h"
+
+namespace moeq {
+
+// Diagnostics (api.cu): launch counter and the optional profiling events.
+void count_launches(int n);
+cudaError_t profile_mark(bool start, cudaStream_t st);
+
+// ------------------------------------------------------------------ GEMV segments
+// One vector of a segment: its source row and its output row.
+struct VecRef {
+  const void* src;  // bf16 row (x) or fp32 row (h), in_dim values
+  float* dst;       // fp32 output row, out_dim values
+};
+
+// A run of rows of one or two matrices (gate and up) multiplied with a set
+// of vectors.  Vectors are either strided (src_base + i*src_stride) or an
+// explicit VecRef list.
+struct Seg {
+  const uint32_t* w[2];
+  const uint16_t* s[2];
+  const uint16_t* b[2];
+  int32_t out_dim;
+  int32_t in_dim;
+  int32_t G;
+  int32_t n_vec;
+  int32_t unit_begin;  // first work unit of this segment
+  int32_t vec_mode;    // 0 strided, 1 list
+  const void* src_base;
+  int64_t src_stride;  // elements
+  float* dst_base;
+  int64_t dst_stride;  // elements
+  const VecRef* vecs;
+};
+
+constexpr int kInlineSegs = 4;
+
+struct GemvArgs {
+  Seg segs[kInlineSegs];    // used when dyn_segs == nullptr
+  int32_t n_segs;
+  int32_t total_units;      // used when dyn_segs == nullptr
+  const Seg* dyn_segs;      // device list written by the decode plan
+  const int32_t* dyn_count; // [0] = number of segments, [1] = total units
+  int32_t slices;           // S: 32-chunk slices per row
+  int* status;
+};
+
+enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
+enum GemvSrc { SRC_BF16 = 0, SRC_F32 = 1 };
+
+// Rows per warp-task and row blocks per CTA for a given slice count.
+struct GemvShape {
+  int R;        // rows per row block (8, 16 or 32)
+  int warps;    // warps per CTA
+  int rbs;      // row blocks per CTA iteration
+};
+GemvShape gemv_shape(int slices, int R);
+
+cudaError_t launch_gemv(int bits, int nl, int nmat, int R, int src, const GemvArgs& a, int grid,
+                        cudaStream_t st);
+
+// ------------------------------------------------------------------ routing
+cudaError_t launch_route_topk(const float* logits, int M, int E, int K, int renorm, float scale,
+                              int32_t* idx, float* w, cudaStream_t st);
+
+// Decode plan: top-K for M tokens, then the grouped work lists for the
+// gate/up and down GEMVs (one segment per distinct expert, plus the shared
+// expert), written into `plan` (device workspace).
+struct DecodePlanArgs {
+  const float* logits;      // [M][E] fp32, or null when idx/w are given
+  const float* sg_logit;    // [M] shared-gate logit, or null
+  const int32_t* idx_in;    // [M][K] when logits == null
+  const float* w_in;
+  int32_t M, E, K, renorm;
+  float router_scale;
+  int32_t* idx_out;         // [M][K]
+  float* w_out;             // [M][K]
+  const uint16_t* x;        // [M][H] bf16
+  int32_t H, I;
+  int32_t has_shared;
+  moeq_qtensor gate, up, down, sh_gate, sh_up, sh_down;
+  float* h;                 // [(M*K + M)][I] fp32 hidden rows (pairs, then shared rows)
+  float* d;                 // [(M*K + M)][H] fp32 down rows
+  float* sigma;             // [M] sigmoid gate values
+  Seg* segs_gu;             // gate/up segments
+  int32_t* count_gu;        // [4]: segs, units; separate shared list: segs, units
+  Seg* segs_dn;             // down segments
+  int32_t* count_dn;        // [4]
+  VecRef* vecs_gu;          // [(M*K + M)]
+  VecRef* vecs_dn;
+  int32_t units_per_seg_gu; // computed on the host from the shapes
+  int32_t units_per_seg_dn;
+  int32_t units_per_seg_gu_sh;
+  int32_t units_per_seg_dn_sh;
+  int32_t shared_same_gu;   // 1: the shared gate/up segment joins the routed launch
+  int32_t shared_same_dn;   // 1: the shared down segment joins the routed launch
+  int* status;
+};
+cudaError_t launch_decode_plan(const DecodePlanArgs& a, cudaStream_t st);
+
+// Codes and/or fp32 weights of one matrix.
+cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, float* w_out,
+                           cudaStream_t st);
+
+// y[t] = sum_k w[t][k] * d[t*K + k] + sigma[t] * d[M*K + t] + residual[t]
+cudaError_t launch_combine(const float* d, const float* w, const float* sigma, int has_shared,
+                           const float* residual, float* y, int M, int K, int H, cudaStream_t st);
+
+}  // namespace moeq

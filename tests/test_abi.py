@@ -1,0 +1,138 @@
+"""The C ABI loads, exports every declared symbol, and rejects bad arguments
+on the host before launching anything (no GPU needed: every call here fails
+its argument checks; fake device addresses are never dereferenced)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from quantized_mixture_experts_affine_b200 import moeq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moeq.h")
+
+A = 1 << 20  # fake, 256-byte aligned device address (never dereferenced)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moeq_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert set(moeq.EXPORTS) <= set(names) and len(names) >= 9
+    lib = C.CDLL(moeq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for s in range(8):
+        assert moeq.status_str(s) and moeq.status_str(s) != "unknown status"
+    assert moeq.status_str(99) == "unknown status"
+    assert "sm_100a" in moeq.version()
+
+
+def qt(out=128, inn=256, bits=4, G=64, w=A, s=A, b=A, n_mats=1):
+    return moeq.qtensor(w, s, b, out, inn, bits, G, n_mats)
+
+
+def rc_qmv(t, M=1, x=A, y=A, expert=0):
+    return moeq.lib().moeq_qmv(C.byref(t), expert, x, M, y, None)
+
+
+def test_qmv_argument_checks():
+    assert rc_qmv(qt(bits=3)) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(G=48)) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(inn=96, G=64)) == moeq.ERR_ALIGNMENT
+    assert rc_qmv(qt(w=A + 4)) == moeq.ERR_ALIGNMENT
+    assert rc_qmv(qt(), x=A + 2) == moeq.ERR_ALIGNMENT
+    assert rc_qmv(qt(w=0)) == moeq.ERR_INVALID_ARG
+    assert rc_qmv(qt(), M=0) == moeq.ERR_INVALID_ARG
+    assert rc_qmv(qt(), M=65) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(), expert=-1) == moeq.ERR_INVALID_ARG
+    assert rc_qmv(qt(inn=16384, bits=8)) == moeq.ERR_UNSUPPORTED   # > 8 slices of 512 B
+    assert moeq.lib().moeq_qmv(None, 0, A, 1, A, None) == moeq.ERR_INVALID_ARG
+
+
+def test_dequant_argument_checks():
+    lib = moeq.lib()
+    assert lib.moeq_dequant(C.byref(qt()), 0, None, None, None) == moeq.ERR_INVALID_ARG
+    assert lib.moeq_dequant(C.byref(qt(bits=5)), 0, A, None, None) == moeq.ERR_UNSUPPORTED
+    # expert > 0 needs expert strides
+    assert lib.moeq_dequant(C.byref(qt()), 1, A, None, None) == moeq.ERR_INVALID_ARG
+
+
+def test_route_argument_checks():
+    lib = moeq.lib()
+    assert lib.moeq_route_topk(A, 4, 8, 9, 1, 1.0, A, A, None) == moeq.ERR_INVALID_ARG
+    assert lib.moeq_route_topk(A, 4, 64, 33, 1, 1.0, A, A, None) == moeq.ERR_UNSUPPORTED
+    assert lib.moeq_route_topk(A, 4, 5000, 4, 1, 1.0, A, A, None) == moeq.ERR_UNSUPPORTED
+    assert lib.moeq_route_topk(A, -1, 8, 2, 1, 1.0, A, A, None) == moeq.ERR_INVALID_ARG
+    assert lib.moeq_route_topk(A, 0, 8, 2, 1, 1.0, None, None, None) == moeq.OK  # nothing to do
+    assert lib.moeq_route_topk(None, 3, 8, 2, 1, 1.0, A, A, None) == moeq.ERR_INVALID_ARG
+
+
+def layer(H=256, I=128, E=8, K=2, bits=4, shared=False):
+    L = moeq.Layer()
+    L.router = qt(E, H, 8)
+    L.gate = qt(I, H, bits, n_mats=E)
+    L.up = qt(I, H, bits, n_mats=E)
+    L.down = qt(H, I, bits, n_mats=E)
+    L.has_shared = int(shared)
+    if shared:
+        L.sh_gate, L.sh_up, L.sh_down = qt(I, H, bits), qt(I, H, bits), qt(H, I, bits)
+        L.sh_expert_gate = qt(1, H, 8)
+    L.hidden, L.inter, L.n_experts, L.top_k, L.renorm, L.router_scale = H, I, E, K, 1, 1.0
+    return L
+
+
+def test_workspace_bytes():
+    L = layer()
+    assert moeq.moeq_workspace_bytes(L, 1, moeq.MODE_DECODE) > 0
+    assert moeq.moeq_workspace_bytes(L, 65, moeq.MODE_DECODE) == 0
+    assert moeq.moeq_workspace_bytes(L, 0, moeq.MODE_DECODE) == 0
+    Ls = layer(shared=True)
+    assert moeq.moeq_workspace_bytes(Ls, 5, moeq.MODE_DECODE) > moeq.moeq_workspace_bytes(L, 5, moeq.MODE_DECODE)
+    bad = layer()
+    bad.top_k = 9
+    assert moeq.moeq_workspace_bytes(bad, 1, moeq.MODE_DECODE) == 0
+    bad = layer()
+    bad.down = qt(255, 128, 4, n_mats=8)  # down must be [H][I]
+    assert moeq.moeq_workspace_bytes(bad, 1, moeq.MODE_DECODE) == 0
+
+
+def fwd(L, M=1, x=A, y=A, ws=A, ws_bytes=None, mode=moeq.MODE_DECODE):
+    if ws_bytes is None:
+        ws_bytes = moeq.moeq_workspace_bytes(L, max(M, 1), mode) - 256
+    return moeq.lib().moeq_layer_forward(C.byref(L), x, M, y, None, None, None, ws, ws_bytes,
+                                         mode, None)
+
+
+def test_forward_argument_checks():
+    L = layer()
+    assert fwd(L) == moeq.ERR_WORKSPACE                 # workspace too small
+    assert fwd(L, ws=None, ws_bytes=1 << 30) == moeq.ERR_WORKSPACE
+    assert fwd(L, x=A + 2, ws_bytes=1 << 30) == moeq.ERR_ALIGNMENT
+    assert fwd(L, ws=A + 16, ws_bytes=1 << 30) == moeq.ERR_ALIGNMENT
+    assert fwd(L, mode=7, ws_bytes=1 << 30) == moeq.ERR_INVALID_ARG
+    assert fwd(L, M=0) == moeq.OK                       # nothing to do
+    assert fwd(L, M=-1) == moeq.ERR_INVALID_ARG
+    assert fwd(L, M=65, ws_bytes=1 << 30) == moeq.ERR_UNSUPPORTED  # decode limit
+    bad = layer()
+    bad.gate = qt(128, 256, 3, n_mats=8)
+    assert fwd(bad, ws_bytes=1 << 30) == moeq.ERR_UNSUPPORTED
+    bad = layer()
+    bad.n_experts = 4                                    # router rows != E
+    assert fwd(bad, ws_bytes=1 << 30) == moeq.ERR_INVALID_ARG
+    lib = moeq.lib()
+    # expert_ffn needs the routing
+    assert lib.moeq_expert_ffn(C.byref(L), A, 2, None, None, None, A, A, 1 << 30,
+                               moeq.MODE_DECODE, None) == moeq.ERR_INVALID_ARG
+
+
+def test_device_status_needs_output():
+    assert moeq.lib().moeq_device_status(None, None) == moeq.ERR_INVALID_ARG

@@ -1,0 +1,212 @@
+"""Decode path on the GPU against the fp64 oracle (through the C ABI).
+
+Bars: unpacked codes and dequantised fp32 weights bit-exact; qmv relative
+L2 <= 1e-5 (24-bit fixed-point input, fp32 sums); routing equal except at
+near-ties; layer outputs relative L2 <= 2e-3 and max abs <= 1e-2.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import check_layer_outputs, rel_l2, NEAR_TIE
+from quantized_mixture_experts_affine_b200 import moeq, synth
+from quantized_mixture_experts_affine_b200.layer import (CONFIGS, expert_ffn, layer_forward,
+                                                         synthetic_layer, Workspace)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+SEED = 0
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def x_tokens(cfg, M, copy=0, seed=SEED):
+    xb = synth.normal_bf16_host(seed, synth.tag(synth.X, copy), M * cfg.H).reshape(M, cfg.H)
+    return xb, dev(xb.view(np.int16)).view(torch.bfloat16)
+
+
+# ------------------------------------------------------------------ generator
+
+@pytest.mark.parametrize("bits,G,rq", [(2, 64, False), (4, 64, False), (8, 64, False),
+                                       (2, 64, True), (4, 32, False), (8, 128, False)])
+def test_device_generator_matches_host(bits, G, rq):
+    tg = synth.tag(synth.GATE, 3)
+    d = synth.tensor_dev(7, tg, 3, 40, 512, bits, G, rq).to_host()
+    h = synth.tensor_host(7, tg, 3, 40, 512, bits, G, rq)
+    assert np.array_equal(d.w, h.w) and np.array_equal(d.s, h.s) and np.array_equal(d.b, h.b)
+    xd = synth.normal_bf16_dev(7, synth.tag(synth.X), 10001).cpu().view(torch.int16).numpy()
+    assert np.array_equal(xd.view(np.uint16), synth.normal_bf16_host(7, synth.tag(synth.X), 10001))
+
+
+# ------------------------------------------------------------------ dequant
+
+@pytest.mark.parametrize("bits,G", [(2, 64), (4, 64), (8, 64), (4, 32), (8, 128), (2, 128)])
+def test_dequant_bit_exact(bits, G):
+    q = synth.tensor_dev(SEED, synth.tag(synth.UP, bits), 3, 72, 512, bits, G)
+    t = moeq.qtensor(q.w, q.s, q.b, 72, 512, bits, G, 3)
+    host = q.to_host()
+    for e in (0, 2):
+        codes = torch.empty((72, 512), dtype=torch.uint8, device="cuda")
+        w = torch.empty((72, 512), dtype=torch.float32, device="cuda")
+        moeq.moeq_dequant(t, e, codes, w)
+        torch.cuda.synchronize()
+        assert np.array_equal(codes.cpu().numpy(), oracle.unpack(host, e))
+        assert np.array_equal(w.cpu().numpy().view(np.uint32),
+                              oracle.dequant_f32(host, e).view(np.uint32))
+    assert moeq.moeq_device_status() == 0
+
+
+# ------------------------------------------------------------------ qmv
+
+QMV_CASES = [  # (bits, G, out, in, M, requant)
+    (8, 64, 128, 2816, 1, False),    # standalone router 2816 -> 128
+    (8, 64, 512, 4096, 3, False),    # 397B-like router
+    (4, 64, 1024, 4096, 2, False),
+    (2, 64, 1024, 4096, 1, True),
+    (4, 64, 4096, 1024, 5, False),
+    (8, 32, 130, 256, 64, False),    # ragged rows, max decode M
+    (4, 128, 96, 768, 7, False),
+    (2, 32, 33, 128, 4, False),
+]
+
+
+@pytest.mark.parametrize("bits,G,out,inn,M,rq", QMV_CASES)
+def test_qmv_parity(bits, G, out, inn, M, rq):
+    tg = synth.tag(synth.ROUTER, 100 + bits)
+    q = synth.tensor_dev(SEED, tg, 2, out, inn, bits, G, rq)
+    t = moeq.qtensor(q.w, q.s, q.b, out, inn, bits, G, 2)
+    xb = synth.normal_bf16_host(SEED, synth.tag(synth.X, 5), M * inn).reshape(M, inn)
+    x = dev(xb.view(np.int16))
+    host = q.to_host()
+    for e in (0, 1):
+        y = torch.full((M, out), float("nan"), device="cuda")
+        moeq.moeq_qmv(t, e, x, M, y)
+        torch.cuda.synchronize()
+        ref = oracle.qmv(host, xb, mat=e)
+        assert rel_l2(y.cpu().numpy(), ref) <= 1e-5, rel_l2(y.cpu().numpy(), ref)
+    assert moeq.moeq_device_status() == 0
+
+
+# ------------------------------------------------------------------ routing
+
+@pytest.mark.parametrize("M,E,K,renorm,scale", [(37, 128, 8, True, 1.0), (5, 512, 4, True, 1.0),
+                                                (64, 8, 2, False, 0.5), (3, 4096, 32, True, 2.0),
+                                                (1, 16, 16, True, 1.0)])
+def test_route_topk_parity(M, E, K, renorm, scale):
+    logits, _ = synth.zipf_logits_host(SEED, synth.tag(synth.LOGITS, E), M, E, 1.1)
+    lg = dev(logits)
+    idx = torch.empty((M, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    moeq.moeq_route_topk(lg, M, E, K, renorm, scale, idx, w)
+    torch.cuda.synchronize()
+    # the decision is taken on the same fp32 logits on both sides
+    io, wo, gap = oracle.route_f32(logits, K, renorm, scale)
+    ig, wg = idx.cpu().numpy(), w.cpu().numpy()
+    for t in range(M):
+        if not np.array_equal(ig[t], io[t]):
+            assert gap[t] < NEAR_TIE or set(ig[t]) == set(io[t]), (t, ig[t], io[t], gap[t])
+    assert np.abs(wg - wo).max() < 2e-6
+    if renorm:
+        assert np.allclose(wg.sum(1), 1.0, atol=1e-6)
+    assert (np.diff(wg, axis=1) <= 1e-7).all()
+
+
+def test_route_ties_lower_index():
+    logits = np.zeros((2, 8), np.float32)
+    logits[1, 3] = 1.0
+    idx = torch.empty((2, 3), dtype=torch.int32, device="cuda")
+    w = torch.empty((2, 3), dtype=torch.float32, device="cuda")
+    moeq.moeq_route_topk(dev(logits), 2, 8, 3, True, 1.0, idx, w)
+    assert idx.cpu().numpy().tolist() == [[0, 1, 2], [3, 0, 1]]
+    assert np.allclose(w.cpu().numpy()[0], 1 / 3)
+
+
+# ------------------------------------------------------------------ layer forward (decode)
+
+def run_decode(cfg_name, Ms, copy=0, residual=False):
+    cfg = CONFIGS[cfg_name]
+    L = synthetic_layer(cfg, SEED, copy)
+    out = []
+    for M in Ms:
+        xb, x = x_tokens(cfg, M, copy=M)
+        res = None
+        res_np = None
+        if residual:
+            res_np = np.linspace(-1, 1, M * cfg.H, dtype=np.float32).reshape(M, cfg.H)
+            res = dev(res_np)
+        y = torch.full((M, cfg.H), float("nan"), device="cuda")
+        y, idx, w = layer_forward(L, x, y=y, residual=res, mode=moeq.MODE_DECODE)
+        torch.cuda.synchronize()
+        assert moeq.moeq_device_status() == 0
+        r = check_layer_outputs(cfg, SEED, copy, xb, y.cpu().numpy(), idx.cpu().numpy(),
+                                w.cpu().numpy(), residual=res_np)
+        out.append(r)
+    return out
+
+
+def test_decode_tiny():
+    run_decode("tiny", [1, 3, 5])
+
+
+def test_decode_tiny_residual():
+    run_decode("tiny", [3], residual=True)
+
+
+def test_decode_30b_like():
+    run_decode("decode_30b", [1, 4])
+
+
+def test_decode_397b_like():
+    run_decode("decode_397b", [1, 8])
+
+
+@pytest.mark.slow
+def test_decode_397b_like_batch64():
+    run_decode("decode_397b", [64])
+
+
+def test_decode_mixed_2bit():
+    run_decode("mixed_2bit", [1, 3])
+
+
+def test_expert_ffn_zipf_routing_decode():
+    """Mixed bank with router logits drawn for a skewed (Zipf 1.1) expert load."""
+    cfg = CONFIGS["mixed_2bit"]
+    L = synthetic_layer(cfg, SEED, 0)
+    M = 64
+    logits, _ = synth.zipf_logits_host(SEED, synth.tag(synth.LOGITS), M, cfg.E, 1.1)
+    idx = torch.empty((M, cfg.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((M, cfg.K), dtype=torch.float32, device="cuda")
+    moeq.moeq_route_topk(dev(logits), M, cfg.E, cfg.K, True, 1.0, idx, w)
+    xb, x = x_tokens(cfg, M, copy=11)
+    y = expert_ffn(L, x, idx, w, mode=moeq.MODE_DECODE)
+    torch.cuda.synchronize()
+    from helpers import oracle_expert_outputs
+    ig = idx.cpu().numpy()
+    # weights in fp64 from the same drawn logits
+    io, wo, _ = oracle.route_f32(logits, cfg.K, True, 1.0)
+    assert np.array_equal(np.sort(ig, 1), np.sort(io, 1))
+    rows = np.arange(0, M, 4)
+    ref = oracle_expert_outputs(cfg, SEED, 0, xb[rows], ig[rows], wo[rows])
+    got = y.cpu().numpy()[rows]
+    assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
+
+
+def test_workspace_reuse_and_poison():
+    """Two calls into the same workspace, outputs poisoned with two values,
+    agree bitwise (no unwritten rows, no dependence on stale workspace)."""
+    cfg = CONFIGS["decode_30b"]
+    L = synthetic_layer(cfg, SEED, 0)
+    xb, x = x_tokens(cfg, 4, copy=3)
+    ws = Workspace(L, 4, moeq.MODE_DECODE)
+    ys = []
+    for poison in (float("nan"), 1e30):
+        ws.buf.fill_(0xA5)
+        y = torch.full((4, cfg.H), poison, device="cuda")
+        layer_forward(L, x, y=y, ws=ws, mode=moeq.MODE_DECODE)
+        ys.append(y.cpu().numpy())
+    assert np.isfinite(ys[0]).all()
+    assert np.array_equal(ys[0].view(np.uint32), ys[1].view(np.uint32))
