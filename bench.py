@@ -32,6 +32,8 @@ sys.path.insert(0, ROOT)
 WORKLOADS = {
     # name: (config, tokens per step)
     "decode_397b_m1": ("decode_397b", 1),
+    # same shapes with a 16-expert bank: small enough for full ncu captures
+    "decode_397b_e16_m1": ("decode_397b_e16", 1),
     "decode_397b_m8": ("decode_397b", 8),
     "decode_30b_m1": ("decode_30b", 1),
     "decode_mixed_2bit_m1": ("mixed_2bit", 1),
@@ -47,9 +49,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_397b_m1", choices=sorted(WORKLOADS))
     ap.add_argument("--copies", type=int, default=8)
-    ap.add_argument("--cpu-sample", type=int, default=16,
+    ap.add_argument("--cpu-sample", type=int, default=8,
                     help="tokens of the bounded oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
@@ -147,31 +150,42 @@ def measured_peaks():
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def cpu_oracle_sample(cfg, n_tokens, seed=0):
-    """The oracle as it stands on a bounded sample: n_tokens single-token
-    forwards of the workload's layer (router, routing, K experts, shared
-    expert), all host cores.  Returns (tokens/s, cores, seconds)."""
-    import numpy as np
-    import oracle
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from helpers import oracle_layer, host_router
-    from quantized_mixture_experts_affine_b200 import synth
-    xb = synth.normal_bf16_host(seed, synth.tag(synth.X, 9999), n_tokens * cfg.H).reshape(
-        n_tokens, cfg.H)
-    R = host_router(cfg, seed, 0)
-    logits = oracle.qmv(R, xb)
-    idx, w, _ = oracle.route(logits, cfg.K, cfg.renorm, cfg.router_scale)
-    experts = np.unique(idx)
-    L = oracle_layer(cfg, seed, 0, experts)           # host weights: not timed
-    remap = {int(e): i for i, e in enumerate(experts)}
-    idx_c = np.vectorize(lambda e: remap[int(e)])(idx).astype(np.int32)
-    cores = oracle.get_threads()
-    t0 = time.perf_counter()
-    logits = oracle.qmv(R, xb)
-    oracle.route(logits, cfg.K, cfg.renorm, cfg.router_scale)
-    oracle.expert_ffn(L, xb, idx_c, w)
-    dt = time.perf_counter() - t0
-    return n_tokens / dt, cores, dt
+class OracleSample:
+    """The oracle as it stands, on a bounded sample of the workload: n_tokens
+    tokens with their router, routed experts and shared expert generated on
+    the host once (not timed).  run(tokens) times the oracle's router qmv,
+    routing and experts + combine for those tokens on all host cores."""
+
+    def __init__(self, cfg, n_tokens, seed=0):
+        import numpy as np
+        import oracle
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from helpers import oracle_layer, host_router
+        from quantized_mixture_experts_affine_b200 import synth
+        self.cfg, self.oracle, self.np = cfg, oracle, np
+        self.xb = synth.normal_bf16_host(seed, synth.tag(synth.X, 9999),
+                                         n_tokens * cfg.H).reshape(n_tokens, cfg.H)
+        self.R = host_router(cfg, seed, 0)
+        logits = oracle.qmv(self.R, self.xb)
+        idx, self.w, _ = oracle.route(logits, cfg.K, cfg.renorm, cfg.router_scale)
+        experts = np.unique(idx)
+        self.L = oracle_layer(cfg, seed, 0, experts)
+        remap = {int(e): i for i, e in enumerate(experts)}
+        self.idx_c = np.vectorize(lambda e: remap[int(e)])(idx).astype(np.int32)
+        self.threads = oracle.get_threads()
+
+    def cores(self, n_rows):
+        """Threads the oracle actually uses for n_rows tokens (it splits tokens)."""
+        return min(self.threads, n_rows)
+
+    def run(self, rows):
+        o, c = self.oracle, self.cfg
+        x = self.xb[rows]
+        t0 = time.perf_counter()
+        logits = o.qmv(self.R, x)
+        o.route(logits, c.K, c.renorm, c.router_scale)
+        o.expert_ffn(self.L, x, self.idx_c[rows], self.w[rows])
+        return time.perf_counter() - t0
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)
@@ -182,23 +196,26 @@ def run_reference(args):
     from quantized_mixture_experts_affine_b200.layer import CONFIGS
     cfg_name, M = WORKLOADS[args.workload]
     cfg = CONFIGS[cfg_name]
-    # each step: one bounded sample of M tokens of the workload
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        cpu_oracle_sample(cfg, M)
-    times = []
-    cores = 0
+    pool = max(M, min(args.cpu_sample, args.steps * M))
+    smp = OracleSample(cfg, pool)
+    for w in range(args.warmup):
+        smp.run(list(range(w * M % pool, w * M % pool + M)) if pool >= M else list(range(M)))
+        if w >= 2:
+            break
+    total = 0.0
     for s in range(args.steps):
-        v, cores, dt = cpu_oracle_sample(cfg, M, seed=0)
-        times.append(dt)
-    total = sum(times)
+        r0 = (s * M) % (pool - M + 1)
+        total += smp.run(list(range(r0, r0 + M)))
     value = M * args.steps / total
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "tokens_per_step": M},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{args.steps} steps x {M} token(s) of {args.workload}"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.cores(M),
+                             "kind": "oracle",
+                             "sample": f"{args.steps} steps of {M} token(s) of {args.workload}, "
+                                       f"drawn from a pool of {pool} tokens"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -288,6 +305,9 @@ def run_ours(args):
     # events recorded around it inside captured graphs
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for e in starts + stops:       # create the CUDA events before capture
+        e.record(st)
+    st.synchronize()
     kgraphs = []
     with torch.cuda.stream(st):
         for g0 in range(W, total_steps, copies):
@@ -307,26 +327,29 @@ def run_ours(args):
 
     # end to end through the public API: pinned host x -> device, forward,
     # y -> pinned host, every step
-    x_host = xs[:K].cpu().pin_memory()
-    y_host = torch.empty((K, M, cfg.H), dtype=torch.float32).pin_memory()
-    xdev = torch.empty((M, cfg.H), dtype=torch.bfloat16, device="cuda")
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with torch.cuda.stream(st):
-        e0.record(st)
-        for i in range(K):
-            c = i % copies
-            xdev.copy_(x_host[i], non_blocking=True)
-            moeq.moeq_layer_forward(layers[c].desc, xdev, M, ys[c], None, idx[c], wts[c], ws.buf,
-                                    ws.bytes, moeq.MODE_DECODE, st)
-            y_host[i].copy_(ys[c], non_blocking=True)
-        e1.record(st)
-    st.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e = M * K * world / (e2e_ms / 1e3)
+    e2e = None
+    if not args.no_e2e:
+        x_host = xs[:K].cpu().pin_memory()
+        y_host = torch.empty((K, M, cfg.H), dtype=torch.float32).pin_memory()
+        xdev = torch.empty((M, cfg.H), dtype=torch.bfloat16, device="cuda")
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(st):
+            e0.record(st)
+            for i in range(K):
+                c = i % copies
+                xdev.copy_(x_host[i], non_blocking=True)
+                moeq.moeq_layer_forward(layers[c].desc, xdev, M, ys[c], None, idx[c], wts[c],
+                                        ws.buf, ws.bytes, moeq.MODE_DECODE, st)
+                y_host[i].copy_(ys[c], non_blocking=True)
+            e1.record(st)
+        st.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": M * K * world / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": M * cfg.H * 2, "d2h_bytes_per_step": M * cfg.H * 4}
     status = moeq.moeq_device_status(st)
 
     line = {
@@ -347,17 +370,18 @@ def run_ours(args):
                      "peak": peak_hbm, "unit": "GB/s", "frac": achieved / peak_hbm,
                      "traffic": None, "bytes_per_launch": gu_bytes, "ms_per_launch": k_ms,
                      "peak_kind": peak_kind},
-        "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": M * cfg.H * 2,
-                "d2h_bytes_per_step": M * cfg.H * 4},
+        "e2e": e2e,
         "gpu_launches": int(launches_per_timed_region),
         "clocks": clk.summary(),
         "device_status": status,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        v, cores, dt = cpu_oracle_sample(cfg, args.cpu_sample)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": f"{args.cpu_sample} tokens of {args.workload} "
-                                          f"({dt:.1f} s)"}
+        smp = OracleSample(cfg, args.cpu_sample)
+        dt = smp.run(list(range(args.cpu_sample)))
+        line["cpu_baseline"] = {"value": args.cpu_sample / dt, "unit": "tokens/s",
+                                "cores": smp.cores(args.cpu_sample), "kind": "oracle",
+                                "sample": f"{args.cpu_sample} tokens of {args.workload}, "
+                                          f"one oracle call ({dt:.2f} s)"}
     for g in graphs + kgraphs:
         g.reset()
     if world > 1:

@@ -148,10 +148,15 @@ moeq_status moeq_route_topk(const float* logits, int32_t M, int32_t E, int32_t K
  *   residual: nullable fp32 [M][H]; y: fp32 [M][H].
  *   ws: device workspace of at least moeq_workspace_bytes(L, M, mode) bytes,
  *   256-byte aligned, owned by the caller, contents ignored on entry.
- * mode: DECODE requires M <= 64; PREFILL requires the prefill constraints
- * (8-bit or 4-bit experts, H and I multiples of 64). The prefill path
- * computes every output row independently of M, so splitting the tokens
- * into chunks gives bit-identical results.
+ * mode: DECODE requires M <= 64 and rows of at most 4096 bytes of codes.
+ * PREFILL requires group_size 64 for every tensor, H, I (and the shared
+ * expert's I) multiples of 128, 4-byte aligned scale/bias arrays, and
+ * values that fit the fp16 tensor-core operands (|x|, |bias| and
+ * |bias + (2^b-1)*scale| at most 65504, nonzero |scale| at least 2^-14);
+ * outside that range the device status reports MOEQ_ERR_RANGE.  The
+ * prefill path computes every output row from its own token with the same
+ * kernels for any M, so splitting the tokens into chunks gives
+ * bit-identical results.
  * idx is not read on the host; an index outside [0,E) found on the device
  * sets MOEQ_ERR_INVALID_ARG in the device status word and expert 0 is used
  * in its place.

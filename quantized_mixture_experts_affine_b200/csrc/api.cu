@@ -41,7 +41,15 @@ namespace moeq {
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 cudaError_t profile_mark(bool start, cudaStream_t st) {
   cudaEvent_t e = start ? t_prof_start : t_prof_stop;
-  return e ? cudaEventRecord(e, st) : cudaSuccess;
+  if (!e) return cudaSuccess;
+  // inside a stream capture a plain record only orders the capture; the
+  // external flag makes it a timestamp node of the graph
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t err = cudaStreamIsCapturing(st, &cs);
+  if (err != cudaSuccess) return err;
+  if (cs == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  return cudaEventRecord(e, st);
 }
 }  // namespace moeq
 

@@ -1,0 +1,485 @@
+// Gather quantised matrix multiply on tcgen05 tensor cores (prefill path).
+//
+// One CTA per SM loops over work items (m-tile of 128 sorted rows of one
+// expert, n-tile of 256 weight rows).  Warp roles:
+//   warps 0-1  A loader: gathers the 128 rows (token rows of x, or the
+//              expert's contiguous hidden rows) with 16-byte cp.async into
+//              the 128B-swizzled K-major A stage;
+//   warp  2    B loader: cp.async of the packed codes of 256 weight rows and
+//              of their bf16 scale/bias pairs for one 64-wide group;
+//   warp  3    MMA issuer: tcgen05.mma (M 128, N 256, K 16) x 4 per group,
+//              fp32 accumulators in TMEM (two 256-column buffers);
+//   warps 4-7  epilogue: tcgen05.ld of the accumulator rows, SwiGLU to fp16
+//              hidden rows, or fp32 output rows scattered to pair order;
+//   warps 8-11 dequantiser: codes -> fp16 weights w = q*scale + bias (one
+//              fused fp16 multiply-add of exact operands) written into the
+//              swizzled B stage.
+// The scale and bias of a 64-wide group are constant along K within a
+// k-block, so dequantising tiles in shared memory applies the affine map of
+// the pages' format exactly once per weight before the tensor-core product.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace moeq {
+namespace gq {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int S1 = 4;  // stages of A, packed B, scale/bias
+constexpr int S2 = 2;  // stages of dequantised B
+constexpr int A_STAGE = BM * BK * 2;   // 16 KB
+constexpr int B_STAGE = BN * BK * 2;   // 32 KB
+constexpr int SB_STAGE = BN * 8;       // scale pair + bias pair per row: 2 KB
+constexpr int THREADS = 384;
+constexpr uint32_t IDESC = tc::idesc_f16_f32(BM, BN);
+
+template <int BITS>
+struct Raw {
+  static constexpr int ROW = BK * BITS / 8;       // packed bytes of one row per k-block
+  static constexpr int STAGE = BN * ROW;          // 16/8/4 KB
+  static constexpr int CHUNKS = ROW / 16;         // 16-byte chunks per row
+};
+
+template <int BITS>
+struct Smem {
+  static constexpr int A_OFF = 0;
+  static constexpr int B_OFF = A_OFF + S1 * A_STAGE;
+  static constexpr int RAW_OFF = B_OFF + S2 * B_STAGE;
+  static constexpr int SB_OFF = RAW_OFF + S1 * Raw<BITS>::STAGE;
+  static constexpr int BAR_OFF = SB_OFF + S1 * SB_STAGE;
+  static constexpr int N_BARS = 5 * S1 + 2 * S2 + 4;
+  static constexpr int TMEM_OFF = BAR_OFF + N_BARS * 8;
+  static constexpr int BYTES = TMEM_OFF + 16;
+  static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024
+};
+
+enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1 };
+enum AMode { A_PAIRS = 0, A_TOKENS = 1, A_ROWS = 2 };
+
+// One expert (or the shared expert, or the router) over a run of sorted rows.
+struct Seg {
+  const uint32_t* w[2];
+  const uint16_t* s[2];
+  const uint16_t* b[2];
+  int32_t n0;         // SWIGLU: rows per source (I); STORE: rows taken from source 0
+  int32_t n_valid;    // STORE: valid weight rows in total (source 0 then source 1)
+  int32_t row_begin;  // first row of the segment in the sorted row space
+  int32_t rows;       // rows of the segment
+  int32_t a_mode;     // AMode
+  int32_t dest_pairs; // STORE: 1 = output row is the pair index sorted_pair[m]
+};
+
+struct Args {
+  const Seg* segs;
+  const int2* tiles;        // (segment, first row within the segment); null: seg0 only
+  const int32_t* n_tiles;   // device count of tiles
+  Seg seg0;                 // the single segment when tiles == null
+  int32_t static_mtiles;    // m-tiles of seg0 when tiles == null
+  int32_t n_tiles_n;        // n-tiles per m-tile
+  int32_t K;                // reduction length, multiple of 128
+  const __half* A;
+  int64_t lda;              // elements
+  const int32_t* sorted_pair;
+  int32_t topk;
+  void* out;
+  int64_t ldo;              // elements
+  int* status;
+};
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Weight row of tile row r (0..255) of n-tile nt: source index, row within
+// the source matrix, validity.
+template <int EPI>
+__device__ __forceinline__ void b_row(const Seg& sg, int nt, int r, int& src, int& q, bool& ok) {
+  if (EPI == EPI_SWIGLU) {
+    src = r >= 128;
+    q = nt * 128 + (r & 127);
+    ok = q < sg.n0;
+  } else {
+    const int g = nt * BN + r;
+    src = g >= sg.n0;
+    q = src ? g - sg.n0 : g;
+    ok = g < sg.n_valid;
+  }
+}
+
+// fp16 operands of the affine map for one group, with the range check of
+// the prefill tiles (scale a normal fp16 value or zero, |bias| and
+// |bias + (2^b - 1) scale| below the fp16 maximum).
+template <int BITS>
+__device__ __forceinline__ void group_h2(uint32_t sbits, uint32_t bbits, __half2& s2, __half2& b2,
+                                         int* status) {
+  const float s = bf16_bits_to_float((uint16_t)sbits);
+  const float b = bf16_bits_to_float((uint16_t)bbits);
+  const float top = fabsf(b + (float)((1 << BITS) - 1) * s);
+  const bool bad = (s != 0.0f && fabsf(s) < 6.103515625e-05f) || fabsf(s) > 65504.0f ||
+                   fabsf(b) > 65504.0f || top > 65504.0f;
+  if (bad) set_status(status, MOEQ_ERR_RANGE);
+  s2 = __float2half2_rn(s);
+  b2 = __float2half2_rn(b);
+}
+
+// Dequantise one 16-byte chunk of packed codes into fp16 weights: 16 (8-bit),
+// 32 (4-bit) or 64 (2-bit) values, written as 16-byte chunks starting at
+// chunk `c16` of row `r` of the swizzled B stage.
+template <int BITS>
+__device__ __forceinline__ void dequant_chunk(uint4 raw, __half2 s2, __half2 b2, uint32_t bstage,
+                                              int r, int c16) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  if (BITS == 8) {
+    // codes q0..q15; half2 (1024 + q_j, 1024 + q_j+1) by byte permutes
+    const __half2 k1024 = __float2half2_rn(1024.0f);
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 lo = __hsub2(u2h(__byte_perm(w[i], 0x64646464u, 0x4140)), k1024);
+      const __half2 hi = __hsub2(u2h(__byte_perm(w[i], 0x64646464u, 0x4342)), k1024);
+      o[2 * i] = h2u(__hfma2(lo, s2, b2));
+      o[2 * i + 1] = h2u(__hfma2(hi, s2, b2));
+    }
+    sts128(bstage + tc::sw128_offset(r, c16), o[0], o[1], o[2], o[3]);
+    sts128(bstage + tc::sw128_offset(r, c16 + 1), o[4], o[5], o[6], o[7]);
+  } else if (BITS == 4) {
+    // byte j holds q_2j (low nibble) and q_2j+1 (high nibble)
+    const __half2 sc = __halves2half2(__float2half_rn(1.0f), __float2half_rn(1.0f / 16.0f));
+    const __half2 of = __halves2half2(__float2half_rn(-1024.0f), __float2half_rn(-64.0f));
+    uint32_t o[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sel = 0x4040u | (uint32_t)j | ((uint32_t)j << 8);
+        const uint32_t t = (__byte_perm(w[i], 0u, sel) & 0x00F0000Fu) | 0x64006400u;
+        const __half2 q = __hfma2(u2h(t), sc, of);  // exact (q_lo, q_hi)
+        o[4 * i + j] = h2u(__hfma2(q, s2, b2));
+      }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      sts128(bstage + tc::sw128_offset(r, c16 + k), o[4 * k], o[4 * k + 1], o[4 * k + 2],
+             o[4 * k + 3]);
+  } else {
+    // byte j holds q_4j .. q_4j+3 in bit pairs
+    const __half2 sc0 = __halves2half2(__float2half_rn(1.0f), __float2half_rn(0.25f));
+    const __half2 of0 = __halves2half2(__float2half_rn(-1024.0f), __float2half_rn(-256.0f));
+    const __half2 sc1 = __halves2half2(__float2half_rn(1.0f / 16.0f), __float2half_rn(1.0f / 64.0f));
+    const __half2 of1 = __halves2half2(__float2half_rn(-64.0f), __float2half_rn(-16.0f));
+    uint32_t o[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sel = 0x4040u | (uint32_t)j | ((uint32_t)j << 8);
+        const uint32_t t = __byte_perm(w[i], 0u, sel);
+        const __half2 q01 = __hfma2(u2h((t & 0x000C0003u) | 0x64006400u), sc0, of0);
+        const __half2 q23 = __hfma2(u2h((t & 0x00C00030u) | 0x64006400u), sc1, of1);
+        o[8 * i + 2 * j] = h2u(__hfma2(q01, s2, b2));
+        o[8 * i + 2 * j + 1] = h2u(__hfma2(q23, s2, b2));
+      }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      sts128(bstage + tc::sw128_offset(r, c16 + k), o[4 * k], o[4 * k + 1], o[4 * k + 2],
+             o[4 * k + 3]);
+  }
+}
+
+__device__ __forceinline__ int2 tile_of(const Args& a, int mt) {
+  return a.tiles ? a.tiles[mt] : make_int2(0, mt * BM);
+}
+
+template <int BITS, int EPI>
+__global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Args a) {
+  using SM = Smem<BITS>;
+  using RW = Raw<BITS>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = tc::smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);
+  uint64_t* full_a = bars;               // S1, A loader -> MMA
+  uint64_t* a_empty = bars + S1;         // S1, MMA -> A loader
+  uint64_t* raw_full = bars + 2 * S1;    // S1, B loader -> dequant
+  uint64_t* raw_empty = bars + 3 * S1;   // S1, dequant -> B loader
+  uint64_t* sb_unused = bars + 4 * S1;   // S1 (reserved)
+  uint64_t* b_full = bars + 5 * S1;      // S2, dequant -> MMA
+  uint64_t* b_empty = b_full + S2;       // S2, MMA -> dequant
+  uint64_t* tmem_full = b_empty + S2;    // 2, MMA -> epilogue
+  uint64_t* tmem_empty = tmem_full + 2;  // 2, epilogue -> MMA
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::TMEM_OFF);
+  (void)sb_unused;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S1; ++i) {
+      tc::mbar_init(&full_a[i], 64);
+      tc::mbar_init(&a_empty[i], 1);
+      tc::mbar_init(&raw_full[i], 32);
+      tc::mbar_init(&raw_empty[i], 128);
+    }
+    for (int i = 0; i < S2; ++i) {
+      tc::mbar_init(&b_full[i], 128);
+      tc::mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&tmem_full[i], 1);
+      tc::mbar_init(&tmem_empty[i], 128);
+    }
+    tc::fence_mbar_init();
+  }
+  if (warp == 3) {
+    tc::tmem_alloc(tmem_holder, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int n_items = (a.tiles ? *a.n_tiles : a.static_mtiles) * a.n_tiles_n;
+  const int KB = a.K / BK;
+  int* status = a.status;
+
+  if (warp < 2) {
+    // ------------------------------------------------------------ A loader
+    const int t = threadIdx.x;  // 0..63: tile rows 2t, 2t+1
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n);
+      const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
+      const __half* src[2];
+      uint32_t nbytes[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int i = 2 * t + j;
+        const bool ok = tile.y + i < sg.rows;
+        const int64_t m = (int64_t)sg.row_begin + tile.y + i;
+        int64_t arow = 0;
+        if (ok) {
+          if (sg.a_mode == A_PAIRS) arow = a.sorted_pair[m] / a.topk;
+          else if (sg.a_mode == A_TOKENS) arow = tile.y + i;
+          else arow = m;
+        }
+        src[j] = a.A + arow * a.lda;
+        nbytes[j] = ok ? 16u : 0u;
+      }
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s = it % S1, ph = (it / S1) & 1u;
+        if (!tc::mbar_wait(&a_empty[s], ph ^ 1u, status)) goto done;
+        const uint32_t st = sbase + SM::A_OFF + s * A_STAGE;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            tc::cp_async16(st + tc::sw128_offset(2 * t + j, c), src[j] + kb * BK + c * 8,
+                           nbytes[j]);
+        tc::cp_async_arrive_noinc(&full_a[s]);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ B loader
+    const int64_t wrow = (int64_t)a.K * BITS / 32;  // words per weight row
+    const int groups = a.K / 64;
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n);
+      const int nt = item % a.n_tiles_n;
+      const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
+      const uint32_t* wp[8];
+      const uint16_t* sp[8];
+      const uint16_t* bp[8];
+      uint32_t ok16[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = lane + 32 * j;
+        int src, q;
+        bool ok;
+        b_row<EPI>(sg, nt, r, src, q, ok);
+        if (!ok) q = 0;
+        wp[j] = sg.w[src] + (int64_t)q * wrow;
+        sp[j] = sg.s[src] + (int64_t)q * groups;
+        bp[j] = sg.b[src] + (int64_t)q * groups;
+        ok16[j] = ok ? 16u : 0u;
+      }
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s = it % S1, ph = (it / S1) & 1u;
+        if (!tc::mbar_wait(&raw_empty[s], ph ^ 1u, status)) goto done;
+        const uint32_t rst = sbase + SM::RAW_OFF + s * RW::STAGE;
+        const uint32_t sbst = sbase + SM::SB_OFF + s * SB_STAGE;
+        const int kb2 = kb & ~1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = lane + 32 * j;
+#pragma unroll
+          for (int c = 0; c < RW::CHUNKS; ++c)
+            tc::cp_async16(rst + r * RW::ROW + c * 16, wp[j] + kb * (RW::ROW / 4) + c * 4,
+                           ok16[j]);
+          tc::cp_async4(sbst + r * 8, sp[j] + kb2, ok16[j] ? 4u : 0u);
+          tc::cp_async4(sbst + r * 8 + 4, bp[j] + kb2, ok16[j] ? 4u : 0u);
+        }
+        tc::cp_async_arrive_noinc(&raw_full[s]);
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t it = 0, tcount = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++tcount) {
+      const uint32_t acc = tcount & 1u, acc_ph = (tcount >> 1) & 1u;
+      if (!tc::mbar_wait(&tmem_empty[acc], acc_ph ^ 1u, status)) goto done;
+      tc::tc_fence_after();
+      const uint32_t d = tmem_base + acc * 256u;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s1 = it % S1, ph1 = (it / S1) & 1u;
+        const uint32_t s2 = it % S2, ph2 = (it / S2) & 1u;
+        if (!tc::mbar_wait(&full_a[s1], ph1, status)) goto done;
+        if (!tc::mbar_wait(&b_full[s2], ph2, status)) goto done;
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_after();
+        if (lane == 0) {
+          const uint32_t aa = sbase + SM::A_OFF + s1 * A_STAGE;
+          const uint32_t ba = sbase + SM::B_OFF + s2 * B_STAGE;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc::mma_f16(d, tc::sw128_kmajor_desc(aa + kk * 32), tc::sw128_kmajor_desc(ba + kk * 32),
+                        IDESC, (kb | kk) != 0);
+          tc::mma_commit(&a_empty[s1]);
+          tc::mma_commit(&b_empty[s2]);
+        }
+        __syncwarp();
+      }
+      if (lane == 0) tc::mma_commit(&tmem_full[acc]);
+      __syncwarp();
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int i = q * 32 + lane;  // tile row = TMEM lane
+    uint32_t tcount = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++tcount) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n);
+      const int nt = item % a.n_tiles_n;
+      const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
+      const uint32_t acc = tcount & 1u, acc_ph = (tcount >> 1) & 1u;
+      if (!tc::mbar_wait(&tmem_full[acc], acc_ph, status)) goto done;
+      tc::tc_fence_after();
+      const bool ok = tile.y + i < sg.rows;
+      const int64_t m = (int64_t)sg.row_begin + tile.y + i;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 256u;
+      if (EPI == EPI_SWIGLU) {
+        __half* out = reinterpret_cast<__half*>(a.out) + m * a.ldo + nt * 128;
+        bool bad = false;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t g[32], u[32];
+          tc::tmem_ld32(tb + c0, g);
+          tc::tmem_ld32(tb + 128 + c0, u);
+          tc::tmem_wait_ld();
+          if (ok && nt * 128 + c0 < sg.n0) {
+            uint32_t o[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float g0 = __uint_as_float(g[2 * k]), g1 = __uint_as_float(g[2 * k + 1]);
+              const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(u[2 * k]);
+              const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(u[2 * k + 1]);
+              bad |= !(fabsf(h0) <= 65504.0f) || !(fabsf(h1) <= 65504.0f);
+              o[k] = h2u(__floats2half2_rn(h0, h1));
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + c0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+          }
+        }
+        if (bad) set_status(status, MOEQ_ERR_RANGE);
+      } else {
+        int64_t dest = m;
+        if (ok && sg.dest_pairs) dest = a.sorted_pair[m];
+        float* out = reinterpret_cast<float*>(a.out) + dest * a.ldo + nt * BN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tc::tmem_ld32(tb + c0, v);
+          tc::tmem_wait_ld();
+          const int col = nt * BN + c0;
+          if (ok && col < sg.n_valid) {
+            if (col + 32 <= sg.n_valid && (((uintptr_t)(out + c0)) & 15) == 0) {
+              uint4* dst = reinterpret_cast<uint4*>(out + c0);
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                dst[k] = make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            } else {
+              const int nv = min(32, sg.n_valid - col);
+              for (int k = 0; k < nv; ++k) out[c0 + k] = __uint_as_float(v[k]);
+            }
+          }
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&tmem_empty[acc]);
+    }
+  } else {
+    // ------------------------------------------------------------ dequantiser
+    const int td = threadIdx.x - 256;  // 0..127
+    constexpr int ITEMS = BN * RW::CHUNKS / 128;  // per thread per stage: 8, 4, 2
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s1 = it % S1, ph1 = (it / S1) & 1u;
+        const uint32_t s2 = it % S2, ph2 = (it / S2) & 1u;
+        if (!tc::mbar_wait(&raw_full[s1], ph1, status)) goto done;
+        if (!tc::mbar_wait(&b_empty[s2], ph2 ^ 1u, status)) goto done;
+        const uint32_t rst = sbase + SM::RAW_OFF + s1 * RW::STAGE;
+        const uint32_t sbst = sbase + SM::SB_OFF + s1 * SB_STAGE;
+        const uint32_t bst = sbase + SM::B_OFF + s2 * B_STAGE;
+        const int hi = kb & 1;
+#pragma unroll
+        for (int k = 0; k < ITEMS; ++k) {
+          const int idx = td + 128 * k;
+          const int r = idx / RW::CHUNKS, c = idx % RW::CHUNKS;
+          const uint4 raw = lds128(rst + r * RW::ROW + c * 16);
+          const uint2 sb = lds64(sbst + r * 8);
+          __half2 s2h, b2h;
+          group_h2<BITS>(hi ? (sb.x >> 16) : (sb.x & 0xFFFFu), hi ? (sb.y >> 16) : (sb.y & 0xFFFFu),
+                         s2h, b2h, status);
+          // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
+          dequant_chunk<BITS>(raw, s2h, b2h, bst, r, c * (16 / BITS));
+        }
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&b_full[s2]);
+        tc::mbar_arrive(&raw_empty[s1]);
+      }
+    }
+  }
+done:
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 3) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace gq
+}  // namespace moeq

@@ -1,14 +1,526 @@
-// Prefill path: placeholder until the tensor-core gather-QMM lands.
+// Prefill path (many tokens): fp16 copy of the tokens, router GEMM, top-K,
+// stable counting sort of the (token, slot) pairs by expert, gate/up
+// gather-QMM with the SwiGLU epilogue, down gather-QMM into pair order,
+// weighted combine.  Every output row is computed from its own token only,
+// with the same kernels and the same K order for any M, so results do not
+// depend on how the tokens are split into calls.
+#include <cuda_fp16.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "gqmm.cuh"
+#include "kernels.h"
 #include "prefill.h"
+#include "route.cuh"
 
 namespace moeq {
 
-size_t prefill_workspace_bytes(const moeq_layer*, int) { return 0; }
+namespace {
 
-moeq_status prefill_forward(const moeq_layer*, const uint16_t*, int, const int32_t*, const float*,
-                            const float*, float*, int32_t*, float*, void*, size_t, int*,
-                            cudaStream_t) {
-  return MOEQ_ERR_UNSUPPORTED;
+constexpr int kSortChunk = 2048;  // pairs per sort block
+
+// ------------------------------------------------------------------ tokens to fp16
+__global__ void __launch_bounds__(256) k_to_f16(const uint16_t* __restrict__ x, int64_t n8,
+                                                __half* __restrict__ y, int* status) {
+  bool bad = false;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
+      bad |= !(fabsf(a) <= 65504.0f) || !(fabsf(b) <= 65504.0f);
+      __half2 h = __floats2half2_rn(a, b);
+      o[j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    reinterpret_cast<uint4*>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (bad) set_status(status, MOEQ_ERR_RANGE);
+}
+
+// ------------------------------------------------------------------ routing (strided logits)
+__global__ void __launch_bounds__(256) k_route_prefill(const float* __restrict__ logits, int64_t ld,
+                                                       int M, int E, int K, int renorm,
+                                                       float scale, int32_t* __restrict__ idx,
+                                                       float* __restrict__ w, int sg_col,
+                                                       float* __restrict__ sigma) {
+  extern __shared__ uint32_t taken_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int words = (E + 31) >> 5;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= M) return;
+  route_token_warp(logits + (int64_t)t * ld, E, K, renorm, scale, idx + (int64_t)t * K,
+                   w + (int64_t)t * K, taken_all + warp * words);
+  if (sigma && lane == 0) sigma[t] = 1.0f / (1.0f + expf(-logits[(int64_t)t * ld + sg_col]));
+}
+
+__global__ void __launch_bounds__(256) k_copy_routing(const int32_t* __restrict__ idx_in,
+                                                      const float* __restrict__ w_in, int64_t n,
+                                                      int32_t* __restrict__ idx,
+                                                      float* __restrict__ w) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    idx[i] = idx_in[i];
+    w[i] = w_in[i];
+  }
+}
+
+__global__ void __launch_bounds__(256) k_sigmoid_col(const float* __restrict__ logits, int64_t ld,
+                                                     int col, int M, float* __restrict__ sigma) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < M; t += gridDim.x * blockDim.x)
+    sigma[t] = 1.0f / (1.0f + expf(-logits[(int64_t)t * ld + col]));
+}
+
+// ------------------------------------------------------------------ stable counting sort
+__device__ __forceinline__ int checked_expert(const int32_t* idx, int64_t p, int E, int* status) {
+  int e = idx[p];
+  if (e < 0 || e >= E) {
+    set_status(status, MOEQ_ERR_INVALID_ARG);
+    e = 0;
+  }
+  return e;
+}
+
+// Per-block expert histogram of kSortChunk pairs.
+__global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, int64_t n, int E,
+                                              int32_t* __restrict__ blockhist, int* status) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t p0 = (int64_t)blockIdx.x * kSortChunk;
+  const int64_t p1 = min(n, p0 + kSortChunk);
+  for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x)
+    atomicAdd(&hist[checked_expert(idx, p, E, status)], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) blockhist[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+struct OffsetsArgs {
+  const int32_t* blockhist;
+  int32_t* blockoff;        // [nb][E]
+  int32_t* expert_off;      // [E]
+  int32_t nb, E, I, H;
+  gq::Seg* segs_gu;         // [E]
+  gq::Seg* segs_dn;         // [E]
+  int2* tiles;              // [max tiles]
+  int32_t* n_tiles;         // [1]
+  moeq_qtensor gate, up, down;
+};
+
+// One CTA: per-expert block offsets and counts, expert offsets (exclusive
+// scan), one gate/up and one down segment per expert and the m-tile list.
+__global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ OffsetsArgs a) {
+  __shared__ int32_t part_rows[1024], part_tiles[1024];
+  const int E = a.E, tid = threadIdx.x;
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = tid * per, e1 = min(E, e0 + per);
+  int32_t cnt[4];  // E <= 4096 -> at most 4 experts per thread
+  int rsum = 0, tsum = 0;
+  for (int e = e0; e < e1; ++e) {
+    int run = 0;
+    for (int b = 0; b < a.nb; ++b) {
+      a.blockoff[(int64_t)b * E + e] = run;
+      run += a.blockhist[(int64_t)b * E + e];
+    }
+    cnt[e - e0] = run;
+    rsum += run;
+    tsum += (run + gq::BM - 1) / gq::BM;
+  }
+  part_rows[tid] = rsum;
+  part_tiles[tid] = tsum;
+  __syncthreads();
+  // exclusive scan over threads (serial by one warp's lane 0 in chunks; 1024 entries)
+  if (tid == 0) {
+    int r = 0, t = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) {
+      const int pr = part_rows[i], pt = part_tiles[i];
+      part_rows[i] = r;
+      part_tiles[i] = t;
+      r += pr;
+      t += pt;
+    }
+    *a.n_tiles = t;
+  }
+  __syncthreads();
+  int row = part_rows[tid], tile = part_tiles[tid];
+  for (int e = e0; e < e1; ++e) {
+    const int c = cnt[e - e0];
+    a.expert_off[e] = row;
+    gq::Seg g;
+    memset(&g, 0, sizeof(g));
+    g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
+    g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
+    g.b[0] = a.gate.biases + (int64_t)e * a.gate.expert_stride_sb;
+    g.w[1] = a.up.w + (int64_t)e * a.up.expert_stride_w;
+    g.s[1] = a.up.scales + (int64_t)e * a.up.expert_stride_sb;
+    g.b[1] = a.up.biases + (int64_t)e * a.up.expert_stride_sb;
+    g.n0 = a.I;
+    g.n_valid = a.I;
+    g.row_begin = row;
+    g.rows = c;
+    g.a_mode = gq::A_PAIRS;
+    g.dest_pairs = 0;
+    a.segs_gu[e] = g;
+    gq::Seg d;
+    memset(&d, 0, sizeof(d));
+    d.w[0] = d.w[1] = a.down.w + (int64_t)e * a.down.expert_stride_w;
+    d.s[0] = d.s[1] = a.down.scales + (int64_t)e * a.down.expert_stride_sb;
+    d.b[0] = d.b[1] = a.down.biases + (int64_t)e * a.down.expert_stride_sb;
+    d.n0 = a.H;
+    d.n_valid = a.H;
+    d.row_begin = row;
+    d.rows = c;
+    d.a_mode = gq::A_ROWS;
+    d.dest_pairs = 1;
+    a.segs_dn[e] = d;
+    const int nt = (c + gq::BM - 1) / gq::BM;
+    for (int j = 0; j < nt; ++j) a.tiles[tile + j] = make_int2(e, j * gq::BM);
+    row += c;
+    tile += nt;
+  }
+}
+
+// Stable scatter: one warp per block of kSortChunk pairs, in pair order.
+__global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx, int64_t n, int E,
+                                                const int32_t* __restrict__ expert_off,
+                                                const int32_t* __restrict__ blockoff,
+                                                int32_t* __restrict__ sorted_pair, int* status) {
+  extern __shared__ int32_t run[];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) run[e] = 0;
+  __syncwarp();
+  const int64_t p0 = (int64_t)blockIdx.x * kSortChunk;
+  const int64_t p1 = min(n, p0 + kSortChunk);
+  const int32_t* boff = blockoff + (int64_t)blockIdx.x * E;
+  for (int64_t base = p0; base < p1; base += 32) {
+    const int64_t p = base + lane;
+    const bool on = p < p1;
+    const int e = on ? checked_expert(idx, p, E, status) : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (on) {
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int64_t pos = (int64_t)expert_off[e] + boff[e] + run[e] + rank;
+      sorted_pair[pos] = (int32_t)p;
+    }
+    __syncwarp();
+    if (on && lane == __ffs(peers) - 1) run[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------------ gather-QMM launch
+template <int BITS, int EPI>
+cudaError_t launch_gqmm_t(const gq::Args& a, int grid, cudaStream_t st) {
+  constexpr int smem = gq::Smem<BITS>::ALLOC;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gq::k_gqmm<BITS, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  gq::k_gqmm<BITS, EPI><<<grid, gq::THREADS, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gqmm(int bits, int epi, const gq::Args& a, int grid, cudaStream_t st) {
+  if (grid <= 0) return cudaSuccess;
+  if (epi == gq::EPI_SWIGLU) {
+    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SWIGLU>(a, grid, st);
+    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SWIGLU>(a, grid, st);
+    return launch_gqmm_t<2, gq::EPI_SWIGLU>(a, grid, st);
+  }
+  if (bits == 8) return launch_gqmm_t<8, gq::EPI_STORE>(a, grid, st);
+  if (bits == 4) return launch_gqmm_t<4, gq::EPI_STORE>(a, grid, st);
+  return launch_gqmm_t<2, gq::EPI_STORE>(a, grid, st);
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+gq::Seg seg_single(const moeq_qtensor& t0, const moeq_qtensor* t1, int rows, int a_mode) {
+  gq::Seg s;
+  memset(&s, 0, sizeof(s));
+  s.w[0] = t0.w;
+  s.s[0] = t0.scales;
+  s.b[0] = t0.biases;
+  const moeq_qtensor& u = t1 ? *t1 : t0;
+  s.w[1] = u.w;
+  s.s[1] = u.scales;
+  s.b[1] = u.biases;
+  s.n0 = t0.out_dim;
+  s.n_valid = t0.out_dim + (t1 ? t1->out_dim : 0);
+  s.row_begin = 0;
+  s.rows = rows;
+  s.a_mode = a_mode;
+  s.dest_pairs = 0;
+  return s;
+}
+
+// ------------------------------------------------------------------ workspace
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~(size_t)255;
+    return o;
+  }
+};
+
+struct PrefillWs {
+  size_t x16, logits, idx, w, sigma, blockhist, blockoff, expert_off, segs_gu, segs_dn, tiles,
+      n_tiles, sorted, h, h_sh, y, total;
+  int64_t ld_logits;
+  int nb;
+};
+
+bool sg_with_router(const moeq_layer* L) {
+  return L->has_shared && L->sh_expert_gate.bits == L->router.bits &&
+         L->sh_expert_gate.group_size == L->router.group_size;
+}
+
+PrefillWs prefill_ws(const moeq_layer* L, int M) {
+  const int E = L->n_experts, K = L->top_k, H = L->hidden, I = L->inter;
+  const int Is = L->has_shared ? L->sh_gate.out_dim : 0;
+  const int64_t n = (int64_t)M * K;
+  PrefillWs w;
+  w.nb = (int)((n + kSortChunk - 1) / kSortChunk);
+  // row stride a multiple of 4 floats: the epilogue stores 16-byte vectors
+  w.ld_logits = (E + (L->has_shared ? 1 : 0) + 3) & ~3;
+  const int64_t max_tiles = n / gq::BM + E + 1;
+  Carve c;
+  w.x16 = c.take((size_t)M * H * 2);
+  w.logits = c.take((size_t)M * w.ld_logits * 4);
+  w.idx = c.take((size_t)n * 4);
+  w.w = c.take((size_t)n * 4);
+  w.sigma = c.take((size_t)M * 4);
+  w.blockhist = c.take((size_t)w.nb * E * 4);
+  w.blockoff = c.take((size_t)w.nb * E * 4);
+  w.expert_off = c.take((size_t)E * 4);
+  w.segs_gu = c.take((size_t)E * sizeof(gq::Seg));
+  w.segs_dn = c.take((size_t)E * sizeof(gq::Seg));
+  w.tiles = c.take((size_t)max_tiles * sizeof(int2));
+  w.n_tiles = c.take(16);
+  w.sorted = c.take((size_t)n * 4);
+  w.h = c.take((size_t)n * I * 2);
+  w.h_sh = c.take((size_t)M * Is * 2);
+  w.y = c.take((size_t)(n + M) * H * 4);
+  w.total = c.off;
+  return w;
+}
+
+moeq_status check_prefill(const moeq_layer* L) {
+  const moeq_qtensor* ts[8] = {&L->router, &L->gate, &L->up, &L->down,
+                               &L->sh_gate, &L->sh_up, &L->sh_down, &L->sh_expert_gate};
+  const int n = L->has_shared ? 8 : 4;
+  for (int i = 0; i < n; ++i) {
+    if (ts[i]->group_size != 64) return MOEQ_ERR_UNSUPPORTED;
+    if (((uintptr_t)ts[i]->scales & 3) || ((uintptr_t)ts[i]->biases & 3)) return MOEQ_ERR_ALIGNMENT;
+    if (ts[i]->in_dim % 128) return MOEQ_ERR_UNSUPPORTED;
+    if (ts[i]->expert_stride_sb % 2) return MOEQ_ERR_ALIGNMENT;
+  }
+  if (L->inter % 128) return MOEQ_ERR_UNSUPPORTED;
+  if (L->has_shared && L->sh_gate.out_dim % 128) return MOEQ_ERR_UNSUPPORTED;
+  return MOEQ_OK;
+}
+
+}  // namespace
+
+size_t prefill_workspace_bytes(const moeq_layer* L, int M) {
+  if (check_prefill(L) != MOEQ_OK) return 0;
+  return prefill_ws(L, M).total;
+}
+
+#define PCK(x)                                              \
+  do {                                                      \
+    if ((x) != cudaSuccess) return MOEQ_ERR_CUDA;           \
+    count_launches(1);                                      \
+  } while (0)
+
+moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const int32_t* idx_in,
+                            const float* w_in, const float* residual, float* y, int32_t* idx_out,
+                            float* w_out, void* ws, size_t ws_bytes, int* status,
+                            cudaStream_t st) {
+  moeq_status s = check_prefill(L);
+  if (s != MOEQ_OK) return s;
+  const int E = L->n_experts, K = L->top_k, H = L->hidden, I = L->inter;
+  const int64_t n = (int64_t)M * K;
+  const PrefillWs lay = prefill_ws(L, M);
+  if (ws_bytes < lay.total) return MOEQ_ERR_WORKSPACE;
+  char* base = (char*)ws;
+  __half* x16 = (__half*)(base + lay.x16);
+  float* logits = (float*)(base + lay.logits);
+  int32_t* idx = idx_out ? idx_out : (int32_t*)(base + lay.idx);
+  float* wts = w_out ? w_out : (float*)(base + lay.w);
+  float* sigma = (float*)(base + lay.sigma);
+  int32_t* blockhist = (int32_t*)(base + lay.blockhist);
+  int32_t* blockoff = (int32_t*)(base + lay.blockoff);
+  int32_t* expert_off = (int32_t*)(base + lay.expert_off);
+  gq::Seg* segs_gu = (gq::Seg*)(base + lay.segs_gu);
+  gq::Seg* segs_dn = (gq::Seg*)(base + lay.segs_dn);
+  int2* tiles = (int2*)(base + lay.tiles);
+  int32_t* n_tiles = (int32_t*)(base + lay.n_tiles);
+  int32_t* sorted = (int32_t*)(base + lay.sorted);
+  __half* h = (__half*)(base + lay.h);
+  __half* h_sh = (__half*)(base + lay.h_sh);
+  float* yrows = (float*)(base + lay.y);
+  const int sms = sm_count();
+  const int mtiles = (M + gq::BM - 1) / gq::BM;
+
+  // 1. fp16 copy of the tokens (range-checked)
+  {
+    const int64_t n8 = (int64_t)M * H / 8;
+    int64_t grid = (n8 + 255) / 256;
+    if (grid > sms * 8) grid = sms * 8;
+    k_to_f16<<<(int)grid, 256, 0, st>>>(x, n8, x16, status);
+    PCK(cudaGetLastError());
+  }
+
+  // 2. router logits (+ the shared-expert gate logit as one more column)
+  const bool sgr = sg_with_router(L);
+  auto gemm_args = [&](const gq::Seg& s0, int n_tiles_n, int Kdim, const __half* A, int64_t lda,
+                       void* out, int64_t ldo) {
+    gq::Args a;
+    memset(&a, 0, sizeof(a));
+    a.seg0 = s0;
+    a.static_mtiles = mtiles;
+    a.n_tiles_n = n_tiles_n;
+    a.K = Kdim;
+    a.A = A;
+    a.lda = lda;
+    a.topk = K;
+    a.out = out;
+    a.ldo = ldo;
+    a.status = status;
+    return a;
+  };
+  if (!idx_in) {
+    const gq::Seg rs = seg_single(L->router, sgr ? &L->sh_expert_gate : nullptr, M, gq::A_TOKENS);
+    const int nt = (rs.n_valid + gq::BN - 1) / gq::BN;
+    const gq::Args a = gemm_args(rs, nt, H, x16, H, logits, lay.ld_logits);
+    const int items = mtiles * nt;
+    PCK(launch_gqmm(L->router.bits, gq::EPI_STORE, a, items < sms ? items : sms, st));
+  }
+  if (L->has_shared && (idx_in || !sgr)) {
+    const gq::Seg gs = seg_single(L->sh_expert_gate, nullptr, M, gq::A_TOKENS);
+    const gq::Args a = gemm_args(gs, 1, H, x16, H, logits + E, lay.ld_logits);
+    PCK(launch_gqmm(L->sh_expert_gate.bits, gq::EPI_STORE, a, mtiles < sms ? mtiles : sms, st));
+  }
+
+  // 3. routing
+  if (!idx_in) {
+    const int warps = 8;
+    const size_t smem = (size_t)warps * ((E + 31) / 32) * 4;
+    k_route_prefill<<<(M + warps - 1) / warps, warps * 32, smem, st>>>(
+        logits, lay.ld_logits, M, E, K, L->renorm, L->router_scale, idx, wts, E,
+        L->has_shared ? sigma : nullptr);
+    PCK(cudaGetLastError());
+  } else {
+    int64_t grid = (n + 255) / 256;
+    if (grid > sms * 8) grid = sms * 8;
+    k_copy_routing<<<(int)grid, 256, 0, st>>>(idx_in, w_in, n, idx, wts);
+    PCK(cudaGetLastError());
+    if (L->has_shared) {
+      k_sigmoid_col<<<(M + 255) / 256, 256, 0, st>>>(logits, lay.ld_logits, E, M, sigma);
+      PCK(cudaGetLastError());
+    }
+  }
+
+  // 4. stable counting sort of the pairs by expert, segments and m-tiles
+  const size_t hsmem = (size_t)E * 4;
+  k_hist<<<lay.nb, 256, hsmem, st>>>(idx, n, E, blockhist, status);
+  PCK(cudaGetLastError());
+  OffsetsArgs oa;
+  memset(&oa, 0, sizeof(oa));
+  oa.blockhist = blockhist;
+  oa.blockoff = blockoff;
+  oa.expert_off = expert_off;
+  oa.nb = lay.nb;
+  oa.E = E;
+  oa.I = I;
+  oa.H = H;
+  oa.segs_gu = segs_gu;
+  oa.segs_dn = segs_dn;
+  oa.tiles = tiles;
+  oa.n_tiles = n_tiles;
+  oa.gate = L->gate;
+  oa.up = L->up;
+  oa.down = L->down;
+  k_offsets<<<1, 1024, 0, st>>>(oa);
+  PCK(cudaGetLastError());
+  k_scatter<<<lay.nb, 32, hsmem, st>>>(idx, n, E, expert_off, blockoff, sorted, status);
+  PCK(cudaGetLastError());
+
+  const int64_t max_mtiles = n / gq::BM + E;
+  // 5. gate/up + SwiGLU for the routed experts (the profiled kernel), then the shared expert
+  {
+    gq::Args a;
+    memset(&a, 0, sizeof(a));
+    a.segs = segs_gu;
+    a.tiles = tiles;
+    a.n_tiles = n_tiles;
+    a.n_tiles_n = I / 128;
+    a.K = H;
+    a.A = x16;
+    a.lda = H;
+    a.sorted_pair = sorted;
+    a.topk = K;
+    a.out = h;
+    a.ldo = I;
+    a.status = status;
+    const int64_t items = max_mtiles * a.n_tiles_n;
+    if (profile_mark(true, st) != cudaSuccess) return MOEQ_ERR_CUDA;
+    PCK(launch_gqmm(L->gate.bits, gq::EPI_SWIGLU, a, items < sms ? (int)items : sms, st));
+    if (profile_mark(false, st) != cudaSuccess) return MOEQ_ERR_CUDA;
+  }
+  if (L->has_shared) {
+    const int Is = L->sh_gate.out_dim;
+    gq::Seg gs = seg_single(L->sh_gate, &L->sh_up, M, gq::A_TOKENS);
+    gs.n0 = Is;
+    const gq::Args a = gemm_args(gs, Is / 128, H, x16, H, h_sh, Is);
+    const int items = mtiles * (Is / 128);
+    PCK(launch_gqmm(L->sh_gate.bits, gq::EPI_SWIGLU, a, items < sms ? items : sms, st));
+  }
+  // 6. down projections into pair order (shared rows after the M*K pair rows)
+  {
+    gq::Args a;
+    memset(&a, 0, sizeof(a));
+    a.segs = segs_dn;
+    a.tiles = tiles;
+    a.n_tiles = n_tiles;
+    a.n_tiles_n = (H + gq::BN - 1) / gq::BN;
+    a.K = I;
+    a.A = h;
+    a.lda = I;
+    a.sorted_pair = sorted;
+    a.topk = K;
+    a.out = yrows;
+    a.ldo = H;
+    a.status = status;
+    const int64_t items = max_mtiles * a.n_tiles_n;
+    PCK(launch_gqmm(L->down.bits, gq::EPI_STORE, a, items < sms ? (int)items : sms, st));
+  }
+  if (L->has_shared) {
+    const int Is = L->sh_gate.out_dim;
+    const gq::Seg ds = seg_single(L->sh_down, nullptr, M, gq::A_ROWS);
+    const gq::Args a = gemm_args(ds, (H + gq::BN - 1) / gq::BN, Is, h_sh, Is,
+                                 yrows + n * (int64_t)H, H);
+    const int items = mtiles * ((H + gq::BN - 1) / gq::BN);
+    PCK(launch_gqmm(L->sh_down.bits, gq::EPI_STORE, a, items < sms ? items : sms, st));
+  }
+  // 7. combine in k order (+ sigmoid-gated shared expert, + residual)
+  PCK(launch_combine(yrows, wts, sigma, L->has_shared, residual, y, M, K, H, st));
+  return MOEQ_OK;
 }
 
 }  // namespace moeq

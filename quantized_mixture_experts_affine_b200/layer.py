@@ -59,6 +59,9 @@ CONFIGS = {
     "decode_30b": LayerConfig("decode_30b", H=2048, I=768, E=128, K=8, expert_bits=4),
     "decode_397b": LayerConfig("decode_397b", H=4096, I=1024, E=512, K=4, expert_bits=4,
                                shared=True, shared_I=1024, shared_bits=4),
+    # the 397B-like shapes with a 16-expert bank (profiling captures)
+    "decode_397b_e16": LayerConfig("decode_397b_e16", H=4096, I=1024, E=16, K=4, expert_bits=4,
+                                   shared=True, shared_I=1024, shared_bits=4),
     "prefill_8bit": LayerConfig("prefill_8bit", H=2048, I=768, E=128, K=8, expert_bits=8),
     "mixed_2bit": LayerConfig("mixed_2bit", H=4096, I=1024, E=512, K=4, expert_bits=2,
                               shared=True, shared_I=1024, shared_bits=4, requant_from4=True),

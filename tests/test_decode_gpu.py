@@ -184,13 +184,14 @@ def test_expert_ffn_zipf_routing_decode():
     xb, x = x_tokens(cfg, M, copy=11)
     y = expert_ffn(L, x, idx, w, mode=moeq.MODE_DECODE)
     torch.cuda.synchronize()
-    from helpers import oracle_expert_outputs
+    from helpers import oracle_expert_outputs, weights_for
     ig = idx.cpu().numpy()
-    # weights in fp64 from the same drawn logits
-    io, wo, _ = oracle.route_f32(logits, cfg.K, True, 1.0)
-    assert np.array_equal(np.sort(ig, 1), np.sort(io, 1))
+    io, _, gap = oracle.route_f32(logits, cfg.K, True, 1.0)
+    assert ((np.sort(ig, 1) == np.sort(io, 1)).all(1) | (gap < NEAR_TIE)).all()
     rows = np.arange(0, M, 4)
-    ref = oracle_expert_outputs(cfg, SEED, 0, xb[rows], ig[rows], wo[rows])
+    # fp64 weights of the GPU's selection from the same drawn logits
+    wref = weights_for(ig[rows], logits[rows], cfg)
+    ref = oracle_expert_outputs(cfg, SEED, 0, xb[rows], ig[rows], wref)
     got = y.cpu().numpy()[rows]
     assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
 

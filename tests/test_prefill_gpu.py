@@ -1,0 +1,201 @@
+"""Prefill path (sort by expert + tcgen05 gather-QMM) on the GPU against the
+fp64 oracle, through the C ABI.
+
+Bars: routing equal except at near-ties; layer outputs relative L2 <= 2e-3
+and max abs <= 1e-2; one-shot and 2048-token chunked outputs bitwise equal;
+outputs poisoned with two different values agree bitwise (no unwritten
+rows), on both sides of the n = M*K = 32768 seam with n % 64 != 0
+(mlx issue 3856: "Silent numerical corruption in single long forward on
+quantized MoE when sequence length % 32 != 0").
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import check_layer_outputs, oracle_expert_outputs, rel_l2, weights_for
+from quantized_mixture_experts_affine_b200 import moeq, synth
+from quantized_mixture_experts_affine_b200.layer import (CONFIGS, Workspace, expert_ffn,
+                                                         layer_forward, synthetic_layer)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+SEED = 0
+P = moeq.MODE_PREFILL
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def x_tokens(cfg, M, copy):
+    xb = synth.normal_bf16_host(SEED, synth.tag(synth.X, copy), M * cfg.H).reshape(M, cfg.H)
+    return xb, dev(xb.view(np.int16)).view(torch.bfloat16)
+
+
+_layers = {}
+
+
+def layer_of(name):
+    if name not in _layers:
+        _layers.clear()
+        torch.cuda.empty_cache()
+        _layers[name] = synthetic_layer(CONFIGS[name], SEED, 0)
+    return _layers[name]
+
+
+def forward(L, x, poison=float("nan"), ws=None):
+    M = x.shape[0]
+    y = torch.full((M, L.cfg.H), poison, device="cuda")
+    y, idx, w = layer_forward(L, x, y=y, ws=ws, mode=P)
+    torch.cuda.synchronize()
+    status = moeq.moeq_device_status()
+    assert status == 0, moeq.status_str(status)
+    return y, idx, w
+
+
+def chunked(L, x, chunk=2048):
+    M = x.shape[0]
+    ys, ids, ws_ = [], [], []
+    ws = Workspace(L, min(chunk, M), P)
+    for s in range(0, M, chunk):
+        y, idx, w = forward(L, x[s:s + chunk], ws=ws)
+        ys.append(y)
+        ids.append(idx)
+        ws_.append(w)
+    return torch.cat(ys), torch.cat(ids), torch.cat(ws_)
+
+
+def bits_equal(a, b):
+    return torch.equal(a.contiguous().view(torch.int32), b.contiguous().view(torch.int32))
+
+
+# ------------------------------------------------------------------ small cases, full parity
+
+@pytest.mark.parametrize("M", [1, 3, 5, 130])
+def test_prefill_tiny(M):
+    cfg = CONFIGS["tiny"]
+    L = layer_of("tiny")
+    xb, x = x_tokens(cfg, M, 40 + M)
+    y, idx, w = forward(L, x)
+    check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
+
+
+def test_prefill_matches_decode_routing_tiny():
+    """Both paths route identically and agree within the layer tolerance."""
+    cfg = CONFIGS["tiny"]
+    L = layer_of("tiny")
+    xb, x = x_tokens(cfg, 37, 7)
+    yp, ip, wp = forward(L, x)
+    yd, idd, wd = layer_forward(L, x, mode=moeq.MODE_DECODE)
+    torch.cuda.synchronize()
+    assert torch.equal(ip, idd)
+    assert rel_l2(yp.cpu().numpy(), yd.cpu().numpy()) < 2e-3
+
+
+def test_prefill_8bit_moderate():
+    """The 8-bit prefill layer at M = 300: several m-tiles per expert, ragged
+    tails; every token checked against the oracle."""
+    cfg = CONFIGS["prefill_8bit"]
+    L = layer_of("prefill_8bit")
+    xb, x = x_tokens(cfg, 300, 3)
+    y, idx, w = forward(L, x)
+    check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
+
+
+def test_prefill_residual_and_expert_ffn():
+    cfg = CONFIGS["prefill_8bit"]
+    L = layer_of("prefill_8bit")
+    M = 77
+    xb, x = x_tokens(cfg, M, 5)
+    res_np = np.linspace(-2, 2, M * cfg.H, dtype=np.float32).reshape(M, cfg.H)
+    y = torch.empty((M, cfg.H), device="cuda")
+    y, idx, w = layer_forward(L, x, y=y, residual=dev(res_np), mode=P)
+    torch.cuda.synchronize()
+    check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy(),
+                        residual=res_np)
+    y2 = expert_ffn(L, x, idx, w, mode=P)
+    y0, _, _ = forward(L, x)
+    torch.cuda.synchronize()
+    assert bits_equal(y2, y0)
+
+
+# ------------------------------------------------------------------ chunking and the 32768 seam
+
+@pytest.mark.parametrize("M", [4097, 4096 + 64])
+def test_prefill_chunk_invariance_seam(M):
+    """n = 8*M crosses 32768 (4097 -> n % 64 = 8; 4160 -> aligned control):
+    one-shot == 2048-chunked bitwise, poison-independent, sampled rows vs
+    the oracle."""
+    cfg = CONFIGS["prefill_8bit"]
+    L = layer_of("prefill_8bit")
+    xb, x = x_tokens(cfg, M, 100 + M)
+    y1, i1, w1 = forward(L, x, poison=float("nan"))
+    y2, i2, w2 = forward(L, x, poison=1e30)
+    assert torch.isfinite(y1).all()
+    assert bits_equal(y1, y2) and torch.equal(i1, i2)
+    yc, ic, wc = chunked(L, x)
+    assert bits_equal(y1, yc) and torch.equal(i1, ic) and bits_equal(w1, wc)
+    rows = np.unique(np.concatenate([np.arange(0, 8), np.arange(M - 8, M),
+                                     np.random.default_rng(M).integers(0, M, 48)]))
+    check_layer_outputs(cfg, SEED, 0, xb, y1.cpu().numpy(), i1.cpu().numpy(), w1.cpu().numpy(),
+                        rows=rows)
+
+
+@pytest.mark.parametrize("M", [16068, 16032, 16384])
+def test_prefill_full_size(M):
+    """The 16k-token prefill workloads (16068 is unaligned: n = 128544,
+    n % 64 = 32): one-shot == chunked bitwise, sampled rows vs oracle
+    including the last rows of the sorted order."""
+    cfg = CONFIGS["prefill_8bit"]
+    L = layer_of("prefill_8bit")
+    xb, x = x_tokens(cfg, M, 200)
+    y1, i1, w1 = forward(L, x)
+    assert torch.isfinite(y1).all()
+    yc, ic, wc = chunked(L, x)
+    assert bits_equal(y1, yc) and torch.equal(i1, ic)
+    ig = i1.cpu().numpy()
+    # tokens whose pairs sit in the last m-tile of some expert
+    rng = np.random.default_rng(M)
+    last = []
+    for e in rng.choice(cfg.E, 6, replace=False):
+        toks = np.nonzero((ig == e).any(1))[0]
+        last.extend(toks[-3:].tolist())
+    rows = np.unique(np.concatenate([np.array(last, dtype=np.int64), [0, M - 1],
+                                     rng.integers(0, M, 40)]))
+    check_layer_outputs(cfg, SEED, 0, xb, y1.cpu().numpy(), ig, w1.cpu().numpy(), rows=rows)
+
+
+# ------------------------------------------------------------------ mixed bank
+
+def test_prefill_mixed_2bit_router():
+    cfg = CONFIGS["mixed_2bit"]
+    L = layer_of("mixed_2bit")
+    xb, x = x_tokens(cfg, 256, 9)
+    y, idx, w = forward(L, x)
+    rows = np.arange(0, 256, 16)
+    check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy(),
+                        rows=rows)
+
+
+def test_prefill_mixed_2bit_zipf_4096():
+    """M = 4096 with router logits drawn for a Zipf(1.1) expert load."""
+    cfg = CONFIGS["mixed_2bit"]
+    L = layer_of("mixed_2bit")
+    M = 4096
+    logits, _ = synth.zipf_logits_host(SEED, synth.tag(synth.LOGITS, 1), M, cfg.E, 1.1)
+    idx = torch.empty((M, cfg.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((M, cfg.K), dtype=torch.float32, device="cuda")
+    moeq.moeq_route_topk(dev(logits), M, cfg.E, cfg.K, True, 1.0, idx, w)
+    xb, x = x_tokens(cfg, M, 12)
+    y = expert_ffn(L, x, idx, w, mode=P)
+    torch.cuda.synchronize()
+    assert moeq.moeq_device_status() == 0
+    ig = idx.cpu().numpy()
+    io, _, gap = oracle.route_f32(logits, cfg.K, True, 1.0)
+    assert ((np.sort(ig, 1) == np.sort(io, 1)).all(1) | (gap < 1e-5)).all()
+    rows = np.random.default_rng(4).integers(0, M, 24)
+    wref = weights_for(ig[rows], logits[rows], cfg)
+    ref = oracle_expert_outputs(cfg, SEED, 0, xb[rows], ig[rows], wref)
+    got = y.cpu().numpy()[rows]
+    assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
