@@ -22,7 +22,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -37,6 +36,12 @@ WORKLOADS = {
     "decode_397b_m8": ("decode_397b", 8),
     "decode_30b_m1": ("decode_30b", 1),
     "decode_mixed_2bit_m1": ("mixed_2bit", 1),
+    # prefill: one call over M tokens per step
+    "prefill_8bit_m16068": ("prefill_8bit", 16068),
+    "prefill_8bit_m16384": ("prefill_8bit", 16384),
+    "prefill_mixed_2bit_m4096": ("mixed_2bit", 4096),
+    # small prefill case for full profiler captures
+    "prefill_8bit_m2048": ("prefill_8bit", 2048),
 }
 METRIC = "qMoE layer tokens/s"
 
@@ -53,6 +58,9 @@ def parse():
                     help="tokens of the bounded oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the secondary prefill measurement of the decode run")
+    ap.add_argument("--prefill-workload", default="prefill_8bit_m16068")
     return ap.parse_args()
 
 
@@ -91,53 +99,74 @@ def max_over_ranks(v, world):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi samples (200 ms) during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled through NVML (read-only) every
+    ~1 ms from a background thread for the duration of the timed region."""
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
-        self.p = None
-        self.path = os.path.join("/tmp", f"moeq_clocks_{os.getpid()}.csv")
+        self.samples = []
+        self.err = None
+        self._stop = False
+        self._thread = None
+
+    def _sample(self, nv, h):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        self.samples.append((sm, r))
+
+    def _run(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            dev = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = self.gpu
+            if dev:
+                ids = [d for d in dev.split(",") if d.strip()]
+                if self.gpu < len(ids) and ids[self.gpu].strip().isdigit():
+                    idx = int(ids[self.gpu])
+            h = nv.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._sample(nv, h)
+            self._ready = True
+            while not self._stop:
+                time.sleep(0.001)
+                self._sample(nv, h)
+            self._sample(nv, h)
+            nv.nvmlShutdown()
+        except Exception as e:  # no NVML: report it, never guess
+            self.err = repr(e)
+            self._ready = True
 
     def __enter__(self):
-        try:
-            self.f = open(self.path, "w")
-            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
-                                      stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.p = None
+        import threading
+        self._ready = False
+        self.max_mhz = None
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        t0 = time.time()
+        while not self._ready and time.time() - t0 < 10:
+            time.sleep(0.001)
         return self
 
     def __exit__(self, *a):
-        if self.p is not None:
-            self.p.terminate()
-            try:
-                self.p.wait(timeout=5)
-            except Exception:
-                self.p.kill()
-            self.f.close()
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=10)
 
     def summary(self):
-        if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+        if self.err or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": [f"clock sampling unavailable: {self.err}"]}
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items()
+                          if r & bit})
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "source": "NVML, ~1 ms period, during the timed region"}
 
 
 def measured_peaks():
@@ -221,6 +250,113 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ prefill measurement
+def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True):
+    """Timed one-shot prefill calls of `workload` (M tokens each): device
+    throughput, the gate/up gather-QMM duration per launch (events around it
+    inside captured graphs), tensor-core roofline and end-to-end rate."""
+    import torch
+    from quantized_mixture_experts_affine_b200 import moeq, synth
+    from quantized_mixture_experts_affine_b200.layer import CONFIGS, Workspace, synthetic_layer
+    cfg_name, M = WORKLOADS[workload]
+    cfg = CONFIGS[cfg_name]
+    L = synthetic_layer(cfg, seed, 0)
+    n_x = 2
+    xs = synth.normal_bf16_dev(seed, synth.tag(synth.X, 555), n_x * M * cfg.H).view(n_x, M, cfg.H)
+    y = torch.empty((M, cfg.H), dtype=torch.float32, device="cuda")
+    idx = torch.empty((M, cfg.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((M, cfg.K), dtype=torch.float32, device="cuda")
+    ws = Workspace(L, M, moeq.MODE_PREFILL)
+    st = torch.cuda.Stream()
+
+    def step(i):
+        moeq.moeq_layer_forward(L.desc, xs[i % n_x], M, y, None, idx, w, ws.buf, ws.bytes,
+                                moeq.MODE_PREFILL, st)
+
+    with torch.cuda.stream(st):
+        for i in range(warmup):
+            step(i)
+    st.synchronize()
+    g = torch.cuda.CUDAGraph()
+    n0 = moeq.moeq_launch_count()
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for i in range(steps):
+                step(i)
+    launches = moeq.moeq_launch_count() - n0
+    with torch.cuda.stream(st):
+        g.replay()
+    st.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        with torch.cuda.stream(st):
+            e0.record(st)
+            g.replay()
+            e1.record(st)
+        st.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    # gate/up gather-QMM per launch
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for e in starts + stops:
+        e.record(st)
+    st.synchronize()
+    kg = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(kg, stream=st):
+            for i in range(steps):
+                moeq.moeq_set_profile_events(starts[i], stops[i])
+                step(i)
+        moeq.moeq_set_profile_events(None, None)
+        kg.replay()
+    st.synchronize()
+    k_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, stops)) / steps, world)
+    n_pairs = M * cfg.K
+    gu_flop = 2.0 * n_pairs * 2 * cfg.I * cfg.H
+    layer_flop = M * cfg.flops_per_token()
+    _, peak_bf16, peak_kind = measured_peaks()
+    out = {"workload": workload, "tokens_per_step": M, "value": M * world / (ms / 1e3),
+           "unit": "tokens/s", "ms_per_step": ms,
+           "layer_tflops": layer_flop / (ms / 1e3) / 1e12,
+           "roofline": {"bound": "tensor", "kernel": "k_gqmm gate/up+SwiGLU (fp16 operands)",
+                        "achieved": gu_flop / (k_ms / 1e3) / 1e12, "peak": peak_bf16,
+                        "unit": "TFLOP/s", "frac": gu_flop / (k_ms / 1e3) / 1e12 / peak_bf16,
+                        "traffic": None, "flop_per_launch": gu_flop, "ms_per_launch": k_ms,
+                        "peak_kind": peak_kind + " bf16 dense (fp16 equal rate)"},
+           "gpu_launches": int(launches), "clocks": clk.summary()}
+    if want_e2e:
+        xh = xs[0].cpu().pin_memory()
+        yh = torch.empty((M, cfg.H), dtype=torch.float32).pin_memory()
+        xdev = torch.empty((M, cfg.H), dtype=torch.bfloat16, device="cuda")
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(st):
+            a0.record(st)
+            for i in range(steps):
+                xdev.copy_(xh, non_blocking=True)
+                moeq.moeq_layer_forward(L.desc, xdev, M, y, None, idx, w, ws.buf, ws.bytes,
+                                        moeq.MODE_PREFILL, st)
+                yh.copy_(y, non_blocking=True)
+            a1.record(st)
+        st.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), world) / steps
+        out["e2e"] = {"value": M * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": M * cfg.H * 2, "d2h_bytes_per_step": M * cfg.H * 4}
+    out["device_status"] = moeq.moeq_device_status(st)
+    g.reset()
+    kg.reset()
+    del L, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import torch
@@ -230,6 +366,8 @@ def run_ours(args):
     rank, world, local = dist_setup(args.gpus)
     cfg_name, M = WORKLOADS[args.workload]
     cfg = CONFIGS[cfg_name]
+    if args.workload.startswith("prefill"):
+        return run_prefill_main(args, rank, world)
     K, W = args.steps, args.warmup
     assert W >= 3, "at least 3 warm-up steps"
     copies = max(1, args.copies)
@@ -384,6 +522,43 @@ def run_ours(args):
                                           f"one oracle call ({dt:.2f} s)"}
     for g in graphs + kgraphs:
         g.reset()
+    if not args.no_prefill:
+        del layers
+        torch.cuda.empty_cache()
+        line["prefill"] = measure_prefill(args.prefill_workload, max(3, min(K, 20)), W, world,
+                                          seed, want_e2e=not args.no_e2e)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_prefill_main(args, rank, world):
+    """A prefill workload as the main line: value = tokens/s of one-shot calls."""
+    cfg_name, M = WORKLOADS[args.workload]
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    p = measure_prefill(args.workload, args.steps, args.warmup, world, 1000 * rank,
+                        want_e2e=not args.no_e2e)
+    line = {"metric": METRIC, "value": p["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": p["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "tokens_per_step": M,
+                       "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (weights, token rows and output rows)",
+                       "cuda_graph": True},
+            "layer_tflops": p["layer_tflops"], "roofline": p["roofline"], "e2e": p.get("e2e"),
+            "gpu_launches": p["gpu_launches"], "clocks": p["clocks"],
+            "device_status": p["device_status"]}
+    if rank == 0 and not args.no_cpu_baseline:
+        from quantized_mixture_experts_affine_b200.layer import CONFIGS
+        smp = OracleSample(CONFIGS[cfg_name], args.cpu_sample)
+        dt = smp.run(list(range(args.cpu_sample)))
+        line["cpu_baseline"] = {"value": args.cpu_sample / dt, "unit": "tokens/s",
+                                "cores": smp.cores(args.cpu_sample), "kind": "oracle",
+                                "sample": f"{args.cpu_sample} tokens of {args.workload}, "
+                                          f"one oracle call ({dt:.2f} s)"}
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -56,7 +56,12 @@ struct Smem {
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024
 };
 
-enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1 };
+// SWIGLU: tile rows 0-127 gate, 128-255 up -> fp16 silu(g)*u.
+// STORE:  256 weight rows -> fp32 outputs.
+// SPLIT:  tile rows 0-127 hold fp16(w) and rows 128-255 fp16(w - fp16(w))
+//         of the same 128 weight rows; output = sum of the two products
+//         (fp32-accurate logits for the routing decision).
+enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_SPLIT = 2 };
 enum AMode { A_PAIRS = 0, A_TOKENS = 1, A_ROWS = 2 };
 
 // One expert (or the shared expert, or the router) over a run of sorted rows.
@@ -120,6 +125,11 @@ __device__ __forceinline__ void b_row(const Seg& sg, int nt, int r, int& src, in
     src = r >= 128;
     q = nt * 128 + (r & 127);
     ok = q < sg.n0;
+  } else if (EPI == EPI_SPLIT) {
+    const int g = nt * 128 + (r & 127);
+    src = g >= sg.n0;
+    q = src ? g - sg.n0 : g;
+    ok = g < sg.n_valid;
   } else {
     const int g = nt * BN + r;
     src = g >= sg.n0;
@@ -209,6 +219,34 @@ __device__ __forceinline__ void dequant_chunk(uint4 raw, __half2 s2, __half2 b2,
 
 __device__ __forceinline__ int2 tile_of(const Args& a, int mt) {
   return a.tiles ? a.tiles[mt] : make_int2(0, mt * BM);
+}
+
+// Split dequantisation for the router tiles: w = fmaf(q, scale, bias) in
+// fp32, written as fp16(w) (LO = false) or fp16(w - fp16(w)) (LO = true).
+template <int BITS, bool LO>
+__device__ __forceinline__ void dequant_chunk_split(uint4 raw, float s, float b, uint32_t bstage,
+                                                    int r, int c16) {
+  constexpr int VPC = 128 / BITS;
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[VPC / 2];
+#pragma unroll
+  for (int i = 0; i < VPC / 2; ++i) {
+    float v[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int k = 2 * i + j;  // value index within the chunk
+      const int word = k / (32 / BITS), pos = k % (32 / BITS);
+      const uint32_t q = (w[word] >> (BITS * pos)) & ((1u << BITS) - 1u);
+      const float wf = __fmaf_rn((float)q, s, b);
+      const float hi = __half2float(__float2half_rn(wf));
+      v[j] = LO ? wf - hi : wf;
+    }
+    o[i] = h2u(__floats2half2_rn(v[0], v[1]));
+  }
+#pragma unroll
+  for (int k = 0; k < VPC / 8; ++k)
+    sts128(bstage + tc::sw128_offset(r, c16 + k), o[4 * k], o[4 * k + 1], o[4 * k + 2],
+           o[4 * k + 3]);
 }
 
 template <int BITS, int EPI>
@@ -413,6 +451,21 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           }
         }
         if (bad) set_status(status, MOEQ_ERR_RANGE);
+      } else if (EPI == EPI_SPLIT) {
+        float* out = reinterpret_cast<float*>(a.out) + m * a.ldo + nt * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t hv[32], lv[32];
+          tc::tmem_ld32(tb + c0, hv);
+          tc::tmem_ld32(tb + 128 + c0, lv);
+          tc::tmem_wait_ld();
+          const int col = nt * 128 + c0;
+          if (ok && col < sg.n_valid) {
+            const int nv = min(32, sg.n_valid - col);
+            for (int k = 0; k < nv; ++k)
+              out[c0 + k] = __uint_as_float(hv[k]) + __uint_as_float(lv[k]);
+          }
+        }
       } else {
         int64_t dest = m;
         if (ok && sg.dest_pairs) dest = a.sorted_pair[m];
@@ -460,11 +513,19 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           const int r = idx / RW::CHUNKS, c = idx % RW::CHUNKS;
           const uint4 raw = lds128(rst + r * RW::ROW + c * 16);
           const uint2 sb = lds64(sbst + r * 8);
-          __half2 s2h, b2h;
-          group_h2<BITS>(hi ? (sb.x >> 16) : (sb.x & 0xFFFFu), hi ? (sb.y >> 16) : (sb.y & 0xFFFFu),
-                         s2h, b2h, status);
+          const uint32_t sbits = hi ? (sb.x >> 16) : (sb.x & 0xFFFFu);
+          const uint32_t bbits = hi ? (sb.y >> 16) : (sb.y & 0xFFFFu);
           // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
-          dequant_chunk<BITS>(raw, s2h, b2h, bst, r, c * (16 / BITS));
+          if (EPI == EPI_SPLIT) {
+            const float sf = bf16_bits_to_float((uint16_t)sbits);
+            const float bf = bf16_bits_to_float((uint16_t)bbits);
+            if (r < 128) dequant_chunk_split<BITS, false>(raw, sf, bf, bst, r, c * (16 / BITS));
+            else dequant_chunk_split<BITS, true>(raw, sf, bf, bst, r, c * (16 / BITS));
+          } else {
+            __half2 s2h, b2h;
+            group_h2<BITS>(sbits, bbits, s2h, b2h, status);
+            dequant_chunk<BITS>(raw, s2h, b2h, bst, r, c * (16 / BITS));
+          }
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(&b_full[s2]);

@@ -227,6 +227,11 @@ cudaError_t launch_gqmm_t(const gq::Args& a, int grid, cudaStream_t st) {
 
 cudaError_t launch_gqmm(int bits, int epi, const gq::Args& a, int grid, cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
+  if (epi == gq::EPI_SPLIT) {
+    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SPLIT>(a, grid, st);
+    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SPLIT>(a, grid, st);
+    return launch_gqmm_t<2, gq::EPI_SPLIT>(a, grid, st);
+  }
   if (epi == gq::EPI_SWIGLU) {
     if (bits == 8) return launch_gqmm_t<8, gq::EPI_SWIGLU>(a, grid, st);
     if (bits == 4) return launch_gqmm_t<4, gq::EPI_SWIGLU>(a, grid, st);
@@ -405,16 +410,17 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     return a;
   };
   if (!idx_in) {
+    // hi/lo split weights: fp32-accurate logits for the top-K decision
     const gq::Seg rs = seg_single(L->router, sgr ? &L->sh_expert_gate : nullptr, M, gq::A_TOKENS);
-    const int nt = (rs.n_valid + gq::BN - 1) / gq::BN;
+    const int nt = (rs.n_valid + 127) / 128;
     const gq::Args a = gemm_args(rs, nt, H, x16, H, logits, lay.ld_logits);
     const int items = mtiles * nt;
-    PCK(launch_gqmm(L->router.bits, gq::EPI_STORE, a, items < sms ? items : sms, st));
+    PCK(launch_gqmm(L->router.bits, gq::EPI_SPLIT, a, items < sms ? items : sms, st));
   }
   if (L->has_shared && (idx_in || !sgr)) {
     const gq::Seg gs = seg_single(L->sh_expert_gate, nullptr, M, gq::A_TOKENS);
     const gq::Args a = gemm_args(gs, 1, H, x16, H, logits + E, lay.ld_logits);
-    PCK(launch_gqmm(L->sh_expert_gate.bits, gq::EPI_STORE, a, mtiles < sms ? mtiles : sms, st));
+    PCK(launch_gqmm(L->sh_expert_gate.bits, gq::EPI_SPLIT, a, mtiles < sms ? mtiles : sms, st));
   }
 
   // 3. routing
