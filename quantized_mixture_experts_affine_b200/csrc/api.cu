@@ -117,12 +117,28 @@ static moeq_status check_layer(const moeq_layer* L) {
   return MOEQ_OK;
 }
 
+// Decode GEMV limits: rows of at most 4096 bytes of codes, an even number
+// of groups per row (4-byte scale/bias copies), 4-byte aligned scale/bias
+// arrays and bank strides, and a work unit that fits one pipeline stage.
+static moeq_status check_gemv_tensor(const moeq_qtensor& t, int nmat) {
+  if (slices_of(t) > 8) return MOEQ_ERR_UNSUPPORTED;
+  if ((t.in_dim / t.group_size) % 2) return MOEQ_ERR_UNSUPPORTED;
+  if (((uintptr_t)t.scales & 3) || ((uintptr_t)t.biases & 3) || (t.expert_stride_sb & 1))
+    return MOEQ_ERR_ALIGNMENT;
+  if (!gemv_fits(t.in_dim, t.bits, nmat, t.group_size)) return MOEQ_ERR_UNSUPPORTED;
+  return MOEQ_OK;
+}
+
 static moeq_status check_decode_shapes(const moeq_layer* L) {
-  const moeq_qtensor* ts[8] = {&L->router, &L->gate, &L->down, &L->sh_gate, &L->sh_down,
-                               &L->sh_expert_gate, nullptr, nullptr};
-  const int n = L->has_shared ? 6 : 3;
-  for (int i = 0; i < n; ++i)
-    if (slices_of(*ts[i]) > 8) return MOEQ_ERR_UNSUPPORTED;
+  moeq_status s;
+  if ((s = check_gemv_tensor(L->router, 1)) != MOEQ_OK) return s;
+  if ((s = check_gemv_tensor(L->gate, 2)) != MOEQ_OK) return s;
+  if ((s = check_gemv_tensor(L->down, 1)) != MOEQ_OK) return s;
+  if (L->has_shared) {
+    if ((s = check_gemv_tensor(L->sh_expert_gate, 1)) != MOEQ_OK) return s;
+    if ((s = check_gemv_tensor(L->sh_gate, 2)) != MOEQ_OK) return s;
+    if ((s = check_gemv_tensor(L->sh_down, 1)) != MOEQ_OK) return s;
+  }
   return MOEQ_OK;
 }
 
@@ -170,12 +186,8 @@ static int resolve_mode(int mode, int M) {
 }
 
 // ------------------------------------------------------------------ GEMV helpers
-static constexpr int kR = 8;  // rows per warp-task on the decode path
-
-static int units_for(int out_dim, int slices) {
-  const GemvShape sh = gemv_shape(slices, kR);
-  const int rows = sh.R * sh.rbs;
-  return (out_dim + rows - 1) / rows;
+static int units_for(const moeq_qtensor& t, int out_dim, int nmat) {
+  return gemv_units(out_dim, gemv_shape(t.in_dim, t.bits, nmat, t.group_size));
 }
 
 static int grid_cap() {
@@ -187,7 +199,29 @@ static int grid_cap() {
       n = 148;
     sms = n;
   }
-  return sms * 2;
+  return sms;
+}
+
+static void set_shape(GemvArgs& a, const moeq_qtensor& t, int nmat) {
+  const GemvShape sh = gemv_shape(t.in_dim, t.bits, nmat, t.group_size);
+  a.in_dim = t.in_dim;
+  a.G = t.group_size;
+  a.slices = sh.S;
+  a.subsets = sh.J;
+  a.rows_per_unit = sh.RU;
+}
+
+// Pull a whole tensor (matrix `expert` of a bank) into L2: codes, scales, biases.
+static int add_prefetch(GemvArgs& a, const moeq_qtensor& t, int expert) {
+  const int64_t words = (int64_t)t.out_dim * t.in_dim * t.bits / 32;
+  const int64_t groups = (int64_t)t.out_dim * (t.in_dim / t.group_size);
+  const void* p[3] = {t.w + (int64_t)expert * t.expert_stride_w,
+                      t.scales + (int64_t)expert * t.expert_stride_sb,
+                      t.biases + (int64_t)expert * t.expert_stride_sb};
+  const int64_t b[3] = {words * 4, groups * 2, groups * 2};
+  for (int i = 0; i < 3 && a.n_pf < kMaxPrefetch; ++i)
+    if (((uintptr_t)p[i] & 15) == 0) a.pf[a.n_pf++] = PrefetchRange{p[i], b[i]};
+  return a.n_pf;
 }
 
 // x [M][in] (bf16) times one matrix -> y with row stride `ystride`.
@@ -204,6 +238,7 @@ static Seg plain_seg(const moeq_qtensor& t, int expert, const void* src, int64_t
   s.out_dim = t.out_dim;
   s.in_dim = t.in_dim;
   s.G = t.group_size;
+  s.bits = t.bits;
   s.n_vec = n_vec;
   s.unit_begin = unit_begin;
   s.vec_mode = 0;
@@ -215,34 +250,39 @@ static Seg plain_seg(const moeq_qtensor& t, int expert, const void* src, int64_t
   return s;
 }
 
-static cudaError_t run_plain(const Seg* segs, int n, int bits, int nl, int slices,
-                             cudaStream_t st) {
+// Segments of one format (the first segment's tensor gives the shape).
+static cudaError_t run_plain(const moeq_qtensor& shape_t, const Seg* segs, int n, int nl,
+                             GemvArgs* pf, cudaStream_t st) {
   GemvArgs a;
-  memset(&a, 0, sizeof(a));
+  if (pf) a = *pf; else memset(&a, 0, sizeof(a));
+  set_shape(a, shape_t, 1);
+  const GemvShape sh = gemv_shape(shape_t.in_dim, shape_t.bits, 1, shape_t.group_size);
   int units = 0;
   for (int i = 0; i < n; ++i) {
     a.segs[i] = segs[i];
     a.segs[i].unit_begin = units;
-    units += units_for(segs[i].out_dim, slices);
+    units += gemv_units(segs[i].out_dim, sh);
   }
   a.n_segs = n;
   a.total_units = units;
-  a.slices = slices;
   a.status = status_ptr();
   const int grid = units < grid_cap() ? units : grid_cap();
-  return launch_gemv(bits, nl, 1, kR, SRC_BF16, a, grid, st);
+  return launch_gemv(shape_t.bits, nl, 1, SRC_BF16, a, grid, st);
 }
 
-static cudaError_t run_dyn(const Seg* segs, const int32_t* count, int bits, int nl, int nmat,
-                           int src, int slices, int max_units, cudaStream_t st) {
+static cudaError_t run_dyn(const moeq_qtensor& shape_t, const Seg* segs, const int32_t* count,
+                           int nl, int nmat, int src, int max_units, cudaStream_t st,
+                           const Seg* pf_segs = nullptr, const int32_t* pf_count = nullptr) {
   GemvArgs a;
   memset(&a, 0, sizeof(a));
+  set_shape(a, shape_t, nmat);
   a.dyn_segs = segs;
   a.dyn_count = count;
-  a.slices = slices;
+  a.pf_segs = pf_segs;
+  a.pf_count = pf_count;
   a.status = status_ptr();
   const int grid = max_units < grid_cap() ? max_units : grid_cap();
-  return launch_gemv(bits, nl, nmat, kR, src, a, grid, st);
+  return launch_gemv(shape_t.bits, nl, nmat, src, a, grid, st);
 }
 
 #define CK(x)                                     \
@@ -282,18 +322,28 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   //    two 8-bit tensors agree in format)
   const moeq_qtensor& R = L->router;
   const moeq_qtensor& SG = L->sh_expert_gate;
-  const int sr = slices_of(R);
-  const bool sg_with_router = L->has_shared && SG.bits == R.bits && slices_of(SG) == sr;
+  const bool sg_with_router = L->has_shared && SG.bits == R.bits &&
+                              SG.group_size == R.group_size && SG.in_dim == R.in_dim;
+  // the shared expert's weights do not depend on the routing: pull them into
+  // L2 while the router streams
+  GemvArgs pf;
+  memset(&pf, 0, sizeof(pf));
+  if (L->has_shared) {
+    add_prefetch(pf, L->sh_gate, 0);
+    add_prefetch(pf, L->sh_up, 0);
+    add_prefetch(pf, L->sh_down, 0);
+  }
   if (!idx_in) {
     Seg segs[2];
     int ns = 0;
     segs[ns++] = plain_seg(R, 0, x, H, logits, E, M, 0);
     if (sg_with_router) segs[ns++] = plain_seg(SG, 0, x, H, sg_logit, 1, M, 0);
-    LAUNCH(run_plain(segs, ns, R.bits, 3, sr, st));
+    LAUNCH(run_plain(R, segs, ns, 3, &pf, st));
+    pf.n_pf = 0;
   }
   if (L->has_shared && (idx_in || !sg_with_router)) {
     Seg s = plain_seg(SG, 0, x, H, sg_logit, 1, M, 0);
-    LAUNCH(run_plain(&s, 1, SG.bits, 3, slices_of(SG), st));
+    LAUNCH(run_plain(SG, &s, 1, 3, &pf, st));
   }
 
   // 2. routing + grouped plan
@@ -331,18 +381,18 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   p.count_dn = counts + 4;
   p.vecs_gu = vecs_gu;
   p.vecs_dn = vecs_dn;
-  const int s_gu = slices_of(L->gate), s_dn = slices_of(L->down);
-  p.units_per_seg_gu = units_for(I, s_gu);
-  p.units_per_seg_dn = units_for(H, s_dn);
-  int s_gu_sh = 0, s_dn_sh = 0;
+  p.units_per_seg_gu = units_for(L->gate, I, 2);
+  p.units_per_seg_dn = units_for(L->down, H, 1);
   if (L->has_shared) {
-    s_gu_sh = slices_of(L->sh_gate);
-    s_dn_sh = slices_of(L->sh_down);
-    p.units_per_seg_gu_sh = units_for(L->sh_gate.out_dim, s_gu_sh);
-    p.units_per_seg_dn_sh = units_for(H, s_dn_sh);
-    p.shared_same_gu = (L->sh_gate.bits == L->gate.bits && s_gu_sh == s_gu);
-    p.shared_same_dn = (L->sh_down.bits == L->down.bits && s_dn_sh == s_dn);
+    p.units_per_seg_gu_sh = units_for(L->sh_gate, L->sh_gate.out_dim, 2);
+    p.units_per_seg_dn_sh = units_for(L->sh_down, H, 1);
+    p.shared_same_gu = (L->sh_gate.bits == L->gate.bits &&
+                        L->sh_gate.group_size == L->gate.group_size);
+    p.shared_same_dn = (L->sh_down.bits == L->down.bits &&
+                        L->sh_down.group_size == L->down.group_size &&
+                        L->sh_down.in_dim == L->down.in_dim);
   }
+  p.prefetch = 0;
   p.status = status_ptr();
   LAUNCH(launch_decode_plan(p, st));
 
@@ -351,15 +401,16 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   const int max_gu = max_entries * p.units_per_seg_gu + (p.shared_same_gu ? p.units_per_seg_gu_sh : 0);
   const int max_dn = max_entries * p.units_per_seg_dn + (p.shared_same_dn ? p.units_per_seg_dn_sh : 0);
   CK(profile_mark(true, st));
-  LAUNCH(run_dyn(segs_gu, counts, L->gate.bits, 2, 2, SRC_BF16, s_gu, max_gu, st));
+  // the gate/up launch also pulls the down projections it will feed into L2
+  LAUNCH(run_dyn(L->gate, segs_gu, counts, 2, 2, SRC_BF16, max_gu, st, segs_dn, counts + 4));
   CK(profile_mark(false, st));
   if (L->has_shared && !p.shared_same_gu)
-    LAUNCH(run_dyn(segs_gu + n, counts + 2, L->sh_gate.bits, 2, 2, SRC_BF16, s_gu_sh,
-                   p.units_per_seg_gu_sh, st));
-  LAUNCH(run_dyn(segs_dn, counts + 4, L->down.bits, 2, 1, SRC_F32, s_dn, max_dn, st));
+    LAUNCH(run_dyn(L->sh_gate, segs_gu + n, counts + 2, 2, 2, SRC_BF16, p.units_per_seg_gu_sh,
+                   st));
+  LAUNCH(run_dyn(L->down, segs_dn, counts + 4, 2, 1, SRC_F32, max_dn, st));
   if (L->has_shared && !p.shared_same_dn)
-    LAUNCH(run_dyn(segs_dn + n, counts + 6, L->sh_down.bits, 2, 1, SRC_F32, s_dn_sh,
-                   p.units_per_seg_dn_sh, st));
+    LAUNCH(run_dyn(L->sh_down, segs_dn + n, counts + 6, 2, 1, SRC_F32, p.units_per_seg_dn_sh,
+                   st));
 
   // 5. weighted combine in k order (+ shared, + residual)
   LAUNCH(launch_combine(d, wts, sigma, L->has_shared, residual, y, M, K, H, st));
@@ -402,10 +453,10 @@ MOEQ_API moeq_status moeq_qmv(const moeq_qtensor* t, int32_t expert, const uint1
   if (s != MOEQ_OK) return s;
   if (expert > 0 && (t->expert_stride_w <= 0 || t->expert_stride_sb <= 0))
     return MOEQ_ERR_INVALID_ARG;
-  if (slices_of(*t) > 8) return MOEQ_ERR_UNSUPPORTED;
+  if ((s = check_gemv_tensor(*t, 1)) != MOEQ_OK) return s;
   if (!aligned(x, 16) || ((int64_t)t->in_dim * 2) % 16 || !aligned(y, 4)) return MOEQ_ERR_ALIGNMENT;
   Seg seg = plain_seg(*t, expert, x, t->in_dim, y, t->out_dim, M, 0);
-  LAUNCH(run_plain(&seg, 1, t->bits, 3, slices_of(*t), (cudaStream_t)stream));
+  LAUNCH(run_plain(*t, &seg, 1, 3, nullptr, (cudaStream_t)stream));
   return MOEQ_OK;
 }
 

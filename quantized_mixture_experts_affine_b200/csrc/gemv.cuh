@@ -169,6 +169,20 @@ __device__ __forceinline__ float chunk_contrib(const uint32_t (&c)[Chunk<BITS>::
   return acc;
 }
 
+__device__ __forceinline__ uint4 gq_lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
 // Transposing butterfly: every lane holds v[0..R); afterwards lane l holds
 // sum over all lanes of v[l % R] (returned).  R in {8, 16, 32}.
 template <int R>

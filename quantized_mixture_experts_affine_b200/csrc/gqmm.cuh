@@ -11,9 +11,9 @@
 //              fp32 accumulators in TMEM (two 256-column buffers);
 //   warps 4-7  epilogue: tcgen05.ld of the accumulator rows, SwiGLU to fp16
 //              hidden rows, or fp32 output rows scattered to pair order;
-//   warps 8-11 dequantiser: codes -> fp16 weights w = q*scale + bias (one
+//   warps 8-15 dequantiser: codes -> fp16 weights w = q*scale + bias (one
 //              fused fp16 multiply-add of exact operands) written into the
-//              swizzled B stage.
+//              swizzled B stage, one weight row per thread.
 // The scale and bias of a 64-wide group are constant along K within a
 // k-block, so dequantising tiles in shared memory applies the affine map of
 // the pages' format exactly once per weight before the tensor-core product.
@@ -28,19 +28,30 @@ namespace moeq {
 namespace gq {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int S1 = 4;  // stages of A, packed B, scale/bias
-constexpr int S2 = 2;  // stages of dequantised B
+constexpr int S1 = 4;  // stages of A (gathered token rows)
+constexpr int SR = 3;  // stages of packed B codes and scale/bias pairs
+constexpr int S2 = 3;  // stages of dequantised B
 constexpr int A_STAGE = BM * BK * 2;   // 16 KB
 constexpr int B_STAGE = BN * BK * 2;   // 32 KB
 constexpr int SB_STAGE = BN * 8;       // scale pair + bias pair per row: 2 KB
-constexpr int THREADS = 384;
+constexpr int DQ_WARPS = 8;            // dequantiser warps: one weight row per thread
+constexpr int THREADS = (8 + DQ_WARPS) * 32;
 constexpr uint32_t IDESC = tc::idesc_f16_f32(BM, BN);
 
+// Packed codes of one k-block in shared memory, one row per dequantiser
+// thread.  Rows are laid out so that eight consecutive rows read by a
+// quarter-warp touch distinct 16-byte bank groups: 8-bit rows (64 bytes)
+// swizzle their 4 chunks by (row >> 1) & 3, 4-bit rows (32 bytes) are
+// padded to 48 bytes, 2-bit rows (16 bytes) are contiguous.
 template <int BITS>
 struct Raw {
   static constexpr int ROW = BK * BITS / 8;       // packed bytes of one row per k-block
-  static constexpr int STAGE = BN * ROW;          // 16/8/4 KB
   static constexpr int CHUNKS = ROW / 16;         // 16-byte chunks per row
+  static constexpr int STRIDE = BITS == 4 ? 48 : ROW;
+  static constexpr int STAGE = BN * STRIDE;
+  __device__ __forceinline__ static int offset(int r, int c) {
+    return BITS == 8 ? r * ROW + ((c ^ ((r >> 1) & 3)) << 4) : r * STRIDE + (c << 4);
+  }
 };
 
 template <int BITS>
@@ -48,19 +59,15 @@ struct Smem {
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = A_OFF + S1 * A_STAGE;
   static constexpr int RAW_OFF = B_OFF + S2 * B_STAGE;
-  static constexpr int SB_OFF = RAW_OFF + S1 * Raw<BITS>::STAGE;
-  static constexpr int BAR_OFF = SB_OFF + S1 * SB_STAGE;
-  static constexpr int N_BARS = 5 * S1 + 2 * S2 + 4;
-  static constexpr int TMEM_OFF = BAR_OFF + N_BARS * 8;
+  static constexpr int SB_OFF = RAW_OFF + SR * Raw<BITS>::STAGE;
+  static constexpr int BAR_OFF = SB_OFF + SR * SB_STAGE;
+  static constexpr int N_BARS = 2 * S1 + 2 * SR + 2 * S2 + 4;
+  static constexpr int ATAB_OFF = BAR_OFF + N_BARS * 8;   // 2 x 128 A-row pointers
+  static constexpr int TMEM_OFF = ATAB_OFF + 2 * BM * 8;
   static constexpr int BYTES = TMEM_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024
 };
 
-// SWIGLU: tile rows 0-127 gate, 128-255 up -> fp16 silu(g)*u.
-// STORE:  256 weight rows -> fp32 outputs.
-// SPLIT:  tile rows 0-127 hold fp16(w) and rows 128-255 fp16(w - fp16(w))
-//         of the same 128 weight rows; output = sum of the two products
-//         (fp32-accurate logits for the routing decision).
 enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_SPLIT = 2 };
 enum AMode { A_PAIRS = 0, A_TOKENS = 1, A_ROWS = 2 };
 
@@ -259,26 +266,27 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);
   uint64_t* full_a = bars;               // S1, A loader -> MMA
   uint64_t* a_empty = bars + S1;         // S1, MMA -> A loader
-  uint64_t* raw_full = bars + 2 * S1;    // S1, B loader -> dequant
-  uint64_t* raw_empty = bars + 3 * S1;   // S1, dequant -> B loader
-  uint64_t* sb_unused = bars + 4 * S1;   // S1 (reserved)
-  uint64_t* b_full = bars + 5 * S1;      // S2, dequant -> MMA
+  uint64_t* raw_full = bars + 2 * S1;    // SR, B loader -> dequant
+  uint64_t* raw_empty = raw_full + SR;   // SR, dequant -> B loader
+  uint64_t* b_full = raw_empty + SR;     // S2, dequant -> MMA
   uint64_t* b_empty = b_full + S2;       // S2, MMA -> dequant
   uint64_t* tmem_full = b_empty + S2;    // 2, MMA -> epilogue
   uint64_t* tmem_empty = tmem_full + 2;  // 2, epilogue -> MMA
+  const __half** atab = reinterpret_cast<const __half**>(smem + SM::ATAB_OFF);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::TMEM_OFF);
-  (void)sb_unused;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < S1; ++i) {
       tc::mbar_init(&full_a[i], 64);
       tc::mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < SR; ++i) {
       tc::mbar_init(&raw_full[i], 32);
-      tc::mbar_init(&raw_empty[i], 128);
+      tc::mbar_init(&raw_empty[i], DQ_WARPS * 32);
     }
     for (int i = 0; i < S2; ++i) {
-      tc::mbar_init(&b_full[i], 128);
+      tc::mbar_init(&b_full[i], DQ_WARPS * 32);
       tc::mbar_init(&b_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -302,37 +310,46 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
 
   if (warp < 2) {
     // ------------------------------------------------------------ A loader
-    const int t = threadIdx.x;  // 0..63: tile rows 2t, 2t+1
-    uint32_t it = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    // 64 threads; the 1024 16-byte chunks of a stage are spread so that each
+    // group of 8 lanes writes the 8 chunks of one row (conflict-free).
+    const int t = threadIdx.x;
+    bool dead = false;
+    uint32_t it = 0, tl = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++tl) {
       const int2 tile = tile_of(a, item / a.n_tiles_n);
       const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
-      const __half* src[2];
-      uint32_t nbytes[2];
+      const __half** tab = atab + (tl & 1) * BM;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int i = 2 * t + j;
         const bool ok = tile.y + i < sg.rows;
         const int64_t m = (int64_t)sg.row_begin + tile.y + i;
-        int64_t arow = 0;
+        const __half* p = nullptr;
         if (ok) {
+          int64_t arow;
           if (sg.a_mode == A_PAIRS) arow = a.sorted_pair[m] / a.topk;
           else if (sg.a_mode == A_TOKENS) arow = tile.y + i;
           else arow = m;
+          p = a.A + arow * a.lda;
         }
-        src[j] = a.A + arow * a.lda;
-        nbytes[j] = ok ? 16u : 0u;
+        tab[i] = p;
       }
+      tc::named_sync(2, 64);
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const uint32_t s = it % S1, ph = (it / S1) & 1u;
-        if (!tc::mbar_wait(&a_empty[s], ph ^ 1u, status)) goto done;
+        // after a wait that ran out both loader warps keep walking the items
+        // (no copies) so they meet at every named barrier
+        if (!dead) dead = !tc::mbar_wait(&a_empty[s], ph ^ 1u, status);
+        if (dead) continue;
         const uint32_t st = sbase + SM::A_OFF + s * A_STAGE;
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            tc::cp_async16(st + tc::sw128_offset(2 * t + j, c), src[j] + kb * BK + c * 8,
-                           nbytes[j]);
+        for (int i = 0; i < 16; ++i) {
+          const int q = t + 64 * i;
+          const int row = q >> 3, c = q & 7;
+          const __half* p = tab[row];
+          tc::cp_async16(st + tc::sw128_offset(row, c), p ? p + kb * BK + c * 8 : a.A,
+                         p ? 16u : 0u);
+        }
         tc::cp_async_arrive_noinc(&full_a[s]);
       }
     }
@@ -362,7 +379,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         ok16[j] = ok ? 16u : 0u;
       }
       for (int kb = 0; kb < KB; ++kb, ++it) {
-        const uint32_t s = it % S1, ph = (it / S1) & 1u;
+        const uint32_t s = it % SR, ph = (it / SR) & 1u;
         if (!tc::mbar_wait(&raw_empty[s], ph ^ 1u, status)) goto done;
         const uint32_t rst = sbase + SM::RAW_OFF + s * RW::STAGE;
         const uint32_t sbst = sbase + SM::SB_OFF + s * SB_STAGE;
@@ -372,8 +389,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           const int r = lane + 32 * j;
 #pragma unroll
           for (int c = 0; c < RW::CHUNKS; ++c)
-            tc::cp_async16(rst + r * RW::ROW + c * 16, wp[j] + kb * (RW::ROW / 4) + c * 4,
-                           ok16[j]);
+            tc::cp_async16(rst + RW::offset(r, c), wp[j] + kb * (RW::ROW / 4) + c * 4, ok16[j]);
           tc::cp_async4(sbst + r * 8, sp[j] + kb2, ok16[j] ? 4u : 0u);
           tc::cp_async4(sbst + r * 8 + 4, bp[j] + kb2, ok16[j] ? 4u : 0u);
         }
@@ -410,7 +426,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
       if (lane == 0) tc::mma_commit(&tmem_full[acc]);
       __syncwarp();
     }
-  } else if (warp < 8) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int i = q * 32 + lane;  // tile row = TMEM lane
@@ -439,8 +455,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
               const float g0 = __uint_as_float(g[2 * k]), g1 = __uint_as_float(g[2 * k + 1]);
-              const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(u[2 * k]);
-              const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(u[2 * k + 1]);
+              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(u[2 * k]);
+              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(u[2 * k + 1]);
               bad |= !(fabsf(h0) <= 65504.0f) || !(fabsf(h1) <= 65504.0f);
               o[k] = h2u(__floats2half2_rn(h0, h1));
             }
@@ -492,44 +508,45 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
       tc::tc_fence_before();
       tc::mbar_arrive(&tmem_empty[acc]);
     }
-  } else {
+  } else if (warp >= 8) {
     // ------------------------------------------------------------ dequantiser
-    const int td = threadIdx.x - 256;  // 0..127
-    constexpr int ITEMS = BN * RW::CHUNKS / 128;  // per thread per stage: 8, 4, 2
+    const int r = threadIdx.x - 256;  // weight row of the tile, 0..255
     uint32_t it = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb, ++it) {
-        const uint32_t s1 = it % S1, ph1 = (it / S1) & 1u;
+        const uint32_t sr = it % SR, phr = (it / SR) & 1u;
         const uint32_t s2 = it % S2, ph2 = (it / S2) & 1u;
-        if (!tc::mbar_wait(&raw_full[s1], ph1, status)) goto done;
+        if (!tc::mbar_wait(&raw_full[sr], phr, status)) goto done;
         if (!tc::mbar_wait(&b_empty[s2], ph2 ^ 1u, status)) goto done;
-        const uint32_t rst = sbase + SM::RAW_OFF + s1 * RW::STAGE;
-        const uint32_t sbst = sbase + SM::SB_OFF + s1 * SB_STAGE;
+        const uint32_t rst = sbase + SM::RAW_OFF + sr * RW::STAGE;
+        const uint32_t sbst = sbase + SM::SB_OFF + sr * SB_STAGE;
         const uint32_t bst = sbase + SM::B_OFF + s2 * B_STAGE;
         const int hi = kb & 1;
+        const uint2 sb = lds64(sbst + r * 8);
+        const uint32_t sbits = hi ? (sb.x >> 16) : (sb.x & 0xFFFFu);
+        const uint32_t bbits = hi ? (sb.y >> 16) : (sb.y & 0xFFFFu);
+        uint4 raw[RW::CHUNKS];
 #pragma unroll
-        for (int k = 0; k < ITEMS; ++k) {
-          const int idx = td + 128 * k;
-          const int r = idx / RW::CHUNKS, c = idx % RW::CHUNKS;
-          const uint4 raw = lds128(rst + r * RW::ROW + c * 16);
-          const uint2 sb = lds64(sbst + r * 8);
-          const uint32_t sbits = hi ? (sb.x >> 16) : (sb.x & 0xFFFFu);
-          const uint32_t bbits = hi ? (sb.y >> 16) : (sb.y & 0xFFFFu);
-          // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
-          if (EPI == EPI_SPLIT) {
-            const float sf = bf16_bits_to_float((uint16_t)sbits);
-            const float bf = bf16_bits_to_float((uint16_t)bbits);
-            if (r < 128) dequant_chunk_split<BITS, false>(raw, sf, bf, bst, r, c * (16 / BITS));
-            else dequant_chunk_split<BITS, true>(raw, sf, bf, bst, r, c * (16 / BITS));
-          } else {
-            __half2 s2h, b2h;
-            group_h2<BITS>(sbits, bbits, s2h, b2h, status);
-            dequant_chunk<BITS>(raw, s2h, b2h, bst, r, c * (16 / BITS));
+        for (int c = 0; c < RW::CHUNKS; ++c) raw[c] = lds128(rst + RW::offset(r, c));
+        tc::mbar_arrive(&raw_empty[sr]);
+        // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
+        if (EPI == EPI_SPLIT) {
+          const float sf = bf16_bits_to_float((uint16_t)sbits);
+          const float bf = bf16_bits_to_float((uint16_t)bbits);
+#pragma unroll
+          for (int c = 0; c < RW::CHUNKS; ++c) {
+            if (r < 128) dequant_chunk_split<BITS, false>(raw[c], sf, bf, bst, r, c * (16 / BITS));
+            else dequant_chunk_split<BITS, true>(raw[c], sf, bf, bst, r, c * (16 / BITS));
           }
+        } else {
+          __half2 s2h, b2h;
+          group_h2<BITS>(sbits, bbits, s2h, b2h, status);
+#pragma unroll
+          for (int c = 0; c < RW::CHUNKS; ++c)
+            dequant_chunk<BITS>(raw[c], s2h, b2h, bst, r, c * (16 / BITS));
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(&b_full[s2]);
-        tc::mbar_arrive(&raw_empty[s1]);
       }
     }
   }

@@ -3,185 +3,444 @@
 #include "gemv.cuh"
 #include "kernels.h"
 #include "route.cuh"
+#include "tc.cuh"
 
 namespace moeq {
 
-GemvShape gemv_shape(int slices, int R) {
-  GemvShape s;
-  s.R = R;
-  s.rbs = slices >= 8 ? 1 : 8 / slices;
-  s.warps = slices * s.rbs;
-  return s;
+GemvShape gemv_shape(int in_dim, int bits, int nmat, int G) {
+  GemvShape sh;
+  const int cpr = in_dim / (128 / bits);
+  sh.S = (cpr + 31) / 32;
+  sh.J = sh.S >= 8 ? 1 : 8 / sh.S;
+  // fewer row subsets when a unit would not fit one stage
+  const int64_t row = (int64_t)in_dim * bits / 8 + 4 * (in_dim / G);
+  while (sh.J > 1 && (int64_t)nmat * sh.J * (8 / nmat) * row > 44 * 1024) sh.J >>= 1;
+  sh.RU = sh.J * (8 / nmat);
+  return sh;
 }
 
-// ============================================================== GEMV kernel
-__device__ __forceinline__ int find_seg(const Seg* segs, int n, int unit) {
-  int lo = 0, hi = n - 1;  // last seg with unit_begin <= unit
+bool gemv_fits(int in_dim, int bits, int nmat, int G) {
+  const GemvShape sh = gemv_shape(in_dim, bits, nmat, G);
+  const int64_t row = (int64_t)in_dim * bits / 8 + 4 * (in_dim / G);
+  return sh.S <= 8 && (int64_t)nmat * sh.RU * row <= 44 * 1024;
+}
+
+int gemv_units(int out_dim, const GemvShape& sh) { return (out_dim + sh.RU - 1) / sh.RU; }
+
+// ============================================================== staged GEMV kernel
+// Persistent CTAs (one per SM).  Warp 8 is the producer: it reads the work
+// description of up to 32 of its CTA's units at once (one unit per lane),
+// then per unit (RU consecutive rows of NMAT matrices of one segment) lane
+// 0 issues bulk copies of the contiguous packed rows into a 4-stage
+// shared-memory ring, and all lanes copy the rows' bf16 scale/bias pairs
+// and the unit's input/output vector references with cp.async.  Warp 9
+// issues the L2 prefetches.  Warps 0..S*J-1 consume: warp (slice s, subset
+// j) keeps its 32-chunk slice of the input vector in registers as
+// fixed-point limbs, takes RU/J rows of each matrix from the stage (one
+// 16-byte chunk per lane per row), reduces the eight row partials of each
+// lane with the transposing butterfly, and the S slices are summed in fixed
+// order through a double-buffered shared-memory exchange guarded by
+// mbarriers (every wait bounded).
+constexpr int GV_CW = 8;                  // consumer warps
+constexpr int GV_PRODUCER = GV_CW;        // producer warp
+constexpr int GV_HELPER = GV_CW + 1;      // L2-prefetch warp
+constexpr int GV_THREADS = (GV_CW + 2) * 32;
+constexpr int GV_STAGES = 4;
+constexpr int GV_STAGE_BYTES = 44 * 1024;
+constexpr int GV_VMAX = 64;               // vector references staged per unit
+constexpr int GV_UB_CAP = 2064;           // segment start units cached in shared memory
+
+// What the consumers need to know about the unit in a stage.
+struct GvMeta {
+  int32_t r0, nrows, n_vec, vec_mode;
+  const void* src_base;
+  int64_t src_stride;
+  float* dst_base;
+  int64_t dst_stride;
+  const VecRef* vecs;
+};
+
+struct GvSmem {
+  static constexpr int META_STRIDE = 64;
+  static constexpr int STAGE_OFF = 0;
+  static constexpr int META_OFF = GV_STAGES * GV_STAGE_BYTES;
+  static constexpr int VEC_OFF = META_OFF + GV_STAGES * META_STRIDE;
+  static constexpr int UB_OFF = VEC_OFF + GV_STAGES * GV_VMAX * 16;
+  static constexpr int BAR_OFF = UB_OFF + GV_UB_CAP * 4;
+  static constexpr int N_BARS = 2 * GV_STAGES + 4;
+  static constexpr int RED_OFF = BAR_OFF + N_BARS * 8;
+  static constexpr int BYTES = RED_OFF + 2 * GV_CW * 8 * 4;
+};
+static_assert(sizeof(GvMeta) <= GvSmem::META_STRIDE, "GvMeta exceeds its slot");
+static_assert(sizeof(VecRef) == 16, "VecRef is copied in 16-byte pieces");
+
+// Last segment whose first unit is <= unit; p[i * stride] is segment i's
+// first unit.
+__device__ __forceinline__ int find_seg(const int32_t* p, int stride, int n, int unit) {
+  int lo = 0, hi = n - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (segs[mid].unit_begin <= unit) lo = mid; else hi = mid - 1;
+    if (p[(int64_t)mid * stride] <= unit) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
-template <int BITS, int NL, int NMAT, int R, int SRC, int EPI>
-__global__ void __launch_bounds__(256) k_gemv(const __grid_constant__ GemvArgs a) {
+// The prefetch ranges into L2 in 32 KB pieces; piece g of the concatenated
+// ranges is issued by CTA g % gridDim.x (lane (g / gridDim.x) % 32 of the
+// calling warp), so every SM's copy engine takes a share.
+__device__ __forceinline__ void prefetch_ranges(const PrefetchRange* pf, int n) {
+  constexpr int64_t PIECE = 32 * 1024;
+  const int lane = threadIdx.x & 31;
+  int64_t g0 = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t pieces = (pf[i].bytes + PIECE - 1) / PIECE;
+    int64_t g = g0 + ((blockIdx.x - g0 % gridDim.x) + gridDim.x) % gridDim.x;
+    for (int64_t j = 0; g < g0 + pieces; g += gridDim.x, ++j) {
+      if ((int)(j % 32) != lane) continue;
+      const int64_t off = (g - g0) * PIECE;
+      const int64_t len = min(PIECE, pf[i].bytes - off) & ~(int64_t)15;
+      if (len > 0) tc::prefetch_l2((const uint8_t*)pf[i].p + off, (uint32_t)len);
+    }
+    g0 += pieces;
+  }
+}
+
+// Matrix 0 (codes, scales, biases) of every listed segment into L2, spread
+// over the CTAs the same way.
+__device__ __forceinline__ void prefetch_segs(const Seg* segs, int n) {
+  constexpr int64_t PIECE = 32 * 1024;
+  const int lane = threadIdx.x & 31;
+  int64_t g0 = 0;
+  for (int i = 0; i < n; ++i) {
+    const Seg& sg = segs[i];
+    const int64_t gr = (int64_t)sg.out_dim * (sg.in_dim / sg.G);
+    const void* p[3] = {sg.w[0], sg.s[0], sg.b[0]};
+    const int64_t bytes[3] = {(int64_t)sg.out_dim * sg.in_dim * sg.bits / 8, gr * 2, gr * 2};
+    for (int k = 0; k < 3; ++k) {
+      const int64_t pieces = (bytes[k] + PIECE - 1) / PIECE;
+      // first global index >= g0 owned by this CTA, then every gridDim.x
+      int64_t g = g0 + ((blockIdx.x - g0 % gridDim.x) + gridDim.x) % gridDim.x;
+      for (int64_t j = 0; g < g0 + pieces; g += gridDim.x, ++j) {
+        if ((int)(j % 32) != lane) continue;
+        const int64_t off = (g - g0) * PIECE;
+        const int64_t len = min(PIECE, bytes[k] - off) & ~(int64_t)15;
+        if (len > 0 && ((uintptr_t)p[k] & 15) == 0)
+          tc::prefetch_l2((const uint8_t*)p[k] + off, (uint32_t)len);
+      }
+      g0 += pieces;
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ T shfl_ptr(T p, int src) {
+  return reinterpret_cast<T>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(p), src));
+}
+
+template <int BITS, int NL, int NMAT, int SRC, int EPI>
+__global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ GemvArgs a) {
   constexpr int VPC = Chunk<BITS>::VPC;
   constexpr int NC = Chunk<BITS>::NC;
   constexpr int NB = SliceVec<BITS, NL>::NB;
-  constexpr int RB = 4;  // rows per load batch
+  constexpr int RPW = 8 / NMAT;  // rows per warp per matrix and unit
   using SrcT = typename std::conditional<SRC == SRC_BF16, SrcBF16, SrcF32>::type;
-  __shared__ float part[8][NMAT][R];
+  extern __shared__ __align__(128) uint8_t gsm[];
+  VecRef* svec = reinterpret_cast<VecRef*>(gsm + GvSmem::VEC_OFF);
+  int32_t* ub = reinterpret_cast<int32_t*>(gsm + GvSmem::UB_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(gsm + GvSmem::BAR_OFF);
+  uint64_t* empty = full + GV_STAGES;
+  uint64_t* red_full = empty + GV_STAGES;  // 2: slices 1..S-1 -> slice 0
+  uint64_t* red_empty = red_full + 2;      // 2: slice 0 -> slices 1..S-1
+  float* red = reinterpret_cast<float*>(gsm + GvSmem::RED_OFF);  // [2][GV_CW][8]
+  const uint32_t sbase = tc::smem_u32(gsm);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = a.slices;
-  const int rbs = (blockDim.x >> 5) / S;
-  const int slice = warp % S, rbl = warp / S;
+  const int S = a.slices, J = a.subsets, RU = a.rows_per_unit;
+  const int W = S * J;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < GV_STAGES; ++i) {
+      tc::mbar_init(&full[i], 1 + 32);
+      tc::mbar_init(&empty[i], GV_CW * 32);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&red_full[i], (uint32_t)((S > 1 ? S - 1 : 1) * J * 8));
+      tc::mbar_init(&red_empty[i], (uint32_t)(J * 8));
+    }
+    tc::fence_mbar_init();
+  }
+  // ranges known before the preceding kernel ends (the shared expert's
+  // weights) go to L2 while it finishes
+  if (warp == GV_HELPER && a.n_pf) prefetch_ranges(a.pf, a.n_pf);
+  __syncthreads();
+  // segment lists and input vectors may come from the preceding kernel
+  tc::grid_dep_wait();
+  tc::grid_dep_launch();
 
   const Seg* segs = a.dyn_segs ? a.dyn_segs : a.segs;
   const int n_segs = a.dyn_segs ? a.dyn_count[0] : a.n_segs;
   const int total_units = a.dyn_segs ? a.dyn_count[1] : a.total_units;
+  const bool ub_cached = n_segs <= GV_UB_CAP;
+  if (ub_cached)
+    for (int i = threadIdx.x; i < n_segs; i += blockDim.x) ub[i] = segs[i].unit_begin;
+  __syncthreads();
 
-  for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x) {
-    const Seg& sg = segs[find_seg(segs, n_segs, unit)];
-    const int lu = unit - sg.unit_begin;
-    const int out_dim = sg.out_dim;
-    const int row0 = (lu * rbs + rbl) * R;
-    const int cpr = sg.in_dim / VPC;
-    const int ch = slice * 32 + lane;
-    const bool lane_on = ch < cpr;
-    const int64_t wpr = (int64_t)sg.in_dim * BITS / 32;
-    const int gpr = sg.in_dim / sg.G;
+  const int row_bytes = a.in_dim * BITS / 8;
+  const int gpr = a.in_dim / a.G;
+  const int cpr = a.in_dim / VPC;
+  // stage layout: codes [NMAT][RU][row_bytes], scales [NMAT][RU*gpr], biases [NMAT][RU*gpr]
+  const int codes_bytes = NMAT * RU * row_bytes;
+  const int sb_bytes = RU * gpr * 2;
+  int* status = a.status;
+
+  if (warp == GV_HELPER) {
+    // ------------------------------------------------------------ L2 prefetch
+    if (a.pf_segs) prefetch_segs(a.pf_segs, a.pf_count[0]);
+  } else if (warp == GV_PRODUCER) {
+    // ------------------------------------------------------------ producer
+    uint32_t it = 0;
+    bool dead = false;
+    for (int base = blockIdx.x; base < total_units && !dead; base += 32 * gridDim.x) {
+      // lane u describes unit base + u * gridDim.x
+      const int mine = base + lane * gridDim.x;
+      int r0 = 0, nrows = 0, n_vec = 0, vec_mode = 0;
+      const uint32_t* w[2] = {nullptr, nullptr};
+      const uint16_t* sp[2] = {nullptr, nullptr};
+      const uint16_t* bp[2] = {nullptr, nullptr};
+      const void* src_base = nullptr;
+      float* dst_base = nullptr;
+      int64_t src_stride = 0, dst_stride = 0;
+      const VecRef* vecs = nullptr;
+      if (mine < total_units) {
+        const int si = ub_cached ? find_seg(ub, 1, n_segs, mine)
+                                 : find_seg(&segs[0].unit_begin, (int)(sizeof(Seg) / 4), n_segs,
+                                            mine);
+        const Seg& sg = segs[si];
+        const int u0 = ub_cached ? ub[si] : sg.unit_begin;
+        r0 = (mine - u0) * RU;
+        nrows = min(RU, sg.out_dim - r0);
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          w[m] = sg.w[m];
+          sp[m] = sg.s[m];
+          bp[m] = sg.b[m];
+        }
+        n_vec = sg.n_vec;
+        vec_mode = sg.vec_mode;
+        src_base = sg.src_base;
+        src_stride = sg.src_stride;
+        dst_base = sg.dst_base;
+        dst_stride = sg.dst_stride;
+        vecs = sg.vecs;
+      }
+      const int nb = min(32, (total_units - base + (int)gridDim.x - 1) / (int)gridDim.x);
+      for (int u = 0; u < nb; ++u, ++it) {
+        const uint32_t s = it % GV_STAGES, ph = (it / GV_STAGES) & 1u;
+        if (!tc::mbar_wait(&empty[s], ph ^ 1u, status)) {
+          dead = true;
+          break;
+        }
+        const int ur0 = __shfl_sync(0xffffffffu, r0, u);
+        const int unr = __shfl_sync(0xffffffffu, nrows, u);
+        const int unv = __shfl_sync(0xffffffffu, n_vec, u);
+        const int uvm = __shfl_sync(0xffffffffu, vec_mode, u);
+        const VecRef* uvecs = shfl_ptr(vecs, u);
+        const uint32_t st = sbase + s * GV_STAGE_BYTES;
+        const uint32_t* uw[2];
+        const uint16_t* usp[2];
+        const uint16_t* ubp[2];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          uw[m] = shfl_ptr(w[m], u);
+          usp[m] = shfl_ptr(sp[m], u);
+          ubp[m] = shfl_ptr(bp[m], u);
+        }
+        const void* usrc = shfl_ptr(src_base, u);
+        float* udst = shfl_ptr(dst_base, u);
+        const int64_t uss = __shfl_sync(0xffffffffu, src_stride, u);
+        const int64_t uds = __shfl_sync(0xffffffffu, dst_stride, u);
+        if (lane == 0) {
+          GvMeta* mt = reinterpret_cast<GvMeta*>(gsm + GvSmem::META_OFF + s * GvSmem::META_STRIDE);
+          mt->r0 = ur0;
+          mt->nrows = unr;
+          mt->n_vec = unv;
+          mt->vec_mode = uvm;
+          mt->src_base = usrc;
+          mt->src_stride = uss;
+          mt->dst_base = udst;
+          mt->dst_stride = uds;
+          mt->vecs = uvecs;
+          tc::mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * unr * row_bytes));
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m)
+            tc::bulk_g2s(st + m * RU * row_bytes,
+                         reinterpret_cast<const uint8_t*>(uw[m]) + (int64_t)ur0 * row_bytes,
+                         (uint32_t)(unr * row_bytes), &full[s]);
+        }
+        const int pairs = unr * gpr / 2;
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          const uint16_t* s0 = usp[m] + (int64_t)ur0 * gpr;
+          const uint16_t* b0 = ubp[m] + (int64_t)ur0 * gpr;
+          const uint32_t sd = st + codes_bytes + m * sb_bytes;
+          const uint32_t bd = st + codes_bytes + NMAT * sb_bytes + m * sb_bytes;
+          for (int p = lane; p < pairs; p += 32) {
+            tc::cp_async4(sd + 4 * p, s0 + 2 * p, 4);
+            tc::cp_async4(bd + 4 * p, b0 + 2 * p, 4);
+          }
+        }
+        if (uvm == 1 && unv <= GV_VMAX) {
+          const uint32_t vd = sbase + GvSmem::VEC_OFF + s * GV_VMAX * 16;
+          for (int v = lane; v < unv; v += 32) tc::cp_async16(vd + 16 * v, uvecs + v, 16);
+        }
+        tc::cp_async_arrive_noinc(&full[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const bool on_w = warp < W;
+    const int sl = warp % S, j = warp / S;
+    const int ch = sl * 32 + lane;
+    const bool lane_on = on_w && ch < cpr;
     int gi[2];
 #pragma unroll
-    for (int pb = 0; pb < 2; ++pb) gi[pb] = (ch * VPC + (pb < NB ? pb : 0) * kXBlock) / sg.G;
-    const uint32_t* wbase[NMAT];
-    const uint16_t* sbase[NMAT];
-    const uint16_t* bbase[NMAT];
+    for (int pb = 0; pb < 2; ++pb) gi[pb] = (ch * VPC + (pb < NB ? pb : 0) * kXBlock) / a.G;
+    SliceVec<BITS, NL> sv;
+    const void* cur_src = nullptr;
+    // After a wait that ran out, every later wait is skipped and no vector
+    // is processed; all waits are bounded, so the CTA always ends.
+    bool timed_out = false;
+    uint32_t it = 0, rc = 0;
+    for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x, ++it) {
+      const uint32_t s = it % GV_STAGES, ph = (it / GV_STAGES) & 1u;
+      if (!timed_out) timed_out = !tc::mbar_wait(&full[s], ph, status);
+      const GvMeta* mp = reinterpret_cast<const GvMeta*>(gsm + GvSmem::META_OFF +
+                                                         s * GvSmem::META_STRIDE);
+      const int n_vec = timed_out ? 0 : mp->n_vec;
+      const uint32_t st = sbase + s * GV_STAGE_BYTES;
+      if (on_w && n_vec > 0) {
+        const int r0 = mp->r0, nrows = mp->nrows, vec_mode = mp->vec_mode;
+        const VecRef* vl = (vec_mode == 1 && n_vec <= GV_VMAX) ? svec + s * GV_VMAX : mp->vecs;
+        for (int v = 0; v < n_vec && !timed_out; ++v) {
+          const void* src;
+          float* dst;
+          if (vec_mode == 0) {
+            src = (SRC == SRC_BF16)
+                      ? (const void*)((const uint16_t*)mp->src_base + (int64_t)v * mp->src_stride)
+                      : (const void*)((const float*)mp->src_base + (int64_t)v * mp->src_stride);
+            dst = mp->dst_base + (int64_t)v * mp->dst_stride;
+          } else {
+            src = vl[v].src;
+            dst = vl[v].dst;
+          }
+          if (src != cur_src) {
+            build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
+            cur_src = src;
+          }
+          float acc[8];
 #pragma unroll
-    for (int m = 0; m < NMAT; ++m) {
-      wbase[m] = sg.w[m];
-      sbase[m] = sg.s[m];
-      bbase[m] = sg.b[m];
-    }
-
-    for (int v = 0; v < sg.n_vec; ++v) {
-      const void* src;
-      float* dst;
-      if (sg.vec_mode == 0) {
-        src = (SRC == SRC_BF16)
-                  ? (const void*)((const uint16_t*)sg.src_base + (int64_t)v * sg.src_stride)
-                  : (const void*)((const float*)sg.src_base + (int64_t)v * sg.src_stride);
-        dst = sg.dst_base + (int64_t)v * sg.dst_stride;
-      } else {
-        src = sg.vecs[v].src;
-        dst = sg.vecs[v].dst;
-      }
-      SliceVec<BITS, NL> sv;
-      build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
-
-      float acc[NMAT][R];
+          for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-      for (int rr = 0; rr < R; rr += RB) {
-        uint4 wv[NMAT][RB];
-        float sf[NMAT][RB][2], bf[NMAT][RB][2];
+            for (int i = 0; i < RPW; ++i) {
+              const int row = j * RPW + i;
+              const bool ok = lane_on && row < nrows;
+              uint4 wv = make_uint4(0, 0, 0, 0);
+              float s2[2] = {0.f, 0.f}, b2[2] = {0.f, 0.f};
+              if (ok) {
+                wv = gq_lds128(st + (m * RU + row) * row_bytes + ch * 16);
+                const uint32_t sd = st + codes_bytes + m * sb_bytes + row * gpr * 2;
+                const uint32_t bd = st + codes_bytes + (NMAT + m) * sb_bytes + row * gpr * 2;
 #pragma unroll
-        for (int i = 0; i < RB; ++i) {
-          const int r = row0 + rr + i;
-          const bool on = lane_on && r < out_dim;
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            if (on) {
-              wv[m][i] = ldg_stream16(wbase[m] + (int64_t)r * wpr + (int64_t)ch * 4);
-#pragma unroll
-              for (int pb = 0; pb < NB; ++pb) {
-                sf[m][i][pb] = bf16_bits_to_float(ldg_u16(sbase[m] + (int64_t)r * gpr + gi[pb]));
-                bf[m][i][pb] = bf16_bits_to_float(ldg_u16(bbase[m] + (int64_t)r * gpr + gi[pb]));
+                for (int pb = 0; pb < NB; ++pb) {
+                  s2[pb] = bf16_bits_to_float(lds_u16(sd + gi[pb] * 2));
+                  b2[pb] = bf16_bits_to_float(lds_u16(bd + gi[pb] * 2));
+                }
+              }
+              uint32_t c[NC];
+              Chunk<BITS>::split(wv, c);
+              acc[m * RPW + i] = chunk_contrib<BITS, NL>(c, sv, s2, b2);
+            }
+          float tot = transpose_reduce<8>(acc);  // lane l: value l % 8
+          if (S > 1) {
+            // slices 1..S-1 hand their partials to slice 0, which adds them
+            // in slice order
+            const uint32_t buf = rc & 1u, rph = (rc >> 1) & 1u;
+            ++rc;
+            float* rb = red + buf * GV_CW * 8;
+            if (sl != 0) {
+              if (!tc::mbar_wait(&red_empty[buf], rph ^ 1u, status)) timed_out = true;
+              if (lane < 8) {
+                rb[warp * 8 + lane] = tot;
+                tc::mbar_arrive(&red_full[buf]);
               }
             } else {
-              wv[m][i] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-              for (int pb = 0; pb < NB; ++pb) sf[m][i][pb] = bf[m][i][pb] = 0.0f;
+              if (!tc::mbar_wait(&red_full[buf], rph, status)) timed_out = true;
+              if (lane < 8) {
+                float t = tot;
+                for (int q = 1; q < S; ++q) t += rb[(j * S + q) * 8 + lane];
+                tot = t;
+                tc::mbar_arrive(&red_empty[buf]);
+              }
             }
-            if (NB == 1) sf[m][i][1] = bf[m][i][1] = 0.0f;
           }
-        }
-#pragma unroll
-        for (int i = 0; i < RB; ++i)
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            uint32_t c[NC];
-            Chunk<BITS>::split(wv[m][i], c);
-            const float s2[2] = {sf[m][i][0], sf[m][i][1]};
-            const float b2[2] = {bf[m][i][0], bf[m][i][1]};
-            acc[m][rr + i] = chunk_contrib<BITS, NL>(c, sv, s2, b2);
-          }
-      }
-      float tot[NMAT];
-#pragma unroll
-      for (int m = 0; m < NMAT; ++m) tot[m] = transpose_reduce<R>(acc[m]);
-      // lane l now holds row (l % R) of this warp's slice
-      bool writer = (lane < R);
-      if (S > 1) {
-        if (lane < R)
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) part[warp][m][lane] = tot[m];
-        __syncthreads();
-        writer = writer && slice == 0;
-        if (writer) {
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            float t = 0.0f;
-            for (int sl = 0; sl < S; ++sl) t += part[rbl * S + sl][m][lane];
-            tot[m] = t;
-          }
-        }
-      }
-      if (writer) {
-        const int r = row0 + lane;
-        if (r < out_dim) {
-          float o;
           if (EPI == EPI_SWIGLU) {
-            const float g = tot[0];
-            o = g / (1.0f + expf(-g)) * tot[NMAT - 1];
+            // values 0..3: gate rows, 4..7: up rows of the same four rows
+            const float u = __shfl_sync(0xffffffffu, tot, (lane + RPW) & 31);
+            const int row = j * RPW + lane;
+            if (sl == 0 && lane < RPW && row < nrows)
+              dst[r0 + row] = __fdividef(tot, 1.0f + __expf(-tot)) * u;
           } else {
-            o = tot[0];
+            const int row = j * RPW + lane;
+            if (sl == 0 && lane < 8 && row < nrows) dst[r0 + row] = tot;
           }
-          dst[r] = o;
         }
       }
-      if (S > 1) __syncthreads();
+      tc::mbar_arrive(&empty[s]);
     }
   }
 }
 
-template <int BITS, int NL, int NMAT, int R, int SRC, int EPI>
-static cudaError_t launch_one(const GemvArgs& a, int grid, int warps, cudaStream_t st) {
-  k_gemv<BITS, NL, NMAT, R, SRC, EPI><<<grid, warps * 32, 0, st>>>(a);
-  return cudaGetLastError();
+template <int BITS, int NL, int NMAT, int SRC, int EPI>
+static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
+  auto kern = k_gemv<BITS, NL, NMAT, SRC, EPI>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GvSmem::BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(GV_THREADS);
+  cfg.dynamicSmemBytes = GvSmem::BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-cudaError_t launch_gemv(int bits, int nl, int nmat, int R, int src, const GemvArgs& a, int grid,
+cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,
                         cudaStream_t st) {
-  const GemvShape sh = gemv_shape(a.slices, R);
   if (grid <= 0) return cudaSuccess;
-  if (R != 8) return cudaErrorInvalidValue;
   // instantiated forms: router / qmv (3 limbs, bf16 tokens), gate/up + SwiGLU
   // (2 limbs, bf16 tokens), down (2 limbs, fp32 hidden rows)
   if (nmat == 2 && nl == 2 && src == SRC_BF16) {
-    if (bits == 8) return launch_one<8, 2, 2, 8, SRC_BF16, EPI_SWIGLU>(a, grid, sh.warps, st);
-    if (bits == 4) return launch_one<4, 2, 2, 8, SRC_BF16, EPI_SWIGLU>(a, grid, sh.warps, st);
-    return launch_one<2, 2, 2, 8, SRC_BF16, EPI_SWIGLU>(a, grid, sh.warps, st);
+    if (bits == 8) return launch_one<8, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st);
+    if (bits == 4) return launch_one<4, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st);
+    return launch_one<2, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st);
   }
   if (nmat == 1 && nl == 3 && src == SRC_BF16) {
-    if (bits == 8) return launch_one<8, 3, 1, 8, SRC_BF16, EPI_PLAIN>(a, grid, sh.warps, st);
-    if (bits == 4) return launch_one<4, 3, 1, 8, SRC_BF16, EPI_PLAIN>(a, grid, sh.warps, st);
-    return launch_one<2, 3, 1, 8, SRC_BF16, EPI_PLAIN>(a, grid, sh.warps, st);
+    if (bits == 8) return launch_one<8, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st);
+    if (bits == 4) return launch_one<4, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st);
+    return launch_one<2, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st);
   }
   if (nmat == 1 && nl == 2 && src == SRC_F32) {
-    if (bits == 8) return launch_one<8, 2, 1, 8, SRC_F32, EPI_PLAIN>(a, grid, sh.warps, st);
-    if (bits == 4) return launch_one<4, 2, 1, 8, SRC_F32, EPI_PLAIN>(a, grid, sh.warps, st);
-    return launch_one<2, 2, 1, 8, SRC_F32, EPI_PLAIN>(a, grid, sh.warps, st);
+    if (bits == 8) return launch_one<8, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st);
+    if (bits == 4) return launch_one<4, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st);
+    return launch_one<2, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -212,6 +471,21 @@ cudaError_t launch_route_topk(const float* logits, int M, int E, int K, int reno
 }
 
 // ============================================================== decode plan
+// Routing warps of the plan kernel: one token each at a time, E floats of
+// staged logits per warp, at most 64 KB of staging.
+__host__ __device__ __forceinline__ int plan_route_warps(int M, int E, int nwarps) {
+  int r = (64 * 1024) / (E * 4);
+  if (r < 1) r = 1;
+  if (r > nwarps) r = nwarps;
+  if (r > M) r = M;
+  return r;
+}
+
+// Shared-memory region after the plan's per-warp bitmaps: n ints.
+__device__ __forceinline__ int32_t* taken_list(uint32_t* sm, int n, int E, int nwarps) {
+  return reinterpret_cast<int32_t*>(sm) + 4 * n + nwarps * ((E + 31) >> 5);
+}
+
 // One CTA (1024 threads).  Routes the M tokens (unless the routing is given),
 // computes the shared-expert gate, sorts the M*K (token, slot) pairs by
 // expert (stable) and writes one gate/up segment and one down segment per
@@ -227,12 +501,17 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
   int32_t* entry_of = head + n;                       // [n] entry index of sorted position
   uint32_t* taken = reinterpret_cast<uint32_t*>(entry_of + n);  // [nwarps][words]
 
-  // 1. routing
+  // 1. routing: R warps, each with its token's logits staged in shared memory
   if (a.logits) {
-    for (int t = warp; t < M; t += nwarps)
-      route_token_warp(a.logits + (int64_t)t * a.E, a.E, K, a.renorm, a.router_scale,
-                       a.idx_out + (int64_t)t * K, a.w_out + (int64_t)t * K,
-                       taken + warp * words);
+    const int R = plan_route_warps(M, a.E, nwarps);
+    float* rows = reinterpret_cast<float*>(taken + nwarps * words);  // [R][E]
+    if (warp < R)
+      for (int t = warp; t < M; t += R) {
+        float* row = rows + (int64_t)warp * a.E;
+        stage_logits_warp(a.logits + (int64_t)t * a.E, row, a.E);
+        route_token_warp(row, a.E, K, a.renorm, a.router_scale, a.idx_out + (int64_t)t * K,
+                         a.w_out + (int64_t)t * K, taken + warp * words);
+      }
   } else {
     for (int p = tid; p < n; p += blockDim.x) {
       a.idx_out[p] = a.idx_in[p];
@@ -285,6 +564,46 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
   __syncthreads();
   const int n_entries = n > 0 ? entry_of[n - 1] + 1 : 0;
 
+  // the selected experts' weights are known now: start pulling them into L2
+  // so the gate/up and down GEMVs read them from there
+  if (a.prefetch) {
+    int32_t* ent = taken_list(sm, n, a.E, nwarps);
+    for (int i = tid; i < n; i += blockDim.x)
+      if (head[i]) ent[entry_of[i]] = key[sorted[i]];
+    __syncthreads();
+    const moeq_qtensor* ts[3] = {&a.gate, &a.up, &a.down};
+    constexpr int64_t PIECE = 32 * 1024;
+    // per expert: 3 tensors x (codes, scales, biases)
+    int64_t sizes[9];
+    for (int k = 0; k < 3; ++k) {
+      const moeq_qtensor& t = *ts[k];
+      const int64_t groups = (int64_t)t.out_dim * (t.in_dim / t.group_size);
+      sizes[3 * k] = (int64_t)t.out_dim * t.in_dim * t.bits / 8;
+      sizes[3 * k + 1] = groups * 2;
+      sizes[3 * k + 2] = groups * 2;
+    }
+    int64_t per_expert = 0;
+    for (int k = 0; k < 9; ++k) per_expert += (sizes[k] + PIECE - 1) / PIECE;
+    for (int64_t q = tid; q < (int64_t)n_entries * per_expert; q += blockDim.x) {
+      const int u = (int)(q / per_expert);
+      int64_t r = q % per_expert;
+      int k = 0;
+      while (r >= (sizes[k] + PIECE - 1) / PIECE) {
+        r -= (sizes[k] + PIECE - 1) / PIECE;
+        ++k;
+      }
+      const moeq_qtensor& t = *ts[k / 3];
+      const int e = ent[u];
+      const uint8_t* base =
+          (k % 3 == 0) ? (const uint8_t*)(t.w + (int64_t)e * t.expert_stride_w)
+          : (k % 3 == 1) ? (const uint8_t*)(t.scales + (int64_t)e * t.expert_stride_sb)
+                         : (const uint8_t*)(t.biases + (int64_t)e * t.expert_stride_sb);
+      const int64_t off = r * PIECE;
+      const int64_t len = min(PIECE, sizes[k] - off) & ~(int64_t)15;
+      if (((uintptr_t)base & 15) == 0 && len > 0) tc::prefetch_l2(base + off, (uint32_t)len);
+    }
+  }
+
   // 3. vector lists and segments, one per distinct expert
   for (int i = tid; i < n; i += blockDim.x) {
     const int p = sorted[i];
@@ -308,6 +627,7 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
       g.out_dim = a.I;
       g.in_dim = a.H;
       g.G = a.gate.group_size;
+      g.bits = a.gate.bits;
       g.n_vec = cnt;
       g.unit_begin = u * a.units_per_seg_gu;
       g.vec_mode = 1;
@@ -324,6 +644,7 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
       dn.out_dim = a.H;
       dn.in_dim = a.I;
       dn.G = a.down.group_size;
+      dn.bits = a.down.bits;
       dn.n_vec = cnt;
       dn.unit_begin = u * a.units_per_seg_dn;
       dn.vec_mode = 1;
@@ -351,6 +672,7 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
       g.out_dim = a.sh_gate.out_dim;
       g.in_dim = a.H;
       g.G = a.sh_gate.group_size;
+      g.bits = a.sh_gate.bits;
       g.n_vec = M;
       g.vec_mode = 0;
       g.src_base = a.x;
@@ -365,6 +687,7 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
       dn.out_dim = a.H;
       dn.in_dim = a.sh_down.in_dim;
       dn.G = a.sh_down.group_size;
+      dn.bits = a.sh_down.bits;
       dn.n_vec = M;
       dn.vec_mode = 0;
       dn.src_base = a.h + (int64_t)n * a.I;
@@ -410,7 +733,8 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
 cudaError_t launch_decode_plan(const DecodePlanArgs& a, cudaStream_t st) {
   const int n = a.M * a.K;
   const int threads = 1024;
-  const size_t smem = (size_t)n * 4 * 4 + (size_t)(threads / 32) * ((a.E + 31) / 32) * 4;
+  size_t smem = (size_t)n * 4 * 5 + (size_t)(threads / 32) * ((a.E + 31) / 32) * 4;
+  if (a.logits) smem += (size_t)plan_route_warps(a.M, a.E, threads / 32) * a.E * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_decode_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);

@@ -29,6 +29,7 @@ struct Seg {
   int32_t out_dim;
   int32_t in_dim;
   int32_t G;
+  int32_t bits;
   int32_t n_vec;
   int32_t unit_begin;  // first work unit of this segment
   int32_t vec_mode;    // 0 strided, 1 list
@@ -40,6 +41,13 @@ struct Seg {
 };
 
 constexpr int kInlineSegs = 4;
+constexpr int kMaxPrefetch = 10;
+
+// A global range to pull into L2 at kernel start (16-byte aligned).
+struct PrefetchRange {
+  const void* p;
+  int64_t bytes;
+};
 
 struct GemvArgs {
   Seg segs[kInlineSegs];    // used when dyn_segs == nullptr
@@ -47,22 +55,37 @@ struct GemvArgs {
   int32_t total_units;      // used when dyn_segs == nullptr
   const Seg* dyn_segs;      // device list written by the decode plan
   const int32_t* dyn_count; // [0] = number of segments, [1] = total units
+  // shape shared by every segment of the launch
+  int32_t in_dim;
+  int32_t G;
   int32_t slices;           // S: 32-chunk slices per row
+  int32_t subsets;          // J: row subsets (warps = S * J)
+  int32_t rows_per_unit;    // RU = J * (8 / NMAT)
+  PrefetchRange pf[kMaxPrefetch];
+  int32_t n_pf;
+  // segments (device list) whose matrix 0 is pulled into L2 at kernel start,
+  // spread over all CTAs (the down projections, from the gate/up launch)
+  const Seg* pf_segs;
+  const int32_t* pf_count;
   int* status;
 };
 
 enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
 enum GemvSrc { SRC_BF16 = 0, SRC_F32 = 1 };
 
-// Rows per warp-task and row blocks per CTA for a given slice count.
+// Work shape of the staged GEMV for rows of `in_dim` codes at `bits`.
 struct GemvShape {
-  int R;        // rows per row block (8, 16 or 32)
-  int warps;    // warps per CTA
-  int rbs;      // row blocks per CTA iteration
+  int S;   // slices of 32 chunks per row
+  int J;   // row subsets
+  int RU;  // rows per unit
 };
-GemvShape gemv_shape(int slices, int R);
+GemvShape gemv_shape(int in_dim, int bits, int nmat, int G);
+bool gemv_fits(int in_dim, int bits, int nmat, int G);
+int gemv_units(int out_dim, const GemvShape& sh);
 
-cudaError_t launch_gemv(int bits, int nl, int nmat, int R, int src, const GemvArgs& a, int grid,
+// Launch with programmatic dependent launch (the kernel waits for its
+// predecessor's results before reading them).
+cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,
                         cudaStream_t st);
 
 // ------------------------------------------------------------------ routing
@@ -98,6 +121,7 @@ struct DecodePlanArgs {
   int32_t units_per_seg_dn;
   int32_t units_per_seg_gu_sh;
   int32_t units_per_seg_dn_sh;
+  int32_t prefetch;         // 1: pull the selected experts' weights into L2
   int32_t shared_same_gu;   // 1: the shared gate/up segment joins the routed launch
   int32_t shared_same_dn;   // 1: the shared down segment joins the routed launch
   int* status;

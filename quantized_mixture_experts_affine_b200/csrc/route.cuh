@@ -62,4 +62,29 @@ __device__ __forceinline__ void route_token_warp(const float* lg, int E, int K, 
   __syncwarp();
 }
 
+// Copies the E logits of one token into the warp's shared-memory row with
+// independent (unrolled, 16-byte where aligned) loads, so the K selection
+// passes of route_token_warp read shared memory instead of issuing one
+// dependent global load per pass and lane.
+__device__ __forceinline__ void stage_logits_warp(const float* __restrict__ lg, float* row, int E) {
+  const int lane = threadIdx.x & 31;
+  if ((((uintptr_t)lg | (uintptr_t)row) & 15) == 0 && (E & 3) == 0) {
+    const float4* g4 = reinterpret_cast<const float4*>(lg);
+    float4* r4 = reinterpret_cast<float4*>(row);
+    const int E4 = E >> 2;
+    int i = lane;
+    for (; i + 96 < E4; i += 128) {
+      const float4 a = g4[i], b = g4[i + 32], c = g4[i + 64], d = g4[i + 96];
+      r4[i] = a;
+      r4[i + 32] = b;
+      r4[i + 64] = c;
+      r4[i + 96] = d;
+    }
+    for (; i < E4; i += 32) r4[i] = g4[i];
+  } else {
+    for (int e = lane; e < E; e += 32) row[e] = lg[e];
+  }
+  __syncwarp();
+}
+
 }  // namespace moeq
