@@ -179,6 +179,37 @@ moeq_status moeq_layer_forward(const moeq_layer* L, const uint16_t* x, int32_t M
  * in `mode` (0 if the arguments are invalid). */
 size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mode);
 
+/*
+ * moeq_layer_forward in DECODE mode with the workspace taken from a fixed
+ * device array inside this library instead of from the caller.  The paper
+ * has no counterpart: the method's pages do not discuss where intermediate
+ * buffers live.  This entry point allocates no device or host memory; it is
+ * for callers that cannot pass a workspace, because they have no device
+ * allocator at the call site or must not allocate while serving (an
+ * allocation can synchronise the device; a pool sized at start-up may not
+ * grow).
+ *   Arguments, layouts and device-side errors are those of
+ *   moeq_layer_forward with mode DECODE (M <= 64).
+ *   Capacity: moeq_static_workspace_capacity() bytes (8 MiB) per device,
+ *   which covers for example H 4096, I 1024, E 512, K 4 with a shared
+ *   expert up to M 64.  When moeq_workspace_bytes(L, M, DECODE) exceeds it
+ *   the call launches nothing and returns MOEQ_ERR_WORKSPACE.
+ *   Set-up: the first call on each device (with that device current) looks
+ *   up the array's device address; make that first call before any stream
+ *   capture begins.  A failed lookup returns MOEQ_ERR_CUDA.
+ *   Sharing: all calls on a device use the same array.  Nothing in it has to
+ *   start at zero, but calls whose work overlaps in time on one device (on
+ *   different streams, or from host threads without ordering between them)
+ *   race on it; order such calls (one stream, or events) yourself.
+ * Errors: those of moeq_layer_forward, and WORKSPACE / CUDA as above.
+ */
+moeq_status moeq_layer_forward_static(const moeq_layer* L, const uint16_t* x, int32_t M,
+                                      float* y, const float* residual, int32_t* idx_out,
+                                      float* w_out, void* stream);
+
+/* Bytes of the fixed per-device workspace of moeq_layer_forward_static. */
+size_t moeq_static_workspace_capacity(void);
+
 /* Reads and clears the device status word of the current device (synchronises
  * `stream`).  *status_out receives MOEQ_OK or the first device error seen. */
 moeq_status moeq_device_status(void* stream, int32_t* status_out);

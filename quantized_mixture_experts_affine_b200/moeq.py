@@ -25,7 +25,8 @@ MODE_AUTO, MODE_DECODE, MODE_PREFILL = 0, 1, 2
 
 EXPORTS = ("moeq_dequant", "moeq_qmv", "moeq_route_topk", "moeq_expert_ffn", "moeq_layer_forward",
            "moeq_workspace_bytes", "moeq_device_status", "moeq_status_str", "moeq_version",
-           "moeq_set_profile_events", "moeq_launch_count")
+           "moeq_set_profile_events", "moeq_launch_count", "moeq_layer_forward_static",
+           "moeq_static_workspace_capacity")
 
 
 class MoeqError(RuntimeError):
@@ -60,6 +61,8 @@ _lib.moeq_expert_ffn.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P
                                  C.c_int32, _P]
 _lib.moeq_layer_forward.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P, _P,
                                     C.c_size_t, C.c_int32, _P]
+_lib.moeq_layer_forward_static.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P, _P]
+_lib.moeq_static_workspace_capacity.restype = C.c_size_t
 _lib.moeq_workspace_bytes.argtypes = [C.POINTER(Layer), C.c_int32, C.c_int32]
 _lib.moeq_workspace_bytes.restype = C.c_size_t
 _lib.moeq_device_status.argtypes = [_P, C.POINTER(C.c_int32)]
@@ -70,7 +73,7 @@ _lib.moeq_set_profile_events.argtypes = [_P, _P]
 _lib.moeq_set_profile_events.restype = C.c_int
 _lib.moeq_launch_count.restype = C.c_uint64
 for _f in ("moeq_dequant", "moeq_qmv", "moeq_route_topk", "moeq_expert_ffn", "moeq_layer_forward",
-           "moeq_device_status"):
+           "moeq_layer_forward_static", "moeq_device_status"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -148,6 +151,18 @@ def moeq_layer_forward(L: Layer, x, M: int, y, residual=None, idx_out=None, w_ou
            _lib.moeq_layer_forward(C.byref(L), _ptr(x), M, _ptr(y), _ptr(residual),
                                    _ptr(idx_out), _ptr(w_out), _ptr(ws), ws_bytes, mode,
                                    _stream(stream)))
+
+
+def moeq_layer_forward_static(L: Layer, x, M: int, y, residual=None, idx_out=None, w_out=None,
+                              stream=None) -> None:
+    """Decode layer forward on the library's fixed per-device workspace."""
+    _check("moeq_layer_forward_static",
+           _lib.moeq_layer_forward_static(C.byref(L), _ptr(x), M, _ptr(y), _ptr(residual),
+                                          _ptr(idx_out), _ptr(w_out), _stream(stream)))
+
+
+def moeq_static_workspace_capacity() -> int:
+    return int(_lib.moeq_static_workspace_capacity())
 
 
 def moeq_set_profile_events(start=None, stop=None) -> None:

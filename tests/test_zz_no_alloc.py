@@ -1,0 +1,82 @@
+"""moeq_layer_forward_static (decode forward on the library's fixed device
+workspace) against moeq_layer_forward with a caller workspace, through the
+C ABI.  Collected last so that it also runs after every other test has used
+the library on the same device.
+
+Bars: two calls in a row each agree with the ordinary entry point within
+the layer tolerance (relative L2 <= 2e-3, max abs <= 1e-2) and route the
+same; a layer whose decode workspace exceeds the fixed capacity is refused
+with MOEQ_ERR_WORKSPACE before anything is launched.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+
+from helpers import MAX_ABS, REL_L2, rel_l2
+from quantized_mixture_experts_affine_b200 import moeq, synth
+from quantized_mixture_experts_affine_b200.layer import CONFIGS, layer_forward, synthetic_layer
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+SEED = 0
+
+
+def x_tokens(cfg, M, copy):
+    xb = synth.normal_bf16_host(SEED, synth.tag(synth.X, copy), M * cfg.H).reshape(M, cfg.H)
+    return torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("name,M", [("decode_397b", 1), ("decode_397b", 64), ("decode_30b", 5)])
+def test_static_matches_caller_workspace(name, M):
+    cfg = CONFIGS[name]
+    L = synthetic_layer(cfg, SEED, 0)
+    assert moeq.moeq_workspace_bytes(L.desc, M, moeq.MODE_DECODE) <= \
+        moeq.moeq_static_workspace_capacity()
+    x = x_tokens(cfg, M, 300 + M)
+    res = torch.linspace(-1, 1, M * cfg.H, device="cuda").reshape(M, cfg.H)
+    y_ref, i_ref, w_ref = layer_forward(L, x, residual=res, mode=moeq.MODE_DECODE)
+    torch.cuda.synchronize()
+    ref = y_ref.cpu().numpy()
+    for poison in (float("nan"), 1e30):  # two calls in a row on the shared array
+        y = torch.full((M, cfg.H), poison, device="cuda")
+        idx = torch.full((M, cfg.K), -1, dtype=torch.int32, device="cuda")
+        w = torch.full((M, cfg.K), poison, device="cuda")
+        moeq.moeq_layer_forward_static(L.desc, x, M, y, residual=res, idx_out=idx, w_out=w)
+        torch.cuda.synchronize()
+        assert moeq.moeq_device_status() == 0
+        got = y.cpu().numpy()
+        assert np.isfinite(got).all()
+        assert rel_l2(got, ref) <= REL_L2 and np.abs(got - ref).max() <= MAX_ABS
+        assert torch.equal(idx, i_ref)
+        assert np.abs(w.cpu().numpy() - w_ref.cpu().numpy()).max() <= 1e-6
+
+
+def test_static_refuses_oversized_workspace():
+    """H 8192, E 512, K 8, I 2048 at M 64 needs about 19 MB of decode
+    workspace: refused on the host; the outputs stay untouched."""
+    buf = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    p = buf.data_ptr()
+    H, I, E, K, M = 8192, 2048, 512, 8, 64
+
+    def qt(out, inn, n):
+        return moeq.qtensor(p, p, p, out, inn, 4, 64, n)
+
+    desc = moeq.Layer()
+    desc.router = moeq.qtensor(p, p, p, E, H, 8, 64, 1)
+    desc.gate, desc.up, desc.down = qt(I, H, E), qt(I, H, E), qt(H, I, E)
+    desc.hidden, desc.inter, desc.n_experts, desc.top_k = H, I, E, K
+    desc.renorm, desc.router_scale, desc.has_shared = 1, 1.0, 0
+    need = moeq.moeq_workspace_bytes(desc, M, moeq.MODE_DECODE)
+    assert need > moeq.moeq_static_workspace_capacity()
+    launches = moeq.moeq_launch_count()
+    rc = moeq.lib().moeq_layer_forward_static(C.byref(desc), p, M, p, None, None, None,
+                                              torch.cuda.current_stream().cuda_stream)
+    assert rc == moeq.ERR_WORKSPACE
+    assert moeq.moeq_launch_count() == launches
+    torch.cuda.synchronize()
+    assert int(buf.count_nonzero()) == 0
+    # within capacity at M 1 for the same layer: accepted by the checks
+    assert moeq.moeq_workspace_bytes(desc, 1, moeq.MODE_DECODE) <= \
+        moeq.moeq_static_workspace_capacity()
