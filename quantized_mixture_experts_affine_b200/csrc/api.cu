@@ -154,7 +154,8 @@ struct Carve {
 };
 
 struct DecodeWs {
-  size_t logits, sg_logit, sigma, idx, w, h, d, segs_gu, segs_dn, counts, vecs_gu, vecs_dn, total;
+  size_t logits, sg_logit, sigma, idx, w, h, d, segs_gu, segs_dn, counts, vecs_gu, vecs_dn, ctr,
+      total;
 };
 
 DecodeWs decode_ws(const moeq_layer* L, int M) {
@@ -175,6 +176,7 @@ DecodeWs decode_ws(const moeq_layer* L, int M) {
   w.counts = c.take(8 * 4);
   w.vecs_gu = c.take(n * sizeof(VecRef));
   w.vecs_dn = c.take(n * sizeof(VecRef));
+  w.ctr = c.take((size_t)H * 4);  // at most one counter per output row
   w.total = c.off;
   return w;
 }
@@ -266,7 +268,13 @@ static cudaError_t run_plain(const moeq_qtensor& shape_t, const Seg* segs, int n
   a.n_segs = n;
   a.total_units = units;
   a.status = status_ptr();
-  const int grid = units < grid_cap() ? units : grid_cap();
+  // a launch that carries L2 prefetches gets enough CTAs to spread them
+  // (one 32 KB piece per CTA and lane); CTAs without a unit only prefetch
+  int64_t pieces = 0;
+  for (int i = 0; i < a.n_pf; ++i) pieces += (a.pf[i].bytes + 32 * 1024 - 1) / (32 * 1024);
+  int grid = units;
+  if (pieces / 8 > grid) grid = (int)(pieces / 8);
+  if (grid > grid_cap()) grid = grid_cap();
   return launch_gemv(shape_t.bits, nl, 1, SRC_BF16, a, grid, st);
 }
 
@@ -383,6 +391,8 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   p.vecs_dn = vecs_dn;
   p.units_per_seg_gu = units_for(L->gate, I, 2);
   p.units_per_seg_dn = units_for(L->down, H, 1);
+  p.ctr = (int32_t*)(base + lay.ctr);
+  p.n_ctr = p.units_per_seg_dn;
   if (L->has_shared) {
     p.units_per_seg_gu_sh = units_for(L->sh_gate, L->sh_gate.out_dim, 2);
     p.units_per_seg_dn_sh = units_for(L->sh_down, H, 1);
@@ -392,28 +402,70 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
                         L->sh_down.group_size == L->down.group_size &&
                         L->sh_down.in_dim == L->down.in_dim);
   }
-  p.prefetch = 0;
   p.status = status_ptr();
-  LAUNCH(launch_decode_plan(p, st));
+  // small steps: every gate/up CTA computes the plan itself (no plan launch)
+  const bool fused_plan =
+      n <= kFusedMaxPairs && (!L->has_shared || p.shared_same_gu) &&
+      plan_scratch_bytes(M, K, E, plan_route_warps(M, E, gemv_threads() / 32)) <=
+          (size_t)gemv_ring_bytes();
+  // the down launch covers every segment: its CTAs also do the combine
+  const bool fuse_combine = !L->has_shared || p.shared_same_dn;
+  if (!fused_plan) LAUNCH(launch_decode_plan(p, st));
 
   // 3. gate/up + SwiGLU, then 4. down, for the routed experts (+ shared)
   const int max_entries = n < E ? n : E;
   const int max_gu = max_entries * p.units_per_seg_gu + (p.shared_same_gu ? p.units_per_seg_gu_sh : 0);
   const int max_dn = max_entries * p.units_per_seg_dn + (p.shared_same_dn ? p.units_per_seg_dn_sh : 0);
   CK(profile_mark(true, st));
-  // the gate/up launch also pulls the down projections it will feed into L2
-  LAUNCH(run_dyn(L->gate, segs_gu, counts, 2, 2, SRC_BF16, max_gu, st, segs_dn, counts + 4));
+  if (fused_plan) {
+    // the gate/up launch plans, and pulls the down projections into L2
+    GemvArgs a;
+    memset(&a, 0, sizeof(a));
+    set_shape(a, L->gate, 2);
+    a.status = status_ptr();
+    a.fused_plan = 1;
+    a.plan = p;
+    const int grid = max_gu < grid_cap() ? max_gu : grid_cap();
+    LAUNCH(launch_gemv(L->gate.bits, 2, 2, SRC_BF16, a, grid, st));
+  } else {
+    // the gate/up launch also pulls the down projections it will feed into L2
+    LAUNCH(run_dyn(L->gate, segs_gu, counts, 2, 2, SRC_BF16, max_gu, st, segs_dn, counts + 4));
+  }
   CK(profile_mark(false, st));
   if (L->has_shared && !p.shared_same_gu)
     LAUNCH(run_dyn(L->sh_gate, segs_gu + n, counts + 2, 2, 2, SRC_BF16, p.units_per_seg_gu_sh,
                    st));
-  LAUNCH(run_dyn(L->down, segs_dn, counts + 4, 2, 1, SRC_F32, max_dn, st));
+  {
+    GemvArgs a;
+    memset(&a, 0, sizeof(a));
+    set_shape(a, L->down, 1);
+    a.dyn_segs = segs_dn;
+    a.dyn_count = counts + 4;
+    a.status = status_ptr();
+    if (fuse_combine) {
+      a.fuse_combine = 1;
+      a.comb.w = wts;
+      a.comb.sigma = sigma;
+      a.comb.residual = residual;
+      a.comb.y = y;
+      a.comb.d = d;
+      a.comb.ctr = p.ctr;
+      a.comb.M = M;
+      a.comb.K = K;
+      a.comb.H = H;
+      a.comb.has_shared = L->has_shared;
+    }
+    const int grid = max_dn < grid_cap() ? max_dn : grid_cap();
+    LAUNCH(launch_gemv(L->down.bits, 2, 1, SRC_F32, a, grid, st));
+  }
   if (L->has_shared && !p.shared_same_dn)
     LAUNCH(run_dyn(L->sh_down, segs_dn + n, counts + 6, 2, 1, SRC_F32, p.units_per_seg_dn_sh,
                    st));
 
-  // 5. weighted combine in k order (+ shared, + residual)
-  LAUNCH(launch_combine(d, wts, sigma, L->has_shared, residual, y, M, K, H, st));
+  // 5. weighted combine in k order (+ shared, + residual), unless the down
+  //    launch did it
+  if (!fuse_combine)
+    LAUNCH(launch_combine(d, wts, sigma, L->has_shared, residual, y, M, K, H, st));
   return MOEQ_OK;
 }
 

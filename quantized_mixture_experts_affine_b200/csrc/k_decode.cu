@@ -28,23 +28,26 @@ bool gemv_fits(int in_dim, int bits, int nmat, int G) {
 int gemv_units(int out_dim, const GemvShape& sh) { return (out_dim + sh.RU - 1) / sh.RU; }
 
 // ============================================================== staged GEMV kernel
-// Persistent CTAs (one per SM).  Warp 8 is the producer: it reads the work
+// Persistent CTAs (one per SM).  Warp 16 is the producer: it reads the work
 // description of up to 32 of its CTA's units at once (one unit per lane),
 // then per unit (RU consecutive rows of NMAT matrices of one segment) lane
 // 0 issues bulk copies of the contiguous packed rows into a 4-stage
 // shared-memory ring, and all lanes copy the rows' bf16 scale/bias pairs
-// and the unit's input/output vector references with cp.async.  Warp 9
-// issues the L2 prefetches.  Warps 0..S*J-1 consume: warp (slice s, subset
-// j) keeps its 32-chunk slice of the input vector in registers as
-// fixed-point limbs, takes RU/J rows of each matrix from the stage (one
-// 16-byte chunk per lane per row), reduces the eight row partials of each
-// lane with the transposing butterfly, and the S slices are summed in fixed
-// order through a double-buffered shared-memory exchange guarded by
-// mbarriers (every wait bounded).
-constexpr int GV_CW = 8;                  // consumer warps
-constexpr int GV_PRODUCER = GV_CW;        // producer warp
-constexpr int GV_HELPER = GV_CW + 1;      // L2-prefetch warp
-constexpr int GV_THREADS = (GV_CW + 2) * 32;
+// and the unit's input/output vector references with cp.async.  Warp 17
+// issues the L2 prefetches.  Warps 0-15 form two consumer groups that take
+// alternate units, so one group computes while the other waits for its
+// stage.  In a group, warps 0..S*J-1 consume: warp (slice s, subset j)
+// keeps its 32-chunk slice of the input vector in registers as fixed-point
+// limbs, takes RU/J rows of each matrix from the stage (one 16-byte chunk
+// per lane per row), reduces the eight row partials of each lane with the
+// transposing butterfly, and the S slices are summed in fixed order through
+// a double-buffered shared-memory exchange guarded by mbarriers (every wait
+// bounded).
+constexpr int GV_CW = 8;                  // consumer warps per group
+constexpr int GV_GROUPS = 2;              // consumer groups, alternating units
+constexpr int GV_PRODUCER = GV_GROUPS * GV_CW;  // producer warp
+constexpr int GV_HELPER = GV_PRODUCER + 1;      // L2-prefetch warp
+constexpr int GV_THREADS = (GV_PRODUCER + 2) * 32;
 constexpr int GV_STAGES = 4;
 constexpr int GV_STAGE_BYTES = 44 * 1024;
 constexpr int GV_VMAX = 64;               // vector references staged per unit
@@ -67,11 +70,24 @@ struct GvSmem {
   static constexpr int VEC_OFF = META_OFF + GV_STAGES * META_STRIDE;
   static constexpr int UB_OFF = VEC_OFF + GV_STAGES * GV_VMAX * 16;
   static constexpr int BAR_OFF = UB_OFF + GV_UB_CAP * 4;
-  static constexpr int N_BARS = 2 * GV_STAGES + 4;
+  static constexpr int N_BARS = 2 * GV_STAGES + 4 * GV_GROUPS;
   static constexpr int RED_OFF = BAR_OFF + N_BARS * 8;
-  static constexpr int BYTES = RED_OFF + 2 * GV_CW * 8 * 4;
+  // the CTA's own plan (gate/up launch that computes it): segments, vector
+  // references, counts, experts; then the fused combine's flags
+  static constexpr int PSEG_OFF = RED_OFF + GV_GROUPS * 2 * GV_CW * 8 * 4;
+  static constexpr int PVEC_OFF = PSEG_OFF + (((kFusedMaxPairs + 1) * (int)sizeof(Seg) + 15) & ~15);
+  static constexpr int PCNT_OFF = PVEC_OFF + kFusedMaxPairs * 16;
+  static constexpr int PEXP_OFF = PCNT_OFF + 8 * 4;
+  static constexpr int FLAG_OFF = PEXP_OFF + kFusedMaxPairs * 4;
+  static constexpr int BYTES = FLAG_OFF + GV_GROUPS * 4;
+  static constexpr int RING_BYTES = GV_STAGES * GV_STAGE_BYTES;
 };
 static_assert(sizeof(GvMeta) <= GvSmem::META_STRIDE, "GvMeta exceeds its slot");
+static_assert(GvSmem::BYTES <= 227 * 1024, "GEMV shared memory exceeds the per-CTA limit");
+static_assert(GvSmem::PSEG_OFF % 16 == 0 && GvSmem::PVEC_OFF % 16 == 0, "plan region alignment");
+
+int gemv_threads() { return GV_THREADS; }
+int gemv_ring_bytes() { return GvSmem::RING_BYTES; }
 static_assert(sizeof(VecRef) == 16, "VecRef is copied in 16-byte pieces");
 
 // Last segment whose first unit is <= unit; p[i * stride] is segment i's
@@ -132,6 +148,58 @@ __device__ __forceinline__ void prefetch_segs(const Seg* segs, int n) {
   }
 }
 
+// Down projections (codes, scales, biases) of the listed experts and of
+// the shared expert into L2, spread over the CTAs in 32 KB pieces.
+__device__ __forceinline__ void prefetch_down(const DecodePlanArgs& p, const int32_t* ent,
+                                              int n_ent) {
+  constexpr int64_t PIECE = 32 * 1024;
+  const int lane = threadIdx.x & 31;
+  const int n_src = n_ent + (p.has_shared ? 1 : 0);
+  int64_t g0 = 0;
+  for (int i = 0; i < n_src; ++i) {
+    const bool sh = i >= n_ent;
+    const moeq_qtensor& t = sh ? p.sh_down : p.down;
+    const int64_t e = sh ? 0 : ent[i];
+    const int64_t gr = (int64_t)t.out_dim * (t.in_dim / t.group_size);
+    const void* ptr[3] = {t.w + e * t.expert_stride_w, t.scales + e * t.expert_stride_sb,
+                          t.biases + e * t.expert_stride_sb};
+    const int64_t bytes[3] = {(int64_t)t.out_dim * t.in_dim * t.bits / 8, gr * 2, gr * 2};
+    for (int k = 0; k < 3; ++k) {
+      const int64_t pieces = (bytes[k] + PIECE - 1) / PIECE;
+      int64_t g = g0 + ((blockIdx.x - g0 % gridDim.x) + gridDim.x) % gridDim.x;
+      for (int64_t j = 0; g < g0 + pieces; g += gridDim.x, ++j) {
+        if ((int)(j % 32) != lane) continue;
+        const int64_t off = (g - g0) * PIECE;
+        const int64_t len = min(PIECE, bytes[k] - off) & ~(int64_t)15;
+        if (len > 0 && ((uintptr_t)ptr[k] & 15) == 0)
+          tc::prefetch_l2((const uint8_t*)ptr[k] + off, (uint32_t)len);
+      }
+      g0 += pieces;
+    }
+  }
+}
+
+__device__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, int R, const PlanSinks& o);
+
+// y[m][r] = sum_k w[m][k] d[m*K + k][r] (+ sigma[m] d[M*K + m][r]) (+ residual[m][r])
+// for rows [r0, r0 + nrows), k in order; the same operations as k_combine.
+// The d rows come from other CTAs of this launch: read through L2.
+__device__ __forceinline__ void combine_rows(const CombineArgs& c, int r0, int nrows, int t,
+                                             int nt) {
+  const int total = c.M * nrows;
+  for (int i = t; i < total; i += nt) {
+    const int m = i / nrows;
+    const int r = r0 + i % nrows;
+    float acc = 0.0f;
+    for (int k = 0; k < c.K; ++k)
+      acc = fmaf(c.w[m * c.K + k], __ldcg(c.d + ((int64_t)m * c.K + k) * c.H + r), acc);
+    if (c.has_shared)
+      acc = fmaf(c.sigma[m], __ldcg(c.d + ((int64_t)c.M * c.K + m) * c.H + r), acc);
+    if (c.residual) acc += c.residual[(int64_t)m * c.H + r];
+    c.y[(int64_t)m * c.H + r] = acc;
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ T shfl_ptr(T p, int src) {
   return reinterpret_cast<T>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(p), src));
@@ -149,9 +217,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   int32_t* ub = reinterpret_cast<int32_t*>(gsm + GvSmem::UB_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(gsm + GvSmem::BAR_OFF);
   uint64_t* empty = full + GV_STAGES;
-  uint64_t* red_full = empty + GV_STAGES;  // 2: slices 1..S-1 -> slice 0
-  uint64_t* red_empty = red_full + 2;      // 2: slice 0 -> slices 1..S-1
-  float* red = reinterpret_cast<float*>(gsm + GvSmem::RED_OFF);  // [2][GV_CW][8]
+  uint64_t* red_full = empty + GV_STAGES;           // [group][2]: slices 1..S-1 -> slice 0
+  uint64_t* red_empty = red_full + 2 * GV_GROUPS;   // [group][2]: slice 0 -> slices 1..S-1
+  float* red = reinterpret_cast<float*>(gsm + GvSmem::RED_OFF);  // [group][2][GV_CW][8]
   const uint32_t sbase = tc::smem_u32(gsm);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -162,7 +230,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
       tc::mbar_init(&full[i], 1 + 32);
       tc::mbar_init(&empty[i], GV_CW * 32);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2 * GV_GROUPS; ++i) {
       tc::mbar_init(&red_full[i], (uint32_t)((S > 1 ? S - 1 : 1) * J * 8));
       tc::mbar_init(&red_empty[i], (uint32_t)(J * 8));
     }
@@ -176,9 +244,41 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   tc::grid_dep_wait();
   tc::grid_dep_launch();
 
-  const Seg* segs = a.dyn_segs ? a.dyn_segs : a.segs;
-  const int n_segs = a.dyn_segs ? a.dyn_count[0] : a.n_segs;
-  const int total_units = a.dyn_segs ? a.dyn_count[1] : a.total_units;
+  const Seg* segs;
+  int n_segs, total_units;
+  int32_t* pcnt = reinterpret_cast<int32_t*>(gsm + GvSmem::PCNT_OFF);
+  int32_t* pexp = reinterpret_cast<int32_t*>(gsm + GvSmem::PEXP_OFF);
+  if (a.fused_plan) {
+    // this CTA's copy of the step's plan, in shared memory; CTA 0 also
+    // writes the routing, the down lists and zeroed combine counters
+    Seg* psegs = reinterpret_cast<Seg*>(gsm + GvSmem::PSEG_OFF);
+    PlanSinks o;
+    memset(&o, 0, sizeof(o));
+    o.segs_gu = psegs;
+    o.count_gu = pcnt;
+    o.vecs_gu = reinterpret_cast<VecRef*>(gsm + GvSmem::PVEC_OFF);
+    o.experts = pexp;
+    o.n_experts = pcnt + 4;
+    if (blockIdx.x == 0) {
+      o.idx = a.plan.idx_out;
+      o.w = a.plan.w_out;
+      o.sigma = a.plan.sigma;
+      o.segs_dn = a.plan.segs_dn;
+      o.count_dn = a.plan.count_dn;
+      o.vecs_dn = a.plan.vecs_dn;
+      o.ctr = a.plan.ctr;
+      o.n_ctr = a.plan.n_ctr;
+    }
+    // the scratch of the plan lives in the (still unused) stage ring
+    plan_cta(a.plan, gsm, plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32), o);
+    segs = psegs;
+    n_segs = pcnt[0];
+    total_units = pcnt[1];
+  } else {
+    segs = a.dyn_segs ? a.dyn_segs : a.segs;
+    n_segs = a.dyn_segs ? a.dyn_count[0] : a.n_segs;
+    total_units = a.dyn_segs ? a.dyn_count[1] : a.total_units;
+  }
   const bool ub_cached = n_segs <= GV_UB_CAP;
   if (ub_cached)
     for (int i = threadIdx.x; i < n_segs; i += blockDim.x) ub[i] = segs[i].unit_begin;
@@ -194,7 +294,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
 
   if (warp == GV_HELPER) {
     // ------------------------------------------------------------ L2 prefetch
-    if (a.pf_segs) prefetch_segs(a.pf_segs, a.pf_count[0]);
+    if (a.fused_plan) prefetch_down(a.plan, pexp, pcnt[4]);
+    else if (a.pf_segs) prefetch_segs(a.pf_segs, a.pf_count[0]);
   } else if (warp == GV_PRODUCER) {
     // ------------------------------------------------------------ producer
     uint32_t it = 0;
@@ -288,7 +389,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
             tc::cp_async4(bd + 4 * p, b0 + 2 * p, 4);
           }
         }
-        if (uvm == 1 && unv <= GV_VMAX) {
+        if (uvm == 1 && unv <= GV_VMAX && !__isShared(uvecs)) {
           const uint32_t vd = sbase + GvSmem::VEC_OFF + s * GV_VMAX * 16;
           for (int v = lane; v < unv; v += 32) tc::cp_async16(vd + 16 * v, uvecs + v, 16);
         }
@@ -297,8 +398,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ consumers
-    const bool on_w = warp < W;
-    const int sl = warp % S, j = warp / S;
+    // group grp takes every GV_GROUPS-th unit of the CTA (stages grp, grp + GV_GROUPS, ...)
+    const int grp = warp / GV_CW, cw = warp % GV_CW;
+    const bool on_w = cw < W;
+    const int sl = cw % S, j = cw / S;
     const int ch = sl * 32 + lane;
     const bool lane_on = on_w && ch < cpr;
     int gi[2];
@@ -309,17 +412,21 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     // After a wait that ran out, every later wait is skipped and no vector
     // is processed; all waits are bounded, so the CTA always ends.
     bool timed_out = false;
-    uint32_t it = 0, rc = 0;
-    for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x, ++it) {
+    uint32_t it = grp, rc = 0;
+    for (int unit = blockIdx.x + grp * gridDim.x; unit < total_units;
+         unit += GV_GROUPS * gridDim.x, it += GV_GROUPS) {
       const uint32_t s = it % GV_STAGES, ph = (it / GV_STAGES) & 1u;
       if (!timed_out) timed_out = !tc::mbar_wait(&full[s], ph, status);
       const GvMeta* mp = reinterpret_cast<const GvMeta*>(gsm + GvSmem::META_OFF +
                                                          s * GvSmem::META_STRIDE);
       const int n_vec = timed_out ? 0 : mp->n_vec;
+      const int r0 = timed_out ? 0 : mp->r0, nrows = timed_out ? 0 : mp->nrows;
       const uint32_t st = sbase + s * GV_STAGE_BYTES;
       if (on_w && n_vec > 0) {
-        const int r0 = mp->r0, nrows = mp->nrows, vec_mode = mp->vec_mode;
-        const VecRef* vl = (vec_mode == 1 && n_vec <= GV_VMAX) ? svec + s * GV_VMAX : mp->vecs;
+        const int vec_mode = mp->vec_mode;
+        const VecRef* vl = (vec_mode == 1 && n_vec <= GV_VMAX && !__isShared(mp->vecs))
+                               ? svec + s * GV_VMAX
+                               : mp->vecs;
         for (int v = 0; v < n_vec && !timed_out; ++v) {
           const void* src;
           float* dst;
@@ -365,20 +472,22 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
             // in slice order
             const uint32_t buf = rc & 1u, rph = (rc >> 1) & 1u;
             ++rc;
-            float* rb = red + buf * GV_CW * 8;
+            float* rb = red + (grp * 2 + buf) * GV_CW * 8;
+            uint64_t* rf = &red_full[grp * 2 + buf];
+            uint64_t* re = &red_empty[grp * 2 + buf];
             if (sl != 0) {
-              if (!tc::mbar_wait(&red_empty[buf], rph ^ 1u, status)) timed_out = true;
+              if (!tc::mbar_wait(re, rph ^ 1u, status)) timed_out = true;
               if (lane < 8) {
-                rb[warp * 8 + lane] = tot;
-                tc::mbar_arrive(&red_full[buf]);
+                rb[cw * 8 + lane] = tot;
+                tc::mbar_arrive(rf);
               }
             } else {
-              if (!tc::mbar_wait(&red_full[buf], rph, status)) timed_out = true;
+              if (!tc::mbar_wait(rf, rph, status)) timed_out = true;
               if (lane < 8) {
                 float t = tot;
                 for (int q = 1; q < S; ++q) t += rb[(j * S + q) * 8 + lane];
                 tot = t;
-                tc::mbar_arrive(&red_empty[buf]);
+                tc::mbar_arrive(re);
               }
             }
           }
@@ -395,6 +504,23 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         }
       }
       tc::mbar_arrive(&empty[s]);
+      if (EPI == EPI_PLAIN && a.fuse_combine) {
+        // the group's stores of this unit are done; the CTA that brings the
+        // row block's count to the number of segments sums the block
+        __threadfence();
+        tc::named_sync(2 + grp, GV_CW * 32);
+        int* flag = reinterpret_cast<int*>(gsm + GvSmem::FLAG_OFF) + grp;
+        if (cw == 0 && lane == 0) {
+          int last = 0;
+          if (n_vec > 0) {
+            last = atomicAdd(&a.comb.ctr[r0 / RU], 1) == n_segs - 1;
+            if (last) __threadfence();
+          }
+          *flag = last;
+        }
+        tc::named_sync(2 + grp, GV_CW * 32);
+        if (*flag) combine_rows(a.comb, r0, nrows, cw * 32 + lane, GV_CW * 32);
+      }
     }
   }
 }
@@ -446,214 +572,229 @@ cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, 
 }
 
 // ============================================================== top-K routing
+// One warp per token; each warp stages its token's logits in shared memory.
 __global__ void __launch_bounds__(256) k_route_topk(const float* __restrict__ logits, int M, int E,
                                                     int K, int renorm, float scale,
                                                     int32_t* __restrict__ idx,
                                                     float* __restrict__ w) {
-  extern __shared__ uint32_t taken_all[];
-  const int warp = threadIdx.x >> 5;
+  extern __shared__ __align__(16) uint8_t rsm[];
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int words = (E + 31) >> 5;
-  uint32_t* taken = taken_all + warp * words;
-  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int wbytes = ((words * 4 + 15) & ~15) + E * 4;
+  uint32_t* taken = reinterpret_cast<uint32_t*>(rsm + warp * wbytes);
+  float* row = reinterpret_cast<float*>(rsm + warp * wbytes + ((words * 4 + 15) & ~15));
+  const int t = blockIdx.x * nw + warp;
   if (t >= M) return;
-  route_token_warp(logits + (int64_t)t * E, E, K, renorm, scale, idx + (int64_t)t * K,
-                   w + (int64_t)t * K, taken);
+  stage_logits_warp(logits + (int64_t)t * E, row, E);
+  route_token_warp(row, E, K, renorm, scale, idx + (int64_t)t * K, w + (int64_t)t * K, taken);
+}
+
+// Warps per routing CTA so that the staged rows fit 48 KB.
+int route_warps_per_cta(int E) {
+  const int wbytes = (((E + 31) / 32 * 4 + 15) & ~15) + E * 4;
+  int w = (48 * 1024) / wbytes;
+  return w < 1 ? 1 : (w > 8 ? 8 : w);
 }
 
 cudaError_t launch_route_topk(const float* logits, int M, int E, int K, int renorm, float scale,
                               int32_t* idx, float* w, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  const int warps = 8;
+  const int warps = route_warps_per_cta(E);
   const int grid = (M + warps - 1) / warps;
-  const size_t smem = (size_t)warps * ((E + 31) / 32) * 4;
+  const size_t smem = (size_t)warps * ((((E + 31) / 32 * 4 + 15) & ~15) + (size_t)E * 4);
   k_route_topk<<<grid, warps * 32, smem, st>>>(logits, M, E, K, renorm, scale, idx, w);
   return cudaGetLastError();
 }
 
 // ============================================================== decode plan
-// Routing warps of the plan kernel: one token each at a time, E floats of
-// staged logits per warp, at most 64 KB of staging.
-__host__ __device__ __forceinline__ int plan_route_warps(int M, int E, int nwarps) {
-  int r = (64 * 1024) / (E * 4);
+__host__ __device__ int plan_route_warps(int M, int E, int nwarps) {
+  int r = kPlanStageBytes / (E * 4);
   if (r < 1) r = 1;
   if (r > nwarps) r = nwarps;
   if (r > M) r = M;
   return r;
 }
 
-// Shared-memory region after the plan's per-warp bitmaps: n ints.
-__device__ __forceinline__ int32_t* taken_list(uint32_t* sm, int n, int E, int nwarps) {
-  return reinterpret_cast<int32_t*>(sm) + 4 * n + nwarps * ((E + 31) >> 5);
+// Scratch of one CTA's plan: routing results, sort keys and the staged
+// logit rows of R routing warps.
+struct PlanScratch {
+  int32_t* sidx;      // [n] routed experts
+  float* sw;          // [n] routed weights
+  float* ssig;        // [M] shared-expert gate values
+  int32_t* key;       // [n] expert of pair
+  int32_t* sorted;    // [n] pairs sorted by (expert, pair)
+  int32_t* head;      // [n] 1 at the first pair of an expert
+  int32_t* entry_of;  // [n] entry index of sorted position
+  uint32_t* taken;    // [R][words] routing bitmaps
+  float* rows;        // [R][E] staged logits (16-byte aligned)
+};
+
+__host__ __device__ size_t plan_scratch_bytes(int M, int K, int E, int R) {
+  const size_t n = (size_t)M * K;
+  size_t b = (7 * n + (size_t)M) * 4 + (size_t)R * ((E + 31) / 32) * 4;
+  b = (b + 15) & ~(size_t)15;
+  return b + (size_t)R * E * 4;
 }
 
-// One CTA (1024 threads).  Routes the M tokens (unless the routing is given),
-// computes the shared-expert gate, sorts the M*K (token, slot) pairs by
-// expert (stable) and writes one gate/up segment and one down segment per
-// distinct expert, then the shared expert's segments.
-__global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ DecodePlanArgs a) {
-  extern __shared__ uint32_t sm[];
+__device__ __forceinline__ PlanScratch plan_scratch(uint8_t* sm, int M, int K, int E, int R) {
+  const int n = M * K;
+  PlanScratch p;
+  p.sidx = reinterpret_cast<int32_t*>(sm);
+  p.sw = reinterpret_cast<float*>(p.sidx + n);
+  p.ssig = p.sw + n;
+  p.key = reinterpret_cast<int32_t*>(p.ssig + M);
+  p.sorted = p.key + n;
+  p.head = p.sorted + n;
+  p.entry_of = p.head + n;
+  p.taken = reinterpret_cast<uint32_t*>(p.entry_of + n);
+  size_t off = (size_t)(7 * n + M) * 4 + (size_t)R * ((E + 31) / 32) * 4;
+  off = (off + 15) & ~(size_t)15;
+  p.rows = reinterpret_cast<float*>(sm + off);
+  return p;
+}
+
+// Computes the routing and the grouped work plan of a decode step in one
+// CTA (every thread of the CTA calls it; it synchronises the CTA):
+//   1. routes the M tokens (or takes the given routing) and the
+//      shared-expert gate;
+//   2. sorts the M*K (token, slot) pairs by expert (stable);
+//   3. lists one gate/up segment and one down segment per distinct expert,
+//      then the shared expert's segments, with the (input, output) vector
+//      references of every pair in sorted order.
+// Each output group of `o` is written only if its pointer is non-null.
+__device__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, int R, const PlanSinks& o) {
   const int M = a.M, K = a.K, n = M * K;
-  const int tid = threadIdx.x, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, nthr = blockDim.x;
   const int words = (a.E + 31) >> 5;
-  int32_t* key = reinterpret_cast<int32_t*>(sm);      // [n] expert of pair
-  int32_t* sorted = key + n;                          // [n] pairs sorted by (expert, pair)
-  int32_t* head = sorted + n;                         // [n] 1 at the first pair of an expert
-  int32_t* entry_of = head + n;                       // [n] entry index of sorted position
-  uint32_t* taken = reinterpret_cast<uint32_t*>(entry_of + n);  // [nwarps][words]
+  const PlanScratch ps = plan_scratch(sm, M, K, a.E, R);
 
   // 1. routing: R warps, each with its token's logits staged in shared memory
   if (a.logits) {
-    const int R = plan_route_warps(M, a.E, nwarps);
-    float* rows = reinterpret_cast<float*>(taken + nwarps * words);  // [R][E]
     if (warp < R)
       for (int t = warp; t < M; t += R) {
-        float* row = rows + (int64_t)warp * a.E;
+        float* row = ps.rows + (int64_t)warp * a.E;
         stage_logits_warp(a.logits + (int64_t)t * a.E, row, a.E);
-        route_token_warp(row, a.E, K, a.renorm, a.router_scale, a.idx_out + (int64_t)t * K,
-                         a.w_out + (int64_t)t * K, taken + warp * words);
+        route_token_warp(row, a.E, K, a.renorm, a.router_scale, ps.sidx + t * K, ps.sw + t * K,
+                         ps.taken + warp * words);
       }
   } else {
-    for (int p = tid; p < n; p += blockDim.x) {
-      a.idx_out[p] = a.idx_in[p];
-      a.w_out[p] = a.w_in[p];
+    for (int p = tid; p < n; p += nthr) {
+      ps.sidx[p] = a.idx_in[p];
+      ps.sw[p] = a.w_in[p];
     }
   }
   if (a.has_shared && a.sg_logit)
-    for (int t = tid; t < M; t += blockDim.x) a.sigma[t] = 1.0f / (1.0f + expf(-a.sg_logit[t]));
+    for (int t = tid; t < M; t += nthr) ps.ssig[t] = 1.0f / (1.0f + expf(-a.sg_logit[t]));
   __syncthreads();
 
-  // 2. stable sort of pairs by expert: rank of key (expert * n + pair)
-  for (int p = tid; p < n; p += blockDim.x) {
-    int e = a.idx_out[p];
+  // routing results out; stable sort of pairs by expert (rank of expert * n + pair)
+  for (int p = tid; p < n; p += nthr) {
+    int e = ps.sidx[p];
+    if (o.idx) {
+      o.idx[p] = e;
+      o.w[p] = ps.sw[p];
+    }
     if (e < 0 || e >= a.E) {
       set_status(a.status, MOEQ_ERR_INVALID_ARG);
       e = 0;
     }
-    key[p] = e;
+    ps.key[p] = e;
   }
+  if (o.sigma && a.has_shared && a.sg_logit)
+    for (int t = tid; t < M; t += nthr) o.sigma[t] = ps.ssig[t];
+  for (int i = tid; i < o.n_ctr; i += nthr) o.ctr[i] = 0;
   __syncthreads();
-  for (int p = tid; p < n; p += blockDim.x) {
-    const int e = key[p];
+  for (int p = tid; p < n; p += nthr) {
+    const int e = ps.key[p];
     int rank = 0;
     for (int q = 0; q < n; ++q) {
-      const int f = key[q];
+      const int f = ps.key[q];
       rank += (f < e) || (f == e && q < p);
     }
-    sorted[rank] = p;
+    ps.sorted[rank] = p;
   }
   __syncthreads();
-  for (int i = tid; i < n; i += blockDim.x)
-    head[i] = (i == 0) || (key[sorted[i]] != key[sorted[i - 1]]);
+  for (int i = tid; i < n; i += nthr)
+    ps.head[i] = (i == 0) || (ps.key[ps.sorted[i]] != ps.key[ps.sorted[i - 1]]);
   __syncthreads();
-  // entry index = inclusive prefix count of heads - 1 (serial scan by warp 0; n <= 2048)
+  // entry index = inclusive prefix count of heads - 1 (scan by warp 0)
   if (warp == 0) {
     int run = 0;
     for (int base = 0; base < n; base += 32) {
       const int i = base + (tid & 31);
-      int h = (i < n) ? head[i] : 0;
+      int h = (i < n) ? ps.head[i] : 0;
       int incl = h;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if ((tid & 31) >= o) incl += y;
+      for (int s = 1; s < 32; s <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, s);
+        if ((tid & 31) >= s) incl += y;
       }
-      if (i < n) entry_of[i] = run + incl - 1;
+      if (i < n) ps.entry_of[i] = run + incl - 1;
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
   __syncthreads();
-  const int n_entries = n > 0 ? entry_of[n - 1] + 1 : 0;
-
-  // the selected experts' weights are known now: start pulling them into L2
-  // so the gate/up and down GEMVs read them from there
-  if (a.prefetch) {
-    int32_t* ent = taken_list(sm, n, a.E, nwarps);
-    for (int i = tid; i < n; i += blockDim.x)
-      if (head[i]) ent[entry_of[i]] = key[sorted[i]];
-    __syncthreads();
-    const moeq_qtensor* ts[3] = {&a.gate, &a.up, &a.down};
-    constexpr int64_t PIECE = 32 * 1024;
-    // per expert: 3 tensors x (codes, scales, biases)
-    int64_t sizes[9];
-    for (int k = 0; k < 3; ++k) {
-      const moeq_qtensor& t = *ts[k];
-      const int64_t groups = (int64_t)t.out_dim * (t.in_dim / t.group_size);
-      sizes[3 * k] = (int64_t)t.out_dim * t.in_dim * t.bits / 8;
-      sizes[3 * k + 1] = groups * 2;
-      sizes[3 * k + 2] = groups * 2;
-    }
-    int64_t per_expert = 0;
-    for (int k = 0; k < 9; ++k) per_expert += (sizes[k] + PIECE - 1) / PIECE;
-    for (int64_t q = tid; q < (int64_t)n_entries * per_expert; q += blockDim.x) {
-      const int u = (int)(q / per_expert);
-      int64_t r = q % per_expert;
-      int k = 0;
-      while (r >= (sizes[k] + PIECE - 1) / PIECE) {
-        r -= (sizes[k] + PIECE - 1) / PIECE;
-        ++k;
-      }
-      const moeq_qtensor& t = *ts[k / 3];
-      const int e = ent[u];
-      const uint8_t* base =
-          (k % 3 == 0) ? (const uint8_t*)(t.w + (int64_t)e * t.expert_stride_w)
-          : (k % 3 == 1) ? (const uint8_t*)(t.scales + (int64_t)e * t.expert_stride_sb)
-                         : (const uint8_t*)(t.biases + (int64_t)e * t.expert_stride_sb);
-      const int64_t off = r * PIECE;
-      const int64_t len = min(PIECE, sizes[k] - off) & ~(int64_t)15;
-      if (((uintptr_t)base & 15) == 0 && len > 0) tc::prefetch_l2(base + off, (uint32_t)len);
-    }
-  }
+  const int n_entries = n > 0 ? ps.entry_of[n - 1] + 1 : 0;
 
   // 3. vector lists and segments, one per distinct expert
-  for (int i = tid; i < n; i += blockDim.x) {
-    const int p = sorted[i];
+  for (int i = tid; i < n; i += nthr) {
+    const int p = ps.sorted[i];
     const int t = p / K;
-    a.vecs_gu[i].src = a.x + (int64_t)t * a.H;
-    a.vecs_gu[i].dst = a.h + (int64_t)p * a.I;
-    a.vecs_dn[i].src = a.h + (int64_t)p * a.I;
-    a.vecs_dn[i].dst = a.d + (int64_t)p * a.H;
-    if (head[i]) {
-      const int u = entry_of[i];
-      const int e = key[p];
+    if (o.vecs_gu) {
+      o.vecs_gu[i].src = a.x + (int64_t)t * a.H;
+      o.vecs_gu[i].dst = a.h + (int64_t)p * a.I;
+    }
+    if (o.vecs_dn) {
+      o.vecs_dn[i].src = a.h + (int64_t)p * a.I;
+      o.vecs_dn[i].dst = a.d + (int64_t)p * a.H;
+    }
+    if (ps.head[i]) {
+      const int u = ps.entry_of[i];
+      const int e = ps.key[p];
       int cnt = 1;
-      while (i + cnt < n && !head[i + cnt]) ++cnt;
-      Seg g;
-      g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
-      g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
-      g.b[0] = a.gate.biases + (int64_t)e * a.gate.expert_stride_sb;
-      g.w[1] = a.up.w + (int64_t)e * a.up.expert_stride_w;
-      g.s[1] = a.up.scales + (int64_t)e * a.up.expert_stride_sb;
-      g.b[1] = a.up.biases + (int64_t)e * a.up.expert_stride_sb;
-      g.out_dim = a.I;
-      g.in_dim = a.H;
-      g.G = a.gate.group_size;
-      g.bits = a.gate.bits;
-      g.n_vec = cnt;
-      g.unit_begin = u * a.units_per_seg_gu;
-      g.vec_mode = 1;
-      g.src_base = nullptr;
-      g.src_stride = 0;
-      g.dst_base = nullptr;
-      g.dst_stride = 0;
-      g.vecs = a.vecs_gu + i;
-      a.segs_gu[u] = g;
-      Seg dn;
-      dn.w[0] = dn.w[1] = a.down.w + (int64_t)e * a.down.expert_stride_w;
-      dn.s[0] = dn.s[1] = a.down.scales + (int64_t)e * a.down.expert_stride_sb;
-      dn.b[0] = dn.b[1] = a.down.biases + (int64_t)e * a.down.expert_stride_sb;
-      dn.out_dim = a.H;
-      dn.in_dim = a.I;
-      dn.G = a.down.group_size;
-      dn.bits = a.down.bits;
-      dn.n_vec = cnt;
-      dn.unit_begin = u * a.units_per_seg_dn;
-      dn.vec_mode = 1;
-      dn.src_base = nullptr;
-      dn.src_stride = 0;
-      dn.dst_base = nullptr;
-      dn.dst_stride = 0;
-      dn.vecs = a.vecs_dn + i;
-      a.segs_dn[u] = dn;
+      while (i + cnt < n && !ps.head[i + cnt]) ++cnt;
+      if (o.experts) o.experts[u] = e;
+      if (o.segs_gu) {
+        Seg g;
+        g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
+        g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
+        g.b[0] = a.gate.biases + (int64_t)e * a.gate.expert_stride_sb;
+        g.w[1] = a.up.w + (int64_t)e * a.up.expert_stride_w;
+        g.s[1] = a.up.scales + (int64_t)e * a.up.expert_stride_sb;
+        g.b[1] = a.up.biases + (int64_t)e * a.up.expert_stride_sb;
+        g.out_dim = a.I;
+        g.in_dim = a.H;
+        g.G = a.gate.group_size;
+        g.bits = a.gate.bits;
+        g.n_vec = cnt;
+        g.unit_begin = u * a.units_per_seg_gu;
+        g.vec_mode = 1;
+        g.src_base = nullptr;
+        g.src_stride = 0;
+        g.dst_base = nullptr;
+        g.dst_stride = 0;
+        g.vecs = o.vecs_gu + i;
+        o.segs_gu[u] = g;
+      }
+      if (o.segs_dn) {
+        Seg dn;
+        dn.w[0] = dn.w[1] = a.down.w + (int64_t)e * a.down.expert_stride_w;
+        dn.s[0] = dn.s[1] = a.down.scales + (int64_t)e * a.down.expert_stride_sb;
+        dn.b[0] = dn.b[1] = a.down.biases + (int64_t)e * a.down.expert_stride_sb;
+        dn.out_dim = a.H;
+        dn.in_dim = a.I;
+        dn.G = a.down.group_size;
+        dn.bits = a.down.bits;
+        dn.n_vec = cnt;
+        dn.unit_begin = u * a.units_per_seg_dn;
+        dn.vec_mode = 1;
+        dn.src_base = nullptr;
+        dn.src_stride = 0;
+        dn.dst_base = nullptr;
+        dn.dst_stride = 0;
+        dn.vecs = o.vecs_dn + i;
+        o.segs_dn[u] = dn;
+      }
     }
   }
   if (tid == 0) {
@@ -661,49 +802,53 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
     int units_gu = n_entries * a.units_per_seg_gu, units_dn = n_entries * a.units_per_seg_dn;
     int sep_gu[2] = {0, 0}, sep_dn[2] = {0, 0};
     if (a.has_shared) {
-      // the shared expert: all M tokens, strided rows after the M*K pair rows
-      Seg g;
-      g.w[0] = a.sh_gate.w;
-      g.s[0] = a.sh_gate.scales;
-      g.b[0] = a.sh_gate.biases;
-      g.w[1] = a.sh_up.w;
-      g.s[1] = a.sh_up.scales;
-      g.b[1] = a.sh_up.biases;
-      g.out_dim = a.sh_gate.out_dim;
-      g.in_dim = a.H;
-      g.G = a.sh_gate.group_size;
-      g.bits = a.sh_gate.bits;
-      g.n_vec = M;
-      g.vec_mode = 0;
-      g.src_base = a.x;
-      g.src_stride = a.H;
-      g.dst_base = a.h + (int64_t)n * a.I;
-      g.dst_stride = a.sh_gate.out_dim;
-      g.vecs = nullptr;
-      Seg dn;
-      dn.w[0] = dn.w[1] = a.sh_down.w;
-      dn.s[0] = dn.s[1] = a.sh_down.scales;
-      dn.b[0] = dn.b[1] = a.sh_down.biases;
-      dn.out_dim = a.H;
-      dn.in_dim = a.sh_down.in_dim;
-      dn.G = a.sh_down.group_size;
-      dn.bits = a.sh_down.bits;
-      dn.n_vec = M;
-      dn.vec_mode = 0;
-      dn.src_base = a.h + (int64_t)n * a.I;
-      dn.src_stride = a.sh_gate.out_dim;
-      dn.dst_base = a.d + (int64_t)n * a.H;
-      dn.dst_stride = a.H;
-      dn.vecs = nullptr;
-      // same bit width as the routed experts: appended to the routed list;
-      // otherwise stored at index n (one past the largest routed list) for a
-      // launch of its own
+      // the shared expert: all M tokens, strided rows after the M*K pair rows;
+      // same format as the routed experts: appended to the routed list;
+      // otherwise stored at index n (one past the largest routed list) for
+      // a launch of its own
       const bool same_gu = a.shared_same_gu != 0;
       const bool same_dn = a.shared_same_dn != 0;
-      g.unit_begin = same_gu ? units_gu : 0;
-      dn.unit_begin = same_dn ? units_dn : 0;
-      a.segs_gu[same_gu ? n_entries : n] = g;
-      a.segs_dn[same_dn ? n_entries : n] = dn;
+      if (o.segs_gu) {
+        Seg g;
+        g.w[0] = a.sh_gate.w;
+        g.s[0] = a.sh_gate.scales;
+        g.b[0] = a.sh_gate.biases;
+        g.w[1] = a.sh_up.w;
+        g.s[1] = a.sh_up.scales;
+        g.b[1] = a.sh_up.biases;
+        g.out_dim = a.sh_gate.out_dim;
+        g.in_dim = a.H;
+        g.G = a.sh_gate.group_size;
+        g.bits = a.sh_gate.bits;
+        g.n_vec = M;
+        g.vec_mode = 0;
+        g.src_base = a.x;
+        g.src_stride = a.H;
+        g.dst_base = a.h + (int64_t)n * a.I;
+        g.dst_stride = a.sh_gate.out_dim;
+        g.vecs = nullptr;
+        g.unit_begin = same_gu ? units_gu : 0;
+        o.segs_gu[same_gu ? n_entries : n] = g;
+      }
+      if (o.segs_dn) {
+        Seg dn;
+        dn.w[0] = dn.w[1] = a.sh_down.w;
+        dn.s[0] = dn.s[1] = a.sh_down.scales;
+        dn.b[0] = dn.b[1] = a.sh_down.biases;
+        dn.out_dim = a.H;
+        dn.in_dim = a.sh_down.in_dim;
+        dn.G = a.sh_down.group_size;
+        dn.bits = a.sh_down.bits;
+        dn.n_vec = M;
+        dn.vec_mode = 0;
+        dn.src_base = a.h + (int64_t)n * a.I;
+        dn.src_stride = a.sh_gate.out_dim;
+        dn.dst_base = a.d + (int64_t)n * a.H;
+        dn.dst_stride = a.H;
+        dn.vecs = nullptr;
+        dn.unit_begin = same_dn ? units_dn : 0;
+        o.segs_dn[same_dn ? n_entries : n] = dn;
+      }
       if (same_gu) {
         nseg_gu += 1;
         units_gu += a.units_per_seg_gu_sh;
@@ -719,29 +864,65 @@ __global__ void __launch_bounds__(1024) k_decode_plan(const __grid_constant__ De
         sep_dn[1] = a.units_per_seg_dn_sh;
       }
     }
-    a.count_gu[0] = nseg_gu;
-    a.count_gu[1] = units_gu;
-    a.count_gu[2] = sep_gu[0];
-    a.count_gu[3] = sep_gu[1];
-    a.count_dn[0] = nseg_dn;
-    a.count_dn[1] = units_dn;
-    a.count_dn[2] = sep_dn[0];
-    a.count_dn[3] = sep_dn[1];
+    if (o.count_gu) {
+      o.count_gu[0] = nseg_gu;
+      o.count_gu[1] = units_gu;
+      o.count_gu[2] = sep_gu[0];
+      o.count_gu[3] = sep_gu[1];
+    }
+    if (o.count_dn) {
+      o.count_dn[0] = nseg_dn;
+      o.count_dn[1] = units_dn;
+      o.count_dn[2] = sep_dn[0];
+      o.count_dn[3] = sep_dn[1];
+    }
+    if (o.n_experts) *o.n_experts = n_entries;
   }
+  __syncthreads();
+}
+
+// The plan as a kernel of its own (one CTA), writing every list to global
+// memory for the GEMV launches that follow.
+constexpr int kPlanThreads = 256;
+__global__ void __launch_bounds__(kPlanThreads) k_decode_plan(const __grid_constant__ DecodePlanArgs a) {
+  extern __shared__ __align__(16) uint8_t psm[];
+  tc::grid_dep_wait();
+  tc::grid_dep_launch();
+  PlanSinks o;
+  memset(&o, 0, sizeof(o));
+  o.idx = a.idx_out;
+  o.w = a.w_out;
+  o.sigma = a.sigma;
+  o.segs_gu = a.segs_gu;
+  o.count_gu = a.count_gu;
+  o.vecs_gu = a.vecs_gu;
+  o.segs_dn = a.segs_dn;
+  o.count_dn = a.count_dn;
+  o.vecs_dn = a.vecs_dn;
+  o.ctr = a.ctr;
+  o.n_ctr = a.n_ctr;
+  plan_cta(a, psm, plan_route_warps(a.M, a.E, kPlanThreads / 32), o);
 }
 
 cudaError_t launch_decode_plan(const DecodePlanArgs& a, cudaStream_t st) {
-  const int n = a.M * a.K;
-  const int threads = 1024;
-  size_t smem = (size_t)n * 4 * 5 + (size_t)(threads / 32) * ((a.E + 31) / 32) * 4;
-  if (a.logits) smem += (size_t)plan_route_warps(a.M, a.E, threads / 32) * a.E * 4;
+  const int R = plan_route_warps(a.M, a.E, kPlanThreads / 32);
+  const size_t smem = plan_scratch_bytes(a.M, a.K, a.E, R);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_decode_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  k_decode_plan<<<1, threads, smem, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kPlanThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_decode_plan, a);
 }
 
 // ============================================================== combine

@@ -46,13 +46,16 @@ __global__ void __launch_bounds__(256) k_route_prefill(const float* __restrict__
                                                        float scale, int32_t* __restrict__ idx,
                                                        float* __restrict__ w, int sg_col,
                                                        float* __restrict__ sigma) {
-  extern __shared__ uint32_t taken_all[];
+  extern __shared__ __align__(16) uint8_t rsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int words = (E + 31) >> 5;
+  const int wbytes = ((words * 4 + 15) & ~15) + E * 4;
+  uint32_t* taken = reinterpret_cast<uint32_t*>(rsm + warp * wbytes);
+  float* row = reinterpret_cast<float*>(rsm + warp * wbytes + ((words * 4 + 15) & ~15));
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= M) return;
-  route_token_warp(logits + (int64_t)t * ld, E, K, renorm, scale, idx + (int64_t)t * K,
-                   w + (int64_t)t * K, taken_all + warp * words);
+  stage_logits_warp(logits + (int64_t)t * ld, row, E);
+  route_token_warp(row, E, K, renorm, scale, idx + (int64_t)t * K, w + (int64_t)t * K, taken);
   if (sigma && lane == 0) sigma[t] = 1.0f / (1.0f + expf(-logits[(int64_t)t * ld + sg_col]));
 }
 
@@ -425,8 +428,8 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
 
   // 3. routing
   if (!idx_in) {
-    const int warps = 8;
-    const size_t smem = (size_t)warps * ((E + 31) / 32) * 4;
+    const int warps = route_warps_per_cta(E);
+    const size_t smem = (size_t)warps * ((((E + 31) / 32 * 4 + 15) & ~15) + (size_t)E * 4);
     k_route_prefill<<<(M + warps - 1) / warps, warps * 32, smem, st>>>(
         logits, lay.ld_logits, M, E, K, L->renorm, L->router_scale, idx, wts, E,
         L->has_shared ? sigma : nullptr);

@@ -49,52 +49,6 @@ struct PrefetchRange {
   int64_t bytes;
 };
 
-struct GemvArgs {
-  Seg segs[kInlineSegs];    // used when dyn_segs == nullptr
-  int32_t n_segs;
-  int32_t total_units;      // used when dyn_segs == nullptr
-  const Seg* dyn_segs;      // device list written by the decode plan
-  const int32_t* dyn_count; // [0] = number of segments, [1] = total units
-  // shape shared by every segment of the launch
-  int32_t in_dim;
-  int32_t G;
-  int32_t slices;           // S: 32-chunk slices per row
-  int32_t subsets;          // J: row subsets (warps = S * J)
-  int32_t rows_per_unit;    // RU = J * (8 / NMAT)
-  PrefetchRange pf[kMaxPrefetch];
-  int32_t n_pf;
-  // segments (device list) whose matrix 0 is pulled into L2 at kernel start,
-  // spread over all CTAs (the down projections, from the gate/up launch)
-  const Seg* pf_segs;
-  const int32_t* pf_count;
-  int* status;
-};
-
-enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
-enum GemvSrc { SRC_BF16 = 0, SRC_F32 = 1 };
-
-// Work shape of the staged GEMV for rows of `in_dim` codes at `bits`.
-struct GemvShape {
-  int S;   // slices of 32 chunks per row
-  int J;   // row subsets
-  int RU;  // rows per unit
-};
-GemvShape gemv_shape(int in_dim, int bits, int nmat, int G);
-bool gemv_fits(int in_dim, int bits, int nmat, int G);
-int gemv_units(int out_dim, const GemvShape& sh);
-
-// Launch with programmatic dependent launch (the kernel waits for its
-// predecessor's results before reading them).
-cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,
-                        cudaStream_t st);
-
-// ------------------------------------------------------------------ routing
-cudaError_t launch_route_topk(const float* logits, int M, int E, int K, int renorm, float scale,
-                              int32_t* idx, float* w, cudaStream_t st);
-
-// Decode plan: top-K for M tokens, then the grouped work lists for the
-// gate/up and down GEMVs (one segment per distinct expert, plus the shared
-// expert), written into `plan` (device workspace).
 struct DecodePlanArgs {
   const float* logits;      // [M][E] fp32, or null when idx/w are given
   const float* sg_logit;    // [M] shared-gate logit, or null
@@ -117,15 +71,109 @@ struct DecodePlanArgs {
   int32_t* count_dn;        // [4]
   VecRef* vecs_gu;          // [(M*K + M)]
   VecRef* vecs_dn;
+  int32_t* ctr;             // [n_ctr] per-row-block counters of the fused combine, zeroed
+  int32_t n_ctr;
   int32_t units_per_seg_gu; // computed on the host from the shapes
   int32_t units_per_seg_dn;
   int32_t units_per_seg_gu_sh;
   int32_t units_per_seg_dn_sh;
-  int32_t prefetch;         // 1: pull the selected experts' weights into L2
   int32_t shared_same_gu;   // 1: the shared gate/up segment joins the routed launch
   int32_t shared_same_dn;   // 1: the shared down segment joins the routed launch
   int* status;
 };
+
+// Where a CTA's plan goes (each group written only when its pointer is set).
+struct PlanSinks {
+  int32_t* idx;
+  float* w;
+  float* sigma;
+  Seg* segs_gu;
+  int32_t* count_gu;
+  VecRef* vecs_gu;
+  Seg* segs_dn;
+  int32_t* count_dn;
+  VecRef* vecs_dn;
+  int32_t* ctr;             // set to zero
+  int32_t n_ctr;
+  int32_t* experts;         // [entries] expert of each entry
+  int32_t* n_experts;
+};
+
+// Staged logits of the plan's routing warps: at most this many bytes.
+constexpr int kPlanStageBytes = 64 * 1024;
+// Largest M*K whose plan the gate/up GEMV computes itself (in every CTA).
+constexpr int kFusedMaxPairs = 64;
+__host__ __device__ int plan_route_warps(int M, int E, int nwarps);
+__host__ __device__ size_t plan_scratch_bytes(int M, int K, int E, int R);
+
+// The weighted combine done by the down GEMV: the CTA that completes the
+// last segment of a row block writes y for those rows.
+struct CombineArgs {
+  const float* w;           // [M][K] routed weights
+  const float* sigma;       // [M] shared-expert gate values
+  const float* residual;    // [M][H] or null
+  float* y;                 // [M][H]
+  const float* d;           // [(M*K + M)][H] down rows
+  int32_t* ctr;             // [row blocks], zero on entry
+  int32_t M, K, H, has_shared;
+};
+
+struct GemvArgs {
+  Seg segs[kInlineSegs];    // used when dyn_segs == nullptr
+  int32_t n_segs;
+  int32_t total_units;      // used when dyn_segs == nullptr
+  const Seg* dyn_segs;      // device list written by the decode plan
+  const int32_t* dyn_count; // [0] = number of segments, [1] = total units
+  // shape shared by every segment of the launch
+  int32_t in_dim;
+  int32_t G;
+  int32_t slices;           // S: 32-chunk slices per row
+  int32_t subsets;          // J: row subsets (warps = S * J)
+  int32_t rows_per_unit;    // RU = J * (8 / NMAT)
+  PrefetchRange pf[kMaxPrefetch];
+  int32_t n_pf;
+  // segments (device list) whose matrix 0 is pulled into L2 at kernel start,
+  // spread over all CTAs (the down projections, from the gate/up launch)
+  const Seg* pf_segs;
+  const int32_t* pf_count;
+  int* status;
+  // gate/up launch: every CTA computes the step's plan itself (M*K <= kFusedMaxPairs)
+  int32_t fused_plan;
+  DecodePlanArgs plan;
+  // down launch: weighted combine by the last CTA of each row block
+  int32_t fuse_combine;
+  CombineArgs comb;
+};
+
+enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
+enum GemvSrc { SRC_BF16 = 0, SRC_F32 = 1 };
+
+// Work shape of the staged GEMV for rows of `in_dim` codes at `bits`.
+struct GemvShape {
+  int S;   // slices of 32 chunks per row
+  int J;   // row subsets
+  int RU;  // rows per unit
+};
+GemvShape gemv_shape(int in_dim, int bits, int nmat, int G);
+bool gemv_fits(int in_dim, int bits, int nmat, int G);
+int gemv_threads();     // threads of a GEMV CTA
+int gemv_ring_bytes();  // bytes of its stage ring (also the scratch of a fused plan)
+int gemv_units(int out_dim, const GemvShape& sh);
+
+// Launch with programmatic dependent launch (the kernel waits for its
+// predecessor's results before reading them).
+cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,
+                        cudaStream_t st);
+
+// ------------------------------------------------------------------ routing
+int route_warps_per_cta(int E);  // warps of a routing CTA (staged logits fit 48 KB)
+cudaError_t launch_route_topk(const float* logits, int M, int E, int K, int renorm, float scale,
+                              int32_t* idx, float* w, cudaStream_t st);
+
+// Decode plan: top-K for M tokens, then the grouped work lists for the
+// gate/up and down GEMVs (one segment per distinct expert, plus the shared
+// expert), written into `plan` (device workspace).
+
 cudaError_t launch_decode_plan(const DecodePlanArgs& a, cudaStream_t st);
 
 // Codes and/or fp32 weights of one matrix.

@@ -163,6 +163,12 @@ def test_decode_397b_like():
     run_decode("decode_397b", [1, 8])
 
 
+def test_decode_30b_like_planned_apart():
+    """M*K = 128 pairs: the plan runs as a launch of its own (above the size
+    the gate/up launch plans itself) while the down launch still combines."""
+    run_decode("decode_30b", [16], residual=True)
+
+
 @pytest.mark.slow
 def test_decode_397b_like_batch64():
     run_decode("decode_397b", [64])
