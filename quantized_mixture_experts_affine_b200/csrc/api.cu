@@ -117,14 +117,11 @@ static moeq_status check_layer(const moeq_layer* L) {
   return MOEQ_OK;
 }
 
-// Decode GEMV limits: rows of at most 4096 bytes of codes, an even number
-// of groups per row (4-byte scale/bias copies), 4-byte aligned scale/bias
-// arrays and bank strides, and a work unit that fits one pipeline stage.
+// Decode GEMV limits: rows of at most 4096 bytes of codes and a work unit
+// that fits one pipeline stage.  (Scale/bias rows are bulk-copied when
+// 16-byte aligned and copied entry by entry otherwise.)
 static moeq_status check_gemv_tensor(const moeq_qtensor& t, int nmat) {
   if (slices_of(t) > 8) return MOEQ_ERR_UNSUPPORTED;
-  if ((t.in_dim / t.group_size) % 2) return MOEQ_ERR_UNSUPPORTED;
-  if (((uintptr_t)t.scales & 3) || ((uintptr_t)t.biases & 3) || (t.expert_stride_sb & 1))
-    return MOEQ_ERR_ALIGNMENT;
   if (!gemv_fits(t.in_dim, t.bits, nmat, t.group_size)) return MOEQ_ERR_UNSUPPORTED;
   return MOEQ_OK;
 }

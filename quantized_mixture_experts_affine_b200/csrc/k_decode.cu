@@ -179,7 +179,8 @@ __device__ __forceinline__ void prefetch_down(const DecodePlanArgs& p, const int
   }
 }
 
-__device__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, int R, const PlanSinks& o);
+__device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, int R,
+                                         const PlanSinks& o);
 
 // y[m][r] = sum_k w[m][k] d[m*K + k][r] (+ sigma[m] d[M*K + m][r]) (+ residual[m][r])
 // for rows [r0, r0 + nrows), k in order; the same operations as k_combine.
@@ -239,50 +240,66 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   // ranges known before the preceding kernel ends (the shared expert's
   // weights) go to L2 while it finishes
   if (warp == GV_HELPER && a.n_pf) prefetch_ranges(a.pf, a.n_pf);
+  // fixed segments (router, qmv): no earlier kernel writes them or the
+  // weights, so the producer starts streaming before the preceding kernel
+  // ends; everyone else waits for it (input vectors, segment lists)
+  const bool static_segs = !a.dyn_segs && !a.fused_plan;
+  if (static_segs)
+    for (int i = threadIdx.x; i < a.n_segs; i += blockDim.x) ub[i] = a.segs[i].unit_begin;
   __syncthreads();
-  // segment lists and input vectors may come from the preceding kernel
-  tc::grid_dep_wait();
+  if (!(static_segs && warp == GV_PRODUCER)) tc::grid_dep_wait();
   tc::grid_dep_launch();
 
   const Seg* segs;
   int n_segs, total_units;
   int32_t* pcnt = reinterpret_cast<int32_t*>(gsm + GvSmem::PCNT_OFF);
   int32_t* pexp = reinterpret_cast<int32_t*>(gsm + GvSmem::PEXP_OFF);
-  if (a.fused_plan) {
-    // this CTA's copy of the step's plan, in shared memory; CTA 0 also
-    // writes the routing, the down lists and zeroed combine counters
-    Seg* psegs = reinterpret_cast<Seg*>(gsm + GvSmem::PSEG_OFF);
-    PlanSinks o;
-    memset(&o, 0, sizeof(o));
-    o.segs_gu = psegs;
-    o.count_gu = pcnt;
-    o.vecs_gu = reinterpret_cast<VecRef*>(gsm + GvSmem::PVEC_OFF);
-    o.experts = pexp;
-    o.n_experts = pcnt + 4;
-    if (blockIdx.x == 0) {
-      o.idx = a.plan.idx_out;
-      o.w = a.plan.w_out;
-      o.sigma = a.plan.sigma;
-      o.segs_dn = a.plan.segs_dn;
-      o.count_dn = a.plan.count_dn;
-      o.vecs_dn = a.plan.vecs_dn;
-      o.ctr = a.plan.ctr;
-      o.n_ctr = a.plan.n_ctr;
-    }
-    // the scratch of the plan lives in the (still unused) stage ring
-    plan_cta(a.plan, gsm, plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32), o);
-    segs = psegs;
-    n_segs = pcnt[0];
-    total_units = pcnt[1];
+  if (static_segs) {
+    segs = a.segs;
+    n_segs = a.n_segs;
+    total_units = a.total_units;
   } else {
-    segs = a.dyn_segs ? a.dyn_segs : a.segs;
-    n_segs = a.dyn_segs ? a.dyn_count[0] : a.n_segs;
-    total_units = a.dyn_segs ? a.dyn_count[1] : a.total_units;
+    bool planned = false;
+    if constexpr (NMAT == 2) {
+      if (a.fused_plan) {
+        // this CTA's copy of the step's plan, in shared memory; CTA 0 also
+        // writes the routing, the down lists and zeroed combine counters
+        Seg* psegs = reinterpret_cast<Seg*>(gsm + GvSmem::PSEG_OFF);
+        PlanSinks o;
+        memset(&o, 0, sizeof(o));
+        o.segs_gu = psegs;
+        o.count_gu = pcnt;
+        o.vecs_gu = reinterpret_cast<VecRef*>(gsm + GvSmem::PVEC_OFF);
+        o.experts = pexp;
+        o.n_experts = pcnt + 4;
+        if (blockIdx.x == 0) {
+          o.idx = a.plan.idx_out;
+          o.w = a.plan.w_out;
+          o.sigma = a.plan.sigma;
+          o.segs_dn = a.plan.segs_dn;
+          o.count_dn = a.plan.count_dn;
+          o.vecs_dn = a.plan.vecs_dn;
+          o.ctr = a.plan.ctr;
+          o.n_ctr = a.plan.n_ctr;
+        }
+        // the scratch of the plan lives in the (still unused) stage ring
+        plan_cta(a.plan, gsm, plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32), o);
+        segs = psegs;
+        n_segs = pcnt[0];
+        total_units = pcnt[1];
+        planned = true;
+      }
+    }
+    if (!planned) {
+      segs = a.dyn_segs;
+      n_segs = a.dyn_count[0];
+      total_units = a.dyn_count[1];
+    }
+    if (n_segs <= GV_UB_CAP)
+      for (int i = threadIdx.x; i < n_segs; i += blockDim.x) ub[i] = segs[i].unit_begin;
+    __syncthreads();
   }
   const bool ub_cached = n_segs <= GV_UB_CAP;
-  if (ub_cached)
-    for (int i = threadIdx.x; i < n_segs; i += blockDim.x) ub[i] = segs[i].unit_begin;
-  __syncthreads();
 
   const int row_bytes = a.in_dim * BITS / 8;
   const int gpr = a.in_dim / a.G;
@@ -359,6 +376,14 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         float* udst = shfl_ptr(dst_base, u);
         const int64_t uss = __shfl_sync(0xffffffffu, src_stride, u);
         const int64_t uds = __shfl_sync(0xffffffffu, dst_stride, u);
+        // scale/bias rows of the unit: contiguous runs of unr * gpr entries,
+        // bulk-copied when 16-byte aligned, else copied entry by entry
+        const int sb_n = unr * gpr;
+        bool sb_bulk = ((sb_n * 2) & 15) == 0 && ((codes_bytes | sb_bytes) & 15) == 0;
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m)
+          sb_bulk = sb_bulk && ((((uintptr_t)(usp[m] + (int64_t)ur0 * gpr)) |
+                                 ((uintptr_t)(ubp[m] + (int64_t)ur0 * gpr))) & 15) == 0;
         if (lane == 0) {
           GvMeta* mt = reinterpret_cast<GvMeta*>(gsm + GvSmem::META_OFF + s * GvSmem::META_STRIDE);
           mt->r0 = ur0;
@@ -370,30 +395,47 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
           mt->dst_base = udst;
           mt->dst_stride = uds;
           mt->vecs = uvecs;
-          tc::mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * unr * row_bytes));
+          tc::mbar_arrive_expect_tx(
+              &full[s], (uint32_t)(NMAT * unr * row_bytes + (sb_bulk ? 2 * NMAT * sb_n * 2 : 0)));
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m)
+          for (int m = 0; m < NMAT; ++m) {
             tc::bulk_g2s(st + m * RU * row_bytes,
                          reinterpret_cast<const uint8_t*>(uw[m]) + (int64_t)ur0 * row_bytes,
                          (uint32_t)(unr * row_bytes), &full[s]);
+            if (sb_bulk) {
+              tc::bulk_g2s(st + codes_bytes + m * sb_bytes, usp[m] + (int64_t)ur0 * gpr,
+                           (uint32_t)(sb_n * 2), &full[s]);
+              tc::bulk_g2s(st + codes_bytes + (NMAT + m) * sb_bytes, ubp[m] + (int64_t)ur0 * gpr,
+                           (uint32_t)(sb_n * 2), &full[s]);
+            }
+          }
         }
-        const int pairs = unr * gpr / 2;
+        if (!sb_bulk) {
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-          const uint16_t* s0 = usp[m] + (int64_t)ur0 * gpr;
-          const uint16_t* b0 = ubp[m] + (int64_t)ur0 * gpr;
-          const uint32_t sd = st + codes_bytes + m * sb_bytes;
-          const uint32_t bd = st + codes_bytes + NMAT * sb_bytes + m * sb_bytes;
-          for (int p = lane; p < pairs; p += 32) {
-            tc::cp_async4(sd + 4 * p, s0 + 2 * p, 4);
-            tc::cp_async4(bd + 4 * p, b0 + 2 * p, 4);
+          for (int m = 0; m < NMAT; ++m) {
+            const uint16_t* s0 = usp[m] + (int64_t)ur0 * gpr;
+            const uint16_t* b0 = ubp[m] + (int64_t)ur0 * gpr;
+            uint16_t* sd = reinterpret_cast<uint16_t*>(gsm + s * GV_STAGE_BYTES + codes_bytes +
+                                                       m * sb_bytes);
+            uint16_t* bd = reinterpret_cast<uint16_t*>(gsm + s * GV_STAGE_BYTES + codes_bytes +
+                                                       (NMAT + m) * sb_bytes);
+            for (int e = lane; e < sb_n; e += 32) {
+              sd[e] = s0[e];
+              bd[e] = b0[e];
+            }
           }
         }
         if (uvm == 1 && unv <= GV_VMAX && !__isShared(uvecs)) {
           const uint32_t vd = sbase + GvSmem::VEC_OFF + s * GV_VMAX * 16;
           for (int v = lane; v < unv; v += 32) tc::cp_async16(vd + 16 * v, uvecs + v, 16);
         }
-        tc::cp_async_arrive_noinc(&full[s]);
+        if (sb_bulk) {
+          tc::cp_async_arrive_noinc(&full[s]);
+        } else {
+          // plain shared-memory stores above: released by an ordinary arrive
+          tc::cp_async_wait_all();
+          tc::mbar_arrive(&full[s]);
+        }
       }
     }
   } else {
@@ -409,6 +451,21 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     for (int pb = 0; pb < 2; ++pb) gi[pb] = (ch * VPC + (pb < NB ? pb : 0) * kXBlock) / a.G;
     SliceVec<BITS, NL> sv;
     const void* cur_src = nullptr;
+    // the first vector's slice is built while the first stage streams in
+    if (on_w) {
+      const int u0 = blockIdx.x + grp * gridDim.x;
+      if (u0 < total_units) {
+        const int si = ub_cached ? find_seg(ub, 1, n_segs, u0)
+                                 : find_seg(&segs[0].unit_begin, (int)(sizeof(Seg) / 4), n_segs,
+                                            u0);
+        const Seg& sg = segs[si];
+        if (sg.n_vec > 0) {
+          const void* src0 = sg.vec_mode == 0 ? sg.src_base : sg.vecs[0].src;
+          build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
+          cur_src = src0;
+        }
+      }
+    }
     // After a wait that ran out, every later wait is skipped and no vector
     // is processed; all waits are bounded, so the CTA always ends.
     bool timed_out = false;
@@ -499,15 +556,18 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
               dst[r0 + row] = __fdividef(tot, 1.0f + __expf(-tot)) * u;
           } else {
             const int row = j * RPW + lane;
-            if (sl == 0 && lane < 8 && row < nrows) dst[r0 + row] = tot;
+            if (sl == 0 && lane < 8 && row < nrows) {
+              dst[r0 + row] = tot;
+              // visible GPU-wide before the row block is counted as done
+              if (a.fuse_combine) __threadfence();
+            }
           }
         }
       }
       tc::mbar_arrive(&empty[s]);
-      if (EPI == EPI_PLAIN && a.fuse_combine) {
+      if (NMAT == 1 && EPI == EPI_PLAIN && a.fuse_combine) {
         // the group's stores of this unit are done; the CTA that brings the
         // row block's count to the number of segments sums the block
-        __threadfence();
         tc::named_sync(2 + grp, GV_CW * 32);
         int* flag = reinterpret_cast<int*>(gsm + GvSmem::FLAG_OFF) + grp;
         if (cw == 0 && lane == 0) {
@@ -585,8 +645,8 @@ __global__ void __launch_bounds__(256) k_route_topk(const float* __restrict__ lo
   float* row = reinterpret_cast<float*>(rsm + warp * wbytes + ((words * 4 + 15) & ~15));
   const int t = blockIdx.x * nw + warp;
   if (t >= M) return;
-  stage_logits_warp(logits + (int64_t)t * E, row, E);
-  route_token_warp(row, E, K, renorm, scale, idx + (int64_t)t * K, w + (int64_t)t * K, taken);
+  route_token_warp(logits + (int64_t)t * E, E, K, renorm, scale, idx + (int64_t)t * K,
+                   w + (int64_t)t * K, row, taken);
 }
 
 // Warps per routing CTA so that the staged rows fit 48 KB.
@@ -653,6 +713,68 @@ __device__ __forceinline__ PlanScratch plan_scratch(uint8_t* sm, int M, int K, i
   return p;
 }
 
+// Vector references of the pair at sorted position i (pair p).
+__device__ __forceinline__ void write_pair_lists(const DecodePlanArgs& a, const PlanSinks& o, int i,
+                                                 int p) {
+  const int t = p / a.K;
+  if (o.vecs_gu) {
+    o.vecs_gu[i].src = a.x + (int64_t)t * a.H;
+    o.vecs_gu[i].dst = a.h + (int64_t)p * a.I;
+  }
+  if (o.vecs_dn) {
+    o.vecs_dn[i].src = a.h + (int64_t)p * a.I;
+    o.vecs_dn[i].dst = a.d + (int64_t)p * a.H;
+  }
+}
+
+// Gate/up and down segments of entry u: expert e, its `cnt` pairs starting
+// at sorted position i.
+__device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const PlanSinks& o, int i,
+                                                  int u, int e, int cnt) {
+  if (o.experts) o.experts[u] = e;
+  if (o.segs_gu) {
+    Seg g;
+    g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
+    g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
+    g.b[0] = a.gate.biases + (int64_t)e * a.gate.expert_stride_sb;
+    g.w[1] = a.up.w + (int64_t)e * a.up.expert_stride_w;
+    g.s[1] = a.up.scales + (int64_t)e * a.up.expert_stride_sb;
+    g.b[1] = a.up.biases + (int64_t)e * a.up.expert_stride_sb;
+    g.out_dim = a.I;
+    g.in_dim = a.H;
+    g.G = a.gate.group_size;
+    g.bits = a.gate.bits;
+    g.n_vec = cnt;
+    g.unit_begin = u * a.units_per_seg_gu;
+    g.vec_mode = 1;
+    g.src_base = nullptr;
+    g.src_stride = 0;
+    g.dst_base = nullptr;
+    g.dst_stride = 0;
+    g.vecs = o.vecs_gu + i;
+    o.segs_gu[u] = g;
+  }
+  if (o.segs_dn) {
+    Seg dn;
+    dn.w[0] = dn.w[1] = a.down.w + (int64_t)e * a.down.expert_stride_w;
+    dn.s[0] = dn.s[1] = a.down.scales + (int64_t)e * a.down.expert_stride_sb;
+    dn.b[0] = dn.b[1] = a.down.biases + (int64_t)e * a.down.expert_stride_sb;
+    dn.out_dim = a.H;
+    dn.in_dim = a.I;
+    dn.G = a.down.group_size;
+    dn.bits = a.down.bits;
+    dn.n_vec = cnt;
+    dn.unit_begin = u * a.units_per_seg_dn;
+    dn.vec_mode = 1;
+    dn.src_base = nullptr;
+    dn.src_stride = 0;
+    dn.dst_base = nullptr;
+    dn.dst_stride = 0;
+    dn.vecs = o.vecs_dn + i;
+    o.segs_dn[u] = dn;
+  }
+}
+
 // Computes the routing and the grouped work plan of a decode step in one
 // CTA (every thread of the CTA calls it; it synchronises the CTA):
 //   1. routes the M tokens (or takes the given routing) and the
@@ -662,21 +784,20 @@ __device__ __forceinline__ PlanScratch plan_scratch(uint8_t* sm, int M, int K, i
 //      then the shared expert's segments, with the (input, output) vector
 //      references of every pair in sorted order.
 // Each output group of `o` is written only if its pointer is non-null.
-__device__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, int R, const PlanSinks& o) {
+__device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, int R,
+                                         const PlanSinks& o) {
   const int M = a.M, K = a.K, n = M * K;
   const int tid = threadIdx.x, warp = tid >> 5, nthr = blockDim.x;
   const int words = (a.E + 31) >> 5;
   const PlanScratch ps = plan_scratch(sm, M, K, a.E, R);
 
-  // 1. routing: R warps, each with its token's logits staged in shared memory
+  // 1. routing: R warps, one token each at a time
   if (a.logits) {
     if (warp < R)
-      for (int t = warp; t < M; t += R) {
-        float* row = ps.rows + (int64_t)warp * a.E;
-        stage_logits_warp(a.logits + (int64_t)t * a.E, row, a.E);
-        route_token_warp(row, a.E, K, a.renorm, a.router_scale, ps.sidx + t * K, ps.sw + t * K,
+      for (int t = warp; t < M; t += R)
+        route_token_warp(a.logits + (int64_t)t * a.E, a.E, K, a.renorm, a.router_scale,
+                         ps.sidx + t * K, ps.sw + t * K, ps.rows + (int64_t)warp * a.E,
                          ps.taken + warp * words);
-      }
   } else {
     for (int p = tid; p < n; p += nthr) {
       ps.sidx[p] = a.idx_in[p];
@@ -686,114 +807,99 @@ __device__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, int R, const Plan
   if (a.has_shared && a.sg_logit)
     for (int t = tid; t < M; t += nthr) ps.ssig[t] = 1.0f / (1.0f + expf(-a.sg_logit[t]));
   __syncthreads();
-
-  // routing results out; stable sort of pairs by expert (rank of expert * n + pair)
-  for (int p = tid; p < n; p += nthr) {
-    int e = ps.sidx[p];
-    if (o.idx) {
-      o.idx[p] = e;
-      o.w[p] = ps.sw[p];
-    }
-    if (e < 0 || e >= a.E) {
-      set_status(a.status, MOEQ_ERR_INVALID_ARG);
-      e = 0;
-    }
-    ps.key[p] = e;
-  }
   if (o.sigma && a.has_shared && a.sg_logit)
     for (int t = tid; t < M; t += nthr) o.sigma[t] = ps.ssig[t];
   for (int i = tid; i < o.n_ctr; i += nthr) o.ctr[i] = 0;
-  __syncthreads();
-  for (int p = tid; p < n; p += nthr) {
-    const int e = ps.key[p];
-    int rank = 0;
-    for (int q = 0; q < n; ++q) {
-      const int f = ps.key[q];
-      rank += (f < e) || (f == e && q < p);
-    }
-    ps.sorted[rank] = p;
-  }
-  __syncthreads();
-  for (int i = tid; i < n; i += nthr)
-    ps.head[i] = (i == 0) || (ps.key[ps.sorted[i]] != ps.key[ps.sorted[i - 1]]);
-  __syncthreads();
-  // entry index = inclusive prefix count of heads - 1 (scan by warp 0)
-  if (warp == 0) {
-    int run = 0;
-    for (int base = 0; base < n; base += 32) {
-      const int i = base + (tid & 31);
-      int h = (i < n) ? ps.head[i] : 0;
-      int incl = h;
-#pragma unroll
-      for (int s = 1; s < 32; s <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, s);
-        if ((tid & 31) >= s) incl += y;
-      }
-      if (i < n) ps.entry_of[i] = run + incl - 1;
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-  }
-  __syncthreads();
-  const int n_entries = n > 0 ? ps.entry_of[n - 1] + 1 : 0;
 
-  // 3. vector lists and segments, one per distinct expert
-  for (int i = tid; i < n; i += nthr) {
-    const int p = ps.sorted[i];
-    const int t = p / K;
-    if (o.vecs_gu) {
-      o.vecs_gu[i].src = a.x + (int64_t)t * a.H;
-      o.vecs_gu[i].dst = a.h + (int64_t)p * a.I;
-    }
-    if (o.vecs_dn) {
-      o.vecs_dn[i].src = a.h + (int64_t)p * a.I;
-      o.vecs_dn[i].dst = a.d + (int64_t)p * a.H;
-    }
-    if (ps.head[i]) {
-      const int u = ps.entry_of[i];
-      const int e = ps.key[p];
-      int cnt = 1;
-      while (i + cnt < n && !ps.head[i + cnt]) ++cnt;
-      if (o.experts) o.experts[u] = e;
-      if (o.segs_gu) {
-        Seg g;
-        g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
-        g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
-        g.b[0] = a.gate.biases + (int64_t)e * a.gate.expert_stride_sb;
-        g.w[1] = a.up.w + (int64_t)e * a.up.expert_stride_w;
-        g.s[1] = a.up.scales + (int64_t)e * a.up.expert_stride_sb;
-        g.b[1] = a.up.biases + (int64_t)e * a.up.expert_stride_sb;
-        g.out_dim = a.I;
-        g.in_dim = a.H;
-        g.G = a.gate.group_size;
-        g.bits = a.gate.bits;
-        g.n_vec = cnt;
-        g.unit_begin = u * a.units_per_seg_gu;
-        g.vec_mode = 1;
-        g.src_base = nullptr;
-        g.src_stride = 0;
-        g.dst_base = nullptr;
-        g.dst_stride = 0;
-        g.vecs = o.vecs_gu + i;
-        o.segs_gu[u] = g;
+  // 2.-3. (the entry count is known to thread 0 afterwards)
+  int n_entries = 0;
+  if (n <= 32) {
+    // warp 0 alone: rank of (expert, pair) by shuffles, runs of equal
+    // experts by a ballot of their first positions
+    if (warp == 0) {
+      const int lane = tid;
+      int e = lane < n ? ps.sidx[lane] : 0;
+      if (lane < n && o.idx) {
+        o.idx[lane] = e;
+        o.w[lane] = ps.sw[lane];
       }
-      if (o.segs_dn) {
-        Seg dn;
-        dn.w[0] = dn.w[1] = a.down.w + (int64_t)e * a.down.expert_stride_w;
-        dn.s[0] = dn.s[1] = a.down.scales + (int64_t)e * a.down.expert_stride_sb;
-        dn.b[0] = dn.b[1] = a.down.biases + (int64_t)e * a.down.expert_stride_sb;
-        dn.out_dim = a.H;
-        dn.in_dim = a.I;
-        dn.G = a.down.group_size;
-        dn.bits = a.down.bits;
-        dn.n_vec = cnt;
-        dn.unit_begin = u * a.units_per_seg_dn;
-        dn.vec_mode = 1;
-        dn.src_base = nullptr;
-        dn.src_stride = 0;
-        dn.dst_base = nullptr;
-        dn.dst_stride = 0;
-        dn.vecs = o.vecs_dn + i;
-        o.segs_dn[u] = dn;
+      if (lane < n && (e < 0 || e >= a.E)) {
+        set_status(a.status, MOEQ_ERR_INVALID_ARG);
+        e = 0;
+      }
+      int rank = 0;
+      for (int q = 0; q < n; ++q) {
+        const int eq = __shfl_sync(0xffffffffu, e, q);
+        rank += (eq < e) || (eq == e && q < lane);
+      }
+      if (lane < n) ps.sorted[rank] = lane;
+      __syncwarp();
+      const int sp = lane < n ? ps.sorted[lane] : 0;  // pair at sorted position `lane`
+      const int se = __shfl_sync(0xffffffffu, e, sp);
+      const int prev = __shfl_up_sync(0xffffffffu, se, 1);
+      const bool head = lane < n && (lane == 0 || se != prev);
+      const uint32_t hb = __ballot_sync(0xffffffffu, head);
+      const uint32_t upto = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
+      const uint32_t later = hb & ~upto;
+      if (lane < n) write_pair_lists(a, o, lane, sp);
+      if (head)
+        write_expert_segs(a, o, lane, __popc(hb & upto) - 1, se,
+                          (later ? __ffs(later) - 1 : n) - lane);
+      n_entries = __popc(hb);
+    }
+  } else {
+    // stable sort of pairs by expert: rank of (expert, pair)
+    for (int p = tid; p < n; p += nthr) {
+      int e = ps.sidx[p];
+      if (o.idx) {
+        o.idx[p] = e;
+        o.w[p] = ps.sw[p];
+      }
+      if (e < 0 || e >= a.E) {
+        set_status(a.status, MOEQ_ERR_INVALID_ARG);
+        e = 0;
+      }
+      ps.key[p] = e;
+    }
+    __syncthreads();
+    for (int p = tid; p < n; p += nthr) {
+      const int e = ps.key[p];
+      int rank = 0;
+      for (int q = 0; q < n; ++q) {
+        const int f = ps.key[q];
+        rank += (f < e) || (f == e && q < p);
+      }
+      ps.sorted[rank] = p;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += nthr)
+      ps.head[i] = (i == 0) || (ps.key[ps.sorted[i]] != ps.key[ps.sorted[i - 1]]);
+    __syncthreads();
+    // entry index = inclusive prefix count of heads - 1 (scan by warp 0)
+    if (warp == 0) {
+      int run = 0;
+      for (int base = 0; base < n; base += 32) {
+        const int i = base + (tid & 31);
+        int h = (i < n) ? ps.head[i] : 0;
+        int incl = h;
+#pragma unroll
+        for (int sft = 1; sft < 32; sft <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, sft);
+          if ((tid & 31) >= sft) incl += y;
+        }
+        if (i < n) ps.entry_of[i] = run + incl - 1;
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    __syncthreads();
+    n_entries = n > 0 ? ps.entry_of[n - 1] + 1 : 0;
+    for (int i = tid; i < n; i += nthr) {
+      const int p = ps.sorted[i];
+      write_pair_lists(a, o, i, p);
+      if (ps.head[i]) {
+        int cnt = 1;
+        while (i + cnt < n && !ps.head[i + cnt]) ++cnt;
+        write_expert_segs(a, o, i, ps.entry_of[i], ps.key[p], cnt);
       }
     }
   }

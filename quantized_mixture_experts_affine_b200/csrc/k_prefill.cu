@@ -54,8 +54,8 @@ __global__ void __launch_bounds__(256) k_route_prefill(const float* __restrict__
   float* row = reinterpret_cast<float*>(rsm + warp * wbytes + ((words * 4 + 15) & ~15));
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= M) return;
-  stage_logits_warp(logits + (int64_t)t * ld, row, E);
-  route_token_warp(row, E, K, renorm, scale, idx + (int64_t)t * K, w + (int64_t)t * K, taken);
+  route_token_warp(logits + (int64_t)t * ld, E, K, renorm, scale, idx + (int64_t)t * K,
+                   w + (int64_t)t * K, row, taken);
   if (sigma && lane == 0) sigma[t] = 1.0f / (1.0f + expf(-logits[(int64_t)t * ld + sg_col]));
 }
 

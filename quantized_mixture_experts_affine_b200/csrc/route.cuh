@@ -6,66 +6,140 @@
 
 namespace moeq {
 
-// One warp routes one token: the K largest of p = softmax(scale * logits)
-// (ties to the lower index), listed by p descending; w = p_k (/ sum of the
-// chosen p when renorm).  `taken` is a per-warp bitmap of E bits in shared
-// memory.
-__device__ __forceinline__ void route_token_warp(const float* lg, int E, int K, int renorm, float scale,
-                                 int32_t* idx, float* w, uint32_t* taken) {
+constexpr int kNoExpert = 0x7fffffff;
+
+// Order-preserving 32-bit key of a logit for the selection: a larger value
+// has a larger key, -0 and +0 share one key, and every NaN maps to 0
+// (below -inf).
+__device__ __forceinline__ uint32_t route_key(float v) {
+  if (v != v) return 0u;
+  const uint32_t b = v == 0.0f ? 0u : __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Register path (E <= 32 * NJ): lane l holds the scaled logits of experts
+// l, l + 32, ...  Each of the K passes takes the warp's largest key with
+// one max-reduction and the lowest expert index holding it with one
+// min-reduction; only the lane that owned the winner rescans its values.
+template <int NJ>
+__device__ __forceinline__ void route_token_regs(const float* __restrict__ lg, int E, int K,
+                                                 int renorm, float scale, int32_t* idx, float* w) {
   const int lane = threadIdx.x & 31;
-  const int words = (E + 31) >> 5;
-  for (int i = lane; i < words; i += 32) taken[i] = 0u;
-  __syncwarp();
-  float psel[kMaxK];
-  float mx = -INFINITY;
-  float chosen_sum = 0.0f;
-  for (int k = 0; k < K; ++k) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) {
-      if (taken[e >> 5] & (1u << (e & 31))) continue;
-      const float v = scale * lg[e];
-      // the first untaken expert is always a candidate (so a choice exists
-      // even when every remaining scaled logit is -inf or NaN)
-      if (v > bv || (v == bv && e < bi) || bi == 0x7fffffff) {
-        bv = v;
-        bi = e;
-      }
-    }
+  float v[NJ];
+  uint32_t key[NJ];
+  uint32_t avail = 0;  // bit j: expert lane + 32 j exists and is not taken
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (ov > bv || (ov == bv && oi < bi) || bi == 0x7fffffff)) {
-        bv = ov;
-        bi = oi;
-      }
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = e < E ? scale * lg[e] : 0.0f;
+    key[j] = route_key(v[j]);
+    if (e < E) avail |= 1u << j;
+  }
+  uint32_t lk = 0;
+  int li = kNoExpert;
+  float lv = 0.0f;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j)
+    if (((avail >> j) & 1u) && (li == kNoExpert || key[j] > lk)) {
+      lk = key[j];
+      li = lane + 32 * j;
+      lv = v[j];
     }
+  float mx = 0.0f, chosen_sum = 0.0f, my_p = 0.0f;
+  int my_i = 0;
+  for (int k = 0; k < K; ++k) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, lk);
+    const uint32_t win = __reduce_min_sync(
+        0xffffffffu, (li != kNoExpert && lk == m) ? (uint32_t)li : 0xffffffffu);
+    const int wl = (int)(win & 31u);
+    const float bv = __shfl_sync(0xffffffffu, lv, wl);
     if (k == 0) mx = bv;
-    if (lane == 0) {
-      taken[bi >> 5] |= 1u << (bi & 31);
-      idx[k] = bi;
+    if (wl == lane && win != 0xffffffffu) {
+      avail &= ~(1u << (win >> 5));
+      lk = 0;
+      li = kNoExpert;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j)
+        if (((avail >> j) & 1u) && (li == kNoExpert || key[j] > lk)) {
+          lk = key[j];
+          li = lane + 32 * j;
+          lv = v[j];
+        }
     }
-    __syncwarp();
     const float p = expf(bv - mx);
-    if (lane == 0 && k < kMaxK) psel[k] = p;
+    if (lane == k) {
+      my_p = p;
+      my_i = (int)win;
+    }
     chosen_sum += p;
   }
   // softmax normaliser over all experts
   float z = 0.0f;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j)
+    if (lane + 32 * j < E) z += expf(v[j] - mx);
+  z = warp_sum(z);
+  const float denom = renorm ? chosen_sum : z;
+  if (lane < K) {
+    idx[lane] = my_i;
+    w[lane] = my_p / denom;
+  }
+  __syncwarp();
+}
+
+// Loop path for large E: logits in (shared) memory, `taken` a per-warp
+// bitmap of E bits in shared memory.
+__device__ __forceinline__ void route_token_loop(const float* lg, int E, int K, int renorm,
+                                                 float scale, int32_t* idx, float* w,
+                                                 uint32_t* taken) {
+  const int lane = threadIdx.x & 31;
+  const int words = (E + 31) >> 5;
+  for (int i = lane; i < words; i += 32) taken[i] = 0u;
+  __syncwarp();
+  float mx = -INFINITY, chosen_sum = 0.0f, my_p = 0.0f;
+  int my_i = 0;
+  for (int k = 0; k < K; ++k) {
+    float bv = -INFINITY;
+    int bi = kNoExpert;
+    uint32_t bk = 0;
+    for (int e = lane; e < E; e += 32) {
+      if (taken[e >> 5] & (1u << (e & 31))) continue;
+      const float v = scale * lg[e];
+      const uint32_t ke = route_key(v);
+      if (bi == kNoExpert || ke > bk) {
+        bk = ke;
+        bv = v;
+        bi = e;
+      }
+    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t win = __reduce_min_sync(
+        0xffffffffu, (bi != kNoExpert && bk == m) ? (uint32_t)bi : 0xffffffffu);
+    bv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
+    bi = win == 0xffffffffu ? kNoExpert : (int)win;
+    if (k == 0) mx = bv;
+    if (lane == 0 && bi != kNoExpert) taken[bi >> 5] |= 1u << (bi & 31);
+    __syncwarp();
+    const float p = expf(bv - mx);
+    if (lane == k) {
+      my_p = p;
+      my_i = bi;
+    }
+    chosen_sum += p;
+  }
+  float z = 0.0f;
   for (int e = lane; e < E; e += 32) z += expf(scale * lg[e] - mx);
   z = warp_sum(z);
-  if (lane == 0) {
-    const float denom = renorm ? chosen_sum : z;
-    for (int k = 0; k < K; ++k) w[k] = psel[k] / denom;
+  const float denom = renorm ? chosen_sum : z;
+  if (lane < K) {
+    idx[lane] = my_i;
+    w[lane] = my_p / denom;
   }
   __syncwarp();
 }
 
 // Copies the E logits of one token into the warp's shared-memory row with
-// independent (unrolled, 16-byte where aligned) loads, so the K selection
-// passes of route_token_warp read shared memory instead of issuing one
-// dependent global load per pass and lane.
+// independent (unrolled, 16-byte where aligned) loads.
 __device__ __forceinline__ void stage_logits_warp(const float* __restrict__ lg, float* row, int E) {
   const int lane = threadIdx.x & 31;
   if ((((uintptr_t)lg | (uintptr_t)row) & 15) == 0 && (E & 3) == 0) {
@@ -85,6 +159,27 @@ __device__ __forceinline__ void stage_logits_warp(const float* __restrict__ lg, 
     for (int e = lane; e < E; e += 32) row[e] = lg[e];
   }
   __syncwarp();
+}
+
+// One warp routes one token: the K largest of p = softmax(scale * logits)
+// (ties to the lower index; NaN logits rank below -inf), listed by p
+// descending; w = p_k (/ sum of the
+// chosen p when renorm).  lg: the token's E logits (global memory);
+// row (E floats) and taken ((E+31)/32 words): the warp's shared scratch,
+// used only when E > 1024.
+__device__ __forceinline__ void route_token_warp(const float* lg, int E, int K, int renorm,
+                                                 float scale, int32_t* idx, float* w, float* row,
+                                                 uint32_t* taken) {
+  if (E <= 32) route_token_regs<1>(lg, E, K, renorm, scale, idx, w);
+  else if (E <= 64) route_token_regs<2>(lg, E, K, renorm, scale, idx, w);
+  else if (E <= 128) route_token_regs<4>(lg, E, K, renorm, scale, idx, w);
+  else if (E <= 256) route_token_regs<8>(lg, E, K, renorm, scale, idx, w);
+  else if (E <= 512) route_token_regs<16>(lg, E, K, renorm, scale, idx, w);
+  else if (E <= 1024) route_token_regs<32>(lg, E, K, renorm, scale, idx, w);
+  else {
+    stage_logits_warp(lg, row, E);
+    route_token_loop(row, E, K, renorm, scale, idx, w, taken);
+  }
 }
 
 }  // namespace moeq

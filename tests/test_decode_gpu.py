@@ -70,6 +70,7 @@ QMV_CASES = [  # (bits, G, out, in, M, requant)
     (8, 32, 130, 256, 64, False),    # ragged rows, max decode M
     (4, 128, 96, 768, 7, False),
     (2, 32, 33, 128, 4, False),
+    (4, 64, 40, 192, 3, False),      # 3 groups per row: scale/bias runs not 16-byte multiples
 ]
 
 
@@ -88,6 +89,26 @@ def test_qmv_parity(bits, G, out, inn, M, rq):
         ref = oracle.qmv(host, xb, mat=e)
         assert rel_l2(y.cpu().numpy(), ref) <= 1e-5, rel_l2(y.cpu().numpy(), ref)
     assert moeq.moeq_device_status() == 0
+
+
+def test_qmv_unaligned_scales():
+    """Scale/bias arrays only 2-byte aligned (offset by one entry): the rows
+    are copied entry by entry instead of in bulk; same results."""
+    bits, G, out, inn, M = 4, 64, 96, 512, 2
+    q = synth.tensor_dev(SEED, synth.tag(synth.ROUTER, 77), 1, out, inn, bits, G)
+    n = q.s.numel()
+    s_buf = torch.zeros(n + 8, dtype=q.s.dtype, device="cuda")
+    b_buf = torch.zeros(n + 8, dtype=q.b.dtype, device="cuda")
+    s_buf[1:n + 1].copy_(q.s.reshape(-1))
+    b_buf[1:n + 1].copy_(q.b.reshape(-1))
+    t = moeq.qtensor(q.w, s_buf[1:].data_ptr(), b_buf[1:].data_ptr(), out, inn, bits, G, 1)
+    xb = synth.normal_bf16_host(SEED, synth.tag(synth.X, 6), M * inn).reshape(M, inn)
+    y = torch.full((M, out), float("nan"), device="cuda")
+    moeq.moeq_qmv(t, 0, dev(xb.view(np.int16)), M, y)
+    torch.cuda.synchronize()
+    assert moeq.moeq_device_status() == 0
+    ref = oracle.qmv(q.to_host(), xb, mat=0)
+    assert rel_l2(y.cpu().numpy(), ref) <= 1e-5
 
 
 # ------------------------------------------------------------------ routing
