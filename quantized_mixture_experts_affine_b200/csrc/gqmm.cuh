@@ -19,6 +19,7 @@
 // the pages' format exactly once per weight before the tensor-core product.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -85,6 +86,11 @@ struct Seg {
 };
 
 struct Args {
+  // contiguous A rows (A_TOKENS, A_ROWS): tiles fetched by the tensor-memory
+  // accelerator from this map (box 64 x 128 fp16, 128-byte swizzle) when
+  // tma_a is set; gathered rows (A_PAIRS) always use cp.async
+  CUtensorMap tmA;
+  int32_t tma_a;
   const Seg* segs;
   const int2* tiles;        // (segment, first row within the segment); null: seg0 only
   const int32_t* n_tiles;   // device count of tiles
@@ -308,7 +314,27 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
   const int KB = a.K / BK;
   int* status = a.status;
 
-  if (warp < 2) {
+  if (warp < 2 && a.tma_a) {
+    // ------------------------------------------------------------ A loader (tensor map)
+    // thread 0 issues one 128-row x 64-column tile per stage; the other 63
+    // threads arrive so the stage barrier keeps its count of 64
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n);
+      const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
+      const int row0 = sg.a_mode == A_TOKENS ? tile.y : sg.row_begin + tile.y;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s = it % S1, ph = (it / S1) & 1u;
+        if (!tc::mbar_wait(&a_empty[s], ph ^ 1u, status)) goto done;
+        if (threadIdx.x == 0) {
+          tc::mbar_arrive_expect_tx(&full_a[s], (uint32_t)A_STAGE);
+          tc::tma_load_2d(sbase + SM::A_OFF + s * A_STAGE, &a.tmA, kb * BK, row0, &full_a[s]);
+        } else {
+          tc::mbar_arrive(&full_a[s]);
+        }
+      }
+    }
+  } else if (warp < 2) {
     // ------------------------------------------------------------ A loader
     // 64 threads; the 1024 16-byte chunks of a stage are spread so that each
     // group of 8 lanes writes the 8 chunks of one row (conflict-free).

@@ -4,6 +4,7 @@
 // weighted combine.  Every output row is computed from its own token only,
 // with the same kernels and the same K order for any M, so results do not
 // depend on how the tokens are split into calls.
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <string.h>
 
@@ -38,6 +39,19 @@ __global__ void __launch_bounds__(256) k_to_f16(const uint16_t* __restrict__ x, 
     reinterpret_cast<uint4*>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
   if (bad) set_status(status, MOEQ_ERR_RANGE);
+}
+
+// Rows of the fp16 tokens in sorted pair order: out[i] = x16[sorted[i] / K]
+// (the gate/up operand as one contiguous matrix, fetched by tensor-map tiles).
+__global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x16,
+                                                     const int32_t* __restrict__ sorted, int K,
+                                                     int64_t n, int row_chunks,
+                                                     uint4* __restrict__ out) {
+  for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
+    const int64_t src = sorted[r] / K;
+    for (int c = threadIdx.x; c < row_chunks; c += blockDim.x)
+      out[r * row_chunks + c] = x16[src * row_chunks + c];
+  }
 }
 
 // ------------------------------------------------------------------ routing (strided logits)
@@ -287,7 +301,7 @@ struct Carve {
 
 struct PrefillWs {
   size_t x16, logits, idx, w, sigma, blockhist, blockoff, expert_off, segs_gu, segs_dn, tiles,
-      n_tiles, sorted, h, h_sh, y, total;
+      n_tiles, sorted, a_sorted, h, h_sh, y, total;
   int64_t ld_logits;
   int nb;
 };
@@ -320,11 +334,46 @@ PrefillWs prefill_ws(const moeq_layer* L, int M) {
   w.tiles = c.take((size_t)max_tiles * sizeof(int2));
   w.n_tiles = c.take(16);
   w.sorted = c.take((size_t)n * 4);
+  w.a_sorted = c.take((size_t)n * H * 2);
   w.h = c.take((size_t)n * I * 2);
   w.h_sh = c.take((size_t)M * Is * 2);
   w.y = c.take((size_t)(n + M) * H * 4);
   w.total = c.off;
   return w;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (null if
+// the driver does not provide it).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Tensor map of an fp16 matrix [rows][K] (row stride lda elements) with a
+// 128-row x 64-column box in the 128-byte swizzled layout of the A stages;
+// rows past the end read as zeros.  Sets a.tma_a on success.
+void set_a_tensor_map(gq::Args& a, const __half* A, int64_t rows, int K, int64_t lda) {
+  a.tma_a = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn || ((uintptr_t)A & 15) || ((lda * 2) & 15) || rows <= 0 || K % gq::BK) return;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)lda * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)gq::BK, (cuuint32_t)gq::BM};
+  const cuuint32_t es[2] = {1, 1};
+  if (fn(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(A), dims, strides, box, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+    a.tma_a = 1;
 }
 
 moeq_status check_prefill(const moeq_layer* L) {
@@ -410,6 +459,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.out = out;
     a.ldo = ldo;
     a.status = status;
+    set_a_tensor_map(a, A, M, Kdim, lda);
     return a;
   };
   if (!idx_in) {
@@ -482,6 +532,15 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.K = H;
     a.A = x16;
     a.lda = H;
+    // the token rows in sorted pair order as one matrix: tensor-map tiles
+    __half* a_sorted = (__half*)(base + lay.a_sorted);
+    set_a_tensor_map(a, a_sorted, n, H, H);
+    if (a.tma_a) {
+      int64_t grid = n < (int64_t)sms * 16 ? n : (int64_t)sms * 16;
+      k_gather_rows<<<(int)grid, 256, 0, st>>>((const uint4*)x16, sorted, K, n, H / 8,
+                                               (uint4*)a_sorted);
+      PCK(cudaGetLastError());
+    }
     a.sorted_pair = sorted;
     a.topk = K;
     a.out = h;
@@ -511,6 +570,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.K = I;
     a.A = h;
     a.lda = I;
+    set_a_tensor_map(a, h, n, I, I);
     a.sorted_pair = sorted;
     a.topk = K;
     a.out = yrows;
