@@ -404,7 +404,7 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   const bool fused_plan =
       n <= kFusedMaxPairs && (!L->has_shared || p.shared_same_gu) &&
       plan_scratch_bytes(M, K, E, plan_route_warps(M, E, gemv_threads() / 32)) <=
-          (size_t)gemv_ring_bytes();
+          (size_t)gemv_plan_scratch_cap();
   // the down launch covers every segment: its CTAs also do the combine
   const bool fuse_combine = !L->has_shared || p.shared_same_dn;
   if (!fused_plan) LAUNCH(launch_decode_plan(p, st));

@@ -87,7 +87,9 @@ static_assert(GvSmem::BYTES <= 227 * 1024, "GEMV shared memory exceeds the per-C
 static_assert(GvSmem::PSEG_OFF % 16 == 0 && GvSmem::PVEC_OFF % 16 == 0, "plan region alignment");
 
 int gemv_threads() { return GV_THREADS; }
-int gemv_ring_bytes() { return GvSmem::RING_BYTES; }
+// A plan computed inside a gate/up launch keeps its scratch in stages 1..3
+// of the ring: stage 0 may already be receiving the shared expert's unit.
+int gemv_plan_scratch_cap() { return GvSmem::RING_BYTES - GV_STAGE_BYTES; }
 static_assert(sizeof(VecRef) == 16, "VecRef is copied in 16-byte pieces");
 
 // Last segment whose first unit is <= unit; p[i * stride] is segment i's
@@ -206,6 +208,91 @@ __device__ __forceinline__ T shfl_ptr(T p, int src) {
   return reinterpret_cast<T>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(p), src));
 }
 
+// One unit of work as the producer issues it.
+struct GvUnit {
+  int r0, nrows, n_vec, vec_mode;
+  const uint32_t* w[2];
+  const uint16_t* s[2];
+  const uint16_t* b[2];
+  const void* src_base;
+  int64_t src_stride;
+  float* dst_base;
+  int64_t dst_stride;
+  const VecRef* vecs;
+};
+
+// Fills stage s with unit u (every producer lane calls; lane 0 writes the
+// stage's description and issues the bulk copies): packed rows, then the
+// scale/bias rows -- contiguous runs of nrows * gpr entries, bulk-copied
+// when 16-byte aligned, else copied entry by entry -- and the unit's vector
+// references when they live in global memory.
+template <int NMAT>
+__device__ __forceinline__ void gv_issue(uint8_t* gsm, uint32_t sbase, uint64_t* full, uint32_t s,
+                                         const GvUnit& u, int row_bytes, int gpr, int RU) {
+  const int lane = threadIdx.x & 31;
+  const int codes_bytes = NMAT * RU * row_bytes;
+  const int sb_bytes = RU * gpr * 2;
+  const uint32_t st = sbase + s * GV_STAGE_BYTES;
+  const int sb_n = u.nrows * gpr;
+  bool sb_bulk = ((sb_n * 2) & 15) == 0 && ((codes_bytes | sb_bytes) & 15) == 0;
+#pragma unroll
+  for (int m = 0; m < NMAT; ++m)
+    sb_bulk = sb_bulk && ((((uintptr_t)(u.s[m] + (int64_t)u.r0 * gpr)) |
+                           ((uintptr_t)(u.b[m] + (int64_t)u.r0 * gpr))) & 15) == 0;
+  if (lane == 0) {
+    GvMeta* mt = reinterpret_cast<GvMeta*>(gsm + GvSmem::META_OFF + s * GvSmem::META_STRIDE);
+    mt->r0 = u.r0;
+    mt->nrows = u.nrows;
+    mt->n_vec = u.n_vec;
+    mt->vec_mode = u.vec_mode;
+    mt->src_base = u.src_base;
+    mt->src_stride = u.src_stride;
+    mt->dst_base = u.dst_base;
+    mt->dst_stride = u.dst_stride;
+    mt->vecs = u.vecs;
+    tc::mbar_arrive_expect_tx(
+        &full[s], (uint32_t)(NMAT * u.nrows * row_bytes + (sb_bulk ? 2 * NMAT * sb_n * 2 : 0)));
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m) {
+      tc::bulk_g2s(st + m * RU * row_bytes,
+                   reinterpret_cast<const uint8_t*>(u.w[m]) + (int64_t)u.r0 * row_bytes,
+                   (uint32_t)(u.nrows * row_bytes), &full[s]);
+      if (sb_bulk) {
+        tc::bulk_g2s(st + codes_bytes + m * sb_bytes, u.s[m] + (int64_t)u.r0 * gpr,
+                     (uint32_t)(sb_n * 2), &full[s]);
+        tc::bulk_g2s(st + codes_bytes + (NMAT + m) * sb_bytes, u.b[m] + (int64_t)u.r0 * gpr,
+                     (uint32_t)(sb_n * 2), &full[s]);
+      }
+    }
+  }
+  if (!sb_bulk) {
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m) {
+      const uint16_t* s0 = u.s[m] + (int64_t)u.r0 * gpr;
+      const uint16_t* b0 = u.b[m] + (int64_t)u.r0 * gpr;
+      uint16_t* sd =
+          reinterpret_cast<uint16_t*>(gsm + s * GV_STAGE_BYTES + codes_bytes + m * sb_bytes);
+      uint16_t* bd = reinterpret_cast<uint16_t*>(gsm + s * GV_STAGE_BYTES + codes_bytes +
+                                                 (NMAT + m) * sb_bytes);
+      for (int e = lane; e < sb_n; e += 32) {
+        sd[e] = s0[e];
+        bd[e] = b0[e];
+      }
+    }
+  }
+  if (u.vec_mode == 1 && u.n_vec <= GV_VMAX && !__isShared(u.vecs)) {
+    const uint32_t vd = sbase + GvSmem::VEC_OFF + s * GV_VMAX * 16;
+    for (int v = lane; v < u.n_vec; v += 32) tc::cp_async16(vd + 16 * v, u.vecs + v, 16);
+  }
+  if (sb_bulk) {
+    tc::cp_async_arrive_noinc(&full[s]);
+  } else {
+    // plain shared-memory stores above: released by an ordinary arrive
+    tc::cp_async_wait_all();
+    tc::mbar_arrive(&full[s]);
+  }
+}
+
 template <int BITS, int NL, int NMAT, int SRC, int EPI>
 __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ GemvArgs a) {
   constexpr int VPC = Chunk<BITS>::VPC;
@@ -237,9 +324,6 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     }
     tc::fence_mbar_init();
   }
-  // ranges known before the preceding kernel ends (the shared expert's
-  // weights) go to L2 while it finishes
-  if (warp == GV_HELPER && a.n_pf) prefetch_ranges(a.pf, a.n_pf);
   // fixed segments (router, qmv): no earlier kernel writes them or the
   // weights, so the producer starts streaming before the preceding kernel
   // ends; everyone else waits for it (input vectors, segment lists)
@@ -247,6 +331,44 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   if (static_segs)
     for (int i = threadIdx.x; i < a.n_segs; i += blockDim.x) ub[i] = a.segs[i].unit_begin;
   __syncthreads();
+  // ranges known before the preceding kernel ends (the shared expert's
+  // weights) go to L2 while it finishes; the other warps do not wait for it
+  if (warp == GV_HELPER && a.n_pf) prefetch_ranges(a.pf, a.n_pf);
+  const int row_bytes = a.in_dim * BITS / 8;
+  const int gpr = a.in_dim / a.G;
+  const int cpr = a.in_dim / VPC;
+  // stage layout: codes [NMAT][RU][row_bytes], scales [NMAT][RU*gpr], biases [NMAT][RU*gpr]
+  const int codes_bytes = NMAT * RU * row_bytes;
+  const int sb_bytes = RU * gpr * 2;
+  int* status = a.status;
+  // a step planned in this launch lists the shared expert first; its
+  // weights do not depend on the routing, so the producer puts this CTA's
+  // first unit of it into stage 0 before the preceding kernel ends
+  int preissued = 0;
+  if constexpr (NMAT == 2) {
+    const DecodePlanArgs& pl = a.plan;
+    if (a.fused_plan && pl.has_shared && warp == GV_PRODUCER &&
+        (int)blockIdx.x < pl.units_per_seg_gu_sh) {
+      GvUnit gu;
+      gu.r0 = blockIdx.x * RU;
+      gu.nrows = min(RU, pl.sh_gate.out_dim - gu.r0);
+      gu.n_vec = pl.M;
+      gu.vec_mode = 0;
+      gu.w[0] = pl.sh_gate.w;
+      gu.s[0] = pl.sh_gate.scales;
+      gu.b[0] = pl.sh_gate.biases;
+      gu.w[1] = pl.sh_up.w;
+      gu.s[1] = pl.sh_up.scales;
+      gu.b[1] = pl.sh_up.biases;
+      gu.src_base = pl.x;
+      gu.src_stride = pl.H;
+      gu.dst_base = pl.h + (int64_t)pl.M * pl.K * pl.I;
+      gu.dst_stride = pl.sh_gate.out_dim;
+      gu.vecs = nullptr;
+      gv_issue<2>(gsm, sbase, full, 0, gu, row_bytes, gpr, RU);
+      preissued = 1;
+    }
+  }
   if (!(static_segs && warp == GV_PRODUCER)) tc::grid_dep_wait();
   tc::grid_dep_launch();
 
@@ -282,8 +404,11 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
           o.ctr = a.plan.ctr;
           o.n_ctr = a.plan.n_ctr;
         }
-        // the scratch of the plan lives in the (still unused) stage ring
-        plan_cta(a.plan, gsm, plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32), o);
+        // the scratch of the plan lives in stages 1..3 of the (still unused)
+        // ring; stage 0 may be receiving the shared expert's unit
+        o.shared_first = a.plan.has_shared;
+        plan_cta(a.plan, gsm + GV_STAGE_BYTES,
+                 plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32), o);
         segs = psegs;
         n_segs = pcnt[0];
         total_units = pcnt[1];
@@ -301,13 +426,6 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   }
   const bool ub_cached = n_segs <= GV_UB_CAP;
 
-  const int row_bytes = a.in_dim * BITS / 8;
-  const int gpr = a.in_dim / a.G;
-  const int cpr = a.in_dim / VPC;
-  // stage layout: codes [NMAT][RU][row_bytes], scales [NMAT][RU*gpr], biases [NMAT][RU*gpr]
-  const int codes_bytes = NMAT * RU * row_bytes;
-  const int sb_bytes = RU * gpr * 2;
-  int* status = a.status;
 
   if (warp == GV_HELPER) {
     // ------------------------------------------------------------ L2 prefetch
@@ -315,9 +433,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     else if (a.pf_segs) prefetch_segs(a.pf_segs, a.pf_count[0]);
   } else if (warp == GV_PRODUCER) {
     // ------------------------------------------------------------ producer
-    uint32_t it = 0;
+    uint32_t it = preissued;
     bool dead = false;
-    for (int base = blockIdx.x; base < total_units && !dead; base += 32 * gridDim.x) {
+    for (int base = blockIdx.x + preissued * gridDim.x; base < total_units && !dead;
+         base += 32 * gridDim.x) {
       // lane u describes unit base + u * gridDim.x
       const int mine = base + lane * gridDim.x;
       int r0 = 0, nrows = 0, n_vec = 0, vec_mode = 0;
@@ -357,85 +476,23 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
           dead = true;
           break;
         }
-        const int ur0 = __shfl_sync(0xffffffffu, r0, u);
-        const int unr = __shfl_sync(0xffffffffu, nrows, u);
-        const int unv = __shfl_sync(0xffffffffu, n_vec, u);
-        const int uvm = __shfl_sync(0xffffffffu, vec_mode, u);
-        const VecRef* uvecs = shfl_ptr(vecs, u);
-        const uint32_t st = sbase + s * GV_STAGE_BYTES;
-        const uint32_t* uw[2];
-        const uint16_t* usp[2];
-        const uint16_t* ubp[2];
+        GvUnit gu;
+        gu.r0 = __shfl_sync(0xffffffffu, r0, u);
+        gu.nrows = __shfl_sync(0xffffffffu, nrows, u);
+        gu.n_vec = __shfl_sync(0xffffffffu, n_vec, u);
+        gu.vec_mode = __shfl_sync(0xffffffffu, vec_mode, u);
+        gu.vecs = shfl_ptr(vecs, u);
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-          uw[m] = shfl_ptr(w[m], u);
-          usp[m] = shfl_ptr(sp[m], u);
-          ubp[m] = shfl_ptr(bp[m], u);
+          gu.w[m] = shfl_ptr(w[m], u);
+          gu.s[m] = shfl_ptr(sp[m], u);
+          gu.b[m] = shfl_ptr(bp[m], u);
         }
-        const void* usrc = shfl_ptr(src_base, u);
-        float* udst = shfl_ptr(dst_base, u);
-        const int64_t uss = __shfl_sync(0xffffffffu, src_stride, u);
-        const int64_t uds = __shfl_sync(0xffffffffu, dst_stride, u);
-        // scale/bias rows of the unit: contiguous runs of unr * gpr entries,
-        // bulk-copied when 16-byte aligned, else copied entry by entry
-        const int sb_n = unr * gpr;
-        bool sb_bulk = ((sb_n * 2) & 15) == 0 && ((codes_bytes | sb_bytes) & 15) == 0;
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m)
-          sb_bulk = sb_bulk && ((((uintptr_t)(usp[m] + (int64_t)ur0 * gpr)) |
-                                 ((uintptr_t)(ubp[m] + (int64_t)ur0 * gpr))) & 15) == 0;
-        if (lane == 0) {
-          GvMeta* mt = reinterpret_cast<GvMeta*>(gsm + GvSmem::META_OFF + s * GvSmem::META_STRIDE);
-          mt->r0 = ur0;
-          mt->nrows = unr;
-          mt->n_vec = unv;
-          mt->vec_mode = uvm;
-          mt->src_base = usrc;
-          mt->src_stride = uss;
-          mt->dst_base = udst;
-          mt->dst_stride = uds;
-          mt->vecs = uvecs;
-          tc::mbar_arrive_expect_tx(
-              &full[s], (uint32_t)(NMAT * unr * row_bytes + (sb_bulk ? 2 * NMAT * sb_n * 2 : 0)));
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            tc::bulk_g2s(st + m * RU * row_bytes,
-                         reinterpret_cast<const uint8_t*>(uw[m]) + (int64_t)ur0 * row_bytes,
-                         (uint32_t)(unr * row_bytes), &full[s]);
-            if (sb_bulk) {
-              tc::bulk_g2s(st + codes_bytes + m * sb_bytes, usp[m] + (int64_t)ur0 * gpr,
-                           (uint32_t)(sb_n * 2), &full[s]);
-              tc::bulk_g2s(st + codes_bytes + (NMAT + m) * sb_bytes, ubp[m] + (int64_t)ur0 * gpr,
-                           (uint32_t)(sb_n * 2), &full[s]);
-            }
-          }
-        }
-        if (!sb_bulk) {
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            const uint16_t* s0 = usp[m] + (int64_t)ur0 * gpr;
-            const uint16_t* b0 = ubp[m] + (int64_t)ur0 * gpr;
-            uint16_t* sd = reinterpret_cast<uint16_t*>(gsm + s * GV_STAGE_BYTES + codes_bytes +
-                                                       m * sb_bytes);
-            uint16_t* bd = reinterpret_cast<uint16_t*>(gsm + s * GV_STAGE_BYTES + codes_bytes +
-                                                       (NMAT + m) * sb_bytes);
-            for (int e = lane; e < sb_n; e += 32) {
-              sd[e] = s0[e];
-              bd[e] = b0[e];
-            }
-          }
-        }
-        if (uvm == 1 && unv <= GV_VMAX && !__isShared(uvecs)) {
-          const uint32_t vd = sbase + GvSmem::VEC_OFF + s * GV_VMAX * 16;
-          for (int v = lane; v < unv; v += 32) tc::cp_async16(vd + 16 * v, uvecs + v, 16);
-        }
-        if (sb_bulk) {
-          tc::cp_async_arrive_noinc(&full[s]);
-        } else {
-          // plain shared-memory stores above: released by an ordinary arrive
-          tc::cp_async_wait_all();
-          tc::mbar_arrive(&full[s]);
-        }
+        gu.src_base = shfl_ptr(src_base, u);
+        gu.dst_base = shfl_ptr(dst_base, u);
+        gu.src_stride = __shfl_sync(0xffffffffu, src_stride, u);
+        gu.dst_stride = __shfl_sync(0xffffffffu, dst_stride, u);
+        gv_issue<NMAT>(gsm, sbase, full, s, gu, row_bytes, gpr, RU);
       }
     }
   } else {
@@ -733,6 +790,9 @@ __device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const
                                                   int u, int e, int cnt) {
   if (o.experts) o.experts[u] = e;
   if (o.segs_gu) {
+    // shared expert first: the routed entries follow it
+    const int gi = o.shared_first ? u + 1 : u;
+    const int gu0 = o.shared_first ? a.units_per_seg_gu_sh : 0;
     Seg g;
     g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
     g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
@@ -745,14 +805,14 @@ __device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const
     g.G = a.gate.group_size;
     g.bits = a.gate.bits;
     g.n_vec = cnt;
-    g.unit_begin = u * a.units_per_seg_gu;
+    g.unit_begin = gu0 + u * a.units_per_seg_gu;
     g.vec_mode = 1;
     g.src_base = nullptr;
     g.src_stride = 0;
     g.dst_base = nullptr;
     g.dst_stride = 0;
     g.vecs = o.vecs_gu + i;
-    o.segs_gu[u] = g;
+    o.segs_gu[gi] = g;
   }
   if (o.segs_dn) {
     Seg dn;
@@ -933,8 +993,13 @@ __device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, i
         g.dst_base = a.h + (int64_t)n * a.I;
         g.dst_stride = a.sh_gate.out_dim;
         g.vecs = nullptr;
-        g.unit_begin = same_gu ? units_gu : 0;
-        o.segs_gu[same_gu ? n_entries : n] = g;
+        if (o.shared_first) {
+          g.unit_begin = 0;
+          o.segs_gu[0] = g;
+        } else {
+          g.unit_begin = same_gu ? units_gu : 0;
+          o.segs_gu[same_gu ? n_entries : n] = g;
+        }
       }
       if (o.segs_dn) {
         Seg dn;

@@ -97,6 +97,9 @@ struct PlanSinks {
   int32_t n_ctr;
   int32_t* experts;         // [entries] expert of each entry
   int32_t* n_experts;
+  // gate/up list with the shared expert first (segment 0, units from 0) and
+  // the routed entries after it
+  int32_t shared_first;
 };
 
 // Staged logits of the plan's routing warps: at most this many bytes.
@@ -157,7 +160,7 @@ struct GemvShape {
 GemvShape gemv_shape(int in_dim, int bits, int nmat, int G);
 bool gemv_fits(int in_dim, int bits, int nmat, int G);
 int gemv_threads();     // threads of a GEMV CTA
-int gemv_ring_bytes();  // bytes of its stage ring (also the scratch of a fused plan)
+int gemv_plan_scratch_cap();  // bytes a plan computed inside a GEMV launch may use
 int gemv_units(int out_dim, const GemvShape& sh);
 
 // Launch with programmatic dependent launch (the kernel waits for its
