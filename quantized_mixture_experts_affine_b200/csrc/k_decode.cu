@@ -744,13 +744,17 @@ struct PlanScratch {
   int32_t* entry_of;  // [n] entry index of sorted position
   uint32_t* taken;    // [R][words] routing bitmaps
   float* rows;        // [R][E] staged logits (16-byte aligned)
+  int32_t* cidx;      // [M][4][K] candidates of the parts of a token
+  float* cval;        // [M][4][K]
+  float* pmax;        // [M][4] largest value of each part
+  float* psum;        // [M][4] sum of exp(v - part maximum)
 };
 
 __host__ __device__ size_t plan_scratch_bytes(int M, int K, int E, int R) {
   const size_t n = (size_t)M * K;
   size_t b = (7 * n + (size_t)M) * 4 + (size_t)R * ((E + 31) / 32) * 4;
   b = (b + 15) & ~(size_t)15;
-  return b + (size_t)R * E * 4;
+  return b + (size_t)R * E * 4 + (size_t)M * 4 * K * 8 + (size_t)M * 4 * 8;
 }
 
 __device__ __forceinline__ PlanScratch plan_scratch(uint8_t* sm, int M, int K, int E, int R) {
@@ -767,6 +771,10 @@ __device__ __forceinline__ PlanScratch plan_scratch(uint8_t* sm, int M, int K, i
   size_t off = (size_t)(7 * n + M) * 4 + (size_t)R * ((E + 31) / 32) * 4;
   off = (off + 15) & ~(size_t)15;
   p.rows = reinterpret_cast<float*>(sm + off);
+  p.cidx = reinterpret_cast<int32_t*>(p.rows + (size_t)R * E);
+  p.cval = reinterpret_cast<float*>(p.cidx + (size_t)M * 4 * K);
+  p.pmax = p.cval + (size_t)M * 4 * K;
+  p.psum = p.pmax + (size_t)M * 4;
   return p;
 }
 
@@ -851,8 +859,23 @@ __device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, i
   const int words = (a.E + 31) >> 5;
   const PlanScratch ps = plan_scratch(sm, M, K, a.E, R);
 
-  // 1. routing: R warps, one token each at a time
-  if (a.logits) {
+  // 1. routing: for few tokens and many experts, four warps per token each
+  //    select candidates from a quarter of the experts and one merges them;
+  //    otherwise R warps, one token each at a time
+  const int WT = (a.logits && a.E >= 256 && M <= 8 && M * 4 <= (nthr >> 5)) ? 4 : 1;
+  if (WT > 1) {
+    if (warp < M * WT) {
+      const int t = warp / WT, part = warp % WT;
+      int32_t* cidx = ps.cidx + t * 4 * K;
+      float* cval = ps.cval + t * 4 * K;
+      route_part(a.logits + (int64_t)t * a.E, a.E, K, a.router_scale, part, WT, cidx + part * K,
+                 cval + part * K, ps.pmax + t * 4 + part, ps.psum + t * 4 + part);
+      tc::named_sync(4 + t, WT * 32);
+      if (part == 0)
+        route_merge_parts(cidx, cval, WT * K, K, a.renorm, ps.pmax + t * 4, ps.psum + t * 4, WT,
+                          ps.sidx + t * K, ps.sw + t * K);
+    }
+  } else if (a.logits) {
     if (warp < R)
       for (int t = warp; t < M; t += R)
         route_token_warp(a.logits + (int64_t)t * a.E, a.E, K, a.renorm, a.router_scale,
