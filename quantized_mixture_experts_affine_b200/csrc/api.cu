@@ -152,7 +152,7 @@ struct Carve {
 
 struct DecodeWs {
   size_t logits, sg_logit, sigma, idx, w, h, d, segs_gu, segs_dn, counts, vecs_gu, vecs_dn, ctr,
-      total;
+      flag, total;
 };
 
 DecodeWs decode_ws(const moeq_layer* L, int M) {
@@ -174,6 +174,7 @@ DecodeWs decode_ws(const moeq_layer* L, int M) {
   w.vecs_gu = c.take(n * sizeof(VecRef));
   w.vecs_dn = c.take(n * sizeof(VecRef));
   w.ctr = c.take((size_t)H * 4);  // at most one counter per output row
+  w.flag = c.take(4);             // "down lists published"
   w.total = c.off;
   return w;
 }
@@ -331,8 +332,19 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
                               SG.group_size == R.group_size && SG.in_dim == R.in_dim;
   // the shared expert's weights do not depend on the routing: pull them into
   // L2 while the router streams
+  // small steps plan inside the gate/up launch (fused plan, below); when
+  // the router runs too, the down launch's producer starts on the plan's
+  // flag instead of on the whole gate/up launch
+  const bool sh_same_gu = L->has_shared && L->sh_gate.bits == L->gate.bits &&
+                          L->sh_gate.group_size == L->gate.group_size;
+  const bool fused_plan =
+      n <= kFusedMaxPairs && (!L->has_shared || sh_same_gu) &&
+      plan_scratch_bytes(M, K, E, plan_route_warps(M, E, gemv_threads() / 32)) <=
+          (size_t)gemv_plan_scratch_cap();
+  int32_t* flag = (fused_plan && !idx_in) ? (int32_t*)(base + lay.flag) : nullptr;
   GemvArgs pf;
   memset(&pf, 0, sizeof(pf));
+  pf.flag_reset = flag;
   if (L->has_shared) {
     add_prefetch(pf, L->sh_gate, 0);
     add_prefetch(pf, L->sh_up, 0);
@@ -345,6 +357,7 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     if (sg_with_router) segs[ns++] = plain_seg(SG, 0, x, H, sg_logit, 1, M, 0);
     LAUNCH(run_plain(R, segs, ns, 3, &pf, st));
     pf.n_pf = 0;
+    pf.flag_reset = nullptr;
   }
   if (L->has_shared && (idx_in || !sg_with_router)) {
     Seg s = plain_seg(SG, 0, x, H, sg_logit, 1, M, 0);
@@ -400,11 +413,6 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
                         L->sh_down.in_dim == L->down.in_dim);
   }
   p.status = status_ptr();
-  // small steps: every gate/up CTA computes the plan itself (no plan launch)
-  const bool fused_plan =
-      n <= kFusedMaxPairs && (!L->has_shared || p.shared_same_gu) &&
-      plan_scratch_bytes(M, K, E, plan_route_warps(M, E, gemv_threads() / 32)) <=
-          (size_t)gemv_plan_scratch_cap();
   // the down launch covers every segment: its CTAs also do the combine
   const bool fuse_combine = !L->has_shared || p.shared_same_dn;
   if (!fused_plan) LAUNCH(launch_decode_plan(p, st));
@@ -422,6 +430,7 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     a.status = status_ptr();
     a.fused_plan = 1;
     a.plan = p;
+    a.flag_set = flag;
     const int grid = max_gu < grid_cap() ? max_gu : grid_cap();
     LAUNCH(launch_gemv(L->gate.bits, 2, 2, SRC_BF16, a, grid, st));
   } else {
@@ -439,6 +448,7 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     a.dyn_segs = segs_dn;
     a.dyn_count = counts + 4;
     a.status = status_ptr();
+    a.flag_wait = flag;
     if (fuse_combine) {
       a.fuse_combine = 1;
       a.comb.w = wts;

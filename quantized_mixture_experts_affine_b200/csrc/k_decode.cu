@@ -208,6 +208,29 @@ __device__ __forceinline__ T shfl_ptr(T p, int src) {
   return reinterpret_cast<T>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(p), src));
 }
 
+// Bounded wait (lane 0 polls, about two seconds) until *p == 1; the warp
+// gets the outcome.  On timeout sets MOEQ_ERR_TIMEOUT.
+__device__ __forceinline__ bool wait_flag(const int32_t* p, int* status) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    const uint64_t t0 = tc::globaltimer_ns();
+    int v;
+    for (;;) {
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+      if (v == 1) break;
+      __nanosleep(128);
+      if (tc::globaltimer_ns() - t0 > 2000000000ull) {
+        set_status(status, MOEQ_ERR_TIMEOUT);
+        ok = false;
+        break;
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok;
+}
+
 // One unit of work as the producer issues it.
 struct GvUnit {
   int r0, nrows, n_vec, vec_mode;
@@ -369,11 +392,15 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
       preissued = 1;
     }
   }
-  if (!(static_segs && warp == GV_PRODUCER)) tc::grid_dep_wait();
+  // the down launch's producer may start on the plan's flag (below)
+  const bool early = a.flag_wait != nullptr;
+  if (!((static_segs || early) && warp == GV_PRODUCER)) tc::grid_dep_wait();
   tc::grid_dep_launch();
+  if (a.flag_reset && blockIdx.x == 0 && threadIdx.x == 0) *a.flag_reset = 0;
 
   const Seg* segs;
   int n_segs, total_units;
+  bool timed_out_p = false;
   int32_t* pcnt = reinterpret_cast<int32_t*>(gsm + GvSmem::PCNT_OFF);
   int32_t* pexp = reinterpret_cast<int32_t*>(gsm + GvSmem::PEXP_OFF);
   if (static_segs) {
@@ -409,6 +436,12 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         o.shared_first = a.plan.has_shared;
         plan_cta(a.plan, gsm + GV_STAGE_BYTES,
                  plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32), o);
+        if (a.flag_set && blockIdx.x == 0 && threadIdx.x == 0) {
+          // CTA 0's lists (written before plan_cta's final barrier) are
+          // visible GPU-wide before the flag
+          __threadfence();
+          atomicExch(a.flag_set, 1);
+        }
         segs = psegs;
         n_segs = pcnt[0];
         total_units = pcnt[1];
@@ -416,15 +449,29 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
       }
     }
     if (!planned) {
+      if (early && warp == GV_PRODUCER) {
+        // wait (bounded) until the plan's down lists are published
+        if (!wait_flag(a.flag_wait, status)) timed_out_p = true;
+      }
       segs = a.dyn_segs;
-      n_segs = a.dyn_count[0];
-      total_units = a.dyn_count[1];
+      n_segs = timed_out_p ? 0 : a.dyn_count[0];
+      total_units = timed_out_p ? 0 : a.dyn_count[1];
     }
-    if (n_segs <= GV_UB_CAP)
-      for (int i = threadIdx.x; i < n_segs; i += blockDim.x) ub[i] = segs[i].unit_begin;
-    __syncthreads();
+    if (early) {
+      // the producer does not join: the others cache the segment starts
+      if (warp != GV_PRODUCER) {
+        if (n_segs <= GV_UB_CAP)
+          for (int i = threadIdx.x; i < n_segs; i += GV_PRODUCER * 32) ub[i] = segs[i].unit_begin;
+        // warps 0..15 and 17 (the helper is warp 17: its 32 threads count)
+        tc::named_sync(1, (GV_THREADS - 32));
+      }
+    } else {
+      if (n_segs <= GV_UB_CAP)
+        for (int i = threadIdx.x; i < n_segs; i += blockDim.x) ub[i] = segs[i].unit_begin;
+      __syncthreads();
+    }
   }
-  const bool ub_cached = n_segs <= GV_UB_CAP;
+  const bool ub_cached = n_segs <= GV_UB_CAP && !(early && warp == GV_PRODUCER);
 
 
   if (warp == GV_HELPER) {

@@ -146,6 +146,13 @@ struct GemvArgs {
   // down launch: weighted combine by the last CTA of each row block
   int32_t fuse_combine;
   CombineArgs comb;
+  // the step's "down lists published" flag: the router launch sets it to 0
+  // after its dependency wait, the gate/up launch that plans the step sets
+  // it to 1 once CTA 0 has written the down lists, and the down launch's
+  // producer starts on it instead of on the dependency wait (null: unused)
+  int32_t* flag_reset;
+  int32_t* flag_set;
+  const int32_t* flag_wait;
 };
 
 enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
