@@ -5,8 +5,9 @@
 //   warps 0-1  A loader: gathers the 128 rows (token rows of x, or the
 //              expert's contiguous hidden rows) with 16-byte cp.async into
 //              the 128B-swizzled K-major A stage;
-//   warp  2    B loader: cp.async of the packed codes of 256 weight rows and
-//              of their bf16 scale/bias pairs for one 64-wide group;
+//   warp  2    B loader: the packed codes of 256 weight rows for one
+//              64-wide group (two tensor-map tiles of 128 rows, or cp.async
+//              per row) and their bf16 scale/bias pairs (cp.async);
 //   warp  3    MMA issuer: tcgen05.mma (M 128, N 256, K 16) x 4 per group,
 //              fp32 accumulators in TMEM (two 256-column buffers);
 //   warps 4-7  epilogue: tcgen05.ld of the accumulator rows, SwiGLU to fp16
@@ -39,19 +40,21 @@ constexpr int DQ_WARPS = 8;            // dequantiser warps: one weight row per 
 constexpr int THREADS = (8 + DQ_WARPS) * 32;
 constexpr uint32_t IDESC = tc::idesc_f16_f32(BM, BN);
 
-// Packed codes of one k-block in shared memory, one row per dequantiser
-// thread.  Rows are laid out so that eight consecutive rows read by a
-// quarter-warp touch distinct 16-byte bank groups: 8-bit rows (64 bytes)
-// swizzle their 4 chunks by (row >> 1) & 3, 4-bit rows (32 bytes) are
-// padded to 48 bytes, 2-bit rows (16 bytes) are contiguous.
+// Packed codes of one k-block in shared memory, one dense row per
+// dequantiser thread, in the layout a tensor-map load writes: 8-bit rows
+// (64 bytes) with the 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3)),
+// 4-bit rows (32 bytes) with the 32-byte swizzle (c ^ ((r >> 2) & 1)), 2-bit
+// rows (16 bytes) plain.  Either way the eight rows a quarter-warp reads
+// touch distinct 16-byte bank groups.
 template <int BITS>
 struct Raw {
   static constexpr int ROW = BK * BITS / 8;       // packed bytes of one row per k-block
   static constexpr int CHUNKS = ROW / 16;         // 16-byte chunks per row
-  static constexpr int STRIDE = BITS == 4 ? 48 : ROW;
-  static constexpr int STAGE = BN * STRIDE;
+  static constexpr int STAGE = BN * ROW;
   __device__ __forceinline__ static int offset(int r, int c) {
-    return BITS == 8 ? r * ROW + ((c ^ ((r >> 1) & 3)) << 4) : r * STRIDE + (c << 4);
+    return BITS == 8   ? r * ROW + ((c ^ ((r >> 1) & 3)) << 4)
+           : BITS == 4 ? r * ROW + ((c ^ ((r >> 2) & 1)) << 4)
+                       : r * ROW + (c << 4);
   }
 };
 
@@ -83,6 +86,7 @@ struct Seg {
   int32_t rows;       // rows of the segment
   int32_t a_mode;     // AMode
   int32_t dest_pairs; // STORE: 1 = output row is the pair index sorted_pair[m]
+  int32_t ex[2];      // matrix index of each source in its code tensor map
 };
 
 struct Args {
@@ -91,6 +95,10 @@ struct Args {
   // tma_a is set; gathered rows (A_PAIRS) always use cp.async
   CUtensorMap tmA;
   int32_t tma_a;
+  // packed codes (SWIGLU: gate and up, STORE: the single source) fetched by
+  // tensor-map tiles of 128 rows x one 64-wide group when tma_b is set
+  CUtensorMap tmB[2];
+  int32_t tma_b;
   const Seg* segs;
   const int2* tiles;        // (segment, first row within the segment); null: seg0 only
   const int32_t* n_tiles;   // device count of tiles
@@ -377,6 +385,55 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
                          p ? 16u : 0u);
         }
         tc::cp_async_arrive_noinc(&full_a[s]);
+      }
+    }
+  } else if (warp == 2 && a.tma_b) {
+    // ------------------------------------------------------------ B loader (tensor maps)
+    // lane 0 fetches the codes as two 128-row tiles; every lane fetches the
+    // scale/bias pairs of its 8 rows
+    const int groups = a.K / 64;
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n);
+      const int nt = item % a.n_tiles_n;
+      const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
+      const uint16_t* sp[8];
+      const uint16_t* bp[8];
+      uint32_t ok4[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = lane + 32 * j;
+        int src, q;
+        bool ok;
+        b_row<EPI>(sg, nt, r, src, q, ok);
+        if (!ok) q = 0;
+        sp[j] = sg.s[src] + (int64_t)q * groups;
+        bp[j] = sg.b[src] + (int64_t)q * groups;
+        ok4[j] = ok ? 4u : 0u;
+      }
+      // (source, first row) of the two 128-row halves of the tile
+      const int src1 = EPI == EPI_SWIGLU ? 1 : 0;
+      const int y0 = EPI == EPI_SWIGLU ? nt * 128 : nt * BN;
+      const int y1 = EPI == EPI_SWIGLU ? nt * 128 : nt * BN + 128;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s = it % SR, ph = (it / SR) & 1u;
+        if (!tc::mbar_wait(&raw_empty[s], ph ^ 1u, status)) goto done;
+        const uint32_t rst = sbase + SM::RAW_OFF + s * RW::STAGE;
+        const uint32_t sbst = sbase + SM::SB_OFF + s * SB_STAGE;
+        if (lane == 0) {
+          tc::mbar_expect_tx(&raw_full[s], (uint32_t)RW::STAGE);
+          tc::tma_load_3d(rst, &a.tmB[0], kb * (RW::ROW / 4), y0, sg.ex[0], &raw_full[s]);
+          tc::tma_load_3d(rst + 128 * RW::ROW, &a.tmB[src1], kb * (RW::ROW / 4), y1,
+                          sg.ex[src1], &raw_full[s]);
+        }
+        const int kb2 = kb & ~1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = lane + 32 * j;
+          tc::cp_async4(sbst + r * 8, sp[j] + kb2, ok4[j]);
+          tc::cp_async4(sbst + r * 8 + 4, bp[j] + kb2, ok4[j]);
+        }
+        tc::cp_async_arrive_noinc(&raw_full[s]);
       }
     }
   } else if (warp == 2) {

@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ Offset
     g.rows = c;
     g.a_mode = gq::A_PAIRS;
     g.dest_pairs = 0;
+    g.ex[0] = g.ex[1] = e;
     a.segs_gu[e] = g;
     gq::Seg d;
     memset(&d, 0, sizeof(d));
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ Offset
     d.rows = c;
     d.a_mode = gq::A_ROWS;
     d.dest_pairs = 1;
+    d.ex[0] = d.ex[1] = e;
     a.segs_dn[e] = d;
     const int nt = (c + gq::BM - 1) / gq::BM;
     for (int j = 0; j < nt; ++j) a.tiles[tile + j] = make_int2(e, j * gq::BM);
@@ -376,6 +378,29 @@ void set_a_tensor_map(gq::Args& a, const __half* A, int64_t rows, int K, int64_t
     a.tma_a = 1;
 }
 
+// Tensor map of a packed code tensor [n_mat][out_dim][in_dim*bits/32 words]
+// with a box of 128 rows x one 64-wide group, written in the swizzle of the
+// raw code stages.  False when the tensor does not meet the map's rules.
+bool code_tensor_map(CUtensorMap* m, const moeq_qtensor& t, int n_mat) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  const int64_t row_words = (int64_t)t.in_dim * t.bits / 32;
+  const int64_t row_bytes = row_words * 4;
+  const int64_t mat_bytes = n_mat > 1 ? t.expert_stride_w * 4 : (int64_t)t.out_dim * row_bytes;
+  if (!fn || ((uintptr_t)t.w & 15) || (row_bytes & 15) || (mat_bytes & 15) || mat_bytes <= 0 ||
+      t.in_dim % gq::BK || n_mat < 1)
+    return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)row_words, (cuuint64_t)t.out_dim, (cuuint64_t)n_mat};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)mat_bytes};
+  const cuuint32_t box[3] = {(cuuint32_t)(gq::BK * t.bits / 32), 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUtensorMapSwizzle swz = t.bits == 8   ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : t.bits == 4 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                               : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(t.w), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 moeq_status check_prefill(const moeq_layer* L) {
   const moeq_qtensor* ts[8] = {&L->router, &L->gate, &L->up, &L->down,
                                &L->sh_gate, &L->sh_up, &L->sh_down, &L->sh_expert_gate};
@@ -546,6 +571,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.out = h;
     a.ldo = I;
     a.status = status;
+    a.tma_b = code_tensor_map(&a.tmB[0], L->gate, E) && code_tensor_map(&a.tmB[1], L->up, E);
     const int64_t items = max_mtiles * a.n_tiles_n;
     if (profile_mark(true, st) != cudaSuccess) return MOEQ_ERR_CUDA;
     PCK(launch_gqmm(L->gate.bits, gq::EPI_SWIGLU, a, items < sms ? (int)items : sms, st));
@@ -555,7 +581,8 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     const int Is = L->sh_gate.out_dim;
     gq::Seg gs = seg_single(L->sh_gate, &L->sh_up, M, gq::A_TOKENS);
     gs.n0 = Is;
-    const gq::Args a = gemm_args(gs, Is / 128, H, x16, H, h_sh, Is);
+    gq::Args a = gemm_args(gs, Is / 128, H, x16, H, h_sh, Is);
+    a.tma_b = code_tensor_map(&a.tmB[0], L->sh_gate, 1) && code_tensor_map(&a.tmB[1], L->sh_up, 1);
     const int items = mtiles * (Is / 128);
     PCK(launch_gqmm(L->sh_gate.bits, gq::EPI_SWIGLU, a, items < sms ? items : sms, st));
   }
@@ -576,14 +603,16 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.out = yrows;
     a.ldo = H;
     a.status = status;
+    a.tma_b = code_tensor_map(&a.tmB[0], L->down, E);
     const int64_t items = max_mtiles * a.n_tiles_n;
     PCK(launch_gqmm(L->down.bits, gq::EPI_STORE, a, items < sms ? (int)items : sms, st));
   }
   if (L->has_shared) {
     const int Is = L->sh_gate.out_dim;
     const gq::Seg ds = seg_single(L->sh_down, nullptr, M, gq::A_ROWS);
-    const gq::Args a = gemm_args(ds, (H + gq::BN - 1) / gq::BN, Is, h_sh, Is,
-                                 yrows + n * (int64_t)H, H);
+    gq::Args a = gemm_args(ds, (H + gq::BN - 1) / gq::BN, Is, h_sh, Is,
+                           yrows + n * (int64_t)H, H);
+    a.tma_b = code_tensor_map(&a.tmB[0], L->sh_down, 1);
     const int items = mtiles * ((H + gq::BN - 1) / gq::BN);
     PCK(launch_gqmm(L->sh_down.bits, gq::EPI_STORE, a, items < sms ? items : sms, st));
   }
