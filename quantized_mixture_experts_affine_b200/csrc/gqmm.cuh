@@ -29,16 +29,10 @@
 namespace moeq {
 namespace gq {
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int S1 = 4;  // stages of A (gathered token rows)
-constexpr int SR = 3;  // stages of packed B codes and scale/bias pairs
-constexpr int S2 = 3;  // stages of dequantised B
-constexpr int A_STAGE = BM * BK * 2;   // 16 KB
-constexpr int B_STAGE = BN * BK * 2;   // 32 KB
-constexpr int SB_STAGE = BN * 8;       // scale pair + bias pair per row: 2 KB
-constexpr int DQ_WARPS = 8;            // dequantiser warps: one weight row per thread
+constexpr int BM = 128, BN = 256, BK = 64;  // per MMA issuer: M = BM (PAIR: 2 BM)
+constexpr int A_STAGE = BM * BK * 2;   // 16 KB: 128 rows of A per CTA
+constexpr int DQ_WARPS = 8;            // dequantiser warps
 constexpr int THREADS = (8 + DQ_WARPS) * 32;
-constexpr uint32_t IDESC = tc::idesc_f16_f32(BM, BN);
 
 // Packed codes of one k-block in shared memory, one dense row per
 // dequantiser thread, in the layout a tensor-map load writes: 8-bit rows
@@ -50,7 +44,6 @@ template <int BITS>
 struct Raw {
   static constexpr int ROW = BK * BITS / 8;       // packed bytes of one row per k-block
   static constexpr int CHUNKS = ROW / 16;         // 16-byte chunks per row
-  static constexpr int STAGE = BN * ROW;
   __device__ __forceinline__ static int offset(int r, int c) {
     return BITS == 8   ? r * ROW + ((c ^ ((r >> 1) & 3)) << 4)
            : BITS == 4 ? r * ROW + ((c ^ ((r >> 2) & 1)) << 4)
@@ -58,12 +51,22 @@ struct Raw {
   }
 };
 
-template <int BITS>
+// Shared-memory plan.  PAIR: each CTA of the pair holds 128 of the 256 B
+// rows, which frees room for deeper rings.
+template <int BITS, bool PAIR>
 struct Smem {
+  static constexpr int BR = PAIR ? BN / 2 : BN;          // B rows in this CTA
+  static constexpr int S1 = PAIR ? 6 : 4;                // A stages
+  static constexpr int SR = PAIR ? 4 : 3;                // packed-code stages
+  static constexpr int S2 = PAIR ? 4 : 3;                // dequantised B stages
+  static constexpr int B_STAGE = BR * BK * 2;
+  static constexpr int RAW_STAGE = BR * Raw<BITS>::ROW;
+  static constexpr int SB_STAGE = BR * 8;                // scale pair + bias pair per row
+  static constexpr uint32_t IDESC = tc::idesc_f16_f32(PAIR ? 2 * BM : BM, BN);
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = A_OFF + S1 * A_STAGE;
   static constexpr int RAW_OFF = B_OFF + S2 * B_STAGE;
-  static constexpr int SB_OFF = RAW_OFF + SR * Raw<BITS>::STAGE;
+  static constexpr int SB_OFF = RAW_OFF + SR * RAW_STAGE;
   static constexpr int BAR_OFF = SB_OFF + SR * SB_STAGE;
   static constexpr int N_BARS = 2 * S1 + 2 * SR + 2 * S2 + 4;
   static constexpr int ATAB_OFF = BAR_OFF + N_BARS * 8;   // 2 x 128 A-row pointers
@@ -238,8 +241,9 @@ __device__ __forceinline__ void dequant_chunk(uint4 raw, __half2 s2, __half2 b2,
   }
 }
 
-__device__ __forceinline__ int2 tile_of(const Args& a, int mt) {
-  return a.tiles ? a.tiles[mt] : make_int2(0, mt * BM);
+// (segment, first row within it) of m-tile mt; `rows` rows per m-tile
+__device__ __forceinline__ int2 tile_of(const Args& a, int mt, int rows) {
+  return a.tiles ? a.tiles[mt] : make_int2(0, mt * rows);
 }
 
 // Split dequantisation for the router tiles: w = fmaf(q, scale, bias) in
@@ -270,10 +274,11 @@ __device__ __forceinline__ void dequant_chunk_split(uint4 raw, float s, float b,
            o[4 * k + 3]);
 }
 
-template <int BITS, int EPI>
+template <int BITS, int EPI, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Args a) {
-  using SM = Smem<BITS>;
+  using SM = Smem<BITS, PAIR>;
   using RW = Raw<BITS>;
+  constexpr int S1 = SM::S1, SR = SM::SR, S2 = SM::S2, BR = SM::BR;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = tc::smem_u32(smem);
@@ -290,9 +295,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::TMEM_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // PAIR: the cluster's two CTAs share every work item; rank 0 issues the
+  // MMAs, each CTA holds half of the A rows, half of the B rows and the
+  // accumulator rows of its A half.  The barriers the MMA issuer waits on
+  // (full_a, b_full, tmem_empty) are rank 0's; the others are per CTA.
+  const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   if (threadIdx.x == 0) {
     for (int i = 0; i < S1; ++i) {
-      tc::mbar_init(&full_a[i], 64);
+      tc::mbar_init(&full_a[i], PAIR ? 1 : 64);
       tc::mbar_init(&a_empty[i], 1);
     }
     for (int i = 0; i < SR; ++i) {
@@ -300,21 +312,27 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
       tc::mbar_init(&raw_empty[i], DQ_WARPS * 32);
     }
     for (int i = 0; i < S2; ++i) {
-      tc::mbar_init(&b_full[i], DQ_WARPS * 32);
+      tc::mbar_init(&b_full[i], PAIR ? 2 * DQ_WARPS : DQ_WARPS * 32);
       tc::mbar_init(&b_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&tmem_full[i], 1);
-      tc::mbar_init(&tmem_empty[i], 128);
+      tc::mbar_init(&tmem_empty[i], PAIR ? 256 : 128);
     }
     tc::fence_mbar_init();
   }
   if (warp == 3) {
-    tc::tmem_alloc(tmem_holder, 512);
-    tc::tmem_relinquish();
+    if (PAIR) {
+      tc::tmem_alloc_pair(tmem_holder, 512);
+      tc::tmem_relinquish_pair();
+    } else {
+      tc::tmem_alloc(tmem_holder, 512);
+      tc::tmem_relinquish();
+    }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  if (PAIR) tc::cluster_sync();
+  else __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -322,13 +340,39 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
   const int KB = a.K / BK;
   int* status = a.status;
 
-  if (warp < 2 && a.tma_a) {
+  if (warp < 2 && PAIR) {
+    // ------------------------------------------------------------ A loader (pair)
+    // warp 0: lane 0 of each CTA fetches its 128 rows per stage; rank 0's
+    // stage barrier expects both CTAs' bytes (warp 1 idles)
+    if (warp == 0) {
+      uint32_t it = 0;
+      for (int item = unit0; item < n_items; item += n_units) {
+        const int2 tile = tile_of(a, item / a.n_tiles_n, PAIR ? 2 * BM : BM);
+        const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
+        const int row0 =
+            (sg.a_mode == A_TOKENS ? 0 : sg.row_begin) + tile.y + (int)rank * BM;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const uint32_t s = it % S1, ph = (it / S1) & 1u;
+          if (!tc::mbar_wait(&a_empty[s], ph ^ 1u, status)) goto done;
+          if (lane == 0) {
+            if (rank == 0) tc::mbar_arrive_expect_tx(&full_a[s], (uint32_t)(2 * A_STAGE));
+            tc::tma_load_2d_pair(sbase + SM::A_OFF + s * A_STAGE, &a.tmA, kb * BK, row0,
+                                 tc::mapa_shared(tc::smem_u32(&full_a[s]), 0));
+          }
+          __syncwarp();
+        }
+      }
+      // every release of this CTA's stages has landed before it may exit
+      for (int j = 0; j < S1; ++j, ++it)
+        if (!tc::mbar_wait(&a_empty[it % S1], ((it / S1) & 1u) ^ 1u, status)) goto done;
+    }
+  } else if (warp < 2 && a.tma_a) {
     // ------------------------------------------------------------ A loader (tensor map)
     // thread 0 issues one 128-row x 64-column tile per stage; the other 63
     // threads arrive so the stage barrier keeps its count of 64
     uint32_t it = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const int2 tile = tile_of(a, item / a.n_tiles_n);
+    for (int item = unit0; item < n_items; item += n_units) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n, PAIR ? 2 * BM : BM);
       const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
       const int row0 = sg.a_mode == A_TOKENS ? tile.y : sg.row_begin + tile.y;
       for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -349,8 +393,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
     const int t = threadIdx.x;
     bool dead = false;
     uint32_t it = 0, tl = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++tl) {
-      const int2 tile = tile_of(a, item / a.n_tiles_n);
+    for (int item = unit0; item < n_items; item += n_units, ++tl) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n, PAIR ? 2 * BM : BM);
       const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
       const __half** tab = atab + (tl & 1) * BM;
 #pragma unroll
@@ -387,71 +431,24 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         tc::cp_async_arrive_noinc(&full_a[s]);
       }
     }
-  } else if (warp == 2 && a.tma_b) {
-    // ------------------------------------------------------------ B loader (tensor maps)
-    // lane 0 fetches the codes as two 128-row tiles; every lane fetches the
-    // scale/bias pairs of its 8 rows
-    const int groups = a.K / 64;
-    uint32_t it = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const int2 tile = tile_of(a, item / a.n_tiles_n);
-      const int nt = item % a.n_tiles_n;
-      const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
-      const uint16_t* sp[8];
-      const uint16_t* bp[8];
-      uint32_t ok4[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int r = lane + 32 * j;
-        int src, q;
-        bool ok;
-        b_row<EPI>(sg, nt, r, src, q, ok);
-        if (!ok) q = 0;
-        sp[j] = sg.s[src] + (int64_t)q * groups;
-        bp[j] = sg.b[src] + (int64_t)q * groups;
-        ok4[j] = ok ? 4u : 0u;
-      }
-      // (source, first row) of the two 128-row halves of the tile
-      const int src1 = EPI == EPI_SWIGLU ? 1 : 0;
-      const int y0 = EPI == EPI_SWIGLU ? nt * 128 : nt * BN;
-      const int y1 = EPI == EPI_SWIGLU ? nt * 128 : nt * BN + 128;
-      for (int kb = 0; kb < KB; ++kb, ++it) {
-        const uint32_t s = it % SR, ph = (it / SR) & 1u;
-        if (!tc::mbar_wait(&raw_empty[s], ph ^ 1u, status)) goto done;
-        const uint32_t rst = sbase + SM::RAW_OFF + s * RW::STAGE;
-        const uint32_t sbst = sbase + SM::SB_OFF + s * SB_STAGE;
-        if (lane == 0) {
-          tc::mbar_expect_tx(&raw_full[s], (uint32_t)RW::STAGE);
-          tc::tma_load_3d(rst, &a.tmB[0], kb * (RW::ROW / 4), y0, sg.ex[0], &raw_full[s]);
-          tc::tma_load_3d(rst + 128 * RW::ROW, &a.tmB[src1], kb * (RW::ROW / 4), y1,
-                          sg.ex[src1], &raw_full[s]);
-        }
-        const int kb2 = kb & ~1;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int r = lane + 32 * j;
-          tc::cp_async4(sbst + r * 8, sp[j] + kb2, ok4[j]);
-          tc::cp_async4(sbst + r * 8 + 4, bp[j] + kb2, ok4[j]);
-        }
-        tc::cp_async_arrive_noinc(&raw_full[s]);
-      }
-    }
   } else if (warp == 2) {
     // ------------------------------------------------------------ B loader
-    const int64_t wrow = (int64_t)a.K * BITS / 32;  // words per weight row
+    // this CTA's BR weight rows of the tile: rows rank*BR + (lane + 32 j)
     const int groups = a.K / 64;
+    const int64_t wrow = (int64_t)a.K * BITS / 32;  // words per weight row
+    constexpr int JR = BR / 32;
     uint32_t it = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const int2 tile = tile_of(a, item / a.n_tiles_n);
+    for (int item = unit0; item < n_items; item += n_units) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n, PAIR ? 2 * BM : BM);
       const int nt = item % a.n_tiles_n;
       const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
-      const uint32_t* wp[8];
-      const uint16_t* sp[8];
-      const uint16_t* bp[8];
-      uint32_t ok16[8];
+      const uint32_t* wp[JR];
+      const uint16_t* sp[JR];
+      const uint16_t* bp[JR];
+      uint32_t ok16[JR];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int r = lane + 32 * j;
+      for (int j = 0; j < JR; ++j) {
+        const int r = (int)rank * BR + lane + 32 * j;
         int src, q;
         bool ok;
         b_row<EPI>(sg, nt, r, src, q, ok);
@@ -461,18 +458,41 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         bp[j] = sg.b[src] + (int64_t)q * groups;
         ok16[j] = ok ? 16u : 0u;
       }
+      // tensor-map halves: (source, first row) of tile rows 0..127 and 128..255
+      const int src1 = EPI == EPI_SWIGLU ? 1 : 0;
+      const int y0 = EPI == EPI_SWIGLU ? nt * 128 : nt * BN;
+      const int y1 = EPI == EPI_SWIGLU ? nt * 128 : nt * BN + 128;
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const uint32_t s = it % SR, ph = (it / SR) & 1u;
         if (!tc::mbar_wait(&raw_empty[s], ph ^ 1u, status)) goto done;
-        const uint32_t rst = sbase + SM::RAW_OFF + s * RW::STAGE;
-        const uint32_t sbst = sbase + SM::SB_OFF + s * SB_STAGE;
+        const uint32_t rst = sbase + SM::RAW_OFF + s * SM::RAW_STAGE;
+        const uint32_t sbst = sbase + SM::SB_OFF + s * SM::SB_STAGE;
         const int kb2 = kb & ~1;
+        if (a.tma_b) {
+          if (lane == 0) {
+            tc::mbar_expect_tx(&raw_full[s], (uint32_t)SM::RAW_STAGE);
+            if (PAIR) {
+              const int src = rank ? src1 : 0;
+              tc::tma_load_3d(rst, &a.tmB[src], kb * (RW::ROW / 4), rank ? y1 : y0, sg.ex[src],
+                              &raw_full[s]);
+            } else {
+              tc::tma_load_3d(rst, &a.tmB[0], kb * (RW::ROW / 4), y0, sg.ex[0], &raw_full[s]);
+              tc::tma_load_3d(rst + 128 * RW::ROW, &a.tmB[src1], kb * (RW::ROW / 4), y1,
+                              sg.ex[src1], &raw_full[s]);
+            }
+          }
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < JR; ++j) {
+            const int r = lane + 32 * j;
+#pragma unroll
+            for (int c = 0; c < RW::CHUNKS; ++c)
+              tc::cp_async16(rst + RW::offset(r, c), wp[j] + kb * (RW::ROW / 4) + c * 4, ok16[j]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < JR; ++j) {
           const int r = lane + 32 * j;
-#pragma unroll
-          for (int c = 0; c < RW::CHUNKS; ++c)
-            tc::cp_async16(rst + RW::offset(r, c), wp[j] + kb * (RW::ROW / 4) + c * 4, ok16[j]);
           tc::cp_async4(sbst + r * 8, sp[j] + kb2, ok16[j] ? 4u : 0u);
           tc::cp_async4(sbst + r * 8 + 4, bp[j] + kb2, ok16[j] ? 4u : 0u);
         }
@@ -481,48 +501,64 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------ MMA issuer
-    uint32_t it = 0, tcount = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++tcount) {
-      const uint32_t acc = tcount & 1u, acc_ph = (tcount >> 1) & 1u;
-      if (!tc::mbar_wait(&tmem_empty[acc], acc_ph ^ 1u, status)) goto done;
-      tc::tc_fence_after();
-      const uint32_t d = tmem_base + acc * 256u;
-      for (int kb = 0; kb < KB; ++kb, ++it) {
-        const uint32_t s1 = it % S1, ph1 = (it / S1) & 1u;
-        const uint32_t s2 = it % S2, ph2 = (it / S2) & 1u;
-        if (!tc::mbar_wait(&full_a[s1], ph1, status)) goto done;
-        if (!tc::mbar_wait(&b_full[s2], ph2, status)) goto done;
-        tc::fence_proxy_async_smem();
+    if (!PAIR || rank == 0) {
+      uint32_t it = 0, tcount = 0;
+      for (int item = unit0; item < n_items; item += n_units, ++tcount) {
+        const uint32_t acc = tcount & 1u, acc_ph = (tcount >> 1) & 1u;
+        if (!tc::mbar_wait(&tmem_empty[acc], acc_ph ^ 1u, status)) goto done;
         tc::tc_fence_after();
-        if (lane == 0) {
-          const uint32_t aa = sbase + SM::A_OFF + s1 * A_STAGE;
-          const uint32_t ba = sbase + SM::B_OFF + s2 * B_STAGE;
+        const uint32_t d = tmem_base + acc * 256u;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const uint32_t s1 = it % S1, ph1 = (it / S1) & 1u;
+          const uint32_t s2 = it % S2, ph2 = (it / S2) & 1u;
+          if (!tc::mbar_wait(&full_a[s1], ph1, status)) goto done;
+          if (!tc::mbar_wait(&b_full[s2], ph2, status)) goto done;
+          tc::fence_proxy_async_smem();
+          tc::tc_fence_after();
+          if (lane == 0) {
+            const uint32_t aa = sbase + SM::A_OFF + s1 * A_STAGE;
+            const uint32_t ba = sbase + SM::B_OFF + s2 * SM::B_STAGE;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            tc::mma_f16(d, tc::sw128_kmajor_desc(aa + kk * 32), tc::sw128_kmajor_desc(ba + kk * 32),
-                        IDESC, (kb | kk) != 0);
-          tc::mma_commit(&a_empty[s1]);
-          tc::mma_commit(&b_empty[s2]);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              if (PAIR)
+                tc::mma_f16_pair(d, tc::sw128_kmajor_desc(aa + kk * 32),
+                                 tc::sw128_kmajor_desc(ba + kk * 32), SM::IDESC, (kb | kk) != 0);
+              else
+                tc::mma_f16(d, tc::sw128_kmajor_desc(aa + kk * 32),
+                            tc::sw128_kmajor_desc(ba + kk * 32), SM::IDESC, (kb | kk) != 0);
+            }
+            if (PAIR) {
+              tc::mma_commit_pair(&a_empty[s1], 3);
+              tc::mma_commit_pair(&b_empty[s2], 3);
+            } else {
+              tc::mma_commit(&a_empty[s1]);
+              tc::mma_commit(&b_empty[s2]);
+            }
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+          if (PAIR) tc::mma_commit_pair(&tmem_full[acc], 3);
+          else tc::mma_commit(&tmem_full[acc]);
         }
         __syncwarp();
       }
-      if (lane == 0) tc::mma_commit(&tmem_full[acc]);
-      __syncwarp();
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int i = q * 32 + lane;  // tile row = TMEM lane
+    const int i = q * 32 + lane;  // accumulator row of this CTA = TMEM lane
     uint32_t tcount = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++tcount) {
-      const int2 tile = tile_of(a, item / a.n_tiles_n);
+    for (int item = unit0; item < n_items; item += n_units, ++tcount) {
+      const int2 tile = tile_of(a, item / a.n_tiles_n, PAIR ? 2 * BM : BM);
       const int nt = item % a.n_tiles_n;
       const Seg& sg = a.tiles ? a.segs[tile.x] : a.seg0;
       const uint32_t acc = tcount & 1u, acc_ph = (tcount >> 1) & 1u;
       if (!tc::mbar_wait(&tmem_full[acc], acc_ph, status)) goto done;
       tc::tc_fence_after();
-      const bool ok = tile.y + i < sg.rows;
-      const int64_t m = (int64_t)sg.row_begin + tile.y + i;
+      const int ty = tile.y + (int)rank * BM + i;  // row within the segment
+      const bool ok = ty < sg.rows;
+      const int64_t m = (int64_t)sg.row_begin + ty;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 256u;
       if (EPI == EPI_SWIGLU) {
         __half* out = reinterpret_cast<__half*>(a.out) + m * a.ldo + nt * 128;
@@ -561,8 +597,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           const int col = nt * 128 + c0;
           if (ok && col < sg.n_valid) {
             const int nv = min(32, sg.n_valid - col);
-            for (int k = 0; k < nv; ++k)
-              out[c0 + k] = __uint_as_float(hv[k]) + __uint_as_float(lv[k]);
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k < nv) out[c0 + k] = __uint_as_float(hv[k]) + __uint_as_float(lv[k]);
           }
         }
       } else {
@@ -583,62 +620,86 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
                 dst[k] = make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
             } else {
               const int nv = min(32, sg.n_valid - col);
-              for (int k = 0; k < nv; ++k) out[c0 + k] = __uint_as_float(v[k]);
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (k < nv) out[c0 + k] = __uint_as_float(v[k]);
             }
           }
         }
       }
       tc::tc_fence_before();
-      tc::mbar_arrive(&tmem_empty[acc]);
+      if (PAIR) tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(&tmem_empty[acc]), 0));
+      else tc::mbar_arrive(&tmem_empty[acc]);
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------ dequantiser
-    const int r = threadIdx.x - 256;  // weight row of the tile, 0..255
+    // one weight row per thread, or (PAIR: 128 rows per CTA) half a row
+    const int t = threadIdx.x - 256;
+    const int r = PAIR ? (t & 127) : t;            // row of this CTA's stages
+    const int rg = (int)rank * BR + r;             // row of the 256-row tile
+    constexpr int CPT = PAIR ? (RW::CHUNKS > 1 ? RW::CHUNKS / 2 : 1) : RW::CHUNKS;
+    const int c_lo = PAIR ? (t >> 7) * CPT : 0;   // first raw chunk of this thread
+    const bool active = c_lo < RW::CHUNKS;
     uint32_t it = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    for (int item = unit0; item < n_items; item += n_units) {
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const uint32_t sr = it % SR, phr = (it / SR) & 1u;
         const uint32_t s2 = it % S2, ph2 = (it / S2) & 1u;
         if (!tc::mbar_wait(&raw_full[sr], phr, status)) goto done;
         if (!tc::mbar_wait(&b_empty[s2], ph2 ^ 1u, status)) goto done;
-        const uint32_t rst = sbase + SM::RAW_OFF + sr * RW::STAGE;
-        const uint32_t sbst = sbase + SM::SB_OFF + sr * SB_STAGE;
-        const uint32_t bst = sbase + SM::B_OFF + s2 * B_STAGE;
+        const uint32_t rst = sbase + SM::RAW_OFF + sr * SM::RAW_STAGE;
+        const uint32_t sbst = sbase + SM::SB_OFF + sr * SM::SB_STAGE;
+        const uint32_t bst = sbase + SM::B_OFF + s2 * SM::B_STAGE;
         const int hi = kb & 1;
         const uint2 sb = lds64(sbst + r * 8);
         const uint32_t sbits = hi ? (sb.x >> 16) : (sb.x & 0xFFFFu);
         const uint32_t bbits = hi ? (sb.y >> 16) : (sb.y & 0xFFFFu);
-        uint4 raw[RW::CHUNKS];
+        uint4 raw[CPT];
 #pragma unroll
-        for (int c = 0; c < RW::CHUNKS; ++c) raw[c] = lds128(rst + RW::offset(r, c));
+        for (int c = 0; c < CPT; ++c)
+          raw[c] = active ? lds128(rst + RW::offset(r, c_lo + c)) : make_uint4(0, 0, 0, 0);
         tc::mbar_arrive(&raw_empty[sr]);
-        // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
-        if (EPI == EPI_SPLIT) {
-          const float sf = bf16_bits_to_float((uint16_t)sbits);
-          const float bf = bf16_bits_to_float((uint16_t)bbits);
+        if (active) {
+          // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
+          if (EPI == EPI_SPLIT) {
+            const float sf = bf16_bits_to_float((uint16_t)sbits);
+            const float bf = bf16_bits_to_float((uint16_t)bbits);
 #pragma unroll
-          for (int c = 0; c < RW::CHUNKS; ++c) {
-            if (r < 128) dequant_chunk_split<BITS, false>(raw[c], sf, bf, bst, r, c * (16 / BITS));
-            else dequant_chunk_split<BITS, true>(raw[c], sf, bf, bst, r, c * (16 / BITS));
+            for (int c = 0; c < CPT; ++c) {
+              if (rg < 128)
+                dequant_chunk_split<BITS, false>(raw[c], sf, bf, bst, r, (c_lo + c) * (16 / BITS));
+              else
+                dequant_chunk_split<BITS, true>(raw[c], sf, bf, bst, r, (c_lo + c) * (16 / BITS));
+            }
+          } else {
+            __half2 s2h, b2h;
+            group_h2<BITS>(sbits, bbits, s2h, b2h, status);
+#pragma unroll
+            for (int c = 0; c < CPT; ++c)
+              dequant_chunk<BITS>(raw[c], s2h, b2h, bst, r, (c_lo + c) * (16 / BITS));
           }
-        } else {
-          __half2 s2h, b2h;
-          group_h2<BITS>(sbits, bbits, s2h, b2h, status);
-#pragma unroll
-          for (int c = 0; c < RW::CHUNKS; ++c)
-            dequant_chunk<BITS>(raw[c], s2h, b2h, bst, r, c * (16 / BITS));
         }
         tc::fence_proxy_async_smem();
-        tc::mbar_arrive(&b_full[s2]);
+        if (PAIR) {
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(&b_full[s2]), 0));
+        } else {
+          tc::mbar_arrive(&b_full[s2]);
+        }
       }
     }
+    if (PAIR)
+      for (int j = 0; j < S2; ++j, ++it)
+        if (!tc::mbar_wait(&b_empty[it % S2], ((it / S2) & 1u) ^ 1u, status)) goto done;
   }
 done:
   tc::tc_fence_before();
-  __syncthreads();
+  if (PAIR) tc::cluster_sync();
+  else __syncthreads();
   if (warp == 3) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem_base, 512);
+    if (PAIR) tc::tmem_dealloc_pair(tmem_base, 512);
+    else tc::tmem_dealloc(tmem_base, 512);
   }
 }
 

@@ -119,6 +119,7 @@ struct OffsetsArgs {
   int32_t* blockoff;        // [nb][E]
   int32_t* expert_off;      // [E]
   int32_t nb, E, I, H;
+  int32_t tile_rows;         // rows per m-tile (128, or 256 for CTA pairs)
   gq::Seg* segs_gu;         // [E]
   gq::Seg* segs_dn;         // [E]
   int2* tiles;              // [max tiles]
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ Offset
     }
     cnt[e - e0] = run;
     rsum += run;
-    tsum += (run + gq::BM - 1) / gq::BM;
+    tsum += (run + a.tile_rows - 1) / a.tile_rows;
   }
   part_rows[tid] = rsum;
   part_tiles[tid] = tsum;
@@ -194,8 +195,8 @@ __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ Offset
     d.dest_pairs = 1;
     d.ex[0] = d.ex[1] = e;
     a.segs_dn[e] = d;
-    const int nt = (c + gq::BM - 1) / gq::BM;
-    for (int j = 0; j < nt; ++j) a.tiles[tile + j] = make_int2(e, j * gq::BM);
+    const int nt = (c + a.tile_rows - 1) / a.tile_rows;
+    for (int j = 0; j < nt; ++j) a.tiles[tile + j] = make_int2(e, j * a.tile_rows);
     row += c;
     tile += nt;
   }
@@ -230,35 +231,73 @@ __global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx,
 }
 
 // ------------------------------------------------------------------ gather-QMM launch
-template <int BITS, int EPI>
-cudaError_t launch_gqmm_t(const gq::Args& a, int grid, cudaStream_t st) {
-  constexpr int smem = gq::Smem<BITS>::ALLOC;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gq::k_gqmm<BITS, EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+int sm_count();
+
+// Launch over `units` work items: one CTA per item up to the co-resident
+// count, or (PAIR) one cluster of two CTAs per item up to the co-resident
+// cluster count.
+template <int BITS, int EPI, bool PAIR>
+cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
+  constexpr int smem = gq::Smem<BITS, PAIR>::ALLOC;
+  auto kern = gq::k_gqmm<BITS, EPI, PAIR>;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.blockDim = dim3(gq::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = PAIR ? 1 : 0;
+  static int max_units = 0;
+  if (!max_units) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attr = true;
+    int n = sm_count();
+    if (PAIR) {
+      cfg.gridDim = dim3(2);
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      if (n <= 0) return cudaErrorInvalidConfiguration;
+    }
+    max_units = n;
   }
-  gq::k_gqmm<BITS, EPI><<<grid, gq::THREADS, smem, st>>>(a);
-  return cudaGetLastError();
+  const int n = units < max_units ? units : max_units;
+  if (n <= 0) return cudaSuccess;
+  cfg.gridDim = dim3(PAIR ? 2 * n : n);
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-cudaError_t launch_gqmm(int bits, int epi, const gq::Args& a, int grid, cudaStream_t st) {
-  if (grid <= 0) return cudaSuccess;
+template <bool PAIR>
+cudaError_t launch_gqmm_p(int bits, int epi, const gq::Args& a, int units, cudaStream_t st) {
   if (epi == gq::EPI_SPLIT) {
-    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SPLIT>(a, grid, st);
-    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SPLIT>(a, grid, st);
-    return launch_gqmm_t<2, gq::EPI_SPLIT>(a, grid, st);
+    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SPLIT, PAIR>(a, units, st);
+    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SPLIT, PAIR>(a, units, st);
+    return launch_gqmm_t<2, gq::EPI_SPLIT, PAIR>(a, units, st);
   }
   if (epi == gq::EPI_SWIGLU) {
-    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SWIGLU>(a, grid, st);
-    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SWIGLU>(a, grid, st);
-    return launch_gqmm_t<2, gq::EPI_SWIGLU>(a, grid, st);
+    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SWIGLU, PAIR>(a, units, st);
+    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SWIGLU, PAIR>(a, units, st);
+    return launch_gqmm_t<2, gq::EPI_SWIGLU, PAIR>(a, units, st);
   }
-  if (bits == 8) return launch_gqmm_t<8, gq::EPI_STORE>(a, grid, st);
-  if (bits == 4) return launch_gqmm_t<4, gq::EPI_STORE>(a, grid, st);
-  return launch_gqmm_t<2, gq::EPI_STORE>(a, grid, st);
+  if (bits == 8) return launch_gqmm_t<8, gq::EPI_STORE, PAIR>(a, units, st);
+  if (bits == 4) return launch_gqmm_t<4, gq::EPI_STORE, PAIR>(a, units, st);
+  return launch_gqmm_t<2, gq::EPI_STORE, PAIR>(a, units, st);
+}
+
+// PAIR launches need the A operand as tensor-map tiles (a.tma_a).
+cudaError_t launch_gqmm(int bits, int epi, bool pair, const gq::Args& a, int64_t units,
+                        cudaStream_t st) {
+  if (units <= 0) return cudaSuccess;
+  const int u = units > (1 << 30) ? (1 << 30) : (int)units;
+  if (pair) {
+    if (!a.tma_a) return cudaErrorInvalidValue;
+    return launch_gqmm_p<true>(bits, epi, a, u, st);
+  }
+  return launch_gqmm_p<false>(bits, epi, a, u, st);
 }
 
 int sm_count() {
@@ -457,7 +496,11 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
   __half* h_sh = (__half*)(base + lay.h_sh);
   float* yrows = (float*)(base + lay.y);
   const int sms = sm_count();
-  const int mtiles = (M + gq::BM - 1) / gq::BM;
+  // CTA pairs (m-tiles of 256 rows) whenever the operands can be tensor-map
+  // tiles; every gather-QMM launch of the call uses the same tiling
+  const bool pair = encode_fn() != nullptr;
+  const int TR = pair ? 2 * gq::BM : gq::BM;
+  const int mtiles = (M + TR - 1) / TR;
 
   // 1. fp16 copy of the tokens (range-checked)
   {
@@ -493,12 +536,12 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     const int nt = (rs.n_valid + 127) / 128;
     const gq::Args a = gemm_args(rs, nt, H, x16, H, logits, lay.ld_logits);
     const int items = mtiles * nt;
-    PCK(launch_gqmm(L->router.bits, gq::EPI_SPLIT, a, items < sms ? items : sms, st));
+    PCK(launch_gqmm(L->router.bits, gq::EPI_SPLIT, pair, a, items, st));
   }
   if (L->has_shared && (idx_in || !sgr)) {
     const gq::Seg gs = seg_single(L->sh_expert_gate, nullptr, M, gq::A_TOKENS);
     const gq::Args a = gemm_args(gs, 1, H, x16, H, logits + E, lay.ld_logits);
-    PCK(launch_gqmm(L->sh_expert_gate.bits, gq::EPI_SPLIT, a, mtiles < sms ? mtiles : sms, st));
+    PCK(launch_gqmm(L->sh_expert_gate.bits, gq::EPI_SPLIT, pair, a, mtiles, st));
   }
 
   // 3. routing
@@ -533,6 +576,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
   oa.E = E;
   oa.I = I;
   oa.H = H;
+  oa.tile_rows = TR;
   oa.segs_gu = segs_gu;
   oa.segs_dn = segs_dn;
   oa.tiles = tiles;
@@ -545,7 +589,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
   k_scatter<<<lay.nb, 32, hsmem, st>>>(idx, n, E, expert_off, blockoff, sorted, status);
   PCK(cudaGetLastError());
 
-  const int64_t max_mtiles = n / gq::BM + E;
+  const int64_t max_mtiles = n / TR + E;
   // 5. gate/up + SwiGLU for the routed experts (the profiled kernel), then the shared expert
   {
     gq::Args a;
@@ -574,7 +618,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.tma_b = code_tensor_map(&a.tmB[0], L->gate, E) && code_tensor_map(&a.tmB[1], L->up, E);
     const int64_t items = max_mtiles * a.n_tiles_n;
     if (profile_mark(true, st) != cudaSuccess) return MOEQ_ERR_CUDA;
-    PCK(launch_gqmm(L->gate.bits, gq::EPI_SWIGLU, a, items < sms ? (int)items : sms, st));
+    PCK(launch_gqmm(L->gate.bits, gq::EPI_SWIGLU, pair, a, items, st));
     if (profile_mark(false, st) != cudaSuccess) return MOEQ_ERR_CUDA;
   }
   if (L->has_shared) {
@@ -584,7 +628,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     gq::Args a = gemm_args(gs, Is / 128, H, x16, H, h_sh, Is);
     a.tma_b = code_tensor_map(&a.tmB[0], L->sh_gate, 1) && code_tensor_map(&a.tmB[1], L->sh_up, 1);
     const int items = mtiles * (Is / 128);
-    PCK(launch_gqmm(L->sh_gate.bits, gq::EPI_SWIGLU, a, items < sms ? items : sms, st));
+    PCK(launch_gqmm(L->sh_gate.bits, gq::EPI_SWIGLU, pair, a, items, st));
   }
   // 6. down projections into pair order (shared rows after the M*K pair rows)
   {
@@ -605,7 +649,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.status = status;
     a.tma_b = code_tensor_map(&a.tmB[0], L->down, E);
     const int64_t items = max_mtiles * a.n_tiles_n;
-    PCK(launch_gqmm(L->down.bits, gq::EPI_STORE, a, items < sms ? (int)items : sms, st));
+    PCK(launch_gqmm(L->down.bits, gq::EPI_STORE, pair, a, items, st));
   }
   if (L->has_shared) {
     const int Is = L->sh_gate.out_dim;
@@ -614,7 +658,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
                            yrows + n * (int64_t)H, H);
     a.tma_b = code_tensor_map(&a.tmB[0], L->sh_down, 1);
     const int items = mtiles * ((H + gq::BN - 1) / gq::BN);
-    PCK(launch_gqmm(L->sh_down.bits, gq::EPI_STORE, a, items < sms ? items : sms, st));
+    PCK(launch_gqmm(L->sh_down.bits, gq::EPI_STORE, pair, a, items, st));
   }
   // 7. combine in k order (+ sigmoid-gated shared expert, + residual)
   PCK(launch_combine(yrows, wts, sigma, L->has_shared, residual, y, M, K, H, st));
