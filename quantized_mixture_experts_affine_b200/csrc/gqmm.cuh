@@ -124,6 +124,14 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
                : "memory");
 }
 
+// 32-byte global store (32-byte aligned address): one full sector per lane.
+__device__ __forceinline__ void stg256(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t a4, uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a0), "r"(a1),
+               "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
@@ -579,10 +587,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
               bad |= !(fabsf(h0) <= 65504.0f) || !(fabsf(h1) <= 65504.0f);
               o[k] = h2u(__floats2half2_rn(h0, h1));
             }
-            uint4* dst = reinterpret_cast<uint4*>(out + c0);
+            if ((((uintptr_t)(out + c0)) & 31) == 0) {
+              stg256(out + c0, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+              stg256(out + c0 + 16, o[8], o[9], o[10], o[11], o[12], o[13], o[14], o[15]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(out + c0);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+            }
           }
         }
         if (bad) set_status(status, MOEQ_ERR_RANGE);
@@ -613,7 +626,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           tc::tmem_wait_ld();
           const int col = nt * BN + c0;
           if (ok && col < sg.n_valid) {
-            if (col + 32 <= sg.n_valid && (((uintptr_t)(out + c0)) & 15) == 0) {
+            if (col + 32 <= sg.n_valid && (((uintptr_t)(out + c0)) & 31) == 0) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                stg256(out + c0 + 8 * k, v[8 * k], v[8 * k + 1], v[8 * k + 2], v[8 * k + 3],
+                       v[8 * k + 4], v[8 * k + 5], v[8 * k + 6], v[8 * k + 7]);
+            } else if (col + 32 <= sg.n_valid && (((uintptr_t)(out + c0)) & 15) == 0) {
               uint4* dst = reinterpret_cast<uint4*>(out + c0);
 #pragma unroll
               for (int k = 0; k < 8; ++k)

@@ -18,7 +18,7 @@ namespace moeq {
 
 namespace {
 
-constexpr int kSortChunk = 2048;  // pairs per sort block
+constexpr int kSortChunk = 512;  // pairs per sort block
 
 // ------------------------------------------------------------------ tokens to fp16
 __global__ void __launch_bounds__(256) k_to_f16(const uint16_t* __restrict__ x, int64_t n8,
@@ -47,10 +47,27 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x
                                                      const int32_t* __restrict__ sorted, int K,
                                                      int64_t n, int row_chunks,
                                                      uint4* __restrict__ out) {
-  for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
-    const int64_t src = sorted[r] / K;
-    for (int c = threadIdx.x; c < row_chunks; c += blockDim.x)
-      out[r * row_chunks + c] = x16[src * row_chunks + c];
+  // one warp per row: every lane's loads of the row in flight, then stores
+  constexpr int U = 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n;
+       r += warps) {
+    const uint4* src = x16 + (int64_t)(sorted[r] / K) * row_chunks;
+    uint4* dst = out + r * row_chunks;
+    for (int c0 = 0; c0 < row_chunks; c0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_chunks) v[u] = src[c];
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_chunks) dst[c] = v[u];
+      }
+    }
   }
 }
 
@@ -111,12 +128,14 @@ __global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, i
   for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x)
     atomicAdd(&hist[checked_expert(idx, p, E, status)], 1);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) blockhist[(int64_t)blockIdx.x * E + e] = hist[e];
+  // expert-major [E][nb]: one expert's block counts are contiguous
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    blockhist[(int64_t)e * gridDim.x + blockIdx.x] = hist[e];
 }
 
 struct OffsetsArgs {
   const int32_t* blockhist;
-  int32_t* blockoff;        // [nb][E]
+  int32_t* blockoff;        // [E][nb]
   int32_t* expert_off;      // [E]
   int32_t nb, E, I, H;
   int32_t tile_rows;         // rows per m-tile (128, or 256 for CTA pairs)
@@ -130,39 +149,77 @@ struct OffsetsArgs {
 // One CTA: per-expert block offsets and counts, expert offsets (exclusive
 // scan), one gate/up and one down segment per expert and the m-tile list.
 __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ OffsetsArgs a) {
-  __shared__ int32_t part_rows[1024], part_tiles[1024];
+  __shared__ int32_t count_s[4096];  // pairs per expert (E <= 4096)
+  __shared__ int32_t part_rows[64], part_tiles[64];
   const int E = a.E, tid = threadIdx.x;
+  const int lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  // 1. per expert (one warp at a time): exclusive scan of its block counts
+  for (int e = wid; e < E; e += nw) {
+    const int32_t* hrow = a.blockhist + (int64_t)e * a.nb;
+    int32_t* orow = a.blockoff + (int64_t)e * a.nb;
+    int carry = 0;
+    for (int b0 = 0; b0 < a.nb; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < a.nb ? hrow[b] : 0;
+      int inc = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+      }
+      if (b < a.nb) orow[b] = carry + inc - v;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) count_s[e] = carry;
+  }
+  __syncthreads();
+  // 2. exclusive scan of (rows, m-tiles) over the experts: each thread sums
+  //    its experts, then shuffles within warps and over the warp totals
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int e0 = tid * per, e1 = min(E, e0 + per);
   int32_t cnt[4];  // E <= 4096 -> at most 4 experts per thread
   int rsum = 0, tsum = 0;
   for (int e = e0; e < e1; ++e) {
-    int run = 0;
-    for (int b = 0; b < a.nb; ++b) {
-      a.blockoff[(int64_t)b * E + e] = run;
-      run += a.blockhist[(int64_t)b * E + e];
-    }
+    const int run = count_s[e];
     cnt[e - e0] = run;
     rsum += run;
     tsum += (run + a.tile_rows - 1) / a.tile_rows;
   }
-  part_rows[tid] = rsum;
-  part_tiles[tid] = tsum;
-  __syncthreads();
-  // exclusive scan over threads (serial by one warp's lane 0 in chunks; 1024 entries)
-  if (tid == 0) {
-    int r = 0, t = 0;
-    for (int i = 0; i < (int)blockDim.x; ++i) {
-      const int pr = part_rows[i], pt = part_tiles[i];
-      part_rows[i] = r;
-      part_tiles[i] = t;
-      r += pr;
-      t += pt;
+  int ir = rsum, itl = tsum;  // inclusive within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int vr = __shfl_up_sync(0xffffffffu, ir, o);
+    const int vt = __shfl_up_sync(0xffffffffu, itl, o);
+    if (lane >= o) {
+      ir += vr;
+      itl += vt;
     }
-    *a.n_tiles = t;
+  }
+  if (lane == 31) {
+    part_rows[wid] = ir;
+    part_tiles[wid] = itl;
   }
   __syncthreads();
-  int row = part_rows[tid], tile = part_tiles[tid];
+  if (wid == 0) {
+    int wr = lane < nw ? part_rows[lane] : 0, wt = lane < nw ? part_tiles[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vr = __shfl_up_sync(0xffffffffu, wr, o);
+      const int vt = __shfl_up_sync(0xffffffffu, wt, o);
+      if (lane >= o) {
+        wr += vr;
+        wt += vt;
+      }
+    }
+    if (lane < nw) {
+      part_rows[32 + lane] = wr;  // inclusive over warps
+      part_tiles[32 + lane] = wt;
+    }
+    if (lane == nw - 1) *a.n_tiles = wt;
+  }
+  __syncthreads();
+  int row = ir - rsum + (wid ? part_rows[32 + wid - 1] : 0);
+  int tile = itl - tsum + (wid ? part_tiles[32 + wid - 1] : 0);
   for (int e = e0; e < e1; ++e) {
     const int c = cnt[e - e0];
     a.expert_off[e] = row;
@@ -207,13 +264,13 @@ __global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx,
                                                 const int32_t* __restrict__ expert_off,
                                                 const int32_t* __restrict__ blockoff,
                                                 int32_t* __restrict__ sorted_pair, int* status) {
-  extern __shared__ int32_t run[];
+  extern __shared__ int32_t run[];  // next sorted position of each expert
   const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) run[e] = 0;
+  for (int e = lane; e < E; e += 32)
+    run[e] = expert_off[e] + blockoff[(int64_t)e * gridDim.x + blockIdx.x];
   __syncwarp();
   const int64_t p0 = (int64_t)blockIdx.x * kSortChunk;
   const int64_t p1 = min(n, p0 + kSortChunk);
-  const int32_t* boff = blockoff + (int64_t)blockIdx.x * E;
   for (int64_t base = p0; base < p1; base += 32) {
     const int64_t p = base + lane;
     const bool on = p < p1;
@@ -221,8 +278,7 @@ __global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx,
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (on) {
       const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int64_t pos = (int64_t)expert_off[e] + boff[e] + run[e] + rank;
-      sorted_pair[pos] = (int32_t)p;
+      sorted_pair[(int64_t)run[e] + rank] = (int32_t)p;
     }
     __syncwarp();
     if (on && lane == __ffs(peers) - 1) run[e] += __popc(peers);
@@ -605,7 +661,8 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     __half* a_sorted = (__half*)(base + lay.a_sorted);
     set_a_tensor_map(a, a_sorted, n, H, H);
     if (a.tma_a) {
-      int64_t grid = n < (int64_t)sms * 16 ? n : (int64_t)sms * 16;
+      int64_t grid = (n + 7) / 8;
+      if (grid > (int64_t)sms * 16) grid = (int64_t)sms * 16;
       k_gather_rows<<<(int)grid, 256, 0, st>>>((const uint4*)x16, sorted, K, n, H / 8,
                                                (uint4*)a_sorted);
       PCK(cudaGetLastError());
