@@ -115,6 +115,7 @@ struct Args {
   int32_t topk;
   void* out;
   int64_t ldo;              // elements
+  int32_t out_f16;          // STORE: fp16 output rows (range-checked) instead of fp32
   int* status;
 };
 
@@ -615,6 +616,37 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
               if (k < nv) out[c0 + k] = __uint_as_float(hv[k]) + __uint_as_float(lv[k]);
           }
         }
+      } else if (a.out_f16) {
+        int64_t dest = m;
+        if (ok && sg.dest_pairs) dest = a.sorted_pair[m];
+        __half* out = reinterpret_cast<__half*>(a.out) + dest * a.ldo + nt * BN;
+        bool bad = false;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tc::tmem_ld32(tb + c0, v);
+          tc::tmem_wait_ld();
+          const int col = nt * BN + c0;
+          if (ok && col < sg.n_valid) {
+            uint32_t o[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float f0 = __uint_as_float(v[2 * k]), f1 = __uint_as_float(v[2 * k + 1]);
+              bad |= !(fabsf(f0) <= 65504.0f) || !(fabsf(f1) <= 65504.0f);
+              o[k] = h2u(__floats2half2_rn(f0, f1));
+            }
+            if (col + 32 <= sg.n_valid && (((uintptr_t)(out + c0)) & 31) == 0) {
+              stg256(out + c0, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+              stg256(out + c0 + 16, o[8], o[9], o[10], o[11], o[12], o[13], o[14], o[15]);
+            } else {
+              const int nv = min(32, sg.n_valid - col);
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (k < nv) out[c0 + k] = __float2half_rn(__uint_as_float(v[k]));
+            }
+          }
+        }
+        if (bad) set_status(status, MOEQ_ERR_RANGE);
       } else {
         int64_t dest = m;
         if (ok && sg.dest_pairs) dest = a.sorted_pair[m];

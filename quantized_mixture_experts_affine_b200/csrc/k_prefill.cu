@@ -71,6 +71,46 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x
   }
 }
 
+// y[t] = sum_k w[t][k] d[t*K + k] (+ sigma[t] d[M*K + t]) (+ residual[t]), k in
+// order, from fp16 down rows in pair order; eight columns per thread.
+__global__ void __launch_bounds__(256) k_combine_h(const uint4* __restrict__ d,
+                                                   const float* __restrict__ w,
+                                                   const float* __restrict__ sigma,
+                                                   int has_shared,
+                                                   const float* __restrict__ residual,
+                                                   float* __restrict__ y, int M, int K, int H) {
+  const int H8 = H >> 3;
+  const int64_t total = (int64_t)M * H8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / H8);
+    const int c8 = (int)(i - (int64_t)t * H8);
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    auto add = [&](float s, const uint4 v) {
+      const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        acc[2 * j] = fmaf(s, f.x, acc[2 * j]);
+        acc[2 * j + 1] = fmaf(s, f.y, acc[2 * j + 1]);
+      }
+    };
+    for (int k = 0; k < K; ++k) add(w[(int64_t)t * K + k], d[((int64_t)t * K + k) * H8 + c8]);
+    if (has_shared) add(sigma[t], d[((int64_t)M * K + t) * H8 + c8]);
+    if (residual) {
+      const float4* r = reinterpret_cast<const float4*>(residual + (int64_t)t * H) + 2 * c8;
+      const float4 r0 = r[0], r1 = r[1];
+      acc[0] += r0.x; acc[1] += r0.y; acc[2] += r0.z; acc[3] += r0.w;
+      acc[4] += r1.x; acc[5] += r1.y; acc[6] += r1.z; acc[7] += r1.w;
+    }
+    float4* o = reinterpret_cast<float4*>(y + (int64_t)t * H) + 2 * c8;
+    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
 // ------------------------------------------------------------------ routing (strided logits)
 __global__ void __launch_bounds__(256) k_route_prefill(const float* __restrict__ logits, int64_t ld,
                                                        int M, int E, int K, int renorm,
@@ -434,7 +474,7 @@ PrefillWs prefill_ws(const moeq_layer* L, int M) {
   w.a_sorted = c.take((size_t)n * H * 2);
   w.h = c.take((size_t)n * I * 2);
   w.h_sh = c.take((size_t)M * Is * 2);
-  w.y = c.take((size_t)(n + M) * H * 4);
+  w.y = c.take((size_t)(n + M) * H * 2);  // fp16 down rows, pair order then shared
   w.total = c.off;
   return w;
 }
@@ -550,7 +590,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
   int32_t* sorted = (int32_t*)(base + lay.sorted);
   __half* h = (__half*)(base + lay.h);
   __half* h_sh = (__half*)(base + lay.h_sh);
-  float* yrows = (float*)(base + lay.y);
+  __half* yrows = (__half*)(base + lay.y);
   const int sms = sm_count();
   // CTA pairs (m-tiles of 256 rows) whenever the operands can be tensor-map
   // tiles; every gather-QMM launch of the call uses the same tiling
@@ -703,6 +743,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.topk = K;
     a.out = yrows;
     a.ldo = H;
+    a.out_f16 = 1;
     a.status = status;
     a.tma_b = code_tensor_map(&a.tmB[0], L->down, E);
     const int64_t items = max_mtiles * a.n_tiles_n;
@@ -713,12 +754,20 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     const gq::Seg ds = seg_single(L->sh_down, nullptr, M, gq::A_ROWS);
     gq::Args a = gemm_args(ds, (H + gq::BN - 1) / gq::BN, Is, h_sh, Is,
                            yrows + n * (int64_t)H, H);
+    a.out_f16 = 1;
     a.tma_b = code_tensor_map(&a.tmB[0], L->sh_down, 1);
     const int items = mtiles * ((H + gq::BN - 1) / gq::BN);
     PCK(launch_gqmm(L->sh_down.bits, gq::EPI_STORE, pair, a, items, st));
   }
   // 7. combine in k order (+ sigmoid-gated shared expert, + residual)
-  PCK(launch_combine(yrows, wts, sigma, L->has_shared, residual, y, M, K, H, st));
+  {
+    const int64_t total = (int64_t)M * (H / 8);
+    int64_t grid = (total + 255) / 256;
+    if (grid > (int64_t)sms * 16) grid = (int64_t)sms * 16;
+    k_combine_h<<<(int)grid, 256, 0, st>>>((const uint4*)yrows, wts, sigma, L->has_shared,
+                                           residual, y, M, K, H);
+    PCK(cudaGetLastError());
+  }
   return MOEQ_OK;
 }
 
