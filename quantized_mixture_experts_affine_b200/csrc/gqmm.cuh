@@ -56,18 +56,24 @@ struct Raw {
 template <int BITS, bool PAIR>
 struct Smem {
   static constexpr int BR = PAIR ? BN / 2 : BN;          // B rows in this CTA
-  static constexpr int S1 = PAIR ? 6 : 4;                // A stages
+  static constexpr int S1 = PAIR ? 6 : 3;                // A stages
   static constexpr int SR = PAIR ? 4 : 3;                // packed-code stages
   static constexpr int S2 = PAIR ? 4 : 3;                // dequantised B stages
   static constexpr int B_STAGE = BR * BK * 2;
   static constexpr int RAW_STAGE = BR * Raw<BITS>::ROW;
-  static constexpr int SB_STAGE = BR * 8;                // scale pair + bias pair per row
+  // scale/bias windows of up to 8 groups (k-blocks): per row 16 bytes of
+  // scales, then 16 of biases.  Two window buffers suffice: the dequantiser
+  // reads a window in its first k-block, before releasing that k-block's raw
+  // stage, and the loader refills the buffer two windows (>= 4 k-blocks)
+  // later, after waiting for the release of the k-block SR (<= 4) back.
+  static constexpr int SB_WIN = BR * 32;
+  static constexpr int NWB = 2;
   static constexpr uint32_t IDESC = tc::idesc_f16_f32(PAIR ? 2 * BM : BM, BN);
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = A_OFF + S1 * A_STAGE;
   static constexpr int RAW_OFF = B_OFF + S2 * B_STAGE;
   static constexpr int SB_OFF = RAW_OFF + SR * RAW_STAGE;
-  static constexpr int BAR_OFF = SB_OFF + SR * SB_STAGE;
+  static constexpr int BAR_OFF = SB_OFF + NWB * SB_WIN;
   static constexpr int N_BARS = 2 * S1 + 2 * SR + 2 * S2 + 4;
   static constexpr int ATAB_OFF = BAR_OFF + N_BARS * 8;   // 2 x 128 A-row pointers
   static constexpr int TMEM_OFF = ATAB_OFF + 2 * BM * 8;
@@ -116,6 +122,8 @@ struct Args {
   void* out;
   int64_t ldo;              // elements
   int32_t out_f16;          // STORE: fp16 output rows (range-checked) instead of fp32
+  int32_t sb_w;             // groups per scale/bias window copy: 8, 4 or 2 (dividing K/64;
+                            // scale/bias rows aligned to 2*sb_w bytes)
   int* status;
 };
 
@@ -138,6 +146,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
 
@@ -444,6 +458,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
     // ------------------------------------------------------------ B loader
     // this CTA's BR weight rows of the tile: rows rank*BR + (lane + 32 j)
     const int groups = a.K / 64;
+    const int W = a.sb_w, wl = W == 8 ? 3 : W == 4 ? 2 : 1;
     const int64_t wrow = (int64_t)a.K * BITS / 32;  // words per weight row
     constexpr int JR = BR / 32;
     uint32_t it = 0;
@@ -475,8 +490,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         const uint32_t s = it % SR, ph = (it / SR) & 1u;
         if (!tc::mbar_wait(&raw_empty[s], ph ^ 1u, status)) goto done;
         const uint32_t rst = sbase + SM::RAW_OFF + s * SM::RAW_STAGE;
-        const uint32_t sbst = sbase + SM::SB_OFF + s * SM::SB_STAGE;
-        const int kb2 = kb & ~1;
+        // a new scale/bias window every sb_w k-blocks (windows counted over
+        // the whole item loop, like the dequantiser)
+        const bool new_win = (kb & (W - 1)) == 0;
+        const uint32_t sbw = sbase + SM::SB_OFF + ((it >> wl) % SM::NWB) * SM::SB_WIN;
         if (a.tma_b) {
           if (lane == 0) {
             tc::mbar_expect_tx(&raw_full[s], (uint32_t)SM::RAW_STAGE);
@@ -499,11 +516,22 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
               tc::cp_async16(rst + RW::offset(r, c), wp[j] + kb * (RW::ROW / 4) + c * 4, ok16[j]);
           }
         }
+        if (new_win) {
 #pragma unroll
-        for (int j = 0; j < JR; ++j) {
-          const int r = lane + 32 * j;
-          tc::cp_async4(sbst + r * 8, sp[j] + kb2, ok16[j] ? 4u : 0u);
-          tc::cp_async4(sbst + r * 8 + 4, bp[j] + kb2, ok16[j] ? 4u : 0u);
+          for (int j = 0; j < JR; ++j) {
+            const int r = lane + 32 * j;
+            const uint32_t d = sbw + r * 32;
+            if (W == 8) {
+              tc::cp_async16(d, sp[j] + kb, ok16[j]);
+              tc::cp_async16(d + 16, bp[j] + kb, ok16[j]);
+            } else if (W == 4) {
+              tc::cp_async8(d, sp[j] + kb, ok16[j] ? 8u : 0u);
+              tc::cp_async8(d + 16, bp[j] + kb, ok16[j] ? 8u : 0u);
+            } else {
+              tc::cp_async4(d, sp[j] + kb, ok16[j] ? 4u : 0u);
+              tc::cp_async4(d + 16, bp[j] + kb, ok16[j] ? 4u : 0u);
+            }
+          }
         }
         tc::cp_async_arrive_noinc(&raw_full[s]);
       }
@@ -522,7 +550,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           const uint32_t s2 = it % S2, ph2 = (it / S2) & 1u;
           if (!tc::mbar_wait(&full_a[s1], ph1, status)) goto done;
           if (!tc::mbar_wait(&b_full[s2], ph2, status)) goto done;
-          tc::fence_proxy_async_smem();
+          // the dequantisers fenced their shared-memory writes to the async
+          // proxy before arriving on b_full
           tc::tc_fence_after();
           if (lane == 0) {
             const uint32_t aa = sbase + SM::A_OFF + s1 * A_STAGE;
@@ -690,6 +719,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
     constexpr int CPT = PAIR ? (RW::CHUNKS > 1 ? RW::CHUNKS / 2 : 1) : RW::CHUNKS;
     const int c_lo = PAIR ? (t >> 7) * CPT : 0;   // first raw chunk of this thread
     const bool active = c_lo < RW::CHUNKS;
+    const int W = a.sb_w, wl = W == 8 ? 3 : W == 4 ? 2 : 1;
+    uint4 swin = make_uint4(0u, 0u, 0u, 0u), bwin = swin;  // scale/bias window (bf16 pairs)
     uint32_t it = 0;
     for (int item = unit0; item < n_items; item += n_units) {
       for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -698,12 +729,28 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         if (!tc::mbar_wait(&raw_full[sr], phr, status)) goto done;
         if (!tc::mbar_wait(&b_empty[s2], ph2 ^ 1u, status)) goto done;
         const uint32_t rst = sbase + SM::RAW_OFF + sr * SM::RAW_STAGE;
-        const uint32_t sbst = sbase + SM::SB_OFF + sr * SM::SB_STAGE;
         const uint32_t bst = sbase + SM::B_OFF + s2 * SM::B_STAGE;
-        const int hi = kb & 1;
-        const uint2 sb = lds64(sbst + r * 8);
-        const uint32_t sbits = hi ? (sb.x >> 16) : (sb.x & 0xFFFFu);
-        const uint32_t bbits = hi ? (sb.y >> 16) : (sb.y & 0xFFFFu);
+        if ((kb & (W - 1)) == 0) {
+          // this row's window of W scales and W biases, kept in registers
+          const uint32_t sbw =
+              sbase + SM::SB_OFF + ((it >> wl) % SM::NWB) * SM::SB_WIN + r * 32;
+          if (W == 8) {
+            swin = lds128(sbw);
+            bwin = lds128(sbw + 16);
+          } else if (W == 4) {
+            const uint2 sv = lds64(sbw), bv = lds64(sbw + 16);
+            swin = make_uint4(sv.x, sv.y, 0u, 0u);
+            bwin = make_uint4(bv.x, bv.y, 0u, 0u);
+          } else {
+            swin = make_uint4(lds32(sbw), 0u, 0u, 0u);
+            bwin = make_uint4(lds32(sbw + 16), 0u, 0u, 0u);
+          }
+        }
+        const int j = kb & (W - 1);
+        const uint32_t sw2 = (j & 4) ? ((j & 2) ? swin.w : swin.z) : ((j & 2) ? swin.y : swin.x);
+        const uint32_t bw2 = (j & 4) ? ((j & 2) ? bwin.w : bwin.z) : ((j & 2) ? bwin.y : bwin.x);
+        const uint32_t sbits = (j & 1) ? (sw2 >> 16) : (sw2 & 0xFFFFu);
+        const uint32_t bbits = (j & 1) ? (bw2 >> 16) : (bw2 & 0xFFFFu);
         uint4 raw[CPT];
 #pragma unroll
         for (int c = 0; c < CPT; ++c)

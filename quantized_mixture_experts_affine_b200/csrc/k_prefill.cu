@@ -536,6 +536,21 @@ bool code_tensor_map(CUtensorMap* m, const moeq_qtensor& t, int n_mat) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Groups per scale/bias window copy of a gather-QMM launch over tensors ts
+// (reduction length K): the largest of 8, 4, 2 that divides K/64 and keeps
+// every matrix's scale and bias rows aligned to the copy size.
+int sb_window(const moeq_qtensor* const* ts, int n, int K) {
+  const int groups = K / 64;
+  for (int W = 8; W > 2; W >>= 1) {
+    bool ok = groups % W == 0;
+    for (int i = 0; i < n && ok; ++i)
+      ok = ((uintptr_t)ts[i]->scales % (2 * W)) == 0 && ((uintptr_t)ts[i]->biases % (2 * W)) == 0 &&
+           (ts[i]->expert_stride_sb * 2) % (2 * W) == 0;
+    if (ok) return W;
+  }
+  return 2;
+}
+
 moeq_status check_prefill(const moeq_layer* L) {
   const moeq_qtensor* ts[8] = {&L->router, &L->gate, &L->up, &L->down,
                                &L->sh_gate, &L->sh_up, &L->sh_down, &L->sh_expert_gate};
@@ -630,13 +645,17 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     // hi/lo split weights: fp32-accurate logits for the top-K decision
     const gq::Seg rs = seg_single(L->router, sgr ? &L->sh_expert_gate : nullptr, M, gq::A_TOKENS);
     const int nt = (rs.n_valid + 127) / 128;
-    const gq::Args a = gemm_args(rs, nt, H, x16, H, logits, lay.ld_logits);
+    gq::Args a = gemm_args(rs, nt, H, x16, H, logits, lay.ld_logits);
+    const moeq_qtensor* ts[2] = {&L->router, &L->sh_expert_gate};
+    a.sb_w = sb_window(ts, sgr ? 2 : 1, H);
     const int items = mtiles * nt;
     PCK(launch_gqmm(L->router.bits, gq::EPI_SPLIT, pair, a, items, st));
   }
   if (L->has_shared && (idx_in || !sgr)) {
     const gq::Seg gs = seg_single(L->sh_expert_gate, nullptr, M, gq::A_TOKENS);
-    const gq::Args a = gemm_args(gs, 1, H, x16, H, logits + E, lay.ld_logits);
+    gq::Args a = gemm_args(gs, 1, H, x16, H, logits + E, lay.ld_logits);
+    const moeq_qtensor* ts[1] = {&L->sh_expert_gate};
+    a.sb_w = sb_window(ts, 1, H);
     PCK(launch_gqmm(L->sh_expert_gate.bits, gq::EPI_SPLIT, pair, a, mtiles, st));
   }
 
@@ -713,6 +732,8 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.ldo = I;
     a.status = status;
     a.tma_b = code_tensor_map(&a.tmB[0], L->gate, E) && code_tensor_map(&a.tmB[1], L->up, E);
+    const moeq_qtensor* ts[2] = {&L->gate, &L->up};
+    a.sb_w = sb_window(ts, 2, H);
     const int64_t items = max_mtiles * a.n_tiles_n;
     if (profile_mark(true, st) != cudaSuccess) return MOEQ_ERR_CUDA;
     PCK(launch_gqmm(L->gate.bits, gq::EPI_SWIGLU, pair, a, items, st));
@@ -724,6 +745,8 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     gs.n0 = Is;
     gq::Args a = gemm_args(gs, Is / 128, H, x16, H, h_sh, Is);
     a.tma_b = code_tensor_map(&a.tmB[0], L->sh_gate, 1) && code_tensor_map(&a.tmB[1], L->sh_up, 1);
+    const moeq_qtensor* ts[2] = {&L->sh_gate, &L->sh_up};
+    a.sb_w = sb_window(ts, 2, H);
     const int items = mtiles * (Is / 128);
     PCK(launch_gqmm(L->sh_gate.bits, gq::EPI_SWIGLU, pair, a, items, st));
   }
@@ -746,6 +769,8 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.out_f16 = 1;
     a.status = status;
     a.tma_b = code_tensor_map(&a.tmB[0], L->down, E);
+    const moeq_qtensor* ts[1] = {&L->down};
+    a.sb_w = sb_window(ts, 1, I);
     const int64_t items = max_mtiles * a.n_tiles_n;
     PCK(launch_gqmm(L->down.bits, gq::EPI_STORE, pair, a, items, st));
   }
@@ -756,6 +781,8 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
                            yrows + n * (int64_t)H, H);
     a.out_f16 = 1;
     a.tma_b = code_tensor_map(&a.tmB[0], L->sh_down, 1);
+    const moeq_qtensor* ts[1] = {&L->sh_down};
+    a.sb_w = sb_window(ts, 1, Is);
     const int items = mtiles * ((H + gq::BN - 1) / gq::BN);
     PCK(launch_gqmm(L->sh_down.bits, gq::EPI_STORE, pair, a, items, st));
   }
