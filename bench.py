@@ -44,6 +44,15 @@ WORKLOADS = {
     "prefill_8bit_m2048": ("prefill_8bit", 2048),
 }
 METRIC = "qMoE layer tokens/s"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# kernel each roofline line names, from one ncu capture of the current
+# kernels on that workload: decode gate/up GEMV (it also carries the down
+# projections' L2 prefetch), prefill gate/up gather-QMM.  Other workloads:
+# not captured (null).
+TRAFFIC = {
+    "decode_397b_m1": 35542016,
+    "prefill_8bit_m16068": 971213056 + 189862656,
+}
 
 
 def parse():
@@ -325,7 +334,8 @@ def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True):
            "roofline": {"bound": "tensor", "kernel": "k_gqmm gate/up+SwiGLU (fp16 operands)",
                         "achieved": gu_flop / (k_ms / 1e3) / 1e12, "peak": peak_bf16,
                         "unit": "TFLOP/s", "frac": gu_flop / (k_ms / 1e3) / 1e12 / peak_bf16,
-                        "traffic": None, "flop_per_launch": gu_flop, "ms_per_launch": k_ms,
+                        "traffic": TRAFFIC.get(workload), "flop_per_launch": gu_flop,
+                        "ms_per_launch": k_ms,
                         "peak_kind": peak_kind + " bf16 dense (fp16 equal rate)"},
            "gpu_launches": int(launches), "clocks": clk.summary()}
     if want_e2e:
@@ -506,7 +516,8 @@ def run_ours(args):
                       "peak_kind": peak_kind},
         "roofline": {"bound": "hbm", "kernel": "k_gemv gate/up+SwiGLU", "achieved": achieved,
                      "peak": peak_hbm, "unit": "GB/s", "frac": achieved / peak_hbm,
-                     "traffic": None, "bytes_per_launch": gu_bytes, "ms_per_launch": k_ms,
+                     "traffic": TRAFFIC.get(args.workload), "bytes_per_launch": gu_bytes,
+                     "ms_per_launch": k_ms,
                      "peak_kind": peak_kind},
         "e2e": e2e,
         "gpu_launches": int(launches_per_timed_region),
