@@ -34,6 +34,7 @@ WORKLOADS = {
     # same shapes with a 16-expert bank: small enough for full ncu captures
     "decode_397b_e16_m1": ("decode_397b_e16", 1),
     "decode_397b_m8": ("decode_397b", 8),
+    "decode_397b_m64": ("decode_397b", 64),
     "decode_30b_m1": ("decode_30b", 1),
     "decode_mixed_2bit_m1": ("mixed_2bit", 1),
     # prefill: one call over M tokens per step

@@ -607,9 +607,12 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
   __half* h_sh = (__half*)(base + lay.h_sh);
   __half* yrows = (__half*)(base + lay.y);
   const int sms = sm_count();
-  // CTA pairs (m-tiles of 256 rows) whenever the operands can be tensor-map
-  // tiles; every gather-QMM launch of the call uses the same tiling
-  const bool pair = encode_fn() != nullptr;
+  // CTA pairs (m-tiles of 256 rows) when the operands can be tensor-map
+  // tiles and the layer routes enough rows to each expert: a 16,384-token
+  // call averages at least 256 rows per expert (64 K >= E).  The choice
+  // depends on the layer only, so chunked and one-shot calls use the same
+  // kernels; every gather-QMM launch of the call uses the same tiling.
+  const bool pair = encode_fn() != nullptr && 64 * K >= E;
   const int TR = pair ? 2 * gq::BM : gq::BM;
   const int mtiles = (M + TR - 1) / TR;
 
