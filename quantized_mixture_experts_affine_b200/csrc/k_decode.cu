@@ -398,6 +398,16 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   tc::grid_dep_launch();
   if (a.flag_reset && blockIdx.x == 0 && threadIdx.x == 0) *a.flag_reset = 0;
 
+  // consumer geometry, and the input slice a consumer warp holds (built
+  // early from token 0's row by the warps the fused plan leaves idle)
+  const int grp = warp / GV_CW, cw = warp % GV_CW;
+  const bool on_w = cw < W;
+  const int sl = cw % S, j = cw / S;
+  const int ch = sl * 32 + lane;
+  const bool lane_on = on_w && ch < cpr;
+  SliceVec<BITS, NL> sv;
+  const void* cur_src = nullptr;
+
   const Seg* segs;
   int n_segs, total_units;
   bool timed_out_p = false;
@@ -434,8 +444,15 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         // the scratch of the plan lives in stages 1..3 of the (still unused)
         // ring; stage 0 may be receiving the shared expert's unit
         o.shared_first = a.plan.has_shared;
-        plan_cta(a.plan, gsm + GV_STAGE_BYTES,
-                 plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32), o);
+        const int pr = plan_route_warps(a.plan.M, a.plan.E, GV_THREADS / 32);
+        // consumer warps the plan does not use build their slice of token
+        // 0's row now (the first vector of the shared expert's units, and
+        // of every unit when M = 1); the others build it after the plan
+        if (warp >= max(pr, 4 * a.plan.M) && warp < GV_PRODUCER && on_w) {
+          build_slice<BITS, NL, SrcT>(a.plan.x, ch, lane_on, sv);
+          cur_src = a.plan.x;
+        }
+        plan_cta(a.plan, gsm + GV_STAGE_BYTES, pr, o);
         if (a.flag_set && blockIdx.x == 0 && threadIdx.x == 0) {
           // CTA 0's lists (written before plan_cta's final barrier) are
           // visible GPU-wide before the flag
@@ -545,16 +562,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   } else {
     // ------------------------------------------------------------ consumers
     // group grp takes every GV_GROUPS-th unit of the CTA (stages grp, grp + GV_GROUPS, ...)
-    const int grp = warp / GV_CW, cw = warp % GV_CW;
-    const bool on_w = cw < W;
-    const int sl = cw % S, j = cw / S;
-    const int ch = sl * 32 + lane;
-    const bool lane_on = on_w && ch < cpr;
     int gi[2];
 #pragma unroll
     for (int pb = 0; pb < 2; ++pb) gi[pb] = (ch * VPC + (pb < NB ? pb : 0) * kXBlock) / a.G;
-    SliceVec<BITS, NL> sv;
-    const void* cur_src = nullptr;
     // the first vector's slice is built while the first stage streams in
     if (on_w) {
       const int u0 = blockIdx.x + grp * gridDim.x;
@@ -565,8 +575,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         const Seg& sg = segs[si];
         if (sg.n_vec > 0) {
           const void* src0 = sg.vec_mode == 0 ? sg.src_base : sg.vecs[0].src;
-          build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
-          cur_src = src0;
+          if (src0 != cur_src) {
+            build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
+            cur_src = src0;
+          }
         }
       }
     }
