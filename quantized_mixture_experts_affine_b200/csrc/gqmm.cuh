@@ -1,20 +1,29 @@
 // Gather quantised matrix multiply on tcgen05 tensor cores (prefill path).
 //
-// One CTA per SM loops over work items (m-tile of 128 sorted rows of one
-// expert, n-tile of 256 weight rows).  Warp roles:
-//   warps 0-1  A loader: gathers the 128 rows (token rows of x, or the
-//              expert's contiguous hidden rows) with 16-byte cp.async into
-//              the 128B-swizzled K-major A stage;
-//   warp  2    B loader: the packed codes of 256 weight rows for one
-//              64-wide group (two tensor-map tiles of 128 rows, or cp.async
-//              per row) and their bf16 scale/bias pairs (cp.async);
-//   warp  3    MMA issuer: tcgen05.mma (M 128, N 256, K 16) x 4 per group,
-//              fp32 accumulators in TMEM (two 256-column buffers);
+// Persistent, warp-specialised.  A work item is an m-tile of one expert's
+// sorted token rows by an n-tile of 256 weight rows, over 64-wide groups
+// (k-blocks).  Two forms:
+//   PAIR   the two CTAs of a cluster share each item: 256 token rows, each
+//          CTA loading 128 of them and dequantising 128 of the weight rows;
+//          rank 0 issues tcgen05.mma.cta_group::2 (M 256, N 256, K 16) over
+//          both CTAs' shared memory and commits to both CTAs' barriers;
+//   single one CTA per item: 128 token rows, 256 weight rows, M 128.
+// Warp roles (per CTA):
+//   warps 0-1  A loader: token rows (or the expert's contiguous hidden rows)
+//              as tensor-map tiles (one thread issues; PAIR: completion
+//              counted on rank 0's barrier), or, without tensor maps, 16-byte
+//              cp.async gathers;
+//   warp  2    B loader: the packed codes of the CTA's weight rows for one
+//              k-block (tensor-map tiles of 128 rows, or cp.async per row) and
+//              the rows' scales and biases once per window of up to 8 groups;
+//   warp  3    MMA issuer (PAIR: rank 0 only), fp32 accumulators in TMEM
+//              (two 256-column buffers);
 //   warps 4-7  epilogue: tcgen05.ld of the accumulator rows, SwiGLU to fp16
-//              hidden rows, or fp32 output rows scattered to pair order;
+//              hidden rows, or output rows (fp16 or fp32) scattered to pair
+//              order, as 32-byte stores;
 //   warps 8-15 dequantiser: codes -> fp16 weights w = q*scale + bias (one
 //              fused fp16 multiply-add of exact operands) written into the
-//              swizzled B stage, one weight row per thread.
+//              swizzled B stage.
 // The scale and bias of a 64-wide group are constant along K within a
 // k-block, so dequantising tiles in shared memory applies the affine map of
 // the pages' format exactly once per weight before the tensor-core product.
