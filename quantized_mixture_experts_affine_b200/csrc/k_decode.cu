@@ -31,10 +31,14 @@ int gemv_units(int out_dim, const GemvShape& sh) { return (out_dim + sh.RU - 1) 
 // Persistent CTAs (one per SM).  Warp 16 is the producer: it reads the work
 // description of up to 32 of its CTA's units at once (one unit per lane),
 // then per unit (RU consecutive rows of NMAT matrices of one segment) lane
-// 0 issues bulk copies of the contiguous packed rows into a 4-stage
-// shared-memory ring, and all lanes copy the rows' bf16 scale/bias pairs
-// and the unit's input/output vector references with cp.async.  Warp 17
-// issues the L2 prefetches.  Warps 0-15 form two consumer groups that take
+// 0 issues bulk copies of the contiguous packed rows and, when 16-byte
+// aligned, of their bf16 scale and bias runs into a 4-stage shared-memory
+// ring (otherwise the lanes copy those entry by entry); the unit's
+// input/output vector references follow by cp.async.  Warp 17 issues the
+// L2 prefetches.  A gate/up launch with a small step computes the step's
+// routing and work lists itself in every CTA (the plan), lists the shared
+// expert first and pre-issues its first unit before the dependency wait;
+// the down launch's producer may start on the plan's published-lists flag.  Warps 0-15 form two consumer groups that take
 // alternate units, so one group computes while the other waits for its
 // stage.  In a group, warps 0..S*J-1 consume: warp (slice s, subset j)
 // keeps its 32-chunk slice of the input vector in registers as fixed-point
