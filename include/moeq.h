@@ -215,6 +215,17 @@ size_t moeq_static_workspace_capacity(void);
 moeq_status moeq_device_status(void* stream, int32_t* status_out);
 
 /*
+ * Failure-path self test (the pages have no counterpart).  Launches one CTA
+ * on `stream` whose two bounded waits, the kinds every kernel of this
+ * library uses, run out: warp 0 waits on an mbarrier phase that never
+ * completes, warp 1 polls a device flag that nothing sets.  Each gives up
+ * after about two seconds, sets MOEQ_ERR_TIMEOUT in the device status word
+ * and returns, so the context stays usable (read the word with
+ * moeq_device_status).  Asynchronous; returns CUDA if the launch fails.
+ */
+moeq_status moeq_selftest_wait_timeout(void* stream);
+
+/*
  * Diagnostics for benchmarks.
  *
  * moeq_set_profile_events: when `start` and `stop` are cudaEvent_t handles

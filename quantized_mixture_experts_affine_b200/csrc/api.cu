@@ -594,6 +594,13 @@ MOEQ_API moeq_status moeq_set_profile_events(void* start, void* stop) {
 
 MOEQ_API uint64_t moeq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+MOEQ_API moeq_status moeq_selftest_wait_timeout(void* stream) {
+  int* p = status_ptr();
+  if (!p) return MOEQ_ERR_CUDA;
+  LAUNCH(launch_wait_probe(p, (cudaStream_t)stream));
+  return MOEQ_OK;
+}
+
 MOEQ_API moeq_status moeq_device_status(void* stream, int32_t* status_out) {
   if (!status_out) return MOEQ_ERR_INVALID_ARG;
   int* p = status_ptr();

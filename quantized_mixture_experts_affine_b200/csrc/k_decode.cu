@@ -1182,6 +1182,30 @@ cudaError_t launch_decode_plan(const DecodePlanArgs& a, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, k_decode_plan, a);
 }
 
+// ============================================================== wait self test
+// Warp 0 waits on an mbarrier phase that never completes, warp 1 on a flag
+// that stays 0; both waits are the bounded ones the kernels above use.
+__device__ int32_t g_never_set = 0;
+
+__global__ void __launch_bounds__(64) k_wait_probe(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    tc::mbar_wait(&bar, 0, status);
+  } else {
+    wait_flag(&g_never_set, status);
+  }
+}
+
+cudaError_t launch_wait_probe(int* status, cudaStream_t st) {
+  k_wait_probe<<<1, 64, 0, st>>>(status);
+  return cudaGetLastError();
+}
+
 // ============================================================== combine
 __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ d,
                                                  const float* __restrict__ w,

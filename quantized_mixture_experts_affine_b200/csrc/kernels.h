@@ -191,6 +191,9 @@ cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, fl
                            cudaStream_t st);
 
 // y[t] = sum_k w[t][k] * d[t*K + k] + sigma[t] * d[M*K + t] + residual[t]
+// Failure-path self test: bounded waits that run out (MOEQ_ERR_TIMEOUT).
+cudaError_t launch_wait_probe(int* status, cudaStream_t st);
+
 cudaError_t launch_combine(const float* d, const float* w, const float* sigma, int has_shared,
                            const float* residual, float* y, int M, int K, int H, cudaStream_t st);
 

@@ -26,7 +26,7 @@ MODE_AUTO, MODE_DECODE, MODE_PREFILL = 0, 1, 2
 EXPORTS = ("moeq_dequant", "moeq_qmv", "moeq_route_topk", "moeq_expert_ffn", "moeq_layer_forward",
            "moeq_workspace_bytes", "moeq_device_status", "moeq_status_str", "moeq_version",
            "moeq_set_profile_events", "moeq_launch_count", "moeq_layer_forward_static",
-           "moeq_static_workspace_capacity")
+           "moeq_static_workspace_capacity", "moeq_selftest_wait_timeout")
 
 
 class MoeqError(RuntimeError):
@@ -66,6 +66,7 @@ _lib.moeq_static_workspace_capacity.restype = C.c_size_t
 _lib.moeq_workspace_bytes.argtypes = [C.POINTER(Layer), C.c_int32, C.c_int32]
 _lib.moeq_workspace_bytes.restype = C.c_size_t
 _lib.moeq_device_status.argtypes = [_P, C.POINTER(C.c_int32)]
+_lib.moeq_selftest_wait_timeout.argtypes = [_P]
 _lib.moeq_status_str.argtypes = [C.c_int32]
 _lib.moeq_status_str.restype = C.c_char_p
 _lib.moeq_version.restype = C.c_char_p
@@ -73,7 +74,7 @@ _lib.moeq_set_profile_events.argtypes = [_P, _P]
 _lib.moeq_set_profile_events.restype = C.c_int
 _lib.moeq_launch_count.restype = C.c_uint64
 for _f in ("moeq_dequant", "moeq_qmv", "moeq_route_topk", "moeq_expert_ffn", "moeq_layer_forward",
-           "moeq_layer_forward_static", "moeq_device_status"):
+           "moeq_layer_forward_static", "moeq_device_status", "moeq_selftest_wait_timeout"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -174,6 +175,10 @@ def moeq_set_profile_events(start=None, stop=None) -> None:
 
 def moeq_launch_count() -> int:
     return int(_lib.moeq_launch_count())
+
+
+def moeq_selftest_wait_timeout(stream=None) -> None:
+    _check("moeq_selftest_wait_timeout", _lib.moeq_selftest_wait_timeout(_stream(stream)))
 
 
 def moeq_device_status(stream=None) -> int:
