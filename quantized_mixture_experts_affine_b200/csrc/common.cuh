@@ -27,18 +27,6 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
   return __uint_as_float(((uint32_t)h) << 16);
 }
 
-// ------------------------------------------------------------------ loads
-// Streaming 16-byte load of packed weights: read once, do not keep in L1.
-__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ uint16_t ldg_u16(const uint16_t* p) { return __ldg(p); }
-
 // ------------------------------------------------------------------ integer dot products
 // d = c + sum_i a.byte[i] * b.byte[i]; a unsigned codes, b signed or unsigned limb.
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
@@ -56,12 +44,6 @@ __device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// Sum within aligned segments of `width` lanes (power of two <= 32).
-__device__ __forceinline__ float segment_sum(float v, int width) {
-  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
