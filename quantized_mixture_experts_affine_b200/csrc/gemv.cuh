@@ -36,6 +36,39 @@ struct SliceVec {
   float xsum[NB];  // sum of the represented values in this chunk's part of the block
 };
 
+// A lane's slice to and from shared memory, word-major ([word][lane]) so
+// that a warp's accesses are conflict-free.  At most 64 words per lane.
+template <int BITS, int NL>
+__device__ __forceinline__ void slice_store(uint32_t* slot, const SliceVec<BITS, NL>& sv,
+                                            int lane) {
+  constexpr int NC = SliceVec<BITS, NL>::NC, NB = SliceVec<BITS, NL>::NB;
+  static_assert(NL * NC + 2 * NB <= 64, "slice exceeds its shared-memory slot");
+#pragma unroll
+  for (int l = 0; l < NL; ++l)
+#pragma unroll
+    for (int r = 0; r < NC; ++r) slot[(l * NC + r) * 32 + lane] = sv.limb[l][r];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    slot[(NL * NC + b) * 32 + lane] = __float_as_uint(sv.xs[b]);
+    slot[(NL * NC + NB + b) * 32 + lane] = __float_as_uint(sv.xsum[b]);
+  }
+}
+
+template <int BITS, int NL>
+__device__ __forceinline__ void slice_load(const uint32_t* slot, SliceVec<BITS, NL>& sv,
+                                           int lane) {
+  constexpr int NC = SliceVec<BITS, NL>::NC, NB = SliceVec<BITS, NL>::NB;
+#pragma unroll
+  for (int l = 0; l < NL; ++l)
+#pragma unroll
+    for (int r = 0; r < NC; ++r) sv.limb[l][r] = slot[(l * NC + r) * 32 + lane];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    sv.xs[b] = __uint_as_float(slot[(NL * NC + b) * 32 + lane]);
+    sv.xsum[b] = __uint_as_float(slot[(NL * NC + NB + b) * 32 + lane]);
+  }
+}
+
 // Value c of the source vector row, as float.
 struct SrcBF16 {
   __device__ __forceinline__ static void load(const void* row, int c0, float* v, int n) {

@@ -83,7 +83,11 @@ struct GvSmem {
   static constexpr int PCNT_OFF = PVEC_OFF + kFusedMaxPairs * 16;
   static constexpr int PEXP_OFF = PCNT_OFF + 8 * 4;
   static constexpr int FLAG_OFF = PEXP_OFF + kFusedMaxPairs * 4;
-  static constexpr int BYTES = FLAG_OFF + GV_GROUPS * 4;
+  // one input slice per consumer group, shared by its warps when they all
+  // hold the same chunk (a single slice: S = 1)
+  static constexpr int SL_OFF = (FLAG_OFF + GV_GROUPS * 4 + 15) & ~15;
+  static constexpr int SL_WORDS = 64 * 32;
+  static constexpr int BYTES = SL_OFF + GV_GROUPS * SL_WORDS * 4;
   static constexpr int RING_BYTES = GV_STAGES * GV_STAGE_BYTES;
 };
 static_assert(sizeof(GvMeta) <= GvSmem::META_STRIDE, "GvMeta exceeds its slot");
@@ -452,7 +456,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         // consumer warps the plan does not use build their slice of token
         // 0's row now (the first vector of the shared expert's units, and
         // of every unit when M = 1); the others build it after the plan
-        if (warp >= max(pr, 4 * a.plan.M) && warp < GV_PRODUCER && on_w) {
+        // (not with a single slice, S = 1: there the group's warps share one
+        // build, which needs every warp of the group to take the same path)
+        if (S > 1 && warp >= max(pr, 4 * a.plan.M) && warp < GV_PRODUCER && on_w) {
           build_slice<BITS, NL, SrcT>(a.plan.x, ch, lane_on, sv);
           cur_src = a.plan.x;
         }
@@ -580,7 +586,20 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         if (sg.n_vec > 0) {
           const void* src0 = sg.vec_mode == 0 ? sg.src_base : sg.vecs[0].src;
           if (src0 != cur_src) {
-            build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
+            if (S == 1 && W > 1) {
+              // every warp of the group holds the same chunk: one loads and
+              // converts the vector, the others copy its slice
+              uint32_t* slot = reinterpret_cast<uint32_t*>(gsm + GvSmem::SL_OFF) +
+                               grp * GvSmem::SL_WORDS;
+              if (cw == 0) {
+                build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
+                slice_store<BITS, NL>(slot, sv, lane);
+              }
+              tc::named_sync(12 + grp, W * 32);
+              if (cw != 0) slice_load<BITS, NL>(slot, sv, lane);
+            } else {
+              build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
+            }
             cur_src = src0;
           }
         }
