@@ -415,6 +415,11 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   const bool lane_on = on_w && ch < cpr;
   SliceVec<BITS, NL> sv;
   const void* cur_src = nullptr;
+  // words of one lane's slice; token 0's slices, built by group 1 during a
+  // fused plan, shared through shared memory when all S of them fit
+  constexpr int SLW = NL * Chunk<BITS>::NC + 2 * SliceVec<BITS, NL>::NB;
+  uint32_t* const sl_base = reinterpret_cast<uint32_t*>(gsm + GvSmem::SL_OFF);
+  bool x_shared = false;
 
   const Seg* segs;
   int n_segs, total_units;
@@ -462,6 +467,12 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
           build_slice<BITS, NL, SrcT>(a.plan.x, ch, lane_on, sv);
           cur_src = a.plan.x;
         }
+        // when the whole of group 1 is idle during the plan, its first
+        // subset's warps leave their slices for the routing warps, which
+        // copy them after the plan instead of loading the row themselves
+        x_shared = S > 1 && S * SLW <= 2 * GvSmem::SL_WORDS / 32 && GV_CW >= max(pr, 4 * a.plan.M);
+        if (x_shared && grp == 1 && j == 0 && on_w)
+          slice_store<BITS, NL>(sl_base + sl * SLW * 32, sv, lane);
         plan_cta(a.plan, gsm + GV_STAGE_BYTES, pr, o);
         if (a.flag_set && blockIdx.x == 0 && threadIdx.x == 0) {
           // CTA 0's lists (written before plan_cta's final barrier) are
@@ -586,7 +597,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         if (sg.n_vec > 0) {
           const void* src0 = sg.vec_mode == 0 ? sg.src_base : sg.vecs[0].src;
           if (src0 != cur_src) {
-            if (S == 1 && W > 1) {
+            if (x_shared && src0 == (const void*)a.plan.x) {
+              slice_load<BITS, NL>(sl_base + sl * SLW * 32, sv, lane);
+            } else if (S == 1 && W > 1) {
               // every warp of the group holds the same chunk: one loads and
               // converts the vector, the others copy its slice
               uint32_t* slot = reinterpret_cast<uint32_t*>(gsm + GvSmem::SL_OFF) +
