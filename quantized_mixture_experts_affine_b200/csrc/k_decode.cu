@@ -92,6 +92,7 @@ struct GvSmem {
 };
 static_assert(sizeof(GvMeta) <= GvSmem::META_STRIDE, "GvMeta exceeds its slot");
 static_assert(GvSmem::BYTES <= 227 * 1024, "GEMV shared memory exceeds the per-CTA limit");
+static_assert(kFusedMaxPairs + 1 <= GV_UB_CAP, "a fused plan's segment starts fit the cache");
 static_assert(GvSmem::PSEG_OFF % 16 == 0 && GvSmem::PVEC_OFF % 16 == 0, "plan region alignment");
 
 int gemv_threads() { return GV_THREADS; }
@@ -444,6 +445,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         o.vecs_gu = reinterpret_cast<VecRef*>(gsm + GvSmem::PVEC_OFF);
         o.experts = pexp;
         o.n_experts = pcnt + 4;
+        o.ub_gu = ub;  // at most kFusedMaxPairs + 1 segments: within GV_UB_CAP
         if (blockIdx.x == 0) {
           o.idx = a.plan.idx_out;
           o.w = a.plan.w_out;
@@ -495,7 +497,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
       n_segs = timed_out_p ? 0 : a.dyn_count[0];
       total_units = timed_out_p ? 0 : a.dyn_count[1];
     }
-    if (early) {
+    if (planned) {
+      // the plan wrote the segment starts; its final barrier published them
+    } else if (early) {
       // the producer does not join: the others cache the segment starts
       if (warp != GV_PRODUCER) {
         if (n_segs <= GV_UB_CAP)
@@ -916,6 +920,7 @@ __device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const
     g.dst_stride = 0;
     g.vecs = o.vecs_gu + i;
     o.segs_gu[gi] = g;
+    if (o.ub_gu) o.ub_gu[gi] = g.unit_begin;
   }
   if (o.segs_dn) {
     Seg dn;
@@ -1114,9 +1119,11 @@ __device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, i
         if (o.shared_first) {
           g.unit_begin = 0;
           o.segs_gu[0] = g;
+          if (o.ub_gu) o.ub_gu[0] = 0;
         } else {
           g.unit_begin = same_gu ? units_gu : 0;
           o.segs_gu[same_gu ? n_entries : n] = g;
+          if (o.ub_gu && same_gu) o.ub_gu[n_entries] = g.unit_begin;
         }
       }
       if (o.segs_dn) {

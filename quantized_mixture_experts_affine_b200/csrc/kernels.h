@@ -100,6 +100,8 @@ struct PlanSinks {
   // gate/up list with the shared expert first (segment 0, units from 0) and
   // the routed entries after it
   int32_t shared_first;
+  // first unit of every gate/up segment (a GEMV's cached segment starts)
+  int32_t* ub_gu;
 };
 
 // Staged logits of the plan's routing warps: at most this many bytes.
