@@ -51,7 +51,7 @@ METRIC = "qMoE layer tokens/s"
 # projections' L2 prefetch), prefill gate/up gather-QMM.  Other workloads:
 # not captured (null).
 TRAFFIC = {
-    "decode_397b_m1": 35612928,
+    "decode_397b_m1": 35535872,
     "prefill_8bit_m16068": 971213056 + 189862656,
 }
 

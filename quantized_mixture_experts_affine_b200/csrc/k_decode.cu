@@ -963,6 +963,10 @@ __device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, i
   //    select candidates from a quarter of the experts and one merges them;
   //    otherwise R warps, one token each at a time
   const int WT = (a.logits && a.E >= 256 && M <= 8 && M * 4 <= (nthr >> 5)) ? 4 : 1;
+  // the shared expert's gate, by the CTA's last warp (idle in a GEMV
+  // launch's plan) while the others route
+  if (a.has_shared && a.sg_logit && warp == (nthr >> 5) - 1)
+    for (int t = tid & 31; t < M; t += 32) ps.ssig[t] = 1.0f / (1.0f + expf(-a.sg_logit[t]));
   if (WT > 1) {
     if (warp < M * WT) {
       const int t = warp / WT, part = warp % WT;
@@ -987,8 +991,6 @@ __device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, i
       ps.sw[p] = a.w_in[p];
     }
   }
-  if (a.has_shared && a.sg_logit)
-    for (int t = tid; t < M; t += nthr) ps.ssig[t] = 1.0f / (1.0f + expf(-a.sg_logit[t]));
   __syncthreads();
   if (o.sigma && a.has_shared && a.sg_logit)
     for (int t = tid; t < M; t += nthr) o.sigma[t] = ps.ssig[t];
