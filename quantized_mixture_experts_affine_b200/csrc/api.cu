@@ -191,15 +191,15 @@ static int units_for(const moeq_qtensor& t, int out_dim, int nmat) {
 }
 
 static int grid_cap() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
+  static int sms[kMaxDevices] = {};
+  const int dev = current_device();
+  if (!sms[dev]) {
+    int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    sms = n;
+    sms[dev] = n;
   }
-  return sms;
+  return sms[dev];
 }
 
 static void set_shape(GemvArgs& a, const moeq_qtensor& t, int nmat) {

@@ -17,6 +17,16 @@ constexpr int kMaxE = 4096;          // experts
 constexpr int kXBlock = 32;          // values per fixed-point block of an input vector
 constexpr int kWaitSpins = 1 << 22;  // bounded device-side waits
 
+// ------------------------------------------------------------------ host: devices
+constexpr int kMaxDevices = 64;  // per-device host caches (launch attributes, SM counts)
+
+// The calling thread's current device, clamped to [0, kMaxDevices).
+inline int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  return dev;
+}
+
 // ------------------------------------------------------------------ status word
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);

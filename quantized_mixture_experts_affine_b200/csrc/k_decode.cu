@@ -744,12 +744,14 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
 template <int BITS, int NL, int NMAT, int SRC, int EPI>
 static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
   auto kern = k_gemv<BITS, NL, NMAT, SRC, EPI>;
-  static bool attr = false;
-  if (!attr) {
+  // the shared-memory opt-in is per device
+  static bool attr[kMaxDevices] = {};
+  const int dev = current_device();
+  if (!attr[dev]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GvSmem::BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

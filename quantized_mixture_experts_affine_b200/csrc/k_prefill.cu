@@ -348,8 +348,10 @@ cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = PAIR ? 1 : 0;
-  static int max_units = 0;
-  if (!max_units) {
+  // co-resident CTAs or clusters, and the shared-memory opt-in, per device
+  static int max_units[kMaxDevices] = {};
+  const int dev = current_device();
+  if (!max_units[dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int n = sm_count();
@@ -359,9 +361,9 @@ cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
       if (e != cudaSuccess) return e;
       if (n <= 0) return cudaErrorInvalidConfiguration;
     }
-    max_units = n;
+    max_units[dev] = n;
   }
-  const int n = units < max_units ? units : max_units;
+  const int n = units < max_units[dev] ? units : max_units[dev];
   if (n <= 0) return cudaSuccess;
   cfg.gridDim = dim3(PAIR ? 2 * n : n);
   return cudaLaunchKernelEx(&cfg, kern, a);
@@ -397,14 +399,15 @@ cudaError_t launch_gqmm(int bits, int epi, bool pair, const gq::Args& a, int64_t
 }
 
 int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
+  static int sms[kMaxDevices] = {};
+  const int dev = current_device();
+  if (!sms[dev]) {
+    int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
+    sms[dev] = n;
   }
-  return n;
+  return sms[dev];
 }
 
 gq::Seg seg_single(const moeq_qtensor& t0, const moeq_qtensor* t1, int rows, int a_mode) {
