@@ -2,6 +2,7 @@
 // and the launch sequences of the decode and prefill paths.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -151,8 +152,8 @@ struct Carve {
 };
 
 struct DecodeWs {
-  size_t logits, sg_logit, sigma, idx, w, h, d, segs_gu, segs_dn, counts, vecs_gu, vecs_dn, ctr,
-      flag, total;
+  size_t gen, flag1, flag2, logits, sg_logit, sigma, idx, w, h, d, segs_gu, segs_dn, counts,
+      vecs_gu, vecs_dn, ctr, flag, total;
 };
 
 DecodeWs decode_ws(const moeq_layer* L, int M) {
@@ -161,7 +162,13 @@ DecodeWs decode_ws(const moeq_layer* L, int M) {
   const size_t n = (size_t)M * K;
   Carve c;
   DecodeWs w;
-  w.logits = c.take((size_t)M * E * 4);
+  // one-launch decode: the previous call's tag (word 0) and two flag arrays
+  w.gen = c.take(8);
+  w.flag1 = c.take((size_t)kFusedMaxGrid * 8);
+  w.flag2 = c.take((size_t)kFusedMaxGrid * 8);
+  // router logits of M tokens (+ one slot: the shared gate logit of the
+  // one-launch decode)
+  w.logits = c.take(((size_t)M * E + 1) * 4);
   w.sg_logit = c.take((size_t)M * 4);
   w.sigma = c.take((size_t)M * 4);
   w.idx = c.take(n * 4);
@@ -302,6 +309,64 @@ static cudaError_t run_dyn(const moeq_qtensor& shape_t, const Seg* segs, const i
     count_launches(1);     \
   } while (0)
 
+// ------------------------------------------------------------------ one-launch decode
+// Shape part of the one-launch decode's arguments for the last layer seen by
+// this host thread (recomputed when the descriptor or grid changes).
+struct FusedCache {
+  bool valid = false, ok = false;
+  moeq_layer L;
+  int grid = 0;
+  bool from_router = false;
+  FusedArgs a;
+  FzMaps m;
+};
+static thread_local FusedCache t_fused;
+
+static bool fused_decode_enabled() {
+  const char* e = getenv("MOEQ_FUSED_DECODE");
+  return e && e[0] == '1' && e[1] == 0;
+}
+
+static const FusedArgs* fused_shape(const moeq_layer* L, int grid, bool from_router) {
+  FusedCache& f = t_fused;
+  if (!f.valid || f.grid != grid || f.from_router != from_router ||
+      memcmp(&f.L, L, sizeof(moeq_layer)) != 0) {
+    f.valid = true;
+    f.L = *L;
+    f.grid = grid;
+    f.from_router = from_router;
+    f.ok = fused_decode_plan(L, grid, from_router, f.a, f.m);
+  }
+  return f.ok ? &f.a : nullptr;
+}
+
+static moeq_status fused_forward(const FusedArgs& shape, const FzMaps& maps, int grid,
+                                 const uint16_t* x,
+                                 const int32_t* idx_in, const float* w_in, const float* residual,
+                                 float* y, int32_t* idx_out, float* w_out, char* base,
+                                 const DecodeWs& lay, cudaStream_t st) {
+  FusedArgs a = shape;
+  a.x = x;
+  a.idx_in = idx_in;
+  a.w_in = w_in;
+  a.residual = residual;
+  a.y = y;
+  a.idx_out = idx_out;
+  a.w_out = w_out;
+  a.gen = (uint64_t*)(base + lay.gen);
+  a.flag1 = (uint64_t*)(base + lay.flag1);
+  a.flag2 = (uint64_t*)(base + lay.flag2);
+  a.logits = (float*)(base + lay.logits);
+  a.h = (float*)(base + lay.h);
+  a.hsh = a.h + (size_t)a.K * a.I;
+  a.status = status_ptr();
+  if (!a.status) return MOEQ_ERR_CUDA;
+  CK(profile_mark(true, st));
+  LAUNCH(launch_fused_decode(a, maps, grid, st));
+  CK(profile_mark(false, st));
+  return MOEQ_OK;
+}
+
 // ------------------------------------------------------------------ decode path
 static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
                                   const int32_t* idx_in, const float* w_in, const float* residual,
@@ -323,6 +388,16 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   int32_t* counts = (int32_t*)(base + lay.counts);
   VecRef* vecs_gu = (VecRef*)(base + lay.vecs_gu);
   VecRef* vecs_dn = (VecRef*)(base + lay.vecs_dn);
+
+  // one token: the whole layer in one launch when its formats allow and the
+  // caller opted in (MOEQ_FUSED_DECODE=1; measured slower than the three
+  // launches below on the 397B-like layer, so not the default)
+  if (M == 1 && fused_decode_enabled()) {
+    const int grid = grid_cap() < kFusedMaxGrid ? grid_cap() : kFusedMaxGrid;
+    if (const FusedArgs* f = fused_shape(L, grid, idx_in == nullptr))
+      return fused_forward(*f, t_fused.m, grid, x, idx_in, w_in, residual, y, idx_out, w_out, base,
+                           lay, st);
+  }
 
   // 1. router logits and the shared-expert gate logit (one launch when the
   //    two 8-bit tensors agree in format)

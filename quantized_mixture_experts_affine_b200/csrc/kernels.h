@@ -1,6 +1,7 @@
 // Host-side launchers shared between the C ABI (api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -187,6 +188,68 @@ cudaError_t launch_route_topk(const float* logits, int M, int E, int K, int reno
 // expert), written into `plan` (device workspace).
 
 cudaError_t launch_decode_plan(const DecodePlanArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------------------ one-launch decode (M = 1)
+constexpr int kFusedMaxK = 8;       // top-K of the one-launch decode
+constexpr int kFusedMaxGrid = 256;  // CTAs (flags per array in the workspace)
+
+// Unit kinds of the one-launch decode, in issue order within a CTA.
+enum FzKindId { FZ_ROUTER = 0, FZ_SGATE = 1, FZ_SHGU = 2, FZ_SHDN = 3, FZ_GU = 4, FZ_DN = 5 };
+// Tensors of the one-launch decode; each has a code map, a scale map and a
+// bias map (map index = 3 * tensor + 0, 1, 2).
+enum FzMapId { FZM_ROUTER = 0, FZM_SGATE, FZM_SHG, FZM_SHU, FZM_SHD, FZM_G, FZM_U, FZM_D, FZM_N };
+
+// Geometry of one unit kind.  A unit holds nbox boxes of RB rows (gate/up:
+// a gate box and an up box of RB intermediate indices); a row's codes are
+// cut into S slabs of slab_bytes, stored at a padded stride of slab_bytes +
+// 16 per (slab, row): box = [S][RB][slab_bytes + 16], box_bytes long,
+// placed box_stride bytes apart (a multiple of 128: tensor copies land on
+// 128-byte aligned shared memory).
+// A box's scale (bias) rows follow the code boxes: [RB][gpr + 8] bf16 each
+// (the 8 padding entries read as zeros), sb_bytes long, sb_stride apart.
+struct FzKind {
+  int32_t row_bytes, gpr, RB, S, slab_bytes, box_bytes, box_stride, nbox, gran;
+  int32_t sb_bytes, sb_stride;
+};
+
+struct FzMaps {
+  CUtensorMap tm[3 * FZM_N];
+};
+
+struct FusedArgs {
+  moeq_qtensor router, sgate, gate, up, down, sh_gate, sh_up, sh_down;
+  int32_t H, I, Ish, E, K, renorm, has_shared, route_from_router;
+  float router_scale;
+  const uint16_t* x;        // [H] bf16
+  const int32_t* idx_in;    // [K] when the routing is given
+  const float* w_in;
+  const float* residual;    // [H] or null
+  float* y;                 // [H]
+  int32_t* idx_out;         // [K] or null
+  float* w_out;
+  uint64_t* gen;            // previous call's tag (workspace word 0)
+  uint64_t* flag1;          // [grid] router logits / shared hidden values published
+  uint64_t* flag2;          // [grid] routed hidden values published
+  float* logits;            // [E + 1]: router logits, then the shared gate logit
+  float* hsh;               // [Ish] shared hidden values
+  float* h;                 // [K][I] routed hidden values
+  int* status;
+  FzKind kind[6];
+  int32_t dgran, drows_max, stage_bytes;
+  int32_t tab_x8, tab_xe, tab_xs, tab_hs, tab_h1;  // bytes of each input table (tab_h1: one expert)
+  int32_t off_args, off_ring, off_xR, off_xE, off_xS, off_hS, off_hl, off_units, off_red,
+      off_dpart, off_bar, smem_bytes;
+  int32_t bits[3];          // router, shared (0: none), routed experts
+};
+
+// Shape part of the arguments, the code tensor maps and the shared-memory
+// layout for `grid` CTAs; false when the layer's formats or sizes are
+// outside what the one-launch decode handles (the multi-launch path runs
+// instead).
+bool fused_decode_plan(const moeq_layer* L, int grid, bool route_from_router, FusedArgs& a,
+                       FzMaps& m);
+int fused_decode_threads();
+cudaError_t launch_fused_decode(const FusedArgs& a, const FzMaps& m, int grid, cudaStream_t st);
 
 // Codes and/or fp32 weights of one matrix.
 cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, float* w_out,

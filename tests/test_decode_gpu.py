@@ -238,3 +238,78 @@ def test_workspace_reuse_and_poison():
         ys.append(y.cpu().numpy())
     assert np.isfinite(ys[0]).all()
     assert np.array_equal(ys[0].view(np.uint32), ys[1].view(np.uint32))
+
+
+# ------------------------------------------------------------------ single token (M = 1)
+# Both decode paths for one token: the default three launches and the opt-in
+# one-launch kernel (MOEQ_FUSED_DECODE=1, read on every call), which runs the
+# layers whose formats it takes (every group 64 wide, rows of whole 8-group
+# runs) and leaves the others to the three launches.
+
+@pytest.fixture(params=["launches", "one_launch"])
+def decode_path(request, monkeypatch):
+    if request.param == "one_launch":
+        monkeypatch.setenv("MOEQ_FUSED_DECODE", "1")
+    else:
+        monkeypatch.delenv("MOEQ_FUSED_DECODE", raising=False)
+    return request.param
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_30b", "decode_397b", "mixed_2bit"])
+def test_single_token_poisoned_workspace(name, decode_path):
+    """The one-launch kernel keeps its inter-CTA flags in the workspace: a
+    workspace filled with three different poisons, then reused for a chain
+    of calls (each call's tag derives from the previous one's), gives
+    bitwise the same output every time, on either path."""
+    cfg = CONFIGS[name]
+    L = synthetic_layer(cfg, SEED, 0)
+    xb, x = x_tokens(cfg, 1, copy=21)
+    ws = Workspace(L, 1, moeq.MODE_DECODE)
+    outs = []
+    for poison in (0xA5, 0x00, 0xFF):
+        ws.buf.fill_(poison)
+        for _ in range(3):
+            y = torch.full((1, cfg.H), float("nan"), device="cuda")
+            y, idx, w = layer_forward(L, x, y=y, ws=ws, mode=moeq.MODE_DECODE)
+            outs.append(y.cpu().numpy().copy())
+    assert moeq.moeq_device_status() == 0
+    check_layer_outputs(cfg, SEED, 0, xb, outs[0], idx.cpu().numpy(), w.cpu().numpy())
+    for o in outs[1:]:
+        assert np.array_equal(o.view(np.uint32), outs[0].view(np.uint32))
+
+
+@pytest.mark.parametrize("name", ["decode_397b", "decode_30b"])
+def test_single_token_many_tokens_in_a_row(name, decode_path):
+    """Different tokens through one workspace, one call each (as a decode
+    loop does); every output matches the oracle."""
+    cfg = CONFIGS[name]
+    L = synthetic_layer(cfg, SEED, 1)
+    ws = Workspace(L, 1, moeq.MODE_DECODE)
+    for t in range(6):
+        xb, x = x_tokens(cfg, 1, copy=400 + t)
+        y, idx, w = layer_forward(L, x, ws=ws, mode=moeq.MODE_DECODE)
+        torch.cuda.synchronize()
+        assert moeq.moeq_device_status() == 0
+        check_layer_outputs(cfg, SEED, 1, xb, y.cpu().numpy(), idx.cpu().numpy(),
+                            w.cpu().numpy())
+
+
+@pytest.mark.parametrize("name", ["decode_397b", "mixed_2bit", "tiny"])
+def test_single_token_given_routing(name, decode_path):
+    """moeq_expert_ffn with M = 1 (routing passed in): experts, shared expert
+    and combine against the oracle, with a residual."""
+    cfg = CONFIGS[name]
+    L = synthetic_layer(cfg, SEED, 0)
+    xb, x = x_tokens(cfg, 1, copy=31)
+    rng = np.random.default_rng(5)
+    ig = np.sort(rng.choice(cfg.E, cfg.K, replace=False)).astype(np.int32)[None, :]
+    wg = rng.random((1, cfg.K)).astype(np.float32)
+    wg /= wg.sum()
+    res_np = np.linspace(-2, 2, cfg.H, dtype=np.float32)[None, :]
+    y = expert_ffn(L, x, dev(ig), dev(wg), residual=dev(res_np), mode=moeq.MODE_DECODE)
+    torch.cuda.synchronize()
+    assert moeq.moeq_device_status() == 0
+    from helpers import oracle_expert_outputs
+    ref = oracle_expert_outputs(cfg, SEED, 0, xb, ig, wg.astype(np.float64), res_np)
+    got = y.cpu().numpy()
+    assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
