@@ -202,11 +202,16 @@ static void orc_route_one(const double* logits, int E, int K, int renorm, double
     z += p[e];
   }
   for (int e = 0; e < E; ++e) p[e] /= z;
+  /* Softmax is strictly increasing in the scaled logit, so the K largest
+   * scores are the K largest scaled logits (ties: lower index first).
+   * Selecting on the logits gives that set even where exp() underflows and
+   * several scores read as 0. */
   double sel = 0.0;
   for (int k = 0; k < K; ++k) {
     int best = -1;
     for (int e = 0; e < E; ++e)
-      if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;
+      if (!taken[e] && (best < 0 || router_scale * logits[e] > router_scale * logits[best]))
+        best = e;
     taken[best] = 1;
     idx[k] = best;
     wts[k] = p[best];
@@ -215,11 +220,14 @@ static void orc_route_one(const double* logits, int E, int K, int renorm, double
   if (renorm)
     for (int k = 0; k < K; ++k) wts[k] /= sel;
   if (gap) {
+    /* relative gap of the K-th and (K+1)-th scores, (p_K - p_next) / p_K =
+     * 1 - exp(l_next - l_K) on the scaled logits (defined under underflow) */
     int next = -1;
     for (int e = 0; e < E; ++e)
-      if (!taken[e] && (next < 0 || p[e] > p[next])) next = e;
-    const double pk = p[idx[K - 1]];
-    *gap = next < 0 ? 1.0 : (pk - p[next]) / pk;
+      if (!taken[e] && (next < 0 || router_scale * logits[e] > router_scale * logits[next]))
+        next = e;
+    *gap = next < 0 ? 1.0
+                    : -expm1(router_scale * logits[next] - router_scale * logits[idx[K - 1]]);
   }
   free(taken);
   free(p);

@@ -420,3 +420,18 @@ def test_threads_do_not_change_results():
     b = oracle.layer(L, x)["out"]
     oracle.set_threads(0)
     assert np.array_equal(a, b)
+
+
+def test_route_under_exp_underflow_selects_by_logit():
+    """Scores that underflow to 0 in fp64 (logit gaps of ~1000) still rank
+    by their logits, as the strictly increasing softmax ranks them; the
+    near-tie gap stays defined (1 - exp(l_next - l_K))."""
+    l = np.array([[0.0, -3000.0, -2000.0, -1000.0, 5.0]])
+    idx, w, gap = oracle.route(l, 3, True, 1.0)
+    assert idx[0].tolist() == [4, 0, 3]
+    e5 = np.exp(-5.0)
+    assert np.allclose(w[0], [1 / (1 + e5), e5 / (1 + e5), 0.0], rtol=1e-14, atol=1e-300)
+    assert gap[0] == 1.0
+    # a negative router scale reverses the order of the logits
+    idx, _, _ = oracle.route(l, 2, True, -1.0)
+    assert idx[0].tolist() == [1, 2]
