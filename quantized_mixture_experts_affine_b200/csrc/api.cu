@@ -22,9 +22,9 @@ __device__ int g_moeq_status;
 
 static int* status_ptr() {
   static std::mutex mu;
-  static int* ptrs[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  static int* ptrs[kMaxDevices] = {nullptr};
+  int dev;
+  if (!current_device(dev)) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
   if (!ptrs[dev]) {
     void* p = nullptr;
@@ -197,17 +197,8 @@ static int units_for(const moeq_qtensor& t, int out_dim, int nmat) {
   return gemv_units(out_dim, gemv_shape(t.in_dim, t.bits, nmat, t.group_size));
 }
 
-static int grid_cap() {
-  static int sms[kMaxDevices] = {};
-  const int dev = current_device();
-  if (!sms[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    sms[dev] = n;
-  }
-  return sms[dev];
-}
+// CTAs of a persistent launch: one per SM (checked non-zero at entry).
+static int grid_cap() { return sm_count(); }
 
 static void set_shape(GemvArgs& a, const moeq_qtensor& t, int nmat) {
   const GemvShape sh = gemv_shape(t.in_dim, t.bits, nmat, t.group_size);
@@ -616,23 +607,35 @@ MOEQ_API size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mod
   return 0;
 }
 
+namespace moeq {
+// The argument checks every layer entry point runs before its workspace
+// check: the layer, M, the mode, and the token, output and residual pointers.
+moeq_status forward_arg_check(const moeq_layer* L, const uint16_t* x, int32_t M, float* y,
+                              const float* residual, int32_t mode) {
+  moeq_status s = check_layer(L);
+  if (s != MOEQ_OK) return s;
+  if (M < 0 || !x || !y) return MOEQ_ERR_INVALID_ARG;
+  if (mode < MOEQ_MODE_AUTO || mode > MOEQ_MODE_PREFILL) return MOEQ_ERR_INVALID_ARG;
+  if (M == 0) return MOEQ_OK;
+  if (!aligned(x, 16) || (L->hidden * 2) % 16 || !aligned(y, 16) || L->hidden % 4)
+    return MOEQ_ERR_ALIGNMENT;
+  if (residual && !aligned(residual, 16)) return MOEQ_ERR_ALIGNMENT;
+  return MOEQ_OK;
+}
+}  // namespace moeq
+
 static moeq_status forward_common(const moeq_layer* L, const uint16_t* x, int32_t M,
                                   const int32_t* idx_in, const float* w_in, const float* residual,
                                   float* y, int32_t* idx_out, float* w_out, void* ws,
                                   size_t ws_bytes, int32_t mode, void* stream) {
-  moeq_status s = check_layer(L);
-  if (s != MOEQ_OK) return s;
-  if (M < 0 || !x || !y) return MOEQ_ERR_INVALID_ARG;
-  if (M == 0) return MOEQ_OK;
-  if (mode < MOEQ_MODE_AUTO || mode > MOEQ_MODE_PREFILL) return MOEQ_ERR_INVALID_ARG;
+  moeq_status s = forward_arg_check(L, x, M, y, residual, mode);
+  if (s != MOEQ_OK || M == 0) return s;
   mode = resolve_mode(mode, M);
-  if (!aligned(x, 16) || (L->hidden * 2) % 16 || !aligned(y, 16) || L->hidden % 4)
-    return MOEQ_ERR_ALIGNMENT;
-  if (residual && !aligned(residual, 16)) return MOEQ_ERR_ALIGNMENT;
   const size_t need = moeq_workspace_bytes(L, M, mode);
   if (need == 0) return MOEQ_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < need) return MOEQ_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return MOEQ_ERR_ALIGNMENT;
+  if (grid_cap() <= 0) return MOEQ_ERR_CUDA;  // no current device to size launches for
   cudaStream_t st = (cudaStream_t)stream;
   if (mode == MOEQ_MODE_DECODE) {
     if (M > kMaxDecodeM) return MOEQ_ERR_UNSUPPORTED;

@@ -4,6 +4,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <stdint.h>
 
 #include "moeq.h"
@@ -20,12 +22,16 @@ constexpr int kWaitSpins = 1 << 22;  // bounded device-side waits
 // ------------------------------------------------------------------ host: devices
 constexpr int kMaxDevices = 64;  // per-device host caches (launch attributes, SM counts)
 
-// The calling thread's current device, clamped to [0, kMaxDevices).
-inline int current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
-  return dev;
+// The calling thread's current device; false when the runtime cannot say or
+// the index is beyond the per-device host caches (callers then fail the call).
+inline bool current_device(int& dev) {
+  dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices;
 }
+
+// SM count of the current device (cached per device); 0 when the device or
+// the attribute cannot be read.
+int sm_count();
 
 // ------------------------------------------------------------------ status word
 __device__ __forceinline__ void set_status(int* status, int code) {

@@ -745,13 +745,14 @@ template <int BITS, int NL, int NMAT, int SRC, int EPI>
 static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
   auto kern = k_gemv<BITS, NL, NMAT, SRC, EPI>;
   // the shared-memory opt-in is per device
-  static bool attr[kMaxDevices] = {};
-  const int dev = current_device();
-  if (!attr[dev]) {
+  static std::atomic<bool> attr[kMaxDevices];
+  int dev;
+  if (!current_device(dev)) return cudaErrorInvalidDevice;
+  if (!attr[dev].load(std::memory_order_acquire)) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GvSmem::BYTES);
     if (e != cudaSuccess) return e;
-    attr[dev] = true;
+    attr[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

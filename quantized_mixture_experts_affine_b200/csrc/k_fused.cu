@@ -870,10 +870,9 @@ template <int BR, int BS, int BE>
 cudaError_t fz_prepare(const FusedArgs& a) {
   auto kern = k_fused_decode<BR, BS, BE>;
   static std::atomic<int> attr_set[kMaxDevices];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int dev;
+  if (!current_device(dev)) return cudaErrorInvalidDevice;
+  cudaError_t e;
   if (attr_set[dev].load(std::memory_order_acquire) >= a.smem_bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
   if (e != cudaSuccess) return e;

@@ -327,7 +327,6 @@ __global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx,
 }
 
 // ------------------------------------------------------------------ gather-QMM launch
-int sm_count();
 
 // Launch over `units` work items: one CTA per item up to the co-resident
 // count, or (PAIR) one cluster of two CTAs per item up to the co-resident
@@ -349,21 +348,24 @@ cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
   cfg.attrs = at;
   cfg.numAttrs = PAIR ? 1 : 0;
   // co-resident CTAs or clusters, and the shared-memory opt-in, per device
-  static int max_units[kMaxDevices] = {};
-  const int dev = current_device();
-  if (!max_units[dev]) {
+  static std::atomic<int> max_units[kMaxDevices];
+  int dev;
+  if (!current_device(dev)) return cudaErrorInvalidDevice;
+  int cap = max_units[dev].load(std::memory_order_acquire);
+  if (cap <= 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    int n = sm_count();
+    cap = sm_count();
+    if (cap <= 0) return cudaErrorInvalidDevice;
     if (PAIR) {
       cfg.gridDim = dim3(2);
-      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      e = cudaOccupancyMaxActiveClusters(&cap, kern, &cfg);
       if (e != cudaSuccess) return e;
-      if (n <= 0) return cudaErrorInvalidConfiguration;
+      if (cap <= 0) return cudaErrorInvalidConfiguration;
     }
-    max_units[dev] = n;
+    max_units[dev].store(cap, std::memory_order_release);
   }
-  const int n = units < max_units[dev] ? units : max_units[dev];
+  const int n = units < cap ? units : cap;
   if (n <= 0) return cudaSuccess;
   cfg.gridDim = dim3(PAIR ? 2 * n : n);
   return cudaLaunchKernelEx(&cfg, kern, a);
@@ -398,17 +400,6 @@ cudaError_t launch_gqmm(int bits, int epi, bool pair, const gq::Args& a, int64_t
   return launch_gqmm_p<false>(bits, epi, a, u, st);
 }
 
-int sm_count() {
-  static int sms[kMaxDevices] = {};
-  const int dev = current_device();
-  if (!sms[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    sms[dev] = n;
-  }
-  return sms[dev];
-}
 
 gq::Seg seg_single(const moeq_qtensor& t0, const moeq_qtensor* t1, int rows, int a_mode) {
   gq::Seg s;
@@ -570,6 +561,19 @@ moeq_status check_prefill(const moeq_layer* L) {
 }
 
 }  // namespace
+
+int sm_count() {
+  static std::atomic<int> sms[kMaxDevices];
+  int dev;
+  if (!current_device(dev)) return 0;
+  int n = sms[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return 0;
+    sms[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
 
 size_t prefill_workspace_bytes(const moeq_layer* L, int M) {
   if (check_prefill(L) != MOEQ_OK) return 0;

@@ -9,6 +9,11 @@
 
 namespace moeq {
 
+// Argument checks shared by the layer entry points (api.cu): the layer, M,
+// the mode, and the x / y / residual pointers, before any workspace check.
+moeq_status forward_arg_check(const moeq_layer* L, const uint16_t* x, int32_t M, float* y,
+                              const float* residual, int32_t mode);
+
 // Diagnostics (api.cu): launch counter and the optional profiling events.
 void count_launches(int n);
 cudaError_t profile_mark(bool start, cudaStream_t st);

@@ -15,6 +15,8 @@
 
 #include <mutex>
 
+#include "common.cuh"
+#include "kernels.h"
 #include "moeq.h"
 
 namespace {
@@ -27,9 +29,9 @@ static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 // device (null if the lookup fails).
 void* static_ws_ptr() {
   static std::mutex mu;
-  static void* ptrs[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  static void* ptrs[moeq::kMaxDevices] = {nullptr};
+  int dev;
+  if (!moeq::current_device(dev)) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
   if (!ptrs[dev]) {
     void* p = nullptr;
@@ -48,10 +50,12 @@ extern "C" __attribute__((visibility("default"))) size_t moeq_static_workspace_c
 extern "C" __attribute__((visibility("default"))) moeq_status moeq_layer_forward_static(
     const moeq_layer* L, const uint16_t* x, int32_t M, float* y, const float* residual,
     int32_t* idx_out, float* w_out, void* stream) {
-  if (M == 0) return moeq_layer_forward(L, x, M, y, residual, idx_out, w_out, nullptr, 0,
-                                        MOEQ_MODE_DECODE, stream);
+  // the ordinary entry point's argument checks come first, so a call fails
+  // with the same status as moeq_layer_forward would; then the capacity
+  const moeq_status s = moeq::forward_arg_check(L, x, M, y, residual, MOEQ_MODE_DECODE);
+  if (s != MOEQ_OK || M == 0) return s;
   const size_t need = moeq_workspace_bytes(L, M, MOEQ_MODE_DECODE);
-  if (need == 0)  // invalid layer or M: let the checks of the ordinary entry point say which
+  if (need == 0)  // beyond the decode path's limits: the ordinary entry point says which
     return moeq_layer_forward(L, x, M, y, residual, idx_out, w_out, nullptr, 0,
                               MOEQ_MODE_DECODE, stream);
   if (need > kStaticWsBytes) return MOEQ_ERR_WORKSPACE;

@@ -136,3 +136,29 @@ def test_forward_argument_checks():
 
 def test_device_status_needs_output():
     assert moeq.lib().moeq_device_status(None, None) == moeq.ERR_INVALID_ARG
+
+
+def fwd_static(L, M=1, x=A, y=A, residual=None):
+    return moeq.lib().moeq_layer_forward_static(C.byref(L), x, M, y, residual, None, None, None)
+
+
+def test_static_entry_checks_arguments_before_capacity():
+    """The fixed-workspace entry runs moeq_layer_forward's argument checks
+    before its capacity check: an oversized layer with a bad pointer reports
+    the pointer, not the workspace."""
+    big = layer(H=8192, I=2048, E=512, K=8)
+    assert moeq.moeq_workspace_bytes(big, 64, moeq.MODE_DECODE) > \
+        moeq.moeq_static_workspace_capacity()
+    assert fwd_static(big, M=64, x=0) == moeq.ERR_INVALID_ARG
+    assert fwd_static(big, M=64, y=0) == moeq.ERR_INVALID_ARG
+    assert fwd_static(big, M=64, x=A + 2) == moeq.ERR_ALIGNMENT
+    assert fwd_static(big, M=64, y=A + 4) == moeq.ERR_ALIGNMENT
+    assert fwd_static(big, M=64, residual=A + 8) == moeq.ERR_ALIGNMENT
+    assert fwd_static(big, M=-1) == moeq.ERR_INVALID_ARG
+    bad = layer()
+    bad.n_experts = 4
+    assert fwd_static(bad) == moeq.ERR_INVALID_ARG
+    assert fwd_static(big, M=0) == moeq.OK
+    # valid pointers: now the capacity decides (nothing launched, no device needed)
+    assert fwd_static(big, M=64) == moeq.ERR_WORKSPACE
+    assert fwd_static(layer(), M=65) == moeq.ERR_UNSUPPORTED
