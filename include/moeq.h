@@ -152,11 +152,20 @@ moeq_status moeq_route_topk(const float* logits, int32_t M, int32_t E, int32_t K
  * PREFILL requires group_size 64 for every tensor, H, I (and the shared
  * expert's I) multiples of 128, 4-byte aligned scale/bias arrays, and
  * values that fit the fp16 tensor-core operands (|x|, |bias| and
- * |bias + (2^b-1)*scale| at most 65504, nonzero |scale| at least 2^-14);
- * outside that range the device status reports MOEQ_ERR_RANGE.  The
+ * |bias + (2^b-1)*scale| at most 65504, every scale exactly representable
+ * as fp16: all bf16 scales of magnitude 2^-17 to 65504 are, and smaller
+ * ones whose lowest significant bit is at least 2^-24; the SwiGLU outputs
+ * and per-expert down rows at most 65504); outside that range the device
+ * status reports MOEQ_ERR_RANGE and the outputs are not valid.  The decode
+ * path has none of these limits.  The
  * prefill path computes every output row from its own token with the same
  * kernels for any M, so splitting the tokens into chunks gives
- * bit-identical results.
+ * bit-identical results.  Only PREFILL mode has that property: AUTO picks
+ * the path per call from that call's M (decode for M <= 64), so a chunked
+ * sequence run in AUTO mode whose last chunk has at most 64 tokens gets
+ * that chunk from the decode path, whose arithmetic differs (the results
+ * agree within the layer tolerance, not bit for bit).  Pass PREFILL for
+ * every chunk to keep chunked and one-shot results bit-identical.
  * idx is not read on the host; an index outside [0,E) found on the device
  * sets MOEQ_ERR_INVALID_ARG in the device status word and expert 0 is used
  * in its place.
@@ -170,6 +179,11 @@ moeq_status moeq_expert_ffn(const moeq_layer* L, const uint16_t* x, int32_t M, c
  * The whole layer: router qmv -> route_topk -> expert_ffn, on the device,
  * with no host round trip.  idx_out/w_out: nullable, receive the routing.
  * Same buffers, workspace and errors as moeq_expert_ffn.
+ * Single-token decode runs as three launches.  With the environment
+ * variable MOEQ_FUSED_DECODE=1 (read on every call) a layer whose tensors
+ * all use group_size 64 with rows of whole 8-group runs runs M = 1 as one
+ * persistent launch instead (same results within the layer tolerance; it
+ * needs every CTA of its grid resident at once, one per SM).
  */
 moeq_status moeq_layer_forward(const moeq_layer* L, const uint16_t* x, int32_t M, float* y,
                                const float* residual, int32_t* idx_out, float* w_out, void* ws,
@@ -189,7 +203,8 @@ size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mode);
  * allocation can synchronise the device; a pool sized at start-up may not
  * grow).
  *   Arguments, layouts and device-side errors are those of
- *   moeq_layer_forward with mode DECODE (M <= 64).
+ *   moeq_layer_forward with mode DECODE (M <= 64); its argument checks
+ *   (layer, M, x, y, residual) run first and fail with the same status.
  *   Capacity: moeq_static_workspace_capacity() bytes (8 MiB) per device,
  *   which covers for example H 4096, I 1024, E 512, K 4 with a shared
  *   expert up to M 64.  When moeq_workspace_bytes(L, M, DECODE) exceeds it

@@ -195,16 +195,18 @@ __device__ __forceinline__ void b_row(const Seg& sg, int nt, int r, int& src, in
 }
 
 // fp16 operands of the affine map for one group, with the range check of
-// the prefill tiles (scale a normal fp16 value or zero, |bias| and
-// |bias + (2^b - 1) scale| below the fp16 maximum).
+// the prefill tiles: the scale exactly representable as fp16 (every bf16
+// scale from 2^-17 to 65504 is, subnormals included, so the fma q*s + b
+// rounds once, as for any normal scale), |bias| and |bias + (2^b - 1) scale|
+// at most the fp16 maximum.
 template <int BITS>
 __device__ __forceinline__ void group_h2(uint32_t sbits, uint32_t bbits, __half2& s2, __half2& b2,
                                          int* status) {
   const float s = bf16_bits_to_float((uint16_t)sbits);
   const float b = bf16_bits_to_float((uint16_t)bbits);
   const float top = fabsf(b + (float)((1 << BITS) - 1) * s);
-  const bool bad = (s != 0.0f && fabsf(s) < 6.103515625e-05f) || fabsf(s) > 65504.0f ||
-                   fabsf(b) > 65504.0f || top > 65504.0f;
+  const bool bad = __half2float(__float2half_rn(s)) != s || !(fabsf(b) <= 65504.0f) ||
+                   !(top <= 65504.0f);
   if (bad) set_status(status, MOEQ_ERR_RANGE);
   s2 = __float2half2_rn(s);
   b2 = __float2half2_rn(b);

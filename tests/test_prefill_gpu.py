@@ -8,6 +8,8 @@ rows), on both sides of the n = M*K = 32768 seam with n % 64 != 0
 (mlx issue 3856: "Silent numerical corruption in single long forward on
 quantized MoE when sequence length % 32 != 0").
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -142,11 +144,11 @@ def test_prefill_chunk_invariance_seam(M):
                         rows=rows)
 
 
-@pytest.mark.parametrize("M", [16068, 16032, 16384])
+@pytest.mark.parametrize("M", [16068, 16065, 16032, 16384])
 def test_prefill_full_size(M):
     """The 16k-token prefill workloads (16068 is unaligned: n = 128544,
-    n % 64 = 32): one-shot == chunked bitwise, sampled rows vs oracle
-    including the last rows of the sorted order."""
+    n % 64 = 32; 16065: n % 64 = 8, M odd): one-shot == chunked bitwise,
+    sampled rows vs oracle including the last rows of the sorted order."""
     cfg = CONFIGS["prefill_8bit"]
     L = layer_of("prefill_8bit")
     xb, x = x_tokens(cfg, M, 200)
@@ -164,6 +166,24 @@ def test_prefill_full_size(M):
     rows = np.unique(np.concatenate([np.array(last, dtype=np.int64), [0, M - 1],
                                      rng.integers(0, M, 40)]))
     check_layer_outputs(cfg, SEED, 0, xb, y1.cpu().numpy(), ig, w1.cpu().numpy(), rows=rows)
+
+
+@pytest.mark.slow
+def test_prefill_full_rows_16068():
+    """Every row of the 16,068-token call against the oracle, on all host
+    cores (about 1.2 TFLOP of fp64 work: minutes).  Runs when
+    MOEQ_FULL_ROWS=1."""
+    if os.environ.get("MOEQ_FULL_ROWS") != "1":
+        pytest.skip("full-row oracle run: set MOEQ_FULL_ROWS=1")
+    cfg = CONFIGS["prefill_8bit"]
+    L = layer_of("prefill_8bit")
+    M = 16068
+    xb, x = x_tokens(cfg, M, 200)
+    y, i, w = forward(L, x)
+    oracle.set_threads(os.cpu_count() or 1)
+    r, m, ties = check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), i.cpu().numpy(),
+                                     w.cpu().numpy())
+    print(f"full rows M={M}: rel_l2 {r:.3e} max_abs {m:.3e} near-tie tokens {ties}")
 
 
 # ------------------------------------------------------------------ mixed bank
@@ -199,3 +219,29 @@ def test_prefill_mixed_2bit_zipf_4096():
     ref = oracle_expert_outputs(cfg, SEED, 0, xb[rows], ig[rows], wref)
     got = y.cpu().numpy()[rows]
     assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
+
+
+def test_auto_mode_picks_the_path_per_call():
+    """AUTO takes the decode path for a call of at most 64 tokens and the
+    prefill path above that, from the call's own M: it is bit for bit one or
+    the other.  So only PREFILL mode makes chunked calls bit-identical to one
+    call; an AUTO chunk of <= 64 tokens agrees with the prefill rows within
+    the layer tolerance only."""
+    L = layer_of("prefill_8bit")
+    cfg = L.cfg
+    xb, x = x_tokens(cfg, 129, copy=77)
+    for M, path in ((64, moeq.MODE_DECODE), (65, P)):
+        ya, ia, wa = layer_forward(L, x[:M], mode=moeq.MODE_AUTO)
+        yb, ib, wb = layer_forward(L, x[:M], mode=path)
+        torch.cuda.synchronize()
+        assert torch.equal(ya.view(torch.int32), yb.view(torch.int32)), M
+        assert torch.equal(ia, ib) and torch.equal(wa.view(torch.int32), wb.view(torch.int32))
+    # 65 + 64 tokens in AUTO mode against one PREFILL call of 129
+    y1, _, _ = forward(L, x)
+    ya, _, _ = layer_forward(L, x[:65], mode=moeq.MODE_AUTO)
+    yb, ib, wb = layer_forward(L, x[65:], mode=moeq.MODE_AUTO)
+    torch.cuda.synchronize()
+    assert torch.equal(ya.view(torch.int32), y1[:65].view(torch.int32))
+    got, ref = yb.cpu().numpy(), y1[65:].cpu().numpy()
+    assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
+    check_layer_outputs(cfg, SEED, 0, xb[65:], got, ib.cpu().numpy(), wb.cpu().numpy())
