@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import sys
@@ -29,22 +30,58 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOADS = {
-    # name: (config, tokens per step)
+    # name: (shape, tokens per step)
     "decode_397b_m1": ("decode_397b", 1),
     # same shapes with a 16-expert bank: small enough for full ncu captures
     "decode_397b_e16_m1": ("decode_397b_e16", 1),
+    "tiny_m1": ("tiny", 1),
+    "tiny_m3": ("tiny", 3),
+    "tiny_m5": ("tiny", 5),
     "decode_397b_m8": ("decode_397b", 8),
     "decode_397b_m64": ("decode_397b", 64),
     "decode_30b_m1": ("decode_30b", 1),
     "decode_mixed_2bit_m1": ("mixed_2bit", 1),
     # prefill: one call over M tokens per step
+    "prefill_8bit_m16032": ("prefill_8bit", 16032),
     "prefill_8bit_m16068": ("prefill_8bit", 16068),
     "prefill_8bit_m16384": ("prefill_8bit", 16384),
+    "prefill_mixed_2bit_m256": ("mixed_2bit", 256),
     "prefill_mixed_2bit_m4096": ("mixed_2bit", 4096),
     # small prefill case for full profiler captures
     "prefill_8bit_m2048": ("prefill_8bit", 2048),
 }
 METRIC = "qMoE layer tokens/s"
+
+
+def shape(name):
+    """Layer shape by name (plain data: loads no library)."""
+    import dataclasses
+    from quantized_mixture_experts_affine_b200.config import CONFIGS
+    if name == "decode_397b_e16":
+        return dataclasses.replace(CONFIGS["decode_397b"], name=name, E=16)
+    return CONFIGS[name]
+
+
+def config_of(workload, world, copies):
+    """The line's `config`: the workload's shape and how the timed steps
+    keep their weights out of L2 (the same dict in both arms)."""
+    cfg_name, M = WORKLOADS[workload]
+    cfg = shape(cfg_name)
+    d = {"workload": workload, "tokens_per_step": M, "hidden": cfg.H, "experts": cfg.E,
+         "top_k": cfg.K, "intermediate": cfg.I, "expert_bits": cfg.expert_bits,
+         "router_bits": cfg.router_bits, "shared_expert": cfg.shared,
+         "shared_intermediate": cfg.shared_I, "group_size": cfg.G,
+         "parallelism": f"replicas{world}"}
+    if workload.startswith("prefill"):
+        d["l2"] = "inputs larger than L2 (weights, token rows and output rows)"
+    else:
+        touched = (cfg.router_bytes() + min(cfg.E, M * cfg.K) * cfg.expert_bytes()
+                   + cfg.shared_bytes())
+        mb = copies * touched / 1e6
+        d["l2"] = (f"{copies} layer copies cycled, fresh tokens per step (up to {mb:.0f} MB "
+                   f"of weights touched per cycle; L2 is 126 MB"
+                   + (", so these weights stay L2-resident)" if mb < 126 else ")"))
+    return d
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
 # kernel each roofline line names, from one ncu capture of the current
 # kernels on that workload: decode gate/up GEMV (it also carries the down
@@ -71,6 +108,9 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the secondary prefill measurement of the decode run")
     ap.add_argument("--prefill-workload", default="prefill_8bit_m16068")
+    ap.add_argument("--sweep", action="store_true",
+                    help="per-config table instead of the benchmark line (one JSON line per row)")
+    ap.add_argument("--sweep-rows", default="", help="comma-separated rows (C1..C5) to run")
     return ap.parse_args()
 
 
@@ -199,8 +239,7 @@ class OracleSample:
     def __init__(self, cfg, n_tokens, seed=0):
         import numpy as np
         import oracle
-        sys.path.insert(0, os.path.join(ROOT, "tests"))
-        from helpers import oracle_layer, host_router
+        from oracle.synthetic import host_router, oracle_layer
         from quantized_mixture_experts_affine_b200 import synth
         self.cfg, self.oracle, self.np = cfg, oracle, np
         self.xb = synth.normal_bf16_host(seed, synth.tag(synth.X, 9999),
@@ -218,14 +257,22 @@ class OracleSample:
         """Threads the oracle actually uses for n_rows tokens (it splits tokens)."""
         return min(self.threads, n_rows)
 
-    def run(self, rows):
+    def run(self, rows, threads=None):
+        """Seconds of the oracle on the sample's tokens `rows` (threads: all
+        host cores when None)."""
         o, c = self.oracle, self.cfg
-        x = self.xb[rows]
-        t0 = time.perf_counter()
-        logits = o.qmv(self.R, x)
-        o.route(logits, c.K, c.renorm, c.router_scale)
-        o.expert_ffn(self.L, x, self.idx_c[rows], self.w[rows])
-        return time.perf_counter() - t0
+        prev = o.get_threads()
+        if threads is not None:
+            o.set_threads(threads)
+        try:
+            x = self.xb[rows]
+            t0 = time.perf_counter()
+            logits = o.qmv(self.R, x)
+            o.route(logits, c.K, c.renorm, c.router_scale)
+            o.expert_ffn(self.L, x, self.idx_c[rows], self.w[rows])
+            return time.perf_counter() - t0
+        finally:
+            o.set_threads(prev)
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)
@@ -233,9 +280,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from quantized_mixture_experts_affine_b200.layer import CONFIGS
     cfg_name, M = WORKLOADS[args.workload]
-    cfg = CONFIGS[cfg_name]
+    cfg = shape(cfg_name)
     pool = max(M, min(args.cpu_sample, args.steps * M))
     smp = OracleSample(cfg, pool)
     for w in range(args.warmup):
@@ -251,7 +297,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "tokens_per_step": M},
+            "config": config_of(args.workload, args.gpus, args.copies),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.cores(M),
                              "kind": "oracle",
                              "sample": f"{args.steps} steps of {M} token(s) of {args.workload}, "
@@ -262,15 +308,35 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ prefill measurement
-def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True):
+def timed_replays(fn, reps, st, world, local):
+    """Device time (max over ranks, ms) of reps calls of fn on stream st,
+    bracketed by a barrier and a synchronize, with the SM clocks sampled."""
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(st):
+            e0.record(st)
+            for _ in range(reps):
+                fn()
+            e1.record(st)
+        st.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1), world), clk
+
+
+def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True, min_ms=100):
     """Timed one-shot prefill calls of `workload` (M tokens each): device
     throughput, the gate/up gather-QMM duration per launch (events around it
     inside captured graphs), tensor-core roofline and end-to-end rate."""
     import torch
     from quantized_mixture_experts_affine_b200 import moeq, synth
-    from quantized_mixture_experts_affine_b200.layer import CONFIGS, Workspace, synthetic_layer
+    from quantized_mixture_experts_affine_b200.layer import Workspace, synthetic_layer
     cfg_name, M = WORKLOADS[workload]
-    cfg = CONFIGS[cfg_name]
+    cfg = shape(cfg_name)
     L = synthetic_layer(cfg, seed, 0)
     n_x = 2
     xs = synth.normal_bf16_dev(seed, synth.tag(synth.X, 555), n_x * M * cfg.H).view(n_x, M, cfg.H)
@@ -298,18 +364,14 @@ def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True):
     with torch.cuda.stream(st):
         g.replay()
     st.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
-        with torch.cuda.stream(st):
-            e0.record(st)
-            g.replay()
-            e1.record(st)
-        st.synchronize()
-    barrier(world)
-    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    ms, clk = timed_replays(lambda: g.replay(), 1, st, world, local)
+    ms /= steps
+    # the same graph replayed for at least min_ms (a long clock record)
+    reps = max(1, math.ceil(min_ms / max(ms * steps, 1e-3)))
+    ms_long, clk_long = timed_replays(lambda: g.replay(), reps, st, world, local)
+    sustained = {"steps": reps * steps, "timed_ms": ms_long, "ms_per_step": ms_long / (reps * steps),
+                 "value": M * world / (ms_long / (reps * steps) / 1e3), "clocks": clk_long.summary()}
     # gate/up gather-QMM per launch
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
@@ -330,9 +392,11 @@ def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True):
     gu_flop = 2.0 * n_pairs * 2 * cfg.I * cfg.H
     layer_flop = M * cfg.flops_per_token()
     _, peak_bf16, peak_kind = measured_peaks()
-    out = {"workload": workload, "tokens_per_step": M, "value": M * world / (ms / 1e3),
-           "unit": "tokens/s", "ms_per_step": ms,
+    out = {"workload": workload, "tokens_per_step": M, "steps": steps,
+           "value": M * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
            "layer_tflops": layer_flop / (ms / 1e3) / 1e12,
+           "layer_frac": layer_flop / (ms / 1e3) / 1e12 / peak_bf16,
+           "sustained": sustained,
            "roofline": {"bound": "tensor", "kernel": "k_gqmm gate/up+SwiGLU (fp16 operands)",
                         "achieved": gu_flop / (k_ms / 1e3) / 1e12, "peak": peak_bf16,
                         "unit": "TFLOP/s", "frac": gu_flop / (k_ms / 1e3) / 1e12 / peak_bf16,
@@ -373,11 +437,11 @@ def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True):
 def run_ours(args):
     import torch
     from quantized_mixture_experts_affine_b200 import moeq, synth
-    from quantized_mixture_experts_affine_b200.layer import CONFIGS, Workspace, synthetic_layer
+    from quantized_mixture_experts_affine_b200.layer import Workspace, synthetic_layer
 
     rank, world, local = dist_setup(args.gpus)
     cfg_name, M = WORKLOADS[args.workload]
-    cfg = CONFIGS[cfg_name]
+    cfg = shape(cfg_name)
     if args.workload.startswith("prefill"):
         return run_prefill_main(args, rank, world)
     K, W = args.steps, args.warmup
@@ -424,22 +488,31 @@ def run_ours(args):
     st.synchronize()
 
     peak_hbm, peak_bf16, peak_kind = measured_peaks()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(st):
-            ev0.record(st)
-            for g in graphs:
-                g.replay()
-            ev1.record(st)
-        st.synchronize()
-    torch.cuda.synchronize()
-    barrier(world)
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+
+    def replay_all():
+        for g in graphs:
+            g.replay()
+
+    # the timed region: exactly the K steps
+    ms_total, clk = timed_replays(replay_all, 1, st, world, local)
     ms_step = ms_total / K
     value = M * K * world / (ms_total / 1e3)
+    # the same K steps replayed for at least 100 ms (a long clock record)
+    reps = max(1, math.ceil(100.0 / max(ms_total, 1e-3)))
+    ms_long, clk_long = timed_replays(replay_all, reps, st, world, local)
+    sustained = {"steps": reps * K, "timed_ms": ms_long, "ms_per_step": ms_long / (reps * K),
+                 "value": M * reps * K * world / (ms_long / 1e3), "clocks": clk_long.summary()}
+    # without a graph: the K steps as eager calls through the C ABI, repeated
+    # for at least 100 ms (host launch cost included)
+    def eager_all():
+        for i in range(W, total_steps):
+            step(i, st)
+    ms_eager1, _ = timed_replays(eager_all, 1, st, world, local)
+    reps_e = max(1, math.ceil(100.0 / max(ms_eager1, 1e-3)))
+    ms_eager, clk_eager = timed_replays(eager_all, reps_e, st, world, local)
+    no_graph = {"steps": reps_e * K, "timed_ms": ms_eager,
+                "ms_per_step": ms_eager / (reps_e * K),
+                "value": M * reps_e * K * world / (ms_eager / 1e3), "clocks": clk_eager.summary()}
 
     # routing actually taken in the last steps -> distinct expert bytes per step
     exp_bytes = cfg.expert_bytes()
@@ -506,13 +579,10 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": args.workload, "tokens_per_step": M, "hidden": cfg.H,
-                   "experts": cfg.E, "top_k": cfg.K, "intermediate": cfg.I,
-                   "expert_bits": cfg.expert_bits, "router_bits": cfg.router_bits,
-                   "shared_expert": cfg.shared, "parallelism": f"replicas{world}",
-                   "l2": f"{copies} layer copies cycled, fresh tokens per step "
-                         f"({copies * layer_bytes / 1e6:.0f} MB touched per cycle > 126 MB L2)",
-                   "cuda_graph": True},
+        "config": config_of(args.workload, world, copies),
+        "cuda_graph": True,
+        "sustained": sustained,
+        "no_graph": no_graph,
         "layer_hbm": {"bytes_per_step": layer_bytes, "achieved_gbs": layer_bytes / (ms_step / 1e3) / 1e9,
                       "peak_gbs": peak_hbm, "frac": layer_bytes / (ms_step / 1e3) / 1e9 / peak_hbm,
                       "peak_kind": peak_kind},
@@ -540,6 +610,7 @@ def run_ours(args):
         torch.cuda.empty_cache()
         line["prefill"] = measure_prefill(args.prefill_workload, max(3, min(K, 20)), W, world,
                                           seed, want_e2e=not args.no_e2e)
+        line["prefill"]["config"] = config_of(args.prefill_workload, world, copies)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -557,16 +628,13 @@ def run_prefill_main(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": p["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic",
-            "config": {"workload": args.workload, "tokens_per_step": M,
-                       "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (weights, token rows and output rows)",
-                       "cuda_graph": True},
-            "layer_tflops": p["layer_tflops"], "roofline": p["roofline"], "e2e": p.get("e2e"),
+            "config": config_of(args.workload, world, args.copies), "cuda_graph": True,
+            "layer_tflops": p["layer_tflops"], "layer_frac": p["layer_frac"],
+            "sustained": p["sustained"], "roofline": p["roofline"], "e2e": p.get("e2e"),
             "gpu_launches": p["gpu_launches"], "clocks": p["clocks"],
             "device_status": p["device_status"]}
     if rank == 0 and not args.no_cpu_baseline:
-        from quantized_mixture_experts_affine_b200.layer import CONFIGS
-        smp = OracleSample(CONFIGS[cfg_name], args.cpu_sample)
+        smp = OracleSample(shape(cfg_name), args.cpu_sample)
         dt = smp.run(list(range(args.cpu_sample)))
         line["cpu_baseline"] = {"value": args.cpu_sample / dt, "unit": "tokens/s",
                                 "cores": smp.cores(args.cpu_sample), "kind": "oracle",
@@ -579,8 +647,125 @@ def run_prefill_main(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ per-config table
+# (row, shape, tokens per call, kind): kind "layer" = moeq_layer_forward in
+# AUTO mode; "zipf" = moeq_route_topk on router logits drawn with a Zipf
+# (s = 1.1) expert load, then moeq_expert_ffn in AUTO mode; "qmv" = the
+# standalone 8-bit router qmv 2816 -> 128.
+SWEEP = [
+    ("C1", "tiny", 1, "layer"), ("C1", "tiny", 3, "layer"), ("C1", "tiny", 5, "layer"),
+    ("C2", "decode_30b", 1, "layer"), ("C2", "router_2816", 1, "qmv"),
+    ("C3", "decode_397b", 1, "layer"), ("C3", "decode_397b", 8, "layer"),
+    ("C3", "decode_397b", 64, "layer"),
+    ("C4", "prefill_8bit", 16032, "layer"), ("C4", "prefill_8bit", 16068, "layer"),
+    ("C4", "prefill_8bit", 16384, "layer"),
+    ("C5", "mixed_2bit", 1, "zipf"), ("C5", "mixed_2bit", 256, "zipf"),
+    ("C5", "mixed_2bit", 4096, "zipf"),
+]
+
+
+def sweep_row(row, name, M, kind, copies, seed=0):
+    """GPU time per call (graph replays, >= 100 ms), tokens/s, roofline
+    fraction, and the oracle on a token sample (1 core and all cores)."""
+    import numpy as np
+    import torch
+    from quantized_mixture_experts_affine_b200 import moeq, synth
+    from quantized_mixture_experts_affine_b200.layer import Workspace, synthetic_layer
+    peak_hbm, peak_bf16, peak_kind = measured_peaks()
+    st = torch.cuda.Stream()
+    out = {"row": row, "shape": name, "tokens_per_call": M, "kind": kind}
+    if kind == "qmv":
+        H, E = 2816, 128
+        Ts = [synth.tensor_dev(seed, synth.tag(synth.ROUTER, 50 + c), 1, E, H, 8, 64)
+              for c in range(copies)]
+        descs = [moeq.qtensor(t.w, t.s, t.b, E, H, 8, 64, 1) for t in Ts]
+        x = synth.normal_bf16_dev(seed, synth.tag(synth.X, 51), H).view(1, H)
+        y = torch.empty((1, E), device="cuda")
+        call = lambda i: moeq.moeq_qmv(descs[i % copies], 0, x, 1, y, st)
+        nbytes = E * H + 4 * E * (H // 64)
+    else:
+        cfg = shape(name)
+        layers = [synthetic_layer(cfg, seed, c) for c in range(copies)]
+        xs = synth.normal_bf16_dev(seed, synth.tag(synth.X, 52), copies * M * cfg.H).view(
+            copies, M, cfg.H)
+        y = torch.empty((M, cfg.H), device="cuda")
+        idx = torch.empty((M, cfg.K), dtype=torch.int32, device="cuda")
+        w = torch.empty((M, cfg.K), device="cuda")
+        ws = Workspace(layers[0], M, moeq.MODE_AUTO)
+        if kind == "zipf":
+            lg, _ = synth.zipf_logits_host(seed, synth.tag(synth.LOGITS, 53), M, cfg.E, 1.1)
+            logits = torch.from_numpy(np.ascontiguousarray(lg)).cuda()
+
+            def call(i):
+                moeq.moeq_route_topk(logits, M, cfg.E, cfg.K, cfg.renorm, cfg.router_scale, idx,
+                                     w, st)
+                moeq.moeq_expert_ffn(layers[i % copies].desc, xs[i % copies], M, idx, w, None, y,
+                                     ws.buf, ws.bytes, moeq.MODE_AUTO, st)
+        else:
+            def call(i):
+                moeq.moeq_layer_forward(layers[i % copies].desc, xs[i % copies], M, y, None, idx,
+                                        w, ws.buf, ws.bytes, moeq.MODE_AUTO, st)
+    with torch.cuda.stream(st):
+        for i in range(3):
+            call(i)
+    st.synchronize()
+    n = copies if M < 1024 else 2
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for i in range(n):
+                call(i)
+        g.replay()
+    st.synchronize()
+    ms1, _ = timed_replays(lambda: g.replay(), 1, st, 1, 0)
+    reps = max(1, math.ceil(100.0 / max(ms1, 1e-3)))
+    ms, clk = timed_replays(lambda: g.replay(), reps, st, 1, 0)
+    ms_call = ms / (reps * n)
+    out.update({"gpu_ms": ms_call, "tokens_per_s": M / (ms_call / 1e3), "timed_ms": ms,
+                "clocks": clk.summary(), "device_status": moeq.moeq_device_status(st)})
+    if kind == "qmv":
+        out["roofline"] = {"bound": "hbm", "bytes": nbytes,
+                           "frac": nbytes / (ms_call / 1e3) / 1e9 / peak_hbm}
+    elif M * cfg.K <= 64 * cfg.K and M <= 64:
+        distinct = len(set(idx.cpu().numpy().ravel().tolist()))
+        nbytes = (0 if kind == "zipf" else cfg.router_bytes()) + distinct * cfg.expert_bytes() \
+            + cfg.shared_bytes()
+        out["roofline"] = {"bound": "hbm", "bytes": nbytes, "distinct_experts": distinct,
+                           "frac": nbytes / (ms_call / 1e3) / 1e9 / peak_hbm}
+    else:
+        flop = M * cfg.flops_per_token() - (2 * M * cfg.E * cfg.H if kind == "zipf" else 0)
+        out["roofline"] = {"bound": "tensor", "flop": flop,
+                           "frac": flop / (ms_call / 1e3) / 1e12 / peak_bf16}
+    out["roofline"]["peak_kind"] = peak_kind
+    del g
+    torch.cuda.empty_cache()
+    if kind != "qmv":
+        smp = OracleSample(cfg, 16)
+        t1 = smp.run([0], threads=1)
+        tn = smp.run(list(range(16)))
+        out["oracle"] = {"one_core_tokens_per_s": 1 / t1, "all_cores_tokens_per_s": 16 / tn,
+                         "cores": smp.cores(16), "sample": "1 token (1 core), 16 tokens (all cores)"}
+    return out
+
+
+def run_sweep(args):
+    import platform
+    import torch
+    torch.cuda.set_device(0)
+    head = {"sweep": "per-config table", "gpu": torch.cuda.get_device_name(0),
+            "host_cores": os.cpu_count(), "cpu": platform.processor() or platform.machine()}
+    print(json.dumps(head), flush=True)
+    for row, name, M, kind in SWEEP:
+        if args.sweep_rows and row not in args.sweep_rows.split(","):
+            continue
+        print(json.dumps(sweep_row(row, name, M, kind, args.copies)), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

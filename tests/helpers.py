@@ -5,8 +5,7 @@ from __future__ import annotations
 import numpy as np
 
 import oracle
-from quantized_mixture_experts_affine_b200 import synth
-from quantized_mixture_experts_affine_b200.layer import LayerConfig
+from oracle.synthetic import host_router, host_tensor, oracle_layer  # noqa: F401
 
 # Pass criteria for layer outputs against the fp64 oracle on the same bf16 inputs.
 REL_L2 = 2e-3
@@ -20,45 +19,6 @@ def rel_l2(a, b) -> float:
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
-
-
-def host_tensor(cfg: LayerConfig, seed: int, kind: int, copy: int, out_dim: int, in_dim: int,
-                bits: int, mats=None, requant=False):
-    """Host copy of a bank (all matrices, or the listed ones stacked in order)."""
-    tg = synth.tag(kind, copy)
-    if mats is None:
-        return synth.tensor_host(seed, tg, 1, out_dim, in_dim, bits, cfg.G, requant)
-    parts = [synth.tensor_host(seed, tg, 1, out_dim, in_dim, bits, cfg.G, requant, first_mat=int(m))
-             for m in mats]
-    return synth.HostQ(np.ascontiguousarray(np.concatenate([p.w for p in parts])),
-                       np.ascontiguousarray(np.concatenate([p.s for p in parts])),
-                       np.ascontiguousarray(np.concatenate([p.b for p in parts])),
-                       out_dim, in_dim, bits, cfg.G, len(parts))
-
-
-def host_router(cfg, seed, copy=0):
-    return host_tensor(cfg, seed, synth.ROUTER, copy, cfg.E, cfg.H, cfg.router_bits)
-
-
-def oracle_layer(cfg: LayerConfig, seed: int, copy: int, experts):
-    """Oracle layer whose banks hold only `experts` (in that order)."""
-    rq = cfg.requant_from4
-    O = oracle.OracleTensor.of
-    kw = {}
-    if cfg.shared:
-        kw = dict(
-            sh_gate=O(host_tensor(cfg, seed, synth.SH_GATE, copy, cfg.shared_I, cfg.H, cfg.shared_bits)),
-            sh_up=O(host_tensor(cfg, seed, synth.SH_UP, copy, cfg.shared_I, cfg.H, cfg.shared_bits)),
-            sh_down=O(host_tensor(cfg, seed, synth.SH_DOWN, copy, cfg.H, cfg.shared_I, cfg.shared_bits)),
-            sh_expert_gate=O(host_tensor(cfg, seed, synth.SH_EXPERT_GATE, copy, 1, cfg.H,
-                                         cfg.shared_gate_bits)))
-    return oracle.OracleLayer(
-        router=O(host_router(cfg, seed, copy)),
-        gate=O(host_tensor(cfg, seed, synth.GATE, copy, cfg.I, cfg.H, cfg.expert_bits, experts, rq)),
-        up=O(host_tensor(cfg, seed, synth.UP, copy, cfg.I, cfg.H, cfg.expert_bits, experts, rq)),
-        down=O(host_tensor(cfg, seed, synth.DOWN, copy, cfg.H, cfg.I, cfg.expert_bits, experts, rq)),
-        H=cfg.H, I=cfg.I, E=len(experts), K=cfg.K, renorm=cfg.renorm,
-        router_scale=cfg.router_scale, **kw)
 
 
 def oracle_expert_outputs(cfg, seed, copy, x_bits, idx, wts, residual=None):
