@@ -20,4 +20,5 @@ from .oracle import (  # noqa: F401
     route_f32,
     expert_ffn,
     layer,
+    rmsnorm,
 )

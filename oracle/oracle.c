@@ -344,3 +344,21 @@ ORC_API void oracle_layer(const orc_layer* L, const uint16_t* x_bf16, int M, con
     free(x);
   }
 }
+
+/*
+ * RMS norm of the combined output, the step the pages run after the
+ * combine ("flash-moe-inference", per-layer pipeline: "CMD3: expert forward
+ * + combine + norm"; rms_norm_pass1 = sum of squares, rms_norm_pass2 =
+ * apply):  out[t][j] = y[t][j] / sqrt((1/H) sum_i y[t][i]^2 + eps) * g[j],
+ * g the bf16 weight vector.  fp64 throughout.
+ */
+ORC_API void oracle_rmsnorm(const double* y, int M, int H, const uint16_t* g_bf16, double eps,
+                            double* out) {
+  for (int t = 0; t < M; ++t) {
+    const double* r = y + (int64_t)t * H;
+    double ss = 0.0;
+    for (int i = 0; i < H; ++i) ss += r[i] * r[i];
+    const double inv = 1.0 / sqrt(ss / H + eps);
+    for (int j = 0; j < H; ++j) out[(int64_t)t * H + j] = r[j] * inv * orc_bf16(g_bf16[j]);
+  }
+}

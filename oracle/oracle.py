@@ -121,6 +121,7 @@ def _L():
                                           P, P]
         _lib.oracle_expert_ffn.argtypes = [C.POINTER(_Layer), P, C.c_int, P, P, P, P]
         _lib.oracle_layer.argtypes = [C.POINTER(_Layer), P, C.c_int, P, P, P, P, P, P]
+        _lib.oracle_rmsnorm.argtypes = [P, C.c_int, C.c_int, P, C.c_double, P]
     return _lib
 
 
@@ -217,3 +218,14 @@ def layer(L: OracleLayer, x_bf16: np.ndarray, residual: np.ndarray | None = None
     _L().oracle_layer(C.byref(cl), _ptr(x), M, _ptr(res), _ptr(out), _ptr(idx), _ptr(w),
                       _ptr(gap), _ptr(logits))
     return dict(out=out, idx=idx, w=w, gap=gap, logits=logits)
+
+
+def rmsnorm(y: np.ndarray, gamma_bf16: np.ndarray, eps: float) -> np.ndarray:
+    """RMS norm of each row of y (fp64 [M][H]) with the bf16 weights gamma
+    ([H] bit patterns): y / sqrt(mean(y^2) + eps) * gamma, in fp64."""
+    y = np.ascontiguousarray(y, np.float64)
+    M, H = y.reshape(-1, y.shape[-1]).shape
+    g = np.ascontiguousarray(gamma_bf16, np.uint16).reshape(H)
+    out = np.empty((M, H), np.float64)
+    _L().oracle_rmsnorm(_ptr(y), M, H, _ptr(g), float(eps), _ptr(out))
+    return out

@@ -212,8 +212,8 @@ def test_zero_scale_groups(M):
 def tiny_scale_layer(exact=True):
     """8-bit experts whose group scales lie in [2^-17, 2^-14) (below the fp16
     normal range, exact as fp16 subnormals) with biases of ordinary size;
-    with exact=False one group of expert 0's gate gets 1.5 * 2^-20, which
-    fp16 cannot hold exactly."""
+    with exact=False the first group of every gate row gets 1.5 * 2^-24,
+    which fp16 cannot hold (its subnormal step is 2^-24)."""
     cfg = EDGE8
     t = host_layer(cfg, copy=3)
     rng = np.random.default_rng(11)
@@ -223,7 +223,7 @@ def tiny_scale_layer(exact=True):
         mag = 2.0 ** rng.integers(-17, -14, h.s.shape) * (1 + rng.integers(0, 8, h.s.shape) / 8)
         h.s[sel] = bf16_bits(mag[sel])
     if not exact:
-        t["gate"].s[:, :, 0] = bf16_bits(1.5 * 2.0 ** -20)
+        t["gate"].s[:, :, 0] = bf16_bits(1.5 * 2.0 ** -24)
     return cfg, t
 
 

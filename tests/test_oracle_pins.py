@@ -435,3 +435,35 @@ def test_route_under_exp_underflow_selects_by_logit():
     # a negative router scale reverses the order of the logits
     idx, _, _ = oracle.route(l, 2, True, -1.0)
     assert idx[0].tolist() == [1, 2]
+
+
+# ------------------------------------------------------------------ RMS norm of the output
+
+def _bf16(v):
+    u = np.asarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def test_rmsnorm_worked_row():
+    """(3, 4): mean square 12.5, so with eps 0 and unit weights the row
+    becomes (3, 4) / sqrt(12.5); weights 2 and 0.5 scale each column."""
+    out = oracle.rmsnorm(np.array([[3.0, 4.0]]), _bf16([1.0, 1.0]), 0.0)
+    assert np.allclose(out, [[3 / np.sqrt(12.5), 4 / np.sqrt(12.5)]], rtol=1e-15)
+    out = oracle.rmsnorm(np.array([[3.0, 4.0]]), _bf16([2.0, 0.5]), 0.0)
+    assert np.allclose(out, [[6 / np.sqrt(12.5), 2 / np.sqrt(12.5)]], rtol=1e-15)
+
+
+def test_rmsnorm_invariants():
+    """With eps 0 and unit weights every output row has mean square 1, and
+    the result does not change when a row is scaled by a positive factor;
+    with eps > 0 a constant row c gives c / sqrt(c^2 + eps)."""
+    rng = np.random.default_rng(3)
+    y = rng.normal(size=(5, 64)) * rng.uniform(0.1, 100, size=(5, 1))
+    one = _bf16(np.ones(64))
+    out = oracle.rmsnorm(y, one, 0.0)
+    assert np.allclose((out ** 2).mean(axis=1), 1.0, rtol=1e-13)
+    assert np.allclose(oracle.rmsnorm(7.5 * y, one, 0.0), out, rtol=1e-13)
+    c = oracle.rmsnorm(np.full((1, 8), 0.5), _bf16(np.ones(8)), 1e-2)
+    assert np.allclose(c, 0.5 / np.sqrt(0.25 + 1e-2), rtol=1e-15)
+    # rows are independent of one another
+    assert np.allclose(oracle.rmsnorm(y[2:3], one, 1e-6), oracle.rmsnorm(y, one, 1e-6)[2:3])
