@@ -189,6 +189,29 @@ moeq_status moeq_layer_forward(const moeq_layer* L, const uint16_t* x, int32_t M
                                const float* residual, int32_t* idx_out, float* w_out, void* ws,
                                size_t ws_bytes, int32_t mode, void* stream);
 
+/*
+ * moeq_layer_forward followed by the step the pages run after the combine,
+ * the RMS norm of the combined output ("flash-moe-inference", per-layer
+ * pipeline "CMD3: expert forward + combine + norm"; Key Metal kernels
+ * rms_norm_pass1 / rms_norm_pass2):
+ *   y[m]         as moeq_layer_forward (fp32 [M][H], the residual stream)
+ *   y_norm[m][j] = bf16( y[m][j] / sqrt((1/H) sum_i y[m][i]^2 + eps) * gamma[j] )
+ *                  (round to nearest even), the next layer's bf16 input.
+ *   gamma: bf16 [H] (device, 16-byte aligned); y_norm: bf16 [M][H] (device,
+ *   16-byte aligned, written whole); eps > 0 and finite.  The sum of
+ *   squares is an fp32 sum in a fixed order, so results are deterministic;
+ *   in PREFILL mode the norm runs inside the combine (one pass over the
+ *   rows) and chunked calls stay bit-identical; in DECODE mode one row-norm
+ *   launch follows the combine.
+ * Same workspace as moeq_layer_forward.  Errors: those of
+ * moeq_layer_forward; INVALID_ARG for a null gamma or y_norm or a bad eps,
+ * ALIGNMENT for a misaligned gamma or y_norm.
+ */
+moeq_status moeq_layer_forward_norm(const moeq_layer* L, const uint16_t* x, int32_t M, float* y,
+                                    const float* residual, const uint16_t* gamma, float eps,
+                                    uint16_t* y_norm, int32_t* idx_out, float* w_out, void* ws,
+                                    size_t ws_bytes, int32_t mode, void* stream);
+
 /* Workspace bytes moeq_expert_ffn / moeq_layer_forward need for M tokens
  * in `mode` (0 if the arguments are invalid). */
 size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mode);

@@ -1,6 +1,7 @@
 // C ABI of libmoeq.so (include/moeq.h): argument checks, workspace layout
 // and the launch sequences of the decode and prefill paths.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -627,7 +628,8 @@ moeq_status forward_arg_check(const moeq_layer* L, const uint16_t* x, int32_t M,
 static moeq_status forward_common(const moeq_layer* L, const uint16_t* x, int32_t M,
                                   const int32_t* idx_in, const float* w_in, const float* residual,
                                   float* y, int32_t* idx_out, float* w_out, void* ws,
-                                  size_t ws_bytes, int32_t mode, void* stream) {
+                                  size_t ws_bytes, int32_t mode, void* stream,
+                                  const NormOut* norm = nullptr) {
   moeq_status s = forward_arg_check(L, x, M, y, residual, mode);
   if (s != MOEQ_OK || M == 0) return s;
   mode = resolve_mode(mode, M);
@@ -640,10 +642,12 @@ static moeq_status forward_common(const moeq_layer* L, const uint16_t* x, int32_
   if (mode == MOEQ_MODE_DECODE) {
     if (M > kMaxDecodeM) return MOEQ_ERR_UNSUPPORTED;
     if ((s = check_decode_shapes(L)) != MOEQ_OK) return s;
-    return decode_forward(L, x, M, idx_in, w_in, residual, y, idx_out, w_out, ws, st);
+    s = decode_forward(L, x, M, idx_in, w_in, residual, y, idx_out, w_out, ws, st);
+    if (s == MOEQ_OK && norm) LAUNCH(launch_rmsnorm_rows(y, M, L->hidden, *norm, st));
+    return s;
   }
   return prefill_forward(L, x, M, idx_in, w_in, residual, y, idx_out, w_out, ws, ws_bytes,
-                         status_ptr(), st);
+                         status_ptr(), st, norm);
 }
 
 MOEQ_API moeq_status moeq_expert_ffn(const moeq_layer* L, const uint16_t* x, int32_t M,
@@ -661,6 +665,20 @@ MOEQ_API moeq_status moeq_layer_forward(const moeq_layer* L, const uint16_t* x, 
                                         void* stream) {
   return forward_common(L, x, M, nullptr, nullptr, residual, y, idx_out, w_out, ws, ws_bytes,
                         mode, stream);
+}
+
+MOEQ_API moeq_status moeq_layer_forward_norm(const moeq_layer* L, const uint16_t* x, int32_t M,
+                                             float* y, const float* residual,
+                                             const uint16_t* gamma, float eps, uint16_t* y_norm,
+                                             int32_t* idx_out, float* w_out, void* ws,
+                                             size_t ws_bytes, int32_t mode, void* stream) {
+  moeq_status s = forward_arg_check(L, x, M, y, residual, mode);
+  if (s != MOEQ_OK || M == 0) return s;
+  if (!gamma || !y_norm || !(eps > 0.0f) || !(eps < INFINITY)) return MOEQ_ERR_INVALID_ARG;
+  if (!aligned(gamma, 16) || !aligned(y_norm, 16)) return MOEQ_ERR_ALIGNMENT;
+  const NormOut n{gamma, eps, y_norm};
+  return forward_common(L, x, M, nullptr, nullptr, residual, y, idx_out, w_out, ws, ws_bytes,
+                        mode, stream, &n);
 }
 
 MOEQ_API moeq_status moeq_set_profile_events(void* start, void* stop) {

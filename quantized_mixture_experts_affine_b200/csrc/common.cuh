@@ -63,6 +63,20 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Sum of one value per thread over a CTA of 256 threads, in a fixed order
+// (warps, then the eight warp totals in order); red: 8 floats of shared memory.
+__device__ __forceinline__ float row_sum_256(float v, float* red) {
+  v = warp_sum(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t += red[i];
+  __syncthreads();
+  return t;
+}
+
+
 // ------------------------------------------------------------------ code registers
 // A 16-byte chunk of a packed row holds VPC = 128/BITS codes in 4 words.
 // It is split into NC = VPC/4 "code registers", each holding 4 codes in its

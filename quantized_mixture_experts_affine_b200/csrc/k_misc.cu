@@ -1,6 +1,8 @@
-// Unpack / dequantise one matrix (bit-exact reference form of the format).
+// Unpack / dequantise one matrix (bit-exact reference form of the format);
+// RMS norm of output rows.
 #include "common.cuh"
 #include "kernels.h"
+#include "prefill.h"
 
 namespace moeq {
 
@@ -47,6 +49,53 @@ cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, fl
     case 4: k_dequant<4><<<(int)grid, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out); break;
     default: k_dequant<8><<<(int)grid, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out); break;
   }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ RMS norm of output rows
+// y_norm[t][j] = bf16(y[t][j] / sqrt((1/H) sum_i y[t][i]^2 + eps) * g[j]),
+// one CTA of 256 threads per row ("flash-moe-inference", rms_norm_pass1/2:
+// the sum of squares, then the scaling).  H a multiple of 8.
+__global__ void __launch_bounds__(256) k_rmsnorm_rows(const float* __restrict__ y, int M, int H,
+                                                      const uint16_t* __restrict__ gamma,
+                                                      float eps, uint16_t* __restrict__ y_norm) {
+  __shared__ float red[8];
+  const int H8 = H >> 3;
+  for (int t = blockIdx.x; t < M; t += gridDim.x) {
+    const float4* r = reinterpret_cast<const float4*>(y + (int64_t)t * H);
+    float ss = 0.0f;
+    for (int i = threadIdx.x; i < 2 * H8; i += 256) {
+      const float4 v = r[i];
+      ss = fmaf(v.x, v.x, ss);
+      ss = fmaf(v.y, v.y, ss);
+      ss = fmaf(v.z, v.z, ss);
+      ss = fmaf(v.w, v.w, ss);
+    }
+    const float inv = 1.0f / sqrtf(row_sum_256(ss, red) / (float)H + eps);
+    uint4* o = reinterpret_cast<uint4*>(y_norm + (int64_t)t * H);
+    const uint4* g = reinterpret_cast<const uint4*>(gamma);
+    for (int i = threadIdx.x; i < H8; i += 256) {
+      const float4 a = r[2 * i], b = r[2 * i + 1];
+      const uint4 gw = g[i];
+      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w};
+      uint32_t out[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = v[2 * j] * inv * __uint_as_float(gg[j] << 16);
+        const float hi = v[2 * j + 1] * inv * __uint_as_float(gg[j] & 0xFFFF0000u);
+        out[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+      }
+      o[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+  }
+}
+
+cudaError_t launch_rmsnorm_rows(const float* y, int M, int H, const NormOut& n, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  const int grid = M < 148 * 8 ? M : 148 * 8;
+  k_rmsnorm_rows<<<grid, 256, 0, st>>>(y, M, H, n.gamma, n.eps, n.y_norm);
   return cudaGetLastError();
 }
 

@@ -111,6 +111,78 @@ __global__ void __launch_bounds__(256) k_combine_h(const uint4* __restrict__ d,
   }
 }
 
+// k_combine_h followed by the RMS norm of each row, in one pass over the
+// fp16 down rows: one CTA per row keeps its NC8 chunks of eight columns per
+// thread in registers while the row's sum of squares is reduced (fixed
+// order), then writes y and y_norm[t][j] = bf16(y[t][j] / sqrt(mean(y[t]^2)
+// + eps) * gamma[j]) ("flash-moe-inference", per-layer pipeline: combine +
+// norm; rms_norm_pass1/2).  H <= 2048 * NC8.
+template <int NC8>
+__global__ void __launch_bounds__(256) k_combine_norm(const uint4* __restrict__ d,
+                                                      const float* __restrict__ w,
+                                                      const float* __restrict__ sigma,
+                                                      int has_shared,
+                                                      const float* __restrict__ residual,
+                                                      float* __restrict__ y, int M, int K, int H,
+                                                      const uint16_t* __restrict__ gamma,
+                                                      float eps, uint16_t* __restrict__ y_norm) {
+  __shared__ float red[8];
+  const int H8 = H >> 3;
+  for (int t = blockIdx.x; t < M; t += gridDim.x) {
+    float acc[NC8][8];
+    float ss = 0.0f;
+#pragma unroll
+    for (int c = 0; c < NC8; ++c) {
+      const int c8 = threadIdx.x + 256 * c;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[c][j] = 0.0f;
+      if (c8 < H8) {
+        auto add = [&](float s, const uint4 v) {
+          const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(h[j]);
+            acc[c][2 * j] = fmaf(s, f.x, acc[c][2 * j]);
+            acc[c][2 * j + 1] = fmaf(s, f.y, acc[c][2 * j + 1]);
+          }
+        };
+        for (int k = 0; k < K; ++k) add(w[(int64_t)t * K + k], d[((int64_t)t * K + k) * H8 + c8]);
+        if (has_shared) add(sigma[t], d[((int64_t)M * K + t) * H8 + c8]);
+        if (residual) {
+          const float4* r = reinterpret_cast<const float4*>(residual + (int64_t)t * H) + 2 * c8;
+          const float4 r0 = r[0], r1 = r[1];
+          acc[c][0] += r0.x; acc[c][1] += r0.y; acc[c][2] += r0.z; acc[c][3] += r0.w;
+          acc[c][4] += r1.x; acc[c][5] += r1.y; acc[c][6] += r1.z; acc[c][7] += r1.w;
+        }
+        float4* o = reinterpret_cast<float4*>(y + (int64_t)t * H) + 2 * c8;
+        o[0] = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+        o[1] = make_float4(acc[c][4], acc[c][5], acc[c][6], acc[c][7]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = fmaf(acc[c][j], acc[c][j], ss);
+      }
+    }
+    const float inv = 1.0f / sqrtf(row_sum_256(ss, red) / (float)H + eps);
+#pragma unroll
+    for (int c = 0; c < NC8; ++c) {
+      const int c8 = threadIdx.x + 256 * c;
+      if (c8 < H8) {
+        const uint4 gw = reinterpret_cast<const uint4*>(gamma)[c8];
+        const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float lo = acc[c][2 * j] * inv * __uint_as_float(gg[j] << 16);
+          const float hi = acc[c][2 * j + 1] * inv * __uint_as_float(gg[j] & 0xFFFF0000u);
+          out[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+        }
+        reinterpret_cast<uint4*>(y_norm + (int64_t)t * H)[c8] =
+            make_uint4(out[0], out[1], out[2], out[3]);
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ routing (strided logits)
 __global__ void __launch_bounds__(256) k_route_prefill(const float* __restrict__ logits, int64_t ld,
                                                        int M, int E, int K, int renorm,
@@ -589,7 +661,7 @@ size_t prefill_workspace_bytes(const moeq_layer* L, int M) {
 moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const int32_t* idx_in,
                             const float* w_in, const float* residual, float* y, int32_t* idx_out,
                             float* w_out, void* ws, size_t ws_bytes, int* status,
-                            cudaStream_t st) {
+                            cudaStream_t st, const NormOut* norm) {
   moeq_status s = check_prefill(L);
   if (s != MOEQ_OK) return s;
   const int E = L->n_experts, K = L->top_k, H = L->hidden, I = L->inter;
@@ -801,9 +873,29 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     const int64_t total = (int64_t)M * (H / 8);
     int64_t grid = (total + 255) / 256;
     if (grid > (int64_t)sms * 16) grid = (int64_t)sms * 16;
-    k_combine_h<<<(int)grid, 256, 0, st>>>((const uint4*)yrows, wts, sigma, L->has_shared,
-                                           residual, y, M, K, H);
-    PCK(cudaGetLastError());
+    const int H8 = H / 8;
+    if (norm && H8 <= 256 * 4) {
+      // combine and norm in one pass: one CTA per row
+      const int g = M < sms * 8 ? M : sms * 8;
+      if (H8 <= 256)
+        k_combine_norm<1><<<g, 256, 0, st>>>((const uint4*)yrows, wts, sigma, L->has_shared,
+                                             residual, y, M, K, H, norm->gamma, norm->eps,
+                                             norm->y_norm);
+      else if (H8 <= 512)
+        k_combine_norm<2><<<g, 256, 0, st>>>((const uint4*)yrows, wts, sigma, L->has_shared,
+                                             residual, y, M, K, H, norm->gamma, norm->eps,
+                                             norm->y_norm);
+      else
+        k_combine_norm<4><<<g, 256, 0, st>>>((const uint4*)yrows, wts, sigma, L->has_shared,
+                                             residual, y, M, K, H, norm->gamma, norm->eps,
+                                             norm->y_norm);
+      PCK(cudaGetLastError());
+    } else {
+      k_combine_h<<<(int)grid, 256, 0, st>>>((const uint4*)yrows, wts, sigma, L->has_shared,
+                                             residual, y, M, K, H);
+      PCK(cudaGetLastError());
+      if (norm) PCK(launch_rmsnorm_rows(y, M, H, *norm, st));
+    }
   }
   return MOEQ_OK;
 }

@@ -96,6 +96,27 @@ def layer_forward(L: DeviceLayer, x, y=None, residual=None, idx=None, w=None, ws
     return y, idx, w
 
 
+def layer_forward_norm(L: DeviceLayer, x, gamma, eps: float, y=None, y_norm=None, residual=None,
+                       idx=None, w=None, ws=None, mode: int = moeq.MODE_AUTO, stream=None):
+    """y = layer(x) and y_norm = bf16 RMS norm of y with weights gamma (bf16
+    [H]); returns (y, y_norm, idx, w)."""
+    import torch
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, L.cfg.H), dtype=torch.float32, device=x.device)
+    if y_norm is None:
+        y_norm = torch.empty((M, L.cfg.H), dtype=torch.bfloat16, device=x.device)
+    if idx is None:
+        idx = torch.empty((M, L.cfg.K), dtype=torch.int32, device=x.device)
+    if w is None:
+        w = torch.empty((M, L.cfg.K), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = Workspace(L, M, mode, x.device)
+    moeq.moeq_layer_forward_norm(L.desc, x, M, y, gamma, eps, y_norm, residual, idx, w, ws.buf,
+                                 ws.bytes, mode, stream)
+    return y, y_norm, idx, w
+
+
 def expert_ffn(L: DeviceLayer, x, idx, w, y=None, residual=None, ws=None,
                mode: int = moeq.MODE_AUTO, stream=None):
     import torch

@@ -26,7 +26,8 @@ MODE_AUTO, MODE_DECODE, MODE_PREFILL = 0, 1, 2
 EXPORTS = ("moeq_dequant", "moeq_qmv", "moeq_route_topk", "moeq_expert_ffn", "moeq_layer_forward",
            "moeq_workspace_bytes", "moeq_device_status", "moeq_status_str", "moeq_version",
            "moeq_set_profile_events", "moeq_launch_count", "moeq_layer_forward_static",
-           "moeq_static_workspace_capacity", "moeq_selftest_wait_timeout")
+           "moeq_static_workspace_capacity", "moeq_selftest_wait_timeout",
+           "moeq_layer_forward_norm")
 
 
 class MoeqError(RuntimeError):
@@ -62,6 +63,8 @@ _lib.moeq_expert_ffn.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P
 _lib.moeq_layer_forward.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P, _P,
                                     C.c_size_t, C.c_int32, _P]
 _lib.moeq_layer_forward_static.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P, _P]
+_lib.moeq_layer_forward_norm.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, C.c_float,
+                                         _P, _P, _P, _P, C.c_size_t, C.c_int32, _P]
 _lib.moeq_static_workspace_capacity.restype = C.c_size_t
 _lib.moeq_workspace_bytes.argtypes = [C.POINTER(Layer), C.c_int32, C.c_int32]
 _lib.moeq_workspace_bytes.restype = C.c_size_t
@@ -74,7 +77,8 @@ _lib.moeq_set_profile_events.argtypes = [_P, _P]
 _lib.moeq_set_profile_events.restype = C.c_int
 _lib.moeq_launch_count.restype = C.c_uint64
 for _f in ("moeq_dequant", "moeq_qmv", "moeq_route_topk", "moeq_expert_ffn", "moeq_layer_forward",
-           "moeq_layer_forward_static", "moeq_device_status", "moeq_selftest_wait_timeout"):
+           "moeq_layer_forward_static", "moeq_device_status", "moeq_selftest_wait_timeout",
+           "moeq_layer_forward_norm"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -152,6 +156,16 @@ def moeq_layer_forward(L: Layer, x, M: int, y, residual=None, idx_out=None, w_ou
            _lib.moeq_layer_forward(C.byref(L), _ptr(x), M, _ptr(y), _ptr(residual),
                                    _ptr(idx_out), _ptr(w_out), _ptr(ws), ws_bytes, mode,
                                    _stream(stream)))
+
+
+def moeq_layer_forward_norm(L: Layer, x, M: int, y, gamma, eps: float, y_norm, residual=None,
+                            idx_out=None, w_out=None, ws=None, ws_bytes: int = 0,
+                            mode: int = MODE_AUTO, stream=None) -> None:
+    """moeq_layer_forward plus y_norm = bf16 RMS norm of y with weights gamma."""
+    _check("moeq_layer_forward_norm",
+           _lib.moeq_layer_forward_norm(C.byref(L), _ptr(x), M, _ptr(y), _ptr(residual),
+                                        _ptr(gamma), float(eps), _ptr(y_norm), _ptr(idx_out),
+                                        _ptr(w_out), _ptr(ws), ws_bytes, mode, _stream(stream)))
 
 
 def moeq_layer_forward_static(L: Layer, x, M: int, y, residual=None, idx_out=None, w_out=None,

@@ -162,3 +162,24 @@ def test_static_entry_checks_arguments_before_capacity():
     # valid pointers: now the capacity decides (nothing launched, no device needed)
     assert fwd_static(big, M=64) == moeq.ERR_WORKSPACE
     assert fwd_static(layer(), M=65) == moeq.ERR_UNSUPPORTED
+
+
+def test_norm_entry_argument_checks():
+    """moeq_layer_forward_norm: the forward's checks first, then gamma,
+    y_norm and eps; nothing is launched on a failed check."""
+    L = layer()
+    f = moeq.lib().moeq_layer_forward_norm
+
+    def call(x=A, y=A, gamma=A, eps=1e-6, y_norm=A, M=1):
+        return f(C.byref(L), x, M, y, None, gamma, eps, y_norm, None, None, A, 1 << 30,
+                 moeq.MODE_DECODE, None)
+    assert call(x=0) == moeq.ERR_INVALID_ARG
+    assert call(gamma=0) == moeq.ERR_INVALID_ARG
+    assert call(y_norm=0) == moeq.ERR_INVALID_ARG
+    assert call(eps=0.0) == moeq.ERR_INVALID_ARG
+    assert call(eps=-1.0) == moeq.ERR_INVALID_ARG
+    assert call(eps=float("inf")) == moeq.ERR_INVALID_ARG
+    assert call(eps=float("nan")) == moeq.ERR_INVALID_ARG
+    assert call(gamma=A + 2) == moeq.ERR_ALIGNMENT
+    assert call(y_norm=A + 8) == moeq.ERR_ALIGNMENT
+    assert call(M=0, gamma=0) == moeq.OK
