@@ -149,8 +149,11 @@ moeq_status moeq_route_topk(const float* logits, int32_t M, int32_t E, int32_t K
  *   ws: device workspace of at least moeq_workspace_bytes(L, M, mode) bytes,
  *   256-byte aligned, owned by the caller, contents ignored on entry.
  * mode: DECODE requires M <= 64 and rows of at most 4096 bytes of codes.
- * PREFILL requires group_size 64 for every tensor, H, I (and the shared
- * expert's I) multiples of 128, 4-byte aligned scale/bias arrays, and
+ * PREFILL requires group sizes of 32, 64 or 128 (32 only for 4- and 8-bit
+ * codes), one group size for gate and up and one for the shared expert's
+ * gate and up, H, I (and the shared expert's I) multiples of 128 and of
+ * 2 * group_size for the tensors that reduce over them, 4-byte aligned
+ * scale/bias arrays, and
  * values that fit the fp16 tensor-core operands (|x|, |bias| and
  * |bias + (2^b-1)*scale| at most 65504, every scale exactly representable
  * as fp16: all bf16 scales of magnitude 2^-17 to 65504 are, and smaller

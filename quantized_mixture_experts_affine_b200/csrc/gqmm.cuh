@@ -131,10 +131,20 @@ struct Args {
   void* out;
   int64_t ldo;              // elements
   int32_t out_f16;          // STORE: fp16 output rows (range-checked) instead of fp32
-  int32_t sb_w;             // groups per scale/bias window copy: 8, 4 or 2 (dividing K/64;
-                            // scale/bias rows aligned to 2*sb_w bytes)
+  int32_t sb_w;             // groups per scale/bias window copy: 8, 4 or 2 (dividing K/G;
+                            // scale/bias rows aligned to 2*sb_w bytes; a window spans
+                            // sb_w*G/64 >= 2 k-blocks)
+  int32_t G;                // group size of the launch's tensors: 32, 64 or 128 (32: not
+                            // 2-bit, whose 16-byte code chunks span two groups)
   int* status;
 };
+
+// k-blocks (of BK = 64 values) spanned by a window of W groups of size G,
+// as a power of two: log2(W * G / 64).
+__host__ __device__ __forceinline__ int win_kb_log2(int W, int G) {
+  const int wl = W == 8 ? 3 : W == 4 ? 2 : 1;
+  return wl + (G == 128 ? 1 : G == 32 ? -1 : 0);
+}
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                        uint32_t d) {
@@ -468,8 +478,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
   } else if (warp == 2) {
     // ------------------------------------------------------------ B loader
     // this CTA's BR weight rows of the tile: rows rank*BR + (lane + 32 j)
-    const int groups = a.K / 64;
-    const int W = a.sb_w, wl = W == 8 ? 3 : W == 4 ? 2 : 1;
+    const int groups = a.K / a.G;
+    const int W = a.sb_w, wl = win_kb_log2(W, a.G);
     const int64_t wrow = (int64_t)a.K * BITS / 32;  // words per weight row
     constexpr int JR = BR / 32;
     uint32_t it = 0;
@@ -501,10 +511,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         const uint32_t s = it % SR, ph = (it / SR) & 1u;
         if (!tc::mbar_wait(&raw_empty[s], ph ^ 1u, status)) goto done;
         const uint32_t rst = sbase + SM::RAW_OFF + s * SM::RAW_STAGE;
-        // a new scale/bias window every sb_w k-blocks (windows counted over
-        // the whole item loop, like the dequantiser)
-        const bool new_win = (kb & (W - 1)) == 0;
+        // a new scale/bias window (W groups) every 2^wl k-blocks (windows
+        // counted over the whole item loop, like the dequantiser); its
+        // first group is group kb * 64 / G of the row
+        const bool new_win = (kb & ((1 << wl) - 1)) == 0;
         const uint32_t sbw = sbase + SM::SB_OFF + ((it >> wl) % SM::NWB) * SM::SB_WIN;
+        const int g0 = a.G == 64 ? kb : a.G == 128 ? kb >> 1 : kb << 1;
         if (a.tma_b) {
           if (lane == 0) {
             tc::mbar_expect_tx(&raw_full[s], (uint32_t)SM::RAW_STAGE);
@@ -533,14 +545,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
             const int r = lane + 32 * j;
             const uint32_t d = sbw + r * 32;
             if (W == 8) {
-              tc::cp_async16(d, sp[j] + kb, ok16[j]);
-              tc::cp_async16(d + 16, bp[j] + kb, ok16[j]);
+              tc::cp_async16(d, sp[j] + g0, ok16[j]);
+              tc::cp_async16(d + 16, bp[j] + g0, ok16[j]);
             } else if (W == 4) {
-              tc::cp_async8(d, sp[j] + kb, ok16[j] ? 8u : 0u);
-              tc::cp_async8(d + 16, bp[j] + kb, ok16[j] ? 8u : 0u);
+              tc::cp_async8(d, sp[j] + g0, ok16[j] ? 8u : 0u);
+              tc::cp_async8(d + 16, bp[j] + g0, ok16[j] ? 8u : 0u);
             } else {
-              tc::cp_async4(d, sp[j] + kb, ok16[j] ? 4u : 0u);
-              tc::cp_async4(d + 16, bp[j] + kb, ok16[j] ? 4u : 0u);
+              tc::cp_async4(d, sp[j] + g0, ok16[j] ? 4u : 0u);
+              tc::cp_async4(d + 16, bp[j] + g0, ok16[j] ? 4u : 0u);
             }
           }
         }
@@ -730,8 +742,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
     constexpr int CPT = PAIR ? (RW::CHUNKS > 1 ? RW::CHUNKS / 2 : 1) : RW::CHUNKS;
     const int c_lo = PAIR ? (t >> 7) * CPT : 0;   // first raw chunk of this thread
     const bool active = c_lo < RW::CHUNKS;
-    const int W = a.sb_w, wl = W == 8 ? 3 : W == 4 ? 2 : 1;
+    const int W = a.sb_w, wl = win_kb_log2(W, a.G);
     uint4 swin = make_uint4(0u, 0u, 0u, 0u), bwin = swin;  // scale/bias window (bf16 pairs)
+    // scale and bias bits of group j of the window
+    auto pick = [&](int j, uint32_t& sbits, uint32_t& bbits) {
+      const uint32_t sw2 = (j & 4) ? ((j & 2) ? swin.w : swin.z) : ((j & 2) ? swin.y : swin.x);
+      const uint32_t bw2 = (j & 4) ? ((j & 2) ? bwin.w : bwin.z) : ((j & 2) ? bwin.y : bwin.x);
+      sbits = (j & 1) ? (sw2 >> 16) : (sw2 & 0xFFFFu);
+      bbits = (j & 1) ? (bw2 >> 16) : (bw2 & 0xFFFFu);
+    };
+    constexpr int VPC = 128 / BITS;  // values of one 16-byte code chunk
     uint32_t it = 0;
     for (int item = unit0; item < n_items; item += n_units) {
       for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -741,7 +761,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         if (!tc::mbar_wait(&b_empty[s2], ph2 ^ 1u, status)) goto done;
         const uint32_t rst = sbase + SM::RAW_OFF + sr * SM::RAW_STAGE;
         const uint32_t bst = sbase + SM::B_OFF + s2 * SM::B_STAGE;
-        if ((kb & (W - 1)) == 0) {
+        const int kbw = kb & ((1 << wl) - 1);  // k-block within the window
+        if (kbw == 0) {
           // this row's window of W scales and W biases, kept in registers
           const uint32_t sbw =
               sbase + SM::SB_OFF + ((it >> wl) % SM::NWB) * SM::SB_WIN + r * 32;
@@ -757,11 +778,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
             bwin = make_uint4(lds32(sbw + 16), 0u, 0u, 0u);
           }
         }
-        const int j = kb & (W - 1);
-        const uint32_t sw2 = (j & 4) ? ((j & 2) ? swin.w : swin.z) : ((j & 2) ? swin.y : swin.x);
-        const uint32_t bw2 = (j & 4) ? ((j & 2) ? bwin.w : bwin.z) : ((j & 2) ? bwin.y : bwin.x);
-        const uint32_t sbits = (j & 1) ? (sw2 >> 16) : (sw2 & 0xFFFFu);
-        const uint32_t bbits = (j & 1) ? (bw2 >> 16) : (bw2 & 0xFFFFu);
+        // group of chunk c: value kbw * 64 + c * VPC of the window, over G
+        uint32_t sbits, bbits;
+        pick(a.G == 64 ? kbw : a.G == 128 ? kbw >> 1 : 2 * kbw + (c_lo * VPC >= 32), sbits, bbits);
         uint4 raw[CPT];
 #pragma unroll
         for (int c = 0; c < CPT; ++c)
@@ -769,11 +788,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         tc::mbar_arrive(&raw_empty[sr]);
         if (active) {
           // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
+          // G = 32 (8- and 4-bit only): chunks of one thread may fall in
+          // both groups of the k-block
+          const bool per_chunk = a.G == 32 && CPT > 1;
           if (EPI == EPI_SPLIT) {
-            const float sf = bf16_bits_to_float((uint16_t)sbits);
-            const float bf = bf16_bits_to_float((uint16_t)bbits);
 #pragma unroll
             for (int c = 0; c < CPT; ++c) {
+              uint32_t sb = sbits, bb = bbits;
+              if (per_chunk) pick(2 * kbw + ((c_lo + c) * VPC >= 32), sb, bb);
+              const float sf = bf16_bits_to_float((uint16_t)sb);
+              const float bf = bf16_bits_to_float((uint16_t)bb);
               if (rg < 128)
                 dequant_chunk_split<BITS, false>(raw[c], sf, bf, bst, r, (c_lo + c) * (16 / BITS));
               else
@@ -783,8 +807,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
             __half2 s2h, b2h;
             group_h2<BITS>(sbits, bbits, s2h, b2h, status);
 #pragma unroll
-            for (int c = 0; c < CPT; ++c)
+            for (int c = 0; c < CPT; ++c) {
+              if (per_chunk && (c_lo + c) * VPC >= 32 && c_lo * VPC < 32) {
+                uint32_t sb, bb;
+                pick(2 * kbw + 1, sb, bb);
+                group_h2<BITS>(sb, bb, s2h, b2h, status);
+              }
               dequant_chunk<BITS>(raw[c], s2h, b2h, bst, r, (c_lo + c) * (16 / BITS));
+            }
           }
         }
         tc::fence_proxy_async_smem();

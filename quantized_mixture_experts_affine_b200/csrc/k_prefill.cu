@@ -603,18 +603,32 @@ bool code_tensor_map(CUtensorMap* m, const moeq_qtensor& t, int n_mat) {
 }
 
 // Groups per scale/bias window copy of a gather-QMM launch over tensors ts
-// (reduction length K): the largest of 8, 4, 2 that divides K/64 and keeps
-// every matrix's scale and bias rows aligned to the copy size.
+// (reduction length K, one group size G for all of them): the largest of 8,
+// 4, 2 that divides K/G, keeps every matrix's scale and bias rows aligned to
+// the copy size and spans at least two k-blocks (W * G / 64 >= 2).  0 when
+// none does or the tensors' group sizes differ.
 int sb_window(const moeq_qtensor* const* ts, int n, int K) {
-  const int groups = K / 64;
-  for (int W = 8; W > 2; W >>= 1) {
+  const int G = ts[0]->group_size;
+  for (int i = 1; i < n; ++i)
+    if (ts[i]->group_size != G) return 0;
+  if (G != 32 && G != 64 && G != 128) return 0;
+  const int groups = K / G;
+  for (int W = 8; W >= 2; W >>= 1) {
+    if (gq::win_kb_log2(W, G) < 1) continue;
     bool ok = groups % W == 0;
     for (int i = 0; i < n && ok; ++i)
       ok = ((uintptr_t)ts[i]->scales % (2 * W)) == 0 && ((uintptr_t)ts[i]->biases % (2 * W)) == 0 &&
            (ts[i]->expert_stride_sb * 2) % (2 * W) == 0;
-    if (ok) return W;
+    if (ok || (W == 2 && groups % 2 == 0)) return W;
   }
-  return 2;
+  return 0;
+}
+
+// Scale/bias window and group size of a launch over tensors ts.
+bool set_window(gq::Args& a, const moeq_qtensor* const* ts, int n, int K) {
+  a.sb_w = sb_window(ts, n, K);
+  a.G = ts[0]->group_size;
+  return a.sb_w != 0;
 }
 
 moeq_status check_prefill(const moeq_layer* L) {
@@ -622,13 +636,30 @@ moeq_status check_prefill(const moeq_layer* L) {
                                &L->sh_gate, &L->sh_up, &L->sh_down, &L->sh_expert_gate};
   const int n = L->has_shared ? 8 : 4;
   for (int i = 0; i < n; ++i) {
-    if (ts[i]->group_size != 64) return MOEQ_ERR_UNSUPPORTED;
+    const int G = ts[i]->group_size;
+    if (G != 32 && G != 64 && G != 128) return MOEQ_ERR_UNSUPPORTED;
+    if (G == 32 && ts[i]->bits == 2) return MOEQ_ERR_UNSUPPORTED;
     if (((uintptr_t)ts[i]->scales & 3) || ((uintptr_t)ts[i]->biases & 3)) return MOEQ_ERR_ALIGNMENT;
     if (ts[i]->in_dim % 128) return MOEQ_ERR_UNSUPPORTED;
     if (ts[i]->expert_stride_sb % 2) return MOEQ_ERR_ALIGNMENT;
   }
   if (L->inter % 128) return MOEQ_ERR_UNSUPPORTED;
   if (L->has_shared && L->sh_gate.out_dim % 128) return MOEQ_ERR_UNSUPPORTED;
+  // every launch's tensors share a group size and admit a scale/bias window
+  const moeq_qtensor* gu[2] = {&L->gate, &L->up};
+  const moeq_qtensor* dn[1] = {&L->down};
+  const moeq_qtensor* rt[2] = {&L->router, &L->sh_expert_gate};
+  if (!sb_window(gu, 2, L->hidden) || !sb_window(dn, 1, L->inter)) return MOEQ_ERR_UNSUPPORTED;
+  if (!sb_window(rt, 1, L->hidden)) return MOEQ_ERR_UNSUPPORTED;
+  if (L->has_shared) {
+    const moeq_qtensor* sgu[2] = {&L->sh_gate, &L->sh_up};
+    const moeq_qtensor* sdn[1] = {&L->sh_down};
+    const moeq_qtensor* sg[1] = {&L->sh_expert_gate};
+    if (!sb_window(sgu, 2, L->hidden) || !sb_window(sdn, 1, L->sh_gate.out_dim) ||
+        !sb_window(sg, 1, L->hidden))
+      return MOEQ_ERR_UNSUPPORTED;
+    if (sg_with_router(L) && !sb_window(rt, 2, L->hidden)) return MOEQ_ERR_UNSUPPORTED;
+  }
   return MOEQ_OK;
 }
 
@@ -729,7 +760,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     const int nt = (rs.n_valid + 127) / 128;
     gq::Args a = gemm_args(rs, nt, H, x16, H, logits, lay.ld_logits);
     const moeq_qtensor* ts[2] = {&L->router, &L->sh_expert_gate};
-    a.sb_w = sb_window(ts, sgr ? 2 : 1, H);
+    if (!set_window(a, ts, sgr ? 2 : 1, H)) return MOEQ_ERR_UNSUPPORTED;
     const int items = mtiles * nt;
     PCK(launch_gqmm(L->router.bits, gq::EPI_SPLIT, pair, a, items, st));
   }
@@ -737,7 +768,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     const gq::Seg gs = seg_single(L->sh_expert_gate, nullptr, M, gq::A_TOKENS);
     gq::Args a = gemm_args(gs, 1, H, x16, H, logits + E, lay.ld_logits);
     const moeq_qtensor* ts[1] = {&L->sh_expert_gate};
-    a.sb_w = sb_window(ts, 1, H);
+    if (!set_window(a, ts, 1, H)) return MOEQ_ERR_UNSUPPORTED;
     PCK(launch_gqmm(L->sh_expert_gate.bits, gq::EPI_SPLIT, pair, a, mtiles, st));
   }
 
@@ -815,7 +846,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.status = status;
     a.tma_b = code_tensor_map(&a.tmB[0], L->gate, E) && code_tensor_map(&a.tmB[1], L->up, E);
     const moeq_qtensor* ts[2] = {&L->gate, &L->up};
-    a.sb_w = sb_window(ts, 2, H);
+    if (!set_window(a, ts, 2, H)) return MOEQ_ERR_UNSUPPORTED;
     const int64_t items = max_mtiles * a.n_tiles_n;
     if (profile_mark(true, st) != cudaSuccess) return MOEQ_ERR_CUDA;
     PCK(launch_gqmm(L->gate.bits, gq::EPI_SWIGLU, pair, a, items, st));
@@ -828,7 +859,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     gq::Args a = gemm_args(gs, Is / 128, H, x16, H, h_sh, Is);
     a.tma_b = code_tensor_map(&a.tmB[0], L->sh_gate, 1) && code_tensor_map(&a.tmB[1], L->sh_up, 1);
     const moeq_qtensor* ts[2] = {&L->sh_gate, &L->sh_up};
-    a.sb_w = sb_window(ts, 2, H);
+    if (!set_window(a, ts, 2, H)) return MOEQ_ERR_UNSUPPORTED;
     const int items = mtiles * (Is / 128);
     PCK(launch_gqmm(L->sh_gate.bits, gq::EPI_SWIGLU, pair, a, items, st));
   }
@@ -852,7 +883,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.status = status;
     a.tma_b = code_tensor_map(&a.tmB[0], L->down, E);
     const moeq_qtensor* ts[1] = {&L->down};
-    a.sb_w = sb_window(ts, 1, I);
+    if (!set_window(a, ts, 1, I)) return MOEQ_ERR_UNSUPPORTED;
     const int64_t items = max_mtiles * a.n_tiles_n;
     PCK(launch_gqmm(L->down.bits, gq::EPI_STORE, pair, a, items, st));
   }
@@ -864,7 +895,7 @@ moeq_status prefill_forward(const moeq_layer* L, const uint16_t* x, int M, const
     a.out_f16 = 1;
     a.tma_b = code_tensor_map(&a.tmB[0], L->sh_down, 1);
     const moeq_qtensor* ts[1] = {&L->sh_down};
-    a.sb_w = sb_window(ts, 1, Is);
+    if (!set_window(a, ts, 1, Is)) return MOEQ_ERR_UNSUPPORTED;
     const int items = mtiles * ((H + gq::BN - 1) / gq::BN);
     PCK(launch_gqmm(L->sh_down.bits, gq::EPI_STORE, pair, a, items, st));
   }
