@@ -89,7 +89,7 @@ def config_of(workload, world, copies):
 # not captured (null).
 TRAFFIC = {
     "decode_397b_m1": 35535872,
-    "prefill_8bit_m16068": 971213056 + 189862656,
+    "prefill_8bit_m16068": 959738624 + 185099264,
 }
 
 

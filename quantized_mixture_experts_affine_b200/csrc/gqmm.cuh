@@ -318,8 +318,11 @@ __device__ __forceinline__ void dequant_chunk_split(uint4 raw, float s, float b,
            o[4 * k + 3]);
 }
 
-template <int BITS, int EPI, bool PAIR>
+// GS: the group size when fixed at compile time (64, the common case, with
+// no group arithmetic left at run time), or 0 to take a.G (32 or 128).
+template <int BITS, int EPI, bool PAIR, int GS>
 __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Args a) {
+  const int G = GS ? GS : a.G;
   using SM = Smem<BITS, PAIR>;
   using RW = Raw<BITS>;
   constexpr int S1 = SM::S1, SR = SM::SR, S2 = SM::S2, BR = SM::BR;
@@ -478,8 +481,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
   } else if (warp == 2) {
     // ------------------------------------------------------------ B loader
     // this CTA's BR weight rows of the tile: rows rank*BR + (lane + 32 j)
-    const int groups = a.K / a.G;
-    const int W = a.sb_w, wl = win_kb_log2(W, a.G);
+    const int groups = a.K / G;
+    const int W = a.sb_w, wl = win_kb_log2(W, G);
     const int64_t wrow = (int64_t)a.K * BITS / 32;  // words per weight row
     constexpr int JR = BR / 32;
     uint32_t it = 0;
@@ -516,7 +519,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         // first group is group kb * 64 / G of the row
         const bool new_win = (kb & ((1 << wl) - 1)) == 0;
         const uint32_t sbw = sbase + SM::SB_OFF + ((it >> wl) % SM::NWB) * SM::SB_WIN;
-        const int g0 = a.G == 64 ? kb : a.G == 128 ? kb >> 1 : kb << 1;
+        const int g0 = G == 64 ? kb : G == 128 ? kb >> 1 : kb << 1;
         if (a.tma_b) {
           if (lane == 0) {
             tc::mbar_expect_tx(&raw_full[s], (uint32_t)SM::RAW_STAGE);
@@ -742,7 +745,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
     constexpr int CPT = PAIR ? (RW::CHUNKS > 1 ? RW::CHUNKS / 2 : 1) : RW::CHUNKS;
     const int c_lo = PAIR ? (t >> 7) * CPT : 0;   // first raw chunk of this thread
     const bool active = c_lo < RW::CHUNKS;
-    const int W = a.sb_w, wl = win_kb_log2(W, a.G);
+    const int W = a.sb_w, wl = win_kb_log2(W, G);
     uint4 swin = make_uint4(0u, 0u, 0u, 0u), bwin = swin;  // scale/bias window (bf16 pairs)
     // scale and bias bits of group j of the window
     auto pick = [&](int j, uint32_t& sbits, uint32_t& bbits) {
@@ -780,7 +783,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         }
         // group of chunk c: value kbw * 64 + c * VPC of the window, over G
         uint32_t sbits, bbits;
-        pick(a.G == 64 ? kbw : a.G == 128 ? kbw >> 1 : 2 * kbw + (c_lo * VPC >= 32), sbits, bbits);
+        pick(G == 64 ? kbw : G == 128 ? kbw >> 1 : 2 * kbw + (c_lo * VPC >= 32), sbits, bbits);
         uint4 raw[CPT];
 #pragma unroll
         for (int c = 0; c < CPT; ++c)
@@ -790,7 +793,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           // packed chunk c holds values [c*128/BITS, (c+1)*128/BITS): fp16 chunk c*16/BITS
           // G = 32 (8- and 4-bit only): chunks of one thread may fall in
           // both groups of the k-block
-          const bool per_chunk = a.G == 32 && CPT > 1;
+          const bool per_chunk = G == 32 && CPT > 1;
           if (EPI == EPI_SPLIT) {
 #pragma unroll
             for (int c = 0; c < CPT; ++c) {

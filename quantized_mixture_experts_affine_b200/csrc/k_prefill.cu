@@ -403,10 +403,10 @@ __global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx,
 // Launch over `units` work items: one CTA per item up to the co-resident
 // count, or (PAIR) one cluster of two CTAs per item up to the co-resident
 // cluster count.
-template <int BITS, int EPI, bool PAIR>
+template <int BITS, int EPI, bool PAIR, int GS>
 cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
   constexpr int smem = gq::Smem<BITS, PAIR>::ALLOC;
-  auto kern = gq::k_gqmm<BITS, EPI, PAIR>;
+  auto kern = gq::k_gqmm<BITS, EPI, PAIR, GS>;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
@@ -443,21 +443,29 @@ cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+// Group size 64 runs the kernel compiled for it; 32 and 128 the one that
+// reads it from the arguments.
+template <int BITS, int EPI, bool PAIR>
+cudaError_t launch_gqmm_g(const gq::Args& a, int units, cudaStream_t st) {
+  if (a.G == 64) return launch_gqmm_t<BITS, EPI, PAIR, 64>(a, units, st);
+  return launch_gqmm_t<BITS, EPI, PAIR, 0>(a, units, st);
+}
+
 template <bool PAIR>
 cudaError_t launch_gqmm_p(int bits, int epi, const gq::Args& a, int units, cudaStream_t st) {
   if (epi == gq::EPI_SPLIT) {
-    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SPLIT, PAIR>(a, units, st);
-    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SPLIT, PAIR>(a, units, st);
-    return launch_gqmm_t<2, gq::EPI_SPLIT, PAIR>(a, units, st);
+    if (bits == 8) return launch_gqmm_g<8, gq::EPI_SPLIT, PAIR>(a, units, st);
+    if (bits == 4) return launch_gqmm_g<4, gq::EPI_SPLIT, PAIR>(a, units, st);
+    return launch_gqmm_g<2, gq::EPI_SPLIT, PAIR>(a, units, st);
   }
   if (epi == gq::EPI_SWIGLU) {
-    if (bits == 8) return launch_gqmm_t<8, gq::EPI_SWIGLU, PAIR>(a, units, st);
-    if (bits == 4) return launch_gqmm_t<4, gq::EPI_SWIGLU, PAIR>(a, units, st);
-    return launch_gqmm_t<2, gq::EPI_SWIGLU, PAIR>(a, units, st);
+    if (bits == 8) return launch_gqmm_g<8, gq::EPI_SWIGLU, PAIR>(a, units, st);
+    if (bits == 4) return launch_gqmm_g<4, gq::EPI_SWIGLU, PAIR>(a, units, st);
+    return launch_gqmm_g<2, gq::EPI_SWIGLU, PAIR>(a, units, st);
   }
-  if (bits == 8) return launch_gqmm_t<8, gq::EPI_STORE, PAIR>(a, units, st);
-  if (bits == 4) return launch_gqmm_t<4, gq::EPI_STORE, PAIR>(a, units, st);
-  return launch_gqmm_t<2, gq::EPI_STORE, PAIR>(a, units, st);
+  if (bits == 8) return launch_gqmm_g<8, gq::EPI_STORE, PAIR>(a, units, st);
+  if (bits == 4) return launch_gqmm_g<4, gq::EPI_STORE, PAIR>(a, units, st);
+  return launch_gqmm_g<2, gq::EPI_STORE, PAIR>(a, units, st);
 }
 
 // PAIR launches need the A operand as tensor-map tiles (a.tma_a).
