@@ -726,16 +726,21 @@ def sweep_row(row, name, M, kind, copies, seed=0):
     if kind == "qmv":
         out["roofline"] = {"bound": "hbm", "bytes": nbytes,
                            "frac": nbytes / (ms_call / 1e3) / 1e9 / peak_hbm}
-    elif M * cfg.K <= 64 * cfg.K and M <= 64:
+    else:
+        # both rooflines: the weight bytes the call must stream (router
+        # unless the routing is given, the distinct routed experts, the
+        # shared expert) and the layer's FLOPs; the bound is the larger
         distinct = len(set(idx.cpu().numpy().ravel().tolist()))
         nbytes = (0 if kind == "zipf" else cfg.router_bytes()) + distinct * cfg.expert_bytes() \
             + cfg.shared_bytes()
-        out["roofline"] = {"bound": "hbm", "bytes": nbytes, "distinct_experts": distinct,
-                           "frac": nbytes / (ms_call / 1e3) / 1e9 / peak_hbm}
-    else:
         flop = M * cfg.flops_per_token() - (2 * M * cfg.E * cfg.H if kind == "zipf" else 0)
-        out["roofline"] = {"bound": "tensor", "flop": flop,
-                           "frac": flop / (ms_call / 1e3) / 1e12 / peak_bf16}
+        hbm = nbytes / (ms_call / 1e3) / 1e9 / peak_hbm
+        ten = flop / (ms_call / 1e3) / 1e12 / peak_bf16
+        out["roofline"] = {"bound": "hbm" if hbm >= ten else "tensor", "bytes": nbytes,
+                           "distinct_experts": distinct, "flop": flop, "hbm_frac": hbm,
+                           "tensor_frac": ten, "frac": max(hbm, ten)}
+    out["path"] = ("decode" if kind != "qmv" and M <= 64 and M * cfg.K <= 96 else
+                   "prefill" if kind != "qmv" else "qmv")
     out["roofline"]["peak_kind"] = peak_kind
     del g
     torch.cuda.empty_cache()

@@ -57,7 +57,7 @@ typedef enum {
 } moeq_status;
 
 typedef enum {
-  MOEQ_MODE_AUTO = 0,    /* decode for M <= 64, prefill otherwise */
+  MOEQ_MODE_AUTO = 0,    /* decode while M*K <= 96 (and M <= 64), prefill beyond */
   MOEQ_MODE_DECODE = 1,  /* HBM-bound split-K quantised matvec path */
   MOEQ_MODE_PREFILL = 2  /* sort-by-expert gather-QMM on tcgen05 tensor cores */
 } moeq_mode;
@@ -164,8 +164,8 @@ moeq_status moeq_route_topk(const float* logits, int32_t M, int32_t E, int32_t K
  * prefill path computes every output row from its own token with the same
  * kernels for any M, so splitting the tokens into chunks gives
  * bit-identical results.  Only PREFILL mode has that property: AUTO picks
- * the path per call from that call's M (decode for M <= 64), so a chunked
- * sequence run in AUTO mode whose last chunk has at most 64 tokens gets
+ * the path per call from that call's M (decode while M*K <= 96), so a
+ * chunked sequence run in AUTO mode whose last chunk is that small gets
  * that chunk from the decode path, whose arithmetic differs (the results
  * agree within the layer tolerance, not bit for bit).  Pass PREFILL for
  * every chunk to keep chunked and one-shot results bit-identical.

@@ -222,26 +222,27 @@ def test_prefill_mixed_2bit_zipf_4096():
 
 
 def test_auto_mode_picks_the_path_per_call():
-    """AUTO takes the decode path for a call of at most 64 tokens and the
-    prefill path above that, from the call's own M: it is bit for bit one or
-    the other.  So only PREFILL mode makes chunked calls bit-identical to one
-    call; an AUTO chunk of <= 64 tokens agrees with the prefill rows within
-    the layer tolerance only."""
+    """AUTO takes the decode path for a call of at most 96 (token, expert)
+    pairs and the prefill path above that, from the call's own M (K = 8
+    here: 12 tokens decode, 13 prefill): it is bit for bit one or the other.
+    So only PREFILL mode makes chunked calls bit-identical to one call; an
+    AUTO chunk on the decode side agrees with the prefill rows within the
+    layer tolerance only."""
     L = layer_of("prefill_8bit")
     cfg = L.cfg
-    xb, x = x_tokens(cfg, 129, copy=77)
-    for M, path in ((64, moeq.MODE_DECODE), (65, P)):
+    xb, x = x_tokens(cfg, 25, copy=77)
+    for M, path in ((12, moeq.MODE_DECODE), (13, P)):
         ya, ia, wa = layer_forward(L, x[:M], mode=moeq.MODE_AUTO)
         yb, ib, wb = layer_forward(L, x[:M], mode=path)
         torch.cuda.synchronize()
         assert torch.equal(ya.view(torch.int32), yb.view(torch.int32)), M
         assert torch.equal(ia, ib) and torch.equal(wa.view(torch.int32), wb.view(torch.int32))
-    # 65 + 64 tokens in AUTO mode against one PREFILL call of 129
+    # 13 + 12 tokens in AUTO mode against one PREFILL call of 25
     y1, _, _ = forward(L, x)
-    ya, _, _ = layer_forward(L, x[:65], mode=moeq.MODE_AUTO)
-    yb, ib, wb = layer_forward(L, x[65:], mode=moeq.MODE_AUTO)
+    ya, _, _ = layer_forward(L, x[:13], mode=moeq.MODE_AUTO)
+    yb, ib, wb = layer_forward(L, x[13:], mode=moeq.MODE_AUTO)
     torch.cuda.synchronize()
-    assert torch.equal(ya.view(torch.int32), y1[:65].view(torch.int32))
-    got, ref = yb.cpu().numpy(), y1[65:].cpu().numpy()
+    assert torch.equal(ya.view(torch.int32), y1[:13].view(torch.int32))
+    got, ref = yb.cpu().numpy(), y1[13:].cpu().numpy()
     assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
-    check_layer_outputs(cfg, SEED, 0, xb[65:], got, ib.cpu().numpy(), wb.cpu().numpy())
+    check_layer_outputs(cfg, SEED, 0, xb[13:], got, ib.cpu().numpy(), wb.cpu().numpy())
