@@ -229,6 +229,19 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def sustained_bf16_peak():
+    """The bf16 dense peak for work timed inside a long run (the power cap
+    holds the clocks below their burst level): the measured sustained figure,
+    else the recipe's fallback of 1.4 PFLOP/s."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops_sustained" in d:
+            return d["bf16_tflops_sustained"], "measured sustained"
+    return 1400.0, "fallback sustained"
+
+
 # ------------------------------------------------------------------ CPU oracle sample
 class OracleSample:
     """The oracle as it stands, on a bounded sample of the workload: n_tokens
@@ -308,6 +321,11 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ prefill measurement
+def layer_flop_of(workload):
+    cfg_name, M = WORKLOADS[workload]
+    return M * shape(cfg_name).flops_per_token()
+
+
 def timed_replays(fn, reps, st, world, local):
     """Device time (max over ranks, ms) of reps calls of fn on stream st,
     bracketed by a barrier and a synchronize, with the SM clocks sampled."""
@@ -370,8 +388,12 @@ def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True, min_ms=
     # the same graph replayed for at least min_ms (a long clock record)
     reps = max(1, math.ceil(min_ms / max(ms * steps, 1e-3)))
     ms_long, clk_long = timed_replays(lambda: g.replay(), reps, st, world, local)
+    sus_peak, sus_kind = sustained_bf16_peak()
     sustained = {"steps": reps * steps, "timed_ms": ms_long, "ms_per_step": ms_long / (reps * steps),
-                 "value": M * world / (ms_long / (reps * steps) / 1e3), "clocks": clk_long.summary()}
+                 "value": M * world / (ms_long / (reps * steps) / 1e3), "clocks": clk_long.summary(),
+                 "layer_tflops": layer_flop_of(workload) / (ms_long / (reps * steps) / 1e3) / 1e12,
+                 "peak_tflops": sus_peak, "peak_kind": sus_kind}
+    sustained["layer_frac"] = sustained["layer_tflops"] / sus_peak
     # gate/up gather-QMM per launch
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]

@@ -616,6 +616,19 @@ __device__ __forceinline__ void prefetch_units(const FzSmem& S, int from, int to
   }
 }
 
+// The routing selection over the logit buffer into the CTA's routing slots
+// (out of line: the early warm-up run and the real selection execute the
+// same code).
+__device__ __noinline__ void route_select(const FusedArgs& a, const FzSmem& S) {
+  const float* lg = a.logits;
+  if (a.E <= 32) route_token_regs<1>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
+  else if (a.E <= 64) route_token_regs<2>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
+  else if (a.E <= 128) route_token_regs<4>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
+  else if (a.E <= 256) route_token_regs<8>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
+  else if (a.E <= 512) route_token_regs<16>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
+  else route_token_regs<32>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
+}
+
 // ------------------------------------------------------------------ compute side
 // Groups of the unit's rows this warp takes.
 __device__ __forceinline__ void warp_groups(const FzKind& g, int warp, int& gb, int& ge) {
@@ -746,18 +759,17 @@ __global__ void __maxnreg__(96) k_fused_decode(const __grid_constant__ FusedArgs
     const uint64_t tag = next_tag(*a.gen);
     for (; seq < n_pre && seq - FZ_NS < n1 && !ld_vol(dead); ++seq)
       if (!issue_unit(S, maps, seq)) break;
+    // While the first flags are outstanding, run the top-K once on whatever
+    // the logit buffer holds (results discarded: the real routing below
+    // overwrites them), so that its code is in the instruction cache when
+    // the routing is on the critical path.
+    if (a.route_from_router && phase1) route_select(a, S);
     // routing: every CTA's logits, shared gate logit and shared hidden values are out
     bool ok = !ld_vol(dead);
     if (ok && phase1) ok = wait_all_flags(a.flag1, P, tag, a.status, dead);
     if (ok) {
       if (a.route_from_router) {
-        const float* lg = a.logits;
-        if (a.E <= 32) route_token_regs<1>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
-        else if (a.E <= 64) route_token_regs<2>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
-        else if (a.E <= 128) route_token_regs<4>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
-        else if (a.E <= 256) route_token_regs<8>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
-        else if (a.E <= 512) route_token_regs<16>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
-        else route_token_regs<32>(lg, a.E, a.K, a.renorm, a.router_scale, S.idx, S.w);
+        route_select(a, S);
       } else if (lane < a.K) {
         int e = a.idx_in[lane];
         if (e < 0 || e >= a.E) {

@@ -266,21 +266,32 @@ __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ Offset
   const int E = a.E, tid = threadIdx.x;
   const int lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
   // 1. per expert (one warp at a time): exclusive scan of its block counts
+  // (the counts of 8 x 32 blocks are loaded before any is scanned, so the
+  // warp waits for one memory round trip per 256 blocks, not per 32)
   for (int e = wid; e < E; e += nw) {
     const int32_t* hrow = a.blockhist + (int64_t)e * a.nb;
     int32_t* orow = a.blockoff + (int64_t)e * a.nb;
     int carry = 0;
-    for (int b0 = 0; b0 < a.nb; b0 += 32) {
-      const int b = b0 + lane;
-      const int v = b < a.nb ? hrow[b] : 0;
-      int inc = v;
+    for (int b00 = 0; b00 < a.nb; b00 += 32 * 8) {
+      int vals[8];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += u;
+      for (int j = 0; j < 8; ++j) {
+        const int b = b00 + 32 * j + lane;
+        vals[j] = b < a.nb ? hrow[b] : 0;
       }
-      if (b < a.nb) orow[b] = carry + inc - v;
-      carry += __shfl_sync(0xffffffffu, inc, 31);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int b = b00 + 32 * j + lane;
+        const int v = vals[j];
+        int inc = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += u;
+        }
+        if (b < a.nb) orow[b] = carry + inc - v;
+        carry += __shfl_sync(0xffffffffu, inc, 31);
+      }
     }
     if (lane == 0) count_s[e] = carry;
   }
@@ -383,10 +394,21 @@ __global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx,
   __syncwarp();
   const int64_t p0 = (int64_t)blockIdx.x * kSortChunk;
   const int64_t p1 = min(n, p0 + kSortChunk);
-  for (int64_t base = p0; base < p1; base += 32) {
+  // the block's expert indices, loaded before the ordered pass (one memory
+  // round trip instead of one per 32 pairs)
+  constexpr int R = kSortChunk / 32;
+  int ev[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t p = p0 + 32 * r + lane;
+    ev[r] = p < p1 ? checked_expert(idx, p, E, status) : -1 - lane;
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t base = p0 + 32 * r;
     const int64_t p = base + lane;
     const bool on = p < p1;
-    const int e = on ? checked_expert(idx, p, E, status) : -1 - lane;
+    const int e = ev[r];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (on) {
       const int rank = __popc(peers & ((1u << lane) - 1u));
