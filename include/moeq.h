@@ -62,17 +62,32 @@ typedef enum {
   MOEQ_MODE_PREFILL = 2  /* sort-by-expert gather-QMM on tcgen05 tensor cores */
 } moeq_mode;
 
+/* Code formats of a tensor. */
+typedef enum {
+  /* w = q * scale + bias per group, bf16 scale and bias ("danveloper/
+   * flash-moe" thread and "flash-moe-inference": the affine format) */
+  MOEQ_FMT_AFFINE = 0,
+  /* MX FP4 (the mlx issue page's mode="mxfp4", bits 4, group_size 32):
+   * each 4-bit code is an E2M1 value (bit 3 sign, bits 2..1 exponent, bit 0
+   * mantissa: 0, 0.5, 1, 1.5, 2, 3, 4, 6, signed) and each group of 32
+   * shares one E8M0 scale byte e, w = e2m1(q) * 2^(e - 127).  scales points
+   * at the uint8 exponents (same shape and strides as the affine scales,
+   * one byte per entry); biases is unused. */
+  MOEQ_FMT_MXFP4 = 1
+} moeq_format;
+
 /* One packed tensor or bank of tensors (device memory). */
 typedef struct {
   const uint32_t* w;        /* codes, [E][out_dim][in_dim*bits/32] */
-  const uint16_t* scales;   /* bf16 bits, [E][out_dim][in_dim/group_size] */
-  const uint16_t* biases;   /* bf16 bits, same shape as scales */
+  const uint16_t* scales;   /* bf16 bits, [E][out_dim][in_dim/group_size] (MXFP4: uint8) */
+  const uint16_t* biases;   /* bf16 bits, same shape as scales (MXFP4: unused) */
   int32_t out_dim;
   int32_t in_dim;
-  int32_t bits;             /* 2, 4 or 8 */
-  int32_t group_size;       /* values per group along in_dim: 64 (or 32, 128) */
+  int32_t bits;             /* 2, 4 or 8 (MXFP4: 4) */
+  int32_t group_size;       /* values per group along in_dim: 64 (or 32, 128; MXFP4: 32) */
   int64_t expert_stride_w;  /* words from one expert's matrix to the next (0: single matrix) */
   int64_t expert_stride_sb; /* scale/bias entries from one expert to the next */
+  int32_t format;           /* moeq_format (0, the affine format, when zero-initialised) */
 } moeq_qtensor;
 
 /*

@@ -61,6 +61,7 @@ typedef struct {
   int32_t out, in, bits, G;
   int64_t stride_w;       /* words between consecutive matrices */
   int64_t stride_sb;      /* scale/bias entries between matrices */
+  int32_t format;         /* 0 affine; 1 MX FP4 (s: uint8 E8M0 exponents, no b) */
 } orc_tensor;
 
 typedef struct {
@@ -114,6 +115,33 @@ static void orc_group(const orc_tensor* t, int mat, int64_t r, int64_t c, double
   *b = orc_bf16(t->b[i]);
 }
 
+/*
+ * MX FP4 ([MLX-3856] mode="mxfp4"; element and scale encodings of the OCP
+ * Microscaling Formats specification v1.0): a 4-bit E2M1 code q has sign
+ * bit 3, exponent bits 2..1 and mantissa bit 0; exponent 0 is subnormal
+ * (value m * 2^-1), exponents 1..3 give 2^(e-1) * (1 + m/2).  A group of
+ * 32 shares the E8M0 byte x: scale 2^(x - 127); x = 255 is NaN.
+ */
+static double orc_e2m1(uint32_t q) {
+  const int sign = (q >> 3) & 1, e = (q >> 1) & 3, m = q & 1;
+  const double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return sign ? -v : v;
+}
+
+static double orc_e8m0(const orc_tensor* t, int mat, int64_t r, int64_t c) {
+  const int64_t groups = t->in / t->G;
+  const uint8_t x = ((const uint8_t*)t->s)[(int64_t)mat * t->stride_sb + r * groups + c / t->G];
+  return x == 255 ? NAN : ldexp(1.0, (int)x - 127);
+}
+
+/* The weight of value c of row r in fp64 (exact for both formats). */
+static double orc_weight(const orc_tensor* t, int mat, int64_t r, int64_t c) {
+  if (t->format == 1) return orc_e2m1(orc_code(t, mat, r, c)) * orc_e8m0(t, mat, r, c);
+  double s, b;
+  orc_group(t, mat, r, c, &s, &b);
+  return (double)orc_code(t, mat, r, c) * s + b;
+}
+
 /* Unpacked codes, one byte per value, [out][in]. */
 ORC_API void oracle_unpack(const orc_tensor* t, int mat, uint8_t* q) {
   for (int64_t r = 0; r < t->out; ++r)
@@ -127,6 +155,12 @@ ORC_API void oracle_unpack(const orc_tensor* t, int mat, uint8_t* q) {
  * bit for bit.
  */
 ORC_API void oracle_dequant_f32(const orc_tensor* t, int mat, float* wout) {
+  if (t->format == 1) {
+    /* MX FP4: e2m1 * 2^(x-127) is exact in fp64; one rounding to fp32 */
+    for (int64_t r = 0; r < t->out; ++r)
+      for (int64_t c = 0; c < t->in; ++c) wout[r * t->in + c] = (float)orc_weight(t, mat, r, c);
+    return;
+  }
   for (int64_t r = 0; r < t->out; ++r)
     for (int64_t c = 0; c < t->in; ++c) {
       const int64_t groups = t->in / t->G;
@@ -145,13 +179,10 @@ static void orc_matvec(const orc_tensor* t, int mat, const double* x, double* y)
   for (int64_t r = 0; r < t->out; ++r) {
     double acc = 0.0;
     for (int g = 0; g < groups; ++g) {
-      double s, b;
-      orc_group(t, mat, r, (int64_t)g * t->G, &s, &b);
       double part = 0.0;
       for (int k = 0; k < t->G; ++k) {
         const int64_t c = (int64_t)g * t->G + k;
-        const double w = (double)orc_code(t, mat, r, c) * s + b;
-        part += w * x[c];
+        part += orc_weight(t, mat, r, c) * x[c];
       }
       acc += part;
     }

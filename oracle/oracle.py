@@ -35,7 +35,7 @@ def build(force: bool = False) -> str:
 class _Tensor(C.Structure):
     _fields_ = [("w", C.c_void_p), ("s", C.c_void_p), ("b", C.c_void_p),
                 ("out", C.c_int32), ("inn", C.c_int32), ("bits", C.c_int32), ("G", C.c_int32),
-                ("stride_w", C.c_int64), ("stride_sb", C.c_int64)]
+                ("stride_w", C.c_int64), ("stride_sb", C.c_int64), ("format", C.c_int32)]
 
 
 class _Layer(C.Structure):
@@ -58,20 +58,26 @@ class OracleTensor:
     in_dim: int
     bits: int
     group_size: int
+    fmt: int = 0   # 0 affine; 1 MX FP4 (s: uint8 E8M0 exponents, b unused)
 
     @classmethod
     def of(cls, t) -> "OracleTensor":
         """Accept any object with the same attribute names (e.g. a generated tensor)."""
-        return cls(t.w, t.s, t.b, t.out_dim, t.in_dim, t.bits, t.group_size)
+        return cls(t.w, t.s, t.b, t.out_dim, t.in_dim, t.bits, t.group_size,
+                   getattr(t, "fmt", 0))
 
     def _c(self) -> _Tensor:
-        for a, dt in ((self.w, np.uint32), (self.s, np.uint16), (self.b, np.uint16)):
+        sdt = np.uint16 if self.fmt == 0 else np.uint8
+        arrays = ((self.w, np.uint32), (self.s, sdt)) + (((self.b, np.uint16),) if self.fmt == 0
+                                                         else ())
+        for a, dt in arrays:
             assert a.dtype == dt and a.flags.c_contiguous, (a.dtype, dt)
         wpr = self.in_dim * self.bits // 32
         gpr = self.in_dim // self.group_size
-        return _Tensor(self.w.ctypes.data, self.s.ctypes.data, self.b.ctypes.data,
+        return _Tensor(self.w.ctypes.data, self.s.ctypes.data,
+                       self.b.ctypes.data if self.fmt == 0 else None,
                        self.out_dim, self.in_dim, self.bits, self.group_size,
-                       self.out_dim * wpr, self.out_dim * gpr)
+                       self.out_dim * wpr, self.out_dim * gpr, self.fmt)
 
     @property
     def n_mats(self) -> int:

@@ -59,15 +59,21 @@ cudaError_t profile_mark(bool start, cudaStream_t st) {
 static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 // Shape/format checks of one tensor.  n_mats: experts addressable (>= 1).
+static bool is_mx(const moeq_qtensor& t) { return t.format == MOEQ_FMT_MXFP4; }
+
 static moeq_status check_tensor(const moeq_qtensor* t, int64_t n_mats) {
-  if (!t || !t->w || !t->scales || !t->biases) return MOEQ_ERR_INVALID_ARG;
+  if (!t) return MOEQ_ERR_INVALID_ARG;
+  if (t->format != MOEQ_FMT_AFFINE && t->format != MOEQ_FMT_MXFP4) return MOEQ_ERR_UNSUPPORTED;
+  const bool mx = is_mx(*t);
+  if (!t->w || !t->scales || (!mx && !t->biases)) return MOEQ_ERR_INVALID_ARG;
   if (t->out_dim <= 0 || t->in_dim <= 0 || n_mats <= 0) return MOEQ_ERR_INVALID_ARG;
   if (t->bits != 2 && t->bits != 4 && t->bits != 8) return MOEQ_ERR_UNSUPPORTED;
   if (t->group_size != 32 && t->group_size != 64 && t->group_size != 128)
     return MOEQ_ERR_UNSUPPORTED;
+  if (mx && (t->bits != 4 || t->group_size != 32)) return MOEQ_ERR_UNSUPPORTED;
   const int vpc = 128 / t->bits;  // codes per 16-byte chunk
   if (t->in_dim % t->group_size || t->in_dim % vpc) return MOEQ_ERR_ALIGNMENT;
-  if (!aligned(t->w, 16) || !aligned(t->scales, 2) || !aligned(t->biases, 2))
+  if (!aligned(t->w, 16) || (!mx && (!aligned(t->scales, 2) || !aligned(t->biases, 2))))
     return MOEQ_ERR_ALIGNMENT;
   const int64_t words = (int64_t)t->out_dim * t->in_dim * t->bits / 32;
   const int64_t groups = (int64_t)t->out_dim * (t->in_dim / t->group_size);
@@ -99,8 +105,11 @@ static moeq_status check_layer(const moeq_layer* L) {
   if (L->gate.out_dim != I || L->gate.in_dim != H) return MOEQ_ERR_INVALID_ARG;
   if (L->up.out_dim != I || L->up.in_dim != H) return MOEQ_ERR_INVALID_ARG;
   if (L->down.out_dim != H || L->down.in_dim != I) return MOEQ_ERR_INVALID_ARG;
-  if (L->gate.bits != L->up.bits || L->gate.group_size != L->up.group_size)
+  if (L->gate.bits != L->up.bits || L->gate.group_size != L->up.group_size ||
+      L->gate.format != L->up.format)
     return MOEQ_ERR_UNSUPPORTED;
+  // MX FP4 is an expert-weight format: the router stays affine
+  if (is_mx(L->router)) return MOEQ_ERR_UNSUPPORTED;
   if (L->has_shared != 0 && L->has_shared != 1) return MOEQ_ERR_INVALID_ARG;
   if (L->has_shared) {
     if ((s = check_tensor(&L->sh_gate, 1)) != MOEQ_OK) return s;
@@ -113,8 +122,10 @@ static moeq_status check_layer(const moeq_layer* L) {
     if (L->sh_down.out_dim != H || L->sh_down.in_dim != Is) return MOEQ_ERR_INVALID_ARG;
     if (L->sh_expert_gate.out_dim != 1 || L->sh_expert_gate.in_dim != H)
       return MOEQ_ERR_INVALID_ARG;
-    if (L->sh_gate.bits != L->sh_up.bits || L->sh_gate.group_size != L->sh_up.group_size)
+    if (L->sh_gate.bits != L->sh_up.bits || L->sh_gate.group_size != L->sh_up.group_size ||
+        L->sh_gate.format != L->sh_up.format)
       return MOEQ_ERR_UNSUPPORTED;
+    if (is_mx(L->sh_expert_gate)) return MOEQ_ERR_UNSUPPORTED;
   }
   return MOEQ_OK;
 }
@@ -128,7 +139,13 @@ static moeq_status check_gemv_tensor(const moeq_qtensor& t, int nmat) {
   return MOEQ_OK;
 }
 
+static bool layer_has_mx(const moeq_layer* L) {
+  return is_mx(L->gate) || is_mx(L->down) ||
+         (L->has_shared && (is_mx(L->sh_gate) || is_mx(L->sh_down)));
+}
+
 static moeq_status check_decode_shapes(const moeq_layer* L) {
+  if (layer_has_mx(L)) return MOEQ_ERR_UNSUPPORTED;
   moeq_status s;
   if ((s = check_gemv_tensor(L->router, 1)) != MOEQ_OK) return s;
   if ((s = check_gemv_tensor(L->gate, 2)) != MOEQ_OK) return s;
@@ -591,6 +608,7 @@ MOEQ_API moeq_status moeq_qmv(const moeq_qtensor* t, int32_t expert, const uint1
   if (expert > 0 && (t->expert_stride_w <= 0 || t->expert_stride_sb <= 0))
     return MOEQ_ERR_INVALID_ARG;
   if ((s = check_gemv_tensor(*t, 1)) != MOEQ_OK) return s;
+  if (is_mx(*t)) return MOEQ_ERR_UNSUPPORTED;
   if (!aligned(x, 16) || ((int64_t)t->in_dim * 2) % 16 || !aligned(y, 4)) return MOEQ_ERR_ALIGNMENT;
   Seg seg = plain_seg(*t, expert, x, t->in_dim, y, t->out_dim, M, 0);
   LAUNCH(run_plain(*t, &seg, 1, 3, nullptr, (cudaStream_t)stream));

@@ -77,6 +77,31 @@ __device__ __forceinline__ float row_sum_256(float v, float* red) {
 }
 
 
+// ------------------------------------------------------------------ MX FP4 codes
+// An E2M1 code q (bit 3 sign, bits 2..1 exponent, bit 0 mantissa) times two
+// is an integer in [-12, 12]; shifted by 12 it is an unsigned code
+// q' = 2 e2m1(q) + 12 in [0, 24], so a group with E8M0 byte e is the affine
+// group w = q' * s + b with s = 2^(e - 128) and b = -12 s, exactly.  The
+// paths run MX FP4 through their affine arithmetic on q'.
+
+// q' of the four codes held one per byte in c (each 0..15): two 8-entry
+// byte tables (the positive and the negative values) indexed by the low 3
+// bits, chosen per byte by the sign bit.
+__device__ __forceinline__ uint32_t mx_q8(uint32_t c) {
+  const uint32_t m = c & 0x07070707u;
+  const uint32_t sel = __byte_perm(m | (m >> 4), 0u, 0x3320u) & 0xFFFFu;  // nibbles m0..m3
+  const uint32_t pos = __byte_perm(0x0F0E0D0Cu, 0x18141210u, sel);  // 12,13,14,15,16,18,20,24
+  const uint32_t neg = __byte_perm(0x090A0B0Cu, 0x00040608u, sel);  // 12,11,10,9,8,6,4,0
+  const uint32_t smask = ((c >> 3) & 0x01010101u) * 0xFFu;
+  return (pos & ~smask) | (neg & smask);
+}
+
+// 2^(e - 127) in fp32 (e = 0: 2^-127, subnormal; e = 255: NaN).
+__device__ __forceinline__ float mx_scale(uint32_t e) {
+  return e == 255u ? __uint_as_float(0x7FC00000u)
+                   : e == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23);
+}
+
 // ------------------------------------------------------------------ code registers
 // A 16-byte chunk of a packed row holds VPC = 128/BITS codes in 4 words.
 // It is split into NC = VPC/4 "code registers", each holding 4 codes in its

@@ -35,8 +35,45 @@ __global__ void __launch_bounds__(256) k_dequant(const uint32_t* __restrict__ w,
   }
 }
 
+// MX FP4: w = e2m1(q) * 2^(e - 127), exact in fp32 (q' * 2^(e - 128) with
+// q' = 2 e2m1(q) + 12, minus 12 * 2^(e - 128)).
+__global__ void __launch_bounds__(256) k_dequant_mx(const uint32_t* __restrict__ w,
+                                                    const uint8_t* __restrict__ ex, int out_dim,
+                                                    int in_dim, uint8_t* __restrict__ q_out,
+                                                    float* __restrict__ w_out) {
+  const int64_t wpr = (int64_t)in_dim / 8;
+  const int64_t total = (int64_t)out_dim * wpr;
+  const int gpr = in_dim / 32;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / wpr;
+    const int64_t c0 = (i % wpr) * 8;
+    const uint32_t word = w[i];
+    const float sc = mx_scale(ex[r * gpr + (int)(c0 / 32)]);
+    const uint32_t lo = mx_q8(word & 0x0F0F0F0Fu), hi = mx_q8((word >> 4) & 0x0F0F0F0Fu);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t q = (word >> (4 * j)) & 15u;
+      const int qq = (int)(((j & 1) ? hi : lo) >> (8 * (j >> 1)) & 255u);  // q' = 2 e2m1 + 12
+      if (q_out) q_out[r * in_dim + c0 + j] = (uint8_t)q;
+      const float mag = (float)abs(qq - 12) * 0.5f * sc;  // |e2m1| * 2^(e-127), exact
+      if (w_out) w_out[r * in_dim + c0 + j] = (q & 8u) ? -mag : mag;  // code 8 is -0
+    }
+  }
+}
+
 cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, float* w_out,
                            cudaStream_t st) {
+  if (t.format == MOEQ_FMT_MXFP4) {
+    const uint32_t* w = t.w + (int64_t)expert * t.expert_stride_w;
+    const uint8_t* e = reinterpret_cast<const uint8_t*>(t.scales) + (int64_t)expert * t.expert_stride_sb;
+    const int64_t total = (int64_t)t.out_dim * t.in_dim / 8;
+    int64_t grid = (total + 255) / 256;
+    if (grid > 148 * 32) grid = 148 * 32;
+    if (grid == 0) return cudaSuccess;
+    k_dequant_mx<<<(int)grid, 256, 0, st>>>(w, e, t.out_dim, t.in_dim, q_out, w_out);
+    return cudaGetLastError();
+  }
   const uint32_t* w = t.w + (int64_t)expert * t.expert_stride_w;
   const uint16_t* s = t.scales + (int64_t)expert * t.expert_stride_sb;
   const uint16_t* b = t.biases + (int64_t)expert * t.expert_stride_sb;

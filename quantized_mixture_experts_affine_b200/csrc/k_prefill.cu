@@ -666,6 +666,7 @@ moeq_status check_prefill(const moeq_layer* L) {
                                &L->sh_gate, &L->sh_up, &L->sh_down, &L->sh_expert_gate};
   const int n = L->has_shared ? 8 : 4;
   for (int i = 0; i < n; ++i) {
+    if (ts[i]->format != MOEQ_FMT_AFFINE) return MOEQ_ERR_UNSUPPORTED;
     const int G = ts[i]->group_size;
     if (G != 32 && G != 64 && G != 128) return MOEQ_ERR_UNSUPPORTED;
     if (G == 32 && ts[i]->bits == 2) return MOEQ_ERR_UNSUPPORTED;

@@ -31,7 +31,7 @@ class DeviceLayer:
 
         def q(t: synth.DevQ):
             return moeq.qtensor(t.w, t.s, t.b, t.out_dim, t.in_dim, t.bits, t.group_size,
-                                t.n_mats)
+                                t.n_mats, getattr(t, "fmt", 0))
         z = moeq.QTensor()
         self.desc = moeq.Layer(q(self.router), q(self.gate), q(self.up), q(self.down),
                                int(c.shared), q(self.sh_gate) if c.shared else z,

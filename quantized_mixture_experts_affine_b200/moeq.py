@@ -41,7 +41,7 @@ class QTensor(C.Structure):
     _fields_ = [("w", C.c_void_p), ("scales", C.c_void_p), ("biases", C.c_void_p),
                 ("out_dim", C.c_int32), ("in_dim", C.c_int32), ("bits", C.c_int32),
                 ("group_size", C.c_int32), ("expert_stride_w", C.c_int64),
-                ("expert_stride_sb", C.c_int64)]
+                ("expert_stride_sb", C.c_int64), ("format", C.c_int32)]
 
 
 class Layer(C.Structure):
@@ -116,11 +116,17 @@ def _check(fn, rc):
         raise MoeqError(fn, rc)
 
 
-def qtensor(w, scales, biases, out_dim, in_dim, bits, group_size=64, n_mats=1) -> QTensor:
-    """Descriptor of a bank of n_mats packed matrices stored back to back."""
+FMT_AFFINE, FMT_MXFP4 = 0, 1
+
+
+def qtensor(w, scales, biases, out_dim, in_dim, bits, group_size=64, n_mats=1,
+            fmt: int = FMT_AFFINE) -> QTensor:
+    """Descriptor of a bank of n_mats packed matrices stored back to back
+    (MX FP4: scales are the uint8 exponents, biases unused)."""
     sw = out_dim * in_dim * bits // 32 if n_mats > 1 else 0
     ssb = out_dim * (in_dim // group_size) if n_mats > 1 else 0
-    return QTensor(_ptr(w), _ptr(scales), _ptr(biases), out_dim, in_dim, bits, group_size, sw, ssb)
+    return QTensor(_ptr(w), _ptr(scales), _ptr(biases) if fmt == FMT_AFFINE else None, out_dim,
+                   in_dim, bits, group_size, sw, ssb, fmt)
 
 
 def moeq_dequant(t: QTensor, expert: int, q_out=None, w_out=None, stream=None) -> None:

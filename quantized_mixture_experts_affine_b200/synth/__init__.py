@@ -39,6 +39,8 @@ def _L():
                                                 i32]
         _lib.moeq_synth_tensor_dev.argtypes = [u64, u64, i32, i32, i32, i32, i32, i32, P, P, P,
                                                P]
+        _lib.moeq_synth_tensor_mx_host.argtypes = [u64, u64, i32, i32, i32, P, P, i32]
+        _lib.moeq_synth_tensor_mx_dev.argtypes = [u64, u64, i32, i32, i32, P, P, P]
         _lib.moeq_synth_normal_bf16_host.argtypes = [u64, u64, i64, P, i32]
         _lib.moeq_synth_normal_bf16_dev.argtypes = [u64, u64, i64, P, P]
         _lib.moeq_synth_zipf_logits_host.argtypes = [u64, u64, i32, i32, C.c_double, P, P]
@@ -49,7 +51,8 @@ def _L():
 @dataclass
 class HostQ:
     """Packed bank in host memory.  w: u32 [n_mats][out][in*bits/32];
-    s, b: u16 (bf16 bits) [n_mats][out][in/G]."""
+    s, b: u16 (bf16 bits) [n_mats][out][in/G].  fmt 1 (MX FP4): s holds the
+    u8 E8M0 exponents, b is empty."""
     w: np.ndarray
     s: np.ndarray
     b: np.ndarray
@@ -58,20 +61,22 @@ class HostQ:
     bits: int
     group_size: int
     n_mats: int
+    fmt: int = 0
 
     @property
     def nbytes(self) -> int:
         return self.w.nbytes + self.s.nbytes + self.b.nbytes
 
     def mat(self, m: int) -> "HostQ":
-        return HostQ(self.w[m:m + 1], self.s[m:m + 1], self.b[m:m + 1], self.out_dim,
-                     self.in_dim, self.bits, self.group_size, 1)
+        return HostQ(self.w[m:m + 1], self.s[m:m + 1], self.b[m:m + 1] if self.fmt == 0 else self.b,
+                     self.out_dim, self.in_dim, self.bits, self.group_size, 1, self.fmt)
 
 
 @dataclass
 class DevQ:
     """Packed bank in device memory (torch tensors; w int32 storage of u32,
-    s/b int16 storage of bf16 bits)."""
+    s/b int16 storage of bf16 bits; fmt 1 (MX FP4): s uint8 exponents, b
+    empty)."""
     w: "object"
     s: "object"
     b: "object"
@@ -80,19 +85,51 @@ class DevQ:
     bits: int
     group_size: int
     n_mats: int
+    fmt: int = 0
 
     @property
     def nbytes(self) -> int:
-        return (self.w.numel() * 4 + self.s.numel() * 2 + self.b.numel() * 2)
+        return (self.w.numel() * 4 + self.s.numel() * self.s.element_size() +
+                self.b.numel() * self.b.element_size())
 
     @property
     def bytes_per_mat(self) -> int:
         return self.nbytes // self.n_mats
 
     def to_host(self) -> HostQ:
-        return HostQ(self.w.cpu().numpy().view(np.uint32), self.s.cpu().numpy().view(np.uint16),
+        sd = np.uint16 if self.fmt == 0 else np.uint8
+        return HostQ(self.w.cpu().numpy().view(np.uint32), self.s.cpu().numpy().view(sd),
                      self.b.cpu().numpy().view(np.uint16), self.out_dim, self.in_dim, self.bits,
-                     self.group_size, self.n_mats)
+                     self.group_size, self.n_mats, self.fmt)
+
+
+def tensor_mx_host(seed: int, tg: int, n_mats: int, out_dim: int, in_dim: int, threads: int = 0,
+                   first_mat: int = 0) -> HostQ:
+    """MX FP4 bank (4-bit E2M1 codes, one E8M0 byte per 32 values) from the
+    same weight streams as tensor_host."""
+    ws, ss = _shapes(n_mats, out_dim, in_dim, 4, 32)
+    w = np.empty(ws, np.uint32)
+    e = np.empty(ss, np.uint8)
+    rc = _L().moeq_synth_tensor_mx_host(seed, tg + first_mat, n_mats, out_dim, in_dim,
+                                        w.ctypes.data, e.ctypes.data, threads)
+    if rc:
+        raise ValueError(f"moeq_synth_tensor_mx_host rc={rc}")
+    return HostQ(w, e, np.zeros(0, np.uint16), out_dim, in_dim, 4, 32, n_mats, 1)
+
+
+def tensor_mx_dev(seed: int, tg: int, n_mats: int, out_dim: int, in_dim: int, device="cuda",
+                  stream=None) -> DevQ:
+    import torch
+    ws, ss = _shapes(n_mats, out_dim, in_dim, 4, 32)
+    w = torch.empty(ws, dtype=torch.int32, device=device)
+    e = torch.empty(ss, dtype=torch.uint8, device=device)
+    st = stream if stream is not None else torch.cuda.current_stream(device)
+    rc = _L().moeq_synth_tensor_mx_dev(seed, tg, n_mats, out_dim, in_dim, w.data_ptr(),
+                                       e.data_ptr(), st.cuda_stream)
+    if rc:
+        raise RuntimeError(f"moeq_synth_tensor_mx_dev rc={rc}")
+    return DevQ(w, e, torch.zeros(0, dtype=torch.int16, device=device), out_dim, in_dim, 4, 32,
+                n_mats, 1)
 
 
 def packed_bytes(out_dim: int, in_dim: int, bits: int, group_size: int = 64) -> int:

@@ -80,6 +80,54 @@ SYN_API int moeq_synth_tensor_dev(uint64_t seed, uint64_t tag, int n_mats, int o
   return cudaGetLastError() == cudaSuccess ? 0 : 10;
 }
 
+/* MX FP4 banks: 4-bit E2M1 codes and one E8M0 byte per group of 32, from
+ * the same weight streams as the affine tensors (syn_make_group_mx). */
+SYN_API int moeq_synth_tensor_mx_host(uint64_t seed, uint64_t tag, int n_mats, int out_dim,
+                                      int in_dim, uint32_t* w, uint8_t* e, int n_threads) {
+  int rc = syn_check_shape(n_mats, out_dim, in_dim, 4, 32);
+  if (rc) return rc;
+  const int64_t words_per_row = (int64_t)in_dim / 8;
+  const int groups = in_dim / 32;
+  const int64_t total_rows = (int64_t)n_mats * out_dim;
+  if (n_threads <= 0) n_threads = omp_get_max_threads();
+#pragma omp parallel for num_threads(n_threads) schedule(static)
+  for (int64_t rr = 0; rr < total_rows; ++rr) {
+    const int m = (int)(rr / out_dim);
+    const int64_t row = rr % out_dim;
+    const uint64_t key = syn_key(seed, tag + (uint64_t)m);
+    for (int g = 0; g < groups; ++g)
+      syn_make_group_mx(key, row, in_dim, g, w + rr * words_per_row, e + rr * groups + g);
+  }
+  return 0;
+}
+
+__global__ void syn_tensor_mx_kernel(uint64_t seed, uint64_t tag, int out_dim, int in_dim,
+                                     int64_t total_groups, uint32_t* w, uint8_t* e) {
+  const int groups = in_dim / 32;
+  const int64_t words_per_row = (int64_t)in_dim / 8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total_groups;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t rr = i / groups;
+    const int g = (int)(i % groups);
+    const int m = (int)(rr / out_dim);
+    const int64_t row = rr % out_dim;
+    const uint64_t key = syn_key(seed, tag + (uint64_t)m);
+    syn_make_group_mx(key, row, in_dim, g, w + rr * words_per_row, e + rr * groups + g);
+  }
+}
+
+SYN_API int moeq_synth_tensor_mx_dev(uint64_t seed, uint64_t tag, int n_mats, int out_dim,
+                                     int in_dim, uint32_t* w, uint8_t* e, void* stream) {
+  int rc = syn_check_shape(n_mats, out_dim, in_dim, 4, 32);
+  if (rc) return rc;
+  const int64_t total_groups = (int64_t)n_mats * out_dim * (in_dim / 32);
+  int64_t blocks = (total_groups + 255) / 256;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  syn_tensor_mx_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+      seed, tag, out_dim, in_dim, total_groups, w, e);
+  return cudaGetLastError() == cudaSuccess ? 0 : 10;
+}
+
 /* n bf16 values ~ N(0,1): element i = bf16_rne(syn_unit_normal(key, i)). */
 SYN_API int moeq_synth_normal_bf16_host(uint64_t seed, uint64_t tag, int64_t n, uint16_t* out,
                                         int n_threads) {

@@ -156,4 +156,64 @@ SYN_HD void syn_make_group(uint64_t key, int64_t row, int in_dim, int g, int G,
   }
 }
 
+/*
+ * MX FP4 (OCP Microscaling Formats v1.0: E2M1 elements, one E8M0 scale per
+ * block of 32; the mlx issue page's mode="mxfp4") of one group of 32 fp32
+ * weights.  Shared exponent X = floor(log2(max|w|)) - 2 (2 = the largest
+ * E2M1 exponent), stored as the byte X + 127 (clamped to 0..254); every
+ * element is w / 2^X (exact) rounded to the nearest E2M1 value, ties to the
+ * even mantissa, magnitudes above 6 saturating to 6; an all-zero group gets
+ * the byte 0 and zero codes.  Codes: bit 3 sign, bits 2..1 exponent, bit 0
+ * mantissa.
+ */
+SYN_HD uint8_t syn_e2m1_code(float v) {
+  const uint8_t sign = v < 0.0f ? 8 : 0;
+  const float a = v < 0.0f ? -v : v;
+  uint8_t m;  /* magnitude code 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6 */
+  if (a <= 0.25f) m = 0;
+  else if (a < 0.75f) m = 1;
+  else if (a <= 1.25f) m = 2;
+  else if (a < 1.75f) m = 3;
+  else if (a <= 2.5f) m = 4;
+  else if (a < 3.5f) m = 5;
+  else if (a <= 5.0f) m = 6;
+  else m = 7;
+  return (uint8_t)(sign | m);
+}
+
+SYN_HD void syn_make_group_mx(uint64_t key, int64_t row, int in_dim, int g, uint32_t* words_row,
+                              uint8_t* e_out) {
+  float w[32];
+  float amax = 0.0f;
+  for (int i = 0; i < 32; ++i) {
+    w[i] = syn_weight(key, (uint64_t)row * (uint64_t)in_dim + (uint64_t)(g * 32 + i));
+    const float a = w[i] < 0.0f ? -w[i] : w[i];
+    amax = a > amax ? a : amax;
+  }
+  uint8_t q[32];
+  uint8_t ebyte = 0;
+  if (amax > 0.0f) {
+    union { float f; uint32_t u; } v;
+    v.f = amax;
+    int ex = (int)((v.u >> 23) & 0xFFu) - 127;   /* floor(log2(amax)), amax normal */
+    if (((v.u >> 23) & 0xFFu) == 0) ex = -127;   /* subnormal: below any scale used here */
+    int X = ex - 2;
+    X = X < -127 ? -127 : (X > 127 ? 127 : X);
+    ebyte = (uint8_t)(X + 127);
+    /* 2^-X as an fp32 power of two (X in [-126, 127]: normal; -127 clamps) */
+    union { float f; uint32_t u; } inv;
+    const int ie = -X + 127;
+    inv.u = (uint32_t)(ie < 1 ? 1 : (ie > 254 ? 254 : ie)) << 23;
+    for (int i = 0; i < 32; ++i) q[i] = syn_e2m1_code(w[i] * inv.f);
+  } else {
+    for (int i = 0; i < 32; ++i) q[i] = 0;
+  }
+  *e_out = ebyte;
+  for (int k = 0; k < 4; ++k) {
+    uint32_t word = 0;
+    for (int j = 0; j < 8; ++j) word |= ((uint32_t)q[k * 8 + j]) << (4 * j);
+    words_row[g * 4 + k] = word;
+  }
+}
+
 #endif

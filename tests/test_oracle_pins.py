@@ -467,3 +467,68 @@ def test_rmsnorm_invariants():
     assert np.allclose(c, 0.5 / np.sqrt(0.25 + 1e-2), rtol=1e-15)
     # rows are independent of one another
     assert np.allclose(oracle.rmsnorm(y[2:3], one, 1e-6), oracle.rmsnorm(y, one, 1e-6)[2:3])
+
+
+# ------------------------------------------------------------------ MX FP4 codes
+
+# The E2M1 element values of the OCP Microscaling Formats specification
+# (v1.0, FP4 E2M1 table): codes 0..7 and their negatives 8..15.
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,
+              -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def _mx_tensor(codes, ebytes):
+    """Host MX FP4 tensor from unpacked codes [out][in] and exponent bytes
+    [out][in/32] (packed here independently of the oracle: 8 codes per word,
+    low nibble first)."""
+    codes = np.asarray(codes, np.uint32)
+    out, inn = codes.shape
+    w = np.zeros((1, out, inn // 8), np.uint32)
+    for j in range(8):
+        w[0] |= codes[:, j::8] << (4 * j)
+    e = np.ascontiguousarray(np.asarray(ebytes, np.uint8).reshape(1, out, inn // 32))
+    return oracle.OracleTensor(w, e, np.zeros(0, np.uint16), out, inn, 4, 32, 1)
+
+
+def test_mxfp4_element_table_and_scale_bytes():
+    codes = np.tile(np.arange(16), 2)[None, :]            # one row of 32 values
+    for x, f in ((127, 1.0), (128, 2.0), (126, 0.5), (120, 2.0 ** -7), (140, 2.0 ** 13)):
+        w = oracle.dequant_f32(_mx_tensor(codes, [[x]]))
+        assert np.array_equal(w[0], np.array(E2M1_TABLE * 2, np.float32) * np.float32(f)), x
+        assert np.array_equal(np.signbit(w[0]), np.signbit(np.array(E2M1_TABLE * 2)))
+    assert np.isnan(oracle.dequant_f32(_mx_tensor(codes, [[255]]))).all()
+    q = oracle.unpack(_mx_tensor(codes, [[127]]))
+    assert np.array_equal(q[0], codes[0])
+
+
+def test_mxfp4_qmv_brute_force():
+    """Random codes and exponents (several groups per row): the oracle's
+    qmv equals a dense fp64 product of the table-decoded weights."""
+    rng = np.random.default_rng(7)
+    out, inn = 5, 128
+    codes = rng.integers(0, 16, (out, inn))
+    eb = rng.integers(110, 140, (out, inn // 32))
+    t = _mx_tensor(codes, eb)
+    dense = np.array(E2M1_TABLE)[codes] * np.ldexp(1.0, np.repeat(eb, 32, axis=1) - 127)
+    xb = _bf16(rng.normal(size=(3, inn)))
+    x = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    got = oracle.qmv(t, xb)
+    assert np.allclose(got, x @ dense.T, rtol=1e-13, atol=1e-300)
+
+
+def test_mxfp4_generator_round_trip():
+    """The generator's MX quantiser: every element within half an E2M1 step
+    (at its magnitude) times the group scale of the fp32 weight, the group
+    maximum mapped into [4, 6], and host and device streams equal by
+    construction (shared recipe)."""
+    H, O = 256, 6
+    t = synth.tensor_mx_host(3, synth.tag(synth.GATE), 1, O, H)
+    w32 = synth.weights_f32_host(3, synth.tag(synth.GATE), 0, O, H)
+    deq = oracle.dequant_f32(oracle.OracleTensor.of(t))
+    scale = np.ldexp(1.0, np.repeat(t.s[0].astype(int), 32, axis=1) - 127)
+    v = np.abs(w32 / scale)
+    step = np.where(v < 2, 0.5, np.where(v < 4, 1.0, 2.0))
+    over = np.maximum(v - 6.0, 0.0)
+    assert (np.abs(deq - w32) <= (step / 2 + over) * scale + 1e-12).all()
+    amax = np.abs(deq).reshape(O, H // 32, 32).max(axis=2) / scale[:, ::32]
+    assert ((amax >= 4.0) & (amax <= 6.0)).all()
