@@ -139,13 +139,7 @@ static moeq_status check_gemv_tensor(const moeq_qtensor& t, int nmat) {
   return MOEQ_OK;
 }
 
-static bool layer_has_mx(const moeq_layer* L) {
-  return is_mx(L->gate) || is_mx(L->down) ||
-         (L->has_shared && (is_mx(L->sh_gate) || is_mx(L->sh_down)));
-}
-
 static moeq_status check_decode_shapes(const moeq_layer* L) {
-  if (layer_has_mx(L)) return MOEQ_ERR_UNSUPPORTED;
   moeq_status s;
   if ((s = check_gemv_tensor(L->router, 1)) != MOEQ_OK) return s;
   if ((s = check_gemv_tensor(L->gate, 2)) != MOEQ_OK) return s;
@@ -233,6 +227,7 @@ static void set_shape(GemvArgs& a, const moeq_qtensor& t, int nmat) {
   const GemvShape sh = gemv_shape(t.in_dim, t.bits, nmat, t.group_size);
   a.in_dim = t.in_dim;
   a.G = t.group_size;
+  a.fmt = t.format;
   a.slices = sh.S;
   a.subsets = sh.J;
   a.rows_per_unit = sh.RU;
@@ -242,11 +237,12 @@ static void set_shape(GemvArgs& a, const moeq_qtensor& t, int nmat) {
 static int add_prefetch(GemvArgs& a, const moeq_qtensor& t, int expert) {
   const int64_t words = (int64_t)t.out_dim * t.in_dim * t.bits / 32;
   const int64_t groups = (int64_t)t.out_dim * (t.in_dim / t.group_size);
+  const bool mx = is_mx(t);
   const void* p[3] = {t.w + (int64_t)expert * t.expert_stride_w,
-                      t.scales + (int64_t)expert * t.expert_stride_sb,
-                      t.biases + (int64_t)expert * t.expert_stride_sb};
-  const int64_t b[3] = {words * 4, groups * 2, groups * 2};
-  for (int i = 0; i < 3 && a.n_pf < kMaxPrefetch; ++i)
+                      scale_at(t, (int64_t)expert * t.expert_stride_sb),
+                      mx ? nullptr : t.biases + (int64_t)expert * t.expert_stride_sb};
+  const int64_t b[3] = {words * 4, groups * (mx ? 1 : 2), mx ? 0 : groups * 2};
+  for (int i = 0; i < (mx ? 2 : 3) && a.n_pf < kMaxPrefetch; ++i)
     if (((uintptr_t)p[i] & 15) == 0) a.pf[a.n_pf++] = PrefetchRange{p[i], b[i]};
   return a.n_pf;
 }
@@ -257,8 +253,8 @@ static Seg plain_seg(const moeq_qtensor& t, int expert, const void* src, int64_t
   Seg s;
   memset(&s, 0, sizeof(s));
   const uint32_t* w = t.w + (int64_t)expert * t.expert_stride_w;
-  const uint16_t* sc = t.scales + (int64_t)expert * t.expert_stride_sb;
-  const uint16_t* bi = t.biases + (int64_t)expert * t.expert_stride_sb;
+  const uint16_t* sc = scale_at(t, (int64_t)expert * t.expert_stride_sb);
+  const uint16_t* bi = is_mx(t) ? nullptr : t.biases + (int64_t)expert * t.expert_stride_sb;
   s.w[0] = s.w[1] = w;
   s.s[0] = s.s[1] = sc;
   s.b[0] = s.b[1] = bi;
@@ -431,7 +427,8 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   // the router runs too, the down launch's producer starts on the plan's
   // flag instead of on the whole gate/up launch
   const bool sh_same_gu = L->has_shared && L->sh_gate.bits == L->gate.bits &&
-                          L->sh_gate.group_size == L->gate.group_size;
+                          L->sh_gate.group_size == L->gate.group_size &&
+                          L->sh_gate.format == L->gate.format;
   const bool fused_plan =
       n <= kFusedMaxPairs && (!L->has_shared || sh_same_gu) &&
       plan_scratch_bytes(M, K, E, plan_route_warps(M, E, gemv_threads() / 32)) <=
@@ -502,9 +499,11 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     p.units_per_seg_gu_sh = units_for(L->sh_gate, L->sh_gate.out_dim, 2);
     p.units_per_seg_dn_sh = units_for(L->sh_down, H, 1);
     p.shared_same_gu = (L->sh_gate.bits == L->gate.bits &&
-                        L->sh_gate.group_size == L->gate.group_size);
+                        L->sh_gate.group_size == L->gate.group_size &&
+                        L->sh_gate.format == L->gate.format);
     p.shared_same_dn = (L->sh_down.bits == L->down.bits &&
                         L->sh_down.group_size == L->down.group_size &&
+                        L->sh_down.format == L->down.format &&
                         L->sh_down.in_dim == L->down.in_dim);
   }
   p.status = status_ptr();
@@ -608,7 +607,6 @@ MOEQ_API moeq_status moeq_qmv(const moeq_qtensor* t, int32_t expert, const uint1
   if (expert > 0 && (t->expert_stride_w <= 0 || t->expert_stride_sb <= 0))
     return MOEQ_ERR_INVALID_ARG;
   if ((s = check_gemv_tensor(*t, 1)) != MOEQ_OK) return s;
-  if (is_mx(*t)) return MOEQ_ERR_UNSUPPORTED;
   if (!aligned(x, 16) || ((int64_t)t->in_dim * 2) % 16 || !aligned(y, 4)) return MOEQ_ERR_ALIGNMENT;
   Seg seg = plain_seg(*t, expert, x, t->in_dim, y, t->out_dim, M, 0);
   LAUNCH(run_plain(*t, &seg, 1, 3, nullptr, (cudaStream_t)stream));

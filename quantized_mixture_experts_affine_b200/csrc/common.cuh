@@ -96,6 +96,16 @@ __device__ __forceinline__ uint32_t mx_q8(uint32_t c) {
   return (pos & ~smask) | (neg & smask);
 }
 
+// Scale array of t advanced by `entries` groups (MX FP4: one byte each,
+// affine: one bf16 each).
+__host__ __device__ __forceinline__ const uint16_t* scale_at(const moeq_qtensor& t,
+                                                             int64_t entries) {
+  return t.format == MOEQ_FMT_MXFP4
+             ? reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(t.scales) +
+                                                 entries)
+             : t.scales + entries;
+}
+
 // 2^(e - 127) in fp32 (e = 0: 2^-127, subnormal; e = 255: NaN).
 __device__ __forceinline__ float mx_scale(uint32_t e) {
   return e == 255u ? __uint_as_float(0x7FC00000u)

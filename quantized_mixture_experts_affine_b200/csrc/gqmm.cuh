@@ -136,6 +136,7 @@ struct Args {
                             // sb_w*G/64 >= 2 k-blocks)
   int32_t G;                // group size of the launch's tensors: 32, 64 or 128 (32: not
                             // 2-bit, whose 16-byte code chunks span two groups)
+  int32_t fmt;              // MOEQ_FMT_*: MX FP4 windows hold one exponent byte per group
   int* status;
 };
 
@@ -220,6 +221,33 @@ __device__ __forceinline__ void group_h2(uint32_t sbits, uint32_t bbits, __half2
   if (bad) set_status(status, MOEQ_ERR_RANGE);
   s2 = __float2half2_rn(s);
   b2 = __float2half2_rn(b);
+}
+
+// MX FP4 group with E8M0 byte e, as the affine group of its codes q' = 2
+// e2m1 + 12: s = 2^(e - 128), b = -12 s, both exact in fp16 for e in
+// [102, 140] (the weights between 6 * 2^-25 and 6 * 2^13); other bytes
+// are outside the prefill tiles' range (MOEQ_ERR_RANGE).
+__device__ __forceinline__ void group_h2_mx(uint32_t e, __half2& s2, __half2& b2, int* status) {
+  if (e < 102u || e > 140u) set_status(status, MOEQ_ERR_RANGE);
+  const float s = __uint_as_float((e >= 1u ? e - 1u : 0u) << 23);  // 2^(e - 128)
+  s2 = __float2half2_rn(s);
+  b2 = __float2half2_rn(-12.0f * s);
+}
+
+// One 16-byte chunk of E2M1 codes (32 values, low nibble first) as two
+// 16-byte chunks of 8-bit codes q' in value order (u0: values 0..15).
+__device__ __forceinline__ void mx_chunk_q8(uint4 raw, uint4& u0, uint4& u1) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t n[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t lo = mx_q8(w[k] & 0x0F0F0F0Fu);         // values 8k + 0, 2, 4, 6
+    const uint32_t hi = mx_q8((w[k] >> 4) & 0x0F0F0F0Fu);  // values 8k + 1, 3, 5, 7
+    n[2 * k] = __byte_perm(lo, hi, 0x5140u);
+    n[2 * k + 1] = __byte_perm(lo, hi, 0x7362u);
+  }
+  u0 = make_uint4(n[0], n[1], n[2], n[3]);
+  u1 = make_uint4(n[4], n[5], n[6], n[7]);
 }
 
 // Dequantise one 16-byte chunk of packed codes into fp16 weights: 16 (8-bit),
@@ -320,9 +348,10 @@ __device__ __forceinline__ void dequant_chunk_split(uint4 raw, float s, float b,
 
 // GS: the group size when fixed at compile time (64, the common case, with
 // no group arithmetic left at run time), or 0 to take a.G (32 or 128).
-template <int BITS, int EPI, bool PAIR, int GS>
+template <int BITS, int EPI, bool PAIR, int GS, bool MX = false>
 __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Args a) {
   const int G = GS ? GS : a.G;
+  static_assert(!MX || (BITS == 4 && GS == 32 && EPI != EPI_SPLIT), "MX FP4: 4-bit, G 32");
   using SM = Smem<BITS, PAIR>;
   using RW = Raw<BITS>;
   constexpr int S1 = SM::S1, SR = SM::SR, S2 = SM::S2, BR = SM::BR;
@@ -502,8 +531,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
         b_row<EPI>(sg, nt, r, src, q, ok);
         if (!ok) q = 0;
         wp[j] = sg.w[src] + (int64_t)q * wrow;
-        sp[j] = sg.s[src] + (int64_t)q * groups;
-        bp[j] = sg.b[src] + (int64_t)q * groups;
+        // (MX FP4: one exponent byte per group, no biases)
+        sp[j] = MX ? reinterpret_cast<const uint16_t*>(
+                         reinterpret_cast<const uint8_t*>(sg.s[src]) + (int64_t)q * groups)
+                   : sg.s[src] + (int64_t)q * groups;
+        bp[j] = MX ? nullptr : sg.b[src] + (int64_t)q * groups;
         ok16[j] = ok ? 16u : 0u;
       }
       // tensor-map halves: (source, first row) of tile rows 0..127 and 128..255
@@ -547,7 +579,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           for (int j = 0; j < JR; ++j) {
             const int r = lane + 32 * j;
             const uint32_t d = sbw + r * 32;
-            if (W == 8) {
+            if (MX) {
+              const uint8_t* e0 = reinterpret_cast<const uint8_t*>(sp[j]) + g0;
+              if (W == 8) tc::cp_async8(d, e0, ok16[j] ? 8u : 0u);
+              else tc::cp_async4(d, e0, ok16[j] ? 4u : 0u);
+            } else if (W == 8) {
               tc::cp_async16(d, sp[j] + g0, ok16[j]);
               tc::cp_async16(d + 16, bp[j] + g0, ok16[j]);
             } else if (W == 4) {
@@ -769,7 +805,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           // this row's window of W scales and W biases, kept in registers
           const uint32_t sbw =
               sbase + SM::SB_OFF + ((it >> wl) % SM::NWB) * SM::SB_WIN + r * 32;
-          if (W == 8) {
+          if (MX) {
+            // W exponent bytes: groups 0..3 in swin.x, 4..7 in swin.y
+            swin = W == 8 ? make_uint4(lds64(sbw).x, lds64(sbw).y, 0u, 0u)
+                          : make_uint4(lds32(sbw), 0u, 0u, 0u);
+          } else if (W == 8) {
             swin = lds128(sbw);
             bwin = lds128(sbw + 16);
           } else if (W == 4) {
@@ -794,7 +834,22 @@ __global__ void __launch_bounds__(THREADS, 1) k_gqmm(const __grid_constant__ Arg
           // G = 32 (8- and 4-bit only): chunks of one thread may fall in
           // both groups of the k-block
           const bool per_chunk = G == 32 && CPT > 1;
-          if (EPI == EPI_SPLIT) {
+          if (MX) {
+            // exponent byte of group j of the window: byte j % 4 of word j / 4
+            auto ebyte = [&](int j) { return ((j < 4 ? swin.x : swin.y) >> (8 * (j & 3))) & 255u; };
+            const int j0 = 2 * kbw + (c_lo * VPC >= 32);
+            __half2 s2h, b2h;
+            group_h2_mx(ebyte(j0), s2h, b2h, status);
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+              if (per_chunk && (c_lo + c) * VPC >= 32 && c_lo * VPC < 32)
+                group_h2_mx(ebyte(2 * kbw + 1), s2h, b2h, status);
+              uint4 u0, u1;
+              mx_chunk_q8(raw[c], u0, u1);
+              dequant_chunk<8>(u0, s2h, b2h, bst, r, (c_lo + c) * 4);
+              dequant_chunk<8>(u1, s2h, b2h, bst, r, (c_lo + c) * 4 + 2);
+            }
+          } else if (EPI == EPI_SPLIT) {
 #pragma unroll
             for (int c = 0; c < CPT; ++c) {
               uint32_t sb = sbits, bb = bbits;

@@ -172,9 +172,11 @@ __device__ __forceinline__ void prefetch_down(const DecodePlanArgs& p, const int
     const moeq_qtensor& t = sh ? p.sh_down : p.down;
     const int64_t e = sh ? 0 : ent[i];
     const int64_t gr = (int64_t)t.out_dim * (t.in_dim / t.group_size);
-    const void* ptr[3] = {t.w + e * t.expert_stride_w, t.scales + e * t.expert_stride_sb,
-                          t.biases + e * t.expert_stride_sb};
-    const int64_t bytes[3] = {(int64_t)t.out_dim * t.in_dim * t.bits / 8, gr * 2, gr * 2};
+    const bool mx = t.format == MOEQ_FMT_MXFP4;
+    const void* ptr[3] = {t.w + e * t.expert_stride_w, scale_at(t, e * t.expert_stride_sb),
+                          mx ? nullptr : t.biases + e * t.expert_stride_sb};
+    const int64_t bytes[3] = {(int64_t)t.out_dim * t.in_dim * t.bits / 8, gr * (mx ? 1 : 2),
+                              mx ? 0 : gr * 2};
     for (int k = 0; k < 3; ++k) {
       const int64_t pieces = (bytes[k] + PIECE - 1) / PIECE;
       int64_t g = g0 + ((blockIdx.x - g0 % gridDim.x) + gridDim.x) % gridDim.x;
@@ -258,19 +260,24 @@ struct GvUnit {
 // scale/bias rows -- contiguous runs of nrows * gpr entries, bulk-copied
 // when 16-byte aligned, else copied entry by entry -- and the unit's vector
 // references when they live in global memory.
-template <int NMAT>
+// (MX: one exponent byte per group in the scale rows, no bias rows.)
+template <int NMAT, bool MX = false>
 __device__ __forceinline__ void gv_issue(uint8_t* gsm, uint32_t sbase, uint64_t* full, uint32_t s,
                                          const GvUnit& u, int row_bytes, int gpr, int RU) {
+  constexpr int ES = MX ? 1 : 2;  // bytes per scale entry
   const int lane = threadIdx.x & 31;
   const int codes_bytes = NMAT * RU * row_bytes;
-  const int sb_bytes = RU * gpr * 2;
+  const int sb_bytes = RU * gpr * ES;
   const uint32_t st = sbase + s * GV_STAGE_BYTES;
   const int sb_n = u.nrows * gpr;
-  bool sb_bulk = ((sb_n * 2) & 15) == 0 && ((codes_bytes | sb_bytes) & 15) == 0;
+  auto srow = [&](int m) {
+    return reinterpret_cast<const uint8_t*>(u.s[m]) + (int64_t)u.r0 * gpr * ES;
+  };
+  bool sb_bulk = ((sb_n * ES) & 15) == 0 && ((codes_bytes | sb_bytes) & 15) == 0;
 #pragma unroll
   for (int m = 0; m < NMAT; ++m)
-    sb_bulk = sb_bulk && ((((uintptr_t)(u.s[m] + (int64_t)u.r0 * gpr)) |
-                           ((uintptr_t)(u.b[m] + (int64_t)u.r0 * gpr))) & 15) == 0;
+    sb_bulk = sb_bulk && ((((uintptr_t)srow(m)) |
+                           (MX ? 0 : (uintptr_t)(u.b[m] + (int64_t)u.r0 * gpr))) & 15) == 0;
   if (lane == 0) {
     GvMeta* mt = reinterpret_cast<GvMeta*>(gsm + GvSmem::META_OFF + s * GvSmem::META_STRIDE);
     mt->r0 = u.r0;
@@ -283,21 +290,29 @@ __device__ __forceinline__ void gv_issue(uint8_t* gsm, uint32_t sbase, uint64_t*
     mt->dst_stride = u.dst_stride;
     mt->vecs = u.vecs;
     tc::mbar_arrive_expect_tx(
-        &full[s], (uint32_t)(NMAT * u.nrows * row_bytes + (sb_bulk ? 2 * NMAT * sb_n * 2 : 0)));
+        &full[s], (uint32_t)(NMAT * u.nrows * row_bytes +
+                             (sb_bulk ? (MX ? 1 : 2) * NMAT * sb_n * ES : 0)));
 #pragma unroll
     for (int m = 0; m < NMAT; ++m) {
       tc::bulk_g2s(st + m * RU * row_bytes,
                    reinterpret_cast<const uint8_t*>(u.w[m]) + (int64_t)u.r0 * row_bytes,
                    (uint32_t)(u.nrows * row_bytes), &full[s]);
       if (sb_bulk) {
-        tc::bulk_g2s(st + codes_bytes + m * sb_bytes, u.s[m] + (int64_t)u.r0 * gpr,
-                     (uint32_t)(sb_n * 2), &full[s]);
-        tc::bulk_g2s(st + codes_bytes + (NMAT + m) * sb_bytes, u.b[m] + (int64_t)u.r0 * gpr,
-                     (uint32_t)(sb_n * 2), &full[s]);
+        tc::bulk_g2s(st + codes_bytes + m * sb_bytes, srow(m), (uint32_t)(sb_n * ES), &full[s]);
+        if (!MX)
+          tc::bulk_g2s(st + codes_bytes + (NMAT + m) * sb_bytes, u.b[m] + (int64_t)u.r0 * gpr,
+                       (uint32_t)(sb_n * 2), &full[s]);
       }
     }
   }
-  if (!sb_bulk) {
+  if (!sb_bulk && MX) {
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m) {
+      const uint8_t* s0 = srow(m);
+      uint8_t* sd = gsm + s * GV_STAGE_BYTES + codes_bytes + m * sb_bytes;
+      for (int e = lane; e < sb_n; e += 32) sd[e] = s0[e];
+    }
+  } else if (!sb_bulk) {
 #pragma unroll
     for (int m = 0; m < NMAT; ++m) {
       const uint16_t* s0 = u.s[m] + (int64_t)u.r0 * gpr;
@@ -325,8 +340,11 @@ __device__ __forceinline__ void gv_issue(uint8_t* gsm, uint32_t sbase, uint64_t*
   }
 }
 
-template <int BITS, int NL, int NMAT, int SRC, int EPI>
+// MX: the segments' tensors are MX FP4 (4-bit E2M1 codes translated to
+// q' = 2 e2m1 + 12 after the split, s = 2^(e - 128), b = -12 s per group).
+template <int BITS, int NL, int NMAT, int SRC, int EPI, bool MX = false>
 __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ GemvArgs a) {
+  static_assert(!MX || BITS == 4, "MX FP4 codes are 4-bit");
   constexpr int VPC = Chunk<BITS>::VPC;
   constexpr int NC = Chunk<BITS>::NC;
   constexpr int NB = SliceVec<BITS, NL>::NB;
@@ -371,7 +389,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   const int cpr = a.in_dim / VPC;
   // stage layout: codes [NMAT][RU][row_bytes], scales [NMAT][RU*gpr], biases [NMAT][RU*gpr]
   const int codes_bytes = NMAT * RU * row_bytes;
-  const int sb_bytes = RU * gpr * 2;
+  const int sb_bytes = RU * gpr * (MX ? 1 : 2);
   int* status = a.status;
   // a step planned in this launch lists the shared expert first; its
   // weights do not depend on the routing, so the producer puts this CTA's
@@ -397,7 +415,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
       gu.dst_base = pl.h + (int64_t)pl.M * pl.K * pl.I;
       gu.dst_stride = pl.sh_gate.out_dim;
       gu.vecs = nullptr;
-      gv_issue<2>(gsm, sbase, full, 0, gu, row_bytes, gpr, RU);
+      gv_issue<2, MX>(gsm, sbase, full, 0, gu, row_bytes, gpr, RU);
       preissued = 1;
     }
   }
@@ -581,7 +599,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         gu.dst_base = shfl_ptr(dst_base, u);
         gu.src_stride = __shfl_sync(0xffffffffu, src_stride, u);
         gu.dst_stride = __shfl_sync(0xffffffffu, dst_stride, u);
-        gv_issue<NMAT>(gsm, sbase, full, s, gu, row_bytes, gpr, RU);
+        gv_issue<NMAT, MX>(gsm, sbase, full, s, gu, row_bytes, gpr, RU);
       }
     }
   } else {
@@ -667,16 +685,27 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
               float s2[2] = {0.f, 0.f}, b2[2] = {0.f, 0.f};
               if (ok) {
                 wv = gq_lds128(st + (m * RU + row) * row_bytes + ch * 16);
-                const uint32_t sd = st + codes_bytes + m * sb_bytes + row * gpr * 2;
-                const uint32_t bd = st + codes_bytes + (NMAT + m) * sb_bytes + row * gpr * 2;
+                if (MX) {
+                  // one group per 32-value chunk: s = 2^(e - 128), b = -12 s
+                  const uint32_t e = lds_u8(st + codes_bytes + m * sb_bytes + row * gpr + gi[0]);
+                  s2[0] = 0.5f * mx_scale(e);
+                  b2[0] = -12.0f * s2[0];
+                } else {
+                  const uint32_t sd = st + codes_bytes + m * sb_bytes + row * gpr * 2;
+                  const uint32_t bd = st + codes_bytes + (NMAT + m) * sb_bytes + row * gpr * 2;
 #pragma unroll
-                for (int pb = 0; pb < NB; ++pb) {
-                  s2[pb] = bf16_bits_to_float(lds_u16(sd + gi[pb] * 2));
-                  b2[pb] = bf16_bits_to_float(lds_u16(bd + gi[pb] * 2));
+                  for (int pb = 0; pb < NB; ++pb) {
+                    s2[pb] = bf16_bits_to_float(lds_u16(sd + gi[pb] * 2));
+                    b2[pb] = bf16_bits_to_float(lds_u16(bd + gi[pb] * 2));
+                  }
                 }
               }
               uint32_t c[NC];
               Chunk<BITS>::split(wv, c);
+              if (MX) {
+#pragma unroll
+                for (int k = 0; k < NC; ++k) c[k] = mx_q8(c[k]);
+              }
               acc[m * RPW + i] = chunk_contrib<BITS, NL>(c, sv, s2, b2);
             }
           float tot = transpose_reduce<8>(acc);  // lane l: value l % 8
@@ -741,9 +770,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   }
 }
 
-template <int BITS, int NL, int NMAT, int SRC, int EPI>
+template <int BITS, int NL, int NMAT, int SRC, int EPI, bool MX = false>
 static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
-  auto kern = k_gemv<BITS, NL, NMAT, SRC, EPI>;
+  auto kern = k_gemv<BITS, NL, NMAT, SRC, EPI, MX>;
   // the shared-memory opt-in is per device
   static std::atomic<bool> attr[kMaxDevices];
   int dev;
@@ -770,6 +799,16 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
 cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,
                         cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
+  if (a.fmt == MOEQ_FMT_MXFP4) {  // 4-bit E2M1 experts (and qmv)
+    if (bits != 4) return cudaErrorInvalidValue;
+    if (nmat == 2 && nl == 2 && src == SRC_BF16)
+      return launch_one<4, 2, 2, SRC_BF16, EPI_SWIGLU, true>(a, grid, st);
+    if (nmat == 1 && nl == 3 && src == SRC_BF16)
+      return launch_one<4, 3, 1, SRC_BF16, EPI_PLAIN, true>(a, grid, st);
+    if (nmat == 1 && nl == 2 && src == SRC_F32)
+      return launch_one<4, 2, 1, SRC_F32, EPI_PLAIN, true>(a, grid, st);
+    return cudaErrorInvalidValue;
+  }
   // instantiated forms: router / qmv (3 limbs, bf16 tokens), gate/up + SwiGLU
   // (2 limbs, bf16 tokens), down (2 limbs, fp32 hidden rows)
   if (nmat == 2 && nl == 2 && src == SRC_BF16) {
@@ -905,10 +944,10 @@ __device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const
     const int gu0 = o.shared_first ? a.units_per_seg_gu_sh : 0;
     Seg g;
     g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
-    g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
+    g.s[0] = scale_at(a.gate, (int64_t)e * a.gate.expert_stride_sb);
     g.b[0] = a.gate.biases + (int64_t)e * a.gate.expert_stride_sb;
     g.w[1] = a.up.w + (int64_t)e * a.up.expert_stride_w;
-    g.s[1] = a.up.scales + (int64_t)e * a.up.expert_stride_sb;
+    g.s[1] = scale_at(a.up, (int64_t)e * a.up.expert_stride_sb);
     g.b[1] = a.up.biases + (int64_t)e * a.up.expert_stride_sb;
     g.out_dim = a.I;
     g.in_dim = a.H;
@@ -928,7 +967,7 @@ __device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const
   if (o.segs_dn) {
     Seg dn;
     dn.w[0] = dn.w[1] = a.down.w + (int64_t)e * a.down.expert_stride_w;
-    dn.s[0] = dn.s[1] = a.down.scales + (int64_t)e * a.down.expert_stride_sb;
+    dn.s[0] = dn.s[1] = scale_at(a.down, (int64_t)e * a.down.expert_stride_sb);
     dn.b[0] = dn.b[1] = a.down.biases + (int64_t)e * a.down.expert_stride_sb;
     dn.out_dim = a.H;
     dn.in_dim = a.I;

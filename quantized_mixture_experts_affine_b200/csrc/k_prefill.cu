@@ -349,10 +349,10 @@ __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ Offset
     gq::Seg g;
     memset(&g, 0, sizeof(g));
     g.w[0] = a.gate.w + (int64_t)e * a.gate.expert_stride_w;
-    g.s[0] = a.gate.scales + (int64_t)e * a.gate.expert_stride_sb;
+    g.s[0] = scale_at(a.gate, (int64_t)e * a.gate.expert_stride_sb);
     g.b[0] = a.gate.biases + (int64_t)e * a.gate.expert_stride_sb;
     g.w[1] = a.up.w + (int64_t)e * a.up.expert_stride_w;
-    g.s[1] = a.up.scales + (int64_t)e * a.up.expert_stride_sb;
+    g.s[1] = scale_at(a.up, (int64_t)e * a.up.expert_stride_sb);
     g.b[1] = a.up.biases + (int64_t)e * a.up.expert_stride_sb;
     g.n0 = a.I;
     g.n_valid = a.I;
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(1024) k_offsets(const __grid_constant__ Offset
     gq::Seg d;
     memset(&d, 0, sizeof(d));
     d.w[0] = d.w[1] = a.down.w + (int64_t)e * a.down.expert_stride_w;
-    d.s[0] = d.s[1] = a.down.scales + (int64_t)e * a.down.expert_stride_sb;
+    d.s[0] = d.s[1] = scale_at(a.down, (int64_t)e * a.down.expert_stride_sb);
     d.b[0] = d.b[1] = a.down.biases + (int64_t)e * a.down.expert_stride_sb;
     d.n0 = a.H;
     d.n_valid = a.H;
@@ -425,10 +425,10 @@ __global__ void __launch_bounds__(32) k_scatter(const int32_t* __restrict__ idx,
 // Launch over `units` work items: one CTA per item up to the co-resident
 // count, or (PAIR) one cluster of two CTAs per item up to the co-resident
 // cluster count.
-template <int BITS, int EPI, bool PAIR, int GS>
+template <int BITS, int EPI, bool PAIR, int GS, bool MX = false>
 cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
   constexpr int smem = gq::Smem<BITS, PAIR>::ALLOC;
-  auto kern = gq::k_gqmm<BITS, EPI, PAIR, GS>;
+  auto kern = gq::k_gqmm<BITS, EPI, PAIR, GS, MX>;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
@@ -469,6 +469,11 @@ cudaError_t launch_gqmm_t(const gq::Args& a, int units, cudaStream_t st) {
 // reads it from the arguments.
 template <int BITS, int EPI, bool PAIR>
 cudaError_t launch_gqmm_g(const gq::Args& a, int units, cudaStream_t st) {
+  if (a.fmt == MOEQ_FMT_MXFP4) {
+    if constexpr (BITS == 4 && EPI != gq::EPI_SPLIT)
+      return launch_gqmm_t<4, EPI, PAIR, 32, true>(a, units, st);
+    return cudaErrorInvalidValue;
+  }
   if (a.G == 64) return launch_gqmm_t<BITS, EPI, PAIR, 64>(a, units, st);
   return launch_gqmm_t<BITS, EPI, PAIR, 0>(a, units, st);
 }
@@ -640,9 +645,20 @@ bool code_tensor_map(CUtensorMap* m, const moeq_qtensor& t, int n_mat) {
 int sb_window(const moeq_qtensor* const* ts, int n, int K) {
   const int G = ts[0]->group_size;
   for (int i = 1; i < n; ++i)
-    if (ts[i]->group_size != G) return 0;
+    if (ts[i]->group_size != G || ts[i]->format != ts[0]->format) return 0;
   if (G != 32 && G != 64 && G != 128) return 0;
   const int groups = K / G;
+  if (ts[0]->format == MOEQ_FMT_MXFP4) {
+    // one exponent byte per group: W-byte copies (W = 8 or 4, two or more
+    // k-blocks per window at G = 32) from W-aligned rows
+    for (int W = 8; W >= 4; W >>= 1) {
+      bool ok = groups % W == 0;
+      for (int i = 0; i < n && ok; ++i)
+        ok = ((uintptr_t)ts[i]->scales % W) == 0 && ts[i]->expert_stride_sb % W == 0;
+      if (ok) return W;
+    }
+    return 0;
+  }
   for (int W = 8; W >= 2; W >>= 1) {
     if (gq::win_kb_log2(W, G) < 1) continue;
     bool ok = groups % W == 0;
@@ -658,6 +674,7 @@ int sb_window(const moeq_qtensor* const* ts, int n, int K) {
 bool set_window(gq::Args& a, const moeq_qtensor* const* ts, int n, int K) {
   a.sb_w = sb_window(ts, n, K);
   a.G = ts[0]->group_size;
+  a.fmt = ts[0]->format;
   return a.sb_w != 0;
 }
 
@@ -666,11 +683,12 @@ moeq_status check_prefill(const moeq_layer* L) {
                                &L->sh_gate, &L->sh_up, &L->sh_down, &L->sh_expert_gate};
   const int n = L->has_shared ? 8 : 4;
   for (int i = 0; i < n; ++i) {
-    if (ts[i]->format != MOEQ_FMT_AFFINE) return MOEQ_ERR_UNSUPPORTED;
     const int G = ts[i]->group_size;
     if (G != 32 && G != 64 && G != 128) return MOEQ_ERR_UNSUPPORTED;
     if (G == 32 && ts[i]->bits == 2) return MOEQ_ERR_UNSUPPORTED;
-    if (((uintptr_t)ts[i]->scales & 3) || ((uintptr_t)ts[i]->biases & 3)) return MOEQ_ERR_ALIGNMENT;
+    if (ts[i]->format == MOEQ_FMT_AFFINE &&
+        (((uintptr_t)ts[i]->scales & 3) || ((uintptr_t)ts[i]->biases & 3)))
+      return MOEQ_ERR_ALIGNMENT;
     if (ts[i]->in_dim % 128) return MOEQ_ERR_UNSUPPORTED;
     if (ts[i]->expert_stride_sb % 2) return MOEQ_ERR_ALIGNMENT;
   }

@@ -138,6 +138,7 @@ struct GemvArgs {
   // shape shared by every segment of the launch
   int32_t in_dim;
   int32_t G;
+  int32_t fmt;              // MOEQ_FMT_* of every segment's tensors
   int32_t slices;           // S: 32-chunk slices per row
   int32_t subsets;          // J: row subsets (warps = S * J)
   int32_t rows_per_unit;    // RU = J * (8 / NMAT)
