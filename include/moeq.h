@@ -230,6 +230,45 @@ moeq_status moeq_layer_forward_norm(const moeq_layer* L, const uint16_t* x, int3
                                     uint16_t* y_norm, int32_t* idx_out, float* w_out, void* ws,
                                     size_t ws_bytes, int32_t mode, void* stream);
 
+/*
+ * Expert streaming from host memory with an HBM expert cache
+ * ("flash-moe-inference", per-layer pipeline "I/O: parallel pread K=4
+ * experts" and the parallel expert loading listing: the routed experts live
+ * in slower storage, the K a token selects are read in parallel, the
+ * operating system's page cache keeps recent ones, LRU).  Here the slower
+ * tier is host memory and the cache holds `slots` experts in HBM, least
+ * recently used out first.  For layers whose expert banks do not fit the
+ * GPU's memory.
+ *
+ * moeq_cache_create: L as moeq_layer_forward, except that gate, up and down
+ *   (all E experts) are in HOST memory (page-locked, e.g. cudaHostAlloc, so
+ *   that the copies run asynchronously); the router and the shared expert
+ *   are in device memory.  slots in [K, E]; max_tokens in [1, 64] with
+ *   max_tokens * K <= slots (one step's experts always fit).  Allocates the
+ *   slot banks and step buffers in device memory (call with the device
+ *   current).  Errors: INVALID_ARG, UNSUPPORTED (shapes outside the decode
+ *   path), CUDA (allocation).
+ * moeq_cache_forward: one decode step of M <= max_tokens tokens on `stream`:
+ *   router qmv and top-K on the device, the selection read back to the host
+ *   (synchronises `stream`), each selected expert not in a slot copied into
+ *   an empty slot or the least recently used slot the step does not use,
+ *   then moeq_expert_ffn on the slots.  Outputs as moeq_layer_forward
+ *   (decode path).  ws: device workspace of moeq_cache_workspace_bytes(c, M)
+ *   bytes.  One stream per cache; not thread-safe.
+ * moeq_cache_stats: distinct experts found in a slot (hits) and copied in
+ *   (misses) over all steps, and the bytes copied from host memory.
+ */
+typedef struct moeq_expert_cache moeq_expert_cache;
+moeq_status moeq_cache_create(const moeq_layer* L, int32_t slots, int32_t max_tokens,
+                              moeq_expert_cache** out);
+size_t moeq_cache_workspace_bytes(const moeq_expert_cache* c, int32_t M);
+moeq_status moeq_cache_forward(moeq_expert_cache* c, const uint16_t* x, int32_t M, float* y,
+                               const float* residual, int32_t* idx_out, float* w_out, void* ws,
+                               size_t ws_bytes, void* stream);
+moeq_status moeq_cache_stats(const moeq_expert_cache* c, uint64_t* hits, uint64_t* misses,
+                             uint64_t* bytes_copied);
+void moeq_cache_destroy(moeq_expert_cache* c);
+
 /* Workspace bytes moeq_expert_ffn / moeq_layer_forward need for M tokens
  * in `mode` (0 if the arguments are invalid). */
 size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mode);

@@ -27,7 +27,8 @@ EXPORTS = ("moeq_dequant", "moeq_qmv", "moeq_route_topk", "moeq_expert_ffn", "mo
            "moeq_workspace_bytes", "moeq_device_status", "moeq_status_str", "moeq_version",
            "moeq_set_profile_events", "moeq_launch_count", "moeq_layer_forward_static",
            "moeq_static_workspace_capacity", "moeq_selftest_wait_timeout",
-           "moeq_layer_forward_norm")
+           "moeq_layer_forward_norm", "moeq_cache_create", "moeq_cache_workspace_bytes",
+           "moeq_cache_forward", "moeq_cache_stats", "moeq_cache_destroy")
 
 
 class MoeqError(RuntimeError):
@@ -63,6 +64,17 @@ _lib.moeq_expert_ffn.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P
 _lib.moeq_layer_forward.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P, _P,
                                     C.c_size_t, C.c_int32, _P]
 _lib.moeq_layer_forward_static.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, _P, _P]
+_lib.moeq_cache_create.argtypes = [C.POINTER(Layer), C.c_int32, C.c_int32, C.POINTER(C.c_void_p)]
+_lib.moeq_cache_create.restype = C.c_int
+_lib.moeq_cache_workspace_bytes.argtypes = [C.c_void_p, C.c_int32]
+_lib.moeq_cache_workspace_bytes.restype = C.c_size_t
+_lib.moeq_cache_forward.argtypes = [C.c_void_p, _P, C.c_int32, _P, _P, _P, _P, _P, C.c_size_t, _P]
+_lib.moeq_cache_forward.restype = C.c_int
+_lib.moeq_cache_stats.argtypes = [C.c_void_p, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64),
+                                  C.POINTER(C.c_uint64)]
+_lib.moeq_cache_stats.restype = C.c_int
+_lib.moeq_cache_destroy.argtypes = [C.c_void_p]
+_lib.moeq_cache_destroy.restype = None
 _lib.moeq_layer_forward_norm.argtypes = [C.POINTER(Layer), _P, C.c_int32, _P, _P, _P, C.c_float,
                                          _P, _P, _P, _P, C.c_size_t, C.c_int32, _P]
 _lib.moeq_static_workspace_capacity.restype = C.c_size_t
@@ -205,3 +217,36 @@ def moeq_device_status(stream=None) -> int:
     v = C.c_int32(0)
     _check("moeq_device_status", _lib.moeq_device_status(_stream(stream), C.byref(v)))
     return int(v.value)
+
+
+class ExpertCache:
+    """moeq_expert_cache: routed expert banks in host memory, `slots` of
+    them cached in HBM (see include/moeq.h).  Keeps the layer descriptor
+    alive; frees the cache on close()."""
+
+    def __init__(self, L: Layer, slots: int, max_tokens: int):
+        self._L = L
+        self._h = C.c_void_p()
+        _check("moeq_cache_create", _lib.moeq_cache_create(C.byref(L), slots, max_tokens,
+                                                           C.byref(self._h)))
+
+    def workspace_bytes(self, M: int) -> int:
+        return int(_lib.moeq_cache_workspace_bytes(self._h, M))
+
+    def forward(self, x, M: int, y, ws, ws_bytes: int, residual=None, idx_out=None, w_out=None,
+                stream=None) -> None:
+        _check("moeq_cache_forward",
+               _lib.moeq_cache_forward(self._h, _ptr(x), M, _ptr(y), _ptr(residual),
+                                       _ptr(idx_out), _ptr(w_out), _ptr(ws), ws_bytes,
+                                       _stream(stream)))
+
+    def stats(self):
+        h, m, b = C.c_uint64(), C.c_uint64(), C.c_uint64()
+        _check("moeq_cache_stats", _lib.moeq_cache_stats(self._h, C.byref(h), C.byref(m),
+                                                         C.byref(b)))
+        return int(h.value), int(m.value), int(b.value)
+
+    def close(self) -> None:
+        if self._h:
+            _lib.moeq_cache_destroy(self._h)
+            self._h = C.c_void_p()

@@ -183,3 +183,21 @@ def test_norm_entry_argument_checks():
     assert call(gamma=A + 2) == moeq.ERR_ALIGNMENT
     assert call(y_norm=A + 8) == moeq.ERR_ALIGNMENT
     assert call(M=0, gamma=0) == moeq.OK
+
+
+def test_cache_create_argument_checks():
+    """moeq_cache_create refuses before touching the device: a missing
+    layer or output, slots outside [K, E], too many tokens for the slots."""
+    f = moeq.lib().moeq_cache_create
+    L = layer(E=8, K=2)
+    h = C.c_void_p()
+    assert f(None, 4, 1, C.byref(h)) == moeq.ERR_INVALID_ARG
+    assert f(C.byref(L), 4, 1, None) == moeq.ERR_INVALID_ARG
+    assert f(C.byref(L), 1, 1, C.byref(h)) == moeq.ERR_INVALID_ARG     # slots < K
+    assert f(C.byref(L), 9, 1, C.byref(h)) == moeq.ERR_INVALID_ARG     # slots > E
+    assert f(C.byref(L), 4, 3, C.byref(h)) == moeq.ERR_INVALID_ARG     # 3 tokens x 2 > 4 slots
+    assert f(C.byref(L), 4, 65, C.byref(h)) == moeq.ERR_INVALID_ARG
+    bad = layer(E=8, K=2)
+    bad.n_experts = 4
+    assert f(C.byref(bad), 4, 1, C.byref(h)) == moeq.ERR_UNSUPPORTED
+    assert not h.value
