@@ -57,7 +57,8 @@ typedef enum {
 } moeq_status;
 
 typedef enum {
-  MOEQ_MODE_AUTO = 0,    /* decode while M*K <= 96 (and M <= 64), prefill beyond */
+  MOEQ_MODE_AUTO = 0,    /* decode while M*K <= 96 (and M <= 64), prefill beyond
+                            (decode up to M = 64 for layers prefill cannot take) */
   MOEQ_MODE_DECODE = 1,  /* HBM-bound split-K quantised matvec path */
   MOEQ_MODE_PREFILL = 2  /* sort-by-expert gather-QMM on tcgen05 tensor cores */
 } moeq_mode;
@@ -83,7 +84,9 @@ typedef struct {
   const uint16_t* biases;   /* bf16 bits, same shape as scales (MXFP4: unused) */
   int32_t out_dim;
   int32_t in_dim;
-  int32_t bits;             /* 2, 4 or 8 (MXFP4: 4) */
+  int32_t bits;             /* 2, 4 or 8; 3 or 6 (decode only): each row one little-endian
+                               bit stream, value i at bits [i*b, (i+1)*b), values may
+                               straddle words, rows of whole 16-byte runs; MXFP4: 4 */
   int32_t group_size;       /* values per group along in_dim: 64 (or 32, 128; MXFP4: 32) */
   int64_t expert_stride_w;  /* words from one expert's matrix to the next (0: single matrix) */
   int64_t expert_stride_sb; /* scale/bias entries from one expert to the next */

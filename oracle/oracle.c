@@ -99,11 +99,17 @@ static float orc_bf16f(uint16_t h) {
  * of a word occupies bits [j*bits, (j+1)*bits) -- low bits first.
  */
 static uint32_t orc_code(const orc_tensor* t, int mat, int64_t r, int64_t c) {
-  const int per_word = 32 / t->bits;
-  const int64_t words_per_row = (int64_t)t->in / per_word;
-  const uint32_t word = t->w[(int64_t)mat * t->stride_w + r * words_per_row + c / per_word];
-  const int j = (int)(c % per_word);
-  return (word >> (t->bits * j)) & ((1u << t->bits) - 1u);
+  /* value c of a row occupies bits [c*bits, (c+1)*bits) of the row's
+   * little-endian stream of u32 words, low bits first; with 3 or 6 bits a
+   * value may straddle two words (cross-word packing) */
+  const int64_t words_per_row = (int64_t)t->in * t->bits / 32;
+  const uint32_t* row = t->w + (int64_t)mat * t->stride_w + r * words_per_row;
+  const int64_t bit = c * t->bits;
+  const int64_t k = bit / 32;
+  const int off = (int)(bit % 32);
+  uint64_t v = row[k] >> off;
+  if (off + t->bits > 32) v |= (uint64_t)row[k + 1] << (32 - off);
+  return (uint32_t)(v & ((1u << t->bits) - 1u));
 }
 
 /* Scale and bias of the group holding value c of row r ([MB-FIX]: groups

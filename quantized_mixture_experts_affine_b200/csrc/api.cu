@@ -67,12 +67,15 @@ static moeq_status check_tensor(const moeq_qtensor* t, int64_t n_mats) {
   const bool mx = is_mx(*t);
   if (!t->w || !t->scales || (!mx && !t->biases)) return MOEQ_ERR_INVALID_ARG;
   if (t->out_dim <= 0 || t->in_dim <= 0 || n_mats <= 0) return MOEQ_ERR_INVALID_ARG;
-  if (t->bits != 2 && t->bits != 4 && t->bits != 8) return MOEQ_ERR_UNSUPPORTED;
+  if (t->bits != 2 && t->bits != 3 && t->bits != 4 && t->bits != 6 && t->bits != 8)
+    return MOEQ_ERR_UNSUPPORTED;
   if (t->group_size != 32 && t->group_size != 64 && t->group_size != 128)
     return MOEQ_ERR_UNSUPPORTED;
   if (mx && (t->bits != 4 || t->group_size != 32)) return MOEQ_ERR_UNSUPPORTED;
-  const int vpc = 128 / t->bits;  // codes per 16-byte chunk
+  const int vpc = chunk_values(t->bits);  // codes per chunk (16 bytes; 3, 6 bits: 32 codes)
   if (t->in_dim % t->group_size || t->in_dim % vpc) return MOEQ_ERR_ALIGNMENT;
+  // rows of whole 16-byte runs (3 bits: in_dim % 128, 6 bits: % 64)
+  if (((int64_t)t->in_dim * t->bits / 8) % 16) return MOEQ_ERR_ALIGNMENT;
   if (!aligned(t->w, 16) || (!mx && (!aligned(t->scales, 2) || !aligned(t->biases, 2))))
     return MOEQ_ERR_ALIGNMENT;
   const int64_t words = (int64_t)t->out_dim * t->in_dim * t->bits / 32;
@@ -86,7 +89,7 @@ static moeq_status check_tensor(const moeq_qtensor* t, int64_t n_mats) {
 
 // Decode GEMV limit: a row is cut into at most 8 slices of 512 bytes.
 static int slices_of(const moeq_qtensor& t) {
-  const int cpr = t.in_dim / (128 / t.bits);
+  const int cpr = t.in_dim / chunk_values(t.bits);
   return (cpr + 31) / 32;
 }
 
@@ -208,10 +211,14 @@ DecodeWs decode_ws(const moeq_layer* L, int M) {
 // times faster on all four.
 constexpr int kAutoDecodePairs = 96;
 
-static int resolve_mode(int mode, int M, int K) {
-  if (mode == MOEQ_MODE_AUTO)
-    return M <= kMaxDecodeM && (int64_t)M * K <= kAutoDecodePairs ? MOEQ_MODE_DECODE
-                                                                   : MOEQ_MODE_PREFILL;
+// (A layer the prefill path cannot take -- 3- or 6-bit codes -- stays on
+// the decode path whenever M allows.)
+static int resolve_mode(int mode, int M, const moeq_layer* L) {
+  if (mode == MOEQ_MODE_AUTO) {
+    if (M <= kMaxDecodeM && (int64_t)M * L->top_k <= kAutoDecodePairs) return MOEQ_MODE_DECODE;
+    if (M <= kMaxDecodeM && prefill_workspace_bytes(L, M) == 0) return MOEQ_MODE_DECODE;
+    return MOEQ_MODE_PREFILL;
+  }
   return mode;
 }
 
@@ -626,7 +633,7 @@ MOEQ_API moeq_status moeq_route_topk(const float* logits, int32_t M, int32_t E, 
 
 MOEQ_API size_t moeq_workspace_bytes(const moeq_layer* L, int32_t M, int32_t mode) {
   if (check_layer(L) != MOEQ_OK || M <= 0) return 0;
-  mode = resolve_mode(mode, M, L->top_k);
+  mode = resolve_mode(mode, M, L);
   if (mode == MOEQ_MODE_DECODE) {
     if (M > kMaxDecodeM) return 0;
     return decode_ws(L, M).total;
@@ -659,7 +666,7 @@ static moeq_status forward_common(const moeq_layer* L, const uint16_t* x, int32_
                                   const NormOut* norm = nullptr) {
   moeq_status s = forward_arg_check(L, x, M, y, residual, mode);
   if (s != MOEQ_OK || M == 0) return s;
-  mode = resolve_mode(mode, M, L->top_k);
+  mode = resolve_mode(mode, M, L);
   const size_t need = moeq_workspace_bytes(L, M, mode);
   if (need == 0) return MOEQ_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < need) return MOEQ_ERR_WORKSPACE;

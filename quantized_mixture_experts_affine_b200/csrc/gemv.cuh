@@ -210,6 +210,18 @@ __device__ __forceinline__ uint4 gq_lds128(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t lds32_gv(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds64_gv(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
   uint16_t v;
   asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));

@@ -9,7 +9,7 @@ namespace moeq {
 
 GemvShape gemv_shape(int in_dim, int bits, int nmat, int G) {
   GemvShape sh;
-  const int cpr = in_dim / (128 / bits);
+  const int cpr = in_dim / chunk_values(bits);
   sh.S = (cpr + 31) / 32;
   sh.J = sh.S >= 8 ? 1 : 8 / sh.S;
   // fewer row subsets when a unit would not fit one stage
@@ -682,9 +682,24 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
               const int row = j * RPW + i;
               const bool ok = lane_on && row < nrows;
               uint4 wv = make_uint4(0, 0, 0, 0);
+              constexpr bool STREAM = BITS == 3 || BITS == 6;  // cross-word packed codes
+              uint32_t ws3[STREAM ? Chunk<BITS>::BYTES / 4 : 1] = {};
               float s2[2] = {0.f, 0.f}, b2[2] = {0.f, 0.f};
               if (ok) {
-                wv = gq_lds128(st + (m * RU + row) * row_bytes + ch * 16);
+                const uint32_t ca = st + (m * RU + row) * row_bytes + ch * Chunk<BITS>::BYTES;
+                if constexpr (BITS == 3) {
+#pragma unroll
+                  for (int q = 0; q < 3; ++q) ws3[q] = lds32_gv(ca + 4 * q);
+                } else if constexpr (BITS == 6) {
+#pragma unroll
+                  for (int q = 0; q < 3; ++q) {
+                    const uint2 v = lds64_gv(ca + 8 * q);
+                    ws3[2 * q] = v.x;
+                    ws3[2 * q + 1] = v.y;
+                  }
+                } else {
+                  wv = gq_lds128(ca);
+                }
                 if (MX) {
                   // one group per 32-value chunk: s = 2^(e - 128), b = -12 s
                   const uint32_t e = lds_u8(st + codes_bytes + m * sb_bytes + row * gpr + gi[0]);
@@ -701,7 +716,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
                 }
               }
               uint32_t c[NC];
-              Chunk<BITS>::split(wv, c);
+              if constexpr (BITS == 3 || BITS == 6) Chunk<BITS>::split_stream(ws3, c);
+              else Chunk<BITS>::split(wv, c);
               if (MX) {
 #pragma unroll
                 for (int k = 0; k < NC; ++k) c[k] = mx_q8(c[k]);
@@ -799,6 +815,18 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
 cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,
                         cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
+  if (bits == 3 || bits == 6) {  // cross-word packed codes
+    if (nmat == 2 && nl == 2 && src == SRC_BF16)
+      return bits == 3 ? launch_one<3, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st)
+                       : launch_one<6, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st);
+    if (nmat == 1 && nl == 3 && src == SRC_BF16)
+      return bits == 3 ? launch_one<3, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st)
+                       : launch_one<6, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st);
+    if (nmat == 1 && nl == 2 && src == SRC_F32)
+      return bits == 3 ? launch_one<3, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st)
+                       : launch_one<6, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st);
+    return cudaErrorInvalidValue;
+  }
   if (a.fmt == MOEQ_FMT_MXFP4) {  // 4-bit E2M1 experts (and qmv)
     if (bits != 4) return cudaErrorInvalidValue;
     if (nmat == 2 && nl == 2 && src == SRC_BF16)

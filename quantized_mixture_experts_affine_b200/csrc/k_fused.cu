@@ -1021,13 +1021,14 @@ bool fused_decode_plan(const moeq_layer* L, int grid, bool route_from_router, Fu
     if (BS != 4 && BS != BE) return false;
     if (L->sh_expert_gate.bits != BR) return false;
   }
-  // every tensor: groups of 64, whole 32-value blocks, at most 8 groups per
-  // compute warp
+  // every tensor: affine, groups of 64, whole 32-value blocks, at most 8
+  // groups per compute warp
   const moeq_qtensor* all[8] = {&R, &Gt, &L->up, &D, &L->sh_gate, &L->sh_up, &L->sh_down,
                                 &L->sh_expert_gate};
   const int n_all = L->has_shared ? 8 : 4;
   for (int i = 0; i < n_all; ++i) {
     const moeq_qtensor& t = *all[i];
+    if (t.format != MOEQ_FMT_AFFINE) return false;  // bf16 scale and bias per group only
     if (t.group_size != FZ_G || t.in_dim % FZ_G || t.in_dim / FZ_G > 8 * FZ_CW) return false;
   }
   memset(&a, 0, sizeof(a));

@@ -35,6 +35,40 @@ __global__ void __launch_bounds__(256) k_dequant(const uint32_t* __restrict__ w,
   }
 }
 
+// 3- and 6-bit codes (a row is one little-endian bit stream): one thread per
+// 32-value chunk of 12 or 24 bytes, spread to bytes as the decode GEMV does.
+template <int BITS>
+__global__ void __launch_bounds__(256) k_dequant_stream(const uint32_t* __restrict__ w,
+                                                        const uint16_t* __restrict__ sc,
+                                                        const uint16_t* __restrict__ bi,
+                                                        int out_dim, int in_dim, int G,
+                                                        uint8_t* __restrict__ q_out,
+                                                        float* __restrict__ w_out) {
+  constexpr int CW = Chunk<BITS>::BYTES / 4;  // words per 32-value chunk
+  const int64_t cpr = in_dim / 32;
+  const int64_t total = (int64_t)out_dim * cpr;
+  const int gpr = in_dim / G;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / cpr;
+    const int64_t c0 = (i % cpr) * 32;
+    uint32_t ws[CW];
+#pragma unroll
+    for (int k = 0; k < CW; ++k) ws[k] = w[i * CW + k];
+    uint32_t c[8];
+    Chunk<BITS>::split_stream(ws, c);
+    const int g = (int)(c0 / G);  // G >= 32: one group per chunk
+    const float s = bf16_bits_to_float(sc[r * gpr + g]);
+    const float b = bf16_bits_to_float(bi[r * gpr + g]);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t q = (c[j / 4] >> (8 * (j % 4))) & 255u;
+      if (q_out) q_out[r * in_dim + c0 + j] = (uint8_t)q;
+      if (w_out) w_out[r * in_dim + c0 + j] = __fmaf_rn((float)q, s, b);
+    }
+  }
+}
+
 // MX FP4: w = e2m1(q) * 2^(e - 127), exact in fp32 (q' * 2^(e - 128) with
 // q' = 2 e2m1(q) + 12, minus 12 * 2^(e - 128)).
 __global__ void __launch_bounds__(256) k_dequant_mx(const uint32_t* __restrict__ w,
@@ -81,6 +115,16 @@ cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, fl
   int64_t grid = (total + 255) / 256;
   if (grid > 148 * 32) grid = 148 * 32;
   if (grid == 0) return cudaSuccess;
+  if (t.bits == 3 || t.bits == 6) {
+    const int64_t chunks = (int64_t)t.out_dim * t.in_dim / 32;
+    int64_t g2 = (chunks + 255) / 256;
+    if (g2 > 148 * 32) g2 = 148 * 32;
+    if (t.bits == 3)
+      k_dequant_stream<3><<<(int)g2, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out);
+    else
+      k_dequant_stream<6><<<(int)g2, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out);
+    return cudaGetLastError();
+  }
   switch (t.bits) {
     case 2: k_dequant<2><<<(int)grid, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out); break;
     case 4: k_dequant<4><<<(int)grid, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out); break;

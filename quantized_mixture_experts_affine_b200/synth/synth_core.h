@@ -146,13 +146,15 @@ SYN_HD void syn_make_group(uint64_t key, int64_t row, int in_dim, int g, int G,
     for (int i = 0; i < G; ++i) w[i] = syn_dequant_f32(q[i], s4, b4);
   }
   syn_quantise_group(w, G, bits, q, scale_out, bias_out);
-  const int per_word = 32 / bits;
-  const int w0 = g * G / per_word;
-  for (int k = 0; k < G / per_word; ++k) {
-    uint32_t word = 0;
-    for (int j = 0; j < per_word; ++j)
-      word |= ((uint32_t)q[k * per_word + j]) << (bits * j);
-    words_row[w0 + k] = word;
+  /* value j of the group at bit (g*G + j)*bits of the row's stream, low bits
+   * first (3 and 6 bits: a value may straddle two words); a group fills
+   * whole words for every G in {32, 64, 128} */
+  const int w0 = g * G * bits / 32, nw = G * bits / 32;
+  for (int k = 0; k < nw; ++k) words_row[w0 + k] = 0;
+  for (int j = 0; j < G; ++j) {
+    const int bit = j * bits, k = bit / 32, off = bit % 32;
+    words_row[w0 + k] |= (uint32_t)q[j] << off;
+    if (off + bits > 32) words_row[w0 + k + 1] |= (uint32_t)q[j] >> (32 - off);
   }
 }
 

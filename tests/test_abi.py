@@ -45,7 +45,9 @@ def rc_qmv(t, M=1, x=A, y=A, expert=0):
 
 
 def test_qmv_argument_checks():
-    assert rc_qmv(qt(bits=3)) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(bits=5)) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(bits=3, inn=192)) == moeq.ERR_ALIGNMENT      # 3-bit rows: in_dim % 128
+    assert rc_qmv(qt(bits=6, inn=96, G=32)) == moeq.ERR_ALIGNMENT  # 6-bit rows: in_dim % 64
     assert rc_qmv(qt(G=48)) == moeq.ERR_UNSUPPORTED
     assert rc_qmv(qt(inn=96, G=64)) == moeq.ERR_ALIGNMENT
     assert rc_qmv(qt(w=A + 4)) == moeq.ERR_ALIGNMENT

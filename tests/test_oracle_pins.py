@@ -30,22 +30,32 @@ def f32_of_bf16(h):
 
 
 def pack(codes, bits):
-    """codes [out][in] (ints) -> u32 words [out][in*bits/32], value j at bits j*b."""
-    codes = np.asarray(codes, np.uint64)
-    per = 32 // bits
+    """codes [out][in] (ints) -> u32 words [out][in*bits/32]: value j of a
+    row at bits [j*b, (j+1)*b) of the row as one little-endian integer (for
+    3 and 6 bits values straddle words), built with Python big integers."""
+    codes = np.asarray(codes, np.int64)
     out, n = codes.shape
-    words = np.zeros((out, n // per), np.uint64)
-    for j in range(per):
-        words |= codes[:, j::per] << np.uint64(bits * j)
-    return words.astype(np.uint32)
+    nw = n * bits // 32
+    words = np.zeros((out, nw), np.uint32)
+    for r in range(out):
+        big = 0
+        for j in range(n):
+            big |= int(codes[r, j]) << (j * bits)
+        for k in range(nw):
+            words[r, k] = (big >> (32 * k)) & 0xFFFFFFFF
+    return words
 
 
 def unpack_np(words, bits, in_dim):
-    per = 32 // bits
-    words = np.asarray(words, np.uint64).reshape(-1, in_dim // per)
+    """Inverse of pack, by Python big integers (independent of the oracle)."""
+    words = np.asarray(words, np.uint32).reshape(-1, in_dim * bits // 32)
     out = np.zeros((words.shape[0], in_dim), np.int64)
-    for j in range(per):
-        out[:, j::per] = (words >> np.uint64(bits * j)) & np.uint64((1 << bits) - 1)
+    for r in range(words.shape[0]):
+        big = 0
+        for k, wv in enumerate(words[r]):
+            big |= int(wv) << (32 * k)
+        for j in range(in_dim):
+            out[r, j] = (big >> (j * bits)) & ((1 << bits) - 1)
     return out
 
 
@@ -109,7 +119,7 @@ def test_words_unpack_low_bits_first(golden):
         assert not q[0, per:].any()
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
 def test_unpack_matches_independent_extraction(bits):
     rng = np.random.default_rng(bits)
     codes = rng.integers(0, 1 << bits, size=(7, 256))
@@ -120,7 +130,7 @@ def test_unpack_matches_independent_extraction(bits):
 
 # ---------------------------------------------------------------- dequant
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
 def test_dequant_endpoints_bit_exact(bits):
     """q = 0 -> bias and q = 2^b-1 -> bias + (2^b-1)*scale, exactly in fp32."""
     rng = np.random.default_rng(10 + bits)
@@ -144,7 +154,8 @@ def test_dequant_matches_single_rounding_everywhere():
     assert np.array_equal(w, dense_f64(q).astype(np.float32))
 
 
-@pytest.mark.parametrize("bits,G", [(2, 64), (4, 64), (8, 64), (4, 32), (8, 128)])
+@pytest.mark.parametrize("bits,G", [(2, 64), (4, 64), (8, 64), (4, 32), (8, 128), (3, 64),
+                                    (6, 32), (3, 128)])
 def test_quantiser_reconstruction_pins_format(bits, G):
     """Generator and oracle agree on the format: dequantised codes sit within
     half a quantisation step of the fp32 draws (a wrong bit order or group
@@ -178,7 +189,8 @@ def test_requantised_2bit_reconstruction():
 # ---------------------------------------------------------------- qmv
 
 @pytest.mark.parametrize("bits,G,out,inn", [(4, 64, 40, 256), (8, 64, 17, 320), (2, 64, 33, 128),
-                                            (4, 32, 9, 96), (8, 128, 5, 384)])
+                                            (4, 32, 9, 96), (8, 128, 5, 384), (3, 64, 11, 256),
+                                            (6, 32, 7, 192), (3, 32, 5, 96)])
 def test_qmv_equals_bruteforce_dense(bits, G, out, inn):
     tg = synth.tag(synth.ROUTER, bits)
     q = synth.tensor_host(11, tg, 2, out, inn, bits, G)
@@ -532,3 +544,21 @@ def test_mxfp4_generator_round_trip():
     assert (np.abs(deq - w32) <= (step / 2 + over) * scale + 1e-12).all()
     amax = np.abs(deq).reshape(O, H // 32, 32).max(axis=2) / scale[:, ::32]
     assert ((amax >= 4.0) & (amax <= 6.0)).all()
+
+
+
+def test_cross_word_packing_by_hand():
+    """3 bits: 32 values in 3 words, value 10 straddling words 0 and 1 (bits
+    30..32) and value 21 words 1 and 2 (bits 63..65); 6 bits: value 5 at bits
+    30..35 straddles words 0 and 1."""
+    codes = np.zeros((1, 32), np.int64)
+    codes[0, 10] = 0b110      # bits 30, 31 = 0, 1 ; bit 32 = 1
+    codes[0, 21] = 0b011      # bit 63 = 1 ; bits 64, 65 = 1, 0
+    t = T(codes, BF16_ONE, 0, 3, 32)
+    assert t.w.tolist() == [[0x80000000, 0x80000001, 0x00000001]]
+    assert np.array_equal(oracle.unpack(t), codes)
+    c6 = np.zeros((1, 32), np.int64)
+    c6[0, 5] = 0b101101       # bits 30, 31 = 1, 0 ; bits 32..35 = 1, 1, 0, 1
+    t6 = T(c6, BF16_ONE, 0, 6, 32)
+    assert t6.w[0, 0] == 0x40000000 and t6.w[0, 1] == 0x0000000B
+    assert np.array_equal(oracle.unpack(t6), c6)
