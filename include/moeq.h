@@ -10,6 +10,11 @@
  *     q, b in {2, 4, 8}, packed 32/b per uint32 word, row-major
  *     ([out_dim][in_dim*b/32] words); value j of a word sits in bits
  *     [j*b, (j+1)*b) (low bits first);
+ *   - b in {3, 5, 6} (the mlx issue page's table runs an affine 5-bit
+ *     model): each row is one little-endian bit stream of u32 words, value
+ *     i at bits [i*b, (i+1)*b), so a value may straddle two words -- the
+ *     same rule, extended to widths that do not divide 32; decode path
+ *     only;
  *   - each row is cut into groups of group_size consecutive inputs
  *     (64 on the pages; 32 and 128 are also accepted) and each group has
  *     one bf16 scale and one bf16 bias, [out_dim][in_dim/group_size] each;
@@ -48,7 +53,8 @@ extern "C" {
 typedef enum {
   MOEQ_OK = 0,
   MOEQ_ERR_INVALID_ARG = 1,  /* null pointer, size <= 0, K > E, index out of range ... */
-  MOEQ_ERR_UNSUPPORTED = 2,  /* bits not in {2,4,8}, group size not in {32,64,128}, sizes beyond limits */
+  MOEQ_ERR_UNSUPPORTED = 2,  /* bits not in {2,3,4,5,6,8} (prefill: {2,4,8}), group size not in
+                                {32,64,128}, sizes beyond limits */
   MOEQ_ERR_ALIGNMENT = 3,    /* pointer not 16-byte aligned, in_dim not a multiple of group_size */
   MOEQ_ERR_WORKSPACE = 4,    /* workspace missing or smaller than moeq_workspace_bytes */
   MOEQ_ERR_CUDA = 5,         /* a CUDA runtime call failed */
@@ -84,7 +90,7 @@ typedef struct {
   const uint16_t* biases;   /* bf16 bits, same shape as scales (MXFP4: unused) */
   int32_t out_dim;
   int32_t in_dim;
-  int32_t bits;             /* 2, 4 or 8; 3 or 6 (decode only): each row one little-endian
+  int32_t bits;             /* 2, 4 or 8; 3, 5 or 6 (decode only): each row one little-endian
                                bit stream, value i at bits [i*b, (i+1)*b), values may
                                straddle words, rows of whole 16-byte runs; MXFP4: 4 */
   int32_t group_size;       /* values per group along in_dim: 64 (or 32, 128; MXFP4: 32) */

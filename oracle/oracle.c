@@ -100,7 +100,7 @@ static float orc_bf16f(uint16_t h) {
  */
 static uint32_t orc_code(const orc_tensor* t, int mat, int64_t r, int64_t c) {
   /* value c of a row occupies bits [c*bits, (c+1)*bits) of the row's
-   * little-endian stream of u32 words, low bits first; with 3 or 6 bits a
+   * little-endian stream of u32 words, low bits first; with 3, 5 or 6 bits a
    * value may straddle two words (cross-word packing) */
   const int64_t words_per_row = (int64_t)t->in * t->bits / 32;
   const uint32_t* row = t->w + (int64_t)mat * t->stride_w + r * words_per_row;

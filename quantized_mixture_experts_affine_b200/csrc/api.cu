@@ -67,14 +67,14 @@ static moeq_status check_tensor(const moeq_qtensor* t, int64_t n_mats) {
   const bool mx = is_mx(*t);
   if (!t->w || !t->scales || (!mx && !t->biases)) return MOEQ_ERR_INVALID_ARG;
   if (t->out_dim <= 0 || t->in_dim <= 0 || n_mats <= 0) return MOEQ_ERR_INVALID_ARG;
-  if (t->bits != 2 && t->bits != 3 && t->bits != 4 && t->bits != 6 && t->bits != 8)
+  if (t->bits < 2 || t->bits > 8 || t->bits == 7)
     return MOEQ_ERR_UNSUPPORTED;
   if (t->group_size != 32 && t->group_size != 64 && t->group_size != 128)
     return MOEQ_ERR_UNSUPPORTED;
   if (mx && (t->bits != 4 || t->group_size != 32)) return MOEQ_ERR_UNSUPPORTED;
-  const int vpc = chunk_values(t->bits);  // codes per chunk (16 bytes; 3, 6 bits: 32 codes)
+  const int vpc = chunk_values(t->bits);  // codes per chunk (16 bytes; 3, 5, 6 bits: 32 codes)
   if (t->in_dim % t->group_size || t->in_dim % vpc) return MOEQ_ERR_ALIGNMENT;
-  // rows of whole 16-byte runs (3 bits: in_dim % 128, 6 bits: % 64)
+  // rows of whole 16-byte runs (3 and 5 bits: in_dim % 128, 6 bits: % 64)
   if (((int64_t)t->in_dim * t->bits / 8) % 16) return MOEQ_ERR_ALIGNMENT;
   if (!aligned(t->w, 16) || (!mx && (!aligned(t->scales, 2) || !aligned(t->biases, 2))))
     return MOEQ_ERR_ALIGNMENT;
@@ -211,7 +211,7 @@ DecodeWs decode_ws(const moeq_layer* L, int M) {
 // times faster on all four.
 constexpr int kAutoDecodePairs = 96;
 
-// (A layer the prefill path cannot take -- 3- or 6-bit codes -- stays on
+// (A layer the prefill path cannot take -- 3-, 5- or 6-bit codes -- stays on
 // the decode path whenever M allows.)
 static int resolve_mode(int mode, int M, const moeq_layer* L) {
   if (mode == MOEQ_MODE_AUTO) {

@@ -121,21 +121,24 @@ __device__ __forceinline__ float mx_scale(uint32_t e) {
 //           reg 2k+1   = (word k >> 4) & 0x0F0F0F0F  (values 8k + 1,3,5,7)
 //   BITS 2: reg 4k+i   = (word k >> 2i) & 0x03030303 (values 16k + i + 0,4,8,12)
 // value_of(BITS, reg, byte) gives the position of a code within the chunk.
-// BITS 3, 6 (cross-word packing): a chunk is 32 values, 12 or 24 bytes of
-// the row's bit stream, spread to one code per byte in value order
+// BITS 3, 5, 6 (cross-word packing): a chunk is 32 values, 12, 20 or 24
+// bytes of the row's bit stream, spread to one code per byte in value order
 //   reg k = values 4k .. 4k+3.
+__host__ __device__ constexpr bool stream_bits(int bits) {
+  return bits == 3 || bits == 5 || bits == 6;
+}
 __host__ __device__ constexpr int chunk_values(int bits) {
-  return bits == 3 || bits == 6 ? 32 : 128 / bits;
+  return stream_bits(bits) ? 32 : 128 / bits;
 }
 
 template <int BITS>
 struct Chunk {
   static constexpr int VPC = chunk_values(BITS);  // values per chunk
-  static constexpr int BYTES = VPC * BITS / 8;     // 16; 12 (3-bit) or 24 (6-bit)
+  static constexpr int BYTES = VPC * BITS / 8;     // 16; 12, 20 or 24 (3, 5, 6 bits)
   static constexpr int NC = VPC / 4;      // code registers per chunk
   static constexpr int NBLK = VPC >= kXBlock ? VPC / kXBlock : 1;  // x blocks touched
   __host__ __device__ static constexpr int value_of(int reg, int byte) {
-    return BITS == 8 || BITS == 3 || BITS == 6 ? reg * 4 + byte
+    return BITS == 8 || stream_bits(BITS) ? reg * 4 + byte
          : BITS == 4 ? (reg >> 1) * 8 + (reg & 1) + 2 * byte
                      : (reg >> 2) * 16 + (reg & 3) + 4 * byte;
   }
@@ -143,9 +146,11 @@ struct Chunk {
   __device__ __forceinline__ static uint32_t spread4(uint32_t v) {
     if (BITS == 3)
       return (v & 0x7u) | ((v & 0x38u) << 5) | ((v & 0x1C0u) << 10) | ((v & 0xE00u) << 15);
+    if (BITS == 5)
+      return (v & 0x1Fu) | ((v & 0x3E0u) << 3) | ((v & 0x7C00u) << 6) | ((v & 0xF8000u) << 9);
     return (v & 0x3Fu) | ((v & 0xFC0u) << 2) | ((v & 0x3F000u) << 4) | ((v & 0xFC0000u) << 6);
   }
-  // The chunk of 3- or 6-bit codes in words w[0 .. BYTES/4) as NC registers.
+  // The chunk of 3-, 5- or 6-bit codes in words w[0 .. BYTES/4) as NC registers.
   __device__ __forceinline__ static void split_stream(const uint32_t* w, uint32_t (&c)[NC]) {
     constexpr int GB = 4 * BITS;  // bits of four values
 #pragma unroll

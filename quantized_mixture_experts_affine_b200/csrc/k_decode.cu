@@ -682,15 +682,15 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
               const int row = j * RPW + i;
               const bool ok = lane_on && row < nrows;
               uint4 wv = make_uint4(0, 0, 0, 0);
-              constexpr bool STREAM = BITS == 3 || BITS == 6;  // cross-word packed codes
+              constexpr bool STREAM = stream_bits(BITS);  // cross-word packed codes
               uint32_t ws3[STREAM ? Chunk<BITS>::BYTES / 4 : 1] = {};
               float s2[2] = {0.f, 0.f}, b2[2] = {0.f, 0.f};
               if (ok) {
                 const uint32_t ca = st + (m * RU + row) * row_bytes + ch * Chunk<BITS>::BYTES;
-                if constexpr (BITS == 3) {
+                if constexpr (BITS == 3 || BITS == 5) {  // 4-byte aligned runs
 #pragma unroll
-                  for (int q = 0; q < 3; ++q) ws3[q] = lds32_gv(ca + 4 * q);
-                } else if constexpr (BITS == 6) {
+                  for (int q = 0; q < Chunk<BITS>::BYTES / 4; ++q) ws3[q] = lds32_gv(ca + 4 * q);
+                } else if constexpr (BITS == 6) {  // 8-byte aligned runs
 #pragma unroll
                   for (int q = 0; q < 3; ++q) {
                     const uint2 v = lds64_gv(ca + 8 * q);
@@ -716,7 +716,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
                 }
               }
               uint32_t c[NC];
-              if constexpr (BITS == 3 || BITS == 6) Chunk<BITS>::split_stream(ws3, c);
+              if constexpr (STREAM) Chunk<BITS>::split_stream(ws3, c);
               else Chunk<BITS>::split(wv, c);
               if (MX) {
 #pragma unroll
@@ -815,15 +815,18 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
 cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,
                         cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
-  if (bits == 3 || bits == 6) {  // cross-word packed codes
+  if (stream_bits(bits)) {  // cross-word packed codes
     if (nmat == 2 && nl == 2 && src == SRC_BF16)
       return bits == 3 ? launch_one<3, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st)
+           : bits == 5 ? launch_one<5, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st)
                        : launch_one<6, 2, 2, SRC_BF16, EPI_SWIGLU>(a, grid, st);
     if (nmat == 1 && nl == 3 && src == SRC_BF16)
       return bits == 3 ? launch_one<3, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st)
+           : bits == 5 ? launch_one<5, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st)
                        : launch_one<6, 3, 1, SRC_BF16, EPI_PLAIN>(a, grid, st);
     if (nmat == 1 && nl == 2 && src == SRC_F32)
       return bits == 3 ? launch_one<3, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st)
+           : bits == 5 ? launch_one<5, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st)
                        : launch_one<6, 2, 1, SRC_F32, EPI_PLAIN>(a, grid, st);
     return cudaErrorInvalidValue;
   }

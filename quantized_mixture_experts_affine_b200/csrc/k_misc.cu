@@ -35,8 +35,9 @@ __global__ void __launch_bounds__(256) k_dequant(const uint32_t* __restrict__ w,
   }
 }
 
-// 3- and 6-bit codes (a row is one little-endian bit stream): one thread per
-// 32-value chunk of 12 or 24 bytes, spread to bytes as the decode GEMV does.
+// 3-, 5- and 6-bit codes (a row is one little-endian bit stream): one thread
+// per 32-value chunk of 12, 20 or 24 bytes, spread to bytes as the decode
+// GEMV does.
 template <int BITS>
 __global__ void __launch_bounds__(256) k_dequant_stream(const uint32_t* __restrict__ w,
                                                         const uint16_t* __restrict__ sc,
@@ -115,12 +116,14 @@ cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, fl
   int64_t grid = (total + 255) / 256;
   if (grid > 148 * 32) grid = 148 * 32;
   if (grid == 0) return cudaSuccess;
-  if (t.bits == 3 || t.bits == 6) {
+  if (stream_bits(t.bits)) {
     const int64_t chunks = (int64_t)t.out_dim * t.in_dim / 32;
     int64_t g2 = (chunks + 255) / 256;
     if (g2 > 148 * 32) g2 = 148 * 32;
     if (t.bits == 3)
       k_dequant_stream<3><<<(int)g2, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out);
+    else if (t.bits == 5)
+      k_dequant_stream<5><<<(int)g2, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out);
     else
       k_dequant_stream<6><<<(int)g2, 256, 0, st>>>(w, s, b, t.out_dim, t.in_dim, t.group_size, q_out, w_out);
     return cudaGetLastError();

@@ -686,7 +686,7 @@ moeq_status check_prefill(const moeq_layer* L) {
     const int G = ts[i]->group_size;
     if (G != 32 && G != 64 && G != 128) return MOEQ_ERR_UNSUPPORTED;
     if (G == 32 && ts[i]->bits == 2) return MOEQ_ERR_UNSUPPORTED;
-    if (ts[i]->bits == 3 || ts[i]->bits == 6) return MOEQ_ERR_UNSUPPORTED;  // decode only
+    if (stream_bits(ts[i]->bits)) return MOEQ_ERR_UNSUPPORTED;  // decode only
     if (ts[i]->format == MOEQ_FMT_AFFINE &&
         (((uintptr_t)ts[i]->scales & 3) || ((uintptr_t)ts[i]->biases & 3)))
       return MOEQ_ERR_ALIGNMENT;

@@ -21,7 +21,7 @@
 
 static int syn_check_shape(int n_mats, int out_dim, int in_dim, int bits, int G) {
   if (n_mats <= 0 || out_dim <= 0 || in_dim <= 0) return 1;
-  if (bits != 2 && bits != 3 && bits != 4 && bits != 6 && bits != 8) return 2;
+  if (bits < 2 || bits > 8 || bits == 7) return 2;
   if (G != 32 && G != 64 && G != 128) return 2;
   if (in_dim % G != 0) return 3;
   return 0;

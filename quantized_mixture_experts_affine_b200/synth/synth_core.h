@@ -147,7 +147,7 @@ SYN_HD void syn_make_group(uint64_t key, int64_t row, int in_dim, int g, int G,
   }
   syn_quantise_group(w, G, bits, q, scale_out, bias_out);
   /* value j of the group at bit (g*G + j)*bits of the row's stream, low bits
-   * first (3 and 6 bits: a value may straddle two words); a group fills
+   * first (3, 5 and 6 bits: a value may straddle two words); a group fills
    * whole words for every G in {32, 64, 128} */
   const int w0 = g * G * bits / 32, nw = G * bits / 32;
   for (int k = 0; k < nw; ++k) words_row[w0 + k] = 0;

@@ -45,7 +45,9 @@ def rc_qmv(t, M=1, x=A, y=A, expert=0):
 
 
 def test_qmv_argument_checks():
-    assert rc_qmv(qt(bits=5)) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(bits=7)) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(bits=1)) == moeq.ERR_UNSUPPORTED
+    assert rc_qmv(qt(bits=5, inn=192)) == moeq.ERR_ALIGNMENT      # 5-bit rows: in_dim % 128
     assert rc_qmv(qt(bits=3, inn=192)) == moeq.ERR_ALIGNMENT      # 3-bit rows: in_dim % 128
     assert rc_qmv(qt(bits=6, inn=96, G=32)) == moeq.ERR_ALIGNMENT  # 6-bit rows: in_dim % 64
     assert rc_qmv(qt(G=48)) == moeq.ERR_UNSUPPORTED
@@ -63,7 +65,7 @@ def test_qmv_argument_checks():
 def test_dequant_argument_checks():
     lib = moeq.lib()
     assert lib.moeq_dequant(C.byref(qt()), 0, None, None, None) == moeq.ERR_INVALID_ARG
-    assert lib.moeq_dequant(C.byref(qt(bits=5)), 0, A, None, None) == moeq.ERR_UNSUPPORTED
+    assert lib.moeq_dequant(C.byref(qt(bits=7)), 0, A, None, None) == moeq.ERR_UNSUPPORTED
     # expert > 0 needs expert strides
     assert lib.moeq_dequant(C.byref(qt()), 1, A, None, None) == moeq.ERR_INVALID_ARG
 

@@ -119,7 +119,7 @@ def test_words_unpack_low_bits_first(golden):
         assert not q[0, per:].any()
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
 def test_unpack_matches_independent_extraction(bits):
     rng = np.random.default_rng(bits)
     codes = rng.integers(0, 1 << bits, size=(7, 256))
@@ -130,7 +130,7 @@ def test_unpack_matches_independent_extraction(bits):
 
 # ---------------------------------------------------------------- dequant
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
 def test_dequant_endpoints_bit_exact(bits):
     """q = 0 -> bias and q = 2^b-1 -> bias + (2^b-1)*scale, exactly in fp32."""
     rng = np.random.default_rng(10 + bits)
@@ -155,7 +155,7 @@ def test_dequant_matches_single_rounding_everywhere():
 
 
 @pytest.mark.parametrize("bits,G", [(2, 64), (4, 64), (8, 64), (4, 32), (8, 128), (3, 64),
-                                    (6, 32), (3, 128)])
+                                    (6, 32), (3, 128), (5, 64), (5, 32)])
 def test_quantiser_reconstruction_pins_format(bits, G):
     """Generator and oracle agree on the format: dequantised codes sit within
     half a quantisation step of the fp32 draws (a wrong bit order or group
@@ -550,7 +550,8 @@ def test_mxfp4_generator_round_trip():
 def test_cross_word_packing_by_hand():
     """3 bits: 32 values in 3 words, value 10 straddling words 0 and 1 (bits
     30..32) and value 21 words 1 and 2 (bits 63..65); 6 bits: value 5 at bits
-    30..35 straddles words 0 and 1."""
+    30..35 straddles words 0 and 1; 5 bits: value 6 at bits 30..34 straddles
+    words 0 and 1, value 12 at bits 60..64 words 1 and 2."""
     codes = np.zeros((1, 32), np.int64)
     codes[0, 10] = 0b110      # bits 30, 31 = 0, 1 ; bit 32 = 1
     codes[0, 21] = 0b011      # bit 63 = 1 ; bits 64, 65 = 1, 0
@@ -562,3 +563,9 @@ def test_cross_word_packing_by_hand():
     t6 = T(c6, BF16_ONE, 0, 6, 32)
     assert t6.w[0, 0] == 0x40000000 and t6.w[0, 1] == 0x0000000B
     assert np.array_equal(oracle.unpack(t6), c6)
+    c5 = np.zeros((1, 32), np.int64)
+    c5[0, 6] = 0b10111        # bits 30, 31 = 1, 1 ; bits 32..34 = 1, 0, 1
+    c5[0, 12] = 0b11001       # bits 60..63 = 1, 0, 0, 1 ; bit 64 = 1
+    t5 = T(c5, BF16_ONE, 0, 5, 32)
+    assert t5.w.tolist() == [[0xC0000000, 0x90000005, 0x00000001, 0, 0]]
+    assert np.array_equal(oracle.unpack(t5), c5)

@@ -1,7 +1,7 @@
-"""3- and 6-bit codes (the mlx issue page's affine bit widths that do not
-divide 32: each row is one little-endian bit stream, value i at bits
-[i*b, (i+1)*b), so a value may straddle two 32-bit words) through the C ABI,
-against the oracle.
+"""3-, 5- and 6-bit codes (affine widths that do not divide 32; the mlx
+issue page's table runs an affine 5-bit model): each row is one
+little-endian bit stream, value i at bits [i*b, (i+1)*b), so a value may
+straddle two 32-bit words.  Through the C ABI, against the oracle.
 
 Bars: the device generator's words equal the host generator's; unpacked
 codes and dequantised fp32 weights bit-exact; qmv relative L2 <= 1e-5;
@@ -35,7 +35,9 @@ def dev(a):
 
 @pytest.mark.parametrize("bits,G,inn,rq", [(3, 32, 512, False), (3, 64, 384, False),
                                            (3, 128, 256, True), (6, 32, 192, False),
-                                           (6, 64, 512, True), (6, 128, 640, False)])
+                                           (6, 64, 512, True), (6, 128, 640, False),
+                                           (5, 32, 384, False), (5, 64, 256, True),
+                                           (5, 128, 512, False)])
 def test_generator_and_dequant_bit_exact(bits, G, inn, rq):
     tg = synth.tag(synth.UP, 30 + bits)
     q = synth.tensor_dev(SEED, tg, 3, 72, inn, bits, G, rq)
@@ -65,6 +67,9 @@ QMV_CASES = [  # (bits, G, out, in, M, requant)
     (6, 128, 96, 4096, 2, False),    # 3 KB rows
     (6, 32, 33, 192, 4, False),      # 144-byte rows, 6 chunks
     (6, 64, 2048, 768, 5, True),     # down width
+    (5, 64, 512, 4096, 1, False),    # 20-byte runs, four slices
+    (5, 32, 70, 384, 9, True),       # ragged rows
+    (5, 128, 2048, 1024, 64, False), # max decode M
 ]
 
 
@@ -95,6 +100,7 @@ LAYERS = [
     shape("decode_30b", expert_bits=6, G=32),
     shape("decode_397b", expert_bits=6, shared_bits=3, G=128),
     shape("mixed_2bit", expert_bits=3),   # 4 -> 3 bit requantised experts, 4-bit shared
+    shape("decode_397b", expert_bits=5, shared_bits=5),
 ]
 
 
