@@ -390,6 +390,57 @@ static moeq_status fused_forward(const FusedArgs& shape, const FzMaps& maps, int
   return MOEQ_OK;
 }
 
+// ------------------------------------------------------------------ single-token decode
+// Shape part of the single-token launches' arguments for the last layer
+// seen by this host thread.
+struct SingleCache {
+  bool valid = false, ok = false;
+  moeq_layer L;
+  int sms = 0;
+  S1Args a;
+};
+static thread_local SingleCache t_single;
+
+// MOEQ_SINGLE_DECODE=0 sends single tokens to the general decode launches.
+static bool single_decode_enabled() {
+  const char* e = getenv("MOEQ_SINGLE_DECODE");
+  return !(e && e[0] == '0' && e[1] == 0);
+}
+
+static const S1Args* single_shape(const moeq_layer* L, int sms) {
+  SingleCache& c = t_single;
+  if (!c.valid || c.sms != sms || memcmp(&c.L, L, sizeof(moeq_layer)) != 0) {
+    c.valid = true;
+    c.L = *L;
+    c.sms = sms;
+    c.ok = single_decode_plan(L, sms, c.a);
+  }
+  return c.ok ? &c.a : nullptr;
+}
+
+static moeq_status single_forward(const S1Args& shape, const uint16_t* x, const float* residual,
+                                  float* y, int32_t* idx, float* wts, char* base,
+                                  const DecodeWs& lay, cudaStream_t st) {
+  S1Args a = shape;
+  a.x = x;
+  a.residual = residual;
+  a.y = y;
+  a.logits = (float*)(base + lay.logits);
+  a.sg_logit = (float*)(base + lay.sg_logit);
+  a.idx = idx;
+  a.w = wts;
+  a.sigma = (float*)(base + lay.sigma);
+  a.h = (float*)(base + lay.h);
+  a.status = status_ptr();
+  if (!a.status) return MOEQ_ERR_CUDA;
+  LAUNCH(launch_single_router(a, st));
+  CK(profile_mark(true, st));
+  LAUNCH(launch_single_gateup(a, st));
+  CK(profile_mark(false, st));
+  LAUNCH(launch_single_down(a, st));
+  return MOEQ_OK;
+}
+
 // ------------------------------------------------------------------ decode path
 static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
                                   const int32_t* idx_in, const float* w_in, const float* residual,
@@ -420,6 +471,12 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     if (const FusedArgs* f = fused_shape(L, grid, idx_in == nullptr))
       return fused_forward(*f, t_fused.m, grid, x, idx_in, w_in, residual, y, idx_out, w_out, base,
                            lay, st);
+  }
+  // one token routed by the router: three lean launches when the formats
+  // allow (k_single.cu)
+  if (M == 1 && !idx_in && single_decode_enabled()) {
+    if (const S1Args* a = single_shape(L, grid_cap()))
+      return single_forward(*a, x, residual, y, idx, wts, base, lay, st);
   }
 
   // 1. router logits and the shared-expert gate logit (one launch when the

@@ -1,0 +1,717 @@
+// Single-token decode (M = 1) in three lean launches.
+//
+// The per-layer pipeline of the flash-moe-inference page ("Per-layer
+// pipeline") runs, for one token, the router matvec, the top-K selection,
+// the K experts' gate/up matvecs with SwiGLU, their down matvecs, and the
+// weighted combine with the sigmoid-gated shared expert.  For one token each
+// phase reads a few MB of weights exactly once, so its time is set by how
+// soon all of its loads are in flight, not by arithmetic.  Each launch here:
+//   - splits every matrix it reads into per-CTA blocks of whole rows (codes,
+//     scales and biases in 16-byte runs), and bulk-copies all of a CTA's
+//     blocks into shared memory at once, one mbarrier per matrix;
+//   - issues the blocks that do not depend on the preceding launch (router
+//     rows, the shared expert's rows) before its programmatic-dependency
+//     wait;
+//   - computes rows with the decode engine's arithmetic (gemv.cuh: exact
+//     dp4a sums of the codes with a fixed-point copy of the input, scale and
+//     bias per group), one warp per row; the input's limbs are built once
+//     per CTA into shared memory and then held in registers.
+// The launches:
+//   R  router rows and the shared-expert gate row -> logits;
+//   G  top-K (one warp per CTA, route.cuh's selection), then the shared and
+//      routed gate/up rows with SwiGLU -> h; also pulls into L2 the routed
+//      down rows that D's CTA of the same index reads;
+//   D  the shared and routed down rows of the CTA's output rows, summed
+//      with the routing weights and the shared gate by the warp that owns
+//      the row (no cross-CTA combine), plus the residual -> y.
+#include <atomic>
+#include <cstring>
+
+#include "gemv.cuh"
+#include "kernels.h"
+#include "route.cuh"
+#include "tc.cuh"
+
+namespace moeq {
+
+namespace {
+
+constexpr int kS1Threads = 256;        // R: 8 warps
+constexpr int kS1WideThreads = 512;    // G and D: 16 warps
+constexpr int kS1RowsPerWarp = 4;      // D: output rows per warp
+constexpr int kS1SlotsPerWarp = 2;     // G: input slots per warp
+// G's registers per thread: 512 x 96 leaves room for an R CTA (256 x 48)
+// on the same SM, so G's CTAs start while R runs
+constexpr int kS1GateUpRegs = 96;
+constexpr uint32_t kS1SmemMax = 227 * 1024;
+constexpr int kS1HeadBytes = 512;      // barriers, routing, shared gate value
+
+struct S1Smem {
+  // head: [0, 256) mbarriers; [256, 320) expert ids; [320, 384) weights;
+  // [384] shared gate value
+  static constexpr int IDX_OFF = 256;
+  static constexpr int W_OFF = 320;
+  static constexpr int SIG_OFF = 384;
+};
+
+__host__ __device__ inline uint32_t s1_al(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Rows [lo, hi) of an n-row matrix for CTA c of `grid`, in units of q rows.
+__host__ __device__ inline void s1_rows(int n, int q, int grid, int c, int& lo, int& hi) {
+  const int64_t nu = n / q;
+  lo = (int)((int64_t)c * nu / grid) * q;
+  hi = (int)((int64_t)(c + 1) * nu / grid) * q;
+}
+
+// Shared-memory region of a block of at most `rows` rows of one matrix
+// (codes, then scales and biases, each 16-byte aligned), `nmat` matrices
+// (gate and up: 2) side by side.
+struct S1Blk {
+  uint32_t codes, sc, bi, bytes;  // offsets of matrix 0; matrix 1 follows at +stride
+  uint32_t stride;
+};
+__host__ __device__ inline S1Blk s1_blk(int rows, int row_bytes, int gpr, int nmat) {
+  S1Blk b;
+  const uint32_t cb = (uint32_t)rows * row_bytes;
+  const uint32_t sbb = s1_al((uint32_t)rows * gpr * 2, 16);
+  b.stride = cb + 2 * sbb;
+  b.codes = 0;
+  b.sc = cb;
+  b.bi = cb + sbb;
+  b.bytes = s1_al(b.stride * nmat, 128);
+  return b;
+}
+
+template <int BITS, int NL>
+constexpr int s1_slw() {
+  return NL * Chunk<BITS>::NC + 2 * SliceVec<BITS, NL>::NB;
+}
+
+// Issues the bulk copies of rows [lo, hi) of one packed matrix (expert e)
+// into a block region; returns the bytes.
+__device__ __forceinline__ uint32_t s1_issue(const moeq_qtensor& t, int64_t e, int lo, int hi,
+                                             uint32_t dst_codes, uint32_t dst_s, uint32_t dst_b,
+                                             uint64_t* bar) {
+  const int n = hi - lo;
+  if (n <= 0) return 0;
+  const int rw = t.in_dim * t.bits / 32;  // words per row
+  const int gpr = t.in_dim / t.group_size;
+  const uint32_t cb = (uint32_t)n * rw * 4, sb = (uint32_t)n * gpr * 2;
+  tc::bulk_g2s(dst_codes, t.w + e * t.expert_stride_w + (int64_t)lo * rw, cb, bar);
+  tc::bulk_g2s(dst_s, t.scales + e * t.expert_stride_sb + (int64_t)lo * gpr, sb, bar);
+  tc::bulk_g2s(dst_b, t.biases + e * t.expert_stride_sb + (int64_t)lo * gpr, sb, bar);
+  return cb + 2 * sb;
+}
+
+__host__ __device__ inline uint32_t s1_bytes(const moeq_qtensor& t, int n) {
+  return n <= 0 ? 0u
+                : (uint32_t)n * (uint32_t)(t.in_dim * t.bits / 8) +
+                      2u * (uint32_t)n * (uint32_t)(t.in_dim / t.group_size) * 2u;
+}
+
+// The CTA's slices of one input vector (cpr chunks) into shared memory,
+// by the threads [t0, t0 + nthr) (whole warps); slot s holds chunks
+// 32 s .. 32 s + 31, word-major.
+template <int BITS, int NL, class SRC>
+__device__ __forceinline__ void s1_build_slices(const void* src, int cpr, uint32_t* base, int t0,
+                                                int nthr) {
+  constexpr int SLW = s1_slw<BITS, NL>();
+  const int lane = threadIdx.x & 31;
+  const int wb = ((int)threadIdx.x - t0) & ~31;
+  for (int c0 = wb; c0 < cpr; c0 += nthr) {
+    const int ch = c0 + lane;
+    SliceVec<BITS, NL> sv;
+    build_slice<BITS, NL, SRC>(src, ch, ch < cpr, sv);
+    slice_store<BITS, NL>(base + (c0 >> 5) * SLW * 32, sv, lane);
+  }
+}
+
+// One lane's part of a row's dot product with the input whose slices the
+// lane holds (chunks ch0 + lane, ch0 + lane + 32, ...).  codes/sc/bi: shared
+// addresses of the row's codes, scales and biases.
+template <int BITS, int NL, int NSL>
+__device__ __forceinline__ float s1_row_part(uint32_t codes, uint32_t sc, uint32_t bi,
+                                             const SliceVec<BITS, NL> (&sv)[NSL], int lane,
+                                             int cpr, int gsh, int ch0 = 0) {
+  constexpr int VPC = Chunk<BITS>::VPC, NC = Chunk<BITS>::NC, NB = SliceVec<BITS, NL>::NB;
+  float acc = 0.0f;
+#pragma unroll
+  for (int s = 0; s < NSL; ++s) {
+    const int ch = ch0 + s * 32 + lane;
+    if (ch < cpr) {
+      const uint4 wv = gq_lds128(codes + ch * 16);
+      uint32_t c[NC];
+      Chunk<BITS>::split(wv, c);
+      float s2[2] = {0.0f, 0.0f}, b2[2] = {0.0f, 0.0f};
+#pragma unroll
+      for (int pb = 0; pb < NB; ++pb) {
+        const int g = (ch * VPC + pb * kXBlock) >> gsh;
+        s2[pb] = bf16_bits_to_float(lds_u16(sc + g * 2));
+        b2[pb] = bf16_bits_to_float(lds_u16(bi + g * 2));
+      }
+      acc += chunk_contrib<BITS, NL>(c, sv[s], s2, b2);
+    }
+  }
+  return acc;
+}
+
+template <int BITS, int NL, int NSL>
+__device__ __forceinline__ void s1_load_slices(const uint32_t* base, SliceVec<BITS, NL> (&sv)[NSL],
+                                               int lane) {
+  constexpr int SLW = s1_slw<BITS, NL>();
+#pragma unroll
+  for (int s = 0; s < NSL; ++s) slice_load<BITS, NL>(base + s * SLW * 32, sv[s], lane);
+}
+
+__device__ __forceinline__ int s1_log2(int g) { return 31 - __clz(g); }
+
+// Waits (bounded) for the copies a CTA issued on the barriers in `mask`
+// before it exits, so that no bulk copy lands in freed shared memory (the
+// phases have completed already unless a wait ran out).
+__device__ __forceinline__ void s1_drain(uint64_t* bars, uint32_t mask, int* status) {
+  for (int m = 0; m < 32; ++m)
+    if ((mask >> m) & 1u) tc::mbar_wait(&bars[m], 0, status);
+}
+
+// ------------------------------------------------------------------ R: router rows
+// Warp w holds input slot w % ns (chunks 32 s .. 32 s + 31, ns = nsR) in
+// registers and takes the rows of row group w / ns; each row's ns partial
+// sums meet in shared memory and are added in slot order.
+__global__ void __launch_bounds__(kS1Threads, 1) k_s1_router(const __grid_constant__ S1Args a) {
+  constexpr int BITS = 8, NL = 3;
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+  float* red = reinterpret_cast<float*>(sm + kS1HeadBytes);  // [row][8]
+  const uint32_t sb = tc::smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const moeq_qtensor& R = a.router;
+  const int rb = a.H * BITS / 8, gpr = a.H / R.group_size;
+  int r0, r1;
+  s1_rows(a.E, a.qR, gridDim.x, blockIdx.x, r0, r1);
+  const bool sg = a.has_shared && blockIdx.x == gridDim.x - 1;
+  const uint32_t blk_off = s1_al(kS1HeadBytes + (a.r_rows_max + 1) * 8 * 4, 128);
+  const S1Blk rbk = s1_blk(a.r_rows_max, rb, gpr, 1);
+  const S1Blk gbk = s1_blk(1, rb, gpr, 1);
+  const uint32_t sg_off = blk_off + rbk.bytes;
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    tc::fence_mbar_init();
+    // the router's weights do not depend on the preceding launch
+    uint32_t bytes = s1_bytes(R, r1 - r0) + (sg ? s1_bytes(a.sg, 1) : 0u);
+    tc::mbar_arrive_expect_tx(bar, bytes);
+    s1_issue(R, 0, r0, r1, sb + blk_off + rbk.codes, sb + blk_off + rbk.sc, sb + blk_off + rbk.bi,
+             bar);
+    if (sg)
+      s1_issue(a.sg, 0, 0, 1, sb + sg_off + gbk.codes, sb + sg_off + gbk.sc, sb + sg_off + gbk.bi,
+               bar);
+  }
+  tc::grid_dep_wait();
+  tc::grid_dep_launch();
+  const int ns = a.nsR, rg = 8 / ns;
+  const int slot = warp % ns, grp = warp / ns;
+  const int cpr = a.H / Chunk<BITS>::VPC;
+  const int ch0 = slot * 32;
+  SliceVec<BITS, NL> sv[1];
+  if (grp < rg) build_slice<BITS, NL, SrcBF16>(a.x, ch0 + lane, ch0 + lane < cpr, sv[0]);
+  __syncthreads();  // the barrier's initialisation is visible to every thread
+  const bool ok = tc::mbar_wait(bar, 0, a.status);
+  const int nr = r1 - r0 + (sg ? 1 : 0);
+  const int gsh = s1_log2(R.group_size);
+  for (int i = grp; ok && grp < rg && i < nr; i += rg) {
+    const bool is_sg = i >= r1 - r0;
+    const uint32_t base = is_sg ? sb + sg_off : sb + blk_off;
+    const S1Blk& k = is_sg ? gbk : rbk;
+    const int j = is_sg ? 0 : i;
+    const float p = s1_row_part<BITS, NL, 1>(base + k.codes + j * rb, base + k.sc + j * gpr * 2,
+                                             base + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
+    const float t = warp_sum(p);
+    if (lane == 0) red[i * 8 + slot] = t;
+  }
+  __syncthreads();
+  if (ok && tid < nr) {
+    float t = 0.0f;
+    for (int q = 0; q < ns; ++q) t += red[tid * 8 + q];
+    if (tid >= r1 - r0) *a.sg_logit = t;
+    else a.logits[r0 + tid] = t;
+  }
+  if (tid == 0) s1_drain(bar, 1u, a.status);
+}
+
+// Rows [lo, hi) of one packed matrix (expert e) into a block region with
+// 16-byte asynchronous copies spread over the CTA's threads (scales and
+// biases are whole 16-byte runs: the row quanta guarantee it).
+__device__ __forceinline__ void s1_async_rows(const moeq_qtensor& t, int64_t e, int lo, int hi,
+                                              uint32_t dst_codes, uint32_t dst_s, uint32_t dst_b,
+                                              int tid, int nthr) {
+  const int n = hi - lo;
+  if (n <= 0) return;
+  const int rw = t.in_dim * t.bits / 32;
+  const int gpr = t.in_dim / t.group_size;
+  const uint8_t* wc = reinterpret_cast<const uint8_t*>(t.w + e * t.expert_stride_w + (int64_t)lo * rw);
+  const uint8_t* ws = reinterpret_cast<const uint8_t*>(t.scales + e * t.expert_stride_sb +
+                                                       (int64_t)lo * gpr);
+  const uint8_t* wb = reinterpret_cast<const uint8_t*>(t.biases + e * t.expert_stride_sb +
+                                                       (int64_t)lo * gpr);
+  const int cb = n * rw * 4, sbb = n * gpr * 2;
+  for (int o = tid * 16; o < cb; o += nthr * 16) tc::cp_async16(dst_codes + o, wc + o, 16);
+  for (int o = tid * 16; o < sbb; o += nthr * 16) {
+    tc::cp_async16(dst_s + o, ws + o, 16);
+    tc::cp_async16(dst_b + o, wb + o, 16);
+  }
+}
+
+// ------------------------------------------------------------------ G: top-K, gate/up + SwiGLU
+// 16 warps.  A row pair (gate row, up row) is split over SGc warps, each
+// holding NSLW input slots (chunks ch0 .. ch0 + 32 NSLW - 1) in registers;
+// the SGc partial sums meet in shared memory and are added in slot order.
+template <int BITS, int NSLW>
+__global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S1Args a) {
+  constexpr int NL = 2, SLW = s1_slw<BITS, NL>();
+  constexpr int NW = kS1WideThreads / 32;
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm);
+  int32_t* sidx = reinterpret_cast<int32_t*>(sm + S1Smem::IDX_OFF);
+  float* sw = reinterpret_cast<float*>(sm + S1Smem::W_OFF);
+  float* ssig = reinterpret_cast<float*>(sm + S1Smem::SIG_OFF);
+  const uint32_t sb = tc::smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = a.K, hs = a.has_shared ? 1 : 0;
+  const int rb = a.H * BITS / 8, gpr = a.H / a.gate.group_size;
+  int g0, g1, s0 = 0, s1 = 0;
+  s1_rows(a.I, a.qG, gridDim.x, blockIdx.x, g0, g1);
+  if (hs) s1_rows(a.Ish, a.qGs, gridDim.x, blockIdx.x, s0, s1);
+  const int SGc = (a.nsG + NSLW - 1) / NSLW, IG = NW / SGc;
+  const uint32_t sl_off = kS1HeadBytes;
+  const uint32_t red_off = s1_al(sl_off + (uint32_t)SGc * NSLW * SLW * 32 * 4, 16);
+  const int items_max = a.g_sh_max + K * a.g_rt_max;
+  const uint32_t blk_off = s1_al(red_off + (uint32_t)items_max * SGc * 8, 128);
+  float* red = reinterpret_cast<float*>(sm + red_off);
+  const S1Blk shb = s1_blk(a.g_sh_max, rb, gpr, 2);
+  const S1Blk rtb = s1_blk(a.g_rt_max, rb, gpr, 2);
+  auto region = [&](int m) -> uint32_t {
+    return sb + blk_off + (m < hs ? 0u : hs * shb.bytes + (uint32_t)(m - hs) * rtb.bytes);
+  };
+  if (tid == 0) {
+    for (int m = 0; m < hs + K; ++m) tc::mbar_init(&bars[m], kS1WideThreads);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  // the shared expert's rows do not depend on the routing
+  if (hs) {
+    const uint32_t r = region(0);
+    s1_async_rows(a.sh_gate, 0, s0, s1, r + shb.codes, r + shb.sc, r + shb.bi, tid, kS1WideThreads);
+    s1_async_rows(a.sh_up, 0, s0, s1, r + shb.stride + shb.codes, r + shb.stride + shb.sc,
+                  r + shb.stride + shb.bi, tid, kS1WideThreads);
+    tc::cp_async_arrive_noinc(&bars[0]);
+  }
+  tc::grid_dep_wait();
+  tc::grid_dep_launch();
+  uint32_t* slices = reinterpret_cast<uint32_t*>(sm + sl_off);
+  const int cpr = a.H / Chunk<BITS>::VPC;
+  if (warp == 0) {
+    // the routing (every CTA computes it; CTA 0 publishes it); the shared
+    // gate's logit is loaded alongside the router logits
+    const float sgl = (hs && lane == 0) ? *a.sg_logit : 0.0f;
+    const float* lg = a.logits;
+    const int E = a.E;
+    if (E <= 32) route_token_regs<1>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else if (E <= 64) route_token_regs<2>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else if (E <= 128) route_token_regs<4>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else if (E <= 256) route_token_regs<8>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else route_token_regs<16>(lg, E, K, a.renorm, a.router_scale, sidx, sw);  // E <= 512
+    if (lane == 0 && hs) *ssig = 1.0f / (1.0f + expf(-sgl));
+    __syncwarp();
+    if (blockIdx.x == 0) {
+      if (lane < K) {
+        a.idx[lane] = sidx[lane];
+        a.w[lane] = sw[lane];
+      }
+      if (lane == 0 && hs) *a.sigma = *ssig;
+    }
+  } else {
+    s1_build_slices<BITS, NL, SrcBF16>(a.x, cpr, slices, 32, kS1WideThreads - 32);
+  }
+  __syncthreads();
+  // the routed experts' rows, by every thread
+  for (int k = 0; k < K; ++k) {
+    const uint32_t r = region(hs + k);
+    const int64_t e = sidx[k];
+    s1_async_rows(a.gate, e, g0, g1, r + rtb.codes, r + rtb.sc, r + rtb.bi, tid, kS1WideThreads);
+    s1_async_rows(a.up, e, g0, g1, r + rtb.stride + rtb.codes, r + rtb.stride + rtb.sc,
+                  r + rtb.stride + rtb.bi, tid, kS1WideThreads);
+    tc::cp_async_arrive_noinc(&bars[hs + k]);
+  }
+  if (warp == 1 && lane < K && (int)blockIdx.x < a.gridD) {
+    // the routed down rows that D's CTA of this index will read, into L2
+    int d0, d1;
+    s1_rows(a.H, a.qD, a.gridD, blockIdx.x, d0, d1);
+    const moeq_qtensor& D = a.down;
+    const int64_t e = sidx[lane];
+    const int rw = D.in_dim * D.bits / 32, dg = D.in_dim / D.group_size;
+    if (d1 > d0) {
+      tc::prefetch_l2(D.w + e * D.expert_stride_w + (int64_t)d0 * rw, (uint32_t)(d1 - d0) * rw * 4);
+      tc::prefetch_l2(D.scales + e * D.expert_stride_sb + (int64_t)d0 * dg,
+                      (uint32_t)(d1 - d0) * dg * 2);
+      tc::prefetch_l2(D.biases + e * D.expert_stride_sb + (int64_t)d0 * dg,
+                      (uint32_t)(d1 - d0) * dg * 2);
+    }
+  }
+  const int ig = warp / SGc, sgi = warp % SGc;
+  const int ch0 = sgi * NSLW * 32;
+  SliceVec<BITS, NL> sv[NSLW];
+  s1_load_slices<BITS, NL, NSLW>(slices + sgi * NSLW * SLW * 32, sv, lane);
+  const int gsh = s1_log2(a.gate.group_size);
+  const int nsh = s1 - s0, nrt = g1 - g0;
+  const int total = nsh + K * nrt;
+  bool ok = true;
+  for (int it = ig; ok && ig < IG && it < total; it += IG) {
+    int m, j;
+    if (it < nsh) {
+      m = 0;
+      j = it;
+    } else {
+      m = hs + (it - nsh) / nrt;
+      j = (it - nsh) % nrt;
+    }
+    ok = tc::mbar_wait(&bars[m], 0, a.status);
+    if (!ok) break;
+    const S1Blk& k = m < hs ? shb : rtb;
+    const uint32_t r = region(m);
+    const float pg = s1_row_part<BITS, NL, NSLW>(r + k.codes + j * rb, r + k.sc + j * gpr * 2,
+                                                 r + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
+    const float pu = s1_row_part<BITS, NL, NSLW>(
+        r + k.stride + k.codes + j * rb, r + k.stride + k.sc + j * gpr * 2,
+        r + k.stride + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
+    const float g = warp_sum(pg), u = warp_sum(pu);
+    if (lane == 0) {
+      red[(it * SGc + sgi) * 2] = g;
+      red[(it * SGc + sgi) * 2 + 1] = u;
+    }
+  }
+  if (!ok && lane == 0) set_status(a.status, MOEQ_ERR_TIMEOUT);
+  const bool all_ok = __syncthreads_and(ok);
+  if (all_ok) {
+    for (int t = tid; t < total; t += kS1WideThreads) {
+      float g = 0.0f, u = 0.0f;
+      for (int q = 0; q < SGc; ++q) {
+        g += red[(t * SGc + q) * 2];
+        u += red[(t * SGc + q) * 2 + 1];
+      }
+      float* dst = t < nsh ? a.h + (int64_t)K * a.I + s0 + t
+                           : a.h + (int64_t)((t - nsh) / nrt) * a.I + g0 + (t - nsh) % nrt;
+      *dst = __fdividef(g, 1.0f + __expf(-g)) * u;
+    }
+  }
+  tc::cp_async_wait_all();
+}
+
+// ------------------------------------------------------------------ D: down rows + combine
+// 16 warps; warp w owns output rows w, w + 16, ... of the CTA's block and
+// sums, for each of them, every matrix's row (shared first, then the routed
+// experts in slot order) weighted by the shared gate or the routing weight.
+template <int BITS, int NSL>
+__global__ void __launch_bounds__(kS1WideThreads, 1) k_s1_down(const __grid_constant__ S1Args a) {
+  constexpr int NL = 2, SLW = s1_slw<BITS, NL>();
+  constexpr int NW = kS1WideThreads / 32;
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm);
+  int32_t* sidx = reinterpret_cast<int32_t*>(sm + S1Smem::IDX_OFF);
+  float* sw = reinterpret_cast<float*>(sm + S1Smem::W_OFF);
+  float* ssig = reinterpret_cast<float*>(sm + S1Smem::SIG_OFF);
+  const uint32_t sb = tc::smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = a.K, hs = a.has_shared ? 1 : 0, NM = hs + K;
+  const moeq_qtensor& D = a.down;
+  int d0, d1;
+  s1_rows(a.H, a.qD, gridDim.x, blockIdx.x, d0, d1);
+  const int rbr = a.I * BITS / 8, gpr_r = a.I / D.group_size;
+  const int rbs = hs ? a.Ish * BITS / 8 : 0, gpr_s = hs ? a.Ish / a.sh_down.group_size : 0;
+  const uint32_t sl_off = kS1HeadBytes;
+  const uint32_t set_words = NSL * SLW * 32;
+  const uint32_t blk_off = s1_al(sl_off + (uint32_t)NM * set_words * 4, 128);
+  const S1Blk shb = s1_blk(a.d_rows_max, hs ? rbs : 16, hs ? gpr_s : 8, 1);
+  const S1Blk rtb = s1_blk(a.d_rows_max, rbr, gpr_r, 1);
+  auto region = [&](int m) -> uint32_t {
+    return sb + blk_off + (m < hs ? 0u : hs * shb.bytes + (uint32_t)(m - hs) * rtb.bytes);
+  };
+  if (tid == 0) {
+    for (int m = 0; m < NM; ++m) tc::mbar_init(&bars[m], kS1WideThreads);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (hs) {
+    const uint32_t r = region(0);
+    s1_async_rows(a.sh_down, 0, d0, d1, r + shb.codes, r + shb.sc, r + shb.bi, tid,
+                  kS1WideThreads);
+    tc::cp_async_arrive_noinc(&bars[0]);
+  }
+  tc::grid_dep_wait();
+  tc::grid_dep_launch();
+  if (tid < K) {
+    sidx[tid] = a.idx[tid];
+    sw[tid] = a.w[tid];
+  }
+  if (tid == 0 && hs) *ssig = *a.sigma;
+  __syncthreads();
+  for (int k = 0; k < K; ++k) {
+    const uint32_t r = region(hs + k);
+    s1_async_rows(D, sidx[k], d0, d1, r + rtb.codes, r + rtb.sc, r + rtb.bi, tid, kS1WideThreads);
+    tc::cp_async_arrive_noinc(&bars[hs + k]);
+  }
+  // the slices of every hidden vector (fp32): matrix m's set at m * set_words;
+  // the warps take (matrix, 32-chunk group) pairs in turn
+  uint32_t* slices = reinterpret_cast<uint32_t*>(sm + sl_off);
+  const int cpr_r = a.I / Chunk<BITS>::VPC, cpr_s = hs ? a.Ish / Chunk<BITS>::VPC : 0;
+  {
+    const int ngrp = ((cpr_r > cpr_s ? cpr_r : cpr_s) + 31) / 32;
+    for (int t = warp; t < NM * ngrp; t += NW) {
+      const int m = t / ngrp, c0 = (t % ngrp) * 32;
+      const bool shm = m < hs;
+      const int cpr = shm ? cpr_s : cpr_r;
+      if (c0 >= cpr) continue;
+      const float* src = shm ? a.h + (int64_t)K * a.I : a.h + (int64_t)(m - hs) * a.I;
+      const int ch = c0 + lane;
+      SliceVec<BITS, NL> v;
+      build_slice<BITS, NL, SrcF32>(src, ch, ch < cpr, v);
+      slice_store<BITS, NL>(slices + m * set_words + (c0 >> 5) * SLW * 32, v, lane);
+    }
+  }
+  __syncthreads();
+  const int gsh = s1_log2(D.group_size);
+  const int nd = d1 - d0;
+  float acc[kS1RowsPerWarp];
+#pragma unroll
+  for (int j = 0; j < kS1RowsPerWarp; ++j) acc[j] = 0.0f;
+  bool ok = true;
+  for (int m = 0; m < NM && ok && warp < nd; ++m) {
+    const bool shm = m < hs;
+    SliceVec<BITS, NL> sv[NSL];
+    s1_load_slices<BITS, NL, NSL>(slices + m * set_words, sv, lane);
+    const float coef = shm ? *ssig : sw[m - hs];
+    const int rb = shm ? rbs : rbr, gpr = shm ? gpr_s : gpr_r, cpr = shm ? cpr_s : cpr_r;
+    const S1Blk& k = shm ? shb : rtb;
+    const uint32_t r = region(m);
+    ok = tc::mbar_wait(&bars[m], 0, a.status);
+    if (!ok) break;
+#pragma unroll
+    for (int j = 0; j < kS1RowsPerWarp; ++j) {
+      const int row = warp + NW * j;
+      if (row < nd)
+        acc[j] += coef * s1_row_part<BITS, NL, NSL>(r + k.codes + row * rb,
+                                                    r + k.sc + row * gpr * 2,
+                                                    r + k.bi + row * gpr * 2, sv, lane, cpr, gsh);
+    }
+  }
+  if (ok) {
+#pragma unroll
+    for (int j = 0; j < kS1RowsPerWarp; ++j) {
+      const int row = warp + NW * j;
+      if (row < nd) {
+        const float t = warp_sum(acc[j]);
+        if (lane == 0) a.y[d0 + row] = t + (a.residual ? a.residual[d0 + row] : 0.0f);
+      }
+    }
+  }
+  tc::cp_async_wait_all();
+}
+
+// ------------------------------------------------------------------ host side
+int gcd_i(int x, int y) {
+  while (y) {
+    const int t = x % y;
+    x = y;
+    y = t;
+  }
+  return x;
+}
+// Rows per block unit so that a block's scales start on a 16-byte boundary.
+int row_quantum(int gpr) { return 16 / gcd_i(16, 2 * gpr); }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool s1_tensor_ok(const moeq_qtensor& t, bool bank) {
+  if (t.format != MOEQ_FMT_AFFINE) return false;
+  if (!(t.bits == 2 || t.bits == 4 || t.bits == 8)) return false;
+  if (!aligned16(t.w) || !aligned16(t.scales) || !aligned16(t.biases)) return false;
+  if (bank && ((t.expert_stride_w % 4) || (t.expert_stride_sb % 8))) return false;
+  return true;
+}
+
+template <class Kern>
+cudaError_t s1_launch(Kern kern, std::atomic<bool>* attr, int grid, int threads, uint32_t smem,
+                      const S1Args& a, cudaStream_t st) {
+  int dev;
+  if (!current_device(dev)) return cudaErrorInvalidDevice;
+  if (!attr[dev].load(std::memory_order_acquire)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kS1SmemMax);
+    // every launch asks for the largest shared-memory carveout, so that a
+    // launch's CTAs can start on an SM the previous launch still occupies
+    // (a different carveout would wait for the SM to drain)
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    attr[dev].store(true, std::memory_order_release);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+cudaError_t launch_r(const S1Args& a, cudaStream_t st) {
+  static std::atomic<bool> attr[kMaxDevices];
+  return s1_launch(k_s1_router, attr, a.gridR, kS1Threads, a.smem_R, a, st);
+}
+template <int BITS, int NSLW>
+cudaError_t launch_g(const S1Args& a, cudaStream_t st) {
+  static std::atomic<bool> attr[kMaxDevices];
+  return s1_launch(k_s1_gateup<BITS, NSLW>, attr, a.gridG, kS1WideThreads, a.smem_G, a, st);
+}
+template <int BITS, int NSL>
+cudaError_t launch_d(const S1Args& a, cudaStream_t st) {
+  static std::atomic<bool> attr[kMaxDevices];
+  return s1_launch(k_s1_down<BITS, NSL>, attr, a.gridD, kS1WideThreads, a.smem_D, a, st);
+}
+
+// Gate/up warps hold 2 input slots each; down warps hold a hidden vector's
+// slots: up to 4 (2-bit rows of 64-value chunks: 2, intermediate 4096).
+template <int BITS>
+cudaError_t launch_g_bits(const S1Args& a, cudaStream_t st) {
+  return launch_g<BITS, kS1SlotsPerWarp>(a, st);
+}
+template <int BITS>
+cudaError_t launch_d_bits(const S1Args& a, cudaStream_t st) {
+  if (a.nsD <= 1) return launch_d<BITS, 1>(a, st);
+  if (BITS == 2 || a.nsD <= 2) return launch_d<BITS, 2>(a, st);
+  return launch_d<BITS == 2 ? 4 : BITS, 4>(a, st);
+}
+
+}  // namespace
+
+bool single_decode_plan(const moeq_layer* L, int sms, S1Args& a) {
+  memset(&a, 0, sizeof(a));
+  const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
+  if (sms < 1 || K < 1 || K > kS1MaxK || E > 512 || E < K) return false;
+  const moeq_qtensor &R = L->router, &Gt = L->gate, &U = L->up, &D = L->down;
+  // router: 8-bit, and the shared-expert gate row in the same format
+  if (R.bits != 8 || !s1_tensor_ok(R, false) || R.out_dim != E || R.in_dim != H) return false;
+  const int BE = Gt.bits, GE = Gt.group_size;
+  for (const moeq_qtensor* t : {&Gt, &U, &D})
+    if (!s1_tensor_ok(*t, true) || t->bits != BE || t->group_size != GE) return false;
+  const bool hs = L->has_shared != 0;
+  const int Ish = hs ? L->sh_gate.out_dim : 0;
+  if (hs) {
+    const moeq_qtensor& SG = L->sh_expert_gate;
+    if (!s1_tensor_ok(SG, false) || SG.bits != R.bits || SG.group_size != R.group_size ||
+        SG.in_dim != H || ((H / SG.group_size) % 8))
+      return false;
+    for (const moeq_qtensor* t : {&L->sh_gate, &L->sh_up, &L->sh_down})
+      if (!s1_tensor_ok(*t, false) || t->bits != BE || t->group_size != GE) return false;
+    if (L->sh_up.out_dim != Ish || L->sh_down.in_dim != Ish || L->sh_down.out_dim != H)
+      return false;
+  }
+  a.H = H;
+  a.I = I;
+  a.Ish = Ish;
+  a.E = E;
+  a.K = K;
+  a.has_shared = hs;
+  a.renorm = L->renorm;
+  a.router_scale = L->router_scale;
+  a.router = R;
+  if (hs) a.sg = L->sh_expert_gate;
+  a.gate = Gt;
+  a.up = U;
+  a.down = D;
+  if (hs) {
+    a.sh_gate = L->sh_gate;
+    a.sh_up = L->sh_up;
+    a.sh_down = L->sh_down;
+  }
+  // row quanta: every block's scales on a 16-byte boundary
+  a.qR = row_quantum(H / R.group_size);
+  a.qG = row_quantum(H / GE);
+  a.qGs = a.qG;
+  int qD = row_quantum(I / GE);
+  if (hs) {
+    const int qs = row_quantum(Ish / GE);
+    qD = qD / gcd_i(qD, qs) * qs;
+  }
+  a.qD = qD;
+  if (E % a.qR || I % a.qG || (hs && Ish % a.qGs) || H % a.qD) return false;
+  // grids and the largest block of a CTA
+  a.gridR = E / a.qR < sms ? E / a.qR : sms;
+  a.gridG = sms;
+  a.gridD = H / a.qD < sms ? H / a.qD : sms;
+  auto most = [](int n, int q, int grid) { return (int)(((n / q) + grid - 1) / grid) * q; };
+  a.r_rows_max = most(E, a.qR, a.gridR);
+  a.g_rt_max = most(I, a.qG, a.gridG);
+  a.g_sh_max = hs ? most(Ish, a.qGs, a.gridG) : 0;
+  a.d_rows_max = most(H, a.qD, a.gridD);
+  if (a.d_rows_max > (kS1WideThreads / 32) * kS1RowsPerWarp) return false;
+  // input slices per lane
+  const int vpc = 128 / BE;
+  if (H % 32 || I % vpc || (hs && Ish % vpc)) return false;
+  a.nsR = (H / 16 + 31) / 32;
+  a.nsG = (H / vpc + 31) / 32;
+  const int cpr_d = (I > Ish ? I : Ish) / vpc;
+  a.nsD = (cpr_d + 31) / 32;
+  if (a.nsR > 8 || a.nsG > 16 || a.nsD > (BE == 2 ? 2 : 4)) return false;
+  // shared memory per launch
+  const int SGc = (a.nsG + kS1SlotsPerWarp - 1) / kS1SlotsPerWarp;  // as k_s1_gateup splits
+  const int nsD = a.nsD <= 1 ? 1 : a.nsD <= 2 ? 2 : 4;  // as launch_d_bits picks
+  const int slwE = 2 * (vpc / 4) + 2 * (BE == 2 ? 2 : 1);
+  {
+    const int rb = H, gpr = H / R.group_size;
+    uint32_t s = s1_al(kS1HeadBytes + (a.r_rows_max + 1) * 8 * 4, 128);
+    s += s1_blk(a.r_rows_max, rb, gpr, 1).bytes + s1_blk(1, rb, gpr, 1).bytes;
+    a.smem_R = s;
+  }
+  {
+    const int rb = H * BE / 8, gpr = H / GE;
+    const uint32_t red = s1_al(kS1HeadBytes + SGc * kS1SlotsPerWarp * slwE * 32 * 4, 16);
+    const int items = a.g_sh_max + K * a.g_rt_max;
+    uint32_t s = s1_al(red + (uint32_t)items * SGc * 8, 128);
+    s += (hs ? s1_blk(a.g_sh_max, rb, gpr, 2).bytes : 0u) +
+         (uint32_t)K * s1_blk(a.g_rt_max, rb, gpr, 2).bytes;
+    a.smem_G = s;
+  }
+  {
+    const int NM = K + (hs ? 1 : 0);
+    uint32_t s = s1_al(kS1HeadBytes + (uint32_t)NM * nsD * slwE * 32 * 4, 128);
+    s += (hs ? s1_blk(a.d_rows_max, Ish * BE / 8, Ish / GE, 1).bytes : 0u) +
+         (uint32_t)K * s1_blk(a.d_rows_max, I * BE / 8, I / GE, 1).bytes;
+    a.smem_D = s;
+  }
+  if (a.smem_R > kS1SmemMax || a.smem_G > kS1SmemMax || a.smem_D > kS1SmemMax) return false;
+  return true;
+}
+
+cudaError_t launch_single_router(const S1Args& a, cudaStream_t st) { return launch_r(a, st); }
+
+cudaError_t launch_single_gateup(const S1Args& a, cudaStream_t st) {
+  switch (a.gate.bits) {
+    case 2: return launch_g_bits<2>(a, st);
+    case 4: return launch_g_bits<4>(a, st);
+    default: return launch_g_bits<8>(a, st);
+  }
+}
+
+cudaError_t launch_single_down(const S1Args& a, cudaStream_t st) {
+  switch (a.down.bits) {
+    case 2: return launch_d_bits<2>(a, st);
+    case 4: return launch_d_bits<4>(a, st);
+    default: return launch_d_bits<8>(a, st);
+  }
+}
+
+}  // namespace moeq

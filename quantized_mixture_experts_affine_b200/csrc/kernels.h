@@ -257,6 +257,45 @@ bool fused_decode_plan(const moeq_layer* L, int grid, bool route_from_router, Fu
 int fused_decode_threads();
 cudaError_t launch_fused_decode(const FusedArgs& a, const FzMaps& m, int grid, cudaStream_t st);
 
+// ------------------------------------------------------------------ single-token decode
+// Three lean launches for M = 1 (k_single.cu): router rows, then top-K with
+// the gate/up rows and SwiGLU, then the down rows with the combine.  Each
+// CTA bulk-copies whole row blocks of every matrix it reads into shared
+// memory at once; blocks that do not depend on the preceding launch are
+// issued before its dependency wait.
+constexpr int kS1MaxK = 16;
+
+struct S1Args {
+  int32_t H, I, Ish, E, K, has_shared, renorm;
+  float router_scale;
+  moeq_qtensor router, sg, gate, up, down, sh_gate, sh_up, sh_down;
+  // row blocks: a matrix's rows split over a grid in units of q rows (the
+  // smallest count whose scales fill whole 16-byte runs)
+  int32_t qR, qG, qGs, qD;
+  int32_t gridR, gridG, gridD;
+  int32_t r_rows_max, g_sh_max, g_rt_max, d_rows_max;  // largest block of a CTA
+  int32_t nsR, nsG, nsD;                               // input slices per lane
+  uint32_t smem_R, smem_G, smem_D;                     // dynamic shared memory
+  const uint16_t* x;      // [H] bf16
+  const float* residual;  // [H] or null
+  float* y;               // [H]
+  float* logits;          // [E]
+  float* sg_logit;        // [1]
+  int32_t* idx;           // [K] routing out
+  float* w;               // [K]
+  float* sigma;           // [1]
+  float* h;               // [K*I + Ish] hidden rows (routed, then shared)
+  int* status;
+};
+
+// Shape part of the arguments for this layer on `sms` SMs; false when the
+// layer's formats or sizes are outside what the three launches take (the
+// general decode path runs it then).
+bool single_decode_plan(const moeq_layer* L, int sms, S1Args& a);
+cudaError_t launch_single_router(const S1Args& a, cudaStream_t st);
+cudaError_t launch_single_gateup(const S1Args& a, cudaStream_t st);
+cudaError_t launch_single_down(const S1Args& a, cudaStream_t st);
+
 // Codes and/or fp32 weights of one matrix.
 cudaError_t launch_dequant(const moeq_qtensor& t, int expert, uint8_t* q_out, float* w_out,
                            cudaStream_t st);

@@ -4,6 +4,8 @@ Bars: unpacked codes and dequantised fp32 weights bit-exact; qmv relative
 L2 <= 1e-5 (24-bit fixed-point input, fp32 sums); routing equal except at
 near-ties; layer outputs relative L2 <= 2e-3 and max abs <= 1e-2.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -250,17 +252,23 @@ def test_workspace_reuse_and_poison():
 
 
 # ------------------------------------------------------------------ single token (M = 1)
-# Both decode paths for one token: the default three launches and the opt-in
-# one-launch kernel (MOEQ_FUSED_DECODE=1, read on every call), which runs the
-# layers whose formats it takes (every group 64 wide, rows of whole 8-group
-# runs) and leaves the others to the three launches.
+# The three decode paths for one token (environment read on every call):
+#   single      the default: three lean launches (router, top-K + gate/up,
+#               down + combine) for the layers whose formats they take;
+#   launches    MOEQ_SINGLE_DECODE=0: the general decode launches with the
+#               in-kernel plan;
+#   one_launch  MOEQ_FUSED_DECODE=1: the opt-in one-launch kernel (every
+#               group 64 wide, rows of whole 8-group runs).
+# A layer a path does not take runs on the general launches.
 
-@pytest.fixture(params=["launches", "one_launch"])
+@pytest.fixture(params=["single", "launches", "one_launch"])
 def decode_path(request, monkeypatch):
+    monkeypatch.delenv("MOEQ_FUSED_DECODE", raising=False)
+    monkeypatch.delenv("MOEQ_SINGLE_DECODE", raising=False)
     if request.param == "one_launch":
         monkeypatch.setenv("MOEQ_FUSED_DECODE", "1")
-    else:
-        monkeypatch.delenv("MOEQ_FUSED_DECODE", raising=False)
+    elif request.param == "launches":
+        monkeypatch.setenv("MOEQ_SINGLE_DECODE", "0")
     return request.param
 
 
@@ -301,6 +309,27 @@ def test_single_token_many_tokens_in_a_row(name, decode_path):
         assert moeq.moeq_device_status() == 0
         check_layer_outputs(cfg, SEED, 1, xb, y.cpu().numpy(), idx.cpu().numpy(),
                             w.cpu().numpy())
+
+
+@pytest.mark.parametrize("name,G", [("decode_30b", 64), ("decode_30b", 128), ("decode_397b", 32),
+                                    ("prefill_8bit", 64), ("prefill_8bit", 32), ("tiny", 64)])
+def test_single_token_residual_group_sizes(name, G, decode_path):
+    """One token with a residual, 4- and 8-bit layers at group sizes 32, 64
+    and 128 (row blocks whose scale runs are 24, 48 or 6 entries per row),
+    against the oracle; a second call into the same workspace is bitwise
+    the same."""
+    cfg = dataclasses.replace(CONFIGS[name], name=f"{name}_g{G}", G=G)
+    L = synthetic_layer(cfg, SEED, 0)
+    xb, x = x_tokens(cfg, 1, copy=51)
+    res_np = np.linspace(-1, 1, cfg.H, dtype=np.float32)[None, :]
+    ws = Workspace(L, 1, moeq.MODE_DECODE)
+    y, idx, w = layer_forward(L, x, residual=dev(res_np), ws=ws, mode=moeq.MODE_DECODE)
+    y2 = layer_forward(L, x, residual=dev(res_np), ws=ws, mode=moeq.MODE_DECODE)[0]
+    torch.cuda.synchronize()
+    assert moeq.moeq_device_status() == 0
+    check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy(),
+                        residual=res_np)
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
 
 
 @pytest.mark.parametrize("name", ["decode_397b", "mixed_2bit", "tiny"])
