@@ -84,13 +84,26 @@ def config_of(workload, world, copies):
     return d
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
 # kernel each roofline line names, from one ncu capture of the current
-# kernels on that workload: decode gate/up GEMV (it also carries the down
+# kernels on that workload: decode gate/up launch (it also carries the down
 # projections' L2 prefetch), prefill gate/up gather-QMM.  Other workloads:
 # not captured (null).
 TRAFFIC = {
-    "decode_397b_m1": 35535872,
+    "decode_397b_m1": 33128960 + 5376,
     "prefill_8bit_m16068": 959738624 + 185099264,
 }
+
+
+def gateup_kernel(cfg, M):
+    """Name of the decode gate/up launch the library runs for this layer and
+    token count: one token of 2-, 4- or 8-bit affine experts (a shared expert
+    in the same format) behind an 8-bit router with at most 512 experts runs
+    on the single-token launches; everything else on the general GEMV."""
+    single = (M == 1 and cfg.expert_bits in (2, 4, 8) and cfg.router_bits == 8
+              and cfg.E <= 512 and cfg.K <= 16
+              and (not cfg.shared or cfg.shared_bits == cfg.expert_bits)
+              and os.environ.get("MOEQ_SINGLE_DECODE") != "0")
+    return ("k_s1_gateup (top-K + gate/up + SwiGLU, single token)" if single
+            else "k_gemv gate/up+SwiGLU")
 
 
 def parse():
@@ -546,7 +559,7 @@ def run_ours(args):
     layer_bytes = cfg.router_bytes() + mean_distinct * exp_bytes + cfg.shared_bytes()
     gu_bytes = mean_distinct * gu_bytes_expert + sh_gu
 
-    # dominant kernel (gate/up GEMV): per-launch durations over the same steps,
+    # dominant kernel (the gate/up launch): per-launch durations over the same steps,
     # events recorded around it inside captured graphs
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -608,7 +621,7 @@ def run_ours(args):
         "layer_hbm": {"bytes_per_step": layer_bytes, "achieved_gbs": layer_bytes / (ms_step / 1e3) / 1e9,
                       "peak_gbs": peak_hbm, "frac": layer_bytes / (ms_step / 1e3) / 1e9 / peak_hbm,
                       "peak_kind": peak_kind},
-        "roofline": {"bound": "hbm", "kernel": "k_gemv gate/up+SwiGLU", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": gateup_kernel(cfg, M), "achieved": achieved,
                      "peak": peak_hbm, "unit": "GB/s", "frac": achieved / peak_hbm,
                      "traffic": TRAFFIC.get(args.workload), "bytes_per_launch": gu_bytes,
                      "ms_per_launch": k_ms,

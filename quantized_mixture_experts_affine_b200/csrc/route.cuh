@@ -73,12 +73,14 @@ __device__ __forceinline__ void route_token_regs(const float* __restrict__ lg, i
     }
     chosen_sum += p;
   }
-  // softmax normaliser over all experts
+  // softmax normaliser over all experts (only without renormalisation)
   float z = 0.0f;
+  if (!renorm) {
 #pragma unroll
-  for (int j = 0; j < NJ; ++j)
-    if (lane + 32 * j < E) z += expf(v[j] - mx);
-  z = warp_sum(z);
+    for (int j = 0; j < NJ; ++j)
+      if (lane + 32 * j < E) z += expf(v[j] - mx);
+    z = warp_sum(z);
+  }
   const float denom = renorm ? chosen_sum : z;
   if (lane < K) {
     idx[lane] = my_i;
