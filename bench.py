@@ -96,11 +96,13 @@ TRAFFIC = {
 def gateup_kernel(cfg, M):
     """Name of the decode gate/up launch the library runs for this layer and
     token count: one token of 2-, 4- or 8-bit affine experts (a shared expert
-    in the same format) behind an 8-bit router with at most 512 experts runs
-    on the single-token launches; everything else on the general GEMV."""
+    of the same width, or 4-bit beside 2-bit experts) behind an 8-bit router
+    with at most 512 experts runs on the single-token launches (their
+    shared-memory limit aside); everything else on the general GEMV."""
+    bs = cfg.shared_bits if cfg.shared else cfg.expert_bits
     single = (M == 1 and cfg.expert_bits in (2, 4, 8) and cfg.router_bits == 8
               and cfg.E <= 512 and cfg.K <= 16
-              and (not cfg.shared or cfg.shared_bits == cfg.expert_bits)
+              and (bs == cfg.expert_bits or (cfg.expert_bits, bs) == (2, 4))
               and os.environ.get("MOEQ_SINGLE_DECODE") != "0")
     return ("k_s1_gateup (top-K + gate/up + SwiGLU, single token)" if single
             else "k_gemv gate/up+SwiGLU")

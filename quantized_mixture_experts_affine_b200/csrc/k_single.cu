@@ -39,7 +39,6 @@ namespace {
 constexpr int kS1Threads = 256;        // R: 8 warps
 constexpr int kS1WideThreads = 512;    // G and D: 16 warps
 constexpr int kS1RowsPerWarp = 4;      // D: output rows per warp
-constexpr int kS1SlotsPerWarp = 2;     // G: input slots per warp
 // G's registers per thread: 512 x 96 leaves room for an R CTA (256 x 48)
 // on the same SM, so G's CTAs start while R runs
 constexpr int kS1GateUpRegs = 96;
@@ -262,12 +261,46 @@ __device__ __forceinline__ void s1_async_rows(const moeq_qtensor& t, int64_t e, 
 
 // ------------------------------------------------------------------ G: top-K, gate/up + SwiGLU
 // 16 warps.  A row pair (gate row, up row) is split over SGc warps, each
-// holding NSLW input slots (chunks ch0 .. ch0 + 32 NSLW - 1) in registers;
-// the SGc partial sums meet in shared memory and are added in slot order.
-template <int BITS, int NSLW>
+// holding s1_slots(BITS) input slots (chunks ch0 .. ch0 + 32 slots - 1) in
+// registers; the SGc partial sums meet in shared memory and are added in
+// slot order.  The shared expert (BSH-bit codes, which may differ from the
+// routed experts' BITS) has slices of its own layout and its own split.
+__host__ __device__ constexpr int s1_slots(int bits) { return bits == 2 ? 1 : 2; }
+
+template <int B, int NSLW>
+__device__ __forceinline__ bool s1_gateup_items(const S1Args& a, int n_items, int nrt, int m0,
+                                                const uint32_t* slices, int sgc, uint32_t sb,
+                                                uint32_t base0, uint32_t stride_m, const S1Blk& k,
+                                                uint64_t* bars, float* red, int warp, int lane,
+                                                int gsh) {
+  constexpr int NL = 2, SLW = s1_slw<B, NL>(), NW = kS1WideThreads / 32;
+  const int ig = warp / sgc, sgi = warp % sgc, IG = NW / sgc;
+  if (ig >= IG) return true;
+  const int rb = a.H * B / 8, gpr = a.H / a.gate.group_size, cpr = a.H / Chunk<B>::VPC;
+  const int ch0 = sgi * NSLW * 32;
+  SliceVec<B, NL> sv[NSLW];
+  s1_load_slices<B, NL, NSLW>(slices + sgi * NSLW * SLW * 32, sv, lane);
+  for (int it = ig; it < n_items; it += IG) {
+    const int mi = it / nrt, j = it % nrt;
+    if (!tc::mbar_wait(&bars[m0 + mi], 0, a.status)) return false;
+    const uint32_t r = sb + base0 + (uint32_t)mi * stride_m;
+    const float pg = s1_row_part<B, NL, NSLW>(r + k.codes + j * rb, r + k.sc + j * gpr * 2,
+                                              r + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
+    const float pu = s1_row_part<B, NL, NSLW>(
+        r + k.stride + k.codes + j * rb, r + k.stride + k.sc + j * gpr * 2,
+        r + k.stride + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
+    const float g = warp_sum(pg), u = warp_sum(pu);
+    if (lane == 0) {
+      red[(it * sgc + sgi) * 2] = g;
+      red[(it * sgc + sgi) * 2 + 1] = u;
+    }
+  }
+  return true;
+}
+
+template <int BITS, int BSH>
 __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S1Args a) {
-  constexpr int NL = 2, SLW = s1_slw<BITS, NL>();
-  constexpr int NW = kS1WideThreads / 32;
+  constexpr int NL = 2, NW = kS1WideThreads / 32;
   extern __shared__ __align__(128) uint8_t sm[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm);
   int32_t* sidx = reinterpret_cast<int32_t*>(sm + S1Smem::IDX_OFF);
@@ -276,21 +309,17 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   const uint32_t sb = tc::smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = a.K, hs = a.has_shared ? 1 : 0;
-  const int rb = a.H * BITS / 8, gpr = a.H / a.gate.group_size;
+  const int gpr = a.H / a.gate.group_size;
   int g0, g1, s0 = 0, s1 = 0;
   s1_rows(a.I, a.qG, gridDim.x, blockIdx.x, g0, g1);
   if (hs) s1_rows(a.Ish, a.qGs, gridDim.x, blockIdx.x, s0, s1);
-  const int SGc = (a.nsG + NSLW - 1) / NSLW, IG = NW / SGc;
-  const uint32_t sl_off = kS1HeadBytes;
-  const uint32_t red_off = s1_al(sl_off + (uint32_t)SGc * NSLW * SLW * 32 * 4, 16);
-  const int items_max = a.g_sh_max + K * a.g_rt_max;
-  const uint32_t blk_off = s1_al(red_off + (uint32_t)items_max * SGc * 8, 128);
-  float* red = reinterpret_cast<float*>(sm + red_off);
-  const S1Blk shb = s1_blk(a.g_sh_max, rb, gpr, 2);
-  const S1Blk rtb = s1_blk(a.g_rt_max, rb, gpr, 2);
-  auto region = [&](int m) -> uint32_t {
-    return sb + blk_off + (m < hs ? 0u : hs * shb.bytes + (uint32_t)(m - hs) * rtb.bytes);
-  };
+  uint32_t* sl_r = reinterpret_cast<uint32_t*>(sm + a.g_sl_r);
+  uint32_t* sl_s = reinterpret_cast<uint32_t*>(sm + a.g_sl_s);
+  float* red_s = reinterpret_cast<float*>(sm + a.g_red);
+  float* red_r = red_s + a.g_sh_max * a.g_sgc_s * 2;
+  const S1Blk shb = s1_blk(a.g_sh_max, a.H * BSH / 8, gpr, 2);
+  const S1Blk rtb = s1_blk(a.g_rt_max, a.H * BITS / 8, gpr, 2);
+  const uint32_t rt_off = a.g_blk + hs * shb.bytes;  // routed block k at rt_off + k * rtb.bytes
   if (tid == 0) {
     for (int m = 0; m < hs + K; ++m) tc::mbar_init(&bars[m], kS1WideThreads);
     tc::fence_mbar_init();
@@ -298,7 +327,7 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   __syncthreads();
   // the shared expert's rows do not depend on the routing
   if (hs) {
-    const uint32_t r = region(0);
+    const uint32_t r = sb + a.g_blk;
     s1_async_rows(a.sh_gate, 0, s0, s1, r + shb.codes, r + shb.sc, r + shb.bi, tid, kS1WideThreads);
     s1_async_rows(a.sh_up, 0, s0, s1, r + shb.stride + shb.codes, r + shb.stride + shb.sc,
                   r + shb.stride + shb.bi, tid, kS1WideThreads);
@@ -306,8 +335,6 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   }
   tc::grid_dep_wait();
   tc::grid_dep_launch();
-  uint32_t* slices = reinterpret_cast<uint32_t*>(sm + sl_off);
-  const int cpr = a.H / Chunk<BITS>::VPC;
   if (warp == 0) {
     // the routing (every CTA computes it; CTA 0 publishes it); the shared
     // gate's logit is loaded alongside the router logits
@@ -329,12 +356,15 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
       if (lane == 0 && hs) *a.sigma = *ssig;
     }
   } else {
-    s1_build_slices<BITS, NL, SrcBF16>(a.x, cpr, slices, 32, kS1WideThreads - 32);
+    s1_build_slices<BITS, NL, SrcBF16>(a.x, a.H / Chunk<BITS>::VPC, sl_r, 32, kS1WideThreads - 32);
+    if (BSH != BITS && hs)
+      s1_build_slices<BSH, NL, SrcBF16>(a.x, a.H / Chunk<BSH>::VPC, sl_s, 32,
+                                        kS1WideThreads - 32);
   }
   __syncthreads();
   // the routed experts' rows, by every thread
   for (int k = 0; k < K; ++k) {
-    const uint32_t r = region(hs + k);
+    const uint32_t r = sb + rt_off + (uint32_t)k * rtb.bytes;
     const int64_t e = sidx[k];
     s1_async_rows(a.gate, e, g0, g1, r + rtb.codes, r + rtb.sc, r + rtb.bi, tid, kS1WideThreads);
     s1_async_rows(a.up, e, g0, g1, r + rtb.stride + rtb.codes, r + rtb.stride + rtb.sc,
@@ -356,49 +386,32 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
                       (uint32_t)(d1 - d0) * dg * 2);
     }
   }
-  const int ig = warp / SGc, sgi = warp % SGc;
-  const int ch0 = sgi * NSLW * 32;
-  SliceVec<BITS, NL> sv[NSLW];
-  s1_load_slices<BITS, NL, NSLW>(slices + sgi * NSLW * SLW * 32, sv, lane);
   const int gsh = s1_log2(a.gate.group_size);
   const int nsh = s1 - s0, nrt = g1 - g0;
-  const int total = nsh + K * nrt;
+  // the shared expert's rows first (their copies were issued first), then
+  // the routed experts' rows
   bool ok = true;
-  for (int it = ig; ok && ig < IG && it < total; it += IG) {
-    int m, j;
-    if (it < nsh) {
-      m = 0;
-      j = it;
-    } else {
-      m = hs + (it - nsh) / nrt;
-      j = (it - nsh) % nrt;
-    }
-    ok = tc::mbar_wait(&bars[m], 0, a.status);
-    if (!ok) break;
-    const S1Blk& k = m < hs ? shb : rtb;
-    const uint32_t r = region(m);
-    const float pg = s1_row_part<BITS, NL, NSLW>(r + k.codes + j * rb, r + k.sc + j * gpr * 2,
-                                                 r + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
-    const float pu = s1_row_part<BITS, NL, NSLW>(
-        r + k.stride + k.codes + j * rb, r + k.stride + k.sc + j * gpr * 2,
-        r + k.stride + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
-    const float g = warp_sum(pg), u = warp_sum(pu);
-    if (lane == 0) {
-      red[(it * SGc + sgi) * 2] = g;
-      red[(it * SGc + sgi) * 2 + 1] = u;
-    }
-  }
+  if (hs && nsh > 0)
+    ok = s1_gateup_items<BSH, s1_slots(BSH)>(a, nsh, nsh, 0, BSH == BITS ? sl_r : sl_s,
+                                             a.g_sgc_s, sb, a.g_blk, 0u, shb, bars, red_s, warp,
+                                             lane, gsh);
+  if (ok && nrt > 0)
+    ok = s1_gateup_items<BITS, s1_slots(BITS)>(a, K * nrt, nrt, hs, sl_r, a.g_sgc_r, sb, rt_off,
+                                               rtb.bytes, rtb, bars, red_r, warp, lane, gsh);
   if (!ok && lane == 0) set_status(a.status, MOEQ_ERR_TIMEOUT);
   const bool all_ok = __syncthreads_and(ok);
   if (all_ok) {
-    for (int t = tid; t < total; t += kS1WideThreads) {
+    for (int t = tid; t < nsh + K * nrt; t += kS1WideThreads) {
+      const bool shr = t < nsh;
+      const int q0 = shr ? t : t - nsh, nq = shr ? a.g_sgc_s : a.g_sgc_r;
+      const float* rr = (shr ? red_s : red_r) + q0 * nq * 2;
       float g = 0.0f, u = 0.0f;
-      for (int q = 0; q < SGc; ++q) {
-        g += red[(t * SGc + q) * 2];
-        u += red[(t * SGc + q) * 2 + 1];
+      for (int q = 0; q < nq; ++q) {
+        g += rr[2 * q];
+        u += rr[2 * q + 1];
       }
-      float* dst = t < nsh ? a.h + (int64_t)K * a.I + s0 + t
-                           : a.h + (int64_t)((t - nsh) / nrt) * a.I + g0 + (t - nsh) % nrt;
+      float* dst = shr ? a.h + (int64_t)K * a.I + s0 + t
+                       : a.h + (int64_t)(q0 / nrt) * a.I + g0 + q0 % nrt;
       *dst = __fdividef(g, 1.0f + __expf(-g)) * u;
     }
   }
@@ -409,9 +422,40 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
 // 16 warps; warp w owns output rows w, w + 16, ... of the CTA's block and
 // sums, for each of them, every matrix's row (shared first, then the routed
 // experts in slot order) weighted by the shared gate or the routing weight.
-template <int BITS, int NSL>
+// The shared down matrix has BSH-bit codes, the routed ones BITS.
+template <int B, int NSL>
+__device__ __forceinline__ bool s1_down_matrix(float (&acc)[kS1RowsPerWarp], const uint32_t* set,
+                                               uint32_t r, const S1Blk& k, int in_dim, float coef,
+                                               uint64_t* bar, int nd, int warp, int lane, int gsh,
+                                               int* status) {
+  constexpr int NL = 2, NW = kS1WideThreads / 32;
+  const int rb = in_dim * B / 8, gpr = in_dim >> gsh, cpr = in_dim / Chunk<B>::VPC;
+  SliceVec<B, NL> sv[NSL];
+  s1_load_slices<B, NL, NSL>(set, sv, lane);
+  if (!tc::mbar_wait(bar, 0, status)) return false;
+#pragma unroll
+  for (int j = 0; j < kS1RowsPerWarp; ++j) {
+    const int row = warp + NW * j;
+    if (row < nd)
+      acc[j] += coef * s1_row_part<B, NL, NSL>(r + k.codes + row * rb, r + k.sc + row * gpr * 2,
+                                               r + k.bi + row * gpr * 2, sv, lane, cpr, gsh);
+  }
+  return true;
+}
+
+template <int B>
+__device__ __forceinline__ void s1_down_slices(const float* src, int cpr, int c0, uint32_t* set,
+                                               int lane) {
+  constexpr int NL = 2, SLW = s1_slw<B, NL>();
+  if (c0 >= cpr) return;
+  const int ch = c0 + lane;
+  SliceVec<B, NL> v;
+  build_slice<B, NL, SrcF32>(src, ch, ch < cpr, v);
+  slice_store<B, NL>(set + (c0 >> 5) * SLW * 32, v, lane);
+}
+
+template <int BITS, int BSH, int NSL>
 __global__ void __launch_bounds__(kS1WideThreads, 1) k_s1_down(const __grid_constant__ S1Args a) {
-  constexpr int NL = 2, SLW = s1_slw<BITS, NL>();
   constexpr int NW = kS1WideThreads / 32;
   extern __shared__ __align__(128) uint8_t sm[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm);
@@ -424,15 +468,12 @@ __global__ void __launch_bounds__(kS1WideThreads, 1) k_s1_down(const __grid_cons
   const moeq_qtensor& D = a.down;
   int d0, d1;
   s1_rows(a.H, a.qD, gridDim.x, blockIdx.x, d0, d1);
-  const int rbr = a.I * BITS / 8, gpr_r = a.I / D.group_size;
-  const int rbs = hs ? a.Ish * BITS / 8 : 0, gpr_s = hs ? a.Ish / a.sh_down.group_size : 0;
-  const uint32_t sl_off = kS1HeadBytes;
-  const uint32_t set_words = NSL * SLW * 32;
-  const uint32_t blk_off = s1_al(sl_off + (uint32_t)NM * set_words * 4, 128);
-  const S1Blk shb = s1_blk(a.d_rows_max, hs ? rbs : 16, hs ? gpr_s : 8, 1);
-  const S1Blk rtb = s1_blk(a.d_rows_max, rbr, gpr_r, 1);
+  const int gsh = s1_log2(D.group_size);
+  const uint32_t set_words = a.d_set_bytes / 4;
+  const S1Blk shb = s1_blk(a.d_rows_max, hs ? a.Ish * BSH / 8 : 16, hs ? a.Ish >> gsh : 8, 1);
+  const S1Blk rtb = s1_blk(a.d_rows_max, a.I * BITS / 8, a.I >> gsh, 1);
   auto region = [&](int m) -> uint32_t {
-    return sb + blk_off + (m < hs ? 0u : hs * shb.bytes + (uint32_t)(m - hs) * rtb.bytes);
+    return sb + a.d_blk + (m < hs ? 0u : hs * shb.bytes + (uint32_t)(m - hs) * rtb.bytes);
   };
   if (tid == 0) {
     for (int m = 0; m < NM; ++m) tc::mbar_init(&bars[m], kS1WideThreads);
@@ -460,47 +501,32 @@ __global__ void __launch_bounds__(kS1WideThreads, 1) k_s1_down(const __grid_cons
   }
   // the slices of every hidden vector (fp32): matrix m's set at m * set_words;
   // the warps take (matrix, 32-chunk group) pairs in turn
-  uint32_t* slices = reinterpret_cast<uint32_t*>(sm + sl_off);
-  const int cpr_r = a.I / Chunk<BITS>::VPC, cpr_s = hs ? a.Ish / Chunk<BITS>::VPC : 0;
+  uint32_t* slices = reinterpret_cast<uint32_t*>(sm + kS1HeadBytes);
+  const int cpr_r = a.I / Chunk<BITS>::VPC, cpr_s = hs ? a.Ish / Chunk<BSH>::VPC : 0;
   {
     const int ngrp = ((cpr_r > cpr_s ? cpr_r : cpr_s) + 31) / 32;
     for (int t = warp; t < NM * ngrp; t += NW) {
       const int m = t / ngrp, c0 = (t % ngrp) * 32;
-      const bool shm = m < hs;
-      const int cpr = shm ? cpr_s : cpr_r;
-      if (c0 >= cpr) continue;
-      const float* src = shm ? a.h + (int64_t)K * a.I : a.h + (int64_t)(m - hs) * a.I;
-      const int ch = c0 + lane;
-      SliceVec<BITS, NL> v;
-      build_slice<BITS, NL, SrcF32>(src, ch, ch < cpr, v);
-      slice_store<BITS, NL>(slices + m * set_words + (c0 >> 5) * SLW * 32, v, lane);
+      if (m < hs)
+        s1_down_slices<BSH>(a.h + (int64_t)K * a.I, cpr_s, c0, slices + m * set_words, lane);
+      else
+        s1_down_slices<BITS>(a.h + (int64_t)(m - hs) * a.I, cpr_r, c0, slices + m * set_words,
+                             lane);
     }
   }
   __syncthreads();
-  const int gsh = s1_log2(D.group_size);
   const int nd = d1 - d0;
   float acc[kS1RowsPerWarp];
 #pragma unroll
   for (int j = 0; j < kS1RowsPerWarp; ++j) acc[j] = 0.0f;
   bool ok = true;
   for (int m = 0; m < NM && ok && warp < nd; ++m) {
-    const bool shm = m < hs;
-    SliceVec<BITS, NL> sv[NSL];
-    s1_load_slices<BITS, NL, NSL>(slices + m * set_words, sv, lane);
-    const float coef = shm ? *ssig : sw[m - hs];
-    const int rb = shm ? rbs : rbr, gpr = shm ? gpr_s : gpr_r, cpr = shm ? cpr_s : cpr_r;
-    const S1Blk& k = shm ? shb : rtb;
-    const uint32_t r = region(m);
-    ok = tc::mbar_wait(&bars[m], 0, a.status);
-    if (!ok) break;
-#pragma unroll
-    for (int j = 0; j < kS1RowsPerWarp; ++j) {
-      const int row = warp + NW * j;
-      if (row < nd)
-        acc[j] += coef * s1_row_part<BITS, NL, NSL>(r + k.codes + row * rb,
-                                                    r + k.sc + row * gpr * 2,
-                                                    r + k.bi + row * gpr * 2, sv, lane, cpr, gsh);
-    }
+    if (m < hs)
+      ok = s1_down_matrix<BSH, NSL>(acc, slices + m * set_words, region(m), shb, a.Ish, *ssig,
+                                    &bars[m], nd, warp, lane, gsh, a.status);
+    else
+      ok = s1_down_matrix<BITS, NSL>(acc, slices + m * set_words, region(m), rtb, a.I,
+                                     sw[m - hs], &bars[m], nd, warp, lane, gsh, a.status);
   }
   if (ok) {
 #pragma unroll
@@ -571,29 +597,32 @@ cudaError_t launch_r(const S1Args& a, cudaStream_t st) {
   static std::atomic<bool> attr[kMaxDevices];
   return s1_launch(k_s1_router, attr, a.gridR, kS1Threads, a.smem_R, a, st);
 }
-template <int BITS, int NSLW>
+template <int BITS, int BSH>
 cudaError_t launch_g(const S1Args& a, cudaStream_t st) {
   static std::atomic<bool> attr[kMaxDevices];
-  return s1_launch(k_s1_gateup<BITS, NSLW>, attr, a.gridG, kS1WideThreads, a.smem_G, a, st);
+  return s1_launch(k_s1_gateup<BITS, BSH>, attr, a.gridG, kS1WideThreads, a.smem_G, a, st);
 }
-template <int BITS, int NSL>
+template <int BITS, int BSH, int NSL>
 cudaError_t launch_d(const S1Args& a, cudaStream_t st) {
   static std::atomic<bool> attr[kMaxDevices];
-  return s1_launch(k_s1_down<BITS, NSL>, attr, a.gridD, kS1WideThreads, a.smem_D, a, st);
+  return s1_launch(k_s1_down<BITS, BSH, NSL>, attr, a.gridD, kS1WideThreads, a.smem_D, a, st);
 }
 
-// Gate/up warps hold 2 input slots each; down warps hold a hidden vector's
-// slots: up to 4 (2-bit rows of 64-value chunks: 2, intermediate 4096).
-template <int BITS>
-cudaError_t launch_g_bits(const S1Args& a, cudaStream_t st) {
-  return launch_g<BITS, kS1SlotsPerWarp>(a, st);
-}
-template <int BITS>
+// Down warps hold a hidden vector's slots: 1, 2 or 4 (2-bit rows of
+// 64-value chunks: 1 or 2, intermediate up to 4096).
+int d_slots(int ns) { return ns <= 1 ? 1 : ns <= 2 ? 2 : 4; }
+template <int BITS, int BSH>
 cudaError_t launch_d_bits(const S1Args& a, cudaStream_t st) {
-  if (a.nsD <= 1) return launch_d<BITS, 1>(a, st);
-  if (BITS == 2 || a.nsD <= 2) return launch_d<BITS, 2>(a, st);
-  return launch_d<BITS == 2 ? 4 : BITS, 4>(a, st);
+  if (a.nsD <= 1) return launch_d<BITS, BSH, 1>(a, st);
+  if (BITS == 2 || a.nsD <= 2) return launch_d<BITS, BSH, 2>(a, st);
+  return launch_d<BITS == 2 ? 4 : BITS, BSH == 2 ? 4 : BSH, 4>(a, st);
 }
+
+// Code widths the launches are built for: routed = shared in {2, 4, 8}, and
+// 2-bit routed experts with a 4-bit shared expert (the requantised bank).
+bool s1_bits_pair(int be, int bs) { return (be == bs && (be == 2 || be == 4 || be == 8)) || (be == 2 && bs == 4); }
+
+int slw_of(int bits) { return 2 * (32 / bits) + 2 * (bits == 2 ? 2 : 1); }  // words per slot
 
 }  // namespace
 
@@ -609,13 +638,15 @@ bool single_decode_plan(const moeq_layer* L, int sms, S1Args& a) {
     if (!s1_tensor_ok(*t, true) || t->bits != BE || t->group_size != GE) return false;
   const bool hs = L->has_shared != 0;
   const int Ish = hs ? L->sh_gate.out_dim : 0;
+  const int BS = hs ? L->sh_gate.bits : BE;
+  if (!s1_bits_pair(BE, BS)) return false;
   if (hs) {
     const moeq_qtensor& SG = L->sh_expert_gate;
     if (!s1_tensor_ok(SG, false) || SG.bits != R.bits || SG.group_size != R.group_size ||
         SG.in_dim != H || ((H / SG.group_size) % 8))
       return false;
     for (const moeq_qtensor* t : {&L->sh_gate, &L->sh_up, &L->sh_down})
-      if (!s1_tensor_ok(*t, false) || t->bits != BE || t->group_size != GE) return false;
+      if (!s1_tensor_ok(*t, false) || t->bits != BS || t->group_size != GE) return false;
     if (L->sh_up.out_dim != Ish || L->sh_down.in_dim != Ish || L->sh_down.out_dim != H)
       return false;
   }
@@ -659,17 +690,19 @@ bool single_decode_plan(const moeq_layer* L, int sms, S1Args& a) {
   a.d_rows_max = most(H, a.qD, a.gridD);
   if (a.d_rows_max > (kS1WideThreads / 32) * kS1RowsPerWarp) return false;
   // input slices per lane
-  const int vpc = 128 / BE;
-  if (H % 32 || I % vpc || (hs && Ish % vpc)) return false;
+  const int vpc = 128 / BE, vps = 128 / BS;
+  if (H % 32 || H % vps || I % vpc || (hs && Ish % vps)) return false;
   a.nsR = (H / 16 + 31) / 32;
   a.nsG = (H / vpc + 31) / 32;
-  const int cpr_d = (I > Ish ? I : Ish) / vpc;
+  const int nsGs = (H / vps + 31) / 32;
+  const int cpr_d = (I / vpc > Ish / vps) ? I / vpc : Ish / vps;
   a.nsD = (cpr_d + 31) / 32;
-  if (a.nsR > 8 || a.nsG > 16 || a.nsD > (BE == 2 ? 2 : 4)) return false;
-  // shared memory per launch
-  const int SGc = (a.nsG + kS1SlotsPerWarp - 1) / kS1SlotsPerWarp;  // as k_s1_gateup splits
-  const int nsD = a.nsD <= 1 ? 1 : a.nsD <= 2 ? 2 : 4;  // as launch_d_bits picks
-  const int slwE = 2 * (vpc / 4) + 2 * (BE == 2 ? 2 : 1);
+  if (a.nsR > 8 || a.nsD > (BE == 2 || BS == 2 ? 2 : 4)) return false;
+  // G: warps per row (slot groups) of the routed and of the shared layout
+  a.g_sgc_r = (a.nsG + s1_slots(BE) - 1) / s1_slots(BE);
+  a.g_sgc_s = hs ? (nsGs + s1_slots(BS) - 1) / s1_slots(BS) : 1;
+  if (a.g_sgc_r > kS1WideThreads / 32 || a.g_sgc_s > kS1WideThreads / 32) return false;
+  // shared memory per launch; the kernels take these offsets as they are
   {
     const int rb = H, gpr = H / R.group_size;
     uint32_t s = s1_al(kS1HeadBytes + (a.r_rows_max + 1) * 8 * 4, 128);
@@ -677,20 +710,28 @@ bool single_decode_plan(const moeq_layer* L, int sms, S1Args& a) {
     a.smem_R = s;
   }
   {
-    const int rb = H * BE / 8, gpr = H / GE;
-    const uint32_t red = s1_al(kS1HeadBytes + SGc * kS1SlotsPerWarp * slwE * 32 * 4, 16);
-    const int items = a.g_sh_max + K * a.g_rt_max;
-    uint32_t s = s1_al(red + (uint32_t)items * SGc * 8, 128);
-    s += (hs ? s1_blk(a.g_sh_max, rb, gpr, 2).bytes : 0u) +
-         (uint32_t)K * s1_blk(a.g_rt_max, rb, gpr, 2).bytes;
-    a.smem_G = s;
+    const int gpr = H / GE;
+    a.g_sl_r = kS1HeadBytes;
+    uint32_t end = a.g_sl_r + (uint32_t)a.g_sgc_r * s1_slots(BE) * slw_of(BE) * 32 * 4;
+    a.g_sl_s = a.g_sl_r;
+    if (hs && BS != BE) {
+      a.g_sl_s = s1_al(end, 16);
+      end = a.g_sl_s + (uint32_t)a.g_sgc_s * s1_slots(BS) * slw_of(BS) * 32 * 4;
+    }
+    a.g_red = s1_al(end, 16);
+    const uint32_t red_floats =
+        2u * ((uint32_t)a.g_sh_max * a.g_sgc_s + (uint32_t)K * a.g_rt_max * a.g_sgc_r);
+    a.g_blk = s1_al(a.g_red + red_floats * 4, 128);
+    a.smem_G = a.g_blk + (hs ? s1_blk(a.g_sh_max, H * BS / 8, gpr, 2).bytes : 0u) +
+               (uint32_t)K * s1_blk(a.g_rt_max, H * BE / 8, gpr, 2).bytes;
   }
   {
     const int NM = K + (hs ? 1 : 0);
-    uint32_t s = s1_al(kS1HeadBytes + (uint32_t)NM * nsD * slwE * 32 * 4, 128);
-    s += (hs ? s1_blk(a.d_rows_max, Ish * BE / 8, Ish / GE, 1).bytes : 0u) +
-         (uint32_t)K * s1_blk(a.d_rows_max, I * BE / 8, I / GE, 1).bytes;
-    a.smem_D = s;
+    const int slw = slw_of(BE) > slw_of(BS) ? slw_of(BE) : slw_of(BS);
+    a.d_set_bytes = (uint32_t)d_slots(a.nsD) * slw * 32 * 4;
+    a.d_blk = s1_al(kS1HeadBytes + (uint32_t)NM * a.d_set_bytes, 128);
+    a.smem_D = a.d_blk + (hs ? s1_blk(a.d_rows_max, Ish * BS / 8, Ish / GE, 1).bytes : 0u) +
+               (uint32_t)K * s1_blk(a.d_rows_max, I * BE / 8, I / GE, 1).bytes;
   }
   if (a.smem_R > kS1SmemMax || a.smem_G > kS1SmemMax || a.smem_D > kS1SmemMax) return false;
   return true;
@@ -699,18 +740,20 @@ bool single_decode_plan(const moeq_layer* L, int sms, S1Args& a) {
 cudaError_t launch_single_router(const S1Args& a, cudaStream_t st) { return launch_r(a, st); }
 
 cudaError_t launch_single_gateup(const S1Args& a, cudaStream_t st) {
+  const int bs = a.has_shared ? a.sh_gate.bits : a.gate.bits;
   switch (a.gate.bits) {
-    case 2: return launch_g_bits<2>(a, st);
-    case 4: return launch_g_bits<4>(a, st);
-    default: return launch_g_bits<8>(a, st);
+    case 2: return bs == 4 ? launch_g<2, 4>(a, st) : launch_g<2, 2>(a, st);
+    case 4: return launch_g<4, 4>(a, st);
+    default: return launch_g<8, 8>(a, st);
   }
 }
 
 cudaError_t launch_single_down(const S1Args& a, cudaStream_t st) {
+  const int bs = a.has_shared ? a.sh_down.bits : a.down.bits;
   switch (a.down.bits) {
-    case 2: return launch_d_bits<2>(a, st);
-    case 4: return launch_d_bits<4>(a, st);
-    default: return launch_d_bits<8>(a, st);
+    case 2: return bs == 4 ? launch_d_bits<2, 4>(a, st) : launch_d_bits<2, 2>(a, st);
+    case 4: return launch_d_bits<4, 4>(a, st);
+    default: return launch_d_bits<8, 8>(a, st);
   }
 }
 

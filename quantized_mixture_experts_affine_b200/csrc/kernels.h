@@ -276,6 +276,12 @@ struct S1Args {
   int32_t r_rows_max, g_sh_max, g_rt_max, d_rows_max;  // largest block of a CTA
   int32_t nsR, nsG, nsD;                               // input slices per lane
   uint32_t smem_R, smem_G, smem_D;                     // dynamic shared memory
+  // G: warps per row pair (routed, shared layout); byte offsets of the
+  // routed and shared input slices, the partial sums and the row blocks
+  int32_t g_sgc_r, g_sgc_s;
+  uint32_t g_sl_r, g_sl_s, g_red, g_blk;
+  // D: bytes of one hidden vector's slices; byte offset of the row blocks
+  uint32_t d_set_bytes, d_blk;
   const uint16_t* x;      // [H] bf16
   const float* residual;  // [H] or null
   float* y;               // [H]

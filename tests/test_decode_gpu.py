@@ -332,6 +332,25 @@ def test_single_token_residual_group_sizes(name, G, decode_path):
     assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
 
 
+@pytest.mark.parametrize("name,be,bs", [("decode_397b", 2, 2), ("decode_397b", 2, 4),
+                                       ("decode_397b", 4, 2), ("decode_397b", 8, 8),
+                                       ("decode_30b", 2, 2), ("decode_30b", 8, 8)])
+def test_single_token_code_widths(name, be, bs, decode_path):
+    """One token through routed / shared code widths the single-token
+    launches take (equal widths, 2-bit routed with a 4-bit shared expert)
+    and ones they leave to the general launches (4-bit routed with a 2-bit
+    shared expert; 8-bit 397B-like rows beyond their shared memory), against
+    the oracle."""
+    cfg = dataclasses.replace(CONFIGS[name], name=f"{name}_b{be}s{bs}", expert_bits=be,
+                              shared_bits=bs)
+    L = synthetic_layer(cfg, SEED, 0)
+    xb, x = x_tokens(cfg, 1, copy=52)
+    y, idx, w = layer_forward(L, x, mode=moeq.MODE_DECODE)
+    torch.cuda.synchronize()
+    assert moeq.moeq_device_status() == 0
+    check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
+
+
 @pytest.mark.parametrize("name", ["decode_397b", "mixed_2bit", "tiny"])
 def test_single_token_given_routing(name, decode_path):
     """moeq_expert_ffn with M = 1 (routing passed in): experts, shared expert
