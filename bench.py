@@ -378,6 +378,8 @@ def measure_prefill(workload, steps, warmup, world, seed, want_e2e=True, min_ms=
     w = torch.empty((M, cfg.K), dtype=torch.float32, device="cuda")
     ws = Workspace(L, M, moeq.MODE_PREFILL)
     st = torch.cuda.Stream()
+    # the weights and tokens are drawn on the current stream: done before st uses them
+    torch.cuda.synchronize()
 
     def step(i):
         moeq.moeq_layer_forward(L.desc, xs[i % n_x], M, y, None, idx, w, ws.buf, ws.bytes,
@@ -742,6 +744,8 @@ def sweep_row(row, name, M, kind, copies, seed=0):
             def call(i):
                 moeq.moeq_layer_forward(layers[i % copies].desc, xs[i % copies], M, y, None, idx,
                                         w, ws.buf, ws.bytes, moeq.MODE_AUTO, st)
+    # the inputs are drawn on the current stream: done before st uses them
+    torch.cuda.synchronize()
     with torch.cuda.stream(st):
         for i in range(3):
             call(i)

@@ -418,11 +418,14 @@ static const S1Args* single_shape(const moeq_layer* L, int sms) {
   return c.ok ? &c.a : nullptr;
 }
 
-static moeq_status single_forward(const S1Args& shape, const uint16_t* x, const float* residual,
-                                  float* y, int32_t* idx, float* wts, char* base,
-                                  const DecodeWs& lay, cudaStream_t st) {
+static moeq_status single_forward(const S1Args& shape, const uint16_t* x, const int32_t* idx_in,
+                                  const float* w_in, const float* residual, float* y,
+                                  int32_t* idx, float* wts, char* base, const DecodeWs& lay,
+                                  cudaStream_t st) {
   S1Args a = shape;
   a.x = x;
+  a.idx_in = idx_in;
+  a.w_in = w_in;
   a.residual = residual;
   a.y = y;
   a.logits = (float*)(base + lay.logits);
@@ -433,7 +436,9 @@ static moeq_status single_forward(const S1Args& shape, const uint16_t* x, const 
   a.h = (float*)(base + lay.h);
   a.status = status_ptr();
   if (!a.status) return MOEQ_ERR_CUDA;
-  LAUNCH(launch_single_router(a, st));
+  // a given routing needs the router launch only for the shared gate's row
+  if (idx_in) a.gridR = 1;
+  if (!idx_in || a.has_shared) LAUNCH(launch_single_router(a, st));
   CK(profile_mark(true, st));
   LAUNCH(launch_single_gateup(a, st));
   CK(profile_mark(false, st));
@@ -472,11 +477,10 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
       return fused_forward(*f, t_fused.m, grid, x, idx_in, w_in, residual, y, idx_out, w_out, base,
                            lay, st);
   }
-  // one token routed by the router: three lean launches when the formats
-  // allow (k_single.cu)
-  if (M == 1 && !idx_in && single_decode_enabled()) {
+  // one token: three lean launches when the formats allow (k_single.cu)
+  if (M == 1 && single_decode_enabled()) {
     if (const S1Args* a = single_shape(L, grid_cap()))
-      return single_forward(*a, x, residual, y, idx, wts, base, lay, st);
+      return single_forward(*a, x, idx_in, w_in, residual, y, idx, wts, base, lay, st);
   }
 
   // 1. router logits and the shared-expert gate logit (one launch when the

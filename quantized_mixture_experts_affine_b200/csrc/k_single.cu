@@ -185,8 +185,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_s1_router(const __grid_consta
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const moeq_qtensor& R = a.router;
   const int rb = a.H * BITS / 8, gpr = a.H / R.group_size;
+  // router rows only when the launch routes (a given routing needs the
+  // shared-gate row alone)
   int r0, r1;
-  s1_rows(a.E, a.qR, gridDim.x, blockIdx.x, r0, r1);
+  s1_rows(a.idx_in ? 0 : a.E, a.qR, gridDim.x, blockIdx.x, r0, r1);
   const bool sg = a.has_shared && blockIdx.x == gridDim.x - 1;
   const uint32_t blk_off = s1_al(kS1HeadBytes + (a.r_rows_max + 1) * 8 * 4, 128);
   const S1Blk rbk = s1_blk(a.r_rows_max, rb, gpr, 1);
@@ -341,7 +343,20 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
     const float sgl = (hs && lane == 0) ? *a.sg_logit : 0.0f;
     const float* lg = a.logits;
     const int E = a.E;
-    if (E <= 32) route_token_regs<1>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    if (a.idx_in) {
+      // the caller's routing; an expert index out of range is reported and
+      // read as expert 0
+      if (lane < K) {
+        int e = a.idx_in[lane];
+        if (e < 0 || e >= E) {
+          set_status(a.status, MOEQ_ERR_INVALID_ARG);
+          e = 0;
+        }
+        sidx[lane] = e;
+        sw[lane] = a.w_in[lane];
+      }
+      __syncwarp();
+    } else if (E <= 32) route_token_regs<1>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
     else if (E <= 64) route_token_regs<2>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
     else if (E <= 128) route_token_regs<4>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
     else if (E <= 256) route_token_regs<8>(lg, E, K, a.renorm, a.router_scale, sidx, sw);

@@ -287,7 +287,9 @@ struct S1Args {
   float* y;               // [H]
   float* logits;          // [E]
   float* sg_logit;        // [1]
-  int32_t* idx;           // [K] routing out
+  const int32_t* idx_in;  // [K] the caller's routing, or null: the router's
+  const float* w_in;      // [K]
+  int32_t* idx;           // [K] routing out (the experts the launches use)
   float* w;               // [K]
   float* sigma;           // [1]
   float* h;               // [K*I + Ish] hidden rows (routed, then shared)

@@ -351,6 +351,25 @@ def test_single_token_code_widths(name, be, bs, decode_path):
     check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
 
 
+def test_single_token_expert_index_out_of_range(decode_path):
+    """A given routing with an expert index out of range: every decode path
+    reports MOEQ_ERR_INVALID_ARG in the device status and reads the index
+    as expert 0 (no access outside the bank)."""
+    cfg = CONFIGS["decode_397b"]
+    L = synthetic_layer(cfg, SEED, 0)
+    xb, x = x_tokens(cfg, 1, copy=33)
+    ig = np.array([[5, cfg.E, 17, 200]], dtype=np.int32)
+    wg = np.array([[0.4, 0.3, 0.2, 0.1]], dtype=np.float32)
+    y = expert_ffn(L, x, dev(ig), dev(wg), mode=moeq.MODE_DECODE)
+    torch.cuda.synchronize()
+    assert moeq.moeq_device_status() == moeq.ERR_INVALID_ARG
+    from helpers import oracle_expert_outputs
+    used = np.array([[5, 0, 17, 200]], dtype=np.int32)
+    ref = oracle_expert_outputs(cfg, SEED, 0, xb, used, wg.astype(np.float64), None)
+    got = y.cpu().numpy()
+    assert rel_l2(got, ref) <= 2e-3 and np.abs(got - ref).max() <= 1e-2
+
+
 @pytest.mark.parametrize("name", ["decode_397b", "mixed_2bit", "tiny"])
 def test_single_token_given_routing(name, decode_path):
     """moeq_expert_ffn with M = 1 (routing passed in): experts, shared expert
