@@ -39,6 +39,7 @@ namespace {
 constexpr int kS1Threads = 256;        // R: 8 warps
 constexpr int kS1WideThreads = 512;    // G and D: 16 warps
 constexpr int kS1RowsPerWarp = 4;      // D: output rows per warp
+constexpr int kS1CopyBar = 1;          // D: named barrier of the copying warps
 // G's registers per thread: 512 x 96 leaves room for an R CTA (256 x 48)
 // on the same SM, so G's CTAs start while R runs
 constexpr int kS1GateUpRegs = 96;
@@ -261,6 +262,90 @@ __device__ __forceinline__ void s1_async_rows(const moeq_qtensor& t, int64_t e, 
   }
 }
 
+// Top-K of one token's E <= 32 NJ logits by one warp with route.cuh's rule
+// (the K largest scaled logits, ties to the lower index, listed by value;
+// weights p_k over the chosen sum with renormalisation, else over the
+// softmax normaliser).  Lane l holds experts NJ l .. NJ l + NJ - 1, loaded
+// with 16-byte loads when NJ is a multiple of 4 (lg 16-byte aligned).
+template <int NJ>
+__device__ __forceinline__ void s1_topk(const float* __restrict__ lg, int E, int K, int renorm,
+                                        float scale, int32_t* idx, float* w) {
+  const int lane = threadIdx.x & 31;
+  const int e0 = lane * NJ;
+  float v[NJ];
+  if (NJ % 4 == 0 && e0 + NJ <= E) {
+#pragma unroll
+    for (int q = 0; q < NJ / 4; ++q) {
+      const float4 f = __ldcg(reinterpret_cast<const float4*>(lg + e0) + q);
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) v[j] = e0 + j < E ? lg[e0 + j] : 0.0f;
+  }
+  uint32_t key[NJ];
+  uint32_t avail = 0;  // bit j: expert e0 + j exists and is not taken
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    v[j] *= scale;
+    key[j] = route_key(v[j]);
+    if (e0 + j < E) avail |= 1u << j;
+  }
+  uint32_t lk = 0;
+  int li = kNoExpert;
+  float lv = 0.0f;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j)
+    if (((avail >> j) & 1u) && (li == kNoExpert || key[j] > lk)) {
+      lk = key[j];
+      li = e0 + j;
+      lv = v[j];
+    }
+  float mx = 0.0f, chosen_sum = 0.0f, my_p = 0.0f;
+  int my_i = 0;
+  for (int k = 0; k < K; ++k) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, lk);
+    const uint32_t win = __reduce_min_sync(
+        0xffffffffu, (li != kNoExpert && lk == m) ? (uint32_t)li : 0xffffffffu);
+    const int wl = (int)(win / NJ);
+    const float bv = __shfl_sync(0xffffffffu, lv, wl & 31);
+    if (k == 0) mx = bv;
+    if (win != 0xffffffffu && wl == lane) {
+      avail &= ~(1u << (win - e0));
+      lk = 0;
+      li = kNoExpert;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j)
+        if (((avail >> j) & 1u) && (li == kNoExpert || key[j] > lk)) {
+          lk = key[j];
+          li = e0 + j;
+          lv = v[j];
+        }
+    }
+    const float p = expf(bv - mx);
+    if (lane == k) {
+      my_p = p;
+      my_i = (int)win;
+    }
+    chosen_sum += p;
+  }
+  float z = 0.0f;
+  if (!renorm) {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j)
+      if (e0 + j < E) z += expf(v[j] - mx);
+    z = warp_sum(z);
+  }
+  if (lane < K) {
+    idx[lane] = my_i;
+    w[lane] = my_p / (renorm ? chosen_sum : z);
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ G: top-K, gate/up + SwiGLU
 // 16 warps.  A row pair (gate row, up row) is split over SGc warps, each
 // holding s1_slots(BITS) input slots (chunks ch0 .. ch0 + 32 slots - 1) in
@@ -302,7 +387,7 @@ __device__ __forceinline__ bool s1_gateup_items(const S1Args& a, int n_items, in
 
 template <int BITS, int BSH>
 __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S1Args a) {
-  constexpr int NL = 2, NW = kS1WideThreads / 32;
+  constexpr int NL = 2;
   extern __shared__ __align__(128) uint8_t sm[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm);
   int32_t* sidx = reinterpret_cast<int32_t*>(sm + S1Smem::IDX_OFF);
@@ -356,11 +441,11 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
         sw[lane] = a.w_in[lane];
       }
       __syncwarp();
-    } else if (E <= 32) route_token_regs<1>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
-    else if (E <= 64) route_token_regs<2>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
-    else if (E <= 128) route_token_regs<4>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
-    else if (E <= 256) route_token_regs<8>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
-    else route_token_regs<16>(lg, E, K, a.renorm, a.router_scale, sidx, sw);  // E <= 512
+    } else if (E <= 32) s1_topk<1>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else if (E <= 64) s1_topk<2>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else if (E <= 128) s1_topk<4>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else if (E <= 256) s1_topk<8>(lg, E, K, a.renorm, a.router_scale, sidx, sw);
+    else s1_topk<16>(lg, E, K, a.renorm, a.router_scale, sidx, sw);  // E <= 512
     if (lane == 0 && hs) *ssig = 1.0f / (1.0f + expf(-sgl));
     __syncwarp();
     if (blockIdx.x == 0) {
@@ -490,8 +575,11 @@ __global__ void __launch_bounds__(kS1WideThreads, 1) k_s1_down(const __grid_cons
   auto region = [&](int m) -> uint32_t {
     return sb + a.d_blk + (m < hs ? 0u : hs * shb.bytes + (uint32_t)(m - hs) * rtb.bytes);
   };
+  // the shared matrix's barrier counts every thread's copies, a routed
+  // matrix's those of the copying warps (the upper half)
+  constexpr int kCopyThreads = kS1WideThreads / 2;
   if (tid == 0) {
-    for (int m = 0; m < NM; ++m) tc::mbar_init(&bars[m], kS1WideThreads);
+    for (int m = 0; m < NM; ++m) tc::mbar_init(&bars[m], m < hs ? kS1WideThreads : kCopyThreads);
     tc::fence_mbar_init();
   }
   __syncthreads();
@@ -503,24 +591,28 @@ __global__ void __launch_bounds__(kS1WideThreads, 1) k_s1_down(const __grid_cons
   }
   tc::grid_dep_wait();
   tc::grid_dep_launch();
-  if (tid < K) {
-    sidx[tid] = a.idx[tid];
-    sw[tid] = a.w[tid];
-  }
-  if (tid == 0 && hs) *ssig = *a.sigma;
-  __syncthreads();
-  for (int k = 0; k < K; ++k) {
-    const uint32_t r = region(hs + k);
-    s1_async_rows(D, sidx[k], d0, d1, r + rtb.codes, r + rtb.sc, r + rtb.bi, tid, kS1WideThreads);
-    tc::cp_async_arrive_noinc(&bars[hs + k]);
-  }
-  // the slices of every hidden vector (fp32): matrix m's set at m * set_words;
-  // the warps take (matrix, 32-chunk group) pairs in turn
   uint32_t* slices = reinterpret_cast<uint32_t*>(sm + kS1HeadBytes);
   const int cpr_r = a.I / Chunk<BITS>::VPC, cpr_s = hs ? a.Ish / Chunk<BSH>::VPC : 0;
-  {
+  if (tid >= kCopyThreads) {
+    // the upper half reads the routing and copies the routed rows while the
+    // lower half builds the hidden vectors' slices
+    const int t = tid - kCopyThreads;
+    if (t < K) {
+      sidx[t] = a.idx[t];
+      sw[t] = a.w[t];
+    }
+    if (t == 0 && hs) *ssig = *a.sigma;
+    tc::named_sync(kS1CopyBar, kCopyThreads);
+    for (int k = 0; k < K; ++k) {
+      const uint32_t r = region(hs + k);
+      s1_async_rows(D, sidx[k], d0, d1, r + rtb.codes, r + rtb.sc, r + rtb.bi, t, kCopyThreads);
+      tc::cp_async_arrive_noinc(&bars[hs + k]);
+    }
+  } else {
+    // the slices of every hidden vector (fp32): matrix m's set at
+    // m * set_words; the warps take (matrix, 32-chunk group) pairs in turn
     const int ngrp = ((cpr_r > cpr_s ? cpr_r : cpr_s) + 31) / 32;
-    for (int t = warp; t < NM * ngrp; t += NW) {
+    for (int t = warp; t < NM * ngrp; t += kCopyThreads / 32) {
       const int m = t / ngrp, c0 = (t % ngrp) * 32;
       if (m < hs)
         s1_down_slices<BSH>(a.h + (int64_t)K * a.I, cpr_s, c0, slices + m * set_words, lane);
