@@ -359,9 +359,10 @@ __device__ __forceinline__ bool s1_gateup_items(const S1Args& a, int n_items, in
                                                 const uint32_t* slices, int sgc, uint32_t sb,
                                                 uint32_t base0, uint32_t stride_m, const S1Blk& k,
                                                 uint64_t* bars, float* red, int warp, int lane,
-                                                int gsh) {
-  constexpr int NL = 2, SLW = s1_slw<B, NL>(), NW = kS1WideThreads / 32;
-  const int ig = warp / sgc, sgi = warp % sgc, IG = NW / sgc;
+                                                int gsh, int nw) {
+  constexpr int NL = 2, SLW = s1_slw<B, NL>();
+  if (warp >= nw) return true;
+  const int ig = warp / sgc, sgi = warp % sgc, IG = nw / sgc;
   if (ig >= IG) return true;
   const int rb = a.H * B / 8, gpr = a.H / a.gate.group_size, cpr = a.H / Chunk<B>::VPC;
   const int ch0 = sgi * NSLW * 32;
@@ -407,8 +408,15 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   const S1Blk shb = s1_blk(a.g_sh_max, a.H * BSH / 8, gpr, 2);
   const S1Blk rtb = s1_blk(a.g_rt_max, a.H * BITS / 8, gpr, 2);
   const uint32_t rt_off = a.g_blk + hs * shb.bytes;  // routed block k at rt_off + k * rtb.bytes
+  // routed rows are copied by the upper half of the warps while the lower
+  // half computes the shared expert's rows when the shared expert is wider
+  // than the routed ones (measured: the 2-bit bank with its 4-bit shared
+  // expert gains 1.6 us per step, equal widths lose 0.2 us); else by every
+  // thread
+  const int copy_lo = (hs && BSH != BITS) ? kS1WideThreads / 2 : 0;
   if (tid == 0) {
-    for (int m = 0; m < hs + K; ++m) tc::mbar_init(&bars[m], kS1WideThreads);
+    for (int m = 0; m < hs + K; ++m)
+      tc::mbar_init(&bars[m], m < hs ? kS1WideThreads : kS1WideThreads - copy_lo);
     tc::fence_mbar_init();
   }
   __syncthreads();
@@ -462,15 +470,18 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
                                         kS1WideThreads - 32);
   }
   __syncthreads();
-  // the routed experts' rows, by every thread
-  for (int k = 0; k < K; ++k) {
-    const uint32_t r = sb + rt_off + (uint32_t)k * rtb.bytes;
-    const int64_t e = sidx[k];
-    s1_async_rows(a.gate, e, g0, g1, r + rtb.codes, r + rtb.sc, r + rtb.bi, tid, kS1WideThreads);
-    s1_async_rows(a.up, e, g0, g1, r + rtb.stride + rtb.codes, r + rtb.stride + rtb.sc,
-                  r + rtb.stride + rtb.bi, tid, kS1WideThreads);
-    tc::cp_async_arrive_noinc(&bars[hs + k]);
-  }
+  // the routed experts' rows (threads copy_lo ..); the lower half starts on
+  // the shared expert's rows meanwhile
+  if (tid >= copy_lo)
+    for (int k = 0; k < K; ++k) {
+      const uint32_t r = sb + rt_off + (uint32_t)k * rtb.bytes;
+      const int64_t e = sidx[k];
+      const int t = tid - copy_lo, nt = kS1WideThreads - copy_lo;
+      s1_async_rows(a.gate, e, g0, g1, r + rtb.codes, r + rtb.sc, r + rtb.bi, t, nt);
+      s1_async_rows(a.up, e, g0, g1, r + rtb.stride + rtb.codes, r + rtb.stride + rtb.sc,
+                    r + rtb.stride + rtb.bi, t, nt);
+      tc::cp_async_arrive_noinc(&bars[hs + k]);
+    }
   if (warp == 1 && lane < K && (int)blockIdx.x < a.gridD) {
     // the routed down rows that D's CTA of this index will read, into L2
     int d0, d1;
@@ -491,13 +502,17 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   // the shared expert's rows first (their copies were issued first), then
   // the routed experts' rows
   bool ok = true;
+  // (the shared rows on the lower half of the warps while the upper half
+  // copies, when a row pair's slot groups fit there)
+  const int nw_sh = copy_lo && a.g_sgc_s <= copy_lo / 32 ? copy_lo / 32 : kS1WideThreads / 32;
   if (hs && nsh > 0)
     ok = s1_gateup_items<BSH, s1_slots(BSH)>(a, nsh, nsh, 0, BSH == BITS ? sl_r : sl_s,
                                              a.g_sgc_s, sb, a.g_blk, 0u, shb, bars, red_s, warp,
-                                             lane, gsh);
+                                             lane, gsh, nw_sh);
   if (ok && nrt > 0)
     ok = s1_gateup_items<BITS, s1_slots(BITS)>(a, K * nrt, nrt, hs, sl_r, a.g_sgc_r, sb, rt_off,
-                                               rtb.bytes, rtb, bars, red_r, warp, lane, gsh);
+                                               rtb.bytes, rtb, bars, red_r, warp, lane, gsh,
+                                               kS1WideThreads / 32);
   if (!ok && lane == 0) set_status(a.status, MOEQ_ERR_TIMEOUT);
   const bool all_ok = __syncthreads_and(ok);
   if (all_ok) {
