@@ -206,11 +206,22 @@ moeq_status moeq_expert_ffn(const moeq_layer* L, const uint16_t* x, int32_t M, c
  * The whole layer: router qmv -> route_topk -> expert_ffn, on the device,
  * with no host round trip.  idx_out/w_out: nullable, receive the routing.
  * Same buffers, workspace and errors as moeq_expert_ffn.
- * Single-token decode runs as three launches.  With the environment
- * variable MOEQ_FUSED_DECODE=1 (read on every call) a layer whose tensors
- * all use group_size 64 with rows of whole 8-group runs runs M = 1 as one
- * persistent launch instead (same results within the layer tolerance; it
- * needs every CTA of its grid resident at once, one per SM).
+ * Single-token decode (M = 1, here and in moeq_expert_ffn) runs as three
+ * lean launches when the layer's formats allow it:
+ *   - 2-, 4- or 8-bit affine experts, with a shared expert of the same
+ *     width or a 4-bit one beside 2-bit experts;
+ *   - an 8-bit router with at most 512 experts, top_k <= 16;
+ *   - each CTA's row blocks fitting in shared memory.
+ * The launches are the router rows, then top-K with gate/up + SwiGLU, then
+ * down + combine.  Other layers and M > 1 use the general decode launches.
+ * Both agree with the oracle within the layer tolerance; each is
+ * deterministic.
+ * The environment variable MOEQ_SINGLE_DECODE=0 (read on every call)
+ * selects the general launches for M = 1.  MOEQ_FUSED_DECODE=1 runs a layer
+ * whose tensors all use group_size 64 with rows of whole 8-group runs as one
+ * persistent launch instead.  That launch gives the same results within the
+ * layer tolerance and needs every CTA of its grid resident at once, one per
+ * SM.
  */
 moeq_status moeq_layer_forward(const moeq_layer* L, const uint16_t* x, int32_t M, float* y,
                                const float* residual, int32_t* idx_out, float* w_out, void* ws,
