@@ -47,25 +47,35 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x
                                                      const int32_t* __restrict__ sorted, int K,
                                                      int64_t n, int row_chunks,
                                                      uint4* __restrict__ out) {
-  // one warp per row: every lane's loads of the row in flight, then stores
+  // one warp per two rows: every lane's loads of both rows in flight, then
+  // streaming (evict-first) stores; the rows are read once, by the gather-QMM
   constexpr int U = 8;
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n;
-       r += warps) {
-    const uint4* src = x16 + (int64_t)(sorted[r] / K) * row_chunks;
-    uint4* dst = out + r * row_chunks;
+  for (int64_t r = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 2; r < n;
+       r += 2 * warps) {
+    const bool two = r + 1 < n;
+    const uint4* src0 = x16 + (int64_t)(sorted[r] / K) * row_chunks;
+    const uint4* src1 = x16 + (int64_t)(sorted[two ? r + 1 : r] / K) * row_chunks;
+    uint4* dst0 = out + r * row_chunks;
+    uint4* dst1 = out + (r + 1) * row_chunks;
     for (int c0 = 0; c0 < row_chunks; c0 += 32 * U) {
-      uint4 v[U];
+      uint4 v[U], w2[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int c = c0 + u * 32 + lane;
-        if (c < row_chunks) v[u] = src[c];
+        if (c < row_chunks) {
+          v[u] = src0[c];
+          w2[u] = src1[c];
+        }
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int c = c0 + u * 32 + lane;
-        if (c < row_chunks) dst[c] = v[u];
+        if (c < row_chunks) {
+          __stcs(dst0 + c, v[u]);
+          if (two) __stcs(dst1 + c, w2[u]);
+        }
       }
     }
   }
