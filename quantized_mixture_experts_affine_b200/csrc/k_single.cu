@@ -39,6 +39,7 @@ namespace {
 constexpr int kS1Threads = 256;        // R: 8 warps
 constexpr int kS1WideThreads = 512;    // G and D: 16 warps
 constexpr int kS1RowsPerWarp = 4;      // D: output rows per warp
+constexpr int kS1SlicesBar = 2;        // G: named barrier of warps 1.. "slices built"
 constexpr int kS1CopyBar = 1;          // D: named barrier of the copying warps
 // G's registers per thread: 512 x 96 leaves room for an R CTA (256 x 48)
 // on the same SM, so G's CTAs start while R runs
@@ -355,22 +356,22 @@ __device__ __forceinline__ void s1_topk(const float* __restrict__ lg, int E, int
 __host__ __device__ constexpr int s1_slots(int bits) { return bits == 2 ? 1 : 2; }
 
 template <int B, int NSLW>
-__device__ __forceinline__ bool s1_gateup_items(const S1Args& a, int n_items, int nrt, int m0,
-                                                const uint32_t* slices, int sgc, uint32_t sb,
-                                                uint32_t base0, uint32_t stride_m, const S1Blk& k,
-                                                uint64_t* bars, float* red, int warp, int lane,
-                                                int gsh, int nw) {
+__device__ __noinline__ bool s1_gateup_items(int H, int* status, int n_items, int nrt, int m0,
+                                             const uint32_t* slices, int sgc, uint32_t sb,
+                                             uint32_t base0, uint32_t stride_m, S1Blk k,
+                                             uint64_t* bars, float* red, int warp, int lane,
+                                             int gsh, int nw) {
   constexpr int NL = 2, SLW = s1_slw<B, NL>();
   if (warp >= nw) return true;
   const int ig = warp / sgc, sgi = warp % sgc, IG = nw / sgc;
   if (ig >= IG) return true;
-  const int rb = a.H * B / 8, gpr = a.H / a.gate.group_size, cpr = a.H / Chunk<B>::VPC;
+  const int rb = H * B / 8, gpr = H >> gsh, cpr = H / Chunk<B>::VPC;
   const int ch0 = sgi * NSLW * 32;
   SliceVec<B, NL> sv[NSLW];
   s1_load_slices<B, NL, NSLW>(slices + sgi * NSLW * SLW * 32, sv, lane);
   for (int it = ig; it < n_items; it += IG) {
     const int mi = it / nrt, j = it % nrt;
-    if (!tc::mbar_wait(&bars[m0 + mi], 0, a.status)) return false;
+    if (!tc::mbar_wait(&bars[m0 + mi], 0, status)) return false;
     const uint32_t r = sb + base0 + (uint32_t)mi * stride_m;
     const float pg = s1_row_part<B, NL, NSLW>(r + k.codes + j * rb, r + k.sc + j * gpr * 2,
                                               r + k.bi + j * gpr * 2, sv, lane, cpr, gsh, ch0);
@@ -408,11 +409,14 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   const S1Blk shb = s1_blk(a.g_sh_max, a.H * BSH / 8, gpr, 2);
   const S1Blk rtb = s1_blk(a.g_rt_max, a.H * BITS / 8, gpr, 2);
   const uint32_t rt_off = a.g_blk + hs * shb.bytes;  // routed block k at rt_off + k * rtb.bytes
-  // routed rows are copied by the upper half of the warps while the lower
-  // half computes the shared expert's rows when the shared expert is wider
-  // than the routed ones (measured: the 2-bit bank with its 4-bit shared
-  // expert gains 1.6 us per step, equal widths lose 0.2 us); else by every
-  // thread
+  // A shared expert of the routed width is computed by warps 1.. while warp
+  // 0 selects the experts (when a row pair's slot groups fit there): 397B-like
+  // layer 23.7 -> 23.1 us per step.  A wider shared expert is computed by the
+  // lower half of the warps while the upper half copies the routed rows
+  // (2-bit bank with its 4-bit shared expert: 27.1 -> 25.4 us).  The item
+  // loop is one out-of-line body for its three uses.
+  constexpr int kShWarps = kS1WideThreads / 32 - 1;
+  const bool early_sh = hs && BSH == BITS && a.g_sgc_s <= kShWarps;
   const int copy_lo = (hs && BSH != BITS) ? kS1WideThreads / 2 : 0;
   if (tid == 0) {
     for (int m = 0; m < hs + K; ++m)
@@ -430,6 +434,7 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   }
   tc::grid_dep_wait();
   tc::grid_dep_launch();
+  bool ok = true;
   if (warp == 0) {
     // the routing (every CTA computes it; CTA 0 publishes it); the shared
     // gate's logit is loaded alongside the router logits
@@ -468,10 +473,16 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
     if (BSH != BITS && hs)
       s1_build_slices<BSH, NL, SrcBF16>(a.x, a.H / Chunk<BSH>::VPC, sl_s, 32,
                                         kS1WideThreads - 32);
+    if (early_sh && s1 > s0) {
+      tc::named_sync(kS1SlicesBar, kS1WideThreads - 32);  // the token's slices are built
+      ok = s1_gateup_items<BSH, s1_slots(BSH)>(a.H, a.status, s1 - s0, s1 - s0, 0,
+                                               BSH == BITS ? sl_r : sl_s, a.g_sgc_s, sb,
+                                               a.g_blk, 0u, shb, bars, red_s, warp - 1, lane,
+                                               s1_log2(a.gate.group_size), kShWarps);
+    }
   }
   __syncthreads();
-  // the routed experts' rows (threads copy_lo ..); the lower half starts on
-  // the shared expert's rows meanwhile
+  // the routed experts' rows, by threads copy_lo ..
   if (tid >= copy_lo)
     for (int k = 0; k < K; ++k) {
       const uint32_t r = sb + rt_off + (uint32_t)k * rtb.bytes;
@@ -499,18 +510,16 @@ __global__ void __maxnreg__(kS1GateUpRegs) k_s1_gateup(const __grid_constant__ S
   }
   const int gsh = s1_log2(a.gate.group_size);
   const int nsh = s1 - s0, nrt = g1 - g0;
-  // the shared expert's rows first (their copies were issued first), then
-  // the routed experts' rows
-  bool ok = true;
-  // (the shared rows on the lower half of the warps while the upper half
-  // copies, when a row pair's slot groups fit there)
+  // the shared rows here unless computed during the selection (on the lower
+  // half of the warps while the upper half copies, when their slot groups
+  // fit there), then the routed experts' rows
   const int nw_sh = copy_lo && a.g_sgc_s <= copy_lo / 32 ? copy_lo / 32 : kS1WideThreads / 32;
-  if (hs && nsh > 0)
-    ok = s1_gateup_items<BSH, s1_slots(BSH)>(a, nsh, nsh, 0, BSH == BITS ? sl_r : sl_s,
+  if (ok && hs && !early_sh && nsh > 0)
+    ok = s1_gateup_items<BSH, s1_slots(BSH)>(a.H, a.status, nsh, nsh, 0, BSH == BITS ? sl_r : sl_s,
                                              a.g_sgc_s, sb, a.g_blk, 0u, shb, bars, red_s, warp,
                                              lane, gsh, nw_sh);
   if (ok && nrt > 0)
-    ok = s1_gateup_items<BITS, s1_slots(BITS)>(a, K * nrt, nrt, hs, sl_r, a.g_sgc_r, sb, rt_off,
+    ok = s1_gateup_items<BITS, s1_slots(BITS)>(a.H, a.status, K * nrt, nrt, hs, sl_r, a.g_sgc_r, sb, rt_off,
                                                rtb.bytes, rtb, bars, red_r, warp, lane, gsh,
                                                kS1WideThreads / 32);
   if (!ok && lane == 0) set_status(a.status, MOEQ_ERR_TIMEOUT);
