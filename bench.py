@@ -88,7 +88,7 @@ def config_of(workload, world, copies):
 # projections' L2 prefetch), prefill gate/up gather-QMM.  Other workloads:
 # not captured (null).
 TRAFFIC = {
-    "decode_397b_m1": 33137664 + 1792,
+    "decode_397b_m1": 33131776 + 0,
     "prefill_8bit_m16068": 959738624 + 185099264,
 }
 

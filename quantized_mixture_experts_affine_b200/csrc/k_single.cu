@@ -191,7 +191,9 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_s1_router(const __grid_consta
   // shared-gate row alone)
   int r0, r1;
   s1_rows(a.idx_in ? 0 : a.E, a.qR, gridDim.x, blockIdx.x, r0, r1);
-  const bool sg = a.has_shared && blockIdx.x == gridDim.x - 1;
+  // the shared-gate row goes to CTA 0, whose block of router rows is the
+  // smallest (row blocks round down)
+  const bool sg = a.has_shared && blockIdx.x == 0;
   const uint32_t blk_off = s1_al(kS1HeadBytes + (a.r_rows_max + 1) * 8 * 4, 128);
   const S1Blk rbk = s1_blk(a.r_rows_max, rb, gpr, 1);
   const S1Blk gbk = s1_blk(1, rb, gpr, 1);
