@@ -351,6 +351,30 @@ def test_single_token_code_widths(name, be, bs, decode_path):
     check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
 
 
+@pytest.mark.parametrize("name,kw", [
+    ("decode_397b", dict(renorm=False, router_scale=0.7)),
+    ("decode_30b", dict(renorm=False)),
+    ("decode_30b", dict(K=1)),
+    ("decode_30b", dict(E=32, K=4)),
+    ("decode_30b", dict(E=40, K=3, router_scale=1.5)),
+], ids=["397b_softmax_w_scale", "30b_softmax_w", "30b_top1", "30b_e32", "30b_e40_k3_scale"])
+def test_routing_variants(name, kw, decode_path):
+    """Weights without renormalisation (softmax over all experts), a router
+    scale, top-1 routing and small or ragged expert counts, on every
+    single-token path (M = 1) and on the general launches (M = 3), against
+    the oracle."""
+    cfg = dataclasses.replace(CONFIGS[name], name=name + "_" + "_".join(f"{k}{v}" for k, v in kw.items()),
+                              **kw)
+    L = synthetic_layer(cfg, SEED, 0)
+    for M in (1, 3):
+        xb, x = x_tokens(cfg, M, copy=60 + M)
+        y, idx, w = layer_forward(L, x, mode=moeq.MODE_DECODE)
+        torch.cuda.synchronize()
+        assert moeq.moeq_device_status() == 0
+        check_layer_outputs(cfg, SEED, 0, xb, y.cpu().numpy(), idx.cpu().numpy(),
+                            w.cpu().numpy())
+
+
 def test_single_token_expert_index_out_of_range(decode_path):
     """A given routing with an expert index out of range: every decode path
     reports MOEQ_ERR_INVALID_ARG in the device status and reads the index
