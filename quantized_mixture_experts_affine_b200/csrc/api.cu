@@ -287,11 +287,25 @@ static cudaError_t run_plain(const moeq_qtensor& shape_t, const Seg* segs, int n
   if (pf) a = *pf; else memset(&a, 0, sizeof(a));
   set_shape(a, shape_t, 1);
   const GemvShape sh = gemv_shape(shape_t.in_dim, shape_t.bits, 1, shape_t.group_size);
+  // Few row blocks and several vectors (the router of a small decode
+  // batch): each row block's vectors are split over several units, so that
+  // both consumer groups of every CTA get work instead of a few CTAs taking
+  // every vector of a block one after another.
+  int blocks = 0;
+  for (int i = 0; i < n; ++i) blocks += gemv_units(segs[i].out_dim, sh);
+  const int want = 2 * grid_cap();
+  int vpu = 0;
+  if (n > 0 && segs[0].n_vec > 1 && blocks > 0 && blocks < want) {
+    const int need = (want + blocks - 1) / blocks;
+    const int nvc = need < segs[0].n_vec ? need : segs[0].n_vec;
+    vpu = (segs[0].n_vec + nvc - 1) / nvc;
+  }
   int units = 0;
   for (int i = 0; i < n; ++i) {
     a.segs[i] = segs[i];
     a.segs[i].unit_begin = units;
-    units += gemv_units(segs[i].out_dim, sh);
+    a.segs[i].vpu = vpu;
+    units += gemv_units(segs[i].out_dim, sh) * seg_vchunks(segs[i].n_vec, vpu);
   }
   a.n_segs = n;
   a.total_units = units;
@@ -564,8 +578,14 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   p.ctr = (int32_t*)(base + lay.ctr);
   p.n_ctr = p.units_per_seg_dn;
   if (L->has_shared) {
-    p.units_per_seg_gu_sh = units_for(L->sh_gate, L->sh_gate.out_dim, 2);
-    p.units_per_seg_dn_sh = units_for(L->sh_down, H, 1);
+    // the shared expert's units hold one token each when there are several:
+    // a unit's tokens run one after another on one consumer group, so M of
+    // them in one unit make that CTA the step's tail
+    p.sh_vpu_gu = M > 1 ? 1 : 0;
+    p.sh_vpu_dn = M > 1 ? 1 : 0;
+    p.units_per_seg_gu_sh =
+        units_for(L->sh_gate, L->sh_gate.out_dim, 2) * seg_vchunks(M, p.sh_vpu_gu);
+    p.units_per_seg_dn_sh = units_for(L->sh_down, H, 1) * seg_vchunks(M, p.sh_vpu_dn);
     p.shared_same_gu = (L->sh_gate.bits == L->gate.bits &&
                         L->sh_gate.group_size == L->gate.group_size &&
                         L->sh_gate.format == L->gate.format);
@@ -623,6 +643,7 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
       a.comb.K = K;
       a.comb.H = H;
       a.comb.has_shared = L->has_shared;
+      a.comb.sh_units = seg_vchunks(M, p.sh_vpu_dn);
     }
     const int grid = max_dn < grid_cap() ? max_dn : grid_cap();
     LAUNCH(launch_gemv(L->down.bits, 2, 1, SRC_F32, a, grid, st));

@@ -399,10 +399,14 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     const DecodePlanArgs& pl = a.plan;
     if (a.fused_plan && pl.has_shared && warp == GV_PRODUCER &&
         (int)blockIdx.x < pl.units_per_seg_gu_sh) {
+      // the shared segment's unit blockIdx.x, mapped as the producer maps it
+      const int nvc = seg_vchunks(pl.M, pl.sh_vpu_gu);
+      const int rbi = (int)blockIdx.x / nvc;
+      const int v0 = ((int)blockIdx.x - rbi * nvc) * pl.sh_vpu_gu;
       GvUnit gu;
-      gu.r0 = blockIdx.x * RU;
+      gu.r0 = rbi * RU;
       gu.nrows = min(RU, pl.sh_gate.out_dim - gu.r0);
-      gu.n_vec = pl.M;
+      gu.n_vec = nvc > 1 ? min(pl.sh_vpu_gu, pl.M - v0) : pl.M;
       gu.vec_mode = 0;
       gu.w[0] = pl.sh_gate.w;
       gu.s[0] = pl.sh_gate.scales;
@@ -410,9 +414,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
       gu.w[1] = pl.sh_up.w;
       gu.s[1] = pl.sh_up.scales;
       gu.b[1] = pl.sh_up.biases;
-      gu.src_base = pl.x;
+      gu.src_base = pl.x + (int64_t)v0 * pl.H;
       gu.src_stride = pl.H;
-      gu.dst_base = pl.h + (int64_t)pl.M * pl.K * pl.I;
+      gu.dst_base = pl.h + (int64_t)pl.M * pl.K * pl.I + (int64_t)v0 * pl.sh_gate.out_dim;
       gu.dst_stride = pl.sh_gate.out_dim;
       gu.vecs = nullptr;
       gv_issue<2, MX>(gsm, sbase, full, 0, gu, row_bytes, gpr, RU);
@@ -560,7 +564,11 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
                                             mine);
         const Seg& sg = segs[si];
         const int u0 = ub_cached ? ub[si] : sg.unit_begin;
-        r0 = (mine - u0) * RU;
+        // a segment split by vectors: units (row block, run of vpu vectors)
+        const int nvc = seg_vchunks(sg.n_vec, sg.vpu);
+        const int rbi = (mine - u0) / nvc;
+        const int v0 = (mine - u0 - rbi * nvc) * sg.vpu;  // 0 when nvc == 1
+        r0 = rbi * RU;
         nrows = min(RU, sg.out_dim - r0);
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
@@ -568,13 +576,22 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
           sp[m] = sg.s[m];
           bp[m] = sg.b[m];
         }
-        n_vec = sg.n_vec;
+        n_vec = nvc > 1 ? min(sg.vpu, sg.n_vec - v0) : sg.n_vec;
         vec_mode = sg.vec_mode;
         src_base = sg.src_base;
         src_stride = sg.src_stride;
         dst_base = sg.dst_base;
         dst_stride = sg.dst_stride;
         vecs = sg.vecs;
+        if (v0 > 0) {
+          if (vec_mode == 0) {
+            src_base = static_cast<const char*>(src_base) +
+                       (int64_t)v0 * src_stride * (SRC == SRC_BF16 ? 2 : 4);
+            dst_base += (int64_t)v0 * dst_stride;
+          } else {
+            vecs += v0;
+          }
+        }
       }
       const int nb = min(32, (total_units - base + (int)gridDim.x - 1) / (int)gridDim.x);
       for (int u = 0; u < nb; ++u, ++it) {
@@ -617,7 +634,15 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
                                             u0);
         const Seg& sg = segs[si];
         if (sg.n_vec > 0) {
-          const void* src0 = sg.vec_mode == 0 ? sg.src_base : sg.vecs[0].src;
+          const int nvc = seg_vchunks(sg.n_vec, sg.vpu);
+          const int lu = u0 - (ub_cached ? ub[si] : sg.unit_begin);
+          const int v0 = (lu - (lu / nvc) * nvc) * sg.vpu;  // 0 when nvc == 1
+          const void* src0 =
+              sg.vec_mode == 0
+                  ? static_cast<const void*>(static_cast<const char*>(sg.src_base) +
+                                             (int64_t)v0 * sg.src_stride *
+                                                 (SRC == SRC_BF16 ? 2 : 4))
+                  : sg.vecs[v0].src;
           if (src0 != cur_src) {
             if (x_shared && src0 == (const void*)a.plan.x) {
               slice_load<BITS, NL>(sl_base + sl * SLW * 32, sv, lane);
@@ -774,7 +799,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
         if (cw == 0 && lane == 0) {
           int last = 0;
           if (n_vec > 0) {
-            last = atomicAdd(&a.comb.ctr[r0 / RU], 1) == n_segs - 1;
+            // every segment covers every row block: one unit each, the
+            // shared one sh_units (split by tokens)
+            const int target = n_segs + (a.comb.has_shared ? a.comb.sh_units - 1 : 0);
+            last = atomicAdd(&a.comb.ctr[r0 / RU], 1) == target - 1;
             if (last) __threadfence();
           }
           *flag = last;
@@ -987,6 +1015,7 @@ __device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const
     g.n_vec = cnt;
     g.unit_begin = gu0 + u * a.units_per_seg_gu;
     g.vec_mode = 1;
+    g.vpu = 0;
     g.src_base = nullptr;
     g.src_stride = 0;
     g.dst_base = nullptr;
@@ -1007,6 +1036,7 @@ __device__ __forceinline__ void write_expert_segs(const DecodePlanArgs& a, const
     dn.n_vec = cnt;
     dn.unit_begin = u * a.units_per_seg_dn;
     dn.vec_mode = 1;
+    dn.vpu = 0;
     dn.src_base = nullptr;
     dn.src_stride = 0;
     dn.dst_base = nullptr;
@@ -1186,6 +1216,7 @@ __device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, i
         g.bits = a.sh_gate.bits;
         g.n_vec = M;
         g.vec_mode = 0;
+        g.vpu = a.sh_vpu_gu;
         g.src_base = a.x;
         g.src_stride = a.H;
         g.dst_base = a.h + (int64_t)n * a.I;
@@ -1212,6 +1243,7 @@ __device__ __forceinline__ void plan_cta(const DecodePlanArgs& a, uint8_t* sm, i
         dn.bits = a.sh_down.bits;
         dn.n_vec = M;
         dn.vec_mode = 0;
+        dn.vpu = a.sh_vpu_dn;
         dn.src_base = a.h + (int64_t)n * a.I;
         dn.src_stride = a.sh_gate.out_dim;
         dn.dst_base = a.d + (int64_t)n * a.H;

@@ -39,6 +39,7 @@ struct Seg {
   int32_t n_vec;
   int32_t unit_begin;  // first work unit of this segment
   int32_t vec_mode;    // 0 strided, 1 list
+  int32_t vpu;         // vectors per work unit (0: all n_vec in one unit)
   const void* src_base;
   int64_t src_stride;  // elements
   float* dst_base;
@@ -81,10 +82,12 @@ struct DecodePlanArgs {
   int32_t n_ctr;
   int32_t units_per_seg_gu; // computed on the host from the shapes
   int32_t units_per_seg_dn;
-  int32_t units_per_seg_gu_sh;
-  int32_t units_per_seg_dn_sh;
+  int32_t units_per_seg_gu_sh;  // row blocks x vector splits of the shared gate/up
+  int32_t units_per_seg_dn_sh;  // row blocks x vector splits of the shared down
   int32_t shared_same_gu;   // 1: the shared gate/up segment joins the routed launch
   int32_t shared_same_dn;   // 1: the shared down segment joins the routed launch
+  int32_t sh_vpu_gu;        // tokens per unit of the shared gate/up segment (0: all M)
+  int32_t sh_vpu_dn;        // tokens per unit of the shared down segment (0: all M)
   int* status;
 };
 
@@ -115,6 +118,11 @@ constexpr int kPlanStageBytes = 64 * 1024;
 // Largest M*K whose plan the gate/up GEMV computes itself (in every CTA).
 constexpr int kFusedMaxPairs = 64;
 __host__ __device__ int plan_route_warps(int M, int E, int nwarps);
+// Units per row block of a segment whose n_vec vectors are split into runs
+// of vpu (vpu = 0: one unit takes them all).
+__host__ __device__ inline int seg_vchunks(int n_vec, int vpu) {
+  return (vpu > 0 && vpu < n_vec) ? (n_vec + vpu - 1) / vpu : 1;
+}
 __host__ __device__ size_t plan_scratch_bytes(int M, int K, int E, int R);
 
 // The weighted combine done by the down GEMV: the CTA that completes the
@@ -127,6 +135,7 @@ struct CombineArgs {
   const float* d;           // [(M*K + M)][H] down rows
   int32_t* ctr;             // [row blocks], zero on entry
   int32_t M, K, H, has_shared;
+  int32_t sh_units;         // units per row block of the shared segment (>= 1)
 };
 
 struct GemvArgs {
