@@ -74,7 +74,7 @@ struct GvSmem {
   static constexpr int VEC_OFF = META_OFF + GV_STAGES * META_STRIDE;
   static constexpr int UB_OFF = VEC_OFF + GV_STAGES * GV_VMAX * 16;
   static constexpr int BAR_OFF = UB_OFF + GV_UB_CAP * 4;
-  static constexpr int N_BARS = 2 * GV_STAGES + 4 * GV_GROUPS;
+  static constexpr int N_BARS = 2 * GV_STAGES + 8 * GV_GROUPS;
   static constexpr int RED_OFF = BAR_OFF + N_BARS * 8;
   // the CTA's own plan (gate/up launch that computes it): segments, vector
   // references, counts, experts; then the fused combine's flags
@@ -357,6 +357,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
   uint64_t* empty = full + GV_STAGES;
   uint64_t* red_full = empty + GV_STAGES;           // [group][2]: slices 1..S-1 -> slice 0
   uint64_t* red_empty = red_full + 2 * GV_GROUPS;   // [group][2]: slice 0 -> slices 1..S-1
+  uint64_t* slot_full = red_empty + 2 * GV_GROUPS;  // [group][2]: built slice -> group
+  uint64_t* slot_empty = slot_full + 2 * GV_GROUPS; // [group][2]: group read it -> builder
   float* red = reinterpret_cast<float*>(gsm + GvSmem::RED_OFF);  // [group][2][GV_CW][8]
   const uint32_t sbase = tc::smem_u32(gsm);
 
@@ -371,6 +373,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     for (int i = 0; i < 2 * GV_GROUPS; ++i) {
       tc::mbar_init(&red_full[i], (uint32_t)((S > 1 ? S - 1 : 1) * J * 8));
       tc::mbar_init(&red_empty[i], (uint32_t)(J * 8));
+      tc::mbar_init(&slot_full[i], 32u);
+      tc::mbar_init(&slot_empty[i], (uint32_t)((W > 1 ? W - 1 : 1) * 32));
     }
     tc::fence_mbar_init();
   }
@@ -625,6 +629,33 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     int gi[2];
 #pragma unroll
     for (int pb = 0; pb < 2; ++pb) gi[pb] = (ch * VPC + (pb < NB ? pb : 0) * kXBlock) / a.G;
+    // With a single slice (S = 1) every warp of the group holds the same
+    // chunk: warp 0 of the group converts each new vector and hands the
+    // slice to the others through a double-buffered slot (full: warp 0's
+    // 32 lanes arrive; empty: the other warps' lanes arrive after copying;
+    // every wait bounded).  Build b uses buffer b & 1.
+    const bool share_build = S == 1 && W > 1 && 2 * SLW * 32 <= GvSmem::SL_WORDS;
+    uint32_t* const sl_grp = sl_base + grp * GvSmem::SL_WORDS;
+    uint32_t nbuild = 0;
+    bool slot_timeout = false;
+    auto group_build = [&](const void* src) {
+      const uint32_t b = nbuild++, buf = b & 1u;
+      uint32_t* slot = sl_grp + buf * SLW * 32;
+      if (cw == 0) {
+        if (b >= 2 && !slot_timeout)
+          slot_timeout = !tc::mbar_wait(&slot_empty[grp * 2 + buf], ((b >> 1) + 1u) & 1u, status);
+        build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
+        slice_store<BITS, NL>(slot, sv, lane);
+        __syncwarp();
+        tc::mbar_arrive(&slot_full[grp * 2 + buf]);
+      } else {
+        if (!slot_timeout)
+          slot_timeout = !tc::mbar_wait(&slot_full[grp * 2 + buf], (b >> 1) & 1u, status);
+        slice_load<BITS, NL>(slot, sv, lane);
+        __syncwarp();
+        tc::mbar_arrive(&slot_empty[grp * 2 + buf]);
+      }
+    };
     // the first vector's slice is built while the first stage streams in
     if (on_w) {
       const int u0 = blockIdx.x + grp * gridDim.x;
@@ -646,17 +677,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
           if (src0 != cur_src) {
             if (x_shared && src0 == (const void*)a.plan.x) {
               slice_load<BITS, NL>(sl_base + sl * SLW * 32, sv, lane);
-            } else if (S == 1 && W > 1) {
-              // every warp of the group holds the same chunk: one loads and
-              // converts the vector, the others copy its slice
-              uint32_t* slot = reinterpret_cast<uint32_t*>(gsm + GvSmem::SL_OFF) +
-                               grp * GvSmem::SL_WORDS;
-              if (cw == 0) {
-                build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
-                slice_store<BITS, NL>(slot, sv, lane);
-              }
-              tc::named_sync(12 + grp, W * 32);
-              if (cw != 0) slice_load<BITS, NL>(slot, sv, lane);
+            } else if (share_build) {
+              group_build(src0);
             } else {
               build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
             }
@@ -696,7 +718,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
             dst = vl[v].dst;
           }
           if (src != cur_src) {
-            build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
+            if (share_build) group_build(src);
+            else build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
             cur_src = src;
           }
           float acc[8];
