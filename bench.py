@@ -34,6 +34,7 @@ WORKLOADS = {
     "decode_397b_m1": ("decode_397b", 1),
     # same shapes with a 16-expert bank: small enough for full ncu captures
     "decode_397b_e16_m1": ("decode_397b_e16", 1),
+    "decode_397b_e64_m8": ("decode_397b_e64", 8),
     "tiny_m1": ("tiny", 1),
     "tiny_m3": ("tiny", 3),
     "tiny_m5": ("tiny", 5),
@@ -57,8 +58,8 @@ def shape(name):
     """Layer shape by name (plain data: loads no library)."""
     import dataclasses
     from quantized_mixture_experts_affine_b200.config import CONFIGS
-    if name == "decode_397b_e16":
-        return dataclasses.replace(CONFIGS["decode_397b"], name=name, E=16)
+    if name in ("decode_397b_e16", "decode_397b_e64"):
+        return dataclasses.replace(CONFIGS["decode_397b"], name=name, E=int(name[-2:]))
     return CONFIGS[name]
 
 
