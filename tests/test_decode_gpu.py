@@ -73,6 +73,9 @@ QMV_CASES = [  # (bits, G, out, in, M, requant)
     (4, 128, 96, 768, 7, False),
     (2, 32, 33, 128, 4, False),
     (4, 64, 40, 192, 3, False),      # 3 groups per row: scale/bias runs not 16-byte multiples
+    # 128 row blocks: each block's tokens are split over units in runs
+    (8, 64, 1024, 4096, 7, False),   # runs of 3, 3, 1 tokens
+    (4, 64, 1024, 4096, 5, False),   # runs of 2, 2, 1 tokens
 ]
 
 
@@ -90,6 +93,28 @@ def test_qmv_parity(bits, G, out, inn, M, rq):
         torch.cuda.synchronize()
         ref = oracle.qmv(host, xb, mat=e)
         assert rel_l2(y.cpu().numpy(), ref) <= 1e-5, rel_l2(y.cpu().numpy(), ref)
+    assert moeq.moeq_device_status() == 0
+
+
+@pytest.mark.parametrize("bits,out,M", [(8, 1024, 7), (4, 1024, 5), (8, 512, 3), (4, 96, 7)])
+def test_qmv_token_split_matches_single_tokens(bits, out, M):
+    """With few row blocks the M tokens of a block are split over several
+    work units (runs of tokens).  Each token's output row must be bitwise
+    the row a one-token call produces: the split only regroups whole vector
+    computations, so a misplaced run shows up as a wrong row."""
+    inn = 4096 if out >= 512 else 768
+    G = 64
+    q = synth.tensor_dev(SEED, synth.tag(synth.ROUTER, 300 + bits), 1, out, inn, bits, G, False)
+    t = moeq.qtensor(q.w, q.s, q.b, out, inn, bits, G, 1)
+    xb = synth.normal_bf16_host(SEED, synth.tag(synth.X, 31), M * inn).reshape(M, inn)
+    x = dev(xb.view(np.int16))
+    y = torch.full((M, out), float("nan"), device="cuda")
+    moeq.moeq_qmv(t, 0, x, M, y)
+    for m in range(M):
+        y1 = torch.full((1, out), float("nan"), device="cuda")
+        moeq.moeq_qmv(t, 0, x[m:m + 1], 1, y1)
+        torch.cuda.synchronize()
+        assert torch.equal(y[m:m + 1], y1), m
     assert moeq.moeq_device_status() == 0
 
 
