@@ -27,6 +27,42 @@ bool gemv_fits(int in_dim, int bits, int nmat, int G) {
 
 int gemv_units(int out_dim, const GemvShape& sh) { return (out_dim + sh.RU - 1) / sh.RU; }
 
+size_t gemv_xslice_words(int H, int bits) {
+  if (bits != 2 && bits != 4 && bits != 8) return 0;
+  const int vpc = chunk_values(bits);
+  const int S = (H / vpc + 31) / 32;
+  const int slw = 2 * (vpc / 4) + 2 * (bits == 2 ? 2 : 1);  // 2 limbs, block scales and sums
+  return (size_t)S * slw * 32;
+}
+
+// One slice (32 chunks) of a token row in the gate/up launch's format, by
+// one warp, into the table (word-major, as slice_load reads it).
+template <int B>
+__device__ __forceinline__ void xslice_one(const uint16_t* row, int H, int sl, uint32_t* out,
+                                           int lane) {
+  const int ch = sl * 32 + lane;
+  SliceVec<B, 2> sv;
+  build_slice<B, 2, SrcBF16>(row, ch, ch < H / Chunk<B>::VPC, sv);
+  slice_store<B, 2>(out, sv, lane);
+}
+
+// The helper warp's share of the token slice table: task t = (token, slice)
+// for t = blockIdx.x, blockIdx.x + gridDim.x, ...
+__device__ __noinline__ void build_xslices(const GemvArgs& a) {
+  const int lane = threadIdx.x & 31;
+  const int tasks = a.xsl_M * a.xsl_S;
+  for (int t = blockIdx.x; t < tasks; t += gridDim.x) {
+    const uint16_t* row = a.xsl_x + (int64_t)(t / a.xsl_S) * a.xsl_H;
+    const int sl = t % a.xsl_S;
+    if (a.xsl_bits == 2)
+      xslice_one<2>(row, a.xsl_H, sl, a.xsl + (size_t)t * (2 * 16 + 4) * 32, lane);
+    else if (a.xsl_bits == 4)
+      xslice_one<4>(row, a.xsl_H, sl, a.xsl + (size_t)t * (2 * 8 + 2) * 32, lane);
+    else if (a.xsl_bits == 8)
+      xslice_one<8>(row, a.xsl_H, sl, a.xsl + (size_t)t * (2 * 4 + 2) * 32, lane);
+  }
+}
+
 // ============================================================== staged GEMV kernel
 // Persistent CTAs (one per SM).  Warp 16 is the producer: it reads the work
 // description of up to 32 of its CTA's units at once (one unit per lane),
@@ -546,6 +582,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     // ------------------------------------------------------------ L2 prefetch
     if (a.fused_plan) prefetch_down(a.plan, pexp, pcnt[4]);
     else if (a.pf_segs) prefetch_segs(a.pf_segs, a.pf_count[0]);
+    // the router launch: the token slice table of the gate/up launch
+    if constexpr (NMAT == 1 && SRC == SRC_BF16 && !MX)
+      if (a.xsl) build_xslices(a);
   } else if (warp == GV_PRODUCER) {
     // ------------------------------------------------------------ producer
     uint32_t it = preissued;
@@ -634,6 +673,20 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     // slice to the others through a double-buffered slot (full: warp 0's
     // 32 lanes arrive; empty: the other warps' lanes arrive after copying;
     // every wait bounded).  Build b uses buffer b & 1.
+    // a token row's slice: copied from the table the router launch built,
+    // else converted here
+    auto vec_slice = [&](const void* src) {
+      if constexpr (NMAT == 2 && SRC == SRC_BF16 && NL == 2 && !MX && !stream_bits(BITS)) {
+        if (a.xsl) {
+          const int64_t off = static_cast<const uint16_t*>(src) - a.xsl_x;
+          if (off >= 0 && off % a.xsl_H == 0 && off / a.xsl_H < a.xsl_M) {
+            slice_load<BITS, NL>(a.xsl + ((off / a.xsl_H) * a.xsl_S + sl) * SLW * 32, sv, lane);
+            return;
+          }
+        }
+      }
+      build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
+    };
     const bool share_build = S == 1 && W > 1 && 2 * SLW * 32 <= GvSmem::SL_WORDS;
     uint32_t* const sl_grp = sl_base + grp * GvSmem::SL_WORDS;
     uint32_t nbuild = 0;
@@ -644,7 +697,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
       if (cw == 0) {
         if (b >= 2 && !slot_timeout)
           slot_timeout = !tc::mbar_wait(&slot_empty[grp * 2 + buf], ((b >> 1) + 1u) & 1u, status);
-        build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
+        vec_slice(src);
         slice_store<BITS, NL>(slot, sv, lane);
         __syncwarp();
         tc::mbar_arrive(&slot_full[grp * 2 + buf]);
@@ -680,7 +733,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
             } else if (share_build) {
               group_build(src0);
             } else {
-              build_slice<BITS, NL, SrcT>(src0, ch, lane_on, sv);
+              vec_slice(src0);
             }
             cur_src = src0;
           }
@@ -719,7 +772,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
           }
           if (src != cur_src) {
             if (share_build) group_build(src);
-            else build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
+            else vec_slice(src);
             cur_src = src;
           }
           float acc[8];

@@ -171,6 +171,13 @@ struct GemvArgs {
   int32_t* flag_reset;
   int32_t* flag_set;
   const int32_t* flag_wait;
+  // token slices in the gate/up launch's fixed-point format (2 limbs,
+  // `bits`-bit chunks), [token][slice][word][lane]: the router launch's
+  // helper warps write them, the gate/up consumers copy a token's slice
+  // instead of converting its row again (table null: unused)
+  uint32_t* xsl;
+  const uint16_t* xsl_x;    // the token rows they were built from, [M][H]
+  int32_t xsl_M, xsl_H, xsl_bits, xsl_S;
 };
 
 enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
@@ -187,6 +194,9 @@ bool gemv_fits(int in_dim, int bits, int nmat, int G);
 int gemv_threads();     // threads of a GEMV CTA
 int gemv_plan_scratch_cap();  // bytes a plan computed inside a GEMV launch may use
 int gemv_units(int out_dim, const GemvShape& sh);
+// Words of one token's slices in the gate/up launch's format (2 limbs) for
+// rows of H codes at `bits` (0: no table for this width).
+size_t gemv_xslice_words(int H, int bits);
 
 // Launch with programmatic dependent launch (the kernel waits for its
 // predecessor's results before reading them).
