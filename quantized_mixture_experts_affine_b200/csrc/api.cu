@@ -524,23 +524,18 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   // several tokens planned in the gate/up launch: the router launch also
   // converts every token row once into the gate/up launch's slice format,
   // which the gate/up consumers copy instead of converting the row per unit
-  GemvArgs xs;
+  TokenSlices xs;
   memset(&xs, 0, sizeof(xs));
   if (M > 1 && fused_plan && !idx_in && L->gate.format == MOEQ_FMT_AFFINE &&
       gemv_xslice_words(H, L->gate.bits) > 0) {
-    xs.xsl = (uint32_t*)(base + lay.xsl);
-    xs.xsl_x = x;
-    xs.xsl_M = M;
-    xs.xsl_H = H;
-    xs.xsl_bits = L->gate.bits;
-    xs.xsl_S = gemv_shape(H, L->gate.bits, 2, L->gate.group_size).S;
+    xs.table = (uint32_t*)(base + lay.xsl);
+    xs.x = x;
+    xs.M = M;
+    xs.H = H;
+    xs.bits = L->gate.bits;
+    xs.S = gemv_shape(H, L->gate.bits, 2, L->gate.group_size).S;
   }
-  pf.xsl = xs.xsl;
-  pf.xsl_x = xs.xsl_x;
-  pf.xsl_M = xs.xsl_M;
-  pf.xsl_H = xs.xsl_H;
-  pf.xsl_bits = xs.xsl_bits;
-  pf.xsl_S = xs.xsl_S;
+  pf.xsl = xs;
   if (L->has_shared) {
     add_prefetch(pf, L->sh_gate, 0);
     add_prefetch(pf, L->sh_up, 0);
@@ -554,7 +549,7 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     LAUNCH(run_plain(R, segs, ns, 3, &pf, st));
     pf.n_pf = 0;
     pf.flag_reset = nullptr;
-    pf.xsl = nullptr;
+    pf.xsl.table = nullptr;
   }
   if (L->has_shared && (idx_in || !sg_with_router)) {
     Seg s = plain_seg(SG, 0, x, H, sg_logit, 1, M, 0);
@@ -636,12 +631,7 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     a.fused_plan = 1;
     a.plan = p;
     a.flag_set = flag;
-    a.xsl = xs.xsl;
-    a.xsl_x = xs.xsl_x;
-    a.xsl_M = xs.xsl_M;
-    a.xsl_H = xs.xsl_H;
-    a.xsl_bits = xs.xsl_bits;
-    a.xsl_S = xs.xsl_S;
+    a.xsl = xs;
     const int grid = max_gu < grid_cap() ? max_gu : grid_cap();
     LAUNCH(launch_gemv(L->gate.bits, 2, 2, SRC_BF16, a, grid, st));
   } else {

@@ -48,18 +48,18 @@ __device__ __forceinline__ void xslice_one(const uint16_t* row, int H, int sl, u
 
 // The helper warp's share of the token slice table: task t = (token, slice)
 // for t = blockIdx.x, blockIdx.x + gridDim.x, ...
-__device__ __noinline__ void build_xslices(const GemvArgs& a) {
+__device__ __noinline__ void build_xslices(const TokenSlices& ts) {
   const int lane = threadIdx.x & 31;
-  const int tasks = a.xsl_M * a.xsl_S;
+  const int tasks = ts.M * ts.S;
   for (int t = blockIdx.x; t < tasks; t += gridDim.x) {
-    const uint16_t* row = a.xsl_x + (int64_t)(t / a.xsl_S) * a.xsl_H;
-    const int sl = t % a.xsl_S;
-    if (a.xsl_bits == 2)
-      xslice_one<2>(row, a.xsl_H, sl, a.xsl + (size_t)t * (2 * 16 + 4) * 32, lane);
-    else if (a.xsl_bits == 4)
-      xslice_one<4>(row, a.xsl_H, sl, a.xsl + (size_t)t * (2 * 8 + 2) * 32, lane);
-    else if (a.xsl_bits == 8)
-      xslice_one<8>(row, a.xsl_H, sl, a.xsl + (size_t)t * (2 * 4 + 2) * 32, lane);
+    const uint16_t* row = ts.x + (int64_t)(t / ts.S) * ts.H;
+    const int sl = t % ts.S;
+    if (ts.bits == 2)
+      xslice_one<2>(row, ts.H, sl, ts.table + (size_t)t * (2 * 16 + 4) * 32, lane);
+    else if (ts.bits == 4)
+      xslice_one<4>(row, ts.H, sl, ts.table + (size_t)t * (2 * 8 + 2) * 32, lane);
+    else if (ts.bits == 8)
+      xslice_one<8>(row, ts.H, sl, ts.table + (size_t)t * (2 * 4 + 2) * 32, lane);
   }
 }
 
@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     else if (a.pf_segs) prefetch_segs(a.pf_segs, a.pf_count[0]);
     // the router launch: the token slice table of the gate/up launch
     if constexpr (NMAT == 1 && SRC == SRC_BF16 && !MX)
-      if (a.xsl) build_xslices(a);
+      if (a.xsl.table) build_xslices(a.xsl);
   } else if (warp == GV_PRODUCER) {
     // ------------------------------------------------------------ producer
     uint32_t it = preissued;
@@ -668,25 +668,26 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     int gi[2];
 #pragma unroll
     for (int pb = 0; pb < 2; ++pb) gi[pb] = (ch * VPC + (pb < NB ? pb : 0) * kXBlock) / a.G;
-    // With a single slice (S = 1) every warp of the group holds the same
-    // chunk: warp 0 of the group converts each new vector and hands the
-    // slice to the others through a double-buffered slot (full: warp 0's
-    // 32 lanes arrive; empty: the other warps' lanes arrive after copying;
-    // every wait bounded).  Build b uses buffer b & 1.
     // a token row's slice: copied from the table the router launch built,
     // else converted here
     auto vec_slice = [&](const void* src) {
       if constexpr (NMAT == 2 && SRC == SRC_BF16 && NL == 2 && !MX && !stream_bits(BITS)) {
-        if (a.xsl) {
-          const int64_t off = static_cast<const uint16_t*>(src) - a.xsl_x;
-          if (off >= 0 && off % a.xsl_H == 0 && off / a.xsl_H < a.xsl_M) {
-            slice_load<BITS, NL>(a.xsl + ((off / a.xsl_H) * a.xsl_S + sl) * SLW * 32, sv, lane);
+        if (a.xsl.table) {
+          const int64_t off = static_cast<const uint16_t*>(src) - a.xsl.x;
+          if (off >= 0 && off % a.xsl.H == 0 && off / a.xsl.H < a.xsl.M) {
+            const int64_t m = off / a.xsl.H;
+            slice_load<BITS, NL>(a.xsl.table + (m * a.xsl.S + sl) * SLW * 32, sv, lane);
             return;
           }
         }
       }
       build_slice<BITS, NL, SrcT>(src, ch, lane_on, sv);
     };
+    // With a single slice (S = 1) every warp of the group holds the same
+    // chunk: warp 0 of the group converts each new vector and hands the
+    // slice to the others through a double-buffered slot (full: warp 0's
+    // 32 lanes arrive; empty: the other warps' lanes arrive after copying;
+    // every wait bounded).  Build b uses buffer b & 1.
     const bool share_build = S == 1 && W > 1 && 2 * SLW * 32 <= GvSmem::SL_WORDS;
     uint32_t* const sl_grp = sl_base + grp * GvSmem::SL_WORDS;
     uint32_t nbuild = 0;

@@ -138,6 +138,14 @@ struct CombineArgs {
   int32_t sh_units;         // units per row block of the shared segment (>= 1)
 };
 
+// Token rows in the gate/up launch's fixed-point format (2 limbs, `bits`-bit
+// chunks), [token][slice][word][lane], as slice_load reads them.
+struct TokenSlices {
+  uint32_t* table;          // null: unused
+  const uint16_t* x;        // the token rows they were built from, [M][H]
+  int32_t M, H, bits, S;    // S: 32-chunk slices per row
+};
+
 struct GemvArgs {
   Seg segs[kInlineSegs];    // used when dyn_segs == nullptr
   int32_t n_segs;
@@ -171,13 +179,9 @@ struct GemvArgs {
   int32_t* flag_reset;
   int32_t* flag_set;
   const int32_t* flag_wait;
-  // token slices in the gate/up launch's fixed-point format (2 limbs,
-  // `bits`-bit chunks), [token][slice][word][lane]: the router launch's
-  // helper warps write them, the gate/up consumers copy a token's slice
-  // instead of converting its row again (table null: unused)
-  uint32_t* xsl;
-  const uint16_t* xsl_x;    // the token rows they were built from, [M][H]
-  int32_t xsl_M, xsl_H, xsl_bits, xsl_S;
+  // the step's token slices (router launch: writes them; gate/up launch:
+  // copies a token's slice instead of converting its row again)
+  TokenSlices xsl;
 };
 
 enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
