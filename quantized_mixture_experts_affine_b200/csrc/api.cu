@@ -324,10 +324,12 @@ static cudaError_t run_plain(const moeq_qtensor& shape_t, const Seg* segs, int n
 
 static cudaError_t run_dyn(const moeq_qtensor& shape_t, const Seg* segs, const int32_t* count,
                            int nl, int nmat, int src, int max_units, cudaStream_t st,
-                           const Seg* pf_segs = nullptr, const int32_t* pf_count = nullptr) {
+                           const Seg* pf_segs = nullptr, const int32_t* pf_count = nullptr,
+                           const TokenSlices* xsl = nullptr) {
   GemvArgs a;
   memset(&a, 0, sizeof(a));
   set_shape(a, shape_t, nmat);
+  if (xsl) a.xsl = *xsl;
   a.dyn_segs = segs;
   a.dyn_count = count;
   a.pf_segs = pf_segs;
@@ -521,12 +523,12 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
   GemvArgs pf;
   memset(&pf, 0, sizeof(pf));
   pf.flag_reset = flag;
-  // several tokens planned in the gate/up launch: the router launch also
-  // converts every token row once into the gate/up launch's slice format,
-  // which the gate/up consumers copy instead of converting the row per unit
+  // several tokens and a router launch: it also converts every token row
+  // once into the gate/up launch's slice format, which the gate/up
+  // consumers copy instead of converting the row for every unit
   TokenSlices xs;
   memset(&xs, 0, sizeof(xs));
-  if (M > 1 && fused_plan && !idx_in && L->gate.format == MOEQ_FMT_AFFINE &&
+  if (M > 1 && !idx_in && L->gate.format == MOEQ_FMT_AFFINE &&
       gemv_xslice_words(H, L->gate.bits) > 0) {
     xs.table = (uint32_t*)(base + lay.xsl);
     xs.x = x;
@@ -636,7 +638,8 @@ static moeq_status decode_forward(const moeq_layer* L, const uint16_t* x, int M,
     LAUNCH(launch_gemv(L->gate.bits, 2, 2, SRC_BF16, a, grid, st));
   } else {
     // the gate/up launch also pulls the down projections it will feed into L2
-    LAUNCH(run_dyn(L->gate, segs_gu, counts, 2, 2, SRC_BF16, max_gu, st, segs_dn, counts + 4));
+    LAUNCH(run_dyn(L->gate, segs_gu, counts, 2, 2, SRC_BF16, max_gu, st, segs_dn, counts + 4,
+                   &xs));
   }
   CK(profile_mark(false, st));
   if (L->has_shared && !p.shared_same_gu)
