@@ -52,7 +52,7 @@ __device__ __noinline__ void build_xslices(const TokenSlices& ts) {
   const int lane = threadIdx.x & 31;
   const int tasks = ts.M * ts.S;
   for (int t = blockIdx.x; t < tasks; t += gridDim.x) {
-    const uint16_t* row = ts.x + (int64_t)(t / ts.S) * ts.H;
+    const uint16_t* row = static_cast<const uint16_t*>(ts.x) + (int64_t)(t / ts.S) * ts.H;
     const int sl = t % ts.S;
     if (ts.bits == 2)
       xslice_one<2>(row, ts.H, sl, ts.table + (size_t)t * (2 * 16 + 4) * 32, lane);
@@ -668,12 +668,16 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     int gi[2];
 #pragma unroll
     for (int pb = 0; pb < 2; ++pb) gi[pb] = (ch * VPC + (pb < NB ? pb : 0) * kXBlock) / a.G;
-    // a token row's slice: copied from the table the router launch built,
-    // else converted here
+    // an input row's slice: copied from the table an earlier launch built
+    // (token rows: the router launch; hidden rows: the slice launch before
+    // the down launch), else converted here
     auto vec_slice = [&](const void* src) {
-      if constexpr (NMAT == 2 && SRC == SRC_BF16 && NL == 2 && !MX && !stream_bits(BITS)) {
+      constexpr bool kTable = !MX && NL == 2 && !stream_bits(BITS) &&
+                              ((NMAT == 2 && SRC == SRC_BF16) || (NMAT == 1 && SRC == SRC_F32));
+      if constexpr (kTable) {
         if (a.xsl.table) {
-          const int64_t off = static_cast<const uint16_t*>(src) - a.xsl.x;
+          using T = typename std::conditional<SRC == SRC_BF16, uint16_t, float>::type;
+          const int64_t off = static_cast<const T*>(src) - static_cast<const T*>(a.xsl.x);
           if (off >= 0 && off % a.xsl.H == 0 && off / a.xsl.H < a.xsl.M) {
             const int64_t m = off / a.xsl.H;
             slice_load<BITS, NL>(a.xsl.table + (m * a.xsl.S + sl) * SLW * 32, sv, lane);
@@ -688,7 +692,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ 
     // slice to the others through a double-buffered slot (full: warp 0's
     // 32 lanes arrive; empty: the other warps' lanes arrive after copying;
     // every wait bounded).  Build b uses buffer b & 1.
-    const bool share_build = S == 1 && W > 1 && 2 * SLW * 32 <= GvSmem::SL_WORDS;
+    const bool share_build =
+        !a.xsl.table && S == 1 && W > 1 && 2 * SLW * 32 <= GvSmem::SL_WORDS;
     uint32_t* const sl_grp = sl_base + grp * GvSmem::SL_WORDS;
     uint32_t nbuild = 0;
     bool slot_timeout = false;
@@ -915,6 +920,43 @@ static cudaError_t launch_one(const GemvArgs& a, int grid, cudaStream_t st) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// Slices of fp32 rows (the hidden rows of a decode step) in the down
+// launch's format, one warp per (row, slice).
+template <int B>
+__global__ void __launch_bounds__(128) k_hslices(const TokenSlices ts) {
+  constexpr int SLW = 2 * Chunk<B>::NC + 2 * SliceVec<B, 2>::NB;
+  // the down launch may be scheduled at once (its producer starts on the
+  // plan's flag); the rows are read after the gate/up launches end
+  tc::grid_dep_launch();
+  tc::grid_dep_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (t >= ts.M * ts.S) return;
+  const int sl = t % ts.S, ch = sl * 32 + lane;
+  const float* row = static_cast<const float*>(ts.x) + (int64_t)(t / ts.S) * ts.H;
+  SliceVec<B, 2> sv;
+  build_slice<B, 2, SrcF32>(row, ch, ch < ts.H / Chunk<B>::VPC, sv);
+  slice_store<B, 2>(ts.table + (size_t)t * SLW * 32, sv, lane);
+}
+
+cudaError_t launch_hslices(const TokenSlices& ts, cudaStream_t st) {
+  const int tasks = ts.M * ts.S;
+  if (!ts.table || tasks <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((tasks + 3) / 4);
+  cfg.blockDim = dim3(128);
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  if (ts.bits == 2) return cudaLaunchKernelEx(&cfg, k_hslices<2>, ts);
+  if (ts.bits == 4) return cudaLaunchKernelEx(&cfg, k_hslices<4>, ts);
+  if (ts.bits == 8) return cudaLaunchKernelEx(&cfg, k_hslices<8>, ts);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_gemv(int bits, int nl, int nmat, int src, const GemvArgs& a, int grid,

@@ -138,11 +138,13 @@ struct CombineArgs {
   int32_t sh_units;         // units per row block of the shared segment (>= 1)
 };
 
-// Token rows in the gate/up launch's fixed-point format (2 limbs, `bits`-bit
-// chunks), [token][slice][word][lane], as slice_load reads them.
+// Input rows of a GEMV launch in its fixed-point format (2 limbs, `bits`-bit
+// chunks), [row][slice][word][lane], as slice_load reads them: the token
+// rows (bf16) for the gate/up launch, the hidden rows (fp32) for the down
+// launch.
 struct TokenSlices {
   uint32_t* table;          // null: unused
-  const uint16_t* x;        // the token rows they were built from, [M][H]
+  const void* x;            // the rows they were built from, [M][H]
   int32_t M, H, bits, S;    // S: 32-chunk slices per row
 };
 
@@ -201,6 +203,9 @@ int gemv_units(int out_dim, const GemvShape& sh);
 // Words of one token's slices in the gate/up launch's format (2 limbs) for
 // rows of H codes at `bits` (0: no table for this width).
 size_t gemv_xslice_words(int H, int bits);
+// Slices of the M fp32 rows of ts.x (stride ts.H) into ts.table, after the
+// preceding launch (the gate/up launches that wrote the rows).
+cudaError_t launch_hslices(const TokenSlices& ts, cudaStream_t st);
 
 // Launch with programmatic dependent launch (the kernel waits for its
 // predecessor's results before reading them).
