@@ -199,8 +199,11 @@ DecodeWs decode_ws(const moeq_layer* L, int M) {
   w.flag = c.take(4);             // "down lists published"
   // the M tokens' slices in the gate/up format (built by the router launch)
   w.xsl = c.take((size_t)M * gemv_xslice_words(H, L->gate.bits) * 4);
-  // the hidden rows' slices in the down format (built by a launch of their own)
-  w.hsl = c.take((n + (size_t)M) * gemv_xslice_words(I, L->down.bits) * 4);
+  // the hidden rows' slices in the down format (built by a launch of their
+  // own; only for steps the gate/up launch plans itself)
+  w.hsl = c.take(n <= (size_t)kFusedMaxPairs
+                     ? (n + (size_t)M) * gemv_xslice_words(I, L->down.bits) * 4
+                     : 0);
   w.total = c.off;
   return w;
 }
